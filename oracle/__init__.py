@@ -1,0 +1,182 @@
+"""CPU oracle for the BitLinear forward (W1.58A8) -- TEST INFRASTRUCTURE.
+
+Only the tests, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline leg
+may import this package.  The product path (the CUDA library and its Python
+binding) never does, and shares no code with it.
+
+Each function is a thin numpy/ctypes wrapper over the plain C in
+``bitnet_oracle.c``; the C file states which passage of the BitNet model page
+each step follows and which reading was taken where the page is silent.
+Every function here is pinned by ``tests/test_oracle_pins.py``.
+"""
+import ctypes
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+def _bind(path):
+    """Load a compiled oracle library and declare its C signatures."""
+    lib = ctypes.CDLL(path)
+    P = ctypes.c_void_p
+    I = ctypes.c_int64
+    F = ctypes.c_float
+    sig = {
+        "oracle_bf16_to_f32": ([P, I, P], None),
+        "oracle_absmean_f64": ([P, I, I], ctypes.c_double),
+        "oracle_gamma": ([P, I, I], F),
+        "oracle_ternarize": ([P, I, I, F, F, P], None),
+        "oracle_pack": ([P, I, I, P], None),
+        "oracle_unpack": ([P, I, I, P], I),
+        "oracle_quant_act": ([P, I, I, P, P, P], None),
+        "oracle_int_matmul": ([P, P, I, I, I, P], None),
+        "oracle_int_dot_samples": ([P, P, I, P, P, I, P], None),
+        "oracle_dequant": ([P, P, F, I, I, P], None),
+        "oracle_relu2_gate": ([P, P, I, P], None),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    return lib
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        _lib = _bind(_build.build())
+    return _lib
+
+
+def _c(a, dtype):
+    a = np.ascontiguousarray(a, dtype=dtype)
+    return a, a.ctypes.data_as(ctypes.c_void_p)
+
+
+QUANT_EPS = 1e-5  # eps of gamma + eps and floor of max|x| (as fp32)
+
+
+def bf16_to_f32(bits):
+    """bf16 bit patterns (uint16) -> float32, exactly."""
+    src, p = _c(bits, np.uint16)
+    out = np.empty(src.shape, np.float32)
+    _load().oracle_bf16_to_f32(p, src.size, out.ctypes.data_as(ctypes.c_void_p))
+    return out
+
+
+def absmean_f64(w):
+    w, p = _c(w, np.float32)
+    n, k = w.shape
+    return float(_load().oracle_absmean_f64(p, n, k))
+
+
+def gamma(w):
+    """gamma = mean|W| (binary64 in canonical row order, rounded to fp32)."""
+    w, p = _c(w, np.float32)
+    n, k = w.shape
+    return np.float32(_load().oracle_gamma(p, n, k))
+
+
+def ternarize(w, gamma_, eps=QUANT_EPS):
+    w, p = _c(w, np.float32)
+    n, k = w.shape
+    out = np.empty((n, k), np.int8)
+    _load().oracle_ternarize(p, n, k, float(gamma_), float(np.float32(eps)),
+                             out.ctypes.data_as(ctypes.c_void_p))
+    return out
+
+
+def pack(w_q):
+    w_q, p = _c(w_q, np.int8)
+    n, k = w_q.shape
+    assert k % 16 == 0
+    out = np.empty((n, k // 4), np.uint8)
+    _load().oracle_pack(p, n, k, out.ctypes.data_as(ctypes.c_void_p))
+    return out
+
+
+def unpack(packed, k):
+    packed, p = _c(packed, np.uint8)
+    n = packed.shape[0]
+    out = np.empty((n, k), np.int8)
+    bad = _load().oracle_unpack(p, n, k, out.ctypes.data_as(ctypes.c_void_p))
+    return out, int(bad)
+
+
+def pack_weights(w, eps=QUANT_EPS):
+    """Whole offline step: returns (packed uint8 [N][K/4], gamma fp32, W_q int8)."""
+    g = gamma(w)
+    w_q = ternarize(w, g, eps)
+    return pack(w_q), g, w_q
+
+
+def quant_act(x):
+    """x: float32 [M][K] (exact bf16 values or fp32). Returns (x_q, s, rowsum)."""
+    x, p = _c(x, np.float32)
+    m, k = x.shape
+    x_q = np.empty((m, k), np.int8)
+    s = np.empty(m, np.float32)
+    rs = np.empty(m, np.int32)
+    _load().oracle_quant_act(p, m, k, x_q.ctypes.data_as(ctypes.c_void_p),
+                             s.ctypes.data_as(ctypes.c_void_p),
+                             rs.ctypes.data_as(ctypes.c_void_p))
+    return x_q, s, rs
+
+
+def int_matmul(x_q, w_q):
+    x_q, px = _c(x_q, np.int8)
+    w_q, pw = _c(w_q, np.int8)
+    m, k = x_q.shape
+    n, k2 = w_q.shape
+    assert k == k2
+    acc = np.empty((m, n), np.int64)
+    _load().oracle_int_matmul(px, pw, m, n, k, acc.ctypes.data_as(ctypes.c_void_p))
+    return acc
+
+
+def int_dot_samples(x_q, w_q, m_idx, n_idx):
+    x_q, px = _c(x_q, np.int8)
+    w_q, pw = _c(w_q, np.int8)
+    mi, pm = _c(m_idx, np.int64)
+    ni, pn = _c(n_idx, np.int64)
+    assert mi.shape == ni.shape
+    acc = np.empty(mi.shape, np.int64)
+    _load().oracle_int_dot_samples(px, pw, x_q.shape[1], pm, pn, mi.size,
+                                   acc.ctypes.data_as(ctypes.c_void_p))
+    return acc
+
+
+def dequant(acc, s, gamma_):
+    acc, pa = _c(acc, np.int64)
+    s, ps = _c(s, np.float32)
+    m, n = acc.shape
+    y = np.empty((m, n), np.float64)
+    _load().oracle_dequant(pa, ps, float(gamma_), m, n, y.ctypes.data_as(ctypes.c_void_p))
+    return y
+
+
+def relu2_gate(g, u):
+    g, pg = _c(g, np.float64)
+    u, pu = _c(u, np.float64)
+    assert g.shape == u.shape
+    h = np.empty(g.shape, np.float64)
+    _load().oracle_relu2_gate(pg, pu, g.size, h.ctypes.data_as(ctypes.c_void_p))
+    return h
+
+
+def bitlinear(x, packed, gamma_, k):
+    """Full forward from already-packed weights: (y fp64, acc int64, x_q, s)."""
+    w_q, bad = unpack(packed, k)
+    assert bad == 0
+    x_q, s, _ = quant_act(x)
+    acc = int_matmul(x_q, w_q)
+    return dequant(acc, s, gamma_), acc, x_q, s
+
+
+def ffn_gate_up(x, packed_g, gamma_g, packed_u, gamma_u, k):
+    """Fused gate/up forward: (h fp64, acc_g, acc_u, x_q, s)."""
+    yg, acc_g, x_q, s = bitlinear(x, packed_g, gamma_g, k)
+    yu, acc_u, _, _ = bitlinear(x, packed_u, gamma_u, k)
+    return relu2_gate(yg, yu), acc_g, acc_u, x_q, s

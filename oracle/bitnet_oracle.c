@@ -1,0 +1,231 @@
+/*
+ * bitnet_oracle.c -- plain, slow CPU oracle for the BitLinear forward (W1.58A8).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path links, loads or calls
+ * this file; only the tests, the smoke check and the benchmark's CPU-baseline
+ * leg do.  It shares no code, header, table or constant generator with the
+ * CUDA library.
+ *
+ * Source of truth: the "BitNet" model page of the transformers documentation
+ * (five translated copies of one page).  Its section "Model details", item
+ * "Quantization", states the scheme:
+ *   - weights are quantised to the ternary values {-1, 0, +1} with absmean
+ *     quantisation;
+ *   - activations are quantised to 8-bit integers with absmax quantisation,
+ *     per token;
+ *   - the pair is called W1.58A8.
+ * Item "Architecture" of the same section says the linear layers are BitLinear
+ * layers, carry no bias, and that the FFN uses squared ReLU (ReLU^2); the
+ * BitNetConfig section gives hidden_act = "relu2".  Section "Model variants"
+ * says the deployable checkpoint stores the 1.58-bit weights packed.
+ *
+ * The page gives no formulas.  This oracle takes the plainest reading:
+ *   gamma  = mean |W| over the whole weight matrix (one scale per matrix)
+ *   W_q    = clamp(round(W / (gamma + eps)), -1, 1), eps = 1e-5
+ *   s_m    = 127 / max_k |x_mk|      (one scale per token = per row of x)
+ *   x_q    = clamp(round(x * s_m), -128, 127)
+ *   acc    = x_q . W_q^T             (exact integers)
+ *   y      = acc * gamma / s_m
+ *   h      = relu(g)^2 * u           (gated FFN: g, u are two BitLinear outputs)
+ * "round" is round-half-to-even everywhere.
+ *
+ * Precision.  The page fixes none.  The quantisers decide integers, so they are
+ * evaluated in IEEE binary32 exactly as written (one fp32 division for s, one
+ * fp32 product x*s rounded once, then round-half-to-even to an integer; one
+ * fp32 add for gamma+eps, one fp32 division W/(gamma+eps)); the GPU takes the
+ * same decisions in the same precision.  gamma is accumulated in binary64 in a
+ * fixed order (each row left to right, then the row sums top to bottom) and
+ * rounded once to binary32.  Everything that does not decide an integer
+ * (dequantisation, the ReLU^2 gate) is computed in binary64.
+ *
+ * Special cases (the page is silent): an all-zero row has max|x| = 0; the
+ * divisor is clamped to 1e-5 so s is finite and x_q = 0.  Inputs are required
+ * to be finite.
+ *
+ * Packed layout (the page only says "packed"; this layout is this project's
+ * choice): code c = W_q + 1 in {0, 1, 2}.  Row n occupies bytes
+ * [n*K/4, (n+1)*K/4).  Weights are grouped by 16; group g of row n is the
+ * little-endian 32-bit word at byte offset n*K/4 + 4*g, and weight
+ * k = 16*g + 4*j + b (j, b in 0..3) sits in byte b at bits 2*j .. 2*j+1.
+ * K must be a multiple of 16 here (the library requires a multiple of 64).
+ *
+ * Build: gcc -O2 -std=c11 -ffp-contract=off -fPIC -shared (no fast-math).
+ */
+#include <math.h>
+#include <stddef.h>
+#include <stdint.h>
+#include <string.h>
+
+#define ORACLE_QUANT_EPS 1e-5f /* floor of max|x| and additive eps of gamma */
+
+/* ---- bf16 input ------------------------------------------------------- */
+
+/* bf16 -> fp32 is exact: the bf16 bits are the top half of the fp32 bits. */
+void oracle_bf16_to_f32(const uint16_t *src, int64_t count, float *dst)
+{
+    for (int64_t i = 0; i < count; ++i) {
+        uint32_t bits = ((uint32_t)src[i]) << 16;
+        float f;
+        memcpy(&f, &bits, sizeof f);
+        dst[i] = f;
+    }
+}
+
+/* ---- absmean weight ternarisation (page: "absmean", ternary) --------- */
+
+/* mean |W| in binary64: each row summed left to right, then the row sums
+ * summed top to bottom, divided by N*K.  Returned unrounded. */
+double oracle_absmean_f64(const float *w, int64_t n_rows, int64_t k_cols)
+{
+    double total = 0.0;
+    for (int64_t n = 0; n < n_rows; ++n) {
+        double row = 0.0;
+        for (int64_t k = 0; k < k_cols; ++k)
+            row += fabs((double)w[n * k_cols + k]);
+        total += row;
+    }
+    return total / (double)(n_rows * k_cols);
+}
+
+/* gamma as stored: the binary64 mean rounded once to binary32. */
+float oracle_gamma(const float *w, int64_t n_rows, int64_t k_cols)
+{
+    return (float)oracle_absmean_f64(w, n_rows, k_cols);
+}
+
+/* W_q = clamp(round_half_even(W / (gamma + eps)), -1, 1), fp32 arithmetic. */
+void oracle_ternarize(const float *w, int64_t n_rows, int64_t k_cols,
+                      float gamma, float eps, int8_t *w_q)
+{
+    const float d = gamma + eps;
+    for (int64_t i = 0; i < n_rows * k_cols; ++i) {
+        float q = nearbyintf(w[i] / d);
+        if (q > 1.0f) q = 1.0f;
+        if (q < -1.0f) q = -1.0f;
+        w_q[i] = (int8_t)q;
+    }
+}
+
+/* ---- 2-bit packing (page: "packed" 1.58-bit weights; layout ours) ---- */
+
+void oracle_pack(const int8_t *w_q, int64_t n_rows, int64_t k_cols, uint8_t *packed)
+{
+    const int64_t row_bytes = k_cols / 4;
+    memset(packed, 0, (size_t)(n_rows * row_bytes));
+    for (int64_t n = 0; n < n_rows; ++n) {
+        for (int64_t k = 0; k < k_cols; ++k) {
+            int64_t group = k / 16;
+            int64_t j = (k % 16) / 4;
+            int64_t b = k % 4;
+            uint8_t code = (uint8_t)(w_q[n * k_cols + k] + 1);
+            packed[n * row_bytes + 4 * group + b] |= (uint8_t)(code << (2 * j));
+        }
+    }
+}
+
+/* Inverse of oracle_pack.  Returns the number of invalid codes (3) seen;
+ * an invalid code decodes to 0. */
+int64_t oracle_unpack(const uint8_t *packed, int64_t n_rows, int64_t k_cols, int8_t *w_q)
+{
+    const int64_t row_bytes = k_cols / 4;
+    int64_t bad = 0;
+    for (int64_t n = 0; n < n_rows; ++n) {
+        for (int64_t k = 0; k < k_cols; ++k) {
+            int64_t group = k / 16;
+            int64_t j = (k % 16) / 4;
+            int64_t b = k % 4;
+            int code = (packed[n * row_bytes + 4 * group + b] >> (2 * j)) & 3;
+            if (code == 3) {
+                ++bad;
+                code = 1;
+            }
+            w_q[n * k_cols + k] = (int8_t)(code - 1);
+        }
+    }
+    return bad;
+}
+
+/* ---- per-token absmax activation quantisation (page: absmax, per token, 8-bit) */
+
+/* x: [m_rows][k_cols] fp32 (bf16 inputs are converted exactly beforehand).
+ * Writes x_q [m_rows][k_cols], s [m_rows] and, if non-NULL, rowsum [m_rows]
+ * (sum of x_q over the row, used by the code-offset form of the product). */
+void oracle_quant_act(const float *x, int64_t m_rows, int64_t k_cols,
+                      int8_t *x_q, float *s, int32_t *rowsum)
+{
+    for (int64_t m = 0; m < m_rows; ++m) {
+        const float *row = x + m * k_cols;
+        float amax = 0.0f;
+        for (int64_t k = 0; k < k_cols; ++k) {
+            float a = fabsf(row[k]);
+            if (a > amax) amax = a;
+        }
+        const float denom = amax > ORACLE_QUANT_EPS ? amax : ORACLE_QUANT_EPS;
+        const float scale = 127.0f / denom;
+        int64_t sum = 0;
+        for (int64_t k = 0; k < k_cols; ++k) {
+            float prod = row[k] * scale;
+            float q = nearbyintf(prod);
+            if (q > 127.0f) q = 127.0f;
+            if (q < -128.0f) q = -128.0f;
+            x_q[m * k_cols + k] = (int8_t)q;
+            sum += (int64_t)q;
+        }
+        s[m] = scale;
+        if (rowsum) rowsum[m] = (int32_t)sum;
+    }
+}
+
+/* ---- exact integer contraction (implied by W1.58A8) -------------------- */
+
+/* acc[m][n] = sum_k x_q[m][k] * w_q[n][k], accumulated in int64. */
+void oracle_int_matmul(const int8_t *x_q, const int8_t *w_q,
+                       int64_t m_rows, int64_t n_rows, int64_t k_cols, int64_t *acc)
+{
+    for (int64_t m = 0; m < m_rows; ++m) {
+        for (int64_t n = 0; n < n_rows; ++n) {
+            int64_t sum = 0;
+            for (int64_t k = 0; k < k_cols; ++k)
+                sum += (int64_t)x_q[m * k_cols + k] * (int64_t)w_q[n * k_cols + k];
+            acc[m * n_rows + n] = sum;
+        }
+    }
+}
+
+/* Same contraction restricted to a list of (m, n) output coordinates, for
+ * spot checks on problems too large to contract in full. */
+void oracle_int_dot_samples(const int8_t *x_q, const int8_t *w_q, int64_t k_cols,
+                            const int64_t *m_idx, const int64_t *n_idx, int64_t count,
+                            int64_t *acc)
+{
+    for (int64_t i = 0; i < count; ++i) {
+        const int8_t *xr = x_q + m_idx[i] * k_cols;
+        const int8_t *wr = w_q + n_idx[i] * k_cols;
+        int64_t sum = 0;
+        for (int64_t k = 0; k < k_cols; ++k)
+            sum += (int64_t)xr[k] * (int64_t)wr[k];
+        acc[i] = sum;
+    }
+}
+
+/* ---- dequantising epilogue -------------------------------------------- */
+
+/* y[m][n] = acc[m][n] * gamma / s[m], in binary64. */
+void oracle_dequant(const int64_t *acc, const float *s, float gamma,
+                    int64_t m_rows, int64_t n_rows, double *y)
+{
+    for (int64_t m = 0; m < m_rows; ++m)
+        for (int64_t n = 0; n < n_rows; ++n)
+            y[m * n_rows + n] = (double)acc[m * n_rows + n] * (double)gamma / (double)s[m];
+}
+
+/* ---- ReLU^2-gated FFN epilogue (page: ReLU^2 in the FFN, hidden_act relu2) */
+
+/* h = relu(g)^2 * u, elementwise, binary64. */
+void oracle_relu2_gate(const double *g, const double *u, int64_t count, double *h)
+{
+    for (int64_t i = 0; i < count; ++i) {
+        double r = g[i] > 0.0 ? g[i] : 0.0;
+        h[i] = r * r * u[i];
+    }
+}

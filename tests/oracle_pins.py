@@ -1,0 +1,318 @@
+"""Pins for the CPU oracle: facts fixed by the BitNet model page's scheme and by
+mathematics, checked against the oracle without retyping its arithmetic.
+
+Each ``pin_*`` function raises AssertionError when the oracle disagrees.  They
+are run by ``test_oracle_pins.py`` against the real oracle and by
+``test_oracle_mutants.py`` against copies of the oracle with planted mistakes
+(each mutant must fail at least one pin).
+
+Kinds of pin used:
+  * a hand-worked example (every value derived by hand, bit patterns included);
+  * hand-built special cases (exact ties, power-of-two scales, zero rows);
+  * invariants that hold for any input (ranges, argmax -> +-127, error bounds);
+  * closed forms for Gaussian latents (E mean|W|, zero fraction of W_q);
+  * independent library routines (exact summation, numpy integer matmul).
+"""
+import math
+from fractions import Fraction
+
+import numpy as np
+
+import oracle
+from ternary_weight_fwd_b200 import synth
+
+
+def _f32_bits(v):
+    return int(np.asarray(v, np.float32).view(np.uint32))
+
+
+# --------------------------------------------------------------------------
+# Hand-worked example.
+#   x = [0.5, -1, 0.25, 2] (bf16-exact)
+#   max|x| = 2, s = 127/2 = 63.5 (0x427E0000, exact)
+#   x*s = [31.75, -63.5, 15.875, 127] -> x_q = [32, -64 (tie -> even), 16, 127]
+#   W = [[0.03, -0.01, 0, -0.05], [0.02, 0.04, -0.02, 0.01]] (fp32)
+#   mean|W| of the fp32 values = 0.0224999998... -> gamma = 0x3CB851EB
+#   d = gamma + 1e-5 = 0x3CB866E4
+#   W/d = [[1.333, -0.444, 0, -2.221], [0.888, 1.777, -0.888, 0.444]]
+#     -> W_q = [[1, 0, 0, -1], [1, 1, -1, 0]]
+#   acc = [32 + (-127), 32 - 64 - 16] = [-95, -48]
+#   y = acc * gamma / s = [-0.0336614..., -0.0170078...]
+# --------------------------------------------------------------------------
+WX = [0.5, -1.0, 0.25, 2.0]
+WW = [[0.03, -0.01, 0.0, -0.05], [0.02, 0.04, -0.02, 0.01]]
+
+
+def pin_worked_example_quant():
+    x = np.array([WX], np.float32)
+    x_q, s, rs = oracle.quant_act(x)
+    assert _f32_bits(s[0]) == 0x427E0000, hex(_f32_bits(s[0]))
+    assert x_q.tolist() == [[32, -64, 16, 127]], x_q
+    assert int(rs[0]) == 111
+
+
+def pin_worked_example_weights():
+    w = np.array(WW, np.float32)
+    g = oracle.gamma(w)
+    assert _f32_bits(g) == 0x3CB851EB, hex(_f32_bits(g))
+    w_q = oracle.ternarize(w, g)
+    assert w_q.tolist() == [[1, 0, 0, -1], [1, 1, -1, 0]], w_q
+
+
+def pin_worked_example_forward():
+    w = np.array(WW, np.float32)
+    # pad K to 16 with zero weights / zero activations (does not change acc)
+    w16 = np.zeros((2, 16), np.float32)
+    w16[:, :4] = w
+    x16 = np.zeros((1, 16), np.float32)
+    x16[0, :4] = WX
+    g = oracle.gamma(w)           # gamma of the 2x4 matrix, as derived above
+    w_q = oracle.ternarize(w16, g)
+    packed = oracle.pack(w_q)
+    # row 0 codes [2,1,1,0, 1 x 12]: byte b = c[b] | c[4+b]<<2 | c[8+b]<<4 | c[12+b]<<6
+    assert packed[0, :4].tolist() == [0x56, 0x55, 0x55, 0x54], packed[0, :4]
+    # row 1 codes [2,2,0,1, 1 x 12]
+    assert packed[1, :4].tolist() == [0x56, 0x56, 0x54, 0x55], packed[1, :4]
+    y, acc, x_q, s = oracle.bitlinear(x16, packed, g, 16)
+    assert acc.tolist() == [[-95, -48]], acc
+    # hand-derived: -95 * 0.0224999990314245 / 63.5 and -48 * ... / 63.5
+    expect = [-95 * 0.022499999031424522 / 63.5, -48 * 0.022499999031424522 / 63.5]
+    assert np.allclose(y[0], expect, rtol=1e-12, atol=0), (y, expect)
+    # the same values printed to 8 digits (the fp32 results the GPU epilogue gives)
+    assert abs(y[0, 0] / -0.033661418 - 1) < 1e-7 and abs(y[0, 1] / -0.017007872 - 1) < 1e-7
+
+
+def pin_bf16_conversion():
+    bits = np.array([0x3F80, 0xC000, 0x4049, 0x0001, 0x8000, 0x7F7F], np.uint16)
+    f = oracle.bf16_to_f32(bits)
+    assert f[0] == 1.0 and f[1] == -2.0 and f[2] == 3.140625
+    assert f[3] == np.float32(2.0 ** -133) and f[4] == 0.0 and np.signbit(f[4])
+    assert f[5] == np.float32(3.3895313892515355e38)
+
+
+def pin_relu2_values():
+    g = np.array([0.5, -0.25, 0.0, 2.0, 3.0])
+    u = np.array([3.0, 7.0, 5.0, -1.0, 0.5])
+    h = oracle.relu2_gate(g, u)
+    # 0.25*3, gate<0 -> 0, gate=0 -> 0, 4*(-1), 9*0.5
+    assert h.tolist() == [0.75, 0.0, 0.0, -4.0, 4.5], h
+
+
+# --------------------------------------------------------------------------
+# Activation quantiser: hand-built exact cases.
+# --------------------------------------------------------------------------
+def pin_quant_ties_unit_scale():
+    # max|x| = 127 -> s = 1 exactly; ties go to the even integer
+    x = np.array([[127.0, 2.5, -2.5, 3.5, 0.5, -0.5, 1.5, -126.5]], np.float32)
+    x_q, s, rs = oracle.quant_act(x)
+    assert float(s[0]) == 1.0
+    assert x_q.tolist() == [[127, 2, -2, 4, 0, 0, 2, -126]], x_q
+    assert int(rs[0]) == 127 + 2 - 2 + 4 + 0 + 0 + 2 - 126
+
+
+def pin_quant_half_scale():
+    # max|x| = 254 -> s = 0.5 exactly
+    x = np.array([[1.0, 3.0, -5.0, -254.0, 7.0]], np.float32)
+    x_q, s, _ = oracle.quant_act(x)
+    assert float(s[0]) == 0.5
+    assert x_q.tolist() == [[0, 2, -2, -127, 4]], x_q
+
+
+def pin_quant_zero_row():
+    x = np.zeros((2, 32), np.float32)
+    x[1, 3] = 1.0
+    x_q, s, rs = oracle.quant_act(x)
+    assert not x_q[0].any() and int(rs[0]) == 0
+    assert float(s[0]) == float(np.float32(127.0) / np.float32(1e-5))
+    assert x_q[1, 3] == 127 and int(rs[1]) == 127
+
+
+def pin_quant_per_token():
+    # each row scaled by its own max; permuting rows permutes everything
+    x = synth.bf16_bits_to_f32(synth.activations(6, 64, 11, "student_t_rows"))
+    x_q, s, rs = oracle.quant_act(x)
+    perm = np.array([3, 0, 5, 1, 4, 2])
+    x_q2, s2, rs2 = oracle.quant_act(x[perm])
+    assert (x_q2 == x_q[perm]).all() and (s2 == s[perm]).all() and (rs2 == rs[perm]).all()
+    # columns: permuting columns permutes x_q and leaves s alone
+    cp = np.random.default_rng(3).permutation(64)
+    x_q3, s3, _ = oracle.quant_act(x[:, cp])
+    assert (x_q3 == x_q[:, cp]).all() and (s3 == s).all()
+
+
+def pin_quant_power_of_two_invariance():
+    # scaling a row by 2^e is exact, so s scales by 2^-e and x_q is unchanged
+    x = synth.bf16_bits_to_f32(synth.activations(4, 256, 12))
+    x_q, s, _ = oracle.quant_act(x)
+    for e in (-3, 5):
+        x_q2, s2, _ = oracle.quant_act(x * np.float32(2.0 ** e))
+        assert (x_q2 == x_q).all()
+        assert (s2 == s * np.float32(2.0 ** -e)).all()
+
+
+def pin_quant_invariants_random():
+    for seed, kind in ((21, "normal"), (22, "outliers"), (23, "student_t_rows")):
+        x = synth.bf16_bits_to_f32(synth.activations(16, 2560, seed, kind))
+        x_q, s, rs = oracle.quant_act(x)
+        assert x_q.min() >= -127 and x_q.max() <= 127          # -128 never produced
+        amax = np.abs(x).max(axis=1)
+        arg = np.abs(x).argmax(axis=1)
+        for m in range(x.shape[0]):                             # row max -> +-127
+            assert x_q[m, arg[m]] == (127 if x[m, arg[m]] > 0 else -127)
+        # s = 127 / max|x| to within one fp32 rounding
+        assert np.all(np.abs(s.astype(np.float64) * amax - 127.0) <= 127.0 * 2.0 ** -23)
+        # rounding error: |x*s - x_q| <= 1/2 (+ one rounding of the product)
+        err = np.abs(x.astype(np.float64) * s[:, None] - x_q)
+        assert err.max() <= 0.5 + 127.0 * 2.0 ** -23, err.max()
+        # signs agree or x_q is zero
+        assert np.all((np.sign(x_q) == np.sign(x)) | (x_q == 0))
+        assert (rs == x_q.astype(np.int64).sum(axis=1)).all()
+
+
+# --------------------------------------------------------------------------
+# Weight ternariser and gamma.
+# --------------------------------------------------------------------------
+def pin_gamma_simple_means():
+    assert float(oracle.gamma(np.array([[1, 2], [3, 4]], np.float32))) == 2.5
+    assert float(oracle.gamma(np.array([[-1, 2], [-3, -4]], np.float32))) == 2.5
+    assert float(oracle.gamma(np.full((3, 16), -0.25, np.float32))) == 0.25
+    # asymmetric shape: rows and columns both count
+    w = np.zeros((2, 16), np.float32)
+    w[1, 15] = 32.0
+    assert float(oracle.gamma(w)) == 1.0
+
+
+def pin_gamma_exact_sum():
+    # mean|W| rounded to fp32 equals the correctly rounded exact mean
+    for (n, k, seed) in ((64, 256, 31), (300, 320, 32), (7, 2560, 33)):
+        w = synth.latent_weights(n, k, seed)
+        exact = Fraction(math.fsum(np.abs(w.astype(np.float64)).ravel())) / (n * k)
+        assert oracle.gamma(w) == np.float32(float(exact))
+        assert abs(oracle.absmean_f64(w) - float(exact)) <= 1e-12 * float(exact)
+
+
+def pin_ternarize_constructed():
+    g = np.float32(1.0)
+    d = np.float32(g + np.float32(1e-5))
+    w = np.array([[0.5 * d, -0.5 * d, d, -d, 2 * d, -3 * d, 0.0, 0.4,
+                   0.51, -0.51, 1.45, -1.55, 100.0, -1e-30, 0.6, -0.6]], np.float32)
+    w_q = oracle.ternarize(w, g)
+    assert w_q.tolist() == [[0, 0, 1, -1, 1, -1, 0, 0, 1, -1, 1, -1, 1, 0, 1, -1]], w_q
+
+
+def pin_ternarize_threshold_random():
+    w = synth.latent_weights(128, 512, 41)
+    g = oracle.gamma(w)
+    w_q = oracle.ternarize(w, g)
+    assert set(np.unique(w_q).tolist()) <= {-1, 0, 1}
+    r = w.astype(np.float64) / (float(g) + 1e-5)
+    far = np.abs(np.abs(r) - 0.5) > 1e-5           # away from the rounding boundary
+    expect = np.where(np.abs(r) > 0.5, np.sign(r), 0)
+    assert (w_q[far] == expect[far]).all()
+
+
+def pin_ternary_closed_forms():
+    # Gaussian latents N(0, s): E|W| = s*sqrt(2/pi); P(|W| < gamma/2) = 2*Phi(sqrt(2/pi)/2) - 1
+    n, k = 2560, 6912
+    w = synth.latent_weights(n, k, 42)
+    g = float(oracle.gamma(w))
+    e_abs = 0.02 * math.sqrt(2.0 / math.pi)
+    assert abs(g / e_abs - 1.0) < 1e-3, g
+    w_q = oracle.ternarize(w, np.float32(g))
+    frac0 = float((w_q == 0).mean())
+    p0 = math.erf(0.5 * math.sqrt(2.0 / math.pi) / math.sqrt(2.0))
+    sd = math.sqrt(p0 * (1 - p0) / (n * k))
+    assert abs(frac0 - p0) < 6 * sd + 2e-4, (frac0, p0)   # + finite-gamma wiggle
+    fp, fm = float((w_q == 1).mean()), float((w_q == -1).mean())
+    assert abs(fp - fm) < 6 * math.sqrt(0.35 / (n * k)) * 2, (fp, fm)
+
+
+# --------------------------------------------------------------------------
+# Packing.
+# --------------------------------------------------------------------------
+def pin_pack_single_weight_probes():
+    base = np.zeros((1, 32), np.int8)
+    assert oracle.pack(base).tolist() == [[0x55] * 8]
+    w = base.copy()
+    w[0, 5] = 1          # group 0, k%16 = 5 -> j = 1, b = 1: byte 1 bits 2..3 = 0b10
+    assert oracle.pack(w).tolist() == [[0x55, 0x59, 0x55, 0x55, 0x55, 0x55, 0x55, 0x55]]
+    w = base.copy()
+    w[0, 18] = -1        # group 1, k%16 = 2 -> j = 0, b = 2: byte 4+2 bits 0..1 = 0b00
+    assert oracle.pack(w).tolist() == [[0x55, 0x55, 0x55, 0x55, 0x55, 0x55, 0x54, 0x55]]
+    w = base.copy()
+    w[0, 31] = 1         # group 1, k%16 = 15 -> j = 3, b = 3: byte 7 bits 6..7 = 0b10
+    assert oracle.pack(w).tolist() == [[0x55, 0x55, 0x55, 0x55, 0x55, 0x55, 0x55, 0x95]]
+    w = np.zeros((2, 16), np.int8)
+    w[1, 0] = -1         # second row starts at byte K/4 = 4
+    assert oracle.pack(w).tolist() == [[0x55] * 4, [0x54, 0x55, 0x55, 0x55]]
+
+
+def pin_pack_roundtrip():
+    r = np.random.default_rng(51)
+    for (n, k) in ((3, 16), (17, 64), (40, 2560)):
+        w_q = r.integers(-1, 2, size=(n, k)).astype(np.int8)
+        packed = oracle.pack(w_q)
+        assert packed.shape == (n, k // 4)
+        back, bad = oracle.unpack(packed, k)
+        assert bad == 0 and (back == w_q).all()
+    planted = oracle.pack(np.zeros((1, 16), np.int8))
+    planted[0, 2] |= 0x30                  # code 3 at k = 2*4 + 2 = 10
+    _, bad = oracle.unpack(planted, 16)
+    assert bad == 1
+
+
+# --------------------------------------------------------------------------
+# Integer contraction and epilogue.
+# --------------------------------------------------------------------------
+def pin_int_matmul_vs_numpy():
+    r = np.random.default_rng(61)
+    for (m, n, k) in ((1, 7, 64), (5, 33, 256), (4, 256, 320)):
+        a = r.integers(-128, 128, size=(m, k)).astype(np.int8)
+        b = r.integers(-1, 2, size=(n, k)).astype(np.int8)
+        acc = oracle.int_matmul(a, b)
+        assert (acc == a.astype(np.int64) @ b.astype(np.int64).T).all()
+        mi = r.integers(0, m, size=20)
+        ni = r.integers(0, n, size=20)
+        assert (oracle.int_dot_samples(a, b, mi, ni) == acc[mi, ni]).all()
+
+
+def pin_dequant_special_values():
+    acc = np.array([[0, 1, -7, 877824]], np.int64)
+    s = np.array([1.0], np.float32)
+    y = oracle.dequant(acc, s, np.float32(1.0))
+    assert y.tolist() == [[0.0, 1.0, -7.0, 877824.0]]
+    s = np.array([0.5], np.float32)
+    y = oracle.dequant(acc, s, np.float32(0.25))          # gamma/s = 0.5
+    assert y.tolist() == [[0.0, 0.5, -3.5, 438912.0]]
+    # row m uses s[m]
+    acc2 = np.array([[4, 8], [4, 8]], np.int64)
+    y2 = oracle.dequant(acc2, np.array([2.0, 4.0], np.float32), np.float32(1.0))
+    assert y2.tolist() == [[2.0, 4.0], [1.0, 2.0]]
+
+
+def pin_forward_error_bound():
+    # y approximates x . (gamma W_q)^T; the only gap is activation rounding:
+    # |y - x.(gamma W_q)^T| <= gamma * sum_k |W_q| * (1/2 + eps') / s
+    x = synth.bf16_bits_to_f32(synth.activations(6, 256, 71, "outliers"))
+    w = synth.latent_weights(48, 256, 72)
+    packed, g, w_q = oracle.pack_weights(w)
+    y, acc, x_q, s = oracle.bitlinear(x, packed, g, 256)
+    ref = x.astype(np.float64) @ (float(g) * w_q.astype(np.float64)).T
+    bound = float(g) * np.abs(w_q).sum(axis=1)[None, :] * (0.5 + 1e-4) / s[:, None].astype(np.float64)
+    assert np.all(np.abs(y - ref) <= bound + 1e-12)
+    assert np.all((y == 0) == (acc == 0)) and np.all(np.sign(y) == np.sign(acc))
+
+
+def pin_ffn_composition():
+    x = synth.bf16_bits_to_f32(synth.activations(3, 64, 81))
+    pg, gg, _ = oracle.pack_weights(synth.latent_weights(32, 64, 82))
+    pu, gu, _ = oracle.pack_weights(synth.latent_weights(32, 64, 83))
+    h, ag, au, _, s = oracle.ffn_gate_up(x, pg, gg, pu, gu, 64)
+    yg = oracle.dequant(ag, s, gg)
+    yu = oracle.dequant(au, s, gu)
+    assert np.all(h[yg <= 0] == 0)
+    pos = yg > 0
+    assert np.allclose(h[pos], (yg[pos] ** 2) * yu[pos], rtol=1e-15, atol=0)
+
+
+ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -1,0 +1,69 @@
+"""Each planted mistake in a copy of the oracle must fail at least one pin.
+
+The mistakes are the plausible ones: a dropped term, a wrong sign, index or
+operand order, a wrong rounding mode, a wrong constant.  Every mutant is a
+textual edit of ``oracle/bitnet_oracle.c`` compiled into a temporary library;
+all edits keep every memory access in bounds.
+"""
+import os
+
+import pytest
+
+import oracle
+import oracle_pins
+from oracle import build as oracle_build
+
+MUTANTS = {
+    "round_half_away": ("float q = nearbyintf(prod);", "float q = roundf(prod);"),
+    "scale_128": ("const float scale = 127.0f / denom;", "const float scale = 128.0f / denom;"),
+    "scale_inverted": ("float prod = row[k] * scale;", "float prod = row[k] / scale;"),
+    "amax_floor_1e-3": ("amax > ORACLE_QUANT_EPS ? amax : ORACLE_QUANT_EPS",
+                        "amax > 1e-3f ? amax : 1e-3f"),
+    "amax_not_abs": ("float a = fabsf(row[k]);", "float a = row[k];"),
+    "rowsum_abs": ("sum += (int64_t)q;", "sum += (int64_t)fabsf(q);"),
+    # (a clamp at -127 instead of -128 would be an equivalent mutant: |x*s| <= 127)
+    "clamp_high_126": ("if (q > 127.0f) q = 127.0f;", "if (q > 126.0f) q = 126.0f;"),
+    "gamma_no_abs": ("row += fabs((double)w[n * k_cols + k]);", "row += (double)w[n * k_cols + k];"),
+    "gamma_rows_only": ("return total / (double)(n_rows * k_cols);", "return total / (double)(k_cols);"),
+    "eps_dropped": ("const float d = gamma + eps;", "const float d = gamma;"),
+    "ternary_no_clamp": ("if (q > 1.0f) q = 1.0f;", ""),
+    "ternary_trunc": ("float q = nearbyintf(w[i] / d);", "float q = truncf(w[i] / d);"),
+    "pack_b_j_swapped": ("packed[n * row_bytes + 4 * group + b] |= (uint8_t)(code << (2 * j));",
+                         "packed[n * row_bytes + 4 * group + j] |= (uint8_t)(code << (2 * b));"),
+    "pack_offset_2": ("uint8_t code = (uint8_t)(w_q[n * k_cols + k] + 1);",
+                      "uint8_t code = (uint8_t)(w_q[n * k_cols + k] + 2);"),
+    "unpack_wrong_shift": ("int code = (packed[n * row_bytes + 4 * group + b] >> (2 * j)) & 3;",
+                           "int code = (packed[n * row_bytes + 4 * group + b] >> (2 * b)) & 3;"),
+    "matmul_k_reversed": ("sum += (int64_t)x_q[m * k_cols + k] * (int64_t)w_q[n * k_cols + k];",
+                          "sum += (int64_t)x_q[m * k_cols + (k_cols - 1 - k)] * (int64_t)w_q[n * k_cols + k];"),
+    "matmul_int8_wrap": ("sum += (int64_t)x_q[m * k_cols + k] * (int64_t)w_q[n * k_cols + k];",
+                         "sum = (int8_t)(sum + x_q[m * k_cols + k] * w_q[n * k_cols + k]);"),
+    "dequant_scale_inverted": ("(double)gamma / (double)s[m];", "(double)s[m] / (double)gamma;"),
+    "dequant_first_row_scale": ("(double)gamma / (double)s[m];", "(double)gamma / (double)s[0];"),
+    "relu_dropped": ("double r = g[i] > 0.0 ? g[i] : 0.0;", "double r = g[i];"),
+    "relu_not_squared": ("h[i] = r * r * u[i];", "h[i] = r * u[i];"),
+    "bf16_shift": ("uint32_t bits = ((uint32_t)src[i]) << 16;", "uint32_t bits = ((uint32_t)src[i]) << 15;"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(oracle_build.SRC).read()
+    assert src.count(old) >= 1, f"mutation site for {name} not found"
+    mutated = src.replace(old, new, 1)
+    path = tmp_path / "mutant.c"
+    path.write_text(mutated)
+    lib = oracle._bind(oracle_build.compile_source(str(path), str(tmp_path / f"lib_{name}.so")))
+    saved = oracle._load()
+    oracle._lib = lib
+    failed = []
+    try:
+        for pin in oracle_pins.ALL_PINS:
+            try:
+                pin()
+            except AssertionError:
+                failed.append(pin.__name__)
+    finally:
+        oracle._lib = saved
+    assert failed, f"mutant {name} passed every pin"
