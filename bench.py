@@ -1,0 +1,545 @@
+#!/usr/bin/env python3
+"""Benchmark of the BitLinear forward on a BitNet b1.58 2B4T-shaped layer stack.
+
+Workload (one "step"): all BitLinear projections of 30 random-init layers
+(hidden 2560, intermediate 6912): q and o (2560 -> 2560), the fused gate/up
+FFN (2560 -> 2 x 6912, relu(gate)^2 * up) and down (6912 -> 2560).  A step is
+one prefill pass over 8 x 512 = 4096 tokens followed by 128 decode steps at
+batch 8, every projection through the library's C ABI (Python binding), each
+phase captured once as CUDA graphs and replayed.  Weights are ternarised and
+packed once before timing (the method does this offline).
+
+Reported metric: BitLinear throughput as tokens/s per layer (token-layers per
+second of device time; prefill and decode tokens both count), with the phase
+breakdown in GB/s (decode, against HBM) and TOPS (prefill, against the int8
+tensor-core peak), a roofline entry for the kernel with the largest share of
+the step, the oracle timed on the host, and an end-to-end figure with
+host<->device copies inside the timed region.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (torchrun, one process per GPU) every rank runs its own replica on
+its own batch (data parallel, no collective on the data path; weak scaling);
+the time is the max over ranks.
+"""
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "BitLinear GB/s and TOPS (% of HBM / INT8 roofline); decode tokens/s per layer"
+UNIT = "tokens/s per layer"
+HIDDEN, INTER = 2560, 6912
+NOMINAL_INT8_PER_BF16 = 2.0  # dense int8 / dense bf16 tensor rate on B200 (4.5 / 2.25 PFLOP/s)
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--layers", type=int, default=30)
+    p.add_argument("--prefill-tokens", type=int, default=4096)
+    p.add_argument("--decode-steps", type=int, default=128)
+    p.add_argument("--decode-batch", type=int, default=8)
+    p.add_argument("--e2e-steps", type=int, default=3)
+    p.add_argument("--cpu-seconds", type=float, default=10.0, help="budget of the oracle CPU baseline")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def workload_config(a, n_gpus):
+    return {
+        "workload": (f"bitnet-b1.58-2b4t BitLinear stack: {a.layers} layers x (q, o {HIDDEN}x{HIDDEN}; "
+                     f"gate/up {HIDDEN}->2x{INTER} + relu2; down {INTER}->{HIDDEN}); "
+                     f"prefill {a.prefill_tokens} tokens (8x512) then {a.decode_steps} decode steps at batch "
+                     f"{a.decode_batch}"),
+        "layers": a.layers, "hidden": HIDDEN, "intermediate": INTER,
+        "prefill_tokens": a.prefill_tokens, "decode_steps": a.decode_steps, "decode_batch": a.decode_batch,
+        "activations": "bf16 N(0,1), fresh per projection; ternary weights from N(0,0.02) latents",
+        "l2": "inputs larger than L2: every pass streams 496 MB of packed weights; prefill activations rotate "
+              "over 168 MB",
+        "parallelism": f"replicas x{n_gpus} (data parallel, no collective)",
+    }
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ oracle (CPU)
+def oracle_layer_sample(tokens, seed=4242):
+    """Bounded CPU sample of the workload: `tokens` tokens through one layer's
+    four projections with the oracle.  Returns (closure, description)."""
+    import numpy as np
+
+    import oracle
+    from ternary_weight_fwd_b200 import synth
+
+    mats = {}
+    for j, (name, n, k) in enumerate((("q", HIDDEN, HIDDEN), ("o", HIDDEN, HIDDEN), ("gate", INTER, HIDDEN),
+                                      ("up", INTER, HIDDEN), ("down", HIDDEN, INTER))):
+        p, g, _ = oracle.pack_weights(synth.latent_weights(n, k, seed + j))
+        mats[name] = (p, g, k)
+    xs = [synth.bf16_bits_to_f32(synth.activations(tokens, HIDDEN, seed + 10 + i)) for i in range(3)]
+
+    def run():
+        oracle.bitlinear(xs[0], *mats["q"])
+        oracle.bitlinear(xs[1], *mats["o"])
+        h = oracle.ffn_gate_up(xs[2], mats["gate"][0], mats["gate"][1], mats["up"][0], mats["up"][1], HIDDEN)[0]
+        oracle.bitlinear(h.astype(np.float32), *mats["down"])
+
+    return run, (f"{tokens} tokens through one layer (q, o, gate/up+relu2, down) with the C oracle, "
+                 f"single thread; tokens/s per layer = tokens / time")
+
+
+def cpu_baseline(budget_s, tokens=8):
+    run, desc = oracle_layer_sample(tokens)
+    run()  # warm
+    times = []
+    t_end = time.perf_counter() + budget_s
+    while time.perf_counter() < t_end or len(times) < 2:
+        t0 = time.perf_counter()
+        run()
+        times.append(time.perf_counter() - t0)
+    mean = statistics.mean(times)
+    return {"value": tokens / mean, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{desc}; {len(times)} repetitions, {sum(times):.1f} s"}
+
+
+def reference_arm(a, n_gpus):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    tokens = a.decode_batch
+    run, desc = oracle_layer_sample(tokens)
+    for _ in range(a.warmup):
+        run()
+    times = []
+    for _ in range(a.steps):
+        t0 = time.perf_counter()
+        run()
+        times.append(time.perf_counter() - t0)
+    ms = 1e3 * statistics.mean(times)
+    value = tokens / (ms / 1e3)
+    cfg = workload_config(a, n_gpus)
+    cfg["sample"] = desc
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": n_gpus,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int64", "data": "synthetic", "config": cfg,
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.out, stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ our arm
+class Stack:
+    """Packed weights, activation pools and output buffers of the layer stack."""
+
+    def __init__(self, a, device, seed):
+        import torch
+
+        import ternary_weight_fwd_b200 as tw
+
+        self.a, self.dev, self.tw, self.torch = a, device, tw, torch
+        gen = torch.Generator(device=device)
+        gen.manual_seed(seed)
+        self.layers = []
+        for _ in range(a.layers):
+            layer = {}
+            for name, n, k in (("q", HIDDEN, HIDDEN), ("o", HIDDEN, HIDDEN), ("gate", INTER, HIDDEN),
+                               ("up", INTER, HIDDEN), ("down", HIDDEN, INTER)):
+                w = torch.randn((n, k), generator=gen, device=device, dtype=torch.float32).mul_(0.02)
+                layer[name] = tw.bitnet_pack_weights(w)
+                del w
+            self.layers.append(layer)
+        torch.cuda.synchronize()
+        M, B = a.prefill_tokens, a.decode_batch
+        self.n_pre = 8   # 8 x 21 MB of bf16 prefill activations (> L2) rotated over the projections
+        self.n_dec = 64
+        self.pre_x = [torch.randn((M, HIDDEN), generator=gen, device=device).to(torch.bfloat16)
+                      for _ in range(self.n_pre)]
+        self.dec_x = [torch.randn((B, HIDDEN), generator=gen, device=device).to(torch.bfloat16)
+                      for _ in range(self.n_dec)]
+        f32 = torch.float32
+        self.pre_out = {"q": torch.empty((M, HIDDEN), dtype=f32, device=device),
+                        "o": torch.empty((M, HIDDEN), dtype=f32, device=device),
+                        "h": torch.empty((M, INTER), dtype=f32, device=device),
+                        "down": torch.empty((M, HIDDEN), dtype=f32, device=device)}
+        self.dec_out = {"q": torch.empty((B, HIDDEN), dtype=f32, device=device),
+                        "o": torch.empty((B, HIDDEN), dtype=f32, device=device),
+                        "h": torch.empty((B, INTER), dtype=f32, device=device),
+                        "down": torch.empty((B, HIDDEN), dtype=f32, device=device)}
+        ws = max(tw.bitnet_workspace_size(M, INTER, INTER), tw.bitnet_workspace_size(M, HIDDEN, HIDDEN))
+        self.ws_pre = torch.empty(ws, dtype=torch.uint8, device=device)
+        self.ws_dec = torch.empty(tw.bitnet_workspace_size(B, INTER, INTER), dtype=torch.uint8, device=device)
+        self.packed_bytes = sum(p.numel() for L in self.layers for (p, _) in L.values())
+
+    # one projection of each kind -------------------------------------------
+    def q(self, l, x, out, ws, s):
+        L = self.layers[l]
+        self.tw.bitnet_linear(x, L["q"][0], L["q"][1], y=out["q"], workspace=ws, stream=s)
+
+    def o(self, l, x, out, ws, s):
+        L = self.layers[l]
+        self.tw.bitnet_linear(x, L["o"][0], L["o"][1], y=out["o"], workspace=ws, stream=s)
+
+    def gate_up(self, l, x, out, ws, s):
+        L = self.layers[l]
+        self.tw.bitnet_ffn_gate_up(x, L["gate"][0], L["gate"][1], L["up"][0], L["up"][1], h=out["h"],
+                                   workspace=ws, stream=s)
+
+    def down(self, l, out, ws, s):
+        L = self.layers[l]
+        self.tw.bitnet_linear(out["h"], L["down"][0], L["down"][1], y=out["down"], workspace=ws, stream=s)
+
+    def prefill_pass(self, s):
+        for l in range(self.a.layers):
+            self.q(l, self.pre_x[(3 * l) % self.n_pre], self.pre_out, self.ws_pre, s)
+            self.o(l, self.pre_x[(3 * l + 1) % self.n_pre], self.pre_out, self.ws_pre, s)
+            self.gate_up(l, self.pre_x[(3 * l + 2) % self.n_pre], self.pre_out, self.ws_pre, s)
+            self.down(l, self.pre_out, self.ws_pre, s)
+
+    def decode_step(self, t, s):
+        for l in range(self.a.layers):
+            base = t * 3 * self.a.layers + 3 * l
+            self.q(l, self.dec_x[base % self.n_dec], self.dec_out, self.ws_dec, s)
+            self.o(l, self.dec_x[(base + 1) % self.n_dec], self.dec_out, self.ws_dec, s)
+            self.gate_up(l, self.dec_x[(base + 2) % self.n_dec], self.dec_out, self.ws_dec, s)
+            self.down(l, self.dec_out, self.ws_dec, s)
+
+
+def capture(torch, stream, fn):
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn(stream)
+    return g
+
+
+def time_graph(torch, stream, graph, reps):
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    graph.replay()
+    stream.synchronize()
+    e0.record(stream)
+    for _ in range(reps):
+        graph.replay()
+    e1.record(stream)
+    e1.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def source_digest():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "ternary_weight_fwd_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode())
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def dram_traffic(kernel_key):
+    """Per-launch DRAM bytes of a kernel from the committed ncu summary, if it was
+    taken on the current kernel sources; otherwise None."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    e = d.get(kernel_key)
+    if not e or e.get("source_digest") != source_digest():
+        return None
+    return e.get("bytes_per_launch")
+
+
+def our_arm(a, n_gpus):
+    import torch
+
+    import ternary_weight_fwd_b200 as tw
+    from ternary_weight_fwd_b200 import build as tw_build
+
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    dist = None
+    if world > 1:
+        import torch.distributed as dist_mod
+        dist = dist_mod
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    if rank == 0:
+        tw_build.build()
+    if dist:
+        dist.barrier()
+    tw.load_library()
+    peaks, peaks_src = load_peaks()
+
+    def barrier():
+        if dist:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if not dist:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    st = Stack(a, dev, seed=1234 + rank)
+    stream = torch.cuda.Stream(device=dev)
+    stream.wait_stream(torch.cuda.current_stream())
+
+    # ---- capture: one prefill pass, decode steps in chunks of 16 ----
+    with torch.cuda.stream(stream):
+        c0 = tw.bitnet_launch_count()
+        g_pre = capture(torch, stream, st.prefill_pass)
+        c1 = tw.bitnet_launch_count()
+        chunk = 16
+        g_dec = []
+        for t0 in range(0, a.decode_steps, chunk):
+            g_dec.append(capture(torch, stream, lambda s, t0=t0: [st.decode_step(t, s) for t in
+                                                                  range(t0, min(t0 + chunk, a.decode_steps))]))
+        c2 = tw.bitnet_launch_count()
+    launches_pre, launches_dec = c1 - c0, c2 - c1
+
+    def run_step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        g_pre.replay()
+        if ev is not None:
+            ev[1].record(stream)
+        for g in g_dec:
+            g.replay()
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(a.warmup):
+        run_step()
+    stream.synchronize()
+    barrier()
+    clocks = ClockSampler(local_rank if world > 1 else torch.cuda.current_device())
+    clocks.start()
+    time.sleep(0.3)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(a.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    barrier()
+    t_start.record(stream)
+    for i in range(a.steps):
+        run_step(evs[i])
+    t_end.record(stream)
+    stream.synchronize()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    total_ms = max_over_ranks(t_start.elapsed_time(t_end))
+    pre_ms = max_over_ranks(statistics.mean(e[0].elapsed_time(e[1]) for e in evs))
+    dec_ms = max_over_ranks(statistics.mean(e[1].elapsed_time(e[2]) for e in evs))
+    barrier()
+    ms_step = total_ms / a.steps
+    assert tw.bitnet_device_status() == 0, "a device-side wait timed out"
+
+    M, B, Lyr = a.prefill_tokens, a.decode_batch, a.layers
+    tokens_step = (M + a.decode_steps * B)
+    value = n_gpus * tokens_step * Lyr / (ms_step / 1e3)
+
+    # ---- phase figures (per replica) ----
+    ops_layer = 2 * HIDDEN * HIDDEN * 2 + 2 * (2 * HIDDEN * INTER) + 2 * INTER * HIDDEN  # per token
+    pre_ops = M * Lyr * ops_layer
+    pre_tops = pre_ops / (pre_ms / 1e3) / 1e12
+    int8_peak_sust = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]) * \
+        NOMINAL_INT8_PER_BF16
+    pk_w = st.packed_bytes
+    act_dec = Lyr * (B * HIDDEN * 2 * 3 + B * INTER * 4 + B * HIDDEN * 4 * 3 + B * INTER * 4)
+    dec_bytes_step = pk_w + act_dec
+    dec_step_ms = dec_ms / a.decode_steps
+    dec_gbs = dec_bytes_step / (dec_step_ms / 1e3) / 1e9
+    hbm_peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    phases = {
+        "prefill_ms": pre_ms, "prefill_tops": pre_tops, "prefill_int8_peak_tops": int8_peak_sust,
+        "prefill_frac_int8": pre_tops / int8_peak_sust,
+        "prefill_tokens_per_s_per_layer": M * Lyr / (pre_ms / 1e3),
+        "decode_ms_per_step": dec_step_ms, "decode_gbs": dec_gbs, "decode_frac_hbm": dec_gbs / hbm_peak,
+        "decode_tokens_per_s_per_layer": B * Lyr / (dec_step_ms / 1e3),
+        "peaks": f"{peaks_src}: HBM {hbm_peak} GB/s; int8 = sustained bf16 x {NOMINAL_INT8_PER_BF16}",
+    }
+
+    # ---- per-kernel averages (CUDA events over graphs of one projection kind) ----
+    kinds = {}
+    R = 4
+    with torch.cuda.stream(stream):
+        specs = {
+            "decode_q_o": (lambda s: [st.q(l, st.dec_x[l % st.n_dec], st.dec_out, st.ws_dec, s)
+                                      for _ in range(R) for l in range(Lyr)],
+                           HIDDEN * HIDDEN // 4 + B * HIDDEN * 2 + B * HIDDEN * 4, "hbm", 2 * Lyr),
+            "decode_gate_up": (lambda s: [st.gate_up(l, st.dec_x[l % st.n_dec], st.dec_out, st.ws_dec, s)
+                                          for _ in range(R) for l in range(Lyr)],
+                               2 * INTER * HIDDEN // 4 + B * HIDDEN * 2 + B * INTER * 4, "hbm", Lyr),
+            "decode_down": (lambda s: [st.down(l, st.dec_out, st.ws_dec, s) for _ in range(R) for l in range(Lyr)],
+                            INTER * HIDDEN // 4 + B * INTER * 4 + B * HIDDEN * 4, "hbm", Lyr),
+            "prefill_q_o": (lambda s: [st.q(l, st.pre_x[l % st.n_pre], st.pre_out, st.ws_pre, s)
+                                       for l in range(Lyr)], 2 * M * HIDDEN * HIDDEN, "tensor", 2 * Lyr),
+            "prefill_gate_up": (lambda s: [st.gate_up(l, st.pre_x[l % st.n_pre], st.pre_out, st.ws_pre, s)
+                                           for l in range(Lyr)], 2 * 2 * M * HIDDEN * INTER, "tensor", Lyr),
+            "prefill_down": (lambda s: [st.down(l, st.pre_out, st.ws_pre, s) for l in range(Lyr)],
+                             2 * M * INTER * HIDDEN, "tensor", Lyr),
+        }
+        for name, (fn, work, bound, per_step) in specs.items():
+            c0 = tw.bitnet_launch_count()
+            g = capture(torch, stream, fn)
+            kern = tw.bitnet_launch_count() - c0
+            n_ops = R * Lyr if name.startswith("decode") else Lyr
+            ms = time_graph(torch, stream, g, 3) / n_ops
+            reps_step = per_step * (a.decode_steps if name.startswith("decode") else 1)
+            kinds[name] = {"us_per_op": ms * 1e3, "kernels_per_op": kern / n_ops, "bound": bound,
+                           "work_per_op": work, "ops_per_step": reps_step,
+                           "share_est": ms * reps_step / ms_step}
+            del g
+    dom = max(kinds, key=lambda k: kinds[k]["share_est"])
+    d = kinds[dom]
+    if d["bound"] == "hbm":
+        achieved = d["work_per_op"] / (d["us_per_op"] / 1e6) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                "frac": achieved / hbm_peak}
+    else:
+        achieved = d["work_per_op"] / (d["us_per_op"] / 1e6) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": int8_peak_sust, "unit": "TFLOP/s",
+                "frac": achieved / int8_peak_sust}
+    roof["traffic"] = dram_traffic(dom)
+    roof["kernel"] = dom
+    roof["peak_source"] = f"{peaks_src} (MEASURED_PEAKS.json)" if peaks_src == "measured" else "fallback"
+    roof["note"] = ("achieved = algorithmic bytes (packed weights + activations in + outputs) per op / "
+                    "mean op time in a CUDA graph of consecutive ops (CUDA events on the launch stream)")
+
+    # ---- end to end: pinned host inputs -> device, step, outputs -> host ----
+    e2e = None
+    if a.e2e_steps > 0:
+        h_pre = [x.cpu().pin_memory() for x in st.pre_x]
+        h_dec = [x.cpu().pin_memory() for x in st.dec_x]
+        outs = list(st.pre_out.values()) + list(st.dec_out.values())
+        h_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+        h2d = sum(x.numel() * x.element_size() for x in h_pre + h_dec)
+        d2h = sum(o.numel() * o.element_size() for o in outs)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        barrier()
+        e0.record(stream)
+        with torch.cuda.stream(stream):
+            for _ in range(a.e2e_steps):
+                for dx, hx in zip(st.pre_x + st.dec_x, h_pre + h_dec):
+                    dx.copy_(hx, non_blocking=True)
+                run_step()
+                for ho, o in zip(h_out, outs):
+                    ho.copy_(o, non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / a.e2e_steps
+        e2e = {"value": n_gpus * tokens_step * Lyr / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+
+    cpu = None
+    if rank == 0 and n_gpus == 1 and not a.no_cpu_baseline:
+        cpu = cpu_baseline(a.cpu_seconds)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": n_gpus, "steps": a.steps,
+            "warmup": a.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int8", "data": "synthetic (seeded random activations and latents)",
+            "config": workload_config(a, n_gpus), "phases": phases, "roofline": roof, "kernels": kinds,
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int((launches_pre + launches_dec) * a.steps),
+            "gpu_launches_per_step": {"prefill": int(launches_pre), "decode": int(launches_dec)},
+            "clocks": clk, "gpu": torch.cuda.get_device_name(dev),
+        }
+        print(json.dumps(line), flush=True)
+    del g_pre, g_dec
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    a = parse_args()
+    n_gpus = int(os.environ.get("WORLD_SIZE", str(a.gpus)))
+    if a.impl == "reference":
+        return reference_arm(a, n_gpus)
+    return our_arm(a, n_gpus)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,217 @@
+/*
+ * bitnet.h -- C ABI of the B200 (sm_100a) BitLinear forward library.
+ *
+ * The operation is the BitLinear layer of BitNet b1.58 as the "BitNet" model
+ * page of the transformers documentation describes it (section "Model
+ * details", items "Architecture" and "Quantization"): weights quantised to
+ * {-1, 0, +1} by absmean quantisation, activations quantised to 8-bit integers
+ * by per-token absmax quantisation (W1.58A8), no bias, and a squared-ReLU FFN
+ * (BitNetConfig: hidden_act = "relu2").  The page gives no formulas; the ones
+ * implemented here are
+ *
+ *   gamma = mean |W|                       (one per weight matrix, fp32)
+ *   W_q   = clamp(rne(W / (gamma + eps)), -1, 1)
+ *   s_m   = 127 / max(max_k |x_mk|, 1e-5)  (one per token = row of x, fp32)
+ *   x_q   = clamp(rne(x * s_m), -128, 127)
+ *   acc   = x_q . W_q^T                    (exact int32)
+ *   y     = (float)acc * (gamma / s_m)     (fp32)
+ *   h     = (g > 0 ? g*g : 0) * u          (gate/up FFN, g and u two BitLinear outputs)
+ *
+ * rne = round half to even.  The quantisers use IEEE fp32 division and one
+ * rounded fp32 product, so their integer results are reproducible exactly.
+ *
+ * Layouts (all row-major, C order):
+ *   x         [M][K]   bf16 or fp32 activations (M tokens, K input features)
+ *   W latent  [N][K]   fp32 (N output features)
+ *   w_packed  [N][K/4] uint8: code c = W_q + 1 in {0,1,2}; within row n the
+ *             little-endian 32-bit word at byte 4*g holds weights
+ *             k = 16g .. 16g+15, weight 16g + 4j + b in byte b, bits 2j..2j+1
+ *   x_q       [M][K]   int8
+ *   y, h      [M][N]   fp32
+ *   acc       [M][N]   int32
+ *
+ * Conventions for every entry point:
+ *   - Pointers are DEVICE pointers unless stated otherwise; the caller owns all
+ *     memory.  The library never allocates or frees device memory and never
+ *     synchronises the stream; work is enqueued on `stream` and runs
+ *     asynchronously.
+ *   - Arguments are validated on the host before anything is launched; on any
+ *     error nothing is launched and the status says why.  After launching,
+ *     a launch error reported by the CUDA runtime is returned as
+ *     BITNET_ERR_CUDA.  Faults that happen later, while the kernels run, are
+ *     reported by the CUDA runtime on the next synchronising call.
+ *   - Shapes: M >= 1, N >= 1, K >= 64 with K % 64 == 0.  Every pointer must be
+ *     16-byte aligned.
+ *   - Inputs must be finite (not checked).
+ *   - Reads of w_packed and gamma may begin before earlier work on the same
+ *     stream has finished (programmatic dependent launch): they must not be
+ *     written by work still in flight on that stream.  Pack, then synchronise
+ *     (or wait on an event) before the first call that reads the result.
+ *     Everything else obeys normal stream order.
+ */
+#ifndef BITNET_H
+#define BITNET_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    BITNET_OK = 0,
+    BITNET_ERR_INVALID_ARG = 1,       /* null pointer, non-positive size, bad enum */
+    BITNET_ERR_UNSUPPORTED_SHAPE = 2, /* K not a positive multiple of 64, sizes too large */
+    BITNET_ERR_MISALIGNED = 3,        /* a pointer is not 16-byte aligned */
+    BITNET_ERR_CUDA = 4,              /* the CUDA runtime reported an error */
+    BITNET_ERR_TIMEOUT = 5,           /* a device-side wait gave up (see bitnet_device_status) */
+    BITNET_ERR_WORKSPACE = 6          /* workspace pointer null or too small */
+} bitnet_status_t;
+
+typedef enum {
+    BITNET_DTYPE_BF16 = 0,
+    BITNET_DTYPE_F32 = 1
+} bitnet_dtype_t;
+
+/* Kernel selection for bitnet_linear / bitnet_ffn_gate_up. */
+typedef enum {
+    BITNET_DISPATCH_AUTO = 0,         /* by M: decode kernels for M <= 64, else prefill */
+    BITNET_DISPATCH_DECODE_FUSED = 1, /* decode kernel quantising x itself (M <= 64) */
+    BITNET_DISPATCH_DECODE = 2,       /* quantiser kernel + decode kernel (M <= 64) */
+    BITNET_DISPATCH_PREFILL = 3       /* quantiser kernel + tcgen05 GEMM (any M) */
+} bitnet_dispatch_t;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *bitnet_status_string(bitnet_status_t status);
+
+/* ABI version of this library: major * 10000 + minor * 100 + patch. */
+int bitnet_version(void);
+
+/*
+ * Workspace needed by bitnet_pack_weights for an [N][K] matrix: N * 8 bytes
+ * (one fp64 partial sum per row).
+ */
+size_t bitnet_pack_workspace_size(int64_t N, int64_t K);
+
+/*
+ * Offline absmean ternarisation and 2-bit packing of one weight matrix
+ * (page: "Quantization" -- ternary {-1, 0, +1} weights by absmean; "Model
+ * variants" -- the deployable weights are stored packed).
+ *
+ *   w          [N][K] fp32 latent weights (device, read)
+ *   eps        additive epsilon of gamma + eps (1e-5 in BitNet b1.58)
+ *   w_packed   [N][K/4] uint8 packed codes (device, written)
+ *   gamma      [1] fp32 (device, written): mean |W|, accumulated in fp64 in a
+ *              fixed order (each row left to right, then the rows top to
+ *              bottom) and rounded once to fp32
+ *   workspace  device scratch of bitnet_pack_workspace_size(N, K) bytes
+ *
+ * Deterministic: identical inputs give identical bytes on every run.
+ */
+bitnet_status_t bitnet_pack_weights(const float *w, int64_t N, int64_t K, float eps,
+                                    uint8_t *w_packed, float *gamma,
+                                    void *workspace, size_t ws_bytes,
+                                    cudaStream_t stream);
+
+/*
+ * Per-token absmax int8 quantisation of activations (page: "Quantization" --
+ * 8-bit activations by absmax, per token).
+ *
+ *   x        [M][K] activations of type x_dtype (device, read)
+ *   x_q      [M][K] int8 (device, written)
+ *   s        [M] fp32 per-token scales s_m = 127 / max(max|x_m|, 1e-5) (device, written)
+ *   rowsum   [M] int32 sum_k x_q[m][k] (device, written; may be NULL)
+ */
+bitnet_status_t bitnet_quant_act(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_t K,
+                                 int8_t *x_q, float *s, int32_t *rowsum,
+                                 cudaStream_t stream);
+
+/*
+ * Workspace needed by bitnet_linear / bitnet_ffn_gate_up for the given shape
+ * (holds the quantised activations, scales and row sums between kernels).
+ */
+size_t bitnet_workspace_size(int64_t M, int64_t N, int64_t K);
+
+/*
+ * BitLinear forward y = dequant(quant(x) . W_q^T) (page: "Architecture" --
+ * BitLinear layers without bias; "Quantization" -- W1.58A8).
+ *
+ *   x          [M][K] activations of type x_dtype (device, read)
+ *   w_packed   [N][K/4] packed ternary weights from bitnet_pack_weights
+ *   gamma      [1] fp32 weight scale from bitnet_pack_weights (device)
+ *   y          [M][N] fp32 output (device, written)
+ *   x_q_out    [M][K] int8 quantised activations (optional, may be NULL)
+ *   s_out      [M] fp32 per-token scales (optional, may be NULL)
+ *   acc_out    [M][N] int32 exact accumulators (optional, may be NULL)
+ *   workspace  device scratch of at least bitnet_workspace_size(M, N, K) bytes
+ *
+ * Small M (decode) streams the packed weights through a GEMV-style kernel;
+ * large M (prefill) runs a tcgen05 int8 tensor-core GEMM.  Both give
+ * bit-identical results.
+ */
+bitnet_status_t bitnet_linear(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_t K,
+                              const uint8_t *w_packed, const float *gamma, int64_t N,
+                              float *y, int8_t *x_q_out, float *s_out, int32_t *acc_out,
+                              void *workspace, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * Gate/up half of the BitNet FFN with the squared-ReLU gate fused in the
+ * epilogue (page: "Architecture" -- ReLU^2 in the FFN; BitNetConfig
+ * hidden_act = "relu2"):
+ *   g = BitLinear_gate(x), u = BitLinear_up(x), h = relu(g)^2 * u.
+ * Both projections share one quantisation of x.
+ *
+ *   x            [M][K] activations (device, read)
+ *   wg_packed    [N][K/4], gamma_g [1]: gate projection
+ *   wu_packed    [N][K/4], gamma_u [1]: up projection
+ *   h            [M][N] fp32 output (device, written)
+ *   acc_g_out, acc_u_out  [M][N] int32 accumulators (optional, may be NULL)
+ *   workspace    as for bitnet_linear
+ *
+ * The down projection is a plain bitnet_linear call with x = h
+ * (x_dtype = BITNET_DTYPE_F32), which quantises h per token again.
+ */
+bitnet_status_t bitnet_ffn_gate_up(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_t K,
+                                   const uint8_t *wg_packed, const float *gamma_g,
+                                   const uint8_t *wu_packed, const float *gamma_u, int64_t N,
+                                   float *h, int32_t *acc_g_out, int32_t *acc_u_out,
+                                   void *workspace, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * Device-side status word.  Kernels whose waits are bounded record
+ * BITNET_ERR_TIMEOUT there (and exit) instead of spinning forever.  This call
+ * synchronises `stream`, copies the word to *status_out and, if clear != 0,
+ * resets it to BITNET_OK.  Returns BITNET_ERR_CUDA if the copy fails.
+ */
+bitnet_status_t bitnet_device_status(int clear, bitnet_status_t *status_out, cudaStream_t stream);
+
+/*
+ * Number of SMs the library sizes its grids for on the current device
+ * (queried once per device).  Returns 0 on error.
+ */
+int bitnet_num_sms(void);
+
+/*
+ * Process-wide kernel selection (a bitnet_dispatch_t value); every selection
+ * computes bit-identical results.  Returns the previous value, or -1 if the
+ * value is not a bitnet_dispatch_t (nothing changed).  A forced decode
+ * selection makes calls with M > 64 (or a K too large for the decode
+ * kernel) return BITNET_ERR_UNSUPPORTED_SHAPE.  Intended for tests and
+ * benchmarks; not synchronised with calls running in other threads.
+ */
+int bitnet_set_dispatch(int dispatch);
+
+/*
+ * Number of kernel launches this library has issued in this process (all
+ * devices, including launches recorded into CUDA graphs during capture).
+ * Monotonic; for measuring how many kernels a sequence of calls enqueues.
+ */
+uint64_t bitnet_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BITNET_H */

@@ -1,0 +1,202 @@
+"""B200-native BitLinear forward (BitNet b1.58, W1.58A8).
+
+Thin Python binding over the C ABI in ``include/bitnet.h`` (library
+``libbitnet_b200.so`` built in-tree by ``ternary_weight_fwd_b200.build``).
+The functions keep the C names; this module only marshals arguments:
+PyTorch tensors are used for device memory and streams, every step of the
+computation runs in the library's CUDA kernels.  There is no fallback: if the
+library is missing the call raises.
+"""
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbitnet_b200.so")
+
+BITNET_OK = 0
+BITNET_ERR_INVALID_ARG = 1
+BITNET_ERR_UNSUPPORTED_SHAPE = 2
+BITNET_ERR_MISALIGNED = 3
+BITNET_ERR_CUDA = 4
+BITNET_ERR_TIMEOUT = 5
+BITNET_ERR_WORKSPACE = 6
+
+BITNET_DTYPE_BF16 = 0
+BITNET_DTYPE_F32 = 1
+
+BITNET_DISPATCH_AUTO = 0
+BITNET_DISPATCH_DECODE_FUSED = 1
+BITNET_DISPATCH_DECODE = 2
+BITNET_DISPATCH_PREFILL = 3
+
+QUANT_EPS = 1e-5
+
+_lib = None
+
+
+class BitnetError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        super().__init__(f"{where}: {bitnet_status_string(status)} ({status})")
+
+
+def load_library(path: str = LIB_PATH):
+    """Load and declare the C ABI.  Raises if the library has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"CUDA library {path} is missing; build it with "
+                           "`python -m ternary_weight_fwd_b200.build` (no CPU fallback exists)")
+    lib = ctypes.CDLL(path)
+    P, I64, SZ, I, F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_int, ctypes.c_float
+    sig = {
+        "bitnet_status_string": ([I], ctypes.c_char_p),
+        "bitnet_version": ([], I),
+        "bitnet_pack_workspace_size": ([I64, I64], SZ),
+        "bitnet_pack_weights": ([P, I64, I64, F, P, P, P, SZ, P], I),
+        "bitnet_quant_act": ([P, I, I64, I64, P, P, P, P], I),
+        "bitnet_workspace_size": ([I64, I64, I64], SZ),
+        "bitnet_linear": ([P, I, I64, I64, P, P, I64, P, P, P, P, P, SZ, P], I),
+        "bitnet_ffn_gate_up": ([P, I, I64, I64, P, P, P, P, I64, P, P, P, P, SZ, P], I),
+        "bitnet_device_status": ([I, ctypes.POINTER(ctypes.c_int), P], I),
+        "bitnet_num_sms": ([], I),
+        "bitnet_set_dispatch": ([I], I),
+        "bitnet_launch_count": ([], ctypes.c_uint64),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    _lib = lib
+    return lib
+
+
+def _check(status, where):
+    if status != BITNET_OK:
+        raise BitnetError(status, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(x):
+    if x.dtype == torch.bfloat16:
+        return BITNET_DTYPE_BF16
+    if x.dtype == torch.float32:
+        return BITNET_DTYPE_F32
+    raise TypeError(f"activations must be bfloat16 or float32, got {x.dtype}")
+
+
+def bitnet_status_string(status: int) -> str:
+    return load_library().bitnet_status_string(int(status)).decode()
+
+
+def bitnet_version() -> int:
+    return load_library().bitnet_version()
+
+
+def bitnet_num_sms() -> int:
+    return load_library().bitnet_num_sms()
+
+
+def bitnet_set_dispatch(dispatch: int) -> int:
+    prev = load_library().bitnet_set_dispatch(int(dispatch))
+    if prev < 0:
+        raise ValueError(f"invalid dispatch {dispatch}")
+    return prev
+
+
+def bitnet_launch_count() -> int:
+    return load_library().bitnet_launch_count()
+
+
+def bitnet_pack_workspace_size(n: int, k: int) -> int:
+    return load_library().bitnet_pack_workspace_size(n, k)
+
+
+def bitnet_workspace_size(m: int, n: int, k: int) -> int:
+    return load_library().bitnet_workspace_size(m, n, k)
+
+
+def bitnet_pack_weights(w, eps=QUANT_EPS, *, w_packed=None, gamma=None, workspace=None, stream=None):
+    """fp32 latent [N][K] -> (packed uint8 [N][K/4], gamma fp32 [1])."""
+    lib = load_library()
+    n, k = w.shape
+    if w_packed is None:
+        w_packed = torch.empty((n, k // 4), dtype=torch.uint8, device=w.device)
+    if gamma is None:
+        gamma = torch.empty(4, dtype=torch.float32, device=w.device)[:1]
+    ws_bytes = lib.bitnet_pack_workspace_size(n, k)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=w.device)
+    _check(lib.bitnet_pack_weights(_ptr(w), n, k, float(eps), _ptr(w_packed), _ptr(gamma), _ptr(workspace),
+                                   workspace.numel(), _stream(stream)), "bitnet_pack_weights")
+    return w_packed, gamma
+
+
+def bitnet_quant_act(x, *, x_q=None, s=None, rowsum=None, want_rowsum=True, stream=None):
+    """[M][K] bf16/fp32 -> (x_q int8 [M][K], s fp32 [M], rowsum int32 [M] or None)."""
+    lib = load_library()
+    m, k = x.shape
+    if x_q is None:
+        x_q = torch.empty((m, k), dtype=torch.int8, device=x.device)
+    if s is None:
+        s = torch.empty(m, dtype=torch.float32, device=x.device)
+    if rowsum is None and want_rowsum:
+        rowsum = torch.empty(m, dtype=torch.int32, device=x.device)
+    _check(lib.bitnet_quant_act(_ptr(x), _dtype_code(x), m, k, _ptr(x_q), _ptr(s), _ptr(rowsum),
+                                _stream(stream)), "bitnet_quant_act")
+    return x_q, s, rowsum
+
+
+def _workspace(workspace, m, n, k, device):
+    need = load_library().bitnet_workspace_size(m, n, k)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=device)
+    return workspace
+
+
+def bitnet_linear(x, w_packed, gamma, *, y=None, x_q_out=None, s_out=None, acc_out=None, workspace=None,
+                  stream=None):
+    """y [M][N] fp32 = BitLinear(x) with packed ternary weights."""
+    lib = load_library()
+    m, k = x.shape
+    n = w_packed.shape[0]
+    if y is None:
+        y = torch.empty((m, n), dtype=torch.float32, device=x.device)
+    workspace = _workspace(workspace, m, n, k, x.device)
+    _check(lib.bitnet_linear(_ptr(x), _dtype_code(x), m, k, _ptr(w_packed), _ptr(gamma), n, _ptr(y),
+                             _ptr(x_q_out), _ptr(s_out), _ptr(acc_out), _ptr(workspace), workspace.numel(),
+                             _stream(stream)), "bitnet_linear")
+    return y
+
+
+def bitnet_ffn_gate_up(x, wg_packed, gamma_g, wu_packed, gamma_u, *, h=None, acc_g_out=None, acc_u_out=None,
+                       workspace=None, stream=None):
+    """h [M][N] fp32 = relu(BitLinear_g(x))^2 * BitLinear_u(x)."""
+    lib = load_library()
+    m, k = x.shape
+    n = wg_packed.shape[0]
+    if h is None:
+        h = torch.empty((m, n), dtype=torch.float32, device=x.device)
+    workspace = _workspace(workspace, m, n, k, x.device)
+    _check(lib.bitnet_ffn_gate_up(_ptr(x), _dtype_code(x), m, k, _ptr(wg_packed), _ptr(gamma_g), _ptr(wu_packed),
+                                  _ptr(gamma_u), n, _ptr(h), _ptr(acc_g_out), _ptr(acc_u_out), _ptr(workspace),
+                                  workspace.numel(), _stream(stream)), "bitnet_ffn_gate_up")
+    return h
+
+
+def bitnet_device_status(clear=True, stream=None) -> int:
+    out = ctypes.c_int(0)
+    _check(load_library().bitnet_device_status(1 if clear else 0, ctypes.byref(out), _stream(stream)),
+           "bitnet_device_status")
+    return out.value

@@ -1,0 +1,462 @@
+// bitnet.cu -- C ABI of the BitLinear forward library (the only translation
+// unit; the kernels live in the .cuh files included below).
+//
+// Host side: argument validation (before anything is launched), kernel
+// selection by M, TMA descriptor encoding, and launches with programmatic
+// dependent launch so consecutive kernels overlap their prologues.
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <utility>
+
+#include "bitnet.h"
+#include "common.cuh"
+#include "decode.cuh"
+#include "pack_quant.cuh"
+#include "prefill.cuh"
+
+namespace bitnet {
+
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int64_t kMaxDim = int64_t(1) << 24;
+constexpr int64_t kMaxK = 65536;
+constexpr int kDecodeMaxM = 64;
+constexpr size_t kSmemLimit = 227 * 1024;
+// Up to this many activation elements (M*K) the decode kernel quantises x in
+// every CTA instead of running the quantiser kernel first.
+constexpr int64_t kFusedQuantMaxElems = 8192;
+
+std::atomic<int> g_dispatch{BITNET_DISPATCH_AUTO};
+std::atomic<uint64_t> g_launches{0};
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+int current_device()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    return dev;
+}
+
+int num_sms_for(int dev)
+{
+    static std::atomic<int> cache[kMaxDevices];
+    if (dev < 0 || dev >= kMaxDevices) return 0;
+    int v = cache[dev].load();
+    if (v > 0) return v;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cache[dev].store(v);
+    return v;
+}
+
+// Raise the dynamic shared-memory limit of a kernel once per device.
+template <typename Kern>
+cudaError_t ensure_smem(Kern *kern, size_t bytes, std::atomic<int> (&done)[kMaxDevices], int dev)
+{
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    if (done[dev].load() >= (int)bytes) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemLimit);
+    if (e == cudaSuccess) done[dev].store((int)kSmemLimit);
+    return e;
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+bitnet_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA; }
+
+bitnet_status_t check_shape(int64_t M, int64_t N, int64_t K)
+{
+    if (M < 1 || N < 1 || K < 1) return BITNET_ERR_INVALID_ARG;
+    if (K % 64 != 0 || K > kMaxK || M > kMaxDim || N > kMaxDim) return BITNET_ERR_UNSUPPORTED_SHAPE;
+    return BITNET_OK;
+}
+
+// ---- workspace layout shared by linear / ffn -------------------------------
+struct Workspace {
+    int8_t *xq;
+    float *s;
+    int32_t *rs;
+};
+
+size_t ws_bytes_for(int64_t M, int64_t K)
+{
+    return align_up((size_t)M * (size_t)K, 256) + 2 * align_up((size_t)M * 4, 256);
+}
+
+Workspace carve(void *ws, int64_t M, int64_t K)
+{
+    char *p = static_cast<char *>(ws);
+    Workspace w;
+    w.xq = reinterpret_cast<int8_t *>(p);
+    p += align_up((size_t)M * (size_t)K, 256);
+    w.s = reinterpret_cast<float *>(p);
+    p += align_up((size_t)M * 4, 256);
+    w.rs = reinterpret_cast<int32_t *>(p);
+    return w;
+}
+
+// ---- TMA descriptors ---------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 2-D uint8 tensor [rows][cols] (row pitch = cols bytes), box [box_rows][box_cols].
+bool encode_u8_2d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows,
+                  uint32_t box_cols, bool swizzle128)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// ---- decode configuration -----------------------------------------------------
+struct DecodeCfg {
+    bool ok;
+    int grid, rg, w_stride, x_stride, rp, ch;
+    size_t smem;
+};
+
+DecodeCfg decode_config(int64_t M, int64_t N, int64_t K, int nmat, bool fused, int sms)
+{
+    DecodeCfg c = {};
+    c.w_stride = (int)(K / 4 + ((16 - (K / 4) % 128) + 128) % 128);
+    c.x_stride = (int)(K + ((64 - K % 128) + 128) % 128);
+    int64_t grid = std::min<int64_t>(sms, cdiv(N, 16));
+    for (;;) {
+        const int64_t rmax = cdiv(N, grid);
+        const int rg = (int)cdiv(rmax, 16);
+        if (rg > DEC_RGM) {
+            grid = cdiv(N, 16 * DEC_RGM);
+            continue;
+        }
+        const int rp = rg * 16 + ((4 - (rg * 16) % 32) + 32) % 32;
+        const size_t smem = DEC_HDR + (size_t)nmat * rg * 16 * c.w_stride + (size_t)nmat * 8 * rp * 4 +
+                            (fused ? (size_t)8 * c.x_stride : 0);
+        if (smem > kSmemLimit) {
+            if (rg == 1) return c; // K too large for the decode kernel
+            grid = cdiv(N, 16 * (rg - 1));
+            continue;
+        }
+        c.grid = (int)grid;
+        c.rg = rg;
+        c.rp = rp;
+        c.smem = smem;
+        break;
+    }
+    const int64_t steps = cdiv(K / 64, DEC_WARPS);
+    c.ch = steps <= 4 ? 4 : (steps <= 8 ? 8 : 16);
+    c.ok = true;
+    return c;
+}
+
+template <int NMAT, bool FUSED, bool XF32, int CH>
+cudaError_t launch_decode_t(const DecodeArgs &a, const DecodeCfg &c, cudaStream_t stream, int dev)
+{
+    static std::atomic<int> done[kMaxDevices];
+    auto kern = k_decode<NMAT, FUSED, XF32, CH>;
+    cudaError_t e = ensure_smem(kern, c.smem, done, dev);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(kern, dim3(c.grid), dim3(DEC_THREADS), c.smem, stream, a);
+}
+
+template <int NMAT>
+cudaError_t launch_decode(const DecodeArgs &a, const DecodeCfg &c, bool fused, bool xf32, cudaStream_t stream,
+                          int dev)
+{
+    if (fused) {
+        return xf32 ? launch_decode_t<NMAT, true, true, 4>(a, c, stream, dev)
+                    : launch_decode_t<NMAT, true, false, 4>(a, c, stream, dev);
+    }
+    switch (c.ch) {
+    case 4: return launch_decode_t<NMAT, false, false, 4>(a, c, stream, dev);
+    case 8: return launch_decode_t<NMAT, false, false, 8>(a, c, stream, dev);
+    default: return launch_decode_t<NMAT, false, false, 16>(a, c, stream, dev);
+    }
+}
+
+cudaError_t launch_quant(const void *x, bool xf32, int64_t M, int64_t K, int8_t *xq, float *s, int32_t *rs,
+                         cudaStream_t stream)
+{
+    const dim3 grid((unsigned)cdiv(M, 8));
+    if (xf32) return launch_pdl(k_quant_rows<true>, grid, dim3(256), 0, stream, x, M, K, xq, s, rs);
+    return launch_pdl(k_quant_rows<false>, grid, dim3(256), 0, stream, x, M, K, xq, s, rs);
+}
+
+bool use_decode(int64_t M, int dispatch)
+{
+    if (dispatch == BITNET_DISPATCH_PREFILL) return false;
+    if (dispatch == BITNET_DISPATCH_DECODE || dispatch == BITNET_DISPATCH_DECODE_FUSED) return M <= kDecodeMaxM;
+    return M <= kDecodeMaxM;
+}
+
+bool use_fused(int64_t M, int64_t K, int dispatch)
+{
+    if (dispatch == BITNET_DISPATCH_DECODE_FUSED) return true;
+    if (dispatch == BITNET_DISPATCH_DECODE) return false;
+    return M * K <= kFusedQuantMaxElems;
+}
+
+// Shared body of bitnet_linear (nmat = 1) and bitnet_ffn_gate_up (nmat = 2).
+bitnet_status_t forward(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_t K, const uint8_t *w0,
+                        const float *gamma0, const uint8_t *w1, const float *gamma1, int64_t N, float *y,
+                        int8_t *x_q_out, float *s_out, int32_t *acc0, int32_t *acc1, void *workspace,
+                        size_t ws_bytes, cudaStream_t stream, int nmat)
+{
+    bitnet_status_t st = check_shape(M, N, K);
+    if (st != BITNET_OK) return st;
+    if (x_dtype != BITNET_DTYPE_BF16 && x_dtype != BITNET_DTYPE_F32) return BITNET_ERR_INVALID_ARG;
+    if (!x || !w0 || !gamma0 || !y || (nmat == 2 && (!w1 || !gamma1))) return BITNET_ERR_INVALID_ARG;
+    const void *ptrs[] = {x, w0, gamma0, w1, gamma1, y, x_q_out, s_out, acc0, acc1, workspace};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return BITNET_ERR_MISALIGNED;
+    if (!workspace || ws_bytes < ws_bytes_for(M, K)) return BITNET_ERR_WORKSPACE;
+    const int dev = current_device();
+    const int sms = num_sms_for(dev);
+    if (sms <= 0) return BITNET_ERR_CUDA;
+    const bool xf32 = x_dtype == BITNET_DTYPE_F32;
+    const int dispatch = g_dispatch.load();
+    Workspace ws = carve(workspace, M, K);
+    int8_t *xq = x_q_out ? x_q_out : ws.xq;
+    float *s = s_out ? s_out : ws.s;
+
+    if (use_decode(M, dispatch)) {
+        bool fused = use_fused(M, K, dispatch);
+        DecodeCfg c = decode_config(M, N, K, nmat, fused, sms);
+        if (!c.ok && fused) {
+            fused = false;
+            c = decode_config(M, N, K, nmat, false, sms);
+        }
+        if (c.ok) {
+            DecodeArgs a = {};
+            a.x = x;
+            a.xq = xq;
+            a.s_in = s;
+            a.rs_in = ws.rs;
+            a.w0 = w0;
+            a.w1 = w1;
+            a.gamma0 = gamma0;
+            a.gamma1 = gamma1;
+            a.y = y;
+            a.acc0 = acc0;
+            a.acc1 = acc1;
+            a.xq_out = fused ? x_q_out : nullptr;
+            a.s_out = fused ? s_out : nullptr;
+            a.M = (int)M;
+            a.N = (int)N;
+            a.K = (int)K;
+            a.grid = c.grid;
+            a.rg = c.rg;
+            a.w_stride = c.w_stride;
+            a.x_stride = c.x_stride;
+            a.rp = c.rp;
+            cudaError_t e = cudaSuccess;
+            if (!fused) e = launch_quant(x, xf32, M, K, xq, s, ws.rs, stream);
+            if (e == cudaSuccess)
+                e = nmat == 1 ? launch_decode<1>(a, c, fused, xf32, stream, dev)
+                              : launch_decode<2>(a, c, fused, xf32, stream, dev);
+            return cuda_status(e);
+        }
+        if (dispatch != BITNET_DISPATCH_AUTO) return BITNET_ERR_UNSUPPORTED_SHAPE;
+    }
+
+    // ---- prefill: quantiser kernel, then the tcgen05 GEMM ----
+    PrefillArgs a = {};
+    a.M = (int)M;
+    a.N = (int)N;
+    a.K = (int)K;
+    a.num_m = (int)cdiv(M, PF_BM);
+    a.num_n = (int)cdiv(N, nmat == 1 ? PF_BN : PF_BN / 2);
+    a.num_k = (int)cdiv(K, PF_BK);
+    a.num_tiles = a.num_m * a.num_n;
+    a.gamma0 = gamma0;
+    a.gamma1 = gamma1;
+    a.s = s;
+    a.y = y;
+    a.acc0 = acc0;
+    a.acc1 = acc1;
+    a.vec_ok = (N % 4) == 0;
+    CUtensorMap tmA, tmB0, tmB1;
+    const uint32_t brows = nmat == 1 ? PF_BN : PF_BN / 2;
+    if (!encode_u8_2d(&tmA, xq, (uint64_t)M, (uint64_t)K, PF_BM, PF_BK, true) ||
+        !encode_u8_2d(&tmB0, w0, (uint64_t)N, (uint64_t)(K / 4), brows, PF_BK / 4, false))
+        return BITNET_ERR_CUDA;
+    if (nmat == 2) {
+        if (!encode_u8_2d(&tmB1, w1, (uint64_t)N, (uint64_t)(K / 4), brows, PF_BK / 4, false))
+            return BITNET_ERR_CUDA;
+    } else {
+        tmB1 = tmB0;
+    }
+    cudaError_t e = launch_quant(x, xf32, M, K, xq, s, nullptr, stream);
+    if (e != cudaSuccess) return BITNET_ERR_CUDA;
+    const int grid = std::min(a.num_tiles, sms);
+    if (nmat == 1) {
+        static std::atomic<int> done[kMaxDevices];
+        e = ensure_smem(k_prefill<false>, PF_SMEM, done, dev);
+        if (e == cudaSuccess)
+            e = launch_pdl(k_prefill<false>, dim3(grid), dim3(PF_THREADS), PF_SMEM, stream, tmA, tmB0, tmB1, a);
+    } else {
+        static std::atomic<int> done[kMaxDevices];
+        e = ensure_smem(k_prefill<true>, PF_SMEM, done, dev);
+        if (e == cudaSuccess)
+            e = launch_pdl(k_prefill<true>, dim3(grid), dim3(PF_THREADS), PF_SMEM, stream, tmA, tmB0, tmB1, a);
+    }
+    return cuda_status(e);
+}
+
+} // namespace
+} // namespace bitnet
+
+using namespace bitnet;
+
+extern "C" {
+
+const char *bitnet_status_string(bitnet_status_t status)
+{
+    switch (status) {
+    case BITNET_OK: return "BITNET_OK";
+    case BITNET_ERR_INVALID_ARG: return "BITNET_ERR_INVALID_ARG";
+    case BITNET_ERR_UNSUPPORTED_SHAPE: return "BITNET_ERR_UNSUPPORTED_SHAPE";
+    case BITNET_ERR_MISALIGNED: return "BITNET_ERR_MISALIGNED";
+    case BITNET_ERR_CUDA: return "BITNET_ERR_CUDA";
+    case BITNET_ERR_TIMEOUT: return "BITNET_ERR_TIMEOUT";
+    case BITNET_ERR_WORKSPACE: return "BITNET_ERR_WORKSPACE";
+    }
+    return "BITNET_ERR_UNKNOWN";
+}
+
+int bitnet_version(void) { return 100; }
+
+size_t bitnet_pack_workspace_size(int64_t N, int64_t K)
+{
+    (void)K;
+    return N > 0 ? (size_t)N * sizeof(double) : 0;
+}
+
+bitnet_status_t bitnet_pack_weights(const float *w, int64_t N, int64_t K, float eps, uint8_t *w_packed,
+                                    float *gamma, void *workspace, size_t ws_bytes, cudaStream_t stream)
+{
+    if (!w || !w_packed || !gamma) return BITNET_ERR_INVALID_ARG;
+    bitnet_status_t st = check_shape(1, N, K);
+    if (st != BITNET_OK) return st;
+    if (!(eps >= 0.0f) || !std::isfinite(eps)) return BITNET_ERR_INVALID_ARG;
+    if (!aligned16(w) || !aligned16(w_packed) || !aligned16(gamma) || (workspace && !aligned16(workspace)))
+        return BITNET_ERR_MISALIGNED;
+    if (!workspace || ws_bytes < bitnet_pack_workspace_size(N, K)) return BITNET_ERR_WORKSPACE;
+    double *rowsum = static_cast<double *>(workspace);
+    g_launches.fetch_add(3, std::memory_order_relaxed);
+    k_pack_rowsum<<<(unsigned)cdiv(N, 128), 128, 0, stream>>>(w, N, K, rowsum);
+    k_pack_gamma<<<1, 1, 0, stream>>>(rowsum, N, K, gamma);
+    const int64_t nwords = N * K / 16;
+    k_pack_codes<<<(unsigned)cdiv(nwords, 256), 256, 0, stream>>>(w, nwords, eps, gamma,
+                                                                   reinterpret_cast<uint32_t *>(w_packed));
+    return cuda_status(cudaGetLastError());
+}
+
+bitnet_status_t bitnet_quant_act(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_t K, int8_t *x_q, float *s,
+                                 int32_t *rowsum, cudaStream_t stream)
+{
+    bitnet_status_t st = check_shape(M, 1, K);
+    if (st != BITNET_OK) return st;
+    if (x_dtype != BITNET_DTYPE_BF16 && x_dtype != BITNET_DTYPE_F32) return BITNET_ERR_INVALID_ARG;
+    if (!x || !x_q || !s) return BITNET_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(x_q) || !aligned16(s) || (rowsum && !aligned16(rowsum)))
+        return BITNET_ERR_MISALIGNED;
+    return cuda_status(launch_quant(x, x_dtype == BITNET_DTYPE_F32, M, K, x_q, s, rowsum, stream));
+}
+
+size_t bitnet_workspace_size(int64_t M, int64_t N, int64_t K)
+{
+    (void)N;
+    if (M < 1 || K < 1) return 0;
+    return ws_bytes_for(M, K);
+}
+
+bitnet_status_t bitnet_linear(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_t K, const uint8_t *w_packed,
+                              const float *gamma, int64_t N, float *y, int8_t *x_q_out, float *s_out,
+                              int32_t *acc_out, void *workspace, size_t ws_bytes, cudaStream_t stream)
+{
+    return forward(x, x_dtype, M, K, w_packed, gamma, nullptr, nullptr, N, y, x_q_out, s_out, acc_out, nullptr,
+                   workspace, ws_bytes, stream, 1);
+}
+
+bitnet_status_t bitnet_ffn_gate_up(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_t K,
+                                   const uint8_t *wg_packed, const float *gamma_g, const uint8_t *wu_packed,
+                                   const float *gamma_u, int64_t N, float *h, int32_t *acc_g_out,
+                                   int32_t *acc_u_out, void *workspace, size_t ws_bytes, cudaStream_t stream)
+{
+    return forward(x, x_dtype, M, K, wg_packed, gamma_g, wu_packed, gamma_u, N, h, nullptr, nullptr, acc_g_out,
+                   acc_u_out, workspace, ws_bytes, stream, 2);
+}
+
+bitnet_status_t bitnet_device_status(int clear, bitnet_status_t *status_out, cudaStream_t stream)
+{
+    if (!status_out) return BITNET_ERR_INVALID_ARG;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return BITNET_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int)) != cudaSuccess) return BITNET_ERR_CUDA;
+    *status_out = static_cast<bitnet_status_t>(v);
+    if (clear) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) return BITNET_ERR_CUDA;
+    }
+    return BITNET_OK;
+}
+
+int bitnet_num_sms(void) { return num_sms_for(current_device()); }
+
+uint64_t bitnet_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int bitnet_set_dispatch(int dispatch)
+{
+    if (dispatch < BITNET_DISPATCH_AUTO || dispatch > BITNET_DISPATCH_PREFILL) return -1;
+    return g_dispatch.exchange(dispatch);
+}
+
+} // extern "C"

@@ -1,0 +1,258 @@
+// common.cuh -- sm_100a PTX helpers shared by the BitLinear kernels.
+//
+// Everything here is a thin wrapper over one documented PTX instruction
+// (mbarrier, bulk/tensor copies, programmatic dependent launch, tcgen05).
+// Every wait on a barrier is bounded: after BITNET_WAIT_LIMIT_NS of wall time
+// the wait records BITNET_ERR_TIMEOUT in the device status word and returns
+// false, and the caller unwinds instead of spinning forever.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "bitnet.h"
+
+#define BITNET_DEVINL __device__ __forceinline__
+
+// Two seconds: far above any legitimate wait in these kernels.
+#ifndef BITNET_WAIT_LIMIT_NS
+#define BITNET_WAIT_LIMIT_NS 2000000000ull
+#endif
+
+namespace bitnet {
+
+// Device status word (one per device).  The library is one translation unit,
+// so this is its only definition.
+__device__ int g_device_status = 0;
+
+BITNET_DEVINL void record_status(int code) { atomicCAS(&g_device_status, 0, code); }
+BITNET_DEVINL bool status_failed() { return *(volatile int *)&g_device_status != 0; }
+
+BITNET_DEVINL uint64_t globaltimer_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+BITNET_DEVINL uint32_t smem_u32(const void *p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ---- mbarrier ------------------------------------------------------------
+
+BITNET_DEVINL void mbar_init(uint64_t *bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+BITNET_DEVINL void fence_mbarrier_init()
+{
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+BITNET_DEVINL void mbar_arrive(uint64_t *bar)
+{
+    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+BITNET_DEVINL void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes)
+{
+    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(
+                     smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+BITNET_DEVINL bool mbar_try_wait(uint32_t bar_addr, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar_addr), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait until the phase with the given parity has completed.  Bounded: returns
+// false (after recording a timeout) if it does not complete in time or if
+// another wait on the device already gave up.
+BITNET_DEVINL bool mbar_wait(uint64_t *bar, uint32_t parity)
+{
+    const uint32_t a = smem_u32(bar);
+    if (mbar_try_wait(a, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t spin = 1;; ++spin) {
+        if (mbar_try_wait(a, parity)) return true;
+        if ((spin & 255u) == 0) {
+            if (status_failed()) return false;
+            if (globaltimer_ns() - t0 > BITNET_WAIT_LIMIT_NS) {
+                record_status(BITNET_ERR_TIMEOUT);
+                return false;
+            }
+        }
+    }
+}
+
+// ---- bulk / tensor copies (async proxy) ----------------------------------
+
+// 1-D bulk copy global -> shared, completion counted on `bar` (bytes % 16 == 0,
+// both addresses 16-byte aligned).
+BITNET_DEVINL void bulk_g2s(void *dst_smem, const void *src_gmem, uint32_t bytes, uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst_smem)),
+        "l"(src_gmem), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// 2-D tiled tensor copy global -> shared (no multicast).  c0 is the innermost
+// coordinate in elements; callers keep c0 * elem_size a multiple of 16 bytes.
+BITNET_DEVINL void tma_load_2d(void *dst_smem, const CUtensorMap *map, int32_t c0, int32_t c1, uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            smem_u32(dst_smem)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+        : "memory");
+}
+
+BITNET_DEVINL void prefetch_tensormap(const CUtensorMap *map)
+{
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// Order this thread's generic-proxy shared-memory writes before later
+// async-proxy (tensor core / TMA) accesses.
+BITNET_DEVINL void fence_proxy_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// ---- programmatic dependent launch -------------------------------------
+
+// Block until the grids this grid depends on have completed and their memory
+// is visible (a no-op when launched without a programmatic dependency).
+BITNET_DEVINL void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Allow the next grid in the stream to start launching.
+BITNET_DEVINL void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// ---- small utilities -----------------------------------------------------
+
+BITNET_DEVINL float warp_max(float v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+BITNET_DEVINL int warp_sum(int v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// Quantise one value: rne(x * s) clamped to [-128, 127], fp32 product rounded once.
+BITNET_DEVINL int quant_one(float x, float s)
+{
+    int q = __float2int_rn(__fmul_rn(x, s));
+    return max(-128, min(127, q));
+}
+
+// s = 127 / max(amax, 1e-5), IEEE fp32 division.
+BITNET_DEVINL float quant_scale(float amax) { return __fdiv_rn(127.0f, fmaxf(amax, 1e-5f)); }
+
+BITNET_DEVINL uint32_t pack4_s8(int a, int b, int c, int d)
+{
+    return (uint32_t)(a & 0xff) | ((uint32_t)(b & 0xff) << 8) | ((uint32_t)(c & 0xff) << 16) |
+           ((uint32_t)(d & 0xff) << 24);
+}
+
+BITNET_DEVINL float bf16_bits_lo(uint32_t w) { return __uint_as_float(w << 16); }
+BITNET_DEVINL float bf16_bits_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// ---- tcgen05 (5th-generation tensor cores, tensor memory) ----------------
+
+BITNET_DEVINL void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+BITNET_DEVINL void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Whole warp: allocate `ncols` TMEM columns, address written to *slot.
+BITNET_DEVINL void tmem_alloc(uint32_t *slot, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)),
+                 "r"(ncols)
+                 : "memory");
+}
+BITNET_DEVINL void tmem_relinquish() { asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;"); }
+BITNET_DEVINL void tmem_dealloc(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
+// 128 bytes, 8-row core groups 1024 bytes apart (SBO), LBO unused (1), sm100
+// descriptor version 1.
+BITNET_DEVINL uint64_t umma_desc_k_sw128(const void *smem_ptr)
+{
+    const uint64_t addr = smem_u32(smem_ptr);
+    return ((addr >> 4) & 0x3FFFull) | (1ull << 16) | ((uint64_t)(1024 >> 4) << 32) | (1ull << 46) |
+           (2ull << 61);
+}
+
+// D[tmem] (+)= A[smem] . B[smem]^T, int8 inputs, int32 accumulators.
+BITNET_DEVINL void umma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive once on `bar` when every tcgen05 operation issued so far by this
+// thread has completed.
+BITNET_DEVINL void umma_commit(uint64_t *bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+// Warp-collective: 32 lanes x 32 consecutive 32-bit columns.
+BITNET_DEVINL void tmem_ld32(uint32_t taddr, uint32_t (&v)[32])
+{
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+                 "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+                 "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+                   "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+                   "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]),
+                   "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]),
+                   "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+                 : "r"(taddr)
+                 : "memory");
+}
+BITNET_DEVINL void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Bounded wait that ignores the failure flag: used only to let this CTA's own
+// in-flight copies / MMAs land before it releases shared or tensor memory.
+BITNET_DEVINL bool mbar_wait_drain(uint64_t *bar, uint32_t parity)
+{
+    const uint32_t a = smem_u32(bar);
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(a, parity))
+        if (globaltimer_ns() - t0 > BITNET_WAIT_LIMIT_NS) return false;
+    return true;
+}
+
+} // namespace bitnet

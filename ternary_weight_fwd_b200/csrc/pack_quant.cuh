@@ -1,0 +1,159 @@
+// pack_quant.cuh -- offline weight ternarisation/packing and the standalone
+// per-token activation quantiser.
+//
+// BitNet model page, section "Model details", item "Quantization": ternary
+// weights by absmean quantisation, 8-bit activations by per-token absmax
+// quantisation; section "Model variants": the deployable weights are packed.
+#pragma once
+
+#include "common.cuh"
+
+namespace bitnet {
+
+// ---------------------------------------------------------------------------
+// gamma = mean|W| in fp64, fixed order: each row left to right (one thread per
+// row), then the row sums top to bottom (one thread).  The order is part of
+// the contract: it makes gamma bit-reproducible against a sequential CPU sum.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(128) k_pack_rowsum(const float *__restrict__ w, int64_t N, int64_t K,
+                                                     double *__restrict__ rowsum)
+{
+    const int64_t n = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (n >= N) return;
+    const float4 *row = reinterpret_cast<const float4 *>(w + n * K);
+    double acc = 0.0;
+    const int64_t nv = K / 4;
+    for (int64_t i = 0; i < nv; ++i) {
+        const float4 v = __ldg(row + i);
+        acc = __dadd_rn(acc, fabs((double)v.x));
+        acc = __dadd_rn(acc, fabs((double)v.y));
+        acc = __dadd_rn(acc, fabs((double)v.z));
+        acc = __dadd_rn(acc, fabs((double)v.w));
+    }
+    rowsum[n] = acc;
+}
+
+__global__ void k_pack_gamma(const double *__restrict__ rowsum, int64_t N, int64_t K, float *__restrict__ gamma)
+{
+    if (blockIdx.x != 0 || threadIdx.x != 0) return;
+    double total = 0.0;
+    for (int64_t n = 0; n < N; ++n) total = __dadd_rn(total, rowsum[n]);
+    gamma[0] = __double2float_rn(__ddiv_rn(total, (double)(N * K)));
+}
+
+// code = clamp(rne(w / d), -1, 1) + 1 with d = gamma + eps (IEEE fp32).
+BITNET_DEVINL uint32_t ternary_code(float w, float d)
+{
+    float q = rintf(__fdiv_rn(w, d));
+    q = fminf(fmaxf(q, -1.0f), 1.0f);
+    return (uint32_t)((int)q + 1);
+}
+
+// One thread per 32-bit word = 16 consecutive weights of a row: weight
+// 16g + 4j + b goes to byte b, bits 2j..2j+1.
+__global__ void __launch_bounds__(256) k_pack_codes(const float *__restrict__ w, int64_t nwords, float eps,
+                                                    const float *__restrict__ gamma, uint32_t *__restrict__ out)
+{
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= nwords) return;
+    const float d = __fadd_rn(gamma[0], eps);
+    const float4 *src = reinterpret_cast<const float4 *>(w) + i * 4;
+    uint32_t word = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float4 v = __ldg(src + j);
+        word |= ternary_code(v.x, d) << (2 * j);
+        word |= ternary_code(v.y, d) << (8 + 2 * j);
+        word |= ternary_code(v.z, d) << (16 + 2 * j);
+        word |= ternary_code(v.w, d) << (24 + 2 * j);
+    }
+    out[i] = word;
+}
+
+// ---------------------------------------------------------------------------
+// Per-token absmax quantiser, one warp per row, natural [M][K] int8 output.
+// s = 127 / max(max|x|, 1e-5); x_q = clamp(rne(x * s), -128, 127).
+// ---------------------------------------------------------------------------
+template <bool XF32>
+BITNET_DEVINL float chunk_absmax(const uint4 v)
+{
+    if constexpr (XF32) {
+        return fmaxf(fmaxf(fabsf(__uint_as_float(v.x)), fabsf(__uint_as_float(v.y))),
+                     fmaxf(fabsf(__uint_as_float(v.z)), fabsf(__uint_as_float(v.w))));
+    } else {
+        // |bf16| bit patterns order like their values; compare in fp32
+        const uint32_t m = 0x7fff7fffu;
+        const uint32_t a = v.x & m, b = v.y & m, c = v.z & m, d = v.w & m;
+        const float f0 = fmaxf(bf16_bits_lo(a), bf16_bits_hi(a));
+        const float f1 = fmaxf(bf16_bits_lo(b), bf16_bits_hi(b));
+        const float f2 = fmaxf(bf16_bits_lo(c), bf16_bits_hi(c));
+        const float f3 = fmaxf(bf16_bits_lo(d), bf16_bits_hi(d));
+        return fmaxf(fmaxf(f0, f1), fmaxf(f2, f3));
+    }
+}
+
+// Quantise one 16-byte chunk (8 bf16 or 4 fp32 values); returns the packed
+// int8 bytes in q.x (.y for bf16) and adds their sum to rs.
+template <bool XF32>
+BITNET_DEVINL uint2 chunk_quant(const uint4 v, float sc, int &rs)
+{
+    uint2 q;
+    if constexpr (XF32) {
+        const int a = quant_one(__uint_as_float(v.x), sc), b = quant_one(__uint_as_float(v.y), sc);
+        const int c = quant_one(__uint_as_float(v.z), sc), d = quant_one(__uint_as_float(v.w), sc);
+        rs += a + b + c + d;
+        q.x = pack4_s8(a, b, c, d);
+        q.y = 0;
+    } else {
+        const int a0 = quant_one(bf16_bits_lo(v.x), sc), a1 = quant_one(bf16_bits_hi(v.x), sc);
+        const int b0 = quant_one(bf16_bits_lo(v.y), sc), b1 = quant_one(bf16_bits_hi(v.y), sc);
+        const int c0 = quant_one(bf16_bits_lo(v.z), sc), c1 = quant_one(bf16_bits_hi(v.z), sc);
+        const int d0 = quant_one(bf16_bits_lo(v.w), sc), d1 = quant_one(bf16_bits_hi(v.w), sc);
+        rs += a0 + a1 + b0 + b1 + c0 + c1 + d0 + d1;
+        q.x = pack4_s8(a0, a1, b0, b1);
+        q.y = pack4_s8(c0, c1, d0, d1);
+    }
+    return q;
+}
+
+template <bool XF32>
+__global__ void __launch_bounds__(256) k_quant_rows(const void *__restrict__ x, int64_t M, int64_t K,
+                                                    int8_t *__restrict__ x_q, float *__restrict__ s,
+                                                    int32_t *__restrict__ rowsum)
+{
+    pdl_launch_dependents();
+    pdl_wait();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t m = (int64_t)blockIdx.x * 8 + warp;
+    if (m >= M) return;
+    constexpr int EPC = XF32 ? 4 : 8; // elements per 16-byte chunk
+    const int64_t nch = K / EPC;
+    const uint4 *row = reinterpret_cast<const uint4 *>(static_cast<const char *>(x) + m * K * (XF32 ? 4 : 2));
+    float amax = 0.0f;
+    int64_t c = lane;
+    for (; c + 96 < nch; c += 128) {
+        const uint4 v0 = __ldg(row + c), v1 = __ldg(row + c + 32), v2 = __ldg(row + c + 64),
+                    v3 = __ldg(row + c + 96);
+        amax = fmaxf(amax, fmaxf(fmaxf(chunk_absmax<XF32>(v0), chunk_absmax<XF32>(v1)),
+                                 fmaxf(chunk_absmax<XF32>(v2), chunk_absmax<XF32>(v3))));
+    }
+    for (; c < nch; c += 32) amax = fmaxf(amax, chunk_absmax<XF32>(__ldg(row + c)));
+    amax = warp_max(amax);
+    const float sc = quant_scale(amax);
+    int rs = 0;
+    int8_t *qrow = x_q + m * K;
+    for (c = lane; c < nch; c += 32) {
+        const uint2 q = chunk_quant<XF32>(__ldg(row + c), sc, rs);
+        if constexpr (XF32)
+            reinterpret_cast<uint32_t *>(qrow)[c] = q.x;
+        else
+            reinterpret_cast<uint2 *>(qrow)[c] = q;
+    }
+    rs = warp_sum(rs);
+    if (lane == 0) {
+        s[m] = sc;
+        if (rowsum) rowsum[m] = rs;
+    }
+}
+
+} // namespace bitnet

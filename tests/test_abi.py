@@ -1,0 +1,118 @@
+"""The C-ABI library builds, loads and exports every declared entry point; host-side
+argument validation works without a GPU (no compute is launched here)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import ternary_weight_fwd_b200 as tw
+from ternary_weight_fwd_b200 import build as tw_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADERS = [os.path.join(ROOT, "include", f) for f in sorted(os.listdir(os.path.join(ROOT, "include")))
+           if f.endswith(".h")]
+
+
+def declared_functions():
+    names = []
+    for h in HEADERS:
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names += re.findall(r"\b(bitnet_[a-z0-9_]+)\s*\(", text)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    tw_build.build()
+    return tw.load_library()
+
+
+def test_header_declares_the_four_calls():
+    names = declared_functions()
+    for n in ("bitnet_pack_weights", "bitnet_quant_act", "bitnet_linear", "bitnet_ffn_gate_up"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    out = subprocess.check_output(["nm", "-D", "--defined-only", tw.LIB_PATH]).decode()
+    exported = set(re.findall(r"\bT (bitnet_[a-z0-9_]+)$", out, flags=re.M))
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+    for n in declared_functions():
+        assert getattr(lib, n) is not None
+
+
+def test_build_targets_sm100a_only():
+    cmd = tw_build.nvcc_cmd("out.so")
+    gencodes = [cmd[i + 1] for i, c in enumerate(cmd) if c == "-gencode"]
+    assert gencodes == ["arch=compute_100a,code=sm_100a"]
+
+
+def test_status_strings(lib):
+    for code, name in [(0, "BITNET_OK"), (1, "BITNET_ERR_INVALID_ARG"), (2, "BITNET_ERR_UNSUPPORTED_SHAPE"),
+                       (3, "BITNET_ERR_MISALIGNED"), (4, "BITNET_ERR_CUDA"), (5, "BITNET_ERR_TIMEOUT"),
+                       (6, "BITNET_ERR_WORKSPACE")]:
+        assert tw.bitnet_status_string(code) == name
+    assert tw.bitnet_status_string(99) == "BITNET_ERR_UNKNOWN"
+
+
+def test_workspace_sizes(lib):
+    assert tw.bitnet_pack_workspace_size(2560, 6912) == 2560 * 8
+    # x_q (M*K rounded to 256) + scales + row sums (each M*4 rounded to 256)
+    assert tw.bitnet_workspace_size(1, 2560, 2560) == 2560 + 256 + 256
+    assert tw.bitnet_workspace_size(4096, 6912, 2560) == 4096 * 2560 + 2 * 16384
+    assert tw.bitnet_workspace_size(0, 1, 64) == 0
+
+
+def test_dispatch_setter(lib):
+    prev = lib.bitnet_set_dispatch(tw.BITNET_DISPATCH_PREFILL)
+    try:
+        assert lib.bitnet_set_dispatch(7) == -1
+        assert lib.bitnet_set_dispatch(tw.BITNET_DISPATCH_DECODE) == tw.BITNET_DISPATCH_PREFILL
+    finally:
+        lib.bitnet_set_dispatch(prev)
+
+
+FAKE = 1 << 20  # a 16-byte aligned non-null "device" address; never dereferenced
+
+
+@pytest.mark.parametrize("case,expect", [
+    (dict(M=0), tw.BITNET_ERR_INVALID_ARG),
+    (dict(N=0), tw.BITNET_ERR_INVALID_ARG),
+    (dict(K=96), tw.BITNET_ERR_UNSUPPORTED_SHAPE),
+    (dict(K=0), tw.BITNET_ERR_INVALID_ARG),
+    (dict(K=65536 + 64), tw.BITNET_ERR_UNSUPPORTED_SHAPE),
+    (dict(x=0), tw.BITNET_ERR_INVALID_ARG),
+    (dict(w=0), tw.BITNET_ERR_INVALID_ARG),
+    (dict(gamma=0), tw.BITNET_ERR_INVALID_ARG),
+    (dict(y=0), tw.BITNET_ERR_INVALID_ARG),
+    (dict(dtype=5), tw.BITNET_ERR_INVALID_ARG),
+    (dict(x=FAKE + 8), tw.BITNET_ERR_MISALIGNED),
+    (dict(y=FAKE + 4), tw.BITNET_ERR_MISALIGNED),
+    (dict(ws=0), tw.BITNET_ERR_WORKSPACE),
+    (dict(ws_bytes=10), tw.BITNET_ERR_WORKSPACE),
+])
+def test_linear_rejects_before_launch(lib, case, expect):
+    a = dict(M=4, N=256, K=256, x=FAKE, w=FAKE, gamma=FAKE, y=FAKE, dtype=0, ws=FAKE, ws_bytes=1 << 20)
+    a.update(case)
+    P = ctypes.c_void_p
+    st = lib.bitnet_linear(P(a["x"] or None), a["dtype"], a["M"], a["K"], P(a["w"] or None),
+                           P(a["gamma"] or None), a["N"], P(a["y"] or None), None, None, None,
+                           P(a["ws"] or None), a["ws_bytes"], None)
+    assert st == expect
+
+
+def test_ffn_and_quant_and_pack_reject_before_launch(lib):
+    P = ctypes.c_void_p
+    assert lib.bitnet_ffn_gate_up(P(FAKE), 0, 4, 256, P(FAKE), P(FAKE), None, P(FAKE), 256, P(FAKE), None, None,
+                                  P(FAKE), 1 << 20, None) == tw.BITNET_ERR_INVALID_ARG
+    assert lib.bitnet_quant_act(P(FAKE), 0, 4, 100, P(FAKE), P(FAKE), None, None) == tw.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert lib.bitnet_quant_act(None, 0, 4, 128, P(FAKE), P(FAKE), None, None) == tw.BITNET_ERR_INVALID_ARG
+    assert lib.bitnet_pack_weights(P(FAKE), 16, 64, 1e-5, P(FAKE), P(FAKE), None, 0, None) == tw.BITNET_ERR_WORKSPACE
+    assert lib.bitnet_pack_weights(P(FAKE), 16, 64, -1.0, P(FAKE), P(FAKE), P(FAKE), 4096, None) == \
+        tw.BITNET_ERR_INVALID_ARG
+    assert lib.bitnet_pack_weights(P(FAKE + 4), 16, 64, 1e-5, P(FAKE), P(FAKE), P(FAKE), 4096, None) == \
+        tw.BITNET_ERR_MISALIGNED
