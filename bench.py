@@ -287,12 +287,13 @@ def capture(torch, stream, fn):
 
 def time_graph(torch, stream, graph, reps):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    graph.replay()
-    stream.synchronize()
-    e0.record(stream)
-    for _ in range(reps):
+    with torch.cuda.stream(stream):
         graph.replay()
-    e1.record(stream)
+        stream.synchronize()
+        e0.record(stream)
+        for _ in range(reps):
+            graph.replay()
+        e1.record(stream)
     e1.synchronize()
     return e0.elapsed_time(e1) / reps
 
@@ -387,22 +388,24 @@ def our_arm(a, n_gpus):
         if ev is not None:
             ev[2].record(stream)
 
-    for _ in range(a.warmup):
-        run_step()
-    stream.synchronize()
-    barrier()
-    clocks = ClockSampler(local_rank if world > 1 else torch.cuda.current_device())
-    clocks.start()
-    time.sleep(0.3)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(a.steps)]
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize()
-    barrier()
-    t_start.record(stream)
-    for i in range(a.steps):
-        run_step(evs[i])
-    t_end.record(stream)
-    stream.synchronize()
+    # graphs replay on the current stream: keep `stream` current for every replay
+    with torch.cuda.stream(stream):
+        for _ in range(a.warmup):
+            run_step()
+        stream.synchronize()
+        barrier()
+        clocks = ClockSampler(local_rank if world > 1 else torch.cuda.current_device())
+        clocks.start()
+        time.sleep(0.3)
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(a.steps)]
+        t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        barrier()
+        t_start.record(stream)
+        for i in range(a.steps):
+            run_step(evs[i])
+        t_end.record(stream)
+        stream.synchronize()
     torch.cuda.synchronize()
     clk = clocks.stop()
     total_ms = max_over_ranks(t_start.elapsed_time(t_end))
