@@ -157,6 +157,34 @@ bitnet_status_t bitnet_linear(const void *x, bitnet_dtype_t x_dtype, int64_t M, 
                               void *workspace, size_t ws_bytes, cudaStream_t stream);
 
 /*
+ * bitnet_linear without a caller-provided workspace, for callers that cannot
+ * allocate device memory when they call: a serving engine that has already
+ * reserved all free HBM for its own pool (KV cache) and hands kernels only
+ * their inputs and outputs, plugin hosts that forbid allocation after
+ * start-up, and latency-critical loops where an allocation's implicit device
+ * synchronisation would stall the pipeline.  The BitNet page has no
+ * counterpart to this call; it is a deployment convenience.
+ *
+ * Arguments and results are those of bitnet_linear without the optional
+ * outputs and the workspace.  Scratch (quantised activations, scales, row
+ * sums) lives in a fixed 8 MiB device array inside this library, held on
+ * every GPU that loads the library until the process exits.  Shapes whose
+ * scratch exceeds it, i.e. M * K + 2 * (M * 4) (each rounded up to 256 bytes)
+ * > 8 MiB, are rejected with BITNET_ERR_WORKSPACE before anything is launched.
+ *
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture.  No call allocates or frees memory.  All calls
+ * share the one array and it keeps the last call's contents (nothing in it
+ * needs to start at zero): calls that can overlap on the GPU -- on different
+ * streams, or on different host threads -- race on it and give wrong
+ * results; order them on one stream or use bitnet_linear.
+ */
+bitnet_status_t bitnet_linear_noalloc(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_t K,
+                                      const uint8_t *w_packed, const float *gamma, int64_t N,
+                                      float *y, cudaStream_t stream);
+
+/*
  * Gate/up half of the BitNet FFN with the squared-ReLU gate fused in the
  * epilogue (page: "Architecture" -- ReLU^2 in the FFN; BitNetConfig
  * hidden_act = "relu2"):

@@ -65,6 +65,7 @@ def load_library(path: str = LIB_PATH):
         "bitnet_num_sms": ([], I),
         "bitnet_set_dispatch": ([I], I),
         "bitnet_launch_count": ([], ctypes.c_uint64),
+        "bitnet_linear_noalloc": ([P, I, I64, I64, P, P, I64, P, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -177,6 +178,21 @@ def bitnet_linear(x, w_packed, gamma, *, y=None, x_q_out=None, s_out=None, acc_o
     _check(lib.bitnet_linear(_ptr(x), _dtype_code(x), m, k, _ptr(w_packed), _ptr(gamma), n, _ptr(y),
                              _ptr(x_q_out), _ptr(s_out), _ptr(acc_out), _ptr(workspace), workspace.numel(),
                              _stream(stream)), "bitnet_linear")
+    return y
+
+
+def bitnet_linear_noalloc(x, w_packed, gamma, *, y=None, stream=None):
+    """bitnet_linear using the library's fixed device scratch instead of a workspace,
+    for callers that cannot allocate at call time.  Only the output may be
+    allocated here, and only when `y` is not given; calls sharing the scratch
+    must not overlap on the GPU."""
+    lib = load_library()
+    m, k = x.shape
+    n = w_packed.shape[0]
+    if y is None:
+        y = torch.empty((m, n), dtype=torch.float32, device=x.device)
+    _check(lib.bitnet_linear_noalloc(_ptr(x), _dtype_code(x), m, k, _ptr(w_packed), _ptr(gamma), n, _ptr(y),
+                                     _stream(stream)), "bitnet_linear_noalloc")
     return y
 
 

@@ -350,6 +350,28 @@ bitnet_status_t forward(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_
     return cuda_status(e);
 }
 
+// ---- fixed scratch for bitnet_linear_noalloc -------------------------------
+// Callers of that entry point cannot allocate, so its scratch is a static
+// device array (every GPU that loads the library holds it until exit).  Host
+// code must not use the symbol as a pointer: it is a host-side stand-in, and
+// the device address is looked up once per device below.
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch on the current device (looked up on the
+// first call per device, with that device current); nullptr on failure.
+void *noalloc_scratch(int dev)
+{
+    static std::atomic<void *> cache[kMaxDevices];
+    if (dev < 0 || dev >= kMaxDevices) return nullptr;
+    void *p = cache[dev].load();
+    if (p) return p;
+    void *q = nullptr;
+    if (cudaGetSymbolAddress(&q, g_noalloc_scratch) != cudaSuccess || q == nullptr) return nullptr;
+    cache[dev].store(q);
+    return q;
+}
+
 } // namespace
 } // namespace bitnet
 
@@ -424,6 +446,20 @@ bitnet_status_t bitnet_linear(const void *x, bitnet_dtype_t x_dtype, int64_t M, 
 {
     return forward(x, x_dtype, M, K, w_packed, gamma, nullptr, nullptr, N, y, x_q_out, s_out, acc_out, nullptr,
                    workspace, ws_bytes, stream, 1);
+}
+
+bitnet_status_t bitnet_linear_noalloc(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_t K,
+                                      const uint8_t *w_packed, const float *gamma, int64_t N, float *y,
+                                      cudaStream_t stream)
+{
+    bitnet_status_t st = check_shape(M, N, K);
+    if (st != BITNET_OK) return st;
+    if (ws_bytes_for(M, K) > kNoAllocScratchBytes) return BITNET_ERR_WORKSPACE;
+    if (!x || !w_packed || !gamma || !y) return BITNET_ERR_INVALID_ARG;
+    void *scratch = noalloc_scratch(current_device());
+    if (!scratch) return BITNET_ERR_CUDA;
+    return forward(x, x_dtype, M, K, w_packed, gamma, nullptr, nullptr, N, y, nullptr, nullptr, nullptr, nullptr,
+                   scratch, kNoAllocScratchBytes, stream, 1);
 }
 
 bitnet_status_t bitnet_ffn_gate_up(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_t K,
