@@ -57,6 +57,12 @@ def parse_args():
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--cpu-seconds", type=float, default=10.0, help="budget of the oracle CPU baseline")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--profile", default=None,
+                   choices=["decode_q_o", "decode_gate_up", "decode_down", "prefill_q_o", "prefill_gate_up",
+                            "prefill_down"],
+                   help="profiling harness: build one layer, run this projection kind --profile-reps times "
+                        "(no graphs, no timing, no JSON) and exit; for ncu captures of one kernel")
+    p.add_argument("--profile-reps", type=int, default=3)
     return p.parse_args()
 
 
@@ -278,6 +284,22 @@ class Stack:
             self.down(l, self.dec_out, self.ws_dec, s)
 
 
+def reduce_max(v, dist, device):
+    """Max of a float over all ranks (identity without a process group)."""
+    if dist is None:
+        return v
+    import torch
+
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_value(n_gpus, tokens_per_replica_step, layers, max_ms_per_step):
+    """Whole-job throughput: every replica processes its own batch (weak scaling)."""
+    return n_gpus * tokens_per_replica_step * layers / (max_ms_per_step / 1e3)
+
+
 def capture(torch, stream, fn):
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=stream):
@@ -354,15 +376,28 @@ def our_arm(a, n_gpus):
             dist.barrier()
 
     def max_over_ranks(v):
-        if not dist:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(v, dist, dev)
 
     st = Stack(a, dev, seed=1234 + rank)
     stream = torch.cuda.Stream(device=dev)
     stream.wait_stream(torch.cuda.current_stream())
+
+    if a.profile:
+        ops = {
+            "decode_q_o": lambda s: st.q(0, st.dec_x[0], st.dec_out, st.ws_dec, s),
+            "decode_gate_up": lambda s: st.gate_up(0, st.dec_x[0], st.dec_out, st.ws_dec, s),
+            "decode_down": lambda s: st.down(0, st.dec_out, st.ws_dec, s),
+            "prefill_q_o": lambda s: st.q(0, st.pre_x[0], st.pre_out, st.ws_pre, s),
+            "prefill_gate_up": lambda s: st.gate_up(0, st.pre_x[0], st.pre_out, st.ws_pre, s),
+            "prefill_down": lambda s: st.down(0, st.pre_out, st.ws_pre, s),
+        }
+        with torch.cuda.stream(stream):
+            for _ in range(a.profile_reps):
+                ops[a.profile](stream)
+        stream.synchronize()
+        assert tw.bitnet_device_status() == 0
+        print(f"profiled {a.profile} x{a.profile_reps}")
+        return 0
 
     # ---- capture: one prefill pass, decode steps in chunks of 16 ----
     with torch.cuda.stream(stream):
@@ -417,7 +452,7 @@ def our_arm(a, n_gpus):
 
     M, B, Lyr = a.prefill_tokens, a.decode_batch, a.layers
     tokens_step = (M + a.decode_steps * B)
-    value = n_gpus * tokens_step * Lyr / (ms_step / 1e3)
+    value = aggregate_value(n_gpus, tokens_step, Lyr, ms_step)
 
     # ---- phase figures (per replica) ----
     ops_layer = 2 * HIDDEN * HIDDEN * 2 + 2 * (2 * HIDDEN * INTER) + 2 * INTER * HIDDEN  # per token
@@ -510,7 +545,7 @@ def our_arm(a, n_gpus):
         e1.record(stream)
         e1.synchronize()
         e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / a.e2e_steps
-        e2e = {"value": n_gpus * tokens_step * Lyr / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        e2e = {"value": aggregate_value(n_gpus, tokens_step, Lyr, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
     cpu = None

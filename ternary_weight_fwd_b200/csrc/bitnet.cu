@@ -16,6 +16,7 @@
 #include "bitnet.h"
 #include "common.cuh"
 #include "decode.cuh"
+#include "decode_cluster.cuh"
 #include "pack_quant.cuh"
 #include "prefill.cuh"
 
@@ -29,9 +30,6 @@ constexpr int64_t kMaxDim = int64_t(1) << 24;
 constexpr int64_t kMaxK = 65536;
 constexpr int kDecodeMaxM = 64;
 constexpr size_t kSmemLimit = 227 * 1024;
-// Up to this many activation elements (M*K) the decode kernel quantises x in
-// every CTA instead of running the quantiser kernel first.
-constexpr int64_t kFusedQuantMaxElems = 8192;
 
 std::atomic<int> g_dispatch{BITNET_DISPATCH_AUTO};
 std::atomic<uint64_t> g_launches{0};
@@ -159,15 +157,15 @@ bool encode_u8_2d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t co
 // ---- decode configuration -----------------------------------------------------
 struct DecodeCfg {
     bool ok;
-    int grid, rg, w_stride, x_stride, rp, ch;
+    int grid, rg, w_stride, rp, ch;
     size_t smem;
 };
 
-DecodeCfg decode_config(int64_t M, int64_t N, int64_t K, int nmat, bool fused, int sms)
+// Row-split decode kernel (quantiser kernel first): one CTA per slice of rows.
+DecodeCfg decode_config(int64_t N, int64_t K, int nmat, int sms)
 {
     DecodeCfg c = {};
     c.w_stride = (int)(K / 4 + ((16 - (K / 4) % 128) + 128) % 128);
-    c.x_stride = (int)(K + ((64 - K % 128) + 128) % 128);
     int64_t grid = std::min<int64_t>(sms, cdiv(N, 16));
     for (;;) {
         const int64_t rmax = cdiv(N, grid);
@@ -177,8 +175,7 @@ DecodeCfg decode_config(int64_t M, int64_t N, int64_t K, int nmat, bool fused, i
             continue;
         }
         const int rp = rg * 16 + ((4 - (rg * 16) % 32) + 32) % 32;
-        const size_t smem = DEC_HDR + (size_t)nmat * rg * 16 * c.w_stride + (size_t)nmat * 8 * rp * 4 +
-                            (fused ? (size_t)8 * c.x_stride : 0);
+        const size_t smem = DEC_HDR + (size_t)nmat * rg * 16 * c.w_stride + (size_t)nmat * 8 * rp * 4;
         if (smem > kSmemLimit) {
             if (rg == 1) return c; // K too large for the decode kernel
             grid = cdiv(N, 16 * (rg - 1));
@@ -196,28 +193,23 @@ DecodeCfg decode_config(int64_t M, int64_t N, int64_t K, int nmat, bool fused, i
     return c;
 }
 
-template <int NMAT, bool FUSED, bool XF32, int CH>
+template <int NMAT, int CH>
 cudaError_t launch_decode_t(const DecodeArgs &a, const DecodeCfg &c, cudaStream_t stream, int dev)
 {
     static std::atomic<int> done[kMaxDevices];
-    auto kern = k_decode<NMAT, FUSED, XF32, CH>;
+    auto kern = k_decode<NMAT, CH>;
     cudaError_t e = ensure_smem(kern, c.smem, done, dev);
     if (e != cudaSuccess) return e;
     return launch_pdl(kern, dim3(c.grid), dim3(DEC_THREADS), c.smem, stream, a);
 }
 
 template <int NMAT>
-cudaError_t launch_decode(const DecodeArgs &a, const DecodeCfg &c, bool fused, bool xf32, cudaStream_t stream,
-                          int dev)
+cudaError_t launch_decode(const DecodeArgs &a, const DecodeCfg &c, cudaStream_t stream, int dev)
 {
-    if (fused) {
-        return xf32 ? launch_decode_t<NMAT, true, true, 4>(a, c, stream, dev)
-                    : launch_decode_t<NMAT, true, false, 4>(a, c, stream, dev);
-    }
     switch (c.ch) {
-    case 4: return launch_decode_t<NMAT, false, false, 4>(a, c, stream, dev);
-    case 8: return launch_decode_t<NMAT, false, false, 8>(a, c, stream, dev);
-    default: return launch_decode_t<NMAT, false, false, 16>(a, c, stream, dev);
+    case 4: return launch_decode_t<NMAT, 4>(a, c, stream, dev);
+    case 8: return launch_decode_t<NMAT, 8>(a, c, stream, dev);
+    default: return launch_decode_t<NMAT, 16>(a, c, stream, dev);
     }
 }
 
@@ -229,18 +221,204 @@ cudaError_t launch_quant(const void *x, bool xf32, int64_t M, int64_t K, int8_t 
     return launch_pdl(k_quant_rows<false>, grid, dim3(256), 0, stream, x, M, K, xq, s, rs);
 }
 
-bool use_decode(int64_t M, int dispatch)
+// ---- cluster (K-split, fused quantiser) decode kernel -------------------------
+struct DcCfg {
+    bool ok;
+    int nc;  // clusters launched
+    int rgw; // row groups per warp
+    size_t smem;
+    DcArgs a;
+};
+
+// Shared-memory layout for `rpc` rows per cluster and cluster size C.
+bool dc_layout(DcArgs &a, size_t &smem, int64_t K, int nmat, bool xf32, int C, int rpc)
 {
-    if (dispatch == BITNET_DISPATCH_PREFILL) return false;
-    if (dispatch == BITNET_DISPATCH_DECODE || dispatch == BITNET_DISPATCH_DECODE_FUSED) return M <= kDecodeMaxM;
-    return M <= kDecodeMaxM;
+    const int KS = (int)(K / 64);
+    a.C = C;
+    a.ks = (int)cdiv(KS, C);
+    if (a.ks > 16) return false; // weight box row must stay <= 256 bytes
+    a.nbox = (int)cdiv(rpc, 256);
+    a.rows_box = (int)align_up((size_t)cdiv(rpc, a.nbox), 8);
+    a.rpc = a.rows_box * a.nbox;
+    if (nmat * cdiv(a.rpc, 16) > 8 * DC_RGW_MAX) return false; // row groups per warp
+    const uint32_t box_w = (uint32_t)a.ks * 16;
+    a.w_mat_bytes = (uint32_t)align_up(align_up((size_t)a.rpc, 16) * box_w, 128);
+    a.xs_row = (uint32_t)align_up((size_t)a.ks * 64 * (xf32 ? 4 : 2), 128);
+    a.xs_off = (uint32_t)(DC_HDR + (size_t)nmat * a.w_mat_bytes);
+    a.xq_stride = (uint32_t)(a.ks * 64 + ((64 - (a.ks * 64) % 128) + 128) % 128);
+    a.xq_off = a.xs_off + 8 * a.xs_row;
+    a.own_rows = (int)cdiv(a.rpc, C);
+    a.orp = (int)align_up((size_t)a.own_rows, 4);
+    if (a.orp % 8 == 0) a.orp += 4; // token rows of a block land 8 banks apart
+    a.blk_bytes = (uint32_t)(nmat * 8 * a.orp * 4);
+    a.part_off = (uint32_t)align_up((size_t)a.xq_off + 8 * (size_t)a.xq_stride, 128);
+    a.recv_off = a.part_off + (uint32_t)align_up((size_t)C * a.blk_bytes, 128);
+    smem = (size_t)a.recv_off + (size_t)C * a.blk_bytes + 128;
+    return smem <= kSmemLimit;
 }
 
-bool use_fused(int64_t M, int64_t K, int dispatch)
+// Row groups per warp for a layout (template argument of the kernel).
+int dc_rgw(const DcArgs &a, int nmat)
 {
-    if (dispatch == BITNET_DISPATCH_DECODE_FUSED) return true;
-    if (dispatch == BITNET_DISPATCH_DECODE) return false;
-    return M * K <= kFusedQuantMaxElems;
+    const int64_t per_warp = cdiv(nmat * cdiv(a.rpc, 16), 8);
+    return per_warp <= 1 ? 1 : per_warp <= 2 ? 2 : per_warp <= 4 ? 4 : 8;
+}
+
+template <int NMAT, bool XF32, int RGW>
+cudaError_t dc_kernel_setup(int dev, int C, size_t smem, int *max_clusters)
+{
+    static std::atomic<int> done[kMaxDevices];
+    auto kern = k_decode_cluster<NMAT, XF32, RGW>;
+    cudaError_t e = ensure_smem(kern, smem, done, dev);
+    if (e != cudaSuccess || !max_clusters) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(C * 64);
+    cfg.blockDim = dim3(DC_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaOccupancyMaxActiveClusters(max_clusters, kern, &cfg);
+}
+
+template <int NMAT, bool XF32>
+cudaError_t dc_setup_rgw(int rgw, int dev, int C, size_t smem, int *max_clusters)
+{
+    switch (rgw) {
+    case 1: return dc_kernel_setup<NMAT, XF32, 1>(dev, C, smem, max_clusters);
+    case 2: return dc_kernel_setup<NMAT, XF32, 2>(dev, C, smem, max_clusters);
+    case 4: return dc_kernel_setup<NMAT, XF32, 4>(dev, C, smem, max_clusters);
+    default: return dc_kernel_setup<NMAT, XF32, 8>(dev, C, smem, max_clusters);
+    }
+}
+
+cudaError_t dc_setup(int nmat, bool xf32, int rgw, int dev, int C, size_t smem, int *max_clusters)
+{
+    if (nmat == 1)
+        return xf32 ? dc_setup_rgw<1, true>(rgw, dev, C, smem, max_clusters)
+                    : dc_setup_rgw<1, false>(rgw, dev, C, smem, max_clusters);
+    return xf32 ? dc_setup_rgw<2, true>(rgw, dev, C, smem, max_clusters)
+                : dc_setup_rgw<2, false>(rgw, dev, C, smem, max_clusters);
+}
+
+// Cluster size C = 8 (K split 8 ways) when K has at least 8 k-steps of 64;
+// rows per cluster sized so that one wave of resident clusters covers N.
+DcCfg dc_config(int64_t N, int64_t K, int nmat, bool xf32, int dev, int sms)
+{
+    struct Entry {
+        int64_t N, K;
+        int nmat, xf32, dev;
+        DcCfg cfg;
+    };
+    static std::mutex mu;
+    static Entry cache[64];
+    static int ncache = 0;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        for (int i = 0; i < ncache; ++i)
+            if (cache[i].N == N && cache[i].K == K && cache[i].nmat == nmat && cache[i].xf32 == (int)xf32 &&
+                cache[i].dev == dev)
+                return cache[i].cfg;
+    }
+    DcCfg c = {};
+    const int KS = (int)(K / 64);
+    const int C = std::min(8, KS);
+    int nc = std::max(1, sms / C);
+    size_t smem = 0;
+    for (int iter = 0; iter < 4; ++iter) {
+        int rpc = (int)align_up((size_t)cdiv(N, nc), 8);
+        while (!dc_layout(c.a, smem, K, nmat, xf32, C, rpc)) {
+            if (rpc <= 8 || cdiv(K / 64, C) > 16) return c; // not supported: caller falls back
+            rpc = (int)align_up((size_t)(rpc / 2), 8);
+        }
+        int resident = 0;
+        c.rgw = dc_rgw(c.a, nmat);
+        if (dc_setup(nmat, xf32, c.rgw, dev, C, smem, &resident) != cudaSuccess || resident < 1) return c;
+        const int want = (int)cdiv(N, c.a.rpc);
+        if (want <= resident || iter == 3) {
+            c.nc = want;
+            break;
+        }
+        nc = resident; // fewer clusters fit: give each more rows and re-check
+    }
+    c.smem = smem;
+    c.ok = true;
+    std::lock_guard<std::mutex> lk(mu);
+    if (ncache < 64) cache[ncache++] = {N, K, nmat, (int)xf32, dev, c};
+    return c;
+}
+
+template <int NMAT, bool XF32, int RGW>
+cudaError_t dc_launch_t(const DcCfg &c, const CUtensorMap &t0, const CUtensorMap &t1, const DcArgs &a,
+                        cudaStream_t stream)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(c.nc * a.C));
+    cfg.blockDim = dim3(DC_THREADS);
+    cfg.dynamicSmemBytes = c.smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = a.C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return cudaLaunchKernelEx(&cfg, k_decode_cluster<NMAT, XF32, RGW>, t0, t1, a);
+}
+
+template <int NMAT, bool XF32>
+cudaError_t dc_launch(const DcCfg &c, const CUtensorMap &t0, const CUtensorMap &t1, const DcArgs &a,
+                      cudaStream_t stream)
+{
+    switch (c.rgw) {
+    case 1: return dc_launch_t<NMAT, XF32, 1>(c, t0, t1, a, stream);
+    case 2: return dc_launch_t<NMAT, XF32, 2>(c, t0, t1, a, stream);
+    case 4: return dc_launch_t<NMAT, XF32, 4>(c, t0, t1, a, stream);
+    default: return dc_launch_t<NMAT, XF32, 8>(c, t0, t1, a, stream);
+    }
+}
+
+bitnet_status_t dc_forward(const DcCfg &c, const void *x, bool xf32, int64_t M, int64_t K, const uint8_t *w0,
+                           const float *gamma0, const uint8_t *w1, const float *gamma1, int64_t N, float *y,
+                           int8_t *x_q_out, float *s_out, int32_t *acc0, int32_t *acc1, cudaStream_t stream,
+                           int nmat)
+{
+    DcArgs a = c.a;
+    a.x = x;
+    a.gamma0 = gamma0;
+    a.gamma1 = gamma1;
+    a.y = y;
+    a.acc0 = acc0;
+    a.acc1 = acc1;
+    a.xq_out = x_q_out;
+    a.s_out = s_out;
+    a.M = (int)M;
+    a.N = (int)N;
+    a.K = (int)K;
+    CUtensorMap t0, t1;
+    const uint32_t box_w = (uint32_t)a.ks * 16;
+    if (!encode_u8_2d(&t0, w0, (uint64_t)N, (uint64_t)(K / 4), (uint32_t)a.rows_box, box_w, false))
+        return BITNET_ERR_CUDA;
+    if (nmat == 2) {
+        if (!encode_u8_2d(&t1, w1, (uint64_t)N, (uint64_t)(K / 4), (uint32_t)a.rows_box, box_w, false))
+            return BITNET_ERR_CUDA;
+    } else {
+        t1 = t0;
+    }
+    cudaError_t e;
+    if (nmat == 1)
+        e = xf32 ? dc_launch<1, true>(c, t0, t1, a, stream) : dc_launch<1, false>(c, t0, t1, a, stream);
+    else
+        e = xf32 ? dc_launch<2, true>(c, t0, t1, a, stream) : dc_launch<2, false>(c, t0, t1, a, stream);
+    return cuda_status(e);
 }
 
 // Shared body of bitnet_linear (nmat = 1) and bitnet_ffn_gate_up (nmat = 2).
@@ -266,16 +444,19 @@ bitnet_status_t forward(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_
     int8_t *xq = x_q_out ? x_q_out : ws.xq;
     float *s = s_out ? s_out : ws.s;
 
-    if (use_decode(M, dispatch)) {
-        bool fused = use_fused(M, K, dispatch);
-        DecodeCfg c = decode_config(M, N, K, nmat, fused, sms);
-        if (!c.ok && fused) {
-            fused = false;
-            c = decode_config(M, N, K, nmat, false, sms);
+    if (M <= kDecodeMaxM && dispatch != BITNET_DISPATCH_PREFILL) {
+        // cluster kernel with the quantiser fused in (automatic choice for decode)
+        if (dispatch != BITNET_DISPATCH_DECODE) {
+            const DcCfg c = dc_config(N, K, nmat, xf32, dev, sms);
+            if (c.ok)
+                return dc_forward(c, x, xf32, M, K, w0, gamma0, w1, gamma1, N, y, x_q_out, s_out, acc0, acc1,
+                                  stream, nmat);
+            if (dispatch == BITNET_DISPATCH_DECODE_FUSED) return BITNET_ERR_UNSUPPORTED_SHAPE;
         }
+        // quantiser kernel, then the row-split decode kernel
+        const DecodeCfg c = decode_config(N, K, nmat, sms);
         if (c.ok) {
             DecodeArgs a = {};
-            a.x = x;
             a.xq = xq;
             a.s_in = s;
             a.rs_in = ws.rs;
@@ -286,24 +467,21 @@ bitnet_status_t forward(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_
             a.y = y;
             a.acc0 = acc0;
             a.acc1 = acc1;
-            a.xq_out = fused ? x_q_out : nullptr;
-            a.s_out = fused ? s_out : nullptr;
             a.M = (int)M;
             a.N = (int)N;
             a.K = (int)K;
             a.grid = c.grid;
             a.rg = c.rg;
             a.w_stride = c.w_stride;
-            a.x_stride = c.x_stride;
             a.rp = c.rp;
-            cudaError_t e = cudaSuccess;
-            if (!fused) e = launch_quant(x, xf32, M, K, xq, s, ws.rs, stream);
+            cudaError_t e = launch_quant(x, xf32, M, K, xq, s, ws.rs, stream);
             if (e == cudaSuccess)
-                e = nmat == 1 ? launch_decode<1>(a, c, fused, xf32, stream, dev)
-                              : launch_decode<2>(a, c, fused, xf32, stream, dev);
+                e = nmat == 1 ? launch_decode<1>(a, c, stream, dev) : launch_decode<2>(a, c, stream, dev);
             return cuda_status(e);
         }
         if (dispatch != BITNET_DISPATCH_AUTO) return BITNET_ERR_UNSUPPORTED_SHAPE;
+    } else if (M > kDecodeMaxM && (dispatch == BITNET_DISPATCH_DECODE || dispatch == BITNET_DISPATCH_DECODE_FUSED)) {
+        return BITNET_ERR_UNSUPPORTED_SHAPE;
     }
 
     // ---- prefill: quantiser kernel, then the tcgen05 GEMM ----

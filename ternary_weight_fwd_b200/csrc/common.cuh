@@ -101,6 +101,87 @@ BITNET_DEVINL bool mbar_wait(uint64_t *bar, uint32_t parity)
     }
 }
 
+// Cluster-scope variant: waits until a phase completed by remote arrivals or
+// remote st.async transactions, and makes the peers' writes visible.
+BITNET_DEVINL bool mbar_try_wait_cluster(uint32_t bar_addr, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar_addr), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+BITNET_DEVINL bool mbar_wait_cluster(uint64_t *bar, uint32_t parity)
+{
+    const uint32_t a = smem_u32(bar);
+    if (mbar_try_wait_cluster(a, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t spin = 1;; ++spin) {
+        if (mbar_try_wait_cluster(a, parity)) return true;
+        if ((spin & 255u) == 0) {
+            if (status_failed()) return false;
+            if (globaltimer_ns() - t0 > BITNET_WAIT_LIMIT_NS) {
+                record_status(BITNET_ERR_TIMEOUT);
+                return false;
+            }
+        }
+    }
+}
+
+// ---- thread-block clusters / distributed shared memory ------------------
+
+BITNET_DEVINL uint32_t cluster_ctarank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+BITNET_DEVINL uint32_t cluster_id_x()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+    return r;
+}
+
+// Whole-cluster barrier (every thread of every CTA), release/acquire.  Used
+// once at kernel start, before any CTA has anything to wait for.
+BITNET_DEVINL void cluster_sync()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Address of the same shared-memory location in CTA `rank` of this cluster.
+BITNET_DEVINL uint32_t mapa_shared(uint32_t local_addr, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_addr), "r"(rank));
+    return r;
+}
+
+// Asynchronous 8-byte store into a peer CTA's shared memory; the peer's
+// mbarrier (same cluster) counts the bytes on arrival.
+BITNET_DEVINL void st_async_v2(uint32_t remote_addr, int a, int b, uint32_t remote_bar)
+{
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.s32 [%0], {%1, %2}, [%3];" ::"r"(
+                     remote_addr),
+                 "r"(a), "r"(b), "r"(remote_bar)
+                 : "memory");
+}
+
+BITNET_DEVINL void st_async_v4f(uint32_t remote_addr, float a, float b, float c, float d, uint32_t remote_bar)
+{
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                     remote_addr),
+                 "f"(a), "f"(b), "f"(c), "f"(d), "r"(remote_bar)
+                 : "memory");
+}
+
 // ---- bulk / tensor copies (async proxy) ----------------------------------
 
 // 1-D bulk copy global -> shared, completion counted on `bar` (bytes % 16 == 0,

@@ -11,8 +11,9 @@
 //    (programmatic dependent launch).  Weights never depend on the previous
 //    kernel, so in a stream of layers the HBM weight stream of kernel i+1
 //    overlaps the tail of kernel i.
-//  * Activations: either quantised in-CTA from x (FUSED, used for small M*K)
-//    or read as int8 x_q from the workspace written by the quantiser kernel.
+//  * Activations: int8 x_q, per-token scales and row sums from the workspace
+//    written by the quantiser kernel (the cluster kernel in decode_cluster.cuh
+//    fuses that step instead; this kernel serves shapes it does not cover).
 //  * Contraction on the legacy integer tensor path, mma.m16n8k32 u8 x s8:
 //    A = 16 weight rows x 32 codes (c = w + 1 in {0,1,2}, unsigned), B = 32 k x
 //    8 tokens (x_q, signed).  One packed 32-bit word gives 16 codes; the four
@@ -34,28 +35,24 @@ constexpr int DEC_RGM = 4;   // max row groups (of 16) per matrix per CTA
 constexpr int DEC_HDR = 1024; // shared-memory header bytes (barriers, per-token scalars)
 
 struct DecodeArgs {
-    const void *x;          // [M][K] bf16/f32 (FUSED)
-    const int8_t *xq;       // [M][K] int8 (non-fused)
-    const float *s_in;      // [M]     (non-fused)
-    const int32_t *rs_in;   // [M]     (non-fused)
+    const int8_t *xq;       // [M][K] int8 quantised activations
+    const float *s_in;      // [M] per-token scales
+    const int32_t *rs_in;   // [M] per-token sums of x_q
     const uint8_t *w0, *w1; // [N][K/4] packed
     const float *gamma0, *gamma1;
     float *y;               // [M][N]
     int32_t *acc0, *acc1;   // [M][N] optional
-    int8_t *xq_out;         // [M][K] optional (FUSED, written by CTA 0)
-    float *s_out;           // [M]    optional (FUSED, written by CTA 0)
     int M, N, K;
     int grid;               // CTAs sharing the N rows
     int rg;                 // row groups per matrix per CTA (<= DEC_RGM)
     int w_stride;           // shared bytes per weight row (== 16 mod 128)
-    int x_stride;           // shared bytes per x_q row (== 64 mod 128, FUSED)
     int rp;                 // reduction row pitch in ints (== 4 mod 32)
 };
 
 BITNET_DEVINL void mma_u8s8_16832(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
                                   uint32_t b1)
 {
-    asm volatile("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
                  "{%0,%1,%2,%3};"
                  : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
                  : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
@@ -84,65 +81,8 @@ BITNET_DEVINL void dec_kstep(int (&acc)[NMAT][DEC_RGM][4], const uint8_t *sW, in
     }
 }
 
-// In-CTA quantisation of tokens [m0, m0+mt) into sX (stride x_stride), per-token
-// s and row sums into tok_s / tok_rs.  All threads participate.
-template <bool XF32>
-BITNET_DEVINL void dec_fused_quant(const DecodeArgs &a, int m0, int mt, uint8_t *sX, float *tok_s, int *tok_rs,
-                                   float *red_max, int *red_rs, bool write_xq)
-{
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    constexpr int EPC = XF32 ? 4 : 8;
-    const int nch = a.K / EPC;
-    const size_t esz = XF32 ? 4 : 2;
-    const char *xb = static_cast<const char *>(a.x);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        if (j < mt) {
-            const uint4 *row = reinterpret_cast<const uint4 *>(xb + (size_t)(m0 + j) * a.K * esz);
-            float mx = 0.0f;
-            for (int c = tid; c < nch; c += DEC_THREADS) mx = fmaxf(mx, chunk_absmax<XF32>(__ldg(row + c)));
-            mx = warp_max(mx);
-            if (lane == 0) red_max[warp * 8 + j] = mx;
-        }
-    }
-    __syncthreads();
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        if (j < mt) {
-            float amax = red_max[j];
-#pragma unroll
-            for (int w = 1; w < DEC_WARPS; ++w) amax = fmaxf(amax, red_max[w * 8 + j]);
-            const float sc = quant_scale(amax);
-            const uint4 *row = reinterpret_cast<const uint4 *>(xb + (size_t)(m0 + j) * a.K * esz);
-            uint8_t *dst = sX + j * a.x_stride;
-            int8_t *gdst = write_xq ? a.xq_out + (size_t)(m0 + j) * a.K : nullptr;
-            int rs = 0;
-            for (int c = tid; c < nch; c += DEC_THREADS) {
-                const uint2 q = chunk_quant<XF32>(__ldg(row + c), sc, rs);
-                if constexpr (XF32) {
-                    reinterpret_cast<uint32_t *>(dst)[c] = q.x;
-                    if (gdst) reinterpret_cast<uint32_t *>(gdst)[c] = q.x;
-                } else {
-                    reinterpret_cast<uint2 *>(dst)[c] = q;
-                    if (gdst) reinterpret_cast<uint2 *>(gdst)[c] = q;
-                }
-            }
-            rs = warp_sum(rs);
-            if (lane == 0) red_rs[warp * 8 + j] = rs;
-            if (tid == 0) tok_s[j] = sc;
-        }
-    }
-    __syncthreads();
-    if (tid < mt) {
-        int rs = 0;
-#pragma unroll
-        for (int w = 0; w < DEC_WARPS; ++w) rs += red_rs[w * 8 + tid];
-        tok_rs[tid] = rs;
-    }
-}
-
-// CH = k-steps per warp held in registers per chunk (non-fused path).
-template <int NMAT, bool FUSED, bool XF32, int CH>
+// CH = k-steps per warp held in registers per chunk.
+template <int NMAT, int CH>
 __global__ void __launch_bounds__(DEC_THREADS, 2) k_decode(const DecodeArgs a)
 {
     extern __shared__ __align__(128) unsigned char smem[];
@@ -150,13 +90,10 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) k_decode(const DecodeArgs a)
     float *tok_s = reinterpret_cast<float *>(smem + 64);    // [8]
     int *tok_rs = reinterpret_cast<int *>(smem + 96);       // [8]
     float *tok_r = reinterpret_cast<float *>(smem + 128);   // [2][8]
-    float *red_max = reinterpret_cast<float *>(smem + 256); // [8 warps][8]
-    int *red_rs = reinterpret_cast<int *>(smem + 512);      // [8 warps][8]
     uint8_t *sW = smem + DEC_HDR;
     const int rg = a.rg;
     const size_t w_bytes = (size_t)NMAT * rg * 16 * a.w_stride;
     int *sRed = reinterpret_cast<int *>(sW + w_bytes); // [NMAT][8 tok][rp]
-    uint8_t *sX = reinterpret_cast<uint8_t *>(sRed + NMAT * 8 * a.rp);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, t4 = lane & 3;
@@ -189,16 +126,10 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) k_decode(const DecodeArgs a)
 
     for (int m0 = 0; m0 < a.M; m0 += 8) {
         const int mt = min(8, a.M - m0);
-        // ---- activations of this 8-token tile ----
-        if constexpr (FUSED) {
-            dec_fused_quant<XF32>(a, m0, mt, sX, tok_s, tok_rs, red_max, red_rs,
-                                  blockIdx.x == 0 && a.xq_out != nullptr);
-            if (blockIdx.x == 0 && a.s_out && tid < mt) a.s_out[m0 + tid] = tok_s[tid];
-        } else {
-            if (tid < mt) {
-                tok_s[tid] = a.s_in[m0 + tid];
-                tok_rs[tid] = a.rs_in[m0 + tid];
-            }
+        // ---- scales and row sums of this 8-token tile (from the quantiser kernel) ----
+        if (tid < mt) {
+            tok_s[tid] = a.s_in[m0 + tid];
+            tok_rs[tid] = a.rs_in[m0 + tid];
         }
         for (int i = tid; i < NMAT * 8 * a.rp; i += DEC_THREADS) sRed[i] = 0;
         __syncthreads();
@@ -220,12 +151,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) k_decode(const DecodeArgs a)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) acc[mat][r][e] = 0;
 
-        if constexpr (FUSED) {
-            for (int ks = warp; ks < KS; ks += DEC_WARPS) {
-                const uint4 xv = *reinterpret_cast<const uint4 *>(sX + g * a.x_stride + ks * 64 + t4 * 16);
-                dec_kstep<NMAT>(acc, sW, a.w_stride, rg, ks, g, t4, xv);
-            }
-        } else {
+        {
             const bool tok_ok = g < mt;
             const int8_t *xrow = a.xq + (size_t)(m0 + (tok_ok ? g : 0)) * a.K + t4 * 16;
             for (int base = warp; base < KS; base += DEC_WARPS * CH) {

@@ -93,6 +93,8 @@ LINEAR_SHAPES = [
     (33, 320, 200, "outliers", "bf16"),       # ragged M, N; K % 128 == 64
     (64, 2560, 2560, "normal", "bf16"),
     (3, 64, 1, "normal", "bf16"),             # minimum K, single output column
+    (5, 576, 300, "normal", "bf16"),          # 9 k-steps over a cluster of 8: ranks without k-steps
+    (40, 1024, 1000, "outliers", "f32"),      # 5 token tiles, fp32 input
 ]
 
 
@@ -158,6 +160,7 @@ def run_ffn(xd, G, U, dispatch, m, n):
 
 
 FFN_SHAPES = [
+    (12, 576, 136, "outliers"),
     (1, 2560, 6912, "normal"),
     (8, 2560, 6912, "normal"),
     (32, 320, 200, "outliers"),
@@ -212,6 +215,27 @@ def test_ffn_chain_down(m):
 
 
 # ---------------------------------------------------------------- cross-checks
+@pytest.mark.parametrize("dispatch,m,kernels", [
+    (tw.BITNET_DISPATCH_AUTO, 8, 1),          # cluster kernel: quantiser fused in
+    (tw.BITNET_DISPATCH_DECODE_FUSED, 64, 1),
+    (tw.BITNET_DISPATCH_DECODE, 8, 2),        # quantiser kernel + row-split decode kernel
+    (tw.BITNET_DISPATCH_PREFILL, 8, 2),       # quantiser kernel + tcgen05 kernel
+    (tw.BITNET_DISPATCH_AUTO, 65, 2),
+])
+def test_kernels_per_call(dispatch, m, kernels):
+    k, n = 2560, 2560
+    W = make_weights(n, k, 1700)
+    xd, _ = make_x(m, k, 1701)
+    tw.bitnet_set_dispatch(dispatch)
+    y = torch.empty((m, n), dtype=torch.float32, device=DEV)
+    ws = torch.empty(tw.bitnet_workspace_size(m, n, k), dtype=torch.uint8, device=DEV)
+    c0 = tw.bitnet_launch_count()
+    tw.bitnet_linear(xd, W["p"], W["g"], y=y, workspace=ws)
+    assert tw.bitnet_launch_count() - c0 == kernels
+    torch.cuda.synchronize()
+
+
+
 def test_all_kernels_agree_bitwise():
     m, k, n = 24, 2560, 6912
     W = make_weights(n, k, 1400)
