@@ -19,6 +19,7 @@
 #include "decode_cluster.cuh"
 #include "pack_quant.cuh"
 #include "prefill.cuh"
+#include "prefill_pair.cuh"
 
 namespace bitnet {
 
@@ -154,6 +155,22 @@ bool encode_u8_2d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t co
     return r == CUDA_SUCCESS;
 }
 
+// 2-D fp32 tensor [rows][cols] (row pitch = cols * 4 bytes), box [box_rows][box_cols], 128-byte swizzle.
+bool encode_f32_2d_sw128(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows,
+                         uint32_t box_cols)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 4};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // ---- decode configuration -----------------------------------------------------
 struct DecodeCfg {
     bool ok;
@@ -236,10 +253,8 @@ bool dc_layout(DcArgs &a, size_t &smem, int64_t K, int nmat, bool xf32, int C, i
     const int KS = (int)(K / 64);
     a.C = C;
     a.ks = (int)cdiv(KS, C);
-    if (a.ks > 16) return false; // weight box row must stay <= 256 bytes
-    a.nbox = (int)cdiv(rpc, 256);
-    a.rows_box = (int)align_up((size_t)cdiv(rpc, a.nbox), 8);
-    a.rpc = a.rows_box * a.nbox;
+    if (a.ks > 16) return false; // at most 1024 k per CTA
+    a.rpc = (int)align_up((size_t)rpc, 8);
     if (nmat * cdiv(a.rpc, 16) > 8 * DC_RGW_MAX) return false; // row groups per warp
     const uint32_t box_w = (uint32_t)a.ks * 16;
     a.w_mat_bytes = (uint32_t)align_up(align_up((size_t)a.rpc, 16) * box_w, 128);
@@ -353,8 +368,7 @@ DcCfg dc_config(int64_t N, int64_t K, int nmat, bool xf32, int dev, int sms)
 }
 
 template <int NMAT, bool XF32, int RGW>
-cudaError_t dc_launch_t(const DcCfg &c, const CUtensorMap &t0, const CUtensorMap &t1, const DcArgs &a,
-                        cudaStream_t stream)
+cudaError_t dc_launch_t(const DcCfg &c, const DcArgs &a, cudaStream_t stream)
 {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(c.nc * a.C));
@@ -371,18 +385,17 @@ cudaError_t dc_launch_t(const DcCfg &c, const CUtensorMap &t0, const CUtensorMap
     cfg.attrs = attr;
     cfg.numAttrs = 2;
     g_launches.fetch_add(1, std::memory_order_relaxed);
-    return cudaLaunchKernelEx(&cfg, k_decode_cluster<NMAT, XF32, RGW>, t0, t1, a);
+    return cudaLaunchKernelEx(&cfg, k_decode_cluster<NMAT, XF32, RGW>, a);
 }
 
 template <int NMAT, bool XF32>
-cudaError_t dc_launch(const DcCfg &c, const CUtensorMap &t0, const CUtensorMap &t1, const DcArgs &a,
-                      cudaStream_t stream)
+cudaError_t dc_launch(const DcCfg &c, const DcArgs &a, cudaStream_t stream)
 {
     switch (c.rgw) {
-    case 1: return dc_launch_t<NMAT, XF32, 1>(c, t0, t1, a, stream);
-    case 2: return dc_launch_t<NMAT, XF32, 2>(c, t0, t1, a, stream);
-    case 4: return dc_launch_t<NMAT, XF32, 4>(c, t0, t1, a, stream);
-    default: return dc_launch_t<NMAT, XF32, 8>(c, t0, t1, a, stream);
+    case 1: return dc_launch_t<NMAT, XF32, 1>(c, a, stream);
+    case 2: return dc_launch_t<NMAT, XF32, 2>(c, a, stream);
+    case 4: return dc_launch_t<NMAT, XF32, 4>(c, a, stream);
+    default: return dc_launch_t<NMAT, XF32, 8>(c, a, stream);
     }
 }
 
@@ -403,22 +416,71 @@ bitnet_status_t dc_forward(const DcCfg &c, const void *x, bool xf32, int64_t M, 
     a.M = (int)M;
     a.N = (int)N;
     a.K = (int)K;
-    CUtensorMap t0, t1;
-    const uint32_t box_w = (uint32_t)a.ks * 16;
-    if (!encode_u8_2d(&t0, w0, (uint64_t)N, (uint64_t)(K / 4), (uint32_t)a.rows_box, box_w, false))
-        return BITNET_ERR_CUDA;
-    if (nmat == 2) {
-        if (!encode_u8_2d(&t1, w1, (uint64_t)N, (uint64_t)(K / 4), (uint32_t)a.rows_box, box_w, false))
-            return BITNET_ERR_CUDA;
-    } else {
-        t1 = t0;
-    }
+    a.w0 = w0;
+    a.w1 = w1;
     cudaError_t e;
     if (nmat == 1)
-        e = xf32 ? dc_launch<1, true>(c, t0, t1, a, stream) : dc_launch<1, false>(c, t0, t1, a, stream);
+        e = xf32 ? dc_launch<1, true>(c, a, stream) : dc_launch<1, false>(c, a, stream);
     else
-        e = xf32 ? dc_launch<2, true>(c, t0, t1, a, stream) : dc_launch<2, false>(c, t0, t1, a, stream);
+        e = xf32 ? dc_launch<2, true>(c, a, stream) : dc_launch<2, false>(c, a, stream);
     return cuda_status(e);
+}
+
+// ---- prefill on CTA pairs ---------------------------------------------------
+template <bool FFN>
+cudaError_t pair_setup(int dev, int *max_pairs)
+{
+    static std::atomic<int> done[kMaxDevices];
+    cudaError_t e = ensure_smem(k_prefill_pair<FFN>, P2_SMEM, done, dev);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * 64);
+    cfg.blockDim = dim3(P2_THREADS);
+    cfg.dynamicSmemBytes = P2_SMEM;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaOccupancyMaxActiveClusters(max_pairs, k_prefill_pair<FFN>, &cfg);
+}
+
+// Co-resident CTA pairs for the pair kernel on this device (0 if unavailable).
+int pair_clusters(int nmat, int dev)
+{
+    static std::atomic<int> cache[2][kMaxDevices];
+    if (dev < 0 || dev >= kMaxDevices) return 0;
+    int v = cache[nmat - 1][dev].load();
+    if (v != 0) return v;
+    int n = 0;
+    cudaError_t e = nmat == 1 ? pair_setup<false>(dev, &n) : pair_setup<true>(dev, &n);
+    v = (e == cudaSuccess && n > 0) ? n : -1;
+    cache[nmat - 1][dev].store(v);
+    return v;
+}
+
+template <bool FFN>
+cudaError_t launch_pair(int npairs, cudaStream_t stream, const CUtensorMap &tmA, const CUtensorMap &tmB0,
+                        const CUtensorMap &tmB1, const CUtensorMap &tmY, const PrefillArgs &a)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(2 * npairs));
+    cfg.blockDim = dim3(P2_THREADS);
+    cfg.dynamicSmemBytes = P2_SMEM;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return cudaLaunchKernelEx(&cfg, k_prefill_pair<FFN>, tmA, tmB0, tmB1, tmY, a);
 }
 
 // Shared body of bitnet_linear (nmat = 1) and bitnet_ffn_gate_up (nmat = 2).
@@ -484,12 +546,13 @@ bitnet_status_t forward(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_
         return BITNET_ERR_UNSUPPORTED_SHAPE;
     }
 
-    // ---- prefill: quantiser kernel, then the tcgen05 GEMM ----
+    // ---- prefill: quantiser kernel, then the tcgen05 GEMM on CTA pairs ----
+    const int pairs = pair_clusters(nmat, dev);
     PrefillArgs a = {};
     a.M = (int)M;
     a.N = (int)N;
     a.K = (int)K;
-    a.num_m = (int)cdiv(M, PF_BM);
+    a.num_m = (int)cdiv(M, pairs > 0 ? 2 * P2_BM : PF_BM);
     a.num_n = (int)cdiv(N, nmat == 1 ? PF_BN : PF_BN / 2);
     a.num_k = (int)cdiv(K, PF_BK);
     a.num_tiles = a.num_m * a.num_n;
@@ -501,7 +564,7 @@ bitnet_status_t forward(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_
     a.acc1 = acc1;
     a.vec_ok = (N % 4) == 0;
     CUtensorMap tmA, tmB0, tmB1;
-    const uint32_t brows = nmat == 1 ? PF_BN : PF_BN / 2;
+    const uint32_t brows = (nmat == 1 && pairs <= 0) ? PF_BN : PF_BN / 2;
     if (!encode_u8_2d(&tmA, xq, (uint64_t)M, (uint64_t)K, PF_BM, PF_BK, true) ||
         !encode_u8_2d(&tmB0, w0, (uint64_t)N, (uint64_t)(K / 4), brows, PF_BK / 4, false))
         return BITNET_ERR_CUDA;
@@ -513,6 +576,15 @@ bitnet_status_t forward(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_
     }
     cudaError_t e = launch_quant(x, xf32, M, K, xq, s, nullptr, stream);
     if (e != cudaSuccess) return BITNET_ERR_CUDA;
+    if (pairs > 0) {
+        // fp32 output through TMA stores (32 x 32 boxes, 128-byte swizzle) when rows are 16-byte multiples
+        CUtensorMap tmY = tmA;
+        if (a.vec_ok && !encode_f32_2d_sw128(&tmY, y, (uint64_t)M, (uint64_t)N, 32, 32)) return BITNET_ERR_CUDA;
+        const int np = std::min(a.num_tiles, pairs);
+        e = nmat == 1 ? launch_pair<false>(np, stream, tmA, tmB0, tmB1, tmY, a)
+                      : launch_pair<true>(np, stream, tmA, tmB0, tmB1, tmY, a);
+        return cuda_status(e);
+    }
     const int grid = std::min(a.num_tiles, sms);
     if (nmat == 1) {
         static std::atomic<int> done[kMaxDevices];

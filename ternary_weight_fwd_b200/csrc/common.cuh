@@ -195,6 +195,19 @@ BITNET_DEVINL void bulk_g2s(void *dst_smem, const void *src_gmem, uint32_t bytes
         : "memory");
 }
 
+// 16-byte asynchronous copy global -> shared (L2 only), Ampere-style.
+BITNET_DEVINL void cp_async16(void *dst_smem, const void *src_gmem)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst_smem)), "l"(src_gmem) : "memory");
+}
+
+// Arrive on `bar` once every cp.async this thread issued so far has landed
+// (the arrival is counted in the barrier's expected count: .noinc).
+BITNET_DEVINL void cp_async_mbar_arrive(uint64_t *bar)
+{
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 // 2-D tiled tensor copy global -> shared (no multicast).  c0 is the innermost
 // coordinate in elements; callers keep c0 * elem_size a multiple of 16 bytes.
 BITNET_DEVINL void tma_load_2d(void *dst_smem, const CUtensorMap *map, int32_t c0, int32_t c1, uint64_t *bar)
@@ -205,6 +218,24 @@ BITNET_DEVINL void tma_load_2d(void *dst_smem, const CUtensorMap *map, int32_t c
         "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
         : "memory");
 }
+
+// 2-D tiled tensor copy shared -> global (bulk-group completion).
+BITNET_DEVINL void tma_store_2d(const CUtensorMap *map, int32_t c0, int32_t c1, const void *src_smem)
+{
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(c0), "r"(c1), "r"(smem_u32(src_smem))
+                 : "memory");
+}
+BITNET_DEVINL void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until at most N committed bulk groups still read their shared source.
+template <int N>
+BITNET_DEVINL void bulk_wait_group_read()
+{
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+// Wait until every committed bulk group has completed (writes performed).
+BITNET_DEVINL void bulk_wait_group_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 BITNET_DEVINL void prefetch_tensormap(const CUtensorMap *map)
 {

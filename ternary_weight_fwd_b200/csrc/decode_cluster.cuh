@@ -8,9 +8,10 @@
 // Why a cluster: a token's scale s = 127 / max_k |x_k| needs the whole row,
 // and every output row needs the whole quantised row.  Instead of every CTA
 // re-reading and re-quantising all of x, the C CTAs of a cluster split K:
-//   1. each CTA bulk-copies its K slice of x (all tokens of the tile) and its
-//      rows x K-slice tile of the packed weights (TMA, issued before the
-//      dependency wait, so the weight stream overlaps the previous kernel);
+//   1. each CTA copies its rows x K-slice tile of the packed weights into
+//      shared memory (16-byte cp.async from every thread, issued before the
+//      dependency wait) and bulk-copies its K slice of x (all tokens of the
+//      tile);
 //   2. it computes per-token partial maxima over its slice and pushes them to
 //      every peer's shared memory (st.async, counted on the peer's mbarrier);
 //   3. every CTA then knows the exact max, so it quantises only its own slice
@@ -37,6 +38,7 @@ constexpr int DC_RGW_MAX = 8; // max row groups (of 16 rows) per warp
 
 struct DcArgs {
     const void *x;
+    const uint8_t *w0, *w1;     // packed [N][K/4]
     const float *gamma0, *gamma1;
     float *y;
     int32_t *acc0, *acc1;
@@ -45,8 +47,6 @@ struct DcArgs {
     int M, N, K;
     int C;         // CTAs per cluster (K split)
     int rpc;       // output rows per cluster (multiple of 8)
-    int rows_box;  // rows per weight TMA box
-    int nbox;      // weight boxes per matrix
     int ks;        // 64-wide k-steps per CTA (the last CTAs may have fewer)
     int own_rows;  // output rows finished by each CTA of the cluster
     int orp;       // row pitch (ints) of a partial-sum block, == 4 mod 8
@@ -74,9 +74,7 @@ BITNET_DEVINL void bulk_s2peer(uint32_t dst_cluster_addr, const void *src_smem, 
 
 // RGW = row groups per warp (1, 2, 4 or 8), chosen by the host for the shape.
 template <int NMAT, bool XF32, int RGW>
-__global__ void __launch_bounds__(DC_THREADS, 2)
-    k_decode_cluster(const __grid_constant__ CUtensorMap tmW0, const __grid_constant__ CUtensorMap tmW1,
-                     const DcArgs a)
+__global__ void __launch_bounds__(DC_THREADS, 2) k_decode_cluster(const DcArgs a)
 {
     extern __shared__ unsigned char dc_smem_raw[];
     unsigned char *smem =
@@ -117,22 +115,43 @@ __global__ void __launch_bounds__(DC_THREADS, 2)
 
     // ---- barriers, then the weight stream (independent of the previous grid) ----
     if (tid == 0) {
-        mbar_init(bar_w, 1);
+        mbar_init(bar_w, DC_THREADS);
         mbar_init(bar_x, 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bar_amax[i], 1);
             mbar_init(&bar_red[i], 1);
         }
         fence_mbarrier_init();
-        if (R > 0 && ksn > 0) {
-            mbar_arrive_expect_tx(bar_w, (uint32_t)(NMAT * a.nbox * a.rows_box) * box_w);
-            for (int m = 0; m < NMAT; ++m)
-                for (int b = 0; b < a.nbox; ++b)
-                    tma_load_2d(sW + m * a.w_mat_bytes + (uint32_t)(b * a.rows_box) * box_w, m ? &tmW1 : &tmW0,
-                                ks0 * 16, (int)(n0 + b * a.rows_box), bar_w);
-        } else {
-            mbar_arrive(bar_w);
+    }
+    __syncthreads();
+    {
+        // this cluster's rows x this CTA's K slice, 16-byte chunks spread over
+        // all threads; (mat, row, chunk) advanced incrementally (no division)
+        const int total = NMAT * R * ksn;
+        if (total > 0) {
+            const int dq = DC_THREADS / ksn, dr = DC_THREADS % ksn;
+            int kc = tid % ksn, row = tid / ksn, mat = 0;
+            while (row >= R && mat < NMAT) {
+                row -= R;
+                ++mat;
+            }
+            const size_t row_bytes = (size_t)a.K / 4;
+            for (int c = tid; c < total; c += DC_THREADS) {
+                const uint8_t *src = (mat ? a.w1 : a.w0) + (size_t)(n0 + row) * row_bytes + (size_t)(ks0 + kc) * 16;
+                cp_async16(sW + mat * a.w_mat_bytes + (uint32_t)row * box_w + kc * 16, src);
+                kc += dr;
+                row += dq;
+                if (kc >= ksn) {
+                    kc -= ksn;
+                    ++row;
+                }
+                while (row >= R && mat < NMAT) {
+                    row -= R;
+                    ++mat;
+                }
+            }
         }
+        cp_async_mbar_arrive(bar_w);
     }
     pdl_launch_dependents();
     pdl_wait();
