@@ -19,7 +19,6 @@
 #include "decode_cluster.cuh"
 #include "pack_quant.cuh"
 #include "prefill.cuh"
-#include "prefill_pair.cuh"
 
 namespace bitnet {
 
@@ -248,7 +247,7 @@ struct DcCfg {
 };
 
 // Shared-memory layout for `rpc` rows per cluster and cluster size C.
-bool dc_layout(DcArgs &a, size_t &smem, int64_t K, int nmat, bool xf32, int C, int rpc)
+bool dc_layout(DcArgs &a, size_t &smem, int64_t K, int nmat, bool xf32, int C, int rpc, bool single_tile)
 {
     const int KS = (int)(K / 64);
     a.C = C;
@@ -266,9 +265,16 @@ bool dc_layout(DcArgs &a, size_t &smem, int64_t K, int nmat, bool xf32, int C, i
     a.orp = (int)align_up((size_t)a.own_rows, 4);
     if (a.orp % 8 == 0) a.orp += 4; // token rows of a block land 8 banks apart
     a.blk_bytes = (uint32_t)(nmat * 8 * a.orp * 4);
-    a.part_off = (uint32_t)align_up((size_t)a.xq_off + 8 * (size_t)a.xq_stride, 128);
-    a.recv_off = a.part_off + (uint32_t)align_up((size_t)C * a.blk_bytes, 128);
-    smem = (size_t)a.recv_off + (size_t)C * a.blk_bytes + 128;
+    const size_t part_bytes = (size_t)C * a.blk_bytes;
+    const size_t after_xq = align_up((size_t)a.xq_off + 8 * (size_t)a.xq_stride, 128);
+    if (single_tile && part_bytes <= (size_t)nmat * a.w_mat_bytes) {
+        a.part_off = DC_HDR; // one token tile: the weights are dead once the contraction is done
+        a.recv_off = (uint32_t)after_xq;
+    } else {
+        a.part_off = (uint32_t)after_xq;
+        a.recv_off = (uint32_t)(after_xq + align_up(part_bytes, 128));
+    }
+    smem = (size_t)a.recv_off + part_bytes + 128;
     return smem <= kSmemLimit;
 }
 
@@ -276,7 +282,7 @@ bool dc_layout(DcArgs &a, size_t &smem, int64_t K, int nmat, bool xf32, int C, i
 int dc_rgw(const DcArgs &a, int nmat)
 {
     const int64_t per_warp = cdiv(nmat * cdiv(a.rpc, 16), 8);
-    return per_warp <= 1 ? 1 : per_warp <= 2 ? 2 : per_warp <= 4 ? 4 : 8;
+    return per_warp <= 4 ? (int)per_warp : per_warp <= 6 ? 6 : 8;
 }
 
 template <int NMAT, bool XF32, int RGW>
@@ -306,7 +312,9 @@ cudaError_t dc_setup_rgw(int rgw, int dev, int C, size_t smem, int *max_clusters
     switch (rgw) {
     case 1: return dc_kernel_setup<NMAT, XF32, 1>(dev, C, smem, max_clusters);
     case 2: return dc_kernel_setup<NMAT, XF32, 2>(dev, C, smem, max_clusters);
+    case 3: return dc_kernel_setup<NMAT, XF32, 3>(dev, C, smem, max_clusters);
     case 4: return dc_kernel_setup<NMAT, XF32, 4>(dev, C, smem, max_clusters);
+    case 6: return dc_kernel_setup<NMAT, XF32, 6>(dev, C, smem, max_clusters);
     default: return dc_kernel_setup<NMAT, XF32, 8>(dev, C, smem, max_clusters);
     }
 }
@@ -322,11 +330,11 @@ cudaError_t dc_setup(int nmat, bool xf32, int rgw, int dev, int C, size_t smem, 
 
 // Cluster size C = 8 (K split 8 ways) when K has at least 8 k-steps of 64;
 // rows per cluster sized so that one wave of resident clusters covers N.
-DcCfg dc_config(int64_t N, int64_t K, int nmat, bool xf32, int dev, int sms)
+DcCfg dc_config(int64_t N, int64_t K, int nmat, bool xf32, bool single_tile, int dev, int sms)
 {
     struct Entry {
         int64_t N, K;
-        int nmat, xf32, dev;
+        int nmat, xf32, single, dev;
         DcCfg cfg;
     };
     static std::mutex mu;
@@ -336,7 +344,7 @@ DcCfg dc_config(int64_t N, int64_t K, int nmat, bool xf32, int dev, int sms)
         std::lock_guard<std::mutex> lk(mu);
         for (int i = 0; i < ncache; ++i)
             if (cache[i].N == N && cache[i].K == K && cache[i].nmat == nmat && cache[i].xf32 == (int)xf32 &&
-                cache[i].dev == dev)
+                cache[i].single == (int)single_tile && cache[i].dev == dev)
                 return cache[i].cfg;
     }
     DcCfg c = {};
@@ -346,7 +354,7 @@ DcCfg dc_config(int64_t N, int64_t K, int nmat, bool xf32, int dev, int sms)
     size_t smem = 0;
     for (int iter = 0; iter < 4; ++iter) {
         int rpc = (int)align_up((size_t)cdiv(N, nc), 8);
-        while (!dc_layout(c.a, smem, K, nmat, xf32, C, rpc)) {
+        while (!dc_layout(c.a, smem, K, nmat, xf32, C, rpc, single_tile)) {
             if (rpc <= 8 || cdiv(K / 64, C) > 16) return c; // not supported: caller falls back
             rpc = (int)align_up((size_t)(rpc / 2), 8);
         }
@@ -363,7 +371,7 @@ DcCfg dc_config(int64_t N, int64_t K, int nmat, bool xf32, int dev, int sms)
     c.smem = smem;
     c.ok = true;
     std::lock_guard<std::mutex> lk(mu);
-    if (ncache < 64) cache[ncache++] = {N, K, nmat, (int)xf32, dev, c};
+    if (ncache < 64) cache[ncache++] = {N, K, nmat, (int)xf32, (int)single_tile, dev, c};
     return c;
 }
 
@@ -394,7 +402,9 @@ cudaError_t dc_launch(const DcCfg &c, const DcArgs &a, cudaStream_t stream)
     switch (c.rgw) {
     case 1: return dc_launch_t<NMAT, XF32, 1>(c, a, stream);
     case 2: return dc_launch_t<NMAT, XF32, 2>(c, a, stream);
+    case 3: return dc_launch_t<NMAT, XF32, 3>(c, a, stream);
     case 4: return dc_launch_t<NMAT, XF32, 4>(c, a, stream);
+    case 6: return dc_launch_t<NMAT, XF32, 6>(c, a, stream);
     default: return dc_launch_t<NMAT, XF32, 8>(c, a, stream);
     }
 }
@@ -426,63 +436,6 @@ bitnet_status_t dc_forward(const DcCfg &c, const void *x, bool xf32, int64_t M, 
     return cuda_status(e);
 }
 
-// ---- prefill on CTA pairs ---------------------------------------------------
-template <bool FFN>
-cudaError_t pair_setup(int dev, int *max_pairs)
-{
-    static std::atomic<int> done[kMaxDevices];
-    cudaError_t e = ensure_smem(k_prefill_pair<FFN>, P2_SMEM, done, dev);
-    if (e != cudaSuccess) return e;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * 64);
-    cfg.blockDim = dim3(P2_THREADS);
-    cfg.dynamicSmemBytes = P2_SMEM;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaOccupancyMaxActiveClusters(max_pairs, k_prefill_pair<FFN>, &cfg);
-}
-
-// Co-resident CTA pairs for the pair kernel on this device (0 if unavailable).
-int pair_clusters(int nmat, int dev)
-{
-    static std::atomic<int> cache[2][kMaxDevices];
-    if (dev < 0 || dev >= kMaxDevices) return 0;
-    int v = cache[nmat - 1][dev].load();
-    if (v != 0) return v;
-    int n = 0;
-    cudaError_t e = nmat == 1 ? pair_setup<false>(dev, &n) : pair_setup<true>(dev, &n);
-    v = (e == cudaSuccess && n > 0) ? n : -1;
-    cache[nmat - 1][dev].store(v);
-    return v;
-}
-
-template <bool FFN>
-cudaError_t launch_pair(int npairs, cudaStream_t stream, const CUtensorMap &tmA, const CUtensorMap &tmB0,
-                        const CUtensorMap &tmB1, const CUtensorMap &tmY, const PrefillArgs &a)
-{
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(2 * npairs));
-    cfg.blockDim = dim3(P2_THREADS);
-    cfg.dynamicSmemBytes = P2_SMEM;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[1].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 2;
-    g_launches.fetch_add(1, std::memory_order_relaxed);
-    return cudaLaunchKernelEx(&cfg, k_prefill_pair<FFN>, tmA, tmB0, tmB1, tmY, a);
-}
-
 // Shared body of bitnet_linear (nmat = 1) and bitnet_ffn_gate_up (nmat = 2).
 bitnet_status_t forward(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_t K, const uint8_t *w0,
                         const float *gamma0, const uint8_t *w1, const float *gamma1, int64_t N, float *y,
@@ -509,7 +462,7 @@ bitnet_status_t forward(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_
     if (M <= kDecodeMaxM && dispatch != BITNET_DISPATCH_PREFILL) {
         // cluster kernel with the quantiser fused in (automatic choice for decode)
         if (dispatch != BITNET_DISPATCH_DECODE) {
-            const DcCfg c = dc_config(N, K, nmat, xf32, dev, sms);
+            const DcCfg c = dc_config(N, K, nmat, xf32, M <= 8, dev, sms);
             if (c.ok)
                 return dc_forward(c, x, xf32, M, K, w0, gamma0, w1, gamma1, N, y, x_q_out, s_out, acc0, acc1,
                                   stream, nmat);
@@ -546,13 +499,12 @@ bitnet_status_t forward(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_
         return BITNET_ERR_UNSUPPORTED_SHAPE;
     }
 
-    // ---- prefill: quantiser kernel, then the tcgen05 GEMM on CTA pairs ----
-    const int pairs = pair_clusters(nmat, dev);
+    // ---- prefill: quantiser kernel, then the tcgen05 GEMM ----
     PrefillArgs a = {};
     a.M = (int)M;
     a.N = (int)N;
     a.K = (int)K;
-    a.num_m = (int)cdiv(M, pairs > 0 ? 2 * P2_BM : PF_BM);
+    a.num_m = (int)cdiv(M, PF_BM);
     a.num_n = (int)cdiv(N, nmat == 1 ? PF_BN : PF_BN / 2);
     a.num_k = (int)cdiv(K, PF_BK);
     a.num_tiles = a.num_m * a.num_n;
@@ -563,8 +515,8 @@ bitnet_status_t forward(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_
     a.acc0 = acc0;
     a.acc1 = acc1;
     a.vec_ok = (N % 4) == 0;
-    CUtensorMap tmA, tmB0, tmB1;
-    const uint32_t brows = (nmat == 1 && pairs <= 0) ? PF_BN : PF_BN / 2;
+    CUtensorMap tmA, tmB0, tmB1, tmY;
+    const uint32_t brows = nmat == 1 ? PF_BN : PF_BN / 2;
     if (!encode_u8_2d(&tmA, xq, (uint64_t)M, (uint64_t)K, PF_BM, PF_BK, true) ||
         !encode_u8_2d(&tmB0, w0, (uint64_t)N, (uint64_t)(K / 4), brows, PF_BK / 4, false))
         return BITNET_ERR_CUDA;
@@ -574,28 +526,22 @@ bitnet_status_t forward(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_
     } else {
         tmB1 = tmB0;
     }
+    // fp32 output through TMA stores (32 x 32 boxes, 128-byte swizzle) when rows are 16-byte multiples
+    tmY = tmA;
+    if (a.vec_ok && !encode_f32_2d_sw128(&tmY, y, (uint64_t)M, (uint64_t)N, 32, 32)) return BITNET_ERR_CUDA;
     cudaError_t e = launch_quant(x, xf32, M, K, xq, s, nullptr, stream);
     if (e != cudaSuccess) return BITNET_ERR_CUDA;
-    if (pairs > 0) {
-        // fp32 output through TMA stores (32 x 32 boxes, 128-byte swizzle) when rows are 16-byte multiples
-        CUtensorMap tmY = tmA;
-        if (a.vec_ok && !encode_f32_2d_sw128(&tmY, y, (uint64_t)M, (uint64_t)N, 32, 32)) return BITNET_ERR_CUDA;
-        const int np = std::min(a.num_tiles, pairs);
-        e = nmat == 1 ? launch_pair<false>(np, stream, tmA, tmB0, tmB1, tmY, a)
-                      : launch_pair<true>(np, stream, tmA, tmB0, tmB1, tmY, a);
-        return cuda_status(e);
-    }
     const int grid = std::min(a.num_tiles, sms);
     if (nmat == 1) {
         static std::atomic<int> done[kMaxDevices];
         e = ensure_smem(k_prefill<false>, PF_SMEM, done, dev);
         if (e == cudaSuccess)
-            e = launch_pdl(k_prefill<false>, dim3(grid), dim3(PF_THREADS), PF_SMEM, stream, tmA, tmB0, tmB1, a);
+            e = launch_pdl(k_prefill<false>, dim3(grid), dim3(PF_THREADS), PF_SMEM, stream, tmA, tmB0, tmB1, tmY, a);
     } else {
         static std::atomic<int> done[kMaxDevices];
         e = ensure_smem(k_prefill<true>, PF_SMEM, done, dev);
         if (e == cudaSuccess)
-            e = launch_pdl(k_prefill<true>, dim3(grid), dim3(PF_THREADS), PF_SMEM, stream, tmA, tmB0, tmB1, a);
+            e = launch_pdl(k_prefill<true>, dim3(grid), dim3(PF_THREADS), PF_SMEM, stream, tmA, tmB0, tmB1, tmY, a);
     }
     return cuda_status(e);
 }

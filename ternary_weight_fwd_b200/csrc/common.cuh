@@ -156,6 +156,11 @@ BITNET_DEVINL void cluster_sync()
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+// Split-phase cluster barrier: every thread arrives (release) and later waits
+// (acquire); work between the two overlaps the barrier's latency.
+BITNET_DEVINL void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
+BITNET_DEVINL void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
+
 // Address of the same shared-memory location in CTA `rank` of this cluster.
 BITNET_DEVINL uint32_t mapa_shared(uint32_t local_addr, uint32_t rank)
 {

@@ -54,6 +54,8 @@ struct DcArgs {
     uint32_t xs_off, xs_row;    // x slice staging: 8 rows
     uint32_t xq_off, xq_stride; // quantised slice: 8 rows (stride == 64 mod 128)
     uint32_t part_off;          // outgoing partial sums [C owners][NMAT][8 tok][orp] int32
+                                // (reuses the weight region when M <= 8: written after the contraction,
+                                // and a single token tile never needs the weights again)
     uint32_t recv_off;          // incoming partial sums [C sources][NMAT][8 tok][orp] int32
     uint32_t blk_bytes;         // bytes of one [NMAT][8][orp] block
 };
@@ -72,7 +74,7 @@ BITNET_DEVINL void bulk_s2peer(uint32_t dst_cluster_addr, const void *src_smem, 
                  : "memory");
 }
 
-// RGW = row groups per warp (1, 2, 4 or 8), chosen by the host for the shape.
+// RGW = row groups per warp (1, 2, 3, 4, 6 or 8), chosen by the host for the shape.
 template <int NMAT, bool XF32, int RGW>
 __global__ void __launch_bounds__(DC_THREADS, 2) k_decode_cluster(const DcArgs a)
 {
@@ -124,6 +126,7 @@ __global__ void __launch_bounds__(DC_THREADS, 2) k_decode_cluster(const DcArgs a
         fence_mbarrier_init();
     }
     __syncthreads();
+    cluster_arrive(); // peers may send to this CTA once every CTA of the cluster has arrived here
     {
         // this cluster's rows x this CTA's K slice, 16-byte chunks spread over
         // all threads; (mat, row, chunk) advanced incrementally (no division)
@@ -167,7 +170,6 @@ __global__ void __launch_bounds__(DC_THREADS, 2) k_decode_cluster(const DcArgs a
         }
     };
     if (tid == 0) issue_x(0, min(8, a.M));
-    cluster_sync(); // every peer's barriers exist before anyone sends to them
 
     const float gam0 = a.gamma0[0];
     const float gam1 = NMAT == 2 ? a.gamma1[0] : 0.0f;
@@ -208,6 +210,7 @@ __global__ void __launch_bounds__(DC_THREADS, 2) k_decode_cluster(const DcArgs a
             if (lane == 0) amax_slot[r * 8 + warp] = mx;
         }
         __syncthreads();
+        if (tile == 0) cluster_wait(); // every peer's barriers exist before anyone sends to them
         if (tid < C && tid != (int)r) {
             const float *v = &amax_slot[r * 8];
             const uint32_t dst = mapa_shared(smem_u32(&amax_slot[r * 8]), tid);
@@ -265,25 +268,48 @@ __global__ void __launch_bounds__(DC_THREADS, 2) k_decode_cluster(const DcArgs a
             for (int h = 0; h < 2; ++h)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) acc[i][h][e] = 0;
-        if (ok) {
+        if (ok && ksn > 0) {
+            // loads of k-step ks+1 are issued before the MMAs of k-step ks
             constexpr uint32_t M3 = 0x03030303u;
             const unsigned char *xq_lane = sXq + g * a.xq_stride + t4 * 16;
+            const uint32_t hi_off = 8 * box_w;
+            uint4 xv = *reinterpret_cast<const uint4 *>(xq_lane);
+            uint32_t wlo[RGW], whi[RGW];
+#pragma unroll
+            for (int i = 0; i < RGW; ++i) {
+                const unsigned char *p = sW + woff[i];
+                wlo[i] = wact[i] ? *reinterpret_cast<const uint32_t *>(p) : 0u;
+                whi[i] = wact[i] ? *reinterpret_cast<const uint32_t *>(p + hi_off) : 0u;
+            }
 #pragma unroll 1
             for (int ks = 0; ks < ksn; ++ks) {
-                const uint4 xv = *reinterpret_cast<const uint4 *>(xq_lane + ks * 64);
+                const bool more = ks + 1 < ksn;
+                const uint4 xn = more ? *reinterpret_cast<const uint4 *>(xq_lane + (ks + 1) * 64) : xv;
+                uint32_t nlo[RGW], nhi[RGW];
+#pragma unroll
+                for (int i = 0; i < RGW; ++i) {
+                    const unsigned char *p = sW + woff[i] + (ks + 1) * 16;
+                    nlo[i] = (wact[i] && more) ? *reinterpret_cast<const uint32_t *>(p) : 0u;
+                    nhi[i] = (wact[i] && more) ? *reinterpret_cast<const uint32_t *>(p + hi_off) : 0u;
+                }
 #pragma unroll
                 for (int i = 0; i < RGW; ++i) {
                     if (wact[i]) {
-                        const unsigned char *p = sW + woff[i] + ks * 16;
-                        const uint32_t lo = *reinterpret_cast<const uint32_t *>(p);
-                        const uint32_t hi = *reinterpret_cast<const uint32_t *>(p + 8 * box_w);
+                        const uint32_t lo = wlo[i], hi = whi[i];
                         mma_u8s8_16832(acc[i][0], lo & M3, hi & M3, (lo >> 2) & M3, (hi >> 2) & M3, xv.x, xv.y);
                         mma_u8s8_16832(acc[i][1], (lo >> 4) & M3, (hi >> 4) & M3, (lo >> 6) & M3, (hi >> 6) & M3,
                                        xv.z, xv.w);
                     }
                 }
+                xv = xn;
+#pragma unroll
+                for (int i = 0; i < RGW; ++i) {
+                    wlo[i] = nlo[i];
+                    whi[i] = nhi[i];
+                }
             }
         }
+        __syncthreads(); // every warp is done with the weights: `part` may reuse their space
 
         // ---- partial sums (code offset removed) into per-owner blocks ----
         {
@@ -314,6 +340,7 @@ __global__ void __launch_bounds__(DC_THREADS, 2) k_decode_cluster(const DcArgs a
             bulk_s2peer(dst, part + tid * blk_ints, a.blk_bytes, mapa_shared(smem_u32(&bar_red[pp]), tid));
         }
         ok = mbar_wait_cluster(&bar_red[pp], ph) && ok;
+        if (m0 + 8 >= a.M) cluster_arrive(); // this CTA needs nothing more from its peers
 
         // ---- owners: sum the C partials, dequantise, gate, store ----
         for (int idx = tid; idx < nown * mt; idx += DC_THREADS) {
@@ -339,8 +366,9 @@ __global__ void __launch_bounds__(DC_THREADS, 2) k_decode_cluster(const DcArgs a
         __syncthreads();
     }
     if (!wready && tid == 0) mbar_wait_drain(bar_w, 0);
-    // no CTA leaves while a peer's bulk copy may still read its shared memory
-    cluster_sync();
+    // no CTA leaves while a peer's bulk copy may still read its shared memory:
+    // every peer has arrived above only after receiving all of its partial sums
+    cluster_wait();
 }
 
 } // namespace bitnet

@@ -6,7 +6,8 @@
 //
 // One persistent CTA per SM, warp-specialised, 448 threads:
 //   warps 0-3  epilogue: tcgen05.ld the int32 tile, dequantise (acc * gamma/s),
-//              optional ReLU^2 gate, store fp32 rows
+//              optional ReLU^2 gate; 32 x 32 fp32 chunks are staged in
+//              128-byte-swizzled shared memory and written by TMA stores
 //   warp 4     producer: TMA (no multicast) of the int8 activation tile
 //              (128 tokens x 128 k, 128-byte swizzle) and of the packed
 //              ternary tile (256 rows x 32 bytes)
@@ -33,7 +34,9 @@ constexpr int PF_BU_BYTES = PF_BN * PF_BK;  // 32 KiB unpacked int8
 constexpr int PF_BP_BYTES = PF_BN * PF_BK / 4; // 8 KiB packed codes
 constexpr int PF_STAGE_BYTES = PF_A_BYTES + PF_BU_BYTES + PF_BP_BYTES;
 constexpr int PF_HDR = 1024;
-constexpr int PF_SMEM = PF_HDR + PF_STAGES * PF_STAGE_BYTES + 1024; // + alignment slack
+constexpr int PF_EPI_BUF = 32 * 128;              // one warp's 32 rows x 32 fp32 columns
+constexpr int PF_EPI_BYTES = 4 * 2 * PF_EPI_BUF;  // 4 epilogue warps, double-buffered
+constexpr int PF_SMEM = PF_HDR + PF_STAGES * PF_STAGE_BYTES + PF_EPI_BYTES + 1024; // + alignment slack
 constexpr int PF_THREADS = 448;
 constexpr int PF_EPI_WARPS = 4;
 constexpr int PF_TMA_WARP = 4;
@@ -118,7 +121,7 @@ BITNET_DEVINL void pf_store_row32_i(int32_t *dst, const uint32_t (&v)[32], int n
 template <bool FFN>
 __global__ void __launch_bounds__(PF_THREADS, 1)
     k_prefill(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
-              const __grid_constant__ CUtensorMap tmB1, const PrefillArgs a)
+              const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmY, const PrefillArgs a)
 {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *smem =
@@ -131,18 +134,19 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     uint64_t *mma_done = acc_empty + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
     unsigned char *stages = smem + PF_HDR;
+    unsigned char *epi_bufs = stages + PF_STAGES * PF_STAGE_BYTES;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < PF_STAGES; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&unpacked[s], PF_UNPACK_THREADS);
+            mbar_init(&unpacked[s], PF_UNPACK_THREADS / 32); // one arrival per unpack warp
             mbar_init(&empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&acc_full[b], 1);
-            mbar_init(&acc_empty[b], PF_EPI_WARPS * 32);
+            mbar_init(&acc_empty[b], PF_EPI_WARPS); // one arrival per epilogue warp
         }
         mbar_init(mma_done, 1);
         fence_mbarrier_init();
@@ -256,7 +260,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 unsigned char *st = stages + stage * PF_STAGE_BYTES;
                 pf_unpack_stage(st + PF_A_BYTES + PF_BU_BYTES, st + PF_A_BYTES, u);
                 fence_proxy_async_smem();
-                mbar_arrive(&unpacked[stage]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&unpacked[stage]);
                 if (++stage == PF_STAGES) {
                     stage = 0;
                     phase ^= 1;
@@ -265,9 +270,35 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         }
     } else {
         // ---------------- epilogue (warps 0-3: TMEM lanes 32w..32w+31) ----------------
+        // fp32 chunks of 32 rows x 32 columns go through a 128-byte-swizzled
+        // staging buffer (chunk j of row l at l*128 + ((j ^ (l & 7)) << 4), so
+        // the writes are conflict-free) and one TMA store; two buffers per warp.
         pdl_wait();
         const float g0 = a.gamma0[0];
         const float g1 = FFN ? a.gamma1[0] : 0.0f;
+        const bool tma_out = a.vec_ok != 0;
+        unsigned char *wbuf = epi_bufs + warp * 2 * PF_EPI_BUF;
+        int nbuf = 0;
+        auto emit = [&](const float (&o)[32], int m, int n, bool mok) {
+            if (tma_out) {
+                unsigned char *buf = wbuf + nbuf * PF_EPI_BUF;
+                if (lane == 0) bulk_wait_group_read<1>(); // the store that used this buffer has read it
+                __syncwarp();
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    *reinterpret_cast<float4 *>(buf + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                        make_float4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&tmY, n, m - lane, buf); // rows/columns outside y are not written
+                    bulk_commit_group();
+                }
+                nbuf ^= 1;
+            } else if (mok && n < a.N) {
+                pf_store_row32(a.y + (size_t)m * a.N + n, o, a.N - n, false);
+            }
+        };
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < a.num_tiles; tile += gridDim.x) {
@@ -280,7 +311,6 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             const float r0 = __fdiv_rn(g0, sm);
             const float r1 = FFN ? __fdiv_rn(g1, sm) : 0.0f;
             const uint32_t tb = tmem_base + ((uint32_t)(warp * 32) << 16) + (uint32_t)(acc * PF_BN);
-            const bool vec = a.vec_ok != 0;
             if constexpr (!FFN) {
 #pragma unroll 1
                 for (int c = 0; c < PF_BN / 32; ++c) {
@@ -288,12 +318,12 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                     tmem_ld32(tb + 32 * c, v);
                     tmem_wait_ld();
                     const int n = nb * PF_BN + 32 * c;
-                    if (mok && n < a.N) {
+                    if (n < a.N) {
                         float o[32];
 #pragma unroll
                         for (int j = 0; j < 32; ++j) o[j] = __fmul_rn((float)(int)v[j], r0);
-                        pf_store_row32(a.y + (size_t)m * a.N + n, o, a.N - n, vec);
-                        if (a.acc0) pf_store_row32_i(a.acc0 + (size_t)m * a.N + n, v, a.N - n, vec, 0);
+                        emit(o, m, n, mok);
+                        if (a.acc0 && mok) pf_store_row32_i(a.acc0 + (size_t)m * a.N + n, v, a.N - n, false, 0);
                     }
                 }
             } else {
@@ -304,7 +334,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                     tmem_ld32(tb + PF_BN / 2 + 32 * c, vu);
                     tmem_wait_ld();
                     const int n = nb * (PF_BN / 2) + 32 * c;
-                    if (mok && n < a.N) {
+                    if (n < a.N) {
                         float o[32];
 #pragma unroll
                         for (int j = 0; j < 32; ++j) {
@@ -313,19 +343,22 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                             const float gp = gv > 0.0f ? gv : 0.0f;
                             o[j] = __fmul_rn(__fmul_rn(gp, gp), uv);
                         }
-                        pf_store_row32(a.y + (size_t)m * a.N + n, o, a.N - n, vec);
-                        if (a.acc0) pf_store_row32_i(a.acc0 + (size_t)m * a.N + n, vg, a.N - n, vec, 0);
-                        if (a.acc1) pf_store_row32_i(a.acc1 + (size_t)m * a.N + n, vu, a.N - n, vec, 0);
+                        emit(o, m, n, mok);
+                        if (mok && a.acc0) pf_store_row32_i(a.acc0 + (size_t)m * a.N + n, vg, a.N - n, false, 0);
+                        if (mok && a.acc1) pf_store_row32_i(a.acc1 + (size_t)m * a.N + n, vu, a.N - n, false, 0);
                     }
                 }
             }
             tc_fence_before();
-            mbar_arrive(&acc_empty[acc]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[acc]);
             if (++acc == 2) {
                 acc = 0;
                 acc_phase ^= 1;
             }
         }
+        if (tma_out && lane == 0) bulk_wait_group_all();
+        __syncwarp();
     }
 
     tc_fence_before();
