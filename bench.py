@@ -57,9 +57,12 @@ def parse_args():
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--cpu-seconds", type=float, default=10.0, help="budget of the oracle CPU baseline")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--decode-path", choices=["sequence", "per-op"], default="sequence",
+                   help="decode step as one persistent bitnet_decode_sequence launch (default) or one "
+                        "bitnet_linear / bitnet_ffn_gate_up call per projection")
     p.add_argument("--profile", default=None,
                    choices=["decode_q_o", "decode_gate_up", "decode_down", "prefill_q_o", "prefill_gate_up",
-                            "prefill_down"],
+                            "prefill_down", "decode_sequence"],
                    help="profiling harness: build one layer, run this projection kind --profile-reps times "
                         "(no graphs, no timing, no JSON) and exit; for ncu captures of one kernel")
     p.add_argument("--profile-reps", type=int, default=3)
@@ -75,6 +78,7 @@ def workload_config(a, n_gpus):
         "layers": a.layers, "hidden": HIDDEN, "intermediate": INTER,
         "prefill_tokens": a.prefill_tokens, "decode_steps": a.decode_steps, "decode_batch": a.decode_batch,
         "activations": "bf16 N(0,1), fresh per projection; ternary weights from N(0,0.02) latents",
+        "decode_path": a.decode_path,
         "l2": "inputs larger than L2: every pass streams 496 MB of packed weights; prefill activations rotate "
               "over 168 MB",
         "parallelism": f"replicas x{n_gpus} (data parallel, no collective)",
@@ -248,6 +252,8 @@ class Stack:
         ws = max(tw.bitnet_workspace_size(M, INTER, INTER), tw.bitnet_workspace_size(M, HIDDEN, HIDDEN))
         self.ws_pre = torch.empty(ws, dtype=torch.uint8, device=device)
         self.ws_dec = torch.empty(tw.bitnet_workspace_size(B, INTER, INTER), dtype=torch.uint8, device=device)
+        self.ws_seq = tw.bitnet_sequence_workspace(device)
+        self.seq_ops = {}
         self.packed_bytes = sum(p.numel() for L in self.layers for (p, _) in L.values())
 
     # one projection of each kind -------------------------------------------
@@ -275,7 +281,25 @@ class Stack:
             self.gate_up(l, self.pre_x[(3 * l + 2) % self.n_pre], self.pre_out, self.ws_pre, s)
             self.down(l, self.pre_out, self.ws_pre, s)
 
+    def decode_ops(self, t):
+        """The projections of decode step t as bitnet_op_t records (one sequence launch)."""
+        if t not in self.seq_ops:
+            tw, out, ops = self.tw, self.dec_out, []
+            for l in range(self.a.layers):
+                L = self.layers[l]
+                base = t * 3 * self.a.layers + 3 * l
+                ops += [tw.linear_op(self.dec_x[base % self.n_dec], L["q"][0], L["q"][1], out["q"]),
+                        tw.linear_op(self.dec_x[(base + 1) % self.n_dec], L["o"][0], L["o"][1], out["o"]),
+                        tw.ffn_gate_up_op(self.dec_x[(base + 2) % self.n_dec], L["gate"][0], L["gate"][1],
+                                          L["up"][0], L["up"][1], out["h"]),
+                        tw.linear_op(out["h"], L["down"][0], L["down"][1], out["down"])]
+            self.seq_ops[t] = ops
+        return self.seq_ops[t]
+
     def decode_step(self, t, s):
+        if self.a.decode_path == "sequence":
+            self.tw.bitnet_decode_sequence(self.decode_ops(t), self.a.decode_batch, self.ws_seq, stream=s)
+            return
         for l in range(self.a.layers):
             base = t * 3 * self.a.layers + 3 * l
             self.q(l, self.dec_x[base % self.n_dec], self.dec_out, self.ws_dec, s)
@@ -390,6 +414,7 @@ def our_arm(a, n_gpus):
             "prefill_q_o": lambda s: st.q(0, st.pre_x[0], st.pre_out, st.ws_pre, s),
             "prefill_gate_up": lambda s: st.gate_up(0, st.pre_x[0], st.pre_out, st.ws_pre, s),
             "prefill_down": lambda s: st.down(0, st.pre_out, st.ws_pre, s),
+            "decode_sequence": lambda s: st.decode_step(0, s),
         }
         with torch.cuda.stream(stream):
             for _ in range(a.profile_reps):
@@ -476,35 +501,44 @@ def our_arm(a, n_gpus):
     }
 
     # ---- per-kernel averages (CUDA events over graphs of one projection kind) ----
+    # Every kind is timed; "in_step" marks the kinds the timed step runs (the decode
+    # step is either one sequence launch or one call per projection).
     kinds = {}
     R = 4
+    seq = a.decode_path == "sequence"
     with torch.cuda.stream(stream):
         specs = {
+            "decode_sequence": (lambda s: [st.decode_step(t, s) for t in range(R)] if seq else None,
+                                dec_bytes_step, "hbm", 1, R, seq),
             "decode_q_o": (lambda s: [st.q(l, st.dec_x[l % st.n_dec], st.dec_out, st.ws_dec, s)
                                       for _ in range(R) for l in range(Lyr)],
-                           HIDDEN * HIDDEN // 4 + B * HIDDEN * 2 + B * HIDDEN * 4, "hbm", 2 * Lyr),
+                           HIDDEN * HIDDEN // 4 + B * HIDDEN * 2 + B * HIDDEN * 4, "hbm", 2 * Lyr, R * Lyr, not seq),
             "decode_gate_up": (lambda s: [st.gate_up(l, st.dec_x[l % st.n_dec], st.dec_out, st.ws_dec, s)
                                           for _ in range(R) for l in range(Lyr)],
-                               2 * INTER * HIDDEN // 4 + B * HIDDEN * 2 + B * INTER * 4, "hbm", Lyr),
+                               2 * INTER * HIDDEN // 4 + B * HIDDEN * 2 + B * INTER * 4, "hbm", Lyr, R * Lyr,
+                               not seq),
             "decode_down": (lambda s: [st.down(l, st.dec_out, st.ws_dec, s) for _ in range(R) for l in range(Lyr)],
-                            INTER * HIDDEN // 4 + B * INTER * 4 + B * HIDDEN * 4, "hbm", Lyr),
+                            INTER * HIDDEN // 4 + B * INTER * 4 + B * HIDDEN * 4, "hbm", Lyr, R * Lyr, not seq),
             "prefill_q_o": (lambda s: [st.q(l, st.pre_x[l % st.n_pre], st.pre_out, st.ws_pre, s)
-                                       for l in range(Lyr)], 2 * M * HIDDEN * HIDDEN, "tensor", 2 * Lyr),
+                                       for l in range(Lyr)], 2 * M * HIDDEN * HIDDEN, "tensor", 2 * Lyr, Lyr, True),
             "prefill_gate_up": (lambda s: [st.gate_up(l, st.pre_x[l % st.n_pre], st.pre_out, st.ws_pre, s)
-                                           for l in range(Lyr)], 2 * 2 * M * HIDDEN * INTER, "tensor", Lyr),
+                                           for l in range(Lyr)], 2 * 2 * M * HIDDEN * INTER, "tensor", Lyr, Lyr,
+                                True),
             "prefill_down": (lambda s: [st.down(l, st.pre_out, st.ws_pre, s) for l in range(Lyr)],
-                             2 * M * INTER * HIDDEN, "tensor", Lyr),
+                             2 * M * INTER * HIDDEN, "tensor", Lyr, Lyr, True),
         }
-        for name, (fn, work, bound, per_step) in specs.items():
+        for name, (fn, work, bound, per_step, n_ops, in_step) in specs.items():
+            if name == "decode_sequence" and not seq:
+                continue
             c0 = tw.bitnet_launch_count()
             g = capture(torch, stream, fn)
             kern = tw.bitnet_launch_count() - c0
-            n_ops = R * Lyr if name.startswith("decode") else Lyr
             ms = time_graph(torch, stream, g, 3) / n_ops
             reps_step = per_step * (a.decode_steps if name.startswith("decode") else 1)
             kinds[name] = {"us_per_op": ms * 1e3, "kernels_per_op": kern / n_ops, "bound": bound,
-                           "work_per_op": work, "ops_per_step": reps_step,
-                           "share_est": ms * reps_step / ms_step}
+                           "work_per_op": work, "in_step": in_step,
+                           "ops_per_step": reps_step if in_step else 0,
+                           "share_est": ms * reps_step / ms_step if in_step else 0.0}
             del g
     dom = max(kinds, key=lambda k: kinds[k]["share_est"])
     d = kinds[dom]
@@ -519,8 +553,13 @@ def our_arm(a, n_gpus):
     roof["traffic"] = dram_traffic(dom)
     roof["kernel"] = dom
     roof["peak_source"] = f"{peaks_src} (MEASURED_PEAKS.json)" if peaks_src == "measured" else "fallback"
-    roof["note"] = ("achieved = algorithmic bytes (packed weights + activations in + outputs) per op / "
-                    "mean op time in a CUDA graph of consecutive ops (CUDA events on the launch stream)")
+    if dom == "decode_sequence":
+        roof["note"] = ("achieved = algorithmic bytes of one decode step (all packed weights of the stack + "
+                        "activations in + outputs) / mean duration of one sequence launch in a CUDA graph of "
+                        "consecutive decode steps (CUDA events on the launch stream)")
+    else:
+        roof["note"] = ("achieved = algorithmic bytes (packed weights + activations in + outputs) per op / "
+                        "mean op time in a CUDA graph of consecutive ops (CUDA events on the launch stream)")
 
     # ---- end to end: pinned host inputs -> device, step, outputs -> host ----
     e2e = None

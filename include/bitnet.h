@@ -207,6 +207,88 @@ bitnet_status_t bitnet_ffn_gate_up(const void *x, bitnet_dtype_t x_dtype, int64_
                                    float *h, int32_t *acc_g_out, int32_t *acc_u_out,
                                    void *workspace, size_t ws_bytes, cudaStream_t stream);
 
+/* ---- decode sequences: many small-M ops in one persistent launch ---------- */
+
+typedef enum {
+    BITNET_OP_LINEAR = 0,     /* y = BitLinear(x), as bitnet_linear */
+    BITNET_OP_FFN_GATE_UP = 1 /* y = relu(BitLinear_gate(x))^2 * BitLinear_up(x), as bitnet_ffn_gate_up */
+} bitnet_op_kind_t;
+
+/* One op of a sequence.  All pointers are device pointers, 16-byte aligned. */
+typedef struct bitnet_op {
+    int32_t kind;          /* bitnet_op_kind_t */
+    int32_t x_dtype;       /* bitnet_dtype_t of x */
+    const void *x;         /* [M][K] activations (read) */
+    int64_t K;             /* in features: multiple of 64, at most 8192 */
+    int64_t N;             /* out features */
+    const uint8_t *w0;     /* [N][K/4] packed: W, or W_gate for the FFN */
+    const float *gamma0;   /* [1] */
+    const uint8_t *w1;     /* [N][K/4] packed W_up (FFN only, else NULL) */
+    const float *gamma1;   /* [1] (FFN only, else NULL) */
+    float *y;              /* [M][N] fp32 output (written): y, or h for the FFN */
+} bitnet_op_t;
+
+#define BITNET_SEQ_MAX_OPS 128
+#define BITNET_SEQ_MAX_M 64
+
+/* Workspace of bitnet_decode_sequence: completion counters (bytes). */
+size_t bitnet_sequence_workspace_size(void);
+
+/*
+ * Host-only planning step of bitnet_decode_sequence (launches nothing, needs
+ * no GPU): validates the ops exactly as bitnet_decode_sequence does and
+ * writes, per op j, the ordering that the sequence kernel will enforce:
+ *   wait_x[j]  latest i < j whose y overlaps op j's x (read after write), or -1
+ *   wait_y[j]  latest i < j whose x or y overlaps op j's y (write after read /
+ *              write after write), or -1
+ * Byte ranges: x covers M*K elements of x_dtype, y covers M*N floats.
+ */
+bitnet_status_t bitnet_sequence_plan(const bitnet_op_t *ops, int32_t n_ops, int64_t M,
+                                     int32_t *wait_x, int32_t *wait_y);
+
+/*
+ * Run ops[0..n_ops) -- every one a decode-size BitLinear or gated FFN over
+ * the same M tokens -- in ONE persistent kernel launch.  The results are
+ * bit-identical to calling bitnet_linear / bitnet_ffn_gate_up for each op in
+ * order on `stream`: an op whose x is an earlier op's y reads that y, and
+ * every output holds what the last op that writes it stored.  The page has
+ * no counterpart to this call: it is the decode-step execution of the
+ * BitLinear layers that the page's model stacks (page: "Architecture").
+ *
+ * Execution: the grid stays resident; each CTA streams its slice of every
+ * op's packed weights into shared memory ahead of the op (weights are read
+ * before any ordering wait), and an op waits for another op only where the
+ * byte ranges of their activations and outputs overlap (see
+ * bitnet_sequence_plan).  Independent ops therefore overlap.
+ *
+ *   ops, n_ops  1 <= n_ops <= BITNET_SEQ_MAX_OPS ops (host array, read
+ *               during the call only; the launch keeps its own copy)
+ *   M           tokens, 1 <= M <= BITNET_SEQ_MAX_M, the same for every op
+ *   workspace   device memory of bitnet_sequence_workspace_size() bytes,
+ *               ZERO-FILLED before its first use; every call leaves it zero
+ *               again (also after a device-side timeout).  Calls that may
+ *               run at the same time need separate workspaces.
+ *
+ * Errors (nothing is launched): BITNET_ERR_INVALID_ARG for a null pointer, a
+ * bad kind or dtype, an op whose y overlaps its own x, any op's weights or
+ * gammas, or the workspace; BITNET_ERR_UNSUPPORTED_SHAPE for K not a
+ * multiple of 64 or above 8192, or an op too large for the per-CTA weight
+ * slice on this GPU; BITNET_ERR_MISALIGNED; BITNET_ERR_WORKSPACE.
+ * The launch is stream-ordered (it starts once earlier work on `stream` has
+ * finished).  Weights and gammas must not be written by other work while it
+ * runs: they are read ahead of every ordering wait.
+ */
+bitnet_status_t bitnet_decode_sequence(const bitnet_op_t *ops, int32_t n_ops, int64_t M,
+                                       void *workspace, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * Cluster size (CTAs splitting K) of the sequence kernel: 4 (default) or 8.
+ * Returns the previous value, or -1 if the value is not allowed (nothing
+ * changed).  Every size gives bit-identical results.  For tests and tuning;
+ * not synchronised with calls running in other threads.
+ */
+int bitnet_set_sequence_cluster(int cluster_size);
+
 /*
  * Device-side status word.  Kernels whose waits are bounded record
  * BITNET_ERR_TIMEOUT there (and exit) instead of spinning forever.  This call

@@ -31,9 +31,22 @@ BITNET_DISPATCH_DECODE_FUSED = 1
 BITNET_DISPATCH_DECODE = 2
 BITNET_DISPATCH_PREFILL = 3
 
+BITNET_OP_LINEAR = 0
+BITNET_OP_FFN_GATE_UP = 1
+BITNET_SEQ_MAX_OPS = 128
+BITNET_SEQ_MAX_M = 64
+
 QUANT_EPS = 1e-5
 
 _lib = None
+
+
+class bitnet_op_t(ctypes.Structure):
+    """One op of bitnet_decode_sequence (mirrors the C struct)."""
+    _fields_ = [("kind", ctypes.c_int32), ("x_dtype", ctypes.c_int32), ("x", ctypes.c_void_p),
+                ("K", ctypes.c_int64), ("N", ctypes.c_int64), ("w0", ctypes.c_void_p),
+                ("gamma0", ctypes.c_void_p), ("w1", ctypes.c_void_p), ("gamma1", ctypes.c_void_p),
+                ("y", ctypes.c_void_p)]
 
 
 class BitnetError(RuntimeError):
@@ -66,6 +79,11 @@ def load_library(path: str = LIB_PATH):
         "bitnet_set_dispatch": ([I], I),
         "bitnet_launch_count": ([], ctypes.c_uint64),
         "bitnet_linear_noalloc": ([P, I, I64, I64, P, P, I64, P, P], I),
+        "bitnet_sequence_workspace_size": ([], SZ),
+        "bitnet_sequence_plan": ([ctypes.POINTER(bitnet_op_t), ctypes.c_int32, I64,
+                                  ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)], I),
+        "bitnet_decode_sequence": ([ctypes.POINTER(bitnet_op_t), ctypes.c_int32, I64, P, SZ, P], I),
+        "bitnet_set_sequence_cluster": ([I], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -216,3 +234,56 @@ def bitnet_device_status(clear=True, stream=None) -> int:
     _check(load_library().bitnet_device_status(1 if clear else 0, ctypes.byref(out), _stream(stream)),
            "bitnet_device_status")
     return out.value
+
+
+# ---- decode sequences -------------------------------------------------------
+def linear_op(x, w_packed, gamma, y):
+    """Describe y = BitLinear(x) as one op of a decode sequence."""
+    return bitnet_op_t(BITNET_OP_LINEAR, _dtype_code(x), x.data_ptr(), x.shape[1], w_packed.shape[0],
+                       w_packed.data_ptr(), gamma.data_ptr(), None, None, y.data_ptr())
+
+
+def ffn_gate_up_op(x, wg_packed, gamma_g, wu_packed, gamma_u, h):
+    """Describe h = relu(BitLinear_g(x))^2 * BitLinear_u(x) as one op of a decode sequence."""
+    return bitnet_op_t(BITNET_OP_FFN_GATE_UP, _dtype_code(x), x.data_ptr(), x.shape[1], wg_packed.shape[0],
+                       wg_packed.data_ptr(), gamma_g.data_ptr(), wu_packed.data_ptr(), gamma_u.data_ptr(),
+                       h.data_ptr())
+
+
+def _op_array(ops):
+    arr = (bitnet_op_t * max(1, len(ops)))()
+    for i, o in enumerate(ops):
+        arr[i] = o
+    return arr
+
+
+def bitnet_sequence_workspace_size() -> int:
+    return load_library().bitnet_sequence_workspace_size()
+
+
+def bitnet_sequence_workspace(device):
+    """A zero-filled workspace for bitnet_decode_sequence (calls leave it zeroed)."""
+    return torch.zeros(bitnet_sequence_workspace_size(), dtype=torch.uint8, device=device)
+
+
+def bitnet_sequence_plan(ops, m):
+    """Host-only: validate `ops` (bitnet_op_t records) for M = m tokens and return
+    (wait_x, wait_y), the earlier op each one waits for before reading x / writing y."""
+    n = len(ops)
+    wx = (ctypes.c_int32 * max(1, n))()
+    wy = (ctypes.c_int32 * max(1, n))()
+    _check(load_library().bitnet_sequence_plan(_op_array(ops), n, m, wx, wy), "bitnet_sequence_plan")
+    return list(wx[:n]), list(wy[:n])
+
+
+def bitnet_decode_sequence(ops, m, workspace, stream=None):
+    """Run `ops` (bitnet_op_t records over the same m tokens) in one persistent launch."""
+    _check(load_library().bitnet_decode_sequence(_op_array(ops), len(ops), m, _ptr(workspace), workspace.numel(),
+                                                 _stream(stream)), "bitnet_decode_sequence")
+
+
+def bitnet_set_sequence_cluster(cluster_size: int) -> int:
+    prev = load_library().bitnet_set_sequence_cluster(int(cluster_size))
+    if prev < 0:
+        raise ValueError(f"invalid sequence cluster size {cluster_size}")
+    return prev

@@ -12,11 +12,13 @@
 #include <cstring>
 #include <mutex>
 #include <utility>
+#include <vector>
 
 #include "bitnet.h"
 #include "common.cuh"
 #include "decode.cuh"
 #include "decode_cluster.cuh"
+#include "decode_seq.cuh"
 #include "pack_quant.cuh"
 #include "prefill.cuh"
 
@@ -229,12 +231,32 @@ cudaError_t launch_decode(const DecodeArgs &a, const DecodeCfg &c, cudaStream_t 
     }
 }
 
+// Per-token quantiser: rows held in registers (one HBM read) when a row fits
+// in 8 warps x 32 lanes x QR_NCH chunks, otherwise the two-pass kernel.
+template <bool XF32>
+cudaError_t launch_quant_t(const void *x, int64_t M, int64_t K, int8_t *xq, float *s, int32_t *rs,
+                           cudaStream_t stream)
+{
+    const int64_t nch = K / (XF32 ? 4 : 8);
+    const int64_t per_warp = 32 * QR_NCH;
+    if (nch <= per_warp)
+        return launch_pdl(k_quant_rows_reg<XF32, 1>, dim3((unsigned)cdiv(M, 8)), dim3(256), 0, stream, x, M, K, xq,
+                          s, rs);
+    if (nch <= 2 * per_warp)
+        return launch_pdl(k_quant_rows_reg<XF32, 2>, dim3((unsigned)cdiv(M, 4)), dim3(256), 0, stream, x, M, K, xq,
+                          s, rs);
+    if (nch <= 4 * per_warp)
+        return launch_pdl(k_quant_rows_reg<XF32, 4>, dim3((unsigned)cdiv(M, 2)), dim3(256), 0, stream, x, M, K, xq,
+                          s, rs);
+    if (nch <= 8 * per_warp)
+        return launch_pdl(k_quant_rows_reg<XF32, 8>, dim3((unsigned)M), dim3(256), 0, stream, x, M, K, xq, s, rs);
+    return launch_pdl(k_quant_rows<XF32>, dim3((unsigned)cdiv(M, 8)), dim3(256), 0, stream, x, M, K, xq, s, rs);
+}
+
 cudaError_t launch_quant(const void *x, bool xf32, int64_t M, int64_t K, int8_t *xq, float *s, int32_t *rs,
                          cudaStream_t stream)
 {
-    const dim3 grid((unsigned)cdiv(M, 8));
-    if (xf32) return launch_pdl(k_quant_rows<true>, grid, dim3(256), 0, stream, x, M, K, xq, s, rs);
-    return launch_pdl(k_quant_rows<false>, grid, dim3(256), 0, stream, x, M, K, xq, s, rs);
+    return xf32 ? launch_quant_t<true>(x, M, K, xq, s, rs, stream) : launch_quant_t<false>(x, M, K, xq, s, rs, stream);
 }
 
 // ---- cluster (K-split, fused quantiser) decode kernel -------------------------
@@ -546,6 +568,204 @@ bitnet_status_t forward(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_
     return cuda_status(e);
 }
 
+// ---- decode sequences: one persistent launch for many ops -----------------
+std::atomic<int> g_seq_cluster{4};
+constexpr int64_t kSeqMaxK = 64 * DS_MAX_KS * 4; // 8192: at most 32 k-steps per CTA with the smallest cluster (4)
+
+struct ByteRange {
+    uintptr_t lo, hi;
+};
+inline bool overlaps(ByteRange a, ByteRange b) { return a.lo < b.hi && b.lo < a.hi; }
+inline ByteRange range_of(const void *p, size_t bytes)
+{
+    const uintptr_t lo = reinterpret_cast<uintptr_t>(p);
+    return {lo, lo + bytes};
+}
+
+// Validation and hazard analysis (host only, shared by plan and run).
+// extra: one more range no op may write or read (the workspace), may be empty.
+bitnet_status_t seq_plan(const bitnet_op_t *ops, int n, int64_t M, int32_t *wait_x, int32_t *wait_y,
+                         ByteRange extra)
+{
+    if (!ops || n < 1 || n > BITNET_SEQ_MAX_OPS || M < 1) return BITNET_ERR_INVALID_ARG;
+    if (M > BITNET_SEQ_MAX_M) return BITNET_ERR_UNSUPPORTED_SHAPE;
+    std::vector<ByteRange> xr(n), yr(n), ro; // ro: weights and gammas (read-only for the launch)
+    ro.reserve(4 * (size_t)n);
+    for (int i = 0; i < n; ++i) {
+        const bitnet_op_t &o = ops[i];
+        if (o.kind != BITNET_OP_LINEAR && o.kind != BITNET_OP_FFN_GATE_UP) return BITNET_ERR_INVALID_ARG;
+        if (o.x_dtype != BITNET_DTYPE_BF16 && o.x_dtype != BITNET_DTYPE_F32) return BITNET_ERR_INVALID_ARG;
+        const bool ffn = o.kind == BITNET_OP_FFN_GATE_UP;
+        if (!o.x || !o.w0 || !o.gamma0 || !o.y || (ffn && (!o.w1 || !o.gamma1))) return BITNET_ERR_INVALID_ARG;
+        const bitnet_status_t st = check_shape(M, o.N, o.K);
+        if (st != BITNET_OK) return st;
+        if (o.K > kSeqMaxK) return BITNET_ERR_UNSUPPORTED_SHAPE;
+        const void *ptrs[] = {o.x, o.w0, o.gamma0, ffn ? o.w1 : nullptr, ffn ? o.gamma1 : nullptr, o.y};
+        for (const void *q : ptrs)
+            if (q && !aligned16(q)) return BITNET_ERR_MISALIGNED;
+        xr[i] = range_of(o.x, (size_t)M * (size_t)o.K * (o.x_dtype == BITNET_DTYPE_F32 ? 4 : 2));
+        yr[i] = range_of(o.y, (size_t)M * (size_t)o.N * 4);
+        if (overlaps(xr[i], yr[i])) return BITNET_ERR_INVALID_ARG;
+        const size_t wbytes = (size_t)o.N * (size_t)(o.K / 4);
+        ro.push_back(range_of(o.w0, wbytes));
+        ro.push_back(range_of(o.gamma0, 4));
+        if (ffn) {
+            ro.push_back(range_of(o.w1, wbytes));
+            ro.push_back(range_of(o.gamma1, 4));
+        }
+    }
+    for (int j = 0; j < n; ++j) {
+        for (const ByteRange &w : ro)
+            if (overlaps(yr[j], w)) return BITNET_ERR_INVALID_ARG;
+        if (extra.hi > extra.lo && (overlaps(yr[j], extra) || overlaps(xr[j], extra))) return BITNET_ERR_INVALID_ARG;
+    }
+    if (extra.hi > extra.lo)
+        for (const ByteRange &w : ro)
+            if (overlaps(w, extra)) return BITNET_ERR_INVALID_ARG;
+    for (int j = 0; j < n; ++j) {
+        int wx = -1, wy = -1;
+        for (int i = 0; i < j; ++i) {
+            if (overlaps(yr[i], xr[j])) wx = i;
+            if (overlaps(yr[i], yr[j]) || overlaps(xr[i], yr[j])) wy = i;
+        }
+        if (wait_x) wait_x[j] = wx;
+        if (wait_y) wait_y[j] = wy;
+    }
+    return BITNET_OK;
+}
+
+// Clusters of C CTAs (one CTA per SM) that are resident at once on `dev`.
+int seq_clusters(int dev, int C)
+{
+    static std::atomic<int> cache[kMaxDevices][9];
+    static std::atomic<int> smem_done[kMaxDevices];
+    if (dev < 0 || dev >= kMaxDevices || C < 1 || C > 8) return 0;
+    int v = cache[dev][C].load();
+    if (v > 0) return v;
+    if (ensure_smem(k_decode_seq, kSmemLimit, smem_done, dev) != cudaSuccess) return 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(C * 64);
+    cfg.blockDim = dim3(DS_THREADS);
+    cfg.dynamicSmemBytes = kSmemLimit;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&v, k_decode_seq, &cfg) != cudaSuccess || v < 1) return 0;
+    cache[dev][C].store(v);
+    return v;
+}
+
+// Per-op layout and the launch-wide shared-memory map for G clusters of C CTAs.
+bitnet_status_t seq_build(DsProgram &p, const bitnet_op_t *ops, int n, int64_t M, int C, int G,
+                          const int32_t *wx, const int32_t *wy)
+{
+    int ks_max = 1;
+    uint32_t blk_max = 0;
+    for (int i = 0; i < n; ++i) {
+        const bitnet_op_t &o = ops[i];
+        DsOp &d = p.ops[i];
+        d = DsOp{};
+        const int nmat = o.kind == BITNET_OP_FFN_GATE_UP ? 2 : 1;
+        const int KS = (int)(o.K / 64);
+        d.ks = (int)cdiv(KS, C);
+        if (d.ks > DS_MAX_KS) return BITNET_ERR_UNSUPPORTED_SHAPE;
+        d.rpc = (int)align_up((size_t)cdiv(o.N, G), 16);
+        const int64_t per_warp = cdiv((int64_t)nmat * (d.rpc / 16), 8);
+        if (per_warp > DS_RGW) return BITNET_ERR_UNSUPPORTED_SHAPE;
+        d.own_rows = d.rpc / C;
+        d.orp = (int)align_up((size_t)d.own_rows, 4);
+        if (d.orp % 8 == 0) d.orp += 4; // token rows of a block land 8 banks apart
+        d.box_w = 16 * (d.ks | 1);      // odd number of 16-byte chunks: conflict-free fragment loads
+        d.x = o.x;
+        d.w0 = o.w0;
+        d.w1 = nmat == 2 ? o.w1 : nullptr;
+        d.gamma0 = o.gamma0;
+        d.gamma1 = nmat == 2 ? o.gamma1 : nullptr;
+        d.y = o.y;
+        d.K = (int)o.K;
+        d.N = (int)o.N;
+        d.nmat = nmat;
+        d.xf32 = o.x_dtype == BITNET_DTYPE_F32;
+        d.wait_x = wx[i];
+        d.wait_y = wy[i];
+        ks_max = std::max(ks_max, d.ks);
+        blk_max = std::max(blk_max, (uint32_t)(nmat * 8 * d.orp * 4));
+    }
+    p.n_ops = n;
+    p.M = (int)M;
+    p.C = C;
+    p.n_ctas = G * C;
+    // x staging: op i uses buffer i % 2, rows as long as the largest K slice among its ops
+    uint32_t pitch[2] = {16, 16};
+    for (int i = 0; i < n; ++i) {
+        const DsOp &d = p.ops[i];
+        pitch[i & 1] = std::max(pitch[i & 1], (uint32_t)(d.ks * 64 * (d.xf32 ? 4 : 2)));
+    }
+    size_t off = DS_HDR;
+    for (int b = 0; b < 2; ++b) {
+        p.xs_off[b] = (uint32_t)off;
+        p.xs_pitch[b] = pitch[b];
+        off = align_up(off + 8 * (size_t)pitch[b], 128);
+    }
+    uint32_t xs = (uint32_t)ks_max * 64;
+    xs += (uint32_t)(((64 - (int)(xs % 128)) + 128) % 128); // == 64 mod 128
+    p.xq_stride = xs;
+    p.xq_off = (uint32_t)off;
+    p.part_off = (uint32_t)align_up(p.xq_off + 8 * (size_t)xs, 128);
+    const size_t part_bytes = align_up((size_t)C * blk_max, 128);
+    p.recv_off = (uint32_t)(p.part_off + part_bytes);
+    p.ring_off = (uint32_t)(p.recv_off + part_bytes);
+    const size_t usable = kSmemLimit - 128; // the kernel aligns its base to 128 bytes
+    if (p.ring_off + 4096 > usable) return BITNET_ERR_UNSUPPORTED_SHAPE;
+    p.ring_bytes = (uint32_t)((usable - p.ring_off) & ~size_t(127));
+    for (int i = 0; i < n; ++i)
+        if (ds_slice_bytes(p.ops[i]) > p.ring_bytes) return BITNET_ERR_UNSUPPORTED_SHAPE;
+    return BITNET_OK;
+}
+
+constexpr size_t kSeqWorkspaceBytes = 1024;
+static_assert(4 * (DS_MAX_OPS + 1) <= (int)kSeqWorkspaceBytes, "sequence counters");
+static_assert(DS_MAX_OPS == BITNET_SEQ_MAX_OPS, "sequence op limit");
+static_assert(sizeof(DsProgram) <= 32000, "kernel parameter space");
+
+bitnet_status_t decode_sequence(const bitnet_op_t *ops, int n, int64_t M, void *workspace, size_t ws_bytes,
+                                cudaStream_t stream)
+{
+    if (workspace && !aligned16(workspace)) return BITNET_ERR_MISALIGNED;
+    int32_t wx[BITNET_SEQ_MAX_OPS], wy[BITNET_SEQ_MAX_OPS];
+    const ByteRange wsr = workspace ? range_of(workspace, kSeqWorkspaceBytes) : ByteRange{0, 0};
+    bitnet_status_t st = seq_plan(ops, n, M, wx, wy, wsr);
+    if (st != BITNET_OK) return st;
+    if (!workspace || ws_bytes < kSeqWorkspaceBytes) return BITNET_ERR_WORKSPACE;
+    const int dev = current_device();
+    const int C = g_seq_cluster.load();
+    const int G = seq_clusters(dev, C);
+    if (G < 1) return BITNET_ERR_CUDA;
+    static DsProgram prog_proto; // zero-initialised template; each call fills a copy
+    DsProgram p = prog_proto;
+    st = seq_build(p, ops, n, M, C, G, wx, wy);
+    if (st != BITNET_OK) return st;
+    p.counters = static_cast<unsigned *>(workspace);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(G * C));
+    cfg.blockDim = dim3(DS_THREADS);
+    cfg.dynamicSmemBytes = kSmemLimit;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return cuda_status(cudaLaunchKernelEx(&cfg, k_decode_seq, p));
+}
+
 // ---- fixed scratch for bitnet_linear_noalloc -------------------------------
 // Callers of that entry point cannot allocate, so its scratch is a static
 // device array (every GPU that loads the library holds it until exit).  Host
@@ -665,6 +885,26 @@ bitnet_status_t bitnet_ffn_gate_up(const void *x, bitnet_dtype_t x_dtype, int64_
 {
     return forward(x, x_dtype, M, K, wg_packed, gamma_g, wu_packed, gamma_u, N, h, nullptr, nullptr, acc_g_out,
                    acc_u_out, workspace, ws_bytes, stream, 2);
+}
+
+size_t bitnet_sequence_workspace_size(void) { return kSeqWorkspaceBytes; }
+
+bitnet_status_t bitnet_sequence_plan(const bitnet_op_t *ops, int32_t n_ops, int64_t M, int32_t *wait_x,
+                                     int32_t *wait_y)
+{
+    return seq_plan(ops, n_ops, M, wait_x, wait_y, ByteRange{0, 0});
+}
+
+bitnet_status_t bitnet_decode_sequence(const bitnet_op_t *ops, int32_t n_ops, int64_t M, void *workspace,
+                                       size_t ws_bytes, cudaStream_t stream)
+{
+    return decode_sequence(ops, n_ops, M, workspace, ws_bytes, stream);
+}
+
+int bitnet_set_sequence_cluster(int cluster_size)
+{
+    if (cluster_size != 4 && cluster_size != 8) return -1;
+    return g_seq_cluster.exchange(cluster_size);
 }
 
 bitnet_status_t bitnet_device_status(int clear, bitnet_status_t *status_out, cudaStream_t stream)

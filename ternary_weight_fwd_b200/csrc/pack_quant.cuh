@@ -156,4 +156,76 @@ __global__ void __launch_bounds__(256) k_quant_rows(const void *__restrict__ x, 
     }
 }
 
+// One-read variant: each row is held in registers between the absmax and the
+// quantise step, so x is read from HBM exactly once (the two-pass kernel above
+// re-reads rows that no longer sit in cache once the input exceeds L2).  WPR
+// warps share a row (8 / WPR rows per 256-thread CTA); every lane holds up to
+// QR_NCH 16-byte chunks of it.  Same arithmetic as k_quant_rows.
+constexpr int QR_NCH = 16;
+
+template <bool XF32, int WPR>
+__global__ void __launch_bounds__(256) k_quant_rows_reg(const void *__restrict__ x, int64_t M, int64_t K,
+                                                        int8_t *__restrict__ x_q, float *__restrict__ s,
+                                                        int32_t *__restrict__ rowsum)
+{
+    __shared__ float red_max[8];
+    __shared__ int red_sum[8];
+    pdl_launch_dependents();
+    pdl_wait();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr int RPC = 8 / WPR; // rows per CTA
+    const int wr = warp % WPR;   // this warp's part of the row
+    const int64_t m = (int64_t)blockIdx.x * RPC + warp / WPR;
+    const bool live = m < M;
+    constexpr int EPC = XF32 ? 4 : 8; // elements per 16-byte chunk
+    const int nch = (int)(K / EPC);
+    const int c0 = wr * 32 + lane;
+    const uint4 *row = reinterpret_cast<const uint4 *>(static_cast<const char *>(x) + (live ? m : 0) * K * (XF32 ? 4 : 2));
+    uint4 v[QR_NCH];
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < QR_NCH; ++i) {
+        const int c = c0 + i * 32 * WPR;
+        if (live && c < nch) {
+            v[i] = __ldg(row + c);
+            amax = fmaxf(amax, chunk_absmax<XF32>(v[i]));
+        }
+    }
+    amax = warp_max(amax);
+    if (WPR > 1) {
+        if (lane == 0) red_max[warp] = amax;
+        __syncthreads();
+        const int w0 = warp - wr;
+#pragma unroll
+        for (int i = 0; i < WPR; ++i) amax = fmaxf(amax, red_max[w0 + i]);
+    }
+    const float sc = quant_scale(amax);
+    int rs = 0;
+    int8_t *qrow = x_q + (live ? m : 0) * K;
+#pragma unroll
+    for (int i = 0; i < QR_NCH; ++i) {
+        const int c = c0 + i * 32 * WPR;
+        if (live && c < nch) {
+            const uint2 q = chunk_quant<XF32>(v[i], sc, rs);
+            if constexpr (XF32)
+                reinterpret_cast<uint32_t *>(qrow)[c] = q.x;
+            else
+                reinterpret_cast<uint2 *>(qrow)[c] = q;
+        }
+    }
+    rs = warp_sum(rs);
+    if (WPR > 1) {
+        if (lane == 0) red_sum[warp] = rs;
+        __syncthreads();
+        rs = 0;
+        const int w0 = warp - wr;
+#pragma unroll
+        for (int i = 0; i < WPR; ++i) rs += red_sum[w0 + i];
+    }
+    if (live && wr == 0 && lane == 0) {
+        s[m] = sc;
+        if (rowsum) rowsum[m] = rs;
+    }
+}
+
 } // namespace bitnet

@@ -46,6 +46,8 @@ def test_pack_deterministic():
     (1, 256, "normal", "bf16"), (4, 256, "normal", "bf16"), (7, 320, "outliers", "bf16"),
     (64, 2560, "student_t_rows", "bf16"), (33, 6912, "outliers", "bf16"), (4096, 2560, "student_t_rows", "bf16"),
     (5, 2560, "normal", "f32"), (300, 6912, "normal", "f32"),
+    # row held by 8 warps (fp32, K = 16384) and the two-pass kernel for rows longer than that
+    (3, 16384, "normal", "f32"), (2, 65536, "outliers", "bf16"), (9, 65536, "normal", "f32"),
 ])
 def test_quant_act_bit_exact(m, k, kind, dtype):
     xd, xf = make_x(m, k, 200 + m + k, kind, dtype)
@@ -95,6 +97,8 @@ LINEAR_SHAPES = [
     (3, 64, 1, "normal", "bf16"),             # minimum K, single output column
     (5, 576, 300, "normal", "bf16"),          # 9 k-steps over a cluster of 8: ranks without k-steps
     (40, 1024, 1000, "outliers", "f32"),      # 5 token tiles, fp32 input
+    (8, 2560, 640, "normal", "bf16"),         # K / V projections of the 2B4T layer (GQA, 5 KV heads)
+    (8, 2560, 3840, "normal", "bf16"),        # fused q|k|v projection
 ]
 
 
@@ -131,7 +135,7 @@ def test_linear_prefill_ragged(m, k, n, kind, dtype):
     assert_rel_close(y, y_ref)
 
 
-@pytest.mark.parametrize("k,n", [(2560, 6912), (6912, 2560)])
+@pytest.mark.parametrize("k,n", [(2560, 6912), (6912, 2560), (2560, 3840), (2560, 640)])
 def test_linear_prefill_full_size_sampled(k, n):
     """M = 4096 prefill at the 2B4T shapes; every output of 48 sampled rows."""
     m = 4096

@@ -1,0 +1,198 @@
+"""Host logic of bitnet_decode_sequence, without a GPU: argument validation and the
+hazard analysis that decides which earlier op each op waits for.
+
+The rule checked here is the one that makes a sequence equal to running its ops
+one after another: op j must not read x before the latest earlier op that writes
+any byte of it has finished (read after write), and must not write y before the
+latest earlier op that reads or writes any byte of it has finished (write after
+read / write after write).  Pointers are synthetic addresses: planning never
+touches memory."""
+import random
+
+import pytest
+
+import ternary_weight_fwd_b200 as tw
+from ternary_weight_fwd_b200 import build as tw_build
+
+BASE = 1 << 40
+
+
+@pytest.fixture(scope="module", autouse=True)
+def lib():
+    tw_build.build()
+    return tw.load_library()
+
+
+def op(kind, x, k, n, y, w0, g0, w1=None, g1=None, f32=False):
+    return tw.bitnet_op_t(kind, tw.BITNET_DTYPE_F32 if f32 else tw.BITNET_DTYPE_BF16, x, k, n, w0, g0, w1, g1, y)
+
+
+def lin(x, k, n, y, w, g=None, f32=False):
+    return op(tw.BITNET_OP_LINEAR, x, k, n, y, w, g if g is not None else w + (n * k // 4 + 255) // 256 * 256,
+              f32=f32)
+
+
+def brute_force(ops, m):
+    """Reference hazard analysis written from the rule above."""
+    def xr(o):
+        return o.x, o.x + m * o.K * (4 if o.x_dtype == tw.BITNET_DTYPE_F32 else 2)
+
+    def yr(o):
+        return o.y, o.y + m * o.N * 4
+
+    def ov(a, b):
+        return a[0] < b[1] and b[0] < a[1]
+
+    wx, wy = [], []
+    for j, oj in enumerate(ops):
+        rx = [i for i in range(j) if ov(yr(ops[i]), xr(oj))]
+        ry = [i for i in range(j) if ov(yr(ops[i]), yr(oj)) or ov(xr(ops[i]), yr(oj))]
+        wx.append(max(rx) if rx else -1)
+        wy.append(max(ry) if ry else -1)
+    return wx, wy
+
+
+def layer_stack(layers, m, shared_outputs=True):
+    """The decode step of a BitNet layer stack: q, o, gate/up (+ReLU^2), down on h."""
+    H, I = 2560, 6912
+    addr = [BASE]
+
+    def alloc(nbytes):
+        a = addr[0]
+        addr[0] += (nbytes + 4095) // 4096 * 4096
+        return a
+
+    ops = []
+    outs = {k: alloc(m * n * 4) for k, n in (("q", H), ("o", H), ("h", I), ("down", H))}
+    for _ in range(layers):
+        xs = [alloc(m * H * 2) for _ in range(3)]
+        if not shared_outputs:
+            outs = {k: alloc(m * n * 4) for k, n in (("q", H), ("o", H), ("h", I), ("down", H))}
+        ops.append(lin(xs[0], H, H, outs["q"], alloc(H * H // 4), alloc(16)))
+        ops.append(lin(xs[1], H, H, outs["o"], alloc(H * H // 4), alloc(16)))
+        ops.append(op(tw.BITNET_OP_FFN_GATE_UP, xs[2], H, I, outs["h"], alloc(I * H // 4), alloc(16),
+                      alloc(I * H // 4), alloc(16)))
+        ops.append(lin(outs["h"], I, H, outs["down"], alloc(H * I // 4), alloc(16), f32=True))
+    return ops
+
+
+def test_layer_stack_dependencies():
+    ops = layer_stack(30, 8)
+    wx, wy = tw.bitnet_sequence_plan(ops, 8)
+    for l in range(30):
+        q, o, gu, dn = 4 * l, 4 * l + 1, 4 * l + 2, 4 * l + 3
+        assert wx[q] == wx[o] == wx[gu] == -1          # fresh inputs
+        assert wx[dn] == gu                            # down reads h
+        if l == 0:
+            assert wy[q] == wy[o] == wy[dn] == -1 and wy[gu] == -1
+        else:
+            assert wy[q] == q - 4 and wy[o] == o - 4   # same output buffers as the previous layer
+            assert wy[gu] == gu - 3                    # h is still read by the previous down
+            assert wy[dn] == dn - 4
+    assert (wx, wy) == brute_force(ops, 8)
+
+
+def test_private_outputs_have_no_write_hazards():
+    ops = layer_stack(4, 3, shared_outputs=False)
+    wx, wy = tw.bitnet_sequence_plan(ops, 3)
+    assert wy == [-1] * len(ops)
+    assert wx == [-1 if j % 4 != 3 else j - 1 for j in range(len(ops))]
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_random_overlaps_match_brute_force(seed):
+    """Random ops over a small arena, so partial overlaps of every kind occur."""
+    r = random.Random(seed)
+    m = r.choice([1, 2, 8, 13, 64])
+    arena = BASE
+    ops = []
+    wbase = BASE + (1 << 30)  # weights live apart from activations
+    for j in range(r.randint(1, 40)):
+        k = 64 * r.randint(1, 8)
+        n = r.randint(1, 300)
+        f32 = r.random() < 0.3
+        x = arena + 16 * r.randint(0, 4000)
+        y = arena + 16 * r.randint(0, 4000)
+        xb = m * k * (4 if f32 else 2)
+        if x < y + m * n * 4 and y < x + xb:  # an op may not overwrite its own input
+            y = x + xb + 16 * r.randint(0, 64)
+        w = wbase + j * (1 << 20)
+        ops.append(lin(x, k, n, y, w, w + (1 << 19), f32=f32))
+    got = tw.bitnet_sequence_plan(ops, m)
+    assert got == brute_force(ops, m)
+
+
+def _status(ops, m, n=None):
+    lib = tw.load_library()
+    arr = tw._op_array(ops)
+    return lib.bitnet_sequence_plan(arr, len(ops) if n is None else n, m, None, None)
+
+
+def test_rejections():
+    good = lin(BASE, 256, 256, BASE + (1 << 20), BASE + (2 << 20))
+    assert _status([good], 4) == tw.BITNET_OK
+    assert _status([good], 0) == tw.BITNET_ERR_INVALID_ARG
+    assert _status([good], 65) == tw.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert _status([good], 4, n=0) == tw.BITNET_ERR_INVALID_ARG
+    assert _status([good] * 129, 4) == tw.BITNET_ERR_INVALID_ARG
+    assert _status([good] * 128, 4) == tw.BITNET_OK
+    # K not a multiple of 64, K above the sequence kernel's limit
+    assert _status([lin(BASE, 96, 256, BASE + (1 << 20), BASE + (2 << 20))], 4) == tw.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert _status([lin(BASE, 8256, 256, BASE + (1 << 22), BASE + (2 << 22))], 4) == \
+        tw.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert _status([lin(BASE, 8192, 256, BASE + (1 << 22), BASE + (2 << 22))], 4) == tw.BITNET_OK
+    # misaligned pointers
+    assert _status([lin(BASE + 8, 256, 256, BASE + (1 << 20), BASE + (2 << 20))], 4) == tw.BITNET_ERR_MISALIGNED
+    assert _status([lin(BASE, 256, 256, BASE + (1 << 20) + 4, BASE + (2 << 20))], 4) == tw.BITNET_ERR_MISALIGNED
+    # null pointers, bad kind / dtype, FFN without its up projection
+    assert _status([lin(0, 256, 256, BASE + (1 << 20), BASE + (2 << 20))], 4) == tw.BITNET_ERR_INVALID_ARG
+    bad = lin(BASE, 256, 256, BASE + (1 << 20), BASE + (2 << 20))
+    bad.kind = 7
+    assert _status([bad], 4) == tw.BITNET_ERR_INVALID_ARG
+    bad = lin(BASE, 256, 256, BASE + (1 << 20), BASE + (2 << 20))
+    bad.x_dtype = 5
+    assert _status([bad], 4) == tw.BITNET_ERR_INVALID_ARG
+    ffn = op(tw.BITNET_OP_FFN_GATE_UP, BASE, 256, 256, BASE + (1 << 20), BASE + (2 << 20), BASE + (3 << 20))
+    assert _status([ffn], 4) == tw.BITNET_ERR_INVALID_ARG
+    # an op overwriting its own input
+    assert _status([lin(BASE, 256, 256, BASE + 256, BASE + (2 << 20))], 4) == tw.BITNET_ERR_INVALID_ARG
+    # an output overwriting weights or a gamma of any op (they are read ahead of every wait)
+    w1 = BASE + (2 << 20)
+    ops = [lin(BASE, 256, 256, BASE + (1 << 20), w1, w1 + (1 << 16)),
+           lin(BASE + (4 << 20), 256, 256, w1 + 1024, BASE + (3 << 20))]
+    assert _status(ops, 4) == tw.BITNET_ERR_INVALID_ARG
+    ops[1] = lin(BASE + (4 << 20), 256, 256, w1 + (1 << 16), BASE + (3 << 20))
+    assert _status(ops, 4) == tw.BITNET_ERR_INVALID_ARG
+
+
+def test_run_rejects_before_launch():
+    """bitnet_decode_sequence validates like the plan and checks the workspace
+    before it looks for a GPU; a valid call without a GPU fails with a CUDA status."""
+    lib = tw.load_library()
+    good = [lin(BASE, 256, 256, BASE + (1 << 20), BASE + (2 << 20))]
+    arr = tw._op_array(good)
+    ws = BASE + (8 << 20)
+    size = tw.bitnet_sequence_workspace_size()
+    assert size >= 4 * (tw.BITNET_SEQ_MAX_OPS + 1)
+    assert lib.bitnet_decode_sequence(arr, 1, 4, None, size, None) == tw.BITNET_ERR_WORKSPACE
+    assert lib.bitnet_decode_sequence(arr, 1, 4, ws, size - 1, None) == tw.BITNET_ERR_WORKSPACE
+    assert lib.bitnet_decode_sequence(arr, 1, 4, ws + 8, size, None) == tw.BITNET_ERR_MISALIGNED
+    # the workspace may not overlap any operand
+    assert lib.bitnet_decode_sequence(arr, 1, 4, BASE + (1 << 20), size, None) == tw.BITNET_ERR_INVALID_ARG
+    assert lib.bitnet_decode_sequence(arr, 1, 4, BASE + (2 << 20), size, None) == tw.BITNET_ERR_INVALID_ARG
+    assert lib.bitnet_decode_sequence(arr, 0, 4, ws, size, None) == tw.BITNET_ERR_INVALID_ARG
+    import torch
+    if not torch.cuda.is_available():
+        assert lib.bitnet_decode_sequence(arr, 1, 4, ws, size, None) == tw.BITNET_ERR_CUDA
+
+
+def test_cluster_size_setter():
+    prev = tw.bitnet_set_sequence_cluster(8)
+    try:
+        assert tw.bitnet_set_sequence_cluster(4) == 8
+        for bad in (0, 1, 2, 3, 16):
+            with pytest.raises(ValueError):
+                tw.bitnet_set_sequence_cluster(bad)
+        assert tw.bitnet_set_sequence_cluster(4) == 4
+    finally:
+        tw.bitnet_set_sequence_cluster(prev)
