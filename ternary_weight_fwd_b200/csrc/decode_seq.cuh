@@ -173,6 +173,22 @@ BITNET_DEVINL bool mbar_spin(uint64_t *bar, uint32_t parity, bool cluster_scope 
     }
 }
 
+// Shared-memory loads through 32-bit shared-window addresses (the operand
+// pointers are built from an aligned integer address, so the compiler would
+// otherwise emit generic loads).
+BITNET_DEVINL uint32_t lds32(uint32_t a)
+{
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+BITNET_DEVINL uint4 lds128(uint32_t a)
+{
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+    return v;
+}
+
 BITNET_DEVINL uint4 ld_cg_v4(const void *p)
 {
     uint4 v;
@@ -453,14 +469,14 @@ __device__ __forceinline__ void ds_op(const DsProgram &p, const DsOp &op, int j,
         {
             constexpr uint32_t M3 = 0x03030303u;
             const int rs0 = tok_rs[2 * t4], rs1 = tok_rs[2 * t4 + 1];
-            const unsigned char *xq_lane = sXq + g * p.xq_stride + t4 * 16;
+            const uint32_t xq_lane = smem_u32(sXq) + g * p.xq_stride + t4 * 16;
             const uint32_t hi_off = 8 * box_w;
             for (int rgi0 = warp; rgi0 < nrgi; rgi0 += 16) {
                 const int rgi1 = rgi0 + 8;
                 const bool two = rgi1 < nrgi;
                 const int mat0 = rgi0 >= RG ? 1 : 0, mat1 = rgi1 >= RG ? 1 : 0;
-                const unsigned char *w0 = sW + mat0 * w_mat_bytes + (uint32_t)((rgi0 - mat0 * RG) * 16 + g) * box_w + t4 * 4;
-                const unsigned char *w1 = sW + mat1 * w_mat_bytes + (uint32_t)((rgi1 - mat1 * RG) * 16 + g) * box_w + t4 * 4;
+                const uint32_t w0 = smem_u32(sW) + mat0 * w_mat_bytes + (uint32_t)((rgi0 - mat0 * RG) * 16 + g) * box_w + t4 * 4;
+                const uint32_t w1 = smem_u32(sW) + mat1 * w_mat_bytes + (uint32_t)((rgi1 - mat1 * RG) * 16 + g) * box_w + t4 * 4;
                 // four independent accumulator chains per row group: k-step parity x k half
                 int a0[4][4] = {}, a1[4][4] = {};
                 if (st.ok && ksn > 0) {
@@ -468,16 +484,16 @@ __device__ __forceinline__ void ds_op(const DsProgram &p, const DsOp &op, int j,
                     for (int ks = 0; ks < ksn; ks += 2) {
                         const bool has2 = ks + 1 < ksn;
                         const int kb = has2 ? ks + 1 : ks;
-                        const uint4 xa = *reinterpret_cast<const uint4 *>(xq_lane + ks * 64);
-                        const uint4 xb2 = *reinterpret_cast<const uint4 *>(xq_lane + kb * 64);
-                        const uint32_t la0 = *reinterpret_cast<const uint32_t *>(w0 + ks * 16);
-                        const uint32_t ha0 = *reinterpret_cast<const uint32_t *>(w0 + hi_off + ks * 16);
-                        const uint32_t lb0 = *reinterpret_cast<const uint32_t *>(w0 + kb * 16);
-                        const uint32_t hb0 = *reinterpret_cast<const uint32_t *>(w0 + hi_off + kb * 16);
-                        const uint32_t la1 = two ? *reinterpret_cast<const uint32_t *>(w1 + ks * 16) : 0u;
-                        const uint32_t ha1 = two ? *reinterpret_cast<const uint32_t *>(w1 + hi_off + ks * 16) : 0u;
-                        const uint32_t lb1 = two ? *reinterpret_cast<const uint32_t *>(w1 + kb * 16) : 0u;
-                        const uint32_t hb1 = two ? *reinterpret_cast<const uint32_t *>(w1 + hi_off + kb * 16) : 0u;
+                        const uint4 xa = lds128(xq_lane + ks * 64);
+                        const uint4 xb2 = lds128(xq_lane + kb * 64);
+                        const uint32_t la0 = lds32(w0 + ks * 16);
+                        const uint32_t ha0 = lds32(w0 + hi_off + ks * 16);
+                        const uint32_t lb0 = lds32(w0 + kb * 16);
+                        const uint32_t hb0 = lds32(w0 + hi_off + kb * 16);
+                        const uint32_t la1 = two ? lds32(w1 + ks * 16) : 0u;
+                        const uint32_t ha1 = two ? lds32(w1 + hi_off + ks * 16) : 0u;
+                        const uint32_t lb1 = two ? lds32(w1 + kb * 16) : 0u;
+                        const uint32_t hb1 = two ? lds32(w1 + hi_off + kb * 16) : 0u;
                         mma_u8s8_16832(a0[0], la0 & M3, ha0 & M3, (la0 >> 2) & M3, (ha0 >> 2) & M3, xa.x, xa.y);
                         mma_u8s8_16832(a0[1], (la0 >> 4) & M3, (ha0 >> 4) & M3, (la0 >> 6) & M3, (ha0 >> 6) & M3,
                                        xa.z, xa.w);
