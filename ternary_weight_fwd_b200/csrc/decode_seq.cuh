@@ -45,11 +45,11 @@ constexpr int DS_COMPUTE = 256;   // eight compute warps
 constexpr int DS_CONTROL = 128;   // control warps: weight copies and completion signals
 constexpr int DS_THREADS = DS_COMPUTE + DS_CONTROL;
 constexpr int DS_SLOTS = 8;       // weight-ring slots (ops in flight)
-constexpr int DS_HDR = 1024;      // header: barriers and per-token scalars
+constexpr int DS_HDR = 1024 + 8 * 96; // header: barriers, per-token scalars, staged op descriptors
 constexpr int DS_MAX_KS = 32;     // 64-wide k-steps per CTA (x slice kept in registers)
 constexpr int DS_RGW = 8;         // row groups (of 16 output rows) per compute warp (host limit)
 
-struct DsOp {
+struct __align__(16) DsOp {
     const void *x;               // [M][K] bf16 or fp32
     const uint8_t *w0, *w1;      // packed [N][K/4]; w1 (up) only for the gated FFN
     const float *gamma0, *gamma1;
@@ -89,6 +89,27 @@ constexpr int DS_AMAX = 384;                       // float [8 ranks][8 tokens]
 constexpr int DS_STARTS = 640;                     // uint32 [DS_SLOTS] ring starts of live slices
 constexpr int DS_RELEASED = 704;                   // uint32: ops whose weight slice is free
 constexpr int DS_DONE = 708;                       // uint32: ops complete on this CTA
+constexpr int DS_DESC_READY = 712;                 // uint32: op descriptors staged in shared memory
+constexpr int DS_Y_CLEAR = 716;                    // uint32: ops whose y-region ordering wait is satisfied
+constexpr int DS_DESC = 1024;                      // DsOp [DS_DESC_SLOTS]: op j in slot j % DS_DESC_SLOTS
+constexpr int DS_DESC_SLOTS = 8;
+
+static_assert(sizeof(DsOp) == 96 && DS_DESC + DS_DESC_SLOTS * 96 <= DS_HDR, "staged op descriptors");
+
+// Op j's descriptor staged in shared memory (slot j % DS_DESC_SLOTS).
+BITNET_DEVINL const DsOp &ds_desc(unsigned char *smem, int j)
+{
+    return *reinterpret_cast<const DsOp *>(smem + DS_DESC + (j % DS_DESC_SLOTS) * (int)sizeof(DsOp));
+}
+
+// Copy op j's descriptor into its shared-memory slot (one thread).
+BITNET_DEVINL void ds_stage_desc(const DsProgram &p, unsigned char *smem, int j)
+{
+    const uint4 *src = reinterpret_cast<const uint4 *>(&p.ops[j]);
+    uint4 *dst = reinterpret_cast<uint4 *>(smem + DS_DESC + (j % DS_DESC_SLOTS) * (int)sizeof(DsOp));
+#pragma unroll
+    for (int i = 0; i < (int)(sizeof(DsOp) / 16); ++i) dst[i] = src[i];
+}
 
 // Where op slices go in the ring.  Positions are virtual (monotone within a
 // launch); a slice never straddles the ring's end.  Producer and consumers
@@ -311,22 +332,25 @@ struct DsState {
     bool ok;
 };
 
-// Bulk-copy one token tile of op `op`'s x slice into staging buffer `b`
-// (thread 0 only).  Rows are this CTA's K slice of tokens m0 .. m0 + mt - 1.
+// Bulk-copy one token tile of op `op`'s x slice into staging buffer `b`, one
+// token row per lane (called by a whole warp).  Rows are this CTA's K slice of
+// tokens m0 .. m0 + mt - 1; lane 0 arms the buffer's mbarrier.
 BITNET_DEVINL void ds_load_x(const DsProgram &p, const DsOp &op, unsigned char *smem, int b, int m0, int mt, int ks0,
-                             int ksn)
+                             int ksn, int lane)
 {
     uint64_t *bar = reinterpret_cast<uint64_t *>(smem + DS_BAR_X) + b;
     const int esz = op.xf32 ? 4 : 2;
     const uint32_t xrow = (uint32_t)ksn * 64 * esz;
     if (ksn <= 0) {
-        mbar_arrive(bar);
+        if (lane == 0) mbar_arrive(bar);
         return;
     }
-    mbar_arrive_expect_tx(bar, (uint32_t)mt * xrow);
-    unsigned char *dst = smem + p.xs_off[b];
-    const char *src = static_cast<const char *>(op.x) + ((size_t)m0 * op.K + (size_t)ks0 * 64) * esz;
-    for (int t = 0; t < mt; ++t) bulk_g2s(dst + t * p.xs_pitch[b], src + (size_t)t * op.K * esz, xrow, bar);
+    if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)mt * xrow);
+    if (lane < mt) {
+        unsigned char *dst = smem + p.xs_off[b] + lane * p.xs_pitch[b];
+        const char *src = static_cast<const char *>(op.x) + ((size_t)(m0 + lane) * op.K + (size_t)ks0 * 64) * esz;
+        bulk_g2s(dst, src, xrow, bar);
+    }
 }
 
 // One op on the compute warps: every token tile of 8, cluster K-split.
@@ -388,19 +412,24 @@ __device__ __forceinline__ void ds_op(const DsProgram &p, const DsOp &op, int j,
         if (tid == 0) {
             mbar_arrive_expect_tx(&bar_amax[pp], (uint32_t)(C - 1) * 32);
             mbar_arrive_expect_tx(&bar_red[pp], (uint32_t)(C - 1) * blk_bytes);
-            if (m0 > 0 || !st.x_ready) {
-                if (m0 == 0 && op.wait_x >= 0) { // x is written by an earlier op of this launch
+        }
+        if (warp == 0 && (m0 > 0 || !st.x_ready)) {
+            if (m0 == 0 && op.wait_x >= 0) { // x is written by an earlier op of this launch
+                if (lane == 0) {
                     if (op.wait_x == j - 1) ds_signal(p, j - 1); // the previous op: publish it right here
                     st.ok = wait_count(&p.counters[op.wait_x], target) && st.ok;
-                    asm volatile("fence.proxy.async.global;" ::: "memory"); // generic writes -> bulk copy reads
                 }
-                ds_load_x(p, op, smem, xb, m0, mt, ks0, ksn);
+                __syncwarp();
+                asm volatile("fence.proxy.async.global;" ::: "memory"); // generic writes -> bulk copy reads
             }
-            if (m0 == 0 && j + 1 < p.n_ops && p.ops[j + 1].wait_x < 0) {
-                // the next op's first tile reads memory no op of this launch writes: fetch it now
-                const DsOp &nx = p.ops[j + 1];
+            ds_load_x(p, op, smem, xb, m0, mt, ks0, ksn, lane);
+        }
+        if (warp == 7 && m0 == 0 && j + 1 < p.n_ops) {
+            // the next op's first tile reads memory no op of this launch writes: fetch it now
+            const DsOp &nx = ds_desc(smem, j + 1);
+            if (nx.wait_x < 0) {
                 const int nks0 = (int)r * nx.ks;
-                ds_load_x(p, nx, smem, xb ^ 1, 0, min(8, p.M), nks0, max(0, min(nx.ks, nx.K / 64 - nks0)));
+                ds_load_x(p, nx, smem, xb ^ 1, 0, min(8, p.M), nks0, max(0, min(nx.ks, nx.K / 64 - nks0)), lane);
             }
         }
 
@@ -545,7 +574,10 @@ __device__ __forceinline__ void ds_op(const DsProgram &p, const DsOp &op, int j,
         st.ok = mbar_spin(&bar_red[pp], ph, true) && st.ok;
         if (last_op && m0 + 8 >= p.M) cluster_arrive(); // nothing more is needed from the peers
         if (m0 == 0 && op.wait_y >= 0) { // y was read or written by an earlier op of this launch
-            if (tid == 0) st.ok = wait_count(&p.counters[op.wait_y], target) && st.ok;
+            // the control warp acquired that op's completion counter (device scope)
+            // and passed it on through this CTA's y-clear counter
+            if (tid == 0)
+                st.ok = wait_local(reinterpret_cast<const uint32_t *>(smem + DS_Y_CLEAR), (uint32_t)j + 1) && st.ok;
             compute_sync();
         }
 
@@ -593,6 +625,8 @@ __global__ void __launch_bounds__(DS_THREADS, 1) k_decode_seq(const __grid_const
         fence_mbarrier_init();
         *reinterpret_cast<volatile uint32_t *>(smem + DS_RELEASED) = 0u;
         *reinterpret_cast<volatile uint32_t *>(smem + DS_DONE) = 0u;
+        *reinterpret_cast<volatile uint32_t *>(smem + DS_DESC_READY) = 0u;
+        *reinterpret_cast<volatile uint32_t *>(smem + DS_Y_CLEAR) = 0u;
     }
     __syncthreads();
     cluster_arrive(); // peers may send to this CTA once every CTA of the cluster has arrived here
@@ -603,14 +637,37 @@ __global__ void __launch_bounds__(DS_THREADS, 1) k_decode_seq(const __grid_const
         ds_issue(p, smem, iss, 0);
         const uint32_t *released = reinterpret_cast<const uint32_t *>(smem + DS_RELEASED);
         const uint32_t *done = reinterpret_cast<const uint32_t *>(smem + DS_DONE);
+        uint32_t *desc_ready = reinterpret_cast<uint32_t *>(smem + DS_DESC_READY);
+        uint32_t *y_clear = reinterpret_cast<uint32_t *>(smem + DS_Y_CLEAR);
+        // y-region waits are acquired here, ahead of the compute warps' epilogues: op 0's now,
+        // op j + 1's once op j is done (ops run in order, so op j + 1's epilogue comes later)
+        auto clear_y = [&](int k) {
+            const int w = p.ops[k].wait_y;
+            if (w >= 0) wait_count(&p.counters[w], (unsigned)p.n_ctas);
+            st_release_cta(y_clear, (uint32_t)k + 1);
+        };
+        // the first op descriptors, staged in shared memory (one op per thread)
+        const int ctid = tid - DS_COMPUTE;
+        if (ctid < DS_DESC_SLOTS && ctid < p.n_ops) ds_stage_desc(p, smem, ctid);
+        control_sync();
+        if (ctid == 0) {
+            st_release_cta(desc_ready, (uint32_t)min(p.n_ops, DS_DESC_SLOTS));
+            clear_y(0);
+        }
         for (int j = 0; j < p.n_ops; ++j) {
             wait_local(released, (uint32_t)j + 1);
             control_sync();
             ds_issue(p, smem, iss, j + 1);
-            // an op the very next op reads is published by compute thread 0 itself
-            if (tid == DS_COMPUTE && !(j + 1 < p.n_ops && p.ops[j + 1].wait_x == j)) {
+            if (ctid == 0) {
                 wait_local(done, (uint32_t)j + 1);
-                ds_signal(p, j);
+                // an op the very next op reads is published by compute thread 0 itself
+                if (!(j + 1 < p.n_ops && p.ops[j + 1].wait_x == j)) ds_signal(p, j);
+                // op j no longer needs its descriptor slot: stage op j + DS_DESC_SLOTS there
+                if (j + DS_DESC_SLOTS < p.n_ops) {
+                    ds_stage_desc(p, smem, j + DS_DESC_SLOTS);
+                    st_release_cta(desc_ready, (uint32_t)(j + DS_DESC_SLOTS + 1));
+                }
+                if (j + 1 < p.n_ops) clear_y(j + 1);
             }
         }
         asm volatile("cp.async.wait_all;" ::: "memory"); // every weight copy has landed
@@ -619,8 +676,11 @@ __global__ void __launch_bounds__(DS_THREADS, 1) k_decode_seq(const __grid_const
     } else {
         uint32_t head = 0;
         DsState st = {0, 0u, false, true};
+        const uint32_t *desc_ready = reinterpret_cast<const uint32_t *>(smem + DS_DESC_READY);
         for (int j = 0; j < p.n_ops; ++j) {
-            const DsOp &op = p.ops[j];
+            // this op's descriptor (and, for warp 7's prefetch, the next one) is staged
+            st.ok = wait_local(desc_ready, (uint32_t)min(j + 2, p.n_ops)) && st.ok;
+            const DsOp &op = ds_desc(smem, j);
             const uint32_t size = ds_slice_bytes(op);
             const uint32_t start = ring_place(head, size, p.ring_bytes);
             head = start + size;
