@@ -247,6 +247,19 @@ bitnet_status_t bitnet_sequence_plan(const bitnet_op_t *ops, int32_t n_ops, int6
                                      int32_t *wait_x, int32_t *wait_y);
 
 /*
+ * Host-only: the order in which bitnet_decode_sequence runs the ops (launches
+ * nothing, needs no GPU).  order[k] = index into ops of the k-th op run.  The
+ * order keeps every pair of ops whose byte ranges conflict (see
+ * bitnet_sequence_plan) in list order, so every op reads, and every output
+ * ends up holding, exactly what running the ops in list order gives; only
+ * independent ops move.  It follows the list, except that an op reading the
+ * output of the op just before it is deferred behind a later ready op (one
+ * that conflicts with nothing still unscheduled before it), so the consumer
+ * waits less for its producer.
+ */
+bitnet_status_t bitnet_sequence_schedule(const bitnet_op_t *ops, int32_t n_ops, int64_t M, int32_t *order);
+
+/*
  * Run ops[0..n_ops) -- every one a decode-size BitLinear or gated FFN over
  * the same M tokens -- in ONE persistent kernel launch.  The results are
  * bit-identical to calling bitnet_linear / bitnet_ffn_gate_up for each op in
@@ -259,7 +272,8 @@ bitnet_status_t bitnet_sequence_plan(const bitnet_op_t *ops, int32_t n_ops, int6
  * op's packed weights into shared memory ahead of the op (weights are read
  * before any ordering wait), and an op waits for another op only where the
  * byte ranges of their activations and outputs overlap (see
- * bitnet_sequence_plan).  Independent ops therefore overlap.
+ * bitnet_sequence_plan), and independent ops may be reordered (see
+ * bitnet_sequence_schedule) with the same results.
  *
  *   ops, n_ops  1 <= n_ops <= BITNET_SEQ_MAX_OPS ops (host array, read
  *               during the call only; the launch keeps its own copy)

@@ -83,6 +83,8 @@ def load_library(path: str = LIB_PATH):
         "bitnet_sequence_plan": ([ctypes.POINTER(bitnet_op_t), ctypes.c_int32, I64,
                                   ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)], I),
         "bitnet_decode_sequence": ([ctypes.POINTER(bitnet_op_t), ctypes.c_int32, I64, P, SZ, P], I),
+        "bitnet_sequence_schedule": ([ctypes.POINTER(bitnet_op_t), ctypes.c_int32, I64,
+                                      ctypes.POINTER(ctypes.c_int32)], I),
         "bitnet_set_sequence_cluster": ([I], I),
     }
     for name, (args, res) in sig.items():
@@ -274,6 +276,14 @@ def bitnet_sequence_plan(ops, m):
     wy = (ctypes.c_int32 * max(1, n))()
     _check(load_library().bitnet_sequence_plan(_op_array(ops), n, m, wx, wy), "bitnet_sequence_plan")
     return list(wx[:n]), list(wy[:n])
+
+
+def bitnet_sequence_schedule(ops, m):
+    """Host-only: the order (indices into `ops`) in which bitnet_decode_sequence runs them."""
+    n = len(ops)
+    order = (ctypes.c_int32 * max(1, n))()
+    _check(load_library().bitnet_sequence_schedule(_op_array(ops), n, m, order), "bitnet_sequence_schedule")
+    return list(order[:n])
 
 
 def bitnet_decode_sequence(ops, m, workspace, stream=None):

@@ -582,14 +582,17 @@ inline ByteRange range_of(const void *p, size_t bytes)
     return {lo, lo + bytes};
 }
 
-// Validation and hazard analysis (host only, shared by plan and run).
-// extra: one more range no op may write or read (the workspace), may be empty.
-bitnet_status_t seq_plan(const bitnet_op_t *ops, int n, int64_t M, int32_t *wait_x, int32_t *wait_y,
-                         ByteRange extra)
+// Validation (host only, shared by plan, schedule and run); fills the byte
+// ranges each op reads (x) and writes (y).  extra: one more range no op may
+// write or read (the workspace), may be empty.
+bitnet_status_t seq_validate(const bitnet_op_t *ops, int n, int64_t M, ByteRange extra, std::vector<ByteRange> &xr,
+                             std::vector<ByteRange> &yr)
 {
     if (!ops || n < 1 || n > BITNET_SEQ_MAX_OPS || M < 1) return BITNET_ERR_INVALID_ARG;
     if (M > BITNET_SEQ_MAX_M) return BITNET_ERR_UNSUPPORTED_SHAPE;
-    std::vector<ByteRange> xr(n), yr(n), ro; // ro: weights and gammas (read-only for the launch)
+    xr.assign(n, ByteRange{0, 0});
+    yr.assign(n, ByteRange{0, 0});
+    std::vector<ByteRange> ro; // weights and gammas (read-only for the launch)
     ro.reserve(4 * (size_t)n);
     for (int i = 0; i < n; ++i) {
         const bitnet_op_t &o = ops[i];
@@ -622,6 +625,22 @@ bitnet_status_t seq_plan(const bitnet_op_t *ops, int n, int64_t M, int32_t *wait
     if (extra.hi > extra.lo)
         for (const ByteRange &w : ro)
             if (overlaps(w, extra)) return BITNET_ERR_INVALID_ARG;
+    return BITNET_OK;
+}
+
+// Op i must precede op j (i before j in the list): one writes what the other reads or writes.
+inline bool hazard(const std::vector<ByteRange> &xr, const std::vector<ByteRange> &yr, int i, int j)
+{
+    return overlaps(yr[i], xr[j]) || overlaps(yr[i], yr[j]) || overlaps(xr[i], yr[j]);
+}
+
+// Hazard waits of the ops in list order (see bitnet_sequence_plan).
+bitnet_status_t seq_plan(const bitnet_op_t *ops, int n, int64_t M, int32_t *wait_x, int32_t *wait_y,
+                         ByteRange extra)
+{
+    std::vector<ByteRange> xr, yr;
+    const bitnet_status_t st = seq_validate(ops, n, M, extra, xr, yr);
+    if (st != BITNET_OK) return st;
     for (int j = 0; j < n; ++j) {
         int wx = -1, wy = -1;
         for (int i = 0; i < j; ++i) {
@@ -630,6 +649,43 @@ bitnet_status_t seq_plan(const bitnet_op_t *ops, int n, int64_t M, int32_t *wait
         }
         if (wait_x) wait_x[j] = wx;
         if (wait_y) wait_y[j] = wy;
+    }
+    return BITNET_OK;
+}
+
+// Execution order (see bitnet_sequence_schedule): a topological order of the
+// hazard graph, so every op reads and leaves exactly what it would in list
+// order.  Greedy, in list order, except that an op reading the output of the
+// op scheduled just before it is deferred while another op is ready: a
+// consumer then waits less for its producer to finish on every CTA.
+bitnet_status_t seq_schedule(const bitnet_op_t *ops, int n, int64_t M, int32_t *order, ByteRange extra)
+{
+    std::vector<ByteRange> xr, yr;
+    const bitnet_status_t st = seq_validate(ops, n, M, extra, xr, yr);
+    if (st != BITNET_OK) return st;
+    std::vector<int> pending(n, 0);              // unscheduled predecessors
+    std::vector<unsigned char> hz((size_t)n * n); // hz[i * n + j]: i must precede j
+    for (int j = 0; j < n; ++j)
+        for (int i = 0; i < j; ++i)
+            if (hazard(xr, yr, i, j)) {
+                hz[(size_t)i * n + j] = 1;
+                ++pending[j];
+            }
+    std::vector<unsigned char> done(n, 0);
+    int last = -1;
+    for (int k = 0; k < n; ++k) {
+        int pick = -1, first = -1;
+        for (int j = 0; j < n && pick < 0; ++j) {
+            if (done[j] || pending[j] != 0) continue;
+            if (first < 0) first = j;
+            if (last < 0 || !overlaps(yr[last], xr[j])) pick = j;
+        }
+        if (pick < 0) pick = first;
+        order[k] = pick;
+        done[pick] = 1;
+        last = pick;
+        for (int j = pick + 1; j < n; ++j)
+            if (hz[(size_t)pick * n + j]) --pending[j];
     }
     return BITNET_OK;
 }
@@ -699,14 +755,23 @@ bitnet_status_t seq_build(DsProgram &p, const bitnet_op_t *ops, int n, int64_t M
     p.M = (int)M;
     p.C = C;
     p.n_ctas = G * C;
-    // x staging: op i uses buffer i % 2, rows as long as the largest K slice among its ops
-    uint32_t pitch[2] = {16, 16};
+    // x staging: ops whose x no op of the launch writes alternate between buffers 0 and 1 (the
+    // next one is fetched while the current one runs); ops reading an earlier op's output use
+    // buffer 2 (loaded when their wait is over).  Rows as long as the largest K slice in the buffer.
+    uint32_t pitch[3] = {16, 16, 16};
+    int alt = 0;
     for (int i = 0; i < n; ++i) {
-        const DsOp &d = p.ops[i];
-        pitch[i & 1] = std::max(pitch[i & 1], (uint32_t)(d.ks * 64 * (d.xf32 ? 4 : 2)));
+        DsOp &d = p.ops[i];
+        if (d.wait_x >= 0) {
+            d.xbuf = 2;
+        } else {
+            d.xbuf = alt;
+            alt ^= 1;
+        }
+        pitch[d.xbuf] = std::max(pitch[d.xbuf], (uint32_t)(d.ks * 64 * (d.xf32 ? 4 : 2)));
     }
     size_t off = DS_HDR;
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < 3; ++b) {
         p.xs_off[b] = (uint32_t)off;
         p.xs_pitch[b] = pitch[b];
         off = align_up(off + 8 * (size_t)pitch[b], 128);
@@ -736,9 +801,14 @@ bitnet_status_t decode_sequence(const bitnet_op_t *ops, int n, int64_t M, void *
                                 cudaStream_t stream)
 {
     if (workspace && !aligned16(workspace)) return BITNET_ERR_MISALIGNED;
-    int32_t wx[BITNET_SEQ_MAX_OPS], wy[BITNET_SEQ_MAX_OPS];
+    int32_t wx[BITNET_SEQ_MAX_OPS], wy[BITNET_SEQ_MAX_OPS], order[BITNET_SEQ_MAX_OPS];
     const ByteRange wsr = workspace ? range_of(workspace, kSeqWorkspaceBytes) : ByteRange{0, 0};
-    bitnet_status_t st = seq_plan(ops, n, M, wx, wy, wsr);
+    bitnet_status_t st = seq_schedule(ops, n, M, order, wsr);
+    if (st != BITNET_OK) return st;
+    bitnet_op_t sched[BITNET_SEQ_MAX_OPS];
+    for (int k = 0; k < n; ++k) sched[k] = ops[order[k]];
+    ops = sched;
+    st = seq_plan(ops, n, M, wx, wy, wsr);
     if (st != BITNET_OK) return st;
     if (!workspace || ws_bytes < kSeqWorkspaceBytes) return BITNET_ERR_WORKSPACE;
     const int dev = current_device();
@@ -899,6 +969,12 @@ bitnet_status_t bitnet_decode_sequence(const bitnet_op_t *ops, int32_t n_ops, in
                                        size_t ws_bytes, cudaStream_t stream)
 {
     return decode_sequence(ops, n_ops, M, workspace, ws_bytes, stream);
+}
+
+bitnet_status_t bitnet_sequence_schedule(const bitnet_op_t *ops, int32_t n_ops, int64_t M, int32_t *order)
+{
+    if (!order) return BITNET_ERR_INVALID_ARG;
+    return seq_schedule(ops, n_ops, M, order, ByteRange{0, 0});
 }
 
 int bitnet_set_sequence_cluster(int cluster_size)

@@ -64,13 +64,15 @@ struct __align__(16) DsOp {
     int box_w;                   // shared bytes per weight row: 16 * odd (conflict-free rows)
     int wait_x;                  // earlier op that must be complete before x is read (-1: none)
     int wait_y;                  // earlier op that must be complete before y is written (-1: none)
+    int xbuf;                    // x staging buffer: 0/1 alternate among ops whose x can be
+                                 // prefetched, 2 for ops that read an earlier op's output
 };
 
 struct DsProgram {
     int n_ops, M, C, n_ctas;
     unsigned *counters;          // [DS_MAX_OPS] completions, then [1] exits (workspace)
-    uint32_t xs_off[2];          // x staging buffers (op j uses buffer j % 2): 8 token rows each
-    uint32_t xs_pitch[2];        // bytes per token row (the largest K slice of the ops using the buffer)
+    uint32_t xs_off[3];          // x staging buffers (DsOp::xbuf): 8 token rows each
+    uint32_t xs_pitch[3];        // bytes per token row (the largest K slice of the ops using the buffer)
     uint32_t xq_off, xq_stride;  // quantised x slice: 8 rows (stride == 64 mod 128)
     uint32_t part_off, recv_off; // outgoing / incoming partial sums, C blocks each
     uint32_t ring_off, ring_bytes;
@@ -81,7 +83,7 @@ struct DsProgram {
 constexpr int DS_BAR_FULL = 0;                     // [DS_SLOTS] weights landed (one cp.async arrival per control thread)
 constexpr int DS_BAR_AMAX = DS_BAR_FULL + 8 * DS_SLOTS; // [2]
 constexpr int DS_BAR_RED = DS_BAR_AMAX + 16;       // [2]
-constexpr int DS_BAR_X = DS_BAR_RED + 16;          // [2] x staging buffer landed (expect_tx + bulk bytes)
+constexpr int DS_BAR_X = DS_BAR_RED + 16;          // [3] x staging buffer landed (expect_tx + bulk bytes)
 constexpr int DS_TOK_S = 256;                      // float [8]
 constexpr int DS_TOK_RS = 288;                     // int [8]
 constexpr int DS_TOK_R = 320;                      // float [16]
@@ -327,7 +329,7 @@ BITNET_DEVINL void ds_signal(const DsProgram &p, int j)
 // Per-CTA launch state shared by the ops (uniform across the CTA's threads).
 struct DsState {
     int tile;        // token tiles done in this launch (exchange barriers and parity)
-    uint32_t xw;     // completed waits on x staging buffer b in bit b (its next parity)
+    uint32_t xw;     // completed waits on x staging buffer b (0..2) in bit b (its next parity)
     bool x_ready;    // this op's first x tile was prefetched into its buffer
     bool ok;
 };
@@ -397,7 +399,7 @@ __device__ __forceinline__ void ds_op(const DsProgram &p, const DsOp &op, int j,
     const int blk_ints = nmat * 8 * orp;
     const uint32_t blk_bytes = (uint32_t)blk_ints * 4;
     const int slot = j % DS_SLOTS;
-    const int xb = j & 1; // this op's x staging buffer
+    const int xb = op.xbuf; // this op's x staging buffer
     const unsigned char *sXs = smem + p.xs_off[xb];
     const uint32_t xs_pitch = p.xs_pitch[xb];
     const unsigned target = (unsigned)p.n_ctas;
@@ -427,9 +429,9 @@ __device__ __forceinline__ void ds_op(const DsProgram &p, const DsOp &op, int j,
         if (warp == 7 && m0 == 0 && j + 1 < p.n_ops) {
             // the next op's first tile reads memory no op of this launch writes: fetch it now
             const DsOp &nx = ds_desc(smem, j + 1);
-            if (nx.wait_x < 0) {
+            if (nx.wait_x < 0) { // its buffer (0/1) is not this op's and no earlier op still uses it
                 const int nks0 = (int)r * nx.ks;
-                ds_load_x(p, nx, smem, xb ^ 1, 0, min(8, p.M), nks0, max(0, min(nx.ks, nx.K / 64 - nks0)), lane);
+                ds_load_x(p, nx, smem, nx.xbuf, 0, min(8, p.M), nks0, max(0, min(nx.ks, nx.K / 64 - nks0)), lane);
             }
         }
 
@@ -620,8 +622,8 @@ __global__ void __launch_bounds__(DS_THREADS, 1) k_decode_seq(const __grid_const
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bars[DS_BAR_AMAX / 8 + i], 1);
             mbar_init(&bars[DS_BAR_RED / 8 + i], 1);
-            mbar_init(&bars[DS_BAR_X / 8 + i], 1);
         }
+        for (int i = 0; i < 3; ++i) mbar_init(&bars[DS_BAR_X / 8 + i], 1);
         fence_mbarrier_init();
         *reinterpret_cast<volatile uint32_t *>(smem + DS_RELEASED) = 0u;
         *reinterpret_cast<volatile uint32_t *>(smem + DS_DONE) = 0u;
@@ -691,7 +693,7 @@ __global__ void __launch_bounds__(DS_THREADS, 1) k_decode_seq(const __grid_const
         // wait gave up): the last phase waited on each staging buffer is drained
         if (tid == 0) {
             uint64_t *bar_x = reinterpret_cast<uint64_t *>(smem + DS_BAR_X);
-            for (int b = 0; b < 2; ++b) mbar_wait_drain(&bar_x[b], ((st.xw >> b) & 1u) ^ 1u);
+            for (int b = 0; b < 3; ++b) mbar_wait_drain(&bar_x[b], ((st.xw >> b) & 1u) ^ 1u);
         }
     }
     __syncthreads();

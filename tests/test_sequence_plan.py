@@ -9,6 +9,7 @@ read / write after write).  Pointers are synthetic addresses: planning never
 touches memory."""
 import random
 
+import numpy as np
 import pytest
 
 import ternary_weight_fwd_b200 as tw
@@ -120,6 +121,84 @@ def test_random_overlaps_match_brute_force(seed):
         ops.append(lin(x, k, n, y, w, w + (1 << 19), f32=f32))
     got = tw.bitnet_sequence_plan(ops, m)
     assert got == brute_force(ops, m)
+
+
+def simulate(ops, m, order, arena_lo, arena_hi):
+    """Run the ops' memory effects in `order` on a byte-stamp model of the activation
+    arena: each op records the stamps it reads and stamps the bytes it writes."""
+    mem = np.zeros(arena_hi - arena_lo, np.int32)
+    reads = {}
+    for j in order:
+        o = ops[j]
+        xb = m * o.K * (4 if o.x_dtype == tw.BITNET_DTYPE_F32 else 2)
+        reads[j] = mem[o.x - arena_lo: o.x - arena_lo + xb].copy()
+        mem[o.y - arena_lo: o.y - arena_lo + m * o.N * 4] = j + 1
+    return reads, mem
+
+
+def is_topological(ops, m, order):
+    pos = {j: k for k, j in enumerate(order)}
+    wx, wy = brute_force(ops, m)
+    def xr(o):
+        return o.x, o.x + m * o.K * (4 if o.x_dtype == tw.BITNET_DTYPE_F32 else 2)
+    def yr(o):
+        return o.y, o.y + m * o.N * 4
+    def ov(a, b):
+        return a[0] < b[1] and b[0] < a[1]
+    for j in range(len(ops)):
+        for i in range(j):
+            if ov(yr(ops[i]), xr(ops[j])) or ov(yr(ops[i]), yr(ops[j])) or ov(xr(ops[i]), yr(ops[j])):
+                if pos[i] > pos[j]:
+                    return False
+    return True
+
+
+def test_schedule_layer_stack_moves_consumers_away_from_producers():
+    ops = layer_stack(30, 8)
+    order = tw.bitnet_sequence_schedule(ops, 8)
+    assert sorted(order) == list(range(len(ops)))
+    assert is_topological(ops, 8, order)
+    # no down projection runs right after the gate/up whose h it reads, except in the
+    # last layer, where no independent op is left to put between them
+    for k in range(1, len(order)):
+        j, prev = order[k], order[k - 1]
+        if j % 4 == 3 and j < len(ops) - 4:
+            assert prev != j - 1, (k, j, prev)
+    assert order[-2:] == [len(ops) - 2, len(ops) - 1]
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_schedule_preserves_every_read_and_the_final_memory(seed):
+    """Random ops over a small arena: the scheduled order reads and leaves exactly
+    what list order does (byte-stamp model), and is a topological order."""
+    r = random.Random(100 + seed)
+    m = r.choice([1, 2, 8])
+    arena = BASE
+    size = 16 * 6000
+    ops = []
+    wbase = BASE + (1 << 30)
+    for j in range(r.randint(2, 48)):
+        k = 64 * r.randint(1, 4)
+        n = r.randint(1, 120)
+        f32 = r.random() < 0.3
+        xb = m * k * (4 if f32 else 2)
+        yb = m * n * 4
+        x = arena + 16 * r.randint(0, (size - xb) // 16)
+        y = arena + 16 * r.randint(0, (size - yb) // 16)
+        if x < y + yb and y < x + xb:
+            continue
+        w = wbase + j * (1 << 20)
+        ops.append(lin(x, k, n, y, w, w + (1 << 19), f32=f32))
+    if not ops:
+        return
+    order = tw.bitnet_sequence_schedule(ops, m)
+    assert sorted(order) == list(range(len(ops)))
+    assert is_topological(ops, m, order)
+    r0, mem0 = simulate(ops, m, range(len(ops)), arena, arena + size)
+    r1, mem1 = simulate(ops, m, order, arena, arena + size)
+    assert np.array_equal(mem0, mem1)
+    for j in range(len(ops)):
+        assert np.array_equal(r0[j], r1[j]), j
 
 
 def _status(ops, m, n=None):
