@@ -716,7 +716,14 @@ int seq_clusters(int dev, int C)
 }
 
 // Per-op layout and the launch-wide shared-memory map for G clusters of C CTAs.
-bitnet_status_t seq_build(DsProgram &p, const bitnet_op_t *ops, int n, int64_t M, int C, int G,
+// Partitions of the grid: op i runs on clusters [cl0[of[i]], cl0[of[i]] + ncl[of[i]]).
+struct SeqParts {
+    int n = 1;
+    int cl0[DS_MAX_PARTS] = {0}, ncl[DS_MAX_PARTS] = {0};
+    std::vector<int> of;
+};
+
+bitnet_status_t seq_build(DsProgram &p, const bitnet_op_t *ops, int n, int64_t M, int C, int G, const SeqParts &parts,
                           const int32_t *wx, const int32_t *wy)
 {
     int ks_max = 1;
@@ -725,11 +732,14 @@ bitnet_status_t seq_build(DsProgram &p, const bitnet_op_t *ops, int n, int64_t M
         const bitnet_op_t &o = ops[i];
         DsOp &d = p.ops[i];
         d = DsOp{};
+        const int part = parts.of[i];
+        d.cl0 = parts.cl0[part];
+        d.ncl = parts.ncl[part];
         const int nmat = o.kind == BITNET_OP_FFN_GATE_UP ? 2 : 1;
         const int KS = (int)(o.K / 64);
         d.ks = (int)cdiv(KS, C);
         if (d.ks > DS_MAX_KS) return BITNET_ERR_UNSUPPORTED_SHAPE;
-        d.rpc = (int)align_up((size_t)cdiv(o.N, G), 16);
+        d.rpc = (int)align_up((size_t)cdiv(o.N, d.ncl), 16);
         const int64_t per_warp = cdiv((int64_t)nmat * (d.rpc / 16), 8);
         if (per_warp > DS_RGW) return BITNET_ERR_UNSUPPORTED_SHAPE;
         d.own_rows = d.rpc / C;
@@ -755,18 +765,43 @@ bitnet_status_t seq_build(DsProgram &p, const bitnet_op_t *ops, int n, int64_t M
     p.M = (int)M;
     p.C = C;
     p.n_ctas = G * C;
+    // partitions: each runs its ops in program order, linked through DsOp::nxt
+    p.n_parts = parts.n;
+    for (int q = 0; q < parts.n; ++q) {
+        p.part_cl0[q] = parts.cl0[q];
+        p.part_ncl[q] = parts.ncl[q];
+        p.part_first[q] = -1;
+    }
+    {
+        int last[DS_MAX_PARTS];
+        for (int q = 0; q < DS_MAX_PARTS; ++q) last[q] = -1;
+        for (int i = 0; i < n; ++i) {
+            const int q = parts.of[i];
+            p.ops[i].nxt = -1;
+            if (last[q] < 0)
+                p.part_first[q] = i;
+            else
+                p.ops[last[q]].nxt = i;
+            last[q] = i;
+            // every op an op waits for runs in its partition
+            if ((wx[i] >= 0 && parts.of[wx[i]] != q) || (wy[i] >= 0 && parts.of[wy[i]] != q))
+                return BITNET_ERR_INVALID_ARG;
+        }
+        for (int q = 0; q < parts.n; ++q)
+            if (p.part_first[q] < 0) return BITNET_ERR_INVALID_ARG;
+    }
     // x staging: ops whose x no op of the launch writes alternate between buffers 0 and 1 (the
     // next one is fetched while the current one runs); ops reading an earlier op's output use
     // buffer 2 (loaded when their wait is over).  Rows as long as the largest K slice in the buffer.
     uint32_t pitch[3] = {16, 16, 16};
-    int alt = 0;
+    int alt[DS_MAX_PARTS] = {0};
     for (int i = 0; i < n; ++i) {
         DsOp &d = p.ops[i];
         if (d.wait_x >= 0) {
             d.xbuf = 2;
         } else {
-            d.xbuf = alt;
-            alt ^= 1;
+            d.xbuf = alt[parts.of[i]];
+            alt[parts.of[i]] ^= 1;
         }
         pitch[d.xbuf] = std::max(pitch[d.xbuf], (uint32_t)(d.ks * 64 * (d.xf32 ? 4 : 2)));
     }
@@ -790,6 +825,60 @@ bitnet_status_t seq_build(DsProgram &p, const bitnet_op_t *ops, int n, int64_t M
     for (int i = 0; i < n; ++i)
         if (ds_slice_bytes(p.ops[i]) > p.ring_bytes) return BITNET_ERR_UNSUPPORTED_SHAPE;
     return BITNET_OK;
+}
+
+// Independent groups of ops run side by side: the connected components of the
+// hazard graph never wait for each other.  The component with the most weight
+// bytes gets most clusters; the rest share the others, sized by their weight
+// bytes, as long as every op's weight slice still fits a CTA's ring.  A single
+// partition (every cluster runs every op) when there is one component or no
+// split fits.
+bitnet_status_t seq_partitioned_build(DsProgram &p, const bitnet_op_t *ops, int n, int64_t M, int C, int G,
+                                      const int32_t *wx, const int32_t *wy)
+{
+    SeqParts one;
+    one.n = 1;
+    one.ncl[0] = G;
+    one.of.assign(n, 0);
+    if (G < 2) return seq_build(p, ops, n, M, C, G, one, wx, wy);
+    // components over the hazard waits (union-find)
+    std::vector<int> root(n);
+    for (int i = 0; i < n; ++i) root[i] = i;
+    auto find = [&](int i) {
+        while (root[i] != i) i = root[i] = root[root[i]];
+        return i;
+    };
+    std::vector<ByteRange> xr, yr;
+    if (seq_validate(ops, n, M, ByteRange{0, 0}, xr, yr) != BITNET_OK) return BITNET_ERR_INVALID_ARG;
+    for (int j = 0; j < n; ++j)
+        for (int i = 0; i < j; ++i)
+            if (hazard(xr, yr, i, j)) root[find(i)] = find(j);
+    std::vector<double> bytes(n, 0.0);
+    double total = 0.0;
+    for (int i = 0; i < n; ++i) {
+        const double b = (ops[i].kind == BITNET_OP_FFN_GATE_UP ? 2.0 : 1.0) * (double)ops[i].N * (double)(ops[i].K / 4);
+        bytes[find(i)] += b;
+        total += b;
+    }
+    int main_root = find(0);
+    for (int i = 0; i < n; ++i)
+        if (bytes[find(i)] > bytes[main_root]) main_root = find(i);
+    const double side = total - bytes[main_root];
+    if (side <= 0.0) return seq_build(p, ops, n, M, C, G, one, wx, wy);
+    SeqParts two;
+    two.n = 2;
+    two.of.resize(n);
+    for (int i = 0; i < n; ++i) two.of[i] = find(i) == main_root ? 1 : 0;
+    const int target = std::min(G - 1, std::max(1, (int)(G * side / total + 0.5)));
+    for (int pass = 0; pass < 2; ++pass)
+        for (int s = pass == 0 ? target : target - 1; pass == 0 ? s < G : s >= 1; s += pass == 0 ? 1 : -1) {
+            two.cl0[0] = 0;
+            two.ncl[0] = s;
+            two.cl0[1] = s;
+            two.ncl[1] = G - s;
+            if (seq_build(p, ops, n, M, C, G, two, wx, wy) == BITNET_OK) return BITNET_OK;
+        }
+    return seq_build(p, ops, n, M, C, G, one, wx, wy);
 }
 
 constexpr size_t kSeqWorkspaceBytes = 1024;
@@ -817,7 +906,7 @@ bitnet_status_t decode_sequence(const bitnet_op_t *ops, int n, int64_t M, void *
     if (G < 1) return BITNET_ERR_CUDA;
     static DsProgram prog_proto; // zero-initialised template; each call fills a copy
     DsProgram p = prog_proto;
-    st = seq_build(p, ops, n, M, C, G, wx, wy);
+    st = seq_partitioned_build(p, ops, n, M, C, G, wx, wy);
     if (st != BITNET_OK) return st;
     p.counters = static_cast<unsigned *>(workspace);
     cudaLaunchConfig_t cfg = {};

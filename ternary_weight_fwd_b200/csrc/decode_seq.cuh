@@ -45,8 +45,9 @@ constexpr int DS_COMPUTE = 256;   // eight compute warps
 constexpr int DS_CONTROL = 128;   // control warps: weight copies and completion signals
 constexpr int DS_THREADS = DS_COMPUTE + DS_CONTROL;
 constexpr int DS_SLOTS = 8;       // weight-ring slots (ops in flight)
-constexpr int DS_HDR = 1024 + 8 * 96; // header: barriers, per-token scalars, staged op descriptors
-constexpr int DS_MAX_KS = 32;     // 64-wide k-steps per CTA (x slice kept in registers)
+constexpr int DS_HDR = 1024 + 8 * 112; // header: barriers, per-token scalars, staged op descriptors
+constexpr int DS_MAX_KS = 32;     // 64-wide k-steps per CTA
+constexpr int DS_MAX_PARTS = 4;   // partitions: independent groups of ops on disjoint clusters
 constexpr int DS_RGW = 8;         // row groups (of 16 output rows) per compute warp (host limit)
 
 struct __align__(16) DsOp {
@@ -66,10 +67,14 @@ struct __align__(16) DsOp {
     int wait_y;                  // earlier op that must be complete before y is written (-1: none)
     int xbuf;                    // x staging buffer: 0/1 alternate among ops whose x can be
                                  // prefetched, 2 for ops that read an earlier op's output
+    int cl0, ncl;                // clusters running this op: [cl0, cl0 + ncl) (its partition)
+    int nxt;                     // next op of the same partition (-1: last)
 };
 
 struct DsProgram {
     int n_ops, M, C, n_ctas;
+    int n_parts;
+    int part_cl0[DS_MAX_PARTS], part_ncl[DS_MAX_PARTS], part_first[DS_MAX_PARTS];
     unsigned *counters;          // [DS_MAX_OPS] completions, then [1] exits (workspace)
     uint32_t xs_off[3];          // x staging buffers (DsOp::xbuf): 8 token rows each
     uint32_t xs_pitch[3];        // bytes per token row (the largest K slice of the ops using the buffer)
@@ -93,22 +98,22 @@ constexpr int DS_RELEASED = 704;                   // uint32: ops whose weight s
 constexpr int DS_DONE = 708;                       // uint32: ops complete on this CTA
 constexpr int DS_DESC_READY = 712;                 // uint32: op descriptors staged in shared memory
 constexpr int DS_Y_CLEAR = 716;                    // uint32: ops whose y-region ordering wait is satisfied
-constexpr int DS_DESC = 1024;                      // DsOp [DS_DESC_SLOTS]: op j in slot j % DS_DESC_SLOTS
+constexpr int DS_DESC = 1024;                      // DsOp [DS_DESC_SLOTS]: this CTA's k-th op in slot k % DS_DESC_SLOTS
 constexpr int DS_DESC_SLOTS = 8;
 
-static_assert(sizeof(DsOp) == 96 && DS_DESC + DS_DESC_SLOTS * 96 <= DS_HDR, "staged op descriptors");
+static_assert(sizeof(DsOp) == 112 && DS_DESC + DS_DESC_SLOTS * 112 <= DS_HDR, "staged op descriptors");
 
-// Op j's descriptor staged in shared memory (slot j % DS_DESC_SLOTS).
-BITNET_DEVINL const DsOp &ds_desc(unsigned char *smem, int j)
+// Descriptor of this CTA's k-th op, staged in shared memory (slot k % DS_DESC_SLOTS).
+BITNET_DEVINL const DsOp &ds_desc(unsigned char *smem, int k)
 {
-    return *reinterpret_cast<const DsOp *>(smem + DS_DESC + (j % DS_DESC_SLOTS) * (int)sizeof(DsOp));
+    return *reinterpret_cast<const DsOp *>(smem + DS_DESC + (k % DS_DESC_SLOTS) * (int)sizeof(DsOp));
 }
 
-// Copy op j's descriptor into its shared-memory slot (one thread).
-BITNET_DEVINL void ds_stage_desc(const DsProgram &p, unsigned char *smem, int j)
+// Stage op j (program index) as this CTA's k-th op (one thread).
+BITNET_DEVINL void ds_stage_desc(const DsProgram &p, unsigned char *smem, int j, int k)
 {
     const uint4 *src = reinterpret_cast<const uint4 *>(&p.ops[j]);
-    uint4 *dst = reinterpret_cast<uint4 *>(smem + DS_DESC + (j % DS_DESC_SLOTS) * (int)sizeof(DsOp));
+    uint4 *dst = reinterpret_cast<uint4 *>(smem + DS_DESC + (k % DS_DESC_SLOTS) * (int)sizeof(DsOp));
 #pragma unroll
     for (int i = 0; i < (int)(sizeof(DsOp) / 16); ++i) dst[i] = src[i];
 }
@@ -256,7 +261,8 @@ BITNET_DEVINL bool wait_count(const unsigned *c, unsigned target)
 // Called before the first op and again each time an op has released its slice.
 struct DsIssue {
     uint32_t head;  // virtual ring position after the last issued slice
-    int issued;     // ops whose copies have been started
+    int issued;     // this CTA's ops whose copies have been started
+    int next;       // program index of the next op to issue (-1: none)
 };
 
 __device__ __forceinline__ void ds_issue(const DsProgram &p, unsigned char *smem, DsIssue &st, int released)
@@ -267,9 +273,9 @@ __device__ __forceinline__ void ds_issue(const DsProgram &p, unsigned char *smem
     const int C = p.C;
     const int r = (int)cluster_ctarank();
     const int cl = blockIdx.x / C;
-    while (st.issued < p.n_ops && st.issued - released < DS_SLOTS) {
-        const int j = st.issued;
-        const DsOp &op = p.ops[j];
+    while (st.next >= 0 && st.issued - released < DS_SLOTS) {
+        const int j = st.issued; // this CTA's ordinal of the op
+        const DsOp &op = p.ops[st.next];
         const uint32_t size = ds_slice_bytes(op);
         const uint32_t start = ring_place(st.head, size, p.ring_bytes);
         // starts[] is written by every control thread with the same value; each reads back its own
@@ -280,7 +286,8 @@ __device__ __forceinline__ void ds_issue(const DsProgram &p, unsigned char *smem
         starts[j % DS_SLOTS] = start;
         st.head = start + size;
         ++st.issued;
-        const int64_t n0 = (int64_t)cl * op.rpc;
+        st.next = op.nxt;
+        const int64_t n0 = (int64_t)(cl - op.cl0) * op.rpc;
         const int64_t rows_left = (int64_t)op.N - n0;
         const int R = rows_left <= 0 ? 0 : (int)(rows_left < op.rpc ? rows_left : op.rpc);
         const int KS = op.K / 64;
@@ -330,7 +337,6 @@ BITNET_DEVINL void ds_signal(const DsProgram &p, int j)
 struct DsState {
     int tile;        // token tiles done in this launch (exchange barriers and parity)
     uint32_t xw;     // completed waits on x staging buffer b (0..2) in bit b (its next parity)
-    bool x_ready;    // this op's first x tile was prefetched into its buffer
     bool ok;
 };
 
@@ -359,8 +365,12 @@ BITNET_DEVINL void ds_load_x(const DsProgram &p, const DsOp &op, unsigned char *
 // `last_op` makes the final tile arrive on the exit phase of the cluster
 // barrier.  The control warp is told when the op's weight slice is free and
 // when the op is complete (it publishes the completion).
-__device__ __forceinline__ void ds_op(const DsProgram &p, const DsOp &op, int j, uint32_t wbase, unsigned char *smem,
-                                      DsState &st, bool last_op)
+//
+// j: the op's program index (completion counters); k: its ordinal among this
+// CTA's ops (ring slot, hand-off counters, staged descriptors); prev: program
+// index of this CTA's previous op (-1: none).
+__device__ __forceinline__ void ds_op(const DsProgram &p, const DsOp &op, int j, int k, int prev, uint32_t wbase,
+                                      unsigned char *smem, DsState &st, bool last_op)
 {
     uint64_t *bar_full = reinterpret_cast<uint64_t *>(smem + DS_BAR_FULL);
     uint64_t *bar_amax = reinterpret_cast<uint64_t *>(smem + DS_BAR_AMAX);
@@ -382,7 +392,7 @@ __device__ __forceinline__ void ds_op(const DsProgram &p, const DsOp &op, int j,
     const int cl = blockIdx.x / C;
     const int nmat = op.nmat;
     const bool xf32 = op.xf32 != 0;
-    const int64_t n0 = (int64_t)cl * op.rpc;
+    const int64_t n0 = (int64_t)(cl - op.cl0) * op.rpc;
     const int64_t rows_left = (int64_t)op.N - n0;
     const int R = rows_left <= 0 ? 0 : (int)(rows_left < op.rpc ? rows_left : op.rpc);
     const int KS = op.K / 64;
@@ -398,11 +408,11 @@ __device__ __forceinline__ void ds_op(const DsProgram &p, const DsOp &op, int j,
     const int orp = op.orp;
     const int blk_ints = nmat * 8 * orp;
     const uint32_t blk_bytes = (uint32_t)blk_ints * 4;
-    const int slot = j % DS_SLOTS;
+    const int slot = k % DS_SLOTS;
     const int xb = op.xbuf; // this op's x staging buffer
     const unsigned char *sXs = smem + p.xs_off[xb];
     const uint32_t xs_pitch = p.xs_pitch[xb];
-    const unsigned target = (unsigned)p.n_ctas;
+    const unsigned target = (unsigned)(op.ncl * C); // CTAs of this partition (every op it waits for is in it)
 
     const float gam0 = op.gamma0[0];
     const float gam1 = nmat == 2 ? op.gamma1[0] : 0.0f;
@@ -415,10 +425,12 @@ __device__ __forceinline__ void ds_op(const DsProgram &p, const DsOp &op, int j,
             mbar_arrive_expect_tx(&bar_amax[pp], (uint32_t)(C - 1) * 32);
             mbar_arrive_expect_tx(&bar_red[pp], (uint32_t)(C - 1) * blk_bytes);
         }
-        if (warp == 0 && (m0 > 0 || !st.x_ready)) {
+        // the first tile of an op that reads nothing this launch writes was fetched
+        // during this CTA's previous op
+        if (warp == 0 && (m0 > 0 || k == 0 || op.wait_x >= 0)) {
             if (m0 == 0 && op.wait_x >= 0) { // x is written by an earlier op of this launch
                 if (lane == 0) {
-                    if (op.wait_x == j - 1) ds_signal(p, j - 1); // the previous op: publish it right here
+                    if (prev >= 0 && op.wait_x == prev) ds_signal(p, prev); // the previous op: publish it right here
                     st.ok = wait_count(&p.counters[op.wait_x], target) && st.ok;
                 }
                 __syncwarp();
@@ -426,9 +438,10 @@ __device__ __forceinline__ void ds_op(const DsProgram &p, const DsOp &op, int j,
             }
             ds_load_x(p, op, smem, xb, m0, mt, ks0, ksn, lane);
         }
-        if (warp == 7 && m0 == 0 && j + 1 < p.n_ops) {
+        if (warp == 7 && m0 == 0 && op.nxt >= 0) {
             // the next op's first tile reads memory no op of this launch writes: fetch it now
-            const DsOp &nx = ds_desc(smem, j + 1);
+            wait_local(reinterpret_cast<const uint32_t *>(smem + DS_DESC_READY), (uint32_t)k + 2);
+            const DsOp &nx = ds_desc(smem, k + 1);
             if (nx.wait_x < 0) { // its buffer (0/1) is not this op's and no earlier op still uses it
                 const int nks0 = (int)r * nx.ks;
                 ds_load_x(p, nx, smem, nx.xbuf, 0, min(8, p.M), nks0, max(0, min(nx.ks, nx.K / 64 - nks0)), lane);
@@ -493,7 +506,7 @@ __device__ __forceinline__ void ds_op(const DsProgram &p, const DsOp &op, int j,
             if (mat < nmat) tok_r[tid] = __fdiv_rn(mat ? gam1 : gam0, tok_s[jj]);
         }
         compute_sync();
-        if (m0 == 0) st.ok = mbar_spin(&bar_full[slot], (uint32_t)(j / DS_SLOTS) & 1u) && st.ok;
+        if (m0 == 0) st.ok = mbar_spin(&bar_full[slot], (uint32_t)(k / DS_SLOTS) & 1u) && st.ok;
 
         // ---- contraction, two row groups at a time; partial sums (code offset
         //      removed) into per-owner blocks ----
@@ -572,14 +585,14 @@ __device__ __forceinline__ void ds_op(const DsProgram &p, const DsOp &op, int j,
         }
         // the slice is free (every compute warp passed the barrier after the
         // contraction): the control warp refills the ring meanwhile
-        if (m0 + 8 >= p.M && tid == 0) st_release_cta(reinterpret_cast<uint32_t *>(smem + DS_RELEASED), (uint32_t)j + 1);
+        if (m0 + 8 >= p.M && tid == 0) st_release_cta(reinterpret_cast<uint32_t *>(smem + DS_RELEASED), (uint32_t)k + 1);
         st.ok = mbar_spin(&bar_red[pp], ph, true) && st.ok;
         if (last_op && m0 + 8 >= p.M) cluster_arrive(); // nothing more is needed from the peers
         if (m0 == 0 && op.wait_y >= 0) { // y was read or written by an earlier op of this launch
             // the control warp acquired that op's completion counter (device scope)
             // and passed it on through this CTA's y-clear counter
             if (tid == 0)
-                st.ok = wait_local(reinterpret_cast<const uint32_t *>(smem + DS_Y_CLEAR), (uint32_t)j + 1) && st.ok;
+                st.ok = wait_local(reinterpret_cast<const uint32_t *>(smem + DS_Y_CLEAR), (uint32_t)k + 1) && st.ok;
             compute_sync();
         }
 
@@ -605,9 +618,7 @@ __device__ __forceinline__ void ds_op(const DsProgram &p, const DsOp &op, int j,
         compute_sync();
     }
     // every store of this op precedes the control warp's completion signal
-    if (tid == 0) st_release_cta(reinterpret_cast<uint32_t *>(smem + DS_DONE), (uint32_t)j + 1);
-    // the next op's first tile was fetched above when it reads nothing this launch writes
-    st.x_ready = j + 1 < p.n_ops && p.ops[j + 1].wait_x < 0;
+    if (tid == 0) st_release_cta(reinterpret_cast<uint32_t *>(smem + DS_DONE), (uint32_t)k + 1);
 }
 
 __global__ void __launch_bounds__(DS_THREADS, 1) k_decode_seq(const __grid_constant__ DsProgram p)
@@ -633,43 +644,62 @@ __global__ void __launch_bounds__(DS_THREADS, 1) k_decode_seq(const __grid_const
     __syncthreads();
     cluster_arrive(); // peers may send to this CTA once every CTA of the cluster has arrived here
 
+    // this CTA's partition: the ops it runs, in program order, linked by DsOp::nxt
+    const int cl = (int)blockIdx.x / p.C;
+    int part = 0;
+    for (int q = 1; q < p.n_parts; ++q)
+        if (cl >= p.part_cl0[q]) part = q;
+    const int first = p.part_first[part];
+
     if (tid >= DS_COMPUTE) {
-        // control warp: keep the weight ring full, publish each op's completion
-        DsIssue iss = {0u, 0};
+        // control warps: keep the weight ring full, publish each op's completion
+        DsIssue iss = {0u, 0, first};
         ds_issue(p, smem, iss, 0);
         const uint32_t *released = reinterpret_cast<const uint32_t *>(smem + DS_RELEASED);
         const uint32_t *done = reinterpret_cast<const uint32_t *>(smem + DS_DONE);
         uint32_t *desc_ready = reinterpret_cast<uint32_t *>(smem + DS_DESC_READY);
         uint32_t *y_clear = reinterpret_cast<uint32_t *>(smem + DS_Y_CLEAR);
-        // y-region waits are acquired here, ahead of the compute warps' epilogues: op 0's now,
-        // op j + 1's once op j is done (ops run in order, so op j + 1's epilogue comes later)
-        auto clear_y = [&](int k) {
-            const int w = p.ops[k].wait_y;
-            if (w >= 0) wait_count(&p.counters[w], (unsigned)p.n_ctas);
+        // y-region waits are acquired here, ahead of the compute warps' epilogues: the first
+        // op's now, the next op's once the current one is done (it runs later)
+        auto clear_y = [&](int j, int k) {
+            const int w = p.ops[j].wait_y;
+            if (w >= 0) wait_count(&p.counters[w], (unsigned)(p.ops[j].ncl * p.C));
             st_release_cta(y_clear, (uint32_t)k + 1);
         };
         // the first op descriptors, staged in shared memory (one op per thread)
         const int ctid = tid - DS_COMPUTE;
-        if (ctid < DS_DESC_SLOTS && ctid < p.n_ops) ds_stage_desc(p, smem, ctid);
+        int staged = 0, stage_next = first; // ops staged so far; program index of the next one
+        {
+            int j = first;
+            for (int q = 0; q < ctid && j >= 0 && q < DS_DESC_SLOTS; ++q) j = p.ops[j].nxt;
+            if (ctid < DS_DESC_SLOTS && j >= 0) ds_stage_desc(p, smem, j, ctid);
+            while (staged < DS_DESC_SLOTS && stage_next >= 0) {
+                stage_next = p.ops[stage_next].nxt;
+                ++staged;
+            }
+        }
         control_sync();
         if (ctid == 0) {
-            st_release_cta(desc_ready, (uint32_t)min(p.n_ops, DS_DESC_SLOTS));
-            clear_y(0);
+            st_release_cta(desc_ready, (uint32_t)staged);
+            clear_y(first, 0);
         }
-        for (int j = 0; j < p.n_ops; ++j) {
-            wait_local(released, (uint32_t)j + 1);
+        int k = 0;
+        for (int j = first; j >= 0; j = p.ops[j].nxt, ++k) {
+            wait_local(released, (uint32_t)k + 1);
             control_sync();
-            ds_issue(p, smem, iss, j + 1);
+            ds_issue(p, smem, iss, k + 1);
             if (ctid == 0) {
-                wait_local(done, (uint32_t)j + 1);
-                // an op the very next op reads is published by compute thread 0 itself
-                if (!(j + 1 < p.n_ops && p.ops[j + 1].wait_x == j)) ds_signal(p, j);
-                // op j no longer needs its descriptor slot: stage op j + DS_DESC_SLOTS there
-                if (j + DS_DESC_SLOTS < p.n_ops) {
-                    ds_stage_desc(p, smem, j + DS_DESC_SLOTS);
-                    st_release_cta(desc_ready, (uint32_t)(j + DS_DESC_SLOTS + 1));
+                wait_local(done, (uint32_t)k + 1);
+                // an op the very next op of this CTA reads is published by compute thread 0 itself
+                const int nx = p.ops[j].nxt;
+                if (!(nx >= 0 && p.ops[nx].wait_x == j)) ds_signal(p, j);
+                // op k no longer needs its descriptor slot: stage the next unstaged op there
+                if (stage_next >= 0) {
+                    ds_stage_desc(p, smem, stage_next, staged);
+                    st_release_cta(desc_ready, (uint32_t)++staged);
+                    stage_next = p.ops[stage_next].nxt;
                 }
-                if (j + 1 < p.n_ops) clear_y(j + 1);
+                if (nx >= 0) clear_y(nx, k + 1);
             }
         }
         asm volatile("cp.async.wait_all;" ::: "memory"); // every weight copy has landed
@@ -677,17 +707,20 @@ __global__ void __launch_bounds__(DS_THREADS, 1) k_decode_seq(const __grid_const
         cluster_arrive();
     } else {
         uint32_t head = 0;
-        DsState st = {0, 0u, false, true};
+        DsState st = {0, 0u, true};
         const uint32_t *desc_ready = reinterpret_cast<const uint32_t *>(smem + DS_DESC_READY);
-        for (int j = 0; j < p.n_ops; ++j) {
-            // this op's descriptor (and, for warp 7's prefetch, the next one) is staged
-            st.ok = wait_local(desc_ready, (uint32_t)min(j + 2, p.n_ops)) && st.ok;
-            const DsOp &op = ds_desc(smem, j);
+        int prev = -1, k = 0;
+        for (int j = first; j >= 0; ++k) {
+            st.ok = wait_local(desc_ready, (uint32_t)k + 1) && st.ok;
+            const DsOp &op = ds_desc(smem, k);
+            const int nxt = op.nxt; // read before the slot can be restaged (after this op)
             const uint32_t size = ds_slice_bytes(op);
             const uint32_t start = ring_place(head, size, p.ring_bytes);
             head = start + size;
             const uint32_t wbase = p.ring_off + start % p.ring_bytes;
-            ds_op(p, op, j, wbase, smem, st, j + 1 == p.n_ops);
+            ds_op(p, op, j, k, prev, wbase, smem, st, nxt < 0);
+            prev = j;
+            j = nxt;
         }
         // every x copy has landed before the CTA may exit (already true unless a
         // wait gave up): the last phase waited on each staging buffer is drained
