@@ -823,14 +823,14 @@ bitnet_status_t seq_build(DsProgram &p, const bitnet_op_t *ops, int n, int64_t M
     if (p.ring_off + 4096 > usable) return BITNET_ERR_UNSUPPORTED_SHAPE;
     p.ring_bytes = (uint32_t)((usable - p.ring_off) & ~size_t(127));
     for (int i = 0; i < n; ++i)
-        if (ds_slice_bytes(p.ops[i]) > p.ring_bytes) return BITNET_ERR_UNSUPPORTED_SHAPE;
+        if ((size_t)ds_piece_bytes(p.ops[i]) * p.ops[i].nmat > p.ring_bytes) return BITNET_ERR_UNSUPPORTED_SHAPE;
     return BITNET_OK;
 }
 
 // Independent groups of ops run side by side: the connected components of the
 // hazard graph never wait for each other.  The component with the most weight
 // bytes gets most clusters; the rest share the others, sized by their weight
-// bytes, as long as every op's weight slice still fits a CTA's ring.  A single
+// bytes, as long as every weight piece still fits a CTA's ring.  A single
 // partition (every cluster runs every op) when there is one component or no
 // split fits.
 bitnet_status_t seq_partitioned_build(DsProgram &p, const bitnet_op_t *ops, int n, int64_t M, int C, int G,
@@ -869,7 +869,9 @@ bitnet_status_t seq_partitioned_build(DsProgram &p, const bitnet_op_t *ops, int 
     two.n = 2;
     two.of.resize(n);
     for (int i = 0; i < n; ++i) two.of[i] = find(i) == main_root ? 1 : 0;
-    const int target = std::min(G - 1, std::max(1, (int)(G * side / total + 0.5)));
+    // the side's share of clusters rounded down: the main component is one long dependency
+    // chain, so its per-op latency (fewer rows per CTA) sets the launch time
+    const int target = std::min(G - 1, std::max(1, (int)(G * side / total)));
     for (int pass = 0; pass < 2; ++pass)
         for (int s = pass == 0 ? target : target - 1; pass == 0 ? s < G : s >= 1; s += pass == 0 ? 1 : -1) {
             two.cl0[0] = 0;

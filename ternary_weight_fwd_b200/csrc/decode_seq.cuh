@@ -44,7 +44,8 @@ constexpr int DS_MAX_OPS = 128;   // ops per launch (kernel-parameter space)
 constexpr int DS_COMPUTE = 256;   // eight compute warps
 constexpr int DS_CONTROL = 128;   // control warps: weight copies and completion signals
 constexpr int DS_THREADS = DS_COMPUTE + DS_CONTROL;
-constexpr int DS_SLOTS = 8;       // weight-ring slots (ops in flight)
+constexpr int DS_SLOTS = 8;       // ops whose weights may be in the ring at once
+constexpr int DS_PSLOTS = 16;     // weight pieces in the ring at once (one per matrix of an op)
 constexpr int DS_HDR = 1024 + 8 * 112; // header: barriers, per-token scalars, staged op descriptors
 constexpr int DS_MAX_KS = 32;     // 64-wide k-steps per CTA
 constexpr int DS_MAX_PARTS = 4;   // partitions: independent groups of ops on disjoint clusters
@@ -85,19 +86,20 @@ struct DsProgram {
 };
 
 // Header offsets.
-constexpr int DS_BAR_FULL = 0;                     // [DS_SLOTS] weights landed (one cp.async arrival per control thread)
-constexpr int DS_BAR_AMAX = DS_BAR_FULL + 8 * DS_SLOTS; // [2]
+constexpr int DS_BAR_FULL = 0;                     // [DS_PSLOTS] weight piece landed (one cp.async arrival per control thread)
+constexpr int DS_BAR_AMAX = DS_BAR_FULL + 8 * DS_PSLOTS; // [2]
 constexpr int DS_BAR_RED = DS_BAR_AMAX + 16;       // [2]
 constexpr int DS_BAR_X = DS_BAR_RED + 16;          // [3] x staging buffer landed (expect_tx + bulk bytes)
 constexpr int DS_TOK_S = 256;                      // float [8]
 constexpr int DS_TOK_RS = 288;                     // int [8]
 constexpr int DS_TOK_R = 320;                      // float [16]
 constexpr int DS_AMAX = 384;                       // float [8 ranks][8 tokens]
-constexpr int DS_STARTS = 640;                     // uint32 [DS_SLOTS] ring starts of live slices
+constexpr int DS_STARTS = 640;                     // uint32 [DS_PSLOTS] ring starts of live pieces
 constexpr int DS_RELEASED = 704;                   // uint32: ops whose weight slice is free
 constexpr int DS_DONE = 708;                       // uint32: ops complete on this CTA
 constexpr int DS_DESC_READY = 712;                 // uint32: op descriptors staged in shared memory
 constexpr int DS_Y_CLEAR = 716;                    // uint32: ops whose y-region ordering wait is satisfied
+constexpr int DS_OP_P0 = 720;                      // uint32 [DS_SLOTS]: first piece of each op in the ring
 constexpr int DS_DESC = 1024;                      // DsOp [DS_DESC_SLOTS]: this CTA's k-th op in slot k % DS_DESC_SLOTS
 constexpr int DS_DESC_SLOTS = 8;
 
@@ -127,7 +129,8 @@ BITNET_DEVINL uint32_t ring_place(uint32_t head, uint32_t size, uint32_t ring)
     return off + size > ring ? head - off + ring : head;
 }
 
-__host__ __device__ __forceinline__ uint32_t ds_slice_bytes(const DsOp &op) { return (uint32_t)(op.nmat * op.rpc * op.box_w); }
+// Ring bytes of one weight piece: this cluster's rows of one matrix x this CTA's K slice.
+__host__ __device__ __forceinline__ uint32_t ds_piece_bytes(const DsOp &op) { return (uint32_t)(op.rpc * op.box_w); }
 
 // Barriers among the compute warps and among the control warps.
 BITNET_DEVINL void compute_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
@@ -260,67 +263,73 @@ BITNET_DEVINL bool wait_count(const unsigned *c, unsigned target)
 // phase).
 // Called before the first op and again each time an op has released its slice.
 struct DsIssue {
-    uint32_t head;  // virtual ring position after the last issued slice
-    int issued;     // this CTA's ops whose copies have been started
-    int next;       // program index of the next op to issue (-1: none)
+    uint32_t head;  // virtual ring position after the last issued piece
+    int issued;     // this CTA's ops whose pieces have all been started
+    int next;       // program index of the op being issued (-1: none)
+    int pieces;     // pieces started so far
+    int mat;        // next matrix of the op being issued
 };
 
 __device__ __forceinline__ void ds_issue(const DsProgram &p, unsigned char *smem, DsIssue &st, int released)
 {
     uint64_t *bar_full = reinterpret_cast<uint64_t *>(smem + DS_BAR_FULL);
     uint32_t *starts = reinterpret_cast<uint32_t *>(smem + DS_STARTS);
+    uint32_t *op_p0 = reinterpret_cast<uint32_t *>(smem + DS_OP_P0);
     const int tid = threadIdx.x - DS_COMPUTE;
     const int C = p.C;
     const int r = (int)cluster_ctarank();
     const int cl = blockIdx.x / C;
+    // starts[] and op_p0[] are written by every control thread with the same values;
+    // each reads back its own
     while (st.next >= 0 && st.issued - released < DS_SLOTS) {
-        const int j = st.issued; // this CTA's ordinal of the op
+        const int k = st.issued; // this CTA's ordinal of the op
         const DsOp &op = p.ops[st.next];
-        const uint32_t size = ds_slice_bytes(op);
-        const uint32_t start = ring_place(st.head, size, p.ring_bytes);
-        // starts[] is written by every control thread with the same value; each reads back its own
-        if (released < j && start + size - starts[released % DS_SLOTS] > p.ring_bytes) break; // no room yet
+        const int q = st.pieces;
+        if (st.mat == 0) op_p0[k % DS_SLOTS] = (uint32_t)q;
+        const uint32_t size = ds_piece_bytes(op);
+        // an op's pieces are placed back to back (no wrap between them, and the host keeps
+        // a whole op within the ring): the up piece always fits once older ops are released
+        const uint32_t start = st.mat == 1 ? st.head : ring_place(st.head, size * op.nmat, p.ring_bytes);
+        // oldest piece still in use: the first piece of op `released`, if that op has begun
+        const int live0 = released < k ? (int)op_p0[released % DS_SLOTS] : (st.mat > 0 ? (int)op_p0[k % DS_SLOTS] : q);
+        if (live0 < q && start + size - starts[live0 % DS_PSLOTS] > p.ring_bytes) break; // no room yet
         // the slot's previous copies have landed (already true unless a consumer gave up
         // waiting for them): no copy is ever in flight into reused memory
-        if (j >= DS_SLOTS) mbar_wait_drain(&bar_full[j % DS_SLOTS], (uint32_t)((j - DS_SLOTS) / DS_SLOTS) & 1u);
-        starts[j % DS_SLOTS] = start;
+        if (q >= DS_PSLOTS) mbar_wait_drain(&bar_full[q % DS_PSLOTS], (uint32_t)((q - DS_PSLOTS) / DS_PSLOTS) & 1u);
+        starts[q % DS_PSLOTS] = start;
         st.head = start + size;
-        ++st.issued;
-        st.next = op.nxt;
+        ++st.pieces;
+        const int mat = st.mat;
+        if (++st.mat == op.nmat) {
+            st.mat = 0;
+            ++st.issued;
+            st.next = op.nxt;
+        }
         const int64_t n0 = (int64_t)(cl - op.cl0) * op.rpc;
         const int64_t rows_left = (int64_t)op.N - n0;
         const int R = rows_left <= 0 ? 0 : (int)(rows_left < op.rpc ? rows_left : op.rpc);
         const int KS = op.K / 64;
         const int ks0 = r * op.ks;
         const int ksn = max(0, min(op.ks, KS - ks0));
-        const int total = op.nmat * R * ksn;
+        const int total = R * ksn;
         if (total > 0 && !status_failed()) {
             unsigned char *dst0 = smem + p.ring_off + start % p.ring_bytes;
-            const uint32_t w_mat_bytes = (uint32_t)(op.rpc * op.box_w);
+            const uint8_t *w = (mat ? op.w1 : op.w0) + (size_t)n0 * (op.K / 4) + (size_t)ks0 * 16;
             const size_t row_bytes = (size_t)op.K / 4;
-            // (mat, row, chunk) of chunk index c = tid + DS_CONTROL i, advanced incrementally
+            // (row, chunk) of chunk index c = tid + DS_CONTROL i, advanced incrementally
             const int dq = DS_CONTROL / ksn, dr = DS_CONTROL % ksn;
-            int kc = tid % ksn, row = tid / ksn, mat = 0;
-            while (row >= R && mat < op.nmat) {
-                row -= R;
-                ++mat;
-            }
+            int kc = tid % ksn, row = tid / ksn;
             for (int c = tid; c < total; c += DS_CONTROL) {
-                const uint8_t *src = (mat ? op.w1 : op.w0) + (size_t)(n0 + row) * row_bytes + (size_t)(ks0 + kc) * 16;
-                cp_async16(dst0 + mat * w_mat_bytes + (uint32_t)row * op.box_w + kc * 16, src);
+                cp_async16(dst0 + (uint32_t)row * op.box_w + kc * 16, w + (size_t)row * row_bytes + (size_t)kc * 16);
                 kc += dr;
                 row += dq;
                 if (kc >= ksn) {
                     kc -= ksn;
                     ++row;
                 }
-                while (row >= R && mat < op.nmat) {
-                    row -= R;
-                    ++mat;
-                }
             }
         }
-        cp_async_mbar_arrive(&bar_full[j % DS_SLOTS]);
+        cp_async_mbar_arrive(&bar_full[q % DS_PSLOTS]);
     }
 }
 
@@ -369,8 +378,10 @@ BITNET_DEVINL void ds_load_x(const DsProgram &p, const DsOp &op, unsigned char *
 // j: the op's program index (completion counters); k: its ordinal among this
 // CTA's ops (ring slot, hand-off counters, staged descriptors); prev: program
 // index of this CTA's previous op (-1: none).
-__device__ __forceinline__ void ds_op(const DsProgram &p, const DsOp &op, int j, int k, int prev, uint32_t wbase,
-                                      unsigned char *smem, DsState &st, bool last_op)
+// q0: ring piece of the op's first matrix (the second, for the gated FFN, is
+// q0 + 1); wb0 / wb1: shared-memory offsets of the two pieces.
+__device__ __forceinline__ void ds_op(const DsProgram &p, const DsOp &op, int j, int k, int prev, int q0,
+                                      uint32_t wb0, uint32_t wb1, unsigned char *smem, DsState &st, bool last_op)
 {
     uint64_t *bar_full = reinterpret_cast<uint64_t *>(smem + DS_BAR_FULL);
     uint64_t *bar_amax = reinterpret_cast<uint64_t *>(smem + DS_BAR_AMAX);
@@ -380,7 +391,6 @@ __device__ __forceinline__ void ds_op(const DsProgram &p, const DsOp &op, int j,
     int *tok_rs = reinterpret_cast<int *>(smem + DS_TOK_RS);
     float *tok_r = reinterpret_cast<float *>(smem + DS_TOK_R);
     float *amax_slot = reinterpret_cast<float *>(smem + DS_AMAX);
-    unsigned char *sW = smem + wbase;
     unsigned char *sXq = smem + p.xq_off;
     int *part = reinterpret_cast<int *>(smem + p.part_off);
     int *recv = reinterpret_cast<int *>(smem + p.recv_off);
@@ -403,12 +413,11 @@ __device__ __forceinline__ void ds_op(const DsProgram &p, const DsOp &op, int j,
     const int RG = op.rpc / 16;
     const int nrgi = nmat * RG; // row groups of the cluster: rgi = warp + 8 i (matrix rgi / RG)
     const uint32_t box_w = (uint32_t)op.box_w;
-    const uint32_t w_mat_bytes = (uint32_t)op.rpc * box_w;
     const int nchunk = ksn * 4 * (xf32 ? 4 : 2); // 16-byte x chunks per token in this slice
     const int orp = op.orp;
     const int blk_ints = nmat * 8 * orp;
     const uint32_t blk_bytes = (uint32_t)blk_ints * 4;
-    const int slot = k % DS_SLOTS;
+    bool up_ready = nmat == 1; // the up projection's piece has landed (gated FFN only)
     const int xb = op.xbuf; // this op's x staging buffer
     const unsigned char *sXs = smem + p.xs_off[xb];
     const uint32_t xs_pitch = p.xs_pitch[xb];
@@ -506,7 +515,7 @@ __device__ __forceinline__ void ds_op(const DsProgram &p, const DsOp &op, int j,
             if (mat < nmat) tok_r[tid] = __fdiv_rn(mat ? gam1 : gam0, tok_s[jj]);
         }
         compute_sync();
-        if (m0 == 0) st.ok = mbar_spin(&bar_full[slot], (uint32_t)(k / DS_SLOTS) & 1u) && st.ok;
+        if (m0 == 0) st.ok = mbar_spin(&bar_full[q0 % DS_PSLOTS], (uint32_t)(q0 / DS_PSLOTS) & 1u) && st.ok;
 
         // ---- contraction, two row groups at a time; partial sums (code offset
         //      removed) into per-owner blocks ----
@@ -519,8 +528,12 @@ __device__ __forceinline__ void ds_op(const DsProgram &p, const DsOp &op, int j,
                 const int rgi1 = rgi0 + 8;
                 const bool two = rgi1 < nrgi;
                 const int mat0 = rgi0 >= RG ? 1 : 0, mat1 = rgi1 >= RG ? 1 : 0;
-                const uint32_t w0 = smem_u32(sW) + mat0 * w_mat_bytes + (uint32_t)((rgi0 - mat0 * RG) * 16 + g) * box_w + t4 * 4;
-                const uint32_t w1 = smem_u32(sW) + mat1 * w_mat_bytes + (uint32_t)((rgi1 - mat1 * RG) * 16 + g) * box_w + t4 * 4;
+                if (!up_ready && (mat0 || (two && mat1))) { // row groups of the up projection from here on
+                    st.ok = mbar_spin(&bar_full[(q0 + 1) % DS_PSLOTS], (uint32_t)((q0 + 1) / DS_PSLOTS) & 1u) && st.ok;
+                    up_ready = true;
+                }
+                const uint32_t w0 = smem_u32(smem) + (mat0 ? wb1 : wb0) + (uint32_t)((rgi0 - mat0 * RG) * 16 + g) * box_w + t4 * 4;
+                const uint32_t w1 = smem_u32(smem) + (mat1 ? wb1 : wb0) + (uint32_t)((rgi1 - mat1 * RG) * 16 + g) * box_w + t4 * 4;
                 // four independent accumulator chains per row group: k-step parity x k half
                 int a0[4][4] = {}, a1[4][4] = {};
                 if (st.ok && ksn > 0) {
@@ -629,7 +642,7 @@ __global__ void __launch_bounds__(DS_THREADS, 1) k_decode_seq(const __grid_const
     const int tid = threadIdx.x;
     if (tid == 0) {
         uint64_t *bars = reinterpret_cast<uint64_t *>(smem);
-        for (int i = 0; i < DS_SLOTS; ++i) mbar_init(&bars[DS_BAR_FULL / 8 + i], DS_CONTROL);
+        for (int i = 0; i < DS_PSLOTS; ++i) mbar_init(&bars[DS_BAR_FULL / 8 + i], DS_CONTROL);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bars[DS_BAR_AMAX / 8 + i], 1);
             mbar_init(&bars[DS_BAR_RED / 8 + i], 1);
@@ -653,7 +666,7 @@ __global__ void __launch_bounds__(DS_THREADS, 1) k_decode_seq(const __grid_const
 
     if (tid >= DS_COMPUTE) {
         // control warps: keep the weight ring full, publish each op's completion
-        DsIssue iss = {0u, 0, first};
+        DsIssue iss = {0u, 0, first, 0, 0};
         ds_issue(p, smem, iss, 0);
         const uint32_t *released = reinterpret_cast<const uint32_t *>(smem + DS_RELEASED);
         const uint32_t *done = reinterpret_cast<const uint32_t *>(smem + DS_DONE);
@@ -709,16 +722,19 @@ __global__ void __launch_bounds__(DS_THREADS, 1) k_decode_seq(const __grid_const
         uint32_t head = 0;
         DsState st = {0, 0u, true};
         const uint32_t *desc_ready = reinterpret_cast<const uint32_t *>(smem + DS_DESC_READY);
-        int prev = -1, k = 0;
+        int prev = -1, k = 0, pieces = 0;
         for (int j = first; j >= 0; ++k) {
             st.ok = wait_local(desc_ready, (uint32_t)k + 1) && st.ok;
             const DsOp &op = ds_desc(smem, k);
             const int nxt = op.nxt; // read before the slot can be restaged (after this op)
-            const uint32_t size = ds_slice_bytes(op);
-            const uint32_t start = ring_place(head, size, p.ring_bytes);
-            head = start + size;
-            const uint32_t wbase = p.ring_off + start % p.ring_bytes;
-            ds_op(p, op, j, k, prev, wbase, smem, st, nxt < 0);
+            // ring positions of the op's pieces: the same sequence the control warps place
+            const uint32_t size = ds_piece_bytes(op);
+            const uint32_t start0 = ring_place(head, size * op.nmat, p.ring_bytes);
+            const uint32_t start1 = start0 + size; // the up projection's piece (gated FFN)
+            head = start0 + size * op.nmat;
+            ds_op(p, op, j, k, prev, pieces, p.ring_off + start0 % p.ring_bytes, p.ring_off + start1 % p.ring_bytes,
+                  smem, st, nxt < 0);
+            pieces += op.nmat;
             prev = j;
             j = nxt;
         }
