@@ -35,6 +35,8 @@ def _bind(path):
         "oracle_int_dot_samples": ([P, P, I, P, P, I, P], None),
         "oracle_dequant": ([P, P, F, I, I, P], None),
         "oracle_relu2_gate": ([P, P, I, P], None),
+        "oracle_sumsq": ([P, I], ctypes.c_double),
+        "oracle_rmsnorm": ([P, P, I, I, F, P, P], None),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -180,3 +182,37 @@ def ffn_gate_up(x, packed_g, gamma_g, packed_u, gamma_u, k):
     yg, acc_g, x_q, s = bitlinear(x, packed_g, gamma_g, k)
     yu, acc_u, _, _ = bitlinear(x, packed_u, gamma_u, k)
     return relu2_gate(yg, yu), acc_g, acc_u, x_q, s
+
+
+RMS_EPS = 1e-5  # rms_norm_eps of BitNetConfig
+
+
+def sumsq(row):
+    """Sum of squares of one row (binary64, the fixed partial/pairing order)."""
+    row, p = _c(row, np.float32)
+    return float(_load().oracle_sumsq(p, row.shape[0]))
+
+
+def rmsnorm(x, g, eps=RMS_EPS):
+    """x: float32 [M][K], g: float32 [K]. Returns (y float32 [M][K], r float32 [M])."""
+    x, px = _c(x, np.float32)
+    g, pg = _c(g, np.float32)
+    m, k = x.shape
+    y = np.empty((m, k), np.float32)
+    r = np.empty(m, np.float32)
+    _load().oracle_rmsnorm(px, pg, m, k, float(eps), y.ctypes.data_as(ctypes.c_void_p),
+                           r.ctypes.data_as(ctypes.c_void_p))
+    return y, r
+
+
+def rmsnorm_quant_act(x, g, eps=RMS_EPS):
+    """RMS normalisation followed by the per-token absmax quantiser: (x_q, s, rowsum, y, r)."""
+    y, r = rmsnorm(x, g, eps)
+    x_q, s, rs = quant_act(y)
+    return x_q, s, rs, y, r
+
+
+def bitlinear_norm(x, g, packed, gamma_, k, eps=RMS_EPS):
+    """BitLinear of the RMS-normalised input: (y fp64, acc, x_q, s)."""
+    xn, _ = rmsnorm(x, g, eps)
+    return bitlinear(xn, packed, gamma_, k)

@@ -229,3 +229,61 @@ void oracle_relu2_gate(const double *g, const double *u, int64_t count, double *
         h[i] = r * r * u[i];
     }
 }
+
+/* ---- RMS normalisation in front of the activation quantiser ------------- */
+
+/* Page, "Model details" / "Architecture": the model uses subln normalisation
+ * and no bias terms in its normalisation layers; BitNetConfig: rms_norm_eps =
+ * 1e-5, the epsilon of the rms normalisation layers.  Reading (the page gives
+ * no formula): y = x / sqrt(mean_k(x_k^2) + eps) * g, with a per-feature
+ * weight g and no bias; BitLinear then quantises y per token as above.
+ *
+ * Order and precision (the page is silent; one ulp in 1/rms can move a
+ * quantised code, so this reading fixes them):
+ *   S_t = sum of x_k^2 over k = t, t + 256, t + 512, ... in ascending k, in
+ *         binary64, for t = 0 .. 255 (x_k^2 of a bf16 or fp32 value is exact);
+ *   the partials of each group t = 32w .. 32w + 31 are combined by pairing
+ *         halves: P_i = S_i + S_{i+16} (i < 16), then P_i + P_{i+8} (i < 8),
+ *         then + P_{i+4}, + P_{i+2}, + P_{i+1}, giving G_w;
+ *   ss  = the same pairing over the 8 group sums: G_i + G_{i+4}, + G_{i+2},
+ *         + G_{i+1};
+ *   r   = (float)(1 / sqrt(ss / K + eps)), every step in binary64 (correctly
+ *         rounded division and square root), rounded once to binary32;
+ *   y_k = (x_k * r) * g_k in binary32, two roundings in this order. */
+
+/* pair v[i] with v[i + n/2] until one value is left (n a power of two) */
+static double oracle_pairing_sum(double *v, int n)
+{
+    for (int half = n / 2; half >= 1; half /= 2)
+        for (int i = 0; i < half; ++i) v[i] = v[i] + v[i + half];
+    return v[0];
+}
+
+double oracle_sumsq(const float *row, int64_t k_cols)
+{
+    double part[256];
+    for (int t = 0; t < 256; ++t) {
+        double acc = 0.0;
+        for (int64_t k = t; k < k_cols; k += 256) acc += (double)row[k] * (double)row[k];
+        part[t] = acc;
+    }
+    double group[8];
+    for (int w = 0; w < 8; ++w) group[w] = oracle_pairing_sum(part + 32 * w, 32);
+    return oracle_pairing_sum(group, 8);
+}
+
+/* x, y: [m_rows][k_cols]; g: [k_cols]; r_out: [m_rows] (may be NULL). */
+void oracle_rmsnorm(const float *x, const float *g, int64_t m_rows, int64_t k_cols, float eps, float *y,
+                    float *r_out)
+{
+    for (int64_t m = 0; m < m_rows; ++m) {
+        const float *row = x + m * k_cols;
+        const double ss = oracle_sumsq(row, k_cols);
+        const float r = (float)(1.0 / sqrt(ss / (double)k_cols + (double)eps));
+        for (int64_t k = 0; k < k_cols; ++k) {
+            const float xr = row[k] * r;
+            y[m * k_cols + k] = xr * g[k];
+        }
+        if (r_out) r_out[m] = r;
+    }
+}

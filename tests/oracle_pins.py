@@ -315,4 +315,78 @@ def pin_ffn_composition():
     assert np.allclose(h[pos], (yg[pos] ** 2) * yu[pos], rtol=1e-15, atol=0)
 
 
+# ---------------------------------------------------------------- RMS normalisation (subln) prologue
+def pin_rmsnorm_exact_integer_sum():
+    """x_k = k + 1: the sum of squares is n(n+1)(2n+1)/6 exactly (every partial and pairing
+    step is an exact integer in binary64); r follows from it by one division and one root."""
+    for n in (64, 512, 2560, 6912):
+        x = np.arange(1, n + 1, dtype=np.float32)
+        exact = n * (n + 1) * (2 * n + 1) // 6
+        assert oracle.sumsq(x) == float(exact)
+        y, r = oracle.rmsnorm(x[None, :], np.ones(n, np.float32))
+        want = np.float32(1.0 / math.sqrt(exact / n + oracle.RMS_EPS))
+        assert r[0] == want
+        # y_k = fl(k * r): monotone, last element = fl(n * r)
+        assert y[0, -1] == np.float32(np.float32(n) * want)
+
+
+def pin_rmsnorm_eps_dominates_tiny_rows():
+    """mean(x^2) << eps: y = x / sqrt(mean + eps) ~ x / sqrt(eps) (eps = 1e-5 must be present)."""
+    x = (synth.activations_f32(3, 256, 301) * np.float32(1e-4)).astype(np.float32)
+    y, r = oracle.rmsnorm(x, np.ones(256, np.float32))
+    ms = np.mean(x.astype(np.float64) ** 2, axis=1)
+    want = 1.0 / np.sqrt(ms + 1e-5)
+    assert np.all(np.abs(r.astype(np.float64) - want) <= 2 ** -23 * want)
+    assert np.all(ms < 1e-6)
+    # the result is far from x / rms(x), which a dropped eps would give
+    assert np.all(r.astype(np.float64) < 0.5 / np.sqrt(ms))
+
+
+def pin_rmsnorm_constant_row_quantises_to_127():
+    """x = c everywhere, g = 1: every y_k equals c * r, so every code is +-127."""
+    for c in (0.75, -3.0, 1e3):
+        x = np.full((1, 320), c, np.float32)
+        x_q, s, rs, y, r = oracle.rmsnorm_quant_act(x, np.ones(320, np.float32))
+        assert abs(float(r[0]) - 1.0 / math.sqrt(c * c + 1e-5)) <= 2 ** -23 / math.sqrt(c * c + 1e-5)
+        assert np.all(y == y[0, 0])
+        assert np.all(x_q == (127 if c > 0 else -127))
+        assert rs[0] == 320 * (127 if c > 0 else -127)
+
+
+def pin_rmsnorm_power_of_two_invariance():
+    """With eps = 0, scaling x by 2^j scales the sum of squares by 4^j exactly and r by 2^-j
+    exactly, so y is bit-identical."""
+    x = synth.bf16_bits_to_f32(synth.activations(4, 2560, 302))
+    g = synth.activations_f32(1, 2560, 303)[0]
+    y0, r0 = oracle.rmsnorm(x, g, eps=0.0)
+    for j in (-3, 5):
+        y1, r1 = oracle.rmsnorm((x * np.float32(2.0 ** j)).astype(np.float32), g, eps=0.0)
+        assert np.array_equal(y0.view(np.uint32), y1.view(np.uint32))
+        assert np.array_equal(r1, (r0 * np.float32(2.0 ** -j)).astype(np.float32))
+
+
+def pin_rmsnorm_weight_per_feature():
+    """y with weight g equals fl(y with unit weight * g_k) element by element."""
+    x = synth.bf16_bits_to_f32(synth.activations(5, 320, 304))
+    g = (synth.activations_f32(1, 320, 305)[0] * np.float32(0.1) + np.float32(1.0)).astype(np.float32)
+    y1, _ = oracle.rmsnorm(x, np.ones(320, np.float32))
+    yg, _ = oracle.rmsnorm(x, g)
+    assert np.array_equal(yg, (y1 * g[None, :]).astype(np.float32))
+
+
+def pin_rmsnorm_sumsq_rounding_bound():
+    """Against the correctly rounded sum (math.fsum): the binary64 partial/pairing sum of n
+    exact squares is within n * 2^-53 relative; the mean square of the output is
+    mean(x^2) / (mean(x^2) + eps) to fp32 accuracy."""
+    for n, seed in ((2560, 306), (6912, 307), (100, 308), (333, 309)):
+        x = synth.bf16_bits_to_f32(synth.activations(2, n, seed, "outliers"))
+        for row in x:
+            exact = math.fsum(float(v) * float(v) for v in row)
+            assert abs(oracle.sumsq(row) - exact) <= n * 2.0 ** -53 * exact
+        y, _ = oracle.rmsnorm(x, np.ones(n, np.float32))
+        ms = np.mean(x.astype(np.float64) ** 2, axis=1)
+        got = np.mean(y.astype(np.float64) ** 2, axis=1)
+        assert np.all(np.abs(got - ms / (ms + 1e-5)) <= 1e-6)
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

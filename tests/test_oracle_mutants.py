@@ -43,6 +43,16 @@ MUTANTS = {
     "relu_dropped": ("double r = g[i] > 0.0 ? g[i] : 0.0;", "double r = g[i];"),
     "relu_not_squared": ("h[i] = r * r * u[i];", "h[i] = r * u[i];"),
     "bf16_shift": ("uint32_t bits = ((uint32_t)src[i]) << 16;", "uint32_t bits = ((uint32_t)src[i]) << 15;"),
+    "rms_eps_dropped": ("1.0 / sqrt(ss / (double)k_cols + (double)eps)", "1.0 / sqrt(ss / (double)k_cols)"),
+    "rms_mean_k_minus_1": ("1.0 / sqrt(ss / (double)k_cols + (double)eps)",
+                           "1.0 / sqrt(ss / (double)(k_cols - 1) + (double)eps)"),
+    "rms_not_inverted": ("(float)(1.0 / sqrt(ss / (double)k_cols + (double)eps));",
+                         "(float)(sqrt(ss / (double)k_cols + (double)eps));"),
+    "rms_weight_dropped": ("y[m * k_cols + k] = xr * g[k];", "y[m * k_cols + k] = xr;"),
+    "rms_weight_first_only": ("y[m * k_cols + k] = xr * g[k];", "y[m * k_cols + k] = xr * g[0];"),
+    "sumsq_stride_255": ("for (int64_t k = t; k < k_cols; k += 256)", "for (int64_t k = t; k < k_cols; k += 255)"),
+    "sumsq_abs": ("acc += (double)row[k] * (double)row[k];", "acc += fabs((double)row[k]);"),
+    "pairing_drops_last_group": ("return oracle_pairing_sum(group, 8);", "return oracle_pairing_sum(group, 4);"),
 }
 
 
