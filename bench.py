@@ -253,6 +253,10 @@ class Stack:
         self.ws_pre = torch.empty(ws, dtype=torch.uint8, device=device)
         self.ws_dec = torch.empty(tw.bitnet_workspace_size(B, INTER, INTER), dtype=torch.uint8, device=device)
         self.ws_seq = tw.bitnet_sequence_workspace(device)
+        self.norm_g = (torch.randn(HIDDEN, generator=gen, device=device) * 0.1 + 1.0).float()
+        self.q_buf = torch.empty((M, HIDDEN), dtype=torch.int8, device=device)
+        self.s_buf = torch.empty(M, dtype=torch.float32, device=device)
+        self.rs_buf = torch.empty(M, dtype=torch.int32, device=device)
         self.seq_ops = {}
         self.packed_bytes = sum(p.numel() for L in self.layers for (p, _) in L.values())
 
@@ -526,6 +530,14 @@ def our_arm(a, n_gpus):
                                 True),
             "prefill_down": (lambda s: [st.down(l, st.pre_out, st.ws_pre, s) for l in range(Lyr)],
                              2 * M * INTER * HIDDEN, "tensor", Lyr, Lyr, True),
+            # the activation quantiser alone, and with the RMS normalisation fused in (not in the step)
+            "prefill_quant": (lambda s: [tw.bitnet_quant_act(st.pre_x[l % st.n_pre], x_q=st.q_buf, s=st.s_buf,
+                                                             rowsum=st.rs_buf, stream=s) for l in range(Lyr)],
+                              M * HIDDEN * 2 + M * HIDDEN + 8 * M, "hbm", 0, Lyr, False),
+            "prefill_rmsnorm_quant": (lambda s: [tw.bitnet_rmsnorm_quant(st.pre_x[l % st.n_pre], st.norm_g, x_q=st.q_buf,
+                                                                         s=st.s_buf, rowsum=st.rs_buf, stream=s)
+                                                 for l in range(Lyr)],
+                                      M * HIDDEN * 2 + HIDDEN * 4 + M * HIDDEN + 8 * M, "hbm", 0, Lyr, False),
         }
         for name, (fn, work, bound, per_step, n_ops, in_step) in specs.items():
             if name == "decode_sequence" and not seq:

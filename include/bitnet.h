@@ -207,6 +207,51 @@ bitnet_status_t bitnet_ffn_gate_up(const void *x, bitnet_dtype_t x_dtype, int64_
                                    float *h, int32_t *acc_g_out, int32_t *acc_u_out,
                                    void *workspace, size_t ws_bytes, cudaStream_t stream);
 
+/* ---- RMS normalisation (subln) fused in front of the quantiser ------------ */
+
+/*
+ * x_q = quant(RMSNorm(x)) in one pass over x (page: "Architecture" -- subln
+ * normalisation, no bias in the normalisation layers; BitNetConfig
+ * rms_norm_eps = 1e-5):
+ *   y_k = (x_k * r) * g_k,  r = 1 / sqrt(mean_k(x_k^2) + eps)
+ * followed by the per-token absmax quantiser of bitnet_quant_act applied to y.
+ * Order and precision are fixed so that results are reproducible: the sum of
+ * squares is accumulated in fp64 as 256 partials (partial t sums k = t,
+ * t + 256, ... in ascending k), combined by pairing halves within each group
+ * of 32 partials (16, 8, 4, 2, 1) and then over the 8 groups (4, 2, 1); r is
+ * computed in fp64 with correctly rounded division and square root and
+ * rounded once to fp32; y is two fp32 products in the order shown.
+ *
+ *   x      [M][K] activations of type x_dtype (device, read); K <= 8192
+ *   g      [K] fp32 normalisation weight (device, read)
+ *   eps    >= 0 (1e-5 in BitNet b1.58)
+ *   x_q, s, rowsum   as bitnet_quant_act, for y
+ */
+bitnet_status_t bitnet_rmsnorm_quant(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_t K,
+                                     const float *g, float eps, int8_t *x_q, float *s, int32_t *rowsum,
+                                     cudaStream_t stream);
+
+/*
+ * bitnet_linear / bitnet_ffn_gate_up applied to RMSNorm(x) (weight g, epsilon
+ * eps, as bitnet_rmsnorm_quant): the normalisation runs inside the
+ * quantisation pass, so x is read once and never written back normalised.
+ * Same arguments, results and workspace as bitnet_linear /
+ * bitnet_ffn_gate_up otherwise (K <= 8192).  For M <= 64 the quantiser and
+ * the decode GEMV are separate kernels (the fused-quantiser decode kernel is
+ * not used); BITNET_DISPATCH_DECODE_FUSED gives BITNET_ERR_UNSUPPORTED_SHAPE.
+ */
+bitnet_status_t bitnet_linear_norm(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_t K,
+                                   const float *g, float eps, const uint8_t *w_packed, const float *gamma,
+                                   int64_t N, float *y, int8_t *x_q_out, float *s_out, int32_t *acc_out,
+                                   void *workspace, size_t ws_bytes, cudaStream_t stream);
+
+bitnet_status_t bitnet_ffn_gate_up_norm(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_t K,
+                                        const float *g, float eps,
+                                        const uint8_t *wg_packed, const float *gamma_g,
+                                        const uint8_t *wu_packed, const float *gamma_u, int64_t N,
+                                        float *h, int32_t *acc_g_out, int32_t *acc_u_out,
+                                        void *workspace, size_t ws_bytes, cudaStream_t stream);
+
 /* ---- decode sequences: many small-M ops in one persistent launch ---------- */
 
 typedef enum {

@@ -79,6 +79,9 @@ def load_library(path: str = LIB_PATH):
         "bitnet_set_dispatch": ([I], I),
         "bitnet_launch_count": ([], ctypes.c_uint64),
         "bitnet_linear_noalloc": ([P, I, I64, I64, P, P, I64, P, P], I),
+        "bitnet_rmsnorm_quant": ([P, I, I64, I64, P, F, P, P, P, P], I),
+        "bitnet_linear_norm": ([P, I, I64, I64, P, F, P, P, I64, P, P, P, P, P, SZ, P], I),
+        "bitnet_ffn_gate_up_norm": ([P, I, I64, I64, P, F, P, P, P, P, I64, P, P, P, P, SZ, P], I),
         "bitnet_sequence_workspace_size": ([], SZ),
         "bitnet_sequence_plan": ([ctypes.POINTER(bitnet_op_t), ctypes.c_int32, I64,
                                   ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)], I),
@@ -228,6 +231,55 @@ def bitnet_ffn_gate_up(x, wg_packed, gamma_g, wu_packed, gamma_u, *, h=None, acc
     _check(lib.bitnet_ffn_gate_up(_ptr(x), _dtype_code(x), m, k, _ptr(wg_packed), _ptr(gamma_g), _ptr(wu_packed),
                                   _ptr(gamma_u), n, _ptr(h), _ptr(acc_g_out), _ptr(acc_u_out), _ptr(workspace),
                                   workspace.numel(), _stream(stream)), "bitnet_ffn_gate_up")
+    return h
+
+
+RMS_EPS = 1e-5
+
+
+def bitnet_rmsnorm_quant(x, g, eps=RMS_EPS, *, x_q=None, s=None, rowsum=None, want_rowsum=True, stream=None):
+    """(x_q int8 [M][K], s fp32 [M], rowsum int32 [M] or None) of RMSNorm(x) with weight g."""
+    lib = load_library()
+    m, k = x.shape
+    if x_q is None:
+        x_q = torch.empty((m, k), dtype=torch.int8, device=x.device)
+    if s is None:
+        s = torch.empty(m, dtype=torch.float32, device=x.device)
+    if rowsum is None and want_rowsum:
+        rowsum = torch.empty(m, dtype=torch.int32, device=x.device)
+    _check(lib.bitnet_rmsnorm_quant(_ptr(x), _dtype_code(x), m, k, _ptr(g), float(eps), _ptr(x_q), _ptr(s),
+                                    _ptr(rowsum), _stream(stream)), "bitnet_rmsnorm_quant")
+    return x_q, s, rowsum
+
+
+def bitnet_linear_norm(x, g, w_packed, gamma, eps=RMS_EPS, *, y=None, x_q_out=None, s_out=None, acc_out=None,
+                       workspace=None, stream=None):
+    """y [M][N] fp32 = BitLinear(RMSNorm(x, g))."""
+    lib = load_library()
+    m, k = x.shape
+    n = w_packed.shape[0]
+    if y is None:
+        y = torch.empty((m, n), dtype=torch.float32, device=x.device)
+    workspace = _workspace(workspace, m, n, k, x.device)
+    _check(lib.bitnet_linear_norm(_ptr(x), _dtype_code(x), m, k, _ptr(g), float(eps), _ptr(w_packed), _ptr(gamma), n,
+                                  _ptr(y), _ptr(x_q_out), _ptr(s_out), _ptr(acc_out), _ptr(workspace),
+                                  workspace.numel(), _stream(stream)), "bitnet_linear_norm")
+    return y
+
+
+def bitnet_ffn_gate_up_norm(x, g, wg_packed, gamma_g, wu_packed, gamma_u, eps=RMS_EPS, *, h=None, acc_g_out=None,
+                            acc_u_out=None, workspace=None, stream=None):
+    """h [M][N] fp32 = relu(BitLinear_g(RMSNorm(x, g)))^2 * BitLinear_u(RMSNorm(x, g))."""
+    lib = load_library()
+    m, k = x.shape
+    n = wg_packed.shape[0]
+    if h is None:
+        h = torch.empty((m, n), dtype=torch.float32, device=x.device)
+    workspace = _workspace(workspace, m, n, k, x.device)
+    _check(lib.bitnet_ffn_gate_up_norm(_ptr(x), _dtype_code(x), m, k, _ptr(g), float(eps), _ptr(wg_packed),
+                                       _ptr(gamma_g), _ptr(wu_packed), _ptr(gamma_u), n, _ptr(h), _ptr(acc_g_out),
+                                       _ptr(acc_u_out), _ptr(workspace), workspace.numel(), _stream(stream)),
+           "bitnet_ffn_gate_up_norm")
     return h
 
 

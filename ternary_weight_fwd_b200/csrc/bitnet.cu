@@ -253,6 +253,28 @@ cudaError_t launch_quant_t(const void *x, int64_t M, int64_t K, int8_t *xq, floa
     return launch_pdl(k_quant_rows<XF32>, dim3((unsigned)cdiv(M, 8)), dim3(256), 0, stream, x, M, K, xq, s, rs);
 }
 
+// RMS normalisation + quantiser: rows of up to 4096 elements on 128 threads (two rows
+// per CTA), longer rows (up to 8192) on 256.
+constexpr int64_t kNormMaxK = 256 * RQ_MAX_PER_THREAD;
+
+template <bool XF32>
+cudaError_t launch_norm_quant_t(const void *x, int64_t M, int64_t K, const float *g, float eps, int8_t *xq, float *s,
+                                int32_t *rs, cudaStream_t stream)
+{
+    if (K <= 128 * RQ_MAX_PER_THREAD)
+        return launch_pdl(k_rmsnorm_quant_rows<XF32, 128>, dim3((unsigned)cdiv(M, 2)), dim3(256), 0, stream, x, M, K,
+                          g, eps, xq, s, rs);
+    return launch_pdl(k_rmsnorm_quant_rows<XF32, 256>, dim3((unsigned)M), dim3(256), 0, stream, x, M, K, g, eps, xq, s,
+                      rs);
+}
+
+cudaError_t launch_norm_quant(const void *x, bool xf32, int64_t M, int64_t K, const float *g, float eps, int8_t *xq,
+                              float *s, int32_t *rs, cudaStream_t stream)
+{
+    return xf32 ? launch_norm_quant_t<true>(x, M, K, g, eps, xq, s, rs, stream)
+                : launch_norm_quant_t<false>(x, M, K, g, eps, xq, s, rs, stream);
+}
+
 cudaError_t launch_quant(const void *x, bool xf32, int64_t M, int64_t K, int8_t *xq, float *s, int32_t *rs,
                          cudaStream_t stream)
 {
@@ -459,16 +481,21 @@ bitnet_status_t dc_forward(const DcCfg &c, const void *x, bool xf32, int64_t M, 
 }
 
 // Shared body of bitnet_linear (nmat = 1) and bitnet_ffn_gate_up (nmat = 2).
+// Shared body of the BitLinear entry points.  norm_g (optional): RMS-normalise
+// x with weight norm_g and epsilon norm_eps before quantising it.
 bitnet_status_t forward(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_t K, const uint8_t *w0,
                         const float *gamma0, const uint8_t *w1, const float *gamma1, int64_t N, float *y,
                         int8_t *x_q_out, float *s_out, int32_t *acc0, int32_t *acc1, void *workspace,
-                        size_t ws_bytes, cudaStream_t stream, int nmat)
+                        size_t ws_bytes, cudaStream_t stream, int nmat, const float *norm_g = nullptr,
+                        float norm_eps = 0.0f)
 {
     bitnet_status_t st = check_shape(M, N, K);
     if (st != BITNET_OK) return st;
     if (x_dtype != BITNET_DTYPE_BF16 && x_dtype != BITNET_DTYPE_F32) return BITNET_ERR_INVALID_ARG;
     if (!x || !w0 || !gamma0 || !y || (nmat == 2 && (!w1 || !gamma1))) return BITNET_ERR_INVALID_ARG;
-    const void *ptrs[] = {x, w0, gamma0, w1, gamma1, y, x_q_out, s_out, acc0, acc1, workspace};
+    if (norm_g && (K > kNormMaxK || !(norm_eps >= 0.0f) || !std::isfinite(norm_eps)))
+        return norm_g && K > kNormMaxK ? BITNET_ERR_UNSUPPORTED_SHAPE : BITNET_ERR_INVALID_ARG;
+    const void *ptrs[] = {x, w0, gamma0, w1, gamma1, y, x_q_out, s_out, acc0, acc1, workspace, norm_g};
     for (const void *p : ptrs)
         if (p && !aligned16(p)) return BITNET_ERR_MISALIGNED;
     if (!workspace || ws_bytes < ws_bytes_for(M, K)) return BITNET_ERR_WORKSPACE;
@@ -481,15 +508,21 @@ bitnet_status_t forward(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_
     int8_t *xq = x_q_out ? x_q_out : ws.xq;
     float *s = s_out ? s_out : ws.s;
 
+    // the normalising quantiser runs as its own kernel ahead of the GEMM
+    auto quantise = [&](int8_t *q, float *sc, int32_t *rs) {
+        return norm_g ? launch_norm_quant(x, xf32, M, K, norm_g, norm_eps, q, sc, rs, stream)
+                      : launch_quant(x, xf32, M, K, q, sc, rs, stream);
+    };
     if (M <= kDecodeMaxM && dispatch != BITNET_DISPATCH_PREFILL) {
         // cluster kernel with the quantiser fused in (automatic choice for decode)
-        if (dispatch != BITNET_DISPATCH_DECODE) {
+        if (dispatch != BITNET_DISPATCH_DECODE && !norm_g) {
             const DcCfg c = dc_config(N, K, nmat, xf32, M <= 8, dev, sms);
             if (c.ok)
                 return dc_forward(c, x, xf32, M, K, w0, gamma0, w1, gamma1, N, y, x_q_out, s_out, acc0, acc1,
                                   stream, nmat);
             if (dispatch == BITNET_DISPATCH_DECODE_FUSED) return BITNET_ERR_UNSUPPORTED_SHAPE;
         }
+        if (norm_g && dispatch == BITNET_DISPATCH_DECODE_FUSED) return BITNET_ERR_UNSUPPORTED_SHAPE;
         // quantiser kernel, then the row-split decode kernel
         const DecodeCfg c = decode_config(N, K, nmat, sms);
         if (c.ok) {
@@ -511,7 +544,7 @@ bitnet_status_t forward(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_
             a.rg = c.rg;
             a.w_stride = c.w_stride;
             a.rp = c.rp;
-            cudaError_t e = launch_quant(x, xf32, M, K, xq, s, ws.rs, stream);
+            cudaError_t e = quantise(xq, s, ws.rs);
             if (e == cudaSuccess)
                 e = nmat == 1 ? launch_decode<1>(a, c, stream, dev) : launch_decode<2>(a, c, stream, dev);
             return cuda_status(e);
@@ -551,7 +584,7 @@ bitnet_status_t forward(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_
     // fp32 output through TMA stores (32 x 32 boxes, 128-byte swizzle) when rows are 16-byte multiples
     tmY = tmA;
     if (a.vec_ok && !encode_f32_2d_sw128(&tmY, y, (uint64_t)M, (uint64_t)N, 32, 32)) return BITNET_ERR_CUDA;
-    cudaError_t e = launch_quant(x, xf32, M, K, xq, s, nullptr, stream);
+    cudaError_t e = quantise(xq, s, nullptr);
     if (e != cudaSuccess) return BITNET_ERR_CUDA;
     const int grid = std::min(a.num_tiles, sms);
     if (nmat == 1) {
@@ -1072,6 +1105,40 @@ int bitnet_set_sequence_cluster(int cluster_size)
 {
     if (cluster_size != 4 && cluster_size != 8) return -1;
     return g_seq_cluster.exchange(cluster_size);
+}
+
+bitnet_status_t bitnet_rmsnorm_quant(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_t K, const float *g,
+                                     float eps, int8_t *x_q, float *s, int32_t *rowsum, cudaStream_t stream)
+{
+    bitnet_status_t st = check_shape(M, 1, K);
+    if (st != BITNET_OK) return st;
+    if (x_dtype != BITNET_DTYPE_BF16 && x_dtype != BITNET_DTYPE_F32) return BITNET_ERR_INVALID_ARG;
+    if (!x || !g || !x_q || !s || !(eps >= 0.0f) || !std::isfinite(eps)) return BITNET_ERR_INVALID_ARG;
+    if (K > kNormMaxK) return BITNET_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(x) || !aligned16(g) || !aligned16(x_q) || !aligned16(s) || (rowsum && !aligned16(rowsum)))
+        return BITNET_ERR_MISALIGNED;
+    return cuda_status(launch_norm_quant(x, x_dtype == BITNET_DTYPE_F32, M, K, g, eps, x_q, s, rowsum, stream));
+}
+
+bitnet_status_t bitnet_linear_norm(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_t K, const float *g,
+                                   float eps, const uint8_t *w_packed, const float *gamma, int64_t N, float *y,
+                                   int8_t *x_q_out, float *s_out, int32_t *acc_out, void *workspace, size_t ws_bytes,
+                                   cudaStream_t stream)
+{
+    if (!g) return BITNET_ERR_INVALID_ARG;
+    return forward(x, x_dtype, M, K, w_packed, gamma, nullptr, nullptr, N, y, x_q_out, s_out, acc_out, nullptr,
+                   workspace, ws_bytes, stream, 1, g, eps);
+}
+
+bitnet_status_t bitnet_ffn_gate_up_norm(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_t K, const float *g,
+                                        float eps, const uint8_t *wg_packed, const float *gamma_g,
+                                        const uint8_t *wu_packed, const float *gamma_u, int64_t N, float *h,
+                                        int32_t *acc_g_out, int32_t *acc_u_out, void *workspace, size_t ws_bytes,
+                                        cudaStream_t stream)
+{
+    if (!g) return BITNET_ERR_INVALID_ARG;
+    return forward(x, x_dtype, M, K, wg_packed, gamma_g, wu_packed, gamma_u, N, h, nullptr, nullptr, acc_g_out,
+                   acc_u_out, workspace, ws_bytes, stream, 2, g, eps);
 }
 
 bitnet_status_t bitnet_device_status(int clear, bitnet_status_t *status_out, cudaStream_t stream)

@@ -228,4 +228,114 @@ __global__ void __launch_bounds__(256) k_quant_rows_reg(const void *__restrict__
     }
 }
 
+// ---------------------------------------------------------------------------
+// RMS normalisation (subln) fused in front of the per-token absmax quantiser:
+// y = (x * r) * g with r = 1 / sqrt(mean(x^2) + eps), then the quantiser on y.
+// BitNet model page, "Model details" / "Architecture" (subln normalisation, no
+// bias) and BitNetConfig (rms_norm_eps).  Each row is held in registers by
+// 128 or 256 threads, so x is read once.  The sum of squares follows the fixed order of this library's
+// definition: per-thread binary64 partials in ascending k, combined within
+// each warp by pairing halves (16, 8, 4, 2, 1) and then over the 8 warps by
+// pairing halves (4, 2, 1); r is computed in binary64 (correctly rounded
+// division and square root) and rounded once to binary32.
+// ---------------------------------------------------------------------------
+constexpr int RQ_PARTIALS = 256;      // binary64 partial sums of squares per row (fixed by the definition)
+constexpr int RQ_MAX_PER_THREAD = 32; // elements a thread holds in registers
+
+// TPR threads per row (128 or 256), 256 / TPR rows per CTA; thread t of a row
+// owns partials t + j * TPR (j < 256 / TPR).  Each warp runs the pairing tree
+// once per partial set, so the group sums (and hence every rounding) are those
+// of the definition whatever TPR is.
+template <bool XF32, int TPR>
+__global__ void __launch_bounds__(256) k_rmsnorm_quant_rows(const void *__restrict__ x, int64_t M, int64_t K,
+                                                            const float *__restrict__ g, float eps,
+                                                            int8_t *__restrict__ x_q, float *__restrict__ s,
+                                                            int32_t *__restrict__ rowsum)
+{
+    constexpr int RPC = 256 / TPR;         // rows per CTA
+    constexpr int WPR = TPR / 32;          // warps per row
+    constexpr int PSETS = RQ_PARTIALS / TPR; // partial sets per thread
+    __shared__ double red_ss[RPC][8];
+    __shared__ float red_max[RPC][WPR];
+    __shared__ int red_sum[RPC][WPR];
+    __shared__ float bcast[RPC][2];
+    pdl_launch_dependents();
+    pdl_wait();
+    const int lr = threadIdx.x / TPR;      // row of this CTA
+    const int t = threadIdx.x % TPR;       // thread within the row
+    const int wr = t >> 5, lane = t & 31;  // warp within the row
+    const int64_t m = (int64_t)blockIdx.x * RPC + lr;
+    const bool live = m < M;
+    float v[RQ_MAX_PER_THREAD];
+    // element e of this thread: partial set j = e % PSETS, step i = e / PSETS, k = t + j * TPR + 256 i
+    const int n = live ? (int)((K + TPR - 1 - t) / TPR) : 0; // elements k = t + TPR * e, e < n
+    if constexpr (XF32) {
+        const float *row = static_cast<const float *>(x) + (live ? m : 0) * K;
+#pragma unroll
+        for (int e = 0; e < RQ_MAX_PER_THREAD; ++e)
+            if (e < n) v[e] = __ldg(row + t + (int64_t)e * TPR);
+    } else {
+        const unsigned short *row = static_cast<const unsigned short *>(x) + (live ? m : 0) * K;
+#pragma unroll
+        for (int e = 0; e < RQ_MAX_PER_THREAD; ++e)
+            if (e < n) v[e] = __uint_as_float((uint32_t)__ldg(row + t + (int64_t)e * TPR) << 16);
+    }
+    // partial j holds k = t + j * TPR + 256 i = t + TPR * (j + PSETS * i), i.e. e = j + PSETS * i
+#pragma unroll
+    for (int j = 0; j < PSETS; ++j) {
+        double part = 0.0;
+#pragma unroll
+        for (int e = j; e < RQ_MAX_PER_THREAD; e += PSETS)
+            if (e < n) part = __dadd_rn(part, __dmul_rn((double)v[e], (double)v[e]));
+        for (int d = 16; d >= 1; d >>= 1) part = __dadd_rn(part, __shfl_down_sync(0xffffffffu, part, d));
+        if (lane == 0) red_ss[lr][wr + j * WPR] = part; // group (t + j * TPR) / 32
+    }
+    __syncthreads();
+    if (t == 0) {
+        double gsum[8];
+        for (int w = 0; w < 8; ++w) gsum[w] = red_ss[lr][w];
+        for (int half = 4; half >= 1; half >>= 1)
+            for (int i = 0; i < half; ++i) gsum[i] = __dadd_rn(gsum[i], gsum[i + half]);
+        const double mean = __ddiv_rn(gsum[0], (double)K);
+        bcast[lr][0] = __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(mean, (double)eps))));
+    }
+    __syncthreads();
+    const float r = bcast[lr][0];
+    float mx = 0.0f;
+#pragma unroll
+    for (int e = 0; e < RQ_MAX_PER_THREAD; ++e)
+        if (e < n) {
+            v[e] = __fmul_rn(__fmul_rn(v[e], r), __ldg(g + t + e * TPR));
+            mx = fmaxf(mx, fabsf(v[e]));
+        }
+    mx = warp_max(mx);
+    if (lane == 0) red_max[lr][wr] = mx;
+    __syncthreads();
+    if (t == 0) {
+        float am = 0.0f;
+        for (int w = 0; w < WPR; ++w) am = fmaxf(am, red_max[lr][w]);
+        bcast[lr][1] = quant_scale(am);
+    }
+    __syncthreads();
+    const float sc = bcast[lr][1];
+    int rs = 0;
+    int8_t *qrow = x_q + (live ? m : 0) * K;
+#pragma unroll
+    for (int e = 0; e < RQ_MAX_PER_THREAD; ++e)
+        if (e < n) {
+            const int q = quant_one(v[e], sc);
+            qrow[t + e * TPR] = (int8_t)q;
+            rs += q;
+        }
+    rs = warp_sum(rs);
+    if (lane == 0) red_sum[lr][wr] = rs;
+    __syncthreads();
+    if (t == 0 && live) {
+        int tot = 0;
+        for (int w = 0; w < WPR; ++w) tot += red_sum[lr][w];
+        s[m] = sc;
+        if (rowsum) rowsum[m] = tot;
+    }
+}
+
 } // namespace bitnet

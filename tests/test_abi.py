@@ -116,3 +116,26 @@ def test_ffn_and_quant_and_pack_reject_before_launch(lib):
         tw.BITNET_ERR_INVALID_ARG
     assert lib.bitnet_pack_weights(P(FAKE + 4), 16, 64, 1e-5, P(FAKE), P(FAKE), P(FAKE), 4096, None) == \
         tw.BITNET_ERR_MISALIGNED
+
+
+def test_norm_entry_points_reject_before_launch(lib):
+    """bitnet_rmsnorm_quant / bitnet_linear_norm validate on the host (no GPU needed)."""
+    P = 1 << 40
+    st = lib.bitnet_rmsnorm_quant
+    assert st(None, 0, 4, 256, P, 1e-5, P, P, None, None) == tw.BITNET_ERR_INVALID_ARG
+    assert st(P, 0, 4, 256, None, 1e-5, P, P, None, None) == tw.BITNET_ERR_INVALID_ARG
+    assert st(P, 0, 4, 256, P, -1.0, P, P, None, None) == tw.BITNET_ERR_INVALID_ARG
+    assert st(P, 0, 4, 256, P, float("nan"), P, P, None, None) == tw.BITNET_ERR_INVALID_ARG
+    assert st(P, 0, 4, 96, P, 1e-5, P, P, None, None) == tw.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert st(P, 0, 4, 8256, P, 1e-5, P, P, None, None) == tw.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert st(P + 4, 0, 4, 256, P, 1e-5, P, P, None, None) == tw.BITNET_ERR_MISALIGNED
+    assert st(P, 0, 4, 256, P + 8, 1e-5, P, P, None, None) == tw.BITNET_ERR_MISALIGNED
+    assert st(P, 7, 4, 256, P, 1e-5, P, P, None, None) == tw.BITNET_ERR_INVALID_ARG
+    ln = lib.bitnet_linear_norm
+    ws = tw.bitnet_workspace_size(4, 256, 256)
+    assert ln(P, 0, 4, 256, None, 1e-5, P, P, 256, P, None, None, None, P, ws, None) == tw.BITNET_ERR_INVALID_ARG
+    assert ln(P, 0, 4, 8256, P, 1e-5, P, P, 256, P, None, None, None, P, ws, None) == \
+        tw.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert ln(P, 0, 4, 256, P + 4, 1e-5, P, P, 256, P, None, None, None, P, ws, None) == tw.BITNET_ERR_MISALIGNED
+    fn = lib.bitnet_ffn_gate_up_norm
+    assert fn(P, 0, 4, 256, None, 1e-5, P, P, P, P, 256, P, None, None, P, ws, None) == tw.BITNET_ERR_INVALID_ARG
