@@ -37,6 +37,10 @@ def _bind(path):
         "oracle_relu2_gate": ([P, P, I, P], None),
         "oracle_sumsq": ([P, I], ctypes.c_double),
         "oracle_rmsnorm": ([P, P, I, I, F, P, P], None),
+        "oracle_quant_act_amax": ([P, I, I, P, P, P, P], None),
+        "oracle_epilogue_f32": ([P, P, P, F, F, I, I, P], None),
+        "oracle_f32_to_bf16": ([P, I, P], None),
+        "oracle_row_absmax": ([P, I, I, P], None),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -114,16 +118,23 @@ def pack_weights(w, eps=QUANT_EPS):
     return pack(w_q), g, w_q
 
 
-def quant_act(x):
-    """x: float32 [M][K] (exact bf16 values or fp32). Returns (x_q, s, rowsum)."""
+def quant_act(x, amax=None):
+    """x: float32 [M][K] (exact bf16 values or fp32). Returns (x_q, s, rowsum).
+
+    amax: optional float32 [M] per-token maxima used instead of max|x|."""
     x, p = _c(x, np.float32)
     m, k = x.shape
     x_q = np.empty((m, k), np.int8)
     s = np.empty(m, np.float32)
     rs = np.empty(m, np.int32)
-    _load().oracle_quant_act(p, m, k, x_q.ctypes.data_as(ctypes.c_void_p),
-                             s.ctypes.data_as(ctypes.c_void_p),
-                             rs.ctypes.data_as(ctypes.c_void_p))
+    out = (x_q.ctypes.data_as(ctypes.c_void_p), s.ctypes.data_as(ctypes.c_void_p),
+           rs.ctypes.data_as(ctypes.c_void_p))
+    if amax is None:
+        _load().oracle_quant_act(p, m, k, *out)
+    else:
+        a, pa = _c(amax, np.float32)
+        assert a.shape == (m,)
+        _load().oracle_quant_act_amax(p, m, k, pa, *out)
     return x_q, s, rs
 
 
@@ -216,3 +227,58 @@ def bitlinear_norm(x, g, packed, gamma_, k, eps=RMS_EPS):
     """BitLinear of the RMS-normalised input: (y fp64, acc, x_q, s)."""
     xn, _ = rmsnorm(x, g, eps)
     return bitlinear(xn, packed, gamma_, k)
+
+
+def epilogue_f32(acc_g, s, gamma_g, acc_u=None, gamma_u=0.0):
+    """The fp32 epilogue value of every output (y32, or h32 when acc_u is given)."""
+    ag, pg = _c(acc_g, np.int64)
+    sv, ps = _c(s, np.float32)
+    m, n = ag.shape
+    pu = None
+    if acc_u is not None:
+        au, pu = _c(acc_u, np.int64)
+        assert au.shape == ag.shape
+    y = np.empty((m, n), np.float32)
+    _load().oracle_epilogue_f32(pg, pu, ps, float(gamma_g), float(gamma_u), m, n,
+                                y.ctypes.data_as(ctypes.c_void_p))
+    return y
+
+
+def f32_to_bf16(v):
+    """float32 -> bf16 bit patterns (uint16), round to nearest even."""
+    src, p = _c(v, np.float32)
+    out = np.empty(src.shape, np.uint16)
+    _load().oracle_f32_to_bf16(p, src.size, out.ctypes.data_as(ctypes.c_void_p))
+    return out
+
+
+def row_absmax(v):
+    """float32 [M][N] -> float32 [M], max |v| of each row."""
+    src, p = _c(v, np.float32)
+    m, n = src.shape
+    out = np.empty(m, np.float32)
+    _load().oracle_row_absmax(p, m, n, out.ctypes.data_as(ctypes.c_void_p))
+    return out
+
+
+def bitlinear_ex(x, packed, gamma_, k, y_dtype="f32", x_amax=None, packed_u=None, gamma_u=None):
+    """BitLinear (or, with packed_u, the gated FFN) with its output as stored.
+
+    Returns (y, y_amax): y float32 [M][N] (y_dtype "f32") or bf16 bit patterns
+    uint16 (y_dtype "bf16"); y_amax float32 [M] = max |stored value| per row.
+    x_amax: optional per-token maxima handed to the quantiser."""
+    w_q, bad = unpack(packed, k)
+    assert bad == 0
+    x_q, s, _ = quant_act(x, x_amax)
+    acc = int_matmul(x_q, w_q)
+    acc_u = None
+    if packed_u is not None:
+        wu, bad = unpack(packed_u, k)
+        assert bad == 0
+        acc_u = int_matmul(x_q, wu)
+    y32 = epilogue_f32(acc, s, gamma_, acc_u, 0.0 if gamma_u is None else gamma_u)
+    if y_dtype == "f32":
+        return y32, row_absmax(y32)
+    assert y_dtype == "bf16"
+    yb = f32_to_bf16(y32)
+    return yb, row_absmax(bf16_to_f32(yb))

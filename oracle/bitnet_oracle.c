@@ -150,8 +150,21 @@ int64_t oracle_unpack(const uint8_t *packed, int64_t n_rows, int64_t k_cols, int
 /* x: [m_rows][k_cols] fp32 (bf16 inputs are converted exactly beforehand).
  * Writes x_q [m_rows][k_cols], s [m_rows] and, if non-NULL, rowsum [m_rows]
  * (sum of x_q over the row, used by the code-offset form of the product). */
+void oracle_quant_act_amax(const float *x, int64_t m_rows, int64_t k_cols, const float *amax_in,
+                           int8_t *x_q, float *s, int32_t *rowsum);
+
 void oracle_quant_act(const float *x, int64_t m_rows, int64_t k_cols,
                       int8_t *x_q, float *s, int32_t *rowsum)
+{
+    oracle_quant_act_amax(x, m_rows, k_cols, NULL, x_q, s, rowsum);
+}
+
+/* Same quantiser with the per-token maximum supplied by the caller (amax_in
+ * [m_rows], NULL: computed from x).  A BitLinear whose input was written by
+ * another BitLinear's epilogue gets max|x| from that epilogue instead of
+ * reducing the row again; given the true maximum the result is identical. */
+void oracle_quant_act_amax(const float *x, int64_t m_rows, int64_t k_cols, const float *amax_in,
+                           int8_t *x_q, float *s, int32_t *rowsum)
 {
     for (int64_t m = 0; m < m_rows; ++m) {
         const float *row = x + m * k_cols;
@@ -160,6 +173,7 @@ void oracle_quant_act(const float *x, int64_t m_rows, int64_t k_cols,
             float a = fabsf(row[k]);
             if (a > amax) amax = a;
         }
+        if (amax_in) amax = amax_in[m];
         const float denom = amax > ORACLE_QUANT_EPS ? amax : ORACLE_QUANT_EPS;
         const float scale = 127.0f / denom;
         int64_t sum = 0;
@@ -285,5 +299,69 @@ void oracle_rmsnorm(const float *x, const float *g, int64_t m_rows, int64_t k_co
             y[m * k_cols + k] = xr * g[k];
         }
         if (r_out) r_out[m] = r;
+    }
+}
+
+/* ---- fp32 epilogue, bf16 outputs and the emitted per-token maximum ------ */
+
+/* Page, "Model details" / "Quantization": the integer product is rescaled by
+ * gamma / s.  The page fixes no output precision.  Reading, so that an output
+ * stored in fp32 or bf16 is one well-defined number:
+ *   r   = fl32(gamma / s)                 (one correctly rounded division)
+ *   y32 = fl32(acc * r)                   (acc is an integer, |acc| < 2^24,
+ *                                          so it converts to binary32 exactly)
+ * and for the gated FFN (page, "Architecture": ReLU^2 in the FFN)
+ *   h32 = fl32(fl32(p * p) * u32),  p = max(g32, 0),  g32, u32 as y32;
+ * a bf16 output is y32 (h32) rounded to the nearest bf16, ties to even. */
+void oracle_epilogue_f32(const int64_t *acc_g, const int64_t *acc_u, const float *s, float gamma_g,
+                         float gamma_u, int64_t m_rows, int64_t n_rows, float *y)
+{
+    for (int64_t m = 0; m < m_rows; ++m) {
+        const float rg = gamma_g / s[m];
+        const float ru = gamma_u / s[m];
+        for (int64_t n = 0; n < n_rows; ++n) {
+            const int64_t i = m * n_rows + n;
+            const float g = (float)acc_g[i] * rg;
+            if (!acc_u) {
+                y[i] = g;
+                continue;
+            }
+            const float u = (float)acc_u[i] * ru;
+            const float p = g > 0.0f ? g : 0.0f;
+            const float pp = p * p;
+            y[i] = pp * u;
+        }
+    }
+}
+
+/* binary32 -> bfloat16 (the upper half of the binary32 encoding), rounded to
+ * nearest with ties to even; a NaN stays a (quiet) NaN. */
+static uint16_t oracle_f32_to_bf16_one(float v)
+{
+    uint32_t bits;
+    memcpy(&bits, &v, sizeof bits);
+    if ((bits & 0x7fffffffu) > 0x7f800000u) return (uint16_t)((bits >> 16) | 0x0040u);
+    uint32_t upper = bits >> 16;
+    const uint32_t lower = bits & 0xffffu;
+    if (lower > 0x8000u || (lower == 0x8000u && (upper & 1u))) upper += 1u;
+    return (uint16_t)upper;
+}
+
+void oracle_f32_to_bf16(const float *src, int64_t count, uint16_t *dst)
+{
+    for (int64_t i = 0; i < count; ++i) dst[i] = oracle_f32_to_bf16_one(src[i]);
+}
+
+/* amax[m] = max over n of |v[m][n]|, the row maxima a BitLinear epilogue
+ * emits for the next quantiser (v: the values as stored, widened to fp32). */
+void oracle_row_absmax(const float *v, int64_t m_rows, int64_t n_rows, float *amax)
+{
+    for (int64_t m = 0; m < m_rows; ++m) {
+        float best = 0.0f;
+        for (int64_t n = 0; n < n_rows; ++n) {
+            const float a = fabsf(v[m * n_rows + n]);
+            if (a > best) best = a;
+        }
+        amax[m] = best;
     }
 }

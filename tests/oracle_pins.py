@@ -389,4 +389,187 @@ def pin_rmsnorm_sumsq_rounding_bound():
         assert np.all(np.abs(got - ms / (ms + 1e-5)) <= 1e-6)
 
 
+# --------------------------------------------------------------------------
+# Output stage: bf16 rounding, the fp32 epilogue value, emitted row maxima and
+# the quantiser fed a maximum from outside.
+# --------------------------------------------------------------------------
+def _bits_to_f32(b):
+    return np.array([b], np.uint32).view(np.float32)
+
+
+def pin_bf16_round_hand_cases():
+    """Bit patterns worked by hand: bf16 keeps the upper 16 bits of binary32;
+    the dropped half decides (above 0x8000 up, below down, exactly 0x8000 to
+    the even upper half)."""
+    cases = [
+        (0x3F800000, 0x3F80),  # 1.0 exact
+        (0x3F808000, 0x3F80),  # 1 + 2^-8: tie, upper 0x3F80 is even -> stays
+        (0x3F818000, 0x3F82),  # 1 + 3*2^-8: tie, upper 0x3F81 odd -> up
+        (0x3F808001, 0x3F81),  # just above the tie -> up
+        (0x3F807FFF, 0x3F80),  # just below the tie -> down
+        (0xBF808000, 0xBF80),  # negative tie: magnitude rounds like the positive one
+        (0xBF818000, 0xBF82),
+        (0x3F80FFFF, 0x3F81),
+        (0x7F7FFFFF, 0x7F80),  # largest finite binary32 rounds up to +inf
+        (0x00008000, 0x0000),  # subnormal tie to the even zero
+        (0x00018000, 0x0002),  # subnormal tie, odd upper -> up
+        (0x80000000, 0x8000),  # -0 keeps its sign
+        (0x7F800000, 0x7F80),  # +inf
+    ]
+    src = np.concatenate([_bits_to_f32(a) for a, _ in cases])
+    got = oracle.f32_to_bf16(src)
+    for (a, want), g in zip(cases, got.tolist()):
+        assert g == want, (hex(a), hex(g), hex(want))
+    # a NaN whose payload sits only in the dropped half must stay a NaN
+    for a in (0x7F800001, 0xFF800001, 0x7FC00000):
+        g = int(oracle.f32_to_bf16(_bits_to_f32(a))[0])
+        assert (g & 0x7F80) == 0x7F80 and (g & 0x007F) != 0, (hex(a), hex(g))
+
+
+def pin_bf16_round_vs_torch():
+    """Against torch's own binary32 -> bfloat16 conversion (round to nearest even)
+    on random finite values of every magnitude, including constructed ties."""
+    import torch
+    rng = np.random.default_rng(77)
+    bits = rng.integers(0, 2**32, 20000, dtype=np.uint64).astype(np.uint32)
+    bits = bits[(bits & 0x7F800000) != 0x7F800000]  # finite only
+    ties = (rng.integers(0, 2**16, 2000, dtype=np.uint64).astype(np.uint32) << 16) | 0x8000
+    ties = ties[(ties & 0x7F800000) != 0x7F800000]
+    v = np.concatenate([bits, ties]).view(np.float32)
+    want = torch.from_numpy(v.copy()).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = oracle.f32_to_bf16(v)
+    bad = np.nonzero(got != want)[0]
+    assert bad.size == 0, [(hex(int(v.view(np.uint32)[i])), hex(int(got[i])), hex(int(want[i]))) for i in bad[:5]]
+
+
+def pin_row_absmax_hand():
+    v = np.array([[1.0, -3.0, 2.0], [-0.5, 0.25, 0.0], [0.0, -0.0, 0.0], [-7.0, -8.0, -1.0]], np.float32)
+    assert oracle.row_absmax(v).tolist() == [3.0, 0.5, 0.0, 8.0]
+
+
+def _rne32(q):
+    """Exact rational -> nearest binary32 value (ties to even), as a Fraction.
+    Normal range only (the pins below stay far from under/overflow)."""
+    if q == 0:
+        return Fraction(0)
+    sign = -1 if q < 0 else 1
+    a = abs(q)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    while Fraction(2) ** e > a:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= a:
+        e += 1
+    # a = m * 2^(e-23) with 2^23 <= m < 2^24
+    m = a / Fraction(2) ** (e - 23)
+    lo = m.numerator // m.denominator
+    rem = m - lo
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and lo % 2 == 1):
+        lo += 1
+    return sign * Fraction(lo) * Fraction(2) ** (e - 23)
+
+
+def pin_epilogue_f32_exact_rounding():
+    """y32 = fl32(acc * fl32(gamma / s)) evaluated in exact rational arithmetic
+    with its own round-to-nearest-even, on triples where rounding gamma / s
+    first changes the result against the single rounding of the exact product
+    (so a fused or binary64 product would fail), plus the gated form
+    h32 = fl32(fl32(p * p) * u32)."""
+    triples = [(3, 0.75, 42.33333206176758), (3, 0.75, 181.42857360839844),
+               (7, 0.75, 42.33333206176758), (100, 0.75, 181.42857360839844),
+               (12345, 0.75, 42.33333206176758), (-12345, 0.75, 42.33333206176758),
+               (1, 0.5, 127.0), (0, 0.8, 3.0)]
+    acc = np.array([[t[0] for t in triples]], np.int64)
+    for gam in sorted({t[1] for t in triples}):
+        for s in sorted({t[2] for t in triples}):
+            s32 = np.float32(s)
+            y = oracle.epilogue_f32(acc, np.array([s32], np.float32), np.float32(gam))[0]
+            r = _rne32(Fraction(float(np.float32(gam))) / Fraction(float(s32)))
+            for a, got in zip(acc[0].tolist(), y.tolist()):
+                want = _rne32(a * r)
+                assert Fraction(got) == want, (a, gam, s, got, float(want))
+    # at least one triple separates the two-rounding value from the exact product's
+    s32 = np.float32(42.33333206176758)
+    r = _rne32(Fraction(0.75) / Fraction(float(s32)))
+    assert _rne32(3 * r) != _rne32(3 * Fraction(0.75) / Fraction(float(s32)))
+    # gated: acc_g, acc_u pairs, signs of both
+    ag = np.array([[5, -5, 17, 100, 0, 33]], np.int64)
+    au = np.array([[7, 7, -9, 3, 4, -1]], np.int64)
+    sg, gg, gu = np.float32(42.33333206176758), np.float32(0.75), np.float32(0.3)
+    h = oracle.epilogue_f32(ag, np.array([sg], np.float32), gg, au, gu)[0]
+    rg = _rne32(Fraction(float(gg)) / Fraction(float(sg)))
+    ru = _rne32(Fraction(float(gu)) / Fraction(float(sg)))
+    for a, b, got in zip(ag[0].tolist(), au[0].tolist(), h.tolist()):
+        g32 = _rne32(a * rg)
+        u32 = _rne32(b * ru)
+        p = g32 if g32 > 0 else Fraction(0)
+        want = _rne32(_rne32(p * p) * u32)
+        assert Fraction(got) == want, (a, b, got, float(want))
+
+
+def pin_epilogue_f32_error_bound():
+    """fp32 epilogue within its rounding bound of the binary64 forward: two
+    roundings (2u) for y, eight (8u) for the gated h, u = 2^-24."""
+    rng = np.random.default_rng(91)
+    m, n, k = 5, 40, 512
+    acc_g = rng.integers(-127 * k // 4, 127 * k // 4, (m, n)).astype(np.int64)
+    acc_u = rng.integers(-127 * k // 4, 127 * k // 4, (m, n)).astype(np.int64)
+    s = (127.0 / rng.uniform(0.01, 30.0, m)).astype(np.float32)
+    gg, gu = np.float32(0.0213), np.float32(0.0377)
+    u = 2.0 ** -24
+    y = oracle.epilogue_f32(acc_g, s, gg).astype(np.float64)
+    y64 = oracle.dequant(acc_g, s, gg)
+    assert np.all(np.abs(y - y64) <= 2.0001 * u * np.abs(y64))
+    h = oracle.epilogue_f32(acc_g, s, gg, acc_u, gu).astype(np.float64)
+    h64 = oracle.relu2_gate(y64, oracle.dequant(acc_u, s, gu))
+    assert np.all(np.abs(h - h64) <= 8.001 * u * np.abs(h64))
+    assert np.all(h[acc_g <= 0] == 0)
+
+
+def pin_quant_given_amax():
+    """The quantiser with a supplied maximum: the true maximum changes nothing;
+    a larger one A gives the codes of the same row with one more element equal
+    to A (whose own code is 127)."""
+    rng = np.random.default_rng(93)
+    x = rng.standard_normal((6, 96)).astype(np.float32)
+    x[2] *= 1e-7  # below the 1e-5 floor
+    x[3, 5] = 41.0
+    true_max = np.abs(x).max(axis=1).astype(np.float32)
+    q0, s0, r0 = oracle.quant_act(x)
+    q1, s1, r1 = oracle.quant_act(x, true_max)
+    assert np.array_equal(q0, q1) and np.array_equal(s0, s1) and np.array_equal(r0, r1)
+    big = (true_max * np.float32(3.5) + np.float32(0.25)).astype(np.float32)
+    qa, sa, ra = oracle.quant_act(x, big)
+    qb, sb, rb = oracle.quant_act(np.concatenate([x, big[:, None]], axis=1))
+    assert np.array_equal(qa, qb[:, :-1]) and np.array_equal(sa, sb)
+    assert np.array_equal(ra.astype(np.int64), rb.astype(np.int64) - qb[:, -1]) and np.all(qb[:, -1] == 127)
+
+
+def pin_bitlinear_ex_output_forms():
+    """bf16 output = the bf16 rounding of the fp32 output; the emitted maxima
+    are the maxima of the stored values; chaining through the emitted maximum
+    equals recomputing it."""
+    rng = np.random.default_rng(95)
+    k, n, m = 128, 32, 4
+    w = synth.latent_weights(n, k, 5)
+    packed, g, _ = oracle.pack_weights(w)
+    wu = synth.latent_weights(n, k, 6)
+    packed_u, gu_, _ = oracle.pack_weights(wu)
+    x = rng.standard_normal((m, k)).astype(np.float32)
+    y32, a32 = oracle.bitlinear_ex(x, packed, g, k, "f32")
+    yb, ab = oracle.bitlinear_ex(x, packed, g, k, "bf16")
+    assert np.array_equal(yb, oracle.f32_to_bf16(y32))
+    widened = (yb.astype(np.uint32) << 16).view(np.float32)
+    assert np.array_equal(ab, np.abs(widened).max(axis=1)) and np.array_equal(a32, np.abs(y32).max(axis=1))
+    y64 = oracle.bitlinear(x, packed, g, k)[0]
+    assert np.all(np.abs(y32 - y64) <= 2.0001 * 2.0 ** -24 * np.abs(y64))
+    h32, _ = oracle.bitlinear_ex(x, packed, g, k, "f32", packed_u=packed_u, gamma_u=gu_)
+    h64 = oracle.ffn_gate_up(x, packed, g, packed_u, gu_, k)[0]
+    assert np.all(np.abs(h32 - h64) <= 8.001 * 2.0 ** -24 * np.abs(h64))
+    # next layer: quantising y through the emitted maximum
+    p2, g2, _ = oracle.pack_weights(np.ascontiguousarray(synth.latent_weights(16, n, 8)))
+    z_a, _ = oracle.bitlinear_ex(widened, p2, g2, n, "f32", x_amax=ab)
+    z_b, _ = oracle.bitlinear_ex(widened, p2, g2, n, "f32")
+    assert np.array_equal(z_a, z_b)
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

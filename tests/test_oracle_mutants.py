@@ -53,6 +53,20 @@ MUTANTS = {
     "sumsq_stride_255": ("for (int64_t k = t; k < k_cols; k += 256)", "for (int64_t k = t; k < k_cols; k += 255)"),
     "sumsq_abs": ("acc += (double)row[k] * (double)row[k];", "acc += fabs((double)row[k]);"),
     "pairing_drops_last_group": ("return oracle_pairing_sum(group, 8);", "return oracle_pairing_sum(group, 4);"),
+    "bf16_truncate": ("if (lower > 0x8000u || (lower == 0x8000u && (upper & 1u))) upper += 1u;", ""),
+    "bf16_ties_away": ("if (lower > 0x8000u || (lower == 0x8000u && (upper & 1u))) upper += 1u;",
+                       "if (lower >= 0x8000u) upper += 1u;"),
+    "bf16_ties_odd": ("(lower == 0x8000u && (upper & 1u))", "(lower == 0x8000u && !(upper & 1u))"),
+    "bf16_nan_unquieted": ("if ((bits & 0x7fffffffu) > 0x7f800000u) return (uint16_t)((bits >> 16) | 0x0040u);", ""),
+    "epi_scale_inverted": ("const float rg = gamma_g / s[m];", "const float rg = s[m] / gamma_g;"),
+    "epi_binary64_product": ("const float g = (float)acc_g[i] * rg;",
+                             "const float g = (float)((double)acc_g[i] * (double)gamma_g / (double)s[m]);"),
+    "epi_relu_dropped": ("const float p = g > 0.0f ? g : 0.0f;", "const float p = g;"),
+    "epi_up_uses_gate_gamma": ("const float ru = gamma_u / s[m];", "const float ru = gamma_g / s[m];"),
+    "epi_not_squared": ("const float pp = p * p;", "const float pp = p;"),
+    "absmax_signed": ("const float a = fabsf(v[m * n_rows + n]);", "const float a = v[m * n_rows + n];"),
+    "absmax_first_column": ("const float a = fabsf(v[m * n_rows + n]);", "const float a = fabsf(v[m * n_rows]);"),
+    "given_amax_ignored": ("if (amax_in) amax = amax_in[m];", ""),
 }
 
 
