@@ -257,6 +257,14 @@ class Stack:
         self.q_buf = torch.empty((M, HIDDEN), dtype=torch.int8, device=device)
         self.s_buf = torch.empty(M, dtype=torch.float32, device=device)
         self.rs_buf = torch.empty(M, dtype=torch.int32, device=device)
+        # bf16 gate/up -> down chain through the emitted per-token maxima of h
+        bf = torch.bfloat16
+        self.pre_hb = torch.empty((M, INTER), dtype=bf, device=device)
+        self.pre_db = torch.empty((M, HIDDEN), dtype=bf, device=device)
+        self.pre_ha = torch.empty(M, dtype=f32, device=device)
+        self.dec_hb = torch.empty((B, INTER), dtype=bf, device=device)
+        self.dec_db = torch.empty((B, HIDDEN), dtype=bf, device=device)
+        self.dec_ha = torch.empty(B, dtype=f32, device=device)
         self.seq_ops = {}
         self.packed_bytes = sum(p.numel() for L in self.layers for (p, _) in L.values())
 
@@ -277,6 +285,13 @@ class Stack:
     def down(self, l, out, ws, s):
         L = self.layers[l]
         self.tw.bitnet_linear(out["h"], L["down"][0], L["down"][1], y=out["down"], workspace=ws, stream=s)
+
+    def ffn_bf16_chain(self, l, x, hb, ha, db, ws, s):
+        """gate/up with bf16 h and its emitted maxima, then down fed those maxima."""
+        L, tw = self.layers[l], self.tw
+        tw.bitnet_ffn_gate_up_ex(x, L["gate"][0], L["gate"][1], L["up"][0], L["up"][1], h=hb, h_amax=ha,
+                                 workspace=ws, stream=s)
+        tw.bitnet_linear_ex(hb, L["down"][0], L["down"][1], x_amax=ha, y=db, workspace=ws, stream=s)
 
     def prefill_pass(self, s):
         for l in range(self.a.layers):
@@ -538,6 +553,17 @@ def our_arm(a, n_gpus):
                                                                          s=st.s_buf, rowsum=st.rs_buf, stream=s)
                                                  for l in range(Lyr)],
                                       M * HIDDEN * 2 + HIDDEN * 4 + M * HIDDEN + 8 * M, "hbm", 0, Lyr, False),
+            # bf16 h with emitted maxima -> down fed them, against prefill_gate_up + prefill_down
+            # (not in the step: the step stores fp32 outputs)
+            "prefill_ffn_bf16_chain": (lambda s: [st.ffn_bf16_chain(l, st.pre_x[l % st.n_pre], st.pre_hb, st.pre_ha,
+                                                                    st.pre_db, st.ws_pre, s) for l in range(Lyr)],
+                                       2 * 2 * M * HIDDEN * INTER + 2 * M * INTER * HIDDEN, "tensor", 0, Lyr,
+                                       False),
+            "decode_ffn_bf16_chain": (lambda s: [st.ffn_bf16_chain(l, st.dec_x[l % st.n_dec], st.dec_hb, st.dec_ha,
+                                                                   st.dec_db, st.ws_dec, s)
+                                                 for _ in range(R) for l in range(Lyr)],
+                                      3 * INTER * HIDDEN // 4 + B * HIDDEN * 2 + 2 * B * INTER * 2 + B * HIDDEN * 2,
+                                      "hbm", 0, R * Lyr, False),
         }
         for name, (fn, work, bound, per_step, n_ops, in_step) in specs.items():
             if name == "decode_sequence" and not seq:

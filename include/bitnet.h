@@ -252,6 +252,52 @@ bitnet_status_t bitnet_ffn_gate_up_norm(const void *x, bitnet_dtype_t x_dtype, i
                                         float *h, int32_t *acc_g_out, int32_t *acc_u_out,
                                         void *workspace, size_t ws_bytes, cudaStream_t stream);
 
+/* ---- output options: bf16 outputs, emitted and given per-token maxima ---- */
+
+/*
+ * bitnet_linear / bitnet_ffn_gate_up with options for chaining BitLinears
+ * (page: "Quantization" -- every BitLinear quantises its input per token by
+ * absmax, so the maximum of each output row is what the next BitLinear's
+ * quantiser needs first).
+ *
+ *   x, x_dtype, M, K, weights, N, workspace, stream: as bitnet_linear /
+ *              bitnet_ffn_gate_up
+ *   x_amax     [M] fp32 (device, read; may be NULL): max_k |x[m][k]| given by
+ *              the caller, typically the y_amax of the BitLinear that wrote x.
+ *              The quantiser uses it instead of reducing the row (and the
+ *              decode kernel skips the exchange of partial maxima between the
+ *              CTAs of a cluster); the result is identical when it is the
+ *              true maximum.  Not allowed together with norm_g (the maxima of
+ *              x are not those of RMSNorm(x)): BITNET_ERR_INVALID_ARG.
+ *   norm_g, norm_eps  optional RMS normalisation in front of the quantiser, as
+ *              bitnet_linear_norm (norm_g NULL: none)
+ *   y (h)      [M][N] output of type y_dtype (h_dtype): BITNET_DTYPE_F32, or
+ *              BITNET_DTYPE_BF16 = the fp32 value rounded to the nearest bf16,
+ *              ties to even.  The fp32 value is fl(acc * fl(gamma / s)) (and
+ *              fl(fl(p * p) * u), p = max(g, 0), for the gated FFN), exactly
+ *              as bitnet_linear / bitnet_ffn_gate_up store it.
+ *   y_amax     [M] fp32 (device, written; may be NULL): max_n |y[m][n]| of the
+ *              values as stored (after bf16 rounding), folded in by the
+ *              epilogues with integer atomicMax on the bit patterns (exact and
+ *              order-independent).  The library zeroes it first (inside the
+ *              quantiser kernel, or with one small kernel ahead of the fused
+ *              decode kernel).  Must not overlap x_amax (BITNET_ERR_INVALID_ARG).
+ *
+ * All pointers 16-byte aligned.  A bf16 y whose rows are not 16-byte
+ * multiples (N % 8 != 0) is written with plain stores instead of tensor
+ * stores.
+ */
+bitnet_status_t bitnet_linear_ex(const void *x, bitnet_dtype_t x_dtype, const float *x_amax, const float *norm_g,
+                                 float norm_eps, int64_t M, int64_t K, const uint8_t *w_packed, const float *gamma,
+                                 int64_t N, void *y, bitnet_dtype_t y_dtype, float *y_amax, void *workspace,
+                                 size_t ws_bytes, cudaStream_t stream);
+
+bitnet_status_t bitnet_ffn_gate_up_ex(const void *x, bitnet_dtype_t x_dtype, const float *x_amax,
+                                      const float *norm_g, float norm_eps, int64_t M, int64_t K,
+                                      const uint8_t *wg_packed, const float *gamma_g, const uint8_t *wu_packed,
+                                      const float *gamma_u, int64_t N, void *h, bitnet_dtype_t h_dtype,
+                                      float *h_amax, void *workspace, size_t ws_bytes, cudaStream_t stream);
+
 /* ---- decode sequences: many small-M ops in one persistent launch ---------- */
 
 typedef enum {

@@ -89,6 +89,8 @@ def load_library(path: str = LIB_PATH):
         "bitnet_sequence_schedule": ([ctypes.POINTER(bitnet_op_t), ctypes.c_int32, I64,
                                       ctypes.POINTER(ctypes.c_int32)], I),
         "bitnet_set_sequence_cluster": ([I], I),
+        "bitnet_linear_ex": ([P, I, P, P, F, I64, I64, P, P, I64, P, I, P, P, SZ, P], I),
+        "bitnet_ffn_gate_up_ex": ([P, I, P, P, F, I64, I64, P, P, P, P, I64, P, I, P, P, SZ, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -280,6 +282,44 @@ def bitnet_ffn_gate_up_norm(x, g, wg_packed, gamma_g, wu_packed, gamma_u, eps=RM
                                        _ptr(gamma_g), _ptr(wu_packed), _ptr(gamma_u), n, _ptr(h), _ptr(acc_g_out),
                                        _ptr(acc_u_out), _ptr(workspace), workspace.numel(), _stream(stream)),
            "bitnet_ffn_gate_up_norm")
+    return h
+
+
+def _out(y, m, n, y_dtype, device):
+    if y is None:
+        y = torch.empty((m, n), dtype=y_dtype, device=device)
+    return y, _dtype_code(y)
+
+
+def bitnet_linear_ex(x, w_packed, gamma, *, x_amax=None, norm_g=None, eps=RMS_EPS, y=None,
+                     y_dtype=torch.float32, y_amax=None, workspace=None, stream=None):
+    """y [M][N] (fp32 or bf16) = BitLinear(x), optionally RMS-normalised first
+    (norm_g), with the per-token maxima of x given (x_amax [M]) and/or those of
+    y emitted into y_amax [M] fp32.  Returns y."""
+    lib = load_library()
+    m, k = x.shape
+    n = w_packed.shape[0]
+    y, yc = _out(y, m, n, y_dtype, x.device)
+    workspace = _workspace(workspace, m, n, k, x.device)
+    _check(lib.bitnet_linear_ex(_ptr(x), _dtype_code(x), _ptr(x_amax), _ptr(norm_g), float(eps), m, k,
+                                _ptr(w_packed), _ptr(gamma), n, _ptr(y), yc, _ptr(y_amax), _ptr(workspace),
+                                workspace.numel(), _stream(stream)), "bitnet_linear_ex")
+    return y
+
+
+def bitnet_ffn_gate_up_ex(x, wg_packed, gamma_g, wu_packed, gamma_u, *, x_amax=None, norm_g=None, eps=RMS_EPS,
+                          h=None, h_dtype=torch.float32, h_amax=None, workspace=None, stream=None):
+    """h [M][N] (fp32 or bf16) = relu(BitLinear_g(x))^2 * BitLinear_u(x) with the
+    options of bitnet_linear_ex.  Returns h."""
+    lib = load_library()
+    m, k = x.shape
+    n = wg_packed.shape[0]
+    h, hc = _out(h, m, n, h_dtype, x.device)
+    workspace = _workspace(workspace, m, n, k, x.device)
+    _check(lib.bitnet_ffn_gate_up_ex(_ptr(x), _dtype_code(x), _ptr(x_amax), _ptr(norm_g), float(eps), m, k,
+                                     _ptr(wg_packed), _ptr(gamma_g), _ptr(wu_packed), _ptr(gamma_u), n, _ptr(h), hc,
+                                     _ptr(h_amax), _ptr(workspace), workspace.numel(), _stream(stream)),
+           "bitnet_ffn_gate_up_ex")
     return h
 
 

@@ -156,18 +156,20 @@ bool encode_u8_2d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t co
     return r == CUDA_SUCCESS;
 }
 
-// 2-D fp32 tensor [rows][cols] (row pitch = cols * 4 bytes), box [box_rows][box_cols], 128-byte swizzle.
-bool encode_f32_2d_sw128(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows,
-                         uint32_t box_cols)
+// 2-D output tensor [rows][cols] of fp32 (128-byte swizzle) or bf16 (64-byte
+// swizzle), box [box_rows][box_cols]: the box rows are exactly one swizzle span.
+bool encode_2d_out(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows,
+                   uint32_t box_cols, bool bf16)
 {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols * 4};
+    cuuint64_t strides[1] = {cols * (bf16 ? 2 : 4)};
     cuuint32_t box[2] = {box_cols, box_rows};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void *>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+    CUresult r = fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+                    const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    bf16 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -232,25 +234,29 @@ cudaError_t launch_decode(const DecodeArgs &a, const DecodeCfg &c, cudaStream_t 
 }
 
 // Per-token quantiser: rows held in registers (one HBM read) when a row fits
-// in 8 warps x 32 lanes x QR_NCH chunks, otherwise the two-pass kernel.
+// in 8 warps x 32 lanes x QR_NCH chunks, otherwise the two-pass kernel (one
+// pass when the row maxima are given).  amax_in: optional given row maxima;
+// amax_zero: optional [M] zeroed for the next kernel's atomicMax.
 template <bool XF32>
 cudaError_t launch_quant_t(const void *x, int64_t M, int64_t K, int8_t *xq, float *s, int32_t *rs,
-                           cudaStream_t stream)
+                           const float *amax_in, float *amax_zero, cudaStream_t stream)
 {
     const int64_t nch = K / (XF32 ? 4 : 8);
     const int64_t per_warp = 32 * QR_NCH;
     if (nch <= per_warp)
         return launch_pdl(k_quant_rows_reg<XF32, 1>, dim3((unsigned)cdiv(M, 8)), dim3(256), 0, stream, x, M, K, xq,
-                          s, rs);
+                          s, rs, amax_in, amax_zero);
     if (nch <= 2 * per_warp)
         return launch_pdl(k_quant_rows_reg<XF32, 2>, dim3((unsigned)cdiv(M, 4)), dim3(256), 0, stream, x, M, K, xq,
-                          s, rs);
+                          s, rs, amax_in, amax_zero);
     if (nch <= 4 * per_warp)
         return launch_pdl(k_quant_rows_reg<XF32, 4>, dim3((unsigned)cdiv(M, 2)), dim3(256), 0, stream, x, M, K, xq,
-                          s, rs);
+                          s, rs, amax_in, amax_zero);
     if (nch <= 8 * per_warp)
-        return launch_pdl(k_quant_rows_reg<XF32, 8>, dim3((unsigned)M), dim3(256), 0, stream, x, M, K, xq, s, rs);
-    return launch_pdl(k_quant_rows<XF32>, dim3((unsigned)cdiv(M, 8)), dim3(256), 0, stream, x, M, K, xq, s, rs);
+        return launch_pdl(k_quant_rows_reg<XF32, 8>, dim3((unsigned)M), dim3(256), 0, stream, x, M, K, xq, s, rs,
+                          amax_in, amax_zero);
+    return launch_pdl(k_quant_rows<XF32>, dim3((unsigned)cdiv(M, 8)), dim3(256), 0, stream, x, M, K, xq, s, rs,
+                      amax_in, amax_zero);
 }
 
 // RMS normalisation + quantiser: rows of up to 4096 elements on 128 threads (two rows
@@ -259,26 +265,27 @@ constexpr int64_t kNormMaxK = 256 * RQ_MAX_PER_THREAD;
 
 template <bool XF32>
 cudaError_t launch_norm_quant_t(const void *x, int64_t M, int64_t K, const float *g, float eps, int8_t *xq, float *s,
-                                int32_t *rs, cudaStream_t stream)
+                                int32_t *rs, float *amax_zero, cudaStream_t stream)
 {
     if (K <= 128 * RQ_MAX_PER_THREAD)
         return launch_pdl(k_rmsnorm_quant_rows<XF32, 128>, dim3((unsigned)cdiv(M, 2)), dim3(256), 0, stream, x, M, K,
-                          g, eps, xq, s, rs);
+                          g, eps, xq, s, rs, amax_zero);
     return launch_pdl(k_rmsnorm_quant_rows<XF32, 256>, dim3((unsigned)M), dim3(256), 0, stream, x, M, K, g, eps, xq, s,
-                      rs);
+                      rs, amax_zero);
 }
 
 cudaError_t launch_norm_quant(const void *x, bool xf32, int64_t M, int64_t K, const float *g, float eps, int8_t *xq,
-                              float *s, int32_t *rs, cudaStream_t stream)
+                              float *s, int32_t *rs, cudaStream_t stream, float *amax_zero = nullptr)
 {
-    return xf32 ? launch_norm_quant_t<true>(x, M, K, g, eps, xq, s, rs, stream)
-                : launch_norm_quant_t<false>(x, M, K, g, eps, xq, s, rs, stream);
+    return xf32 ? launch_norm_quant_t<true>(x, M, K, g, eps, xq, s, rs, amax_zero, stream)
+                : launch_norm_quant_t<false>(x, M, K, g, eps, xq, s, rs, amax_zero, stream);
 }
 
 cudaError_t launch_quant(const void *x, bool xf32, int64_t M, int64_t K, int8_t *xq, float *s, int32_t *rs,
-                         cudaStream_t stream)
+                         cudaStream_t stream, const float *amax_in = nullptr, float *amax_zero = nullptr)
 {
-    return xf32 ? launch_quant_t<true>(x, M, K, xq, s, rs, stream) : launch_quant_t<false>(x, M, K, xq, s, rs, stream);
+    return xf32 ? launch_quant_t<true>(x, M, K, xq, s, rs, amax_in, amax_zero, stream)
+                : launch_quant_t<false>(x, M, K, xq, s, rs, amax_in, amax_zero, stream);
 }
 
 // ---- cluster (K-split, fused quantiser) decode kernel -------------------------
@@ -453,16 +460,28 @@ cudaError_t dc_launch(const DcCfg &c, const DcArgs &a, cudaStream_t stream)
     }
 }
 
+// Input and output options of the BitLinear entry points (the plain entry
+// points use the defaults): x_amax = given per-token maxima of x; y_bf16 =
+// store y as bf16; y_amax = emit the per-token maxima of y.
+struct IoOpts {
+    const float *x_amax = nullptr;
+    bool y_bf16 = false;
+    float *y_amax = nullptr;
+};
+
 bitnet_status_t dc_forward(const DcCfg &c, const void *x, bool xf32, int64_t M, int64_t K, const uint8_t *w0,
-                           const float *gamma0, const uint8_t *w1, const float *gamma1, int64_t N, float *y,
+                           const float *gamma0, const uint8_t *w1, const float *gamma1, int64_t N, void *y,
                            int8_t *x_q_out, float *s_out, int32_t *acc0, int32_t *acc1, cudaStream_t stream,
-                           int nmat)
+                           int nmat, const IoOpts &io)
 {
     DcArgs a = c.a;
     a.x = x;
+    a.x_amax = io.x_amax;
     a.gamma0 = gamma0;
     a.gamma1 = gamma1;
     a.y = y;
+    a.y_bf16 = io.y_bf16 ? 1 : 0;
+    a.y_amax = io.y_amax;
     a.acc0 = acc0;
     a.acc1 = acc1;
     a.xq_out = x_q_out;
@@ -472,7 +491,10 @@ bitnet_status_t dc_forward(const DcCfg &c, const void *x, bool xf32, int64_t M, 
     a.K = (int)K;
     a.w0 = w0;
     a.w1 = w1;
-    cudaError_t e;
+    cudaError_t e = cudaSuccess;
+    // the maxima are folded in with atomicMax by every cluster: zero them first
+    if (io.y_amax) e = launch_pdl(k_zero_f32, dim3(1), dim3(128), 0, stream, io.y_amax, (int)M);
+    if (e != cudaSuccess) return cuda_status(e);
     if (nmat == 1)
         e = xf32 ? dc_launch<1, true>(c, a, stream) : dc_launch<1, false>(c, a, stream);
     else
@@ -480,14 +502,15 @@ bitnet_status_t dc_forward(const DcCfg &c, const void *x, bool xf32, int64_t M, 
     return cuda_status(e);
 }
 
-// Shared body of bitnet_linear (nmat = 1) and bitnet_ffn_gate_up (nmat = 2).
-// Shared body of the BitLinear entry points.  norm_g (optional): RMS-normalise
-// x with weight norm_g and epsilon norm_eps before quantising it.
+// Shared body of the BitLinear entry points (nmat = 1: BitLinear, 2: gated
+// FFN gate/up).  norm_g (optional): RMS-normalise x with weight norm_g and
+// epsilon norm_eps before quantising it.  io: given maxima of x, bf16 output,
+// emitted maxima of y.
 bitnet_status_t forward(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_t K, const uint8_t *w0,
-                        const float *gamma0, const uint8_t *w1, const float *gamma1, int64_t N, float *y,
+                        const float *gamma0, const uint8_t *w1, const float *gamma1, int64_t N, void *y,
                         int8_t *x_q_out, float *s_out, int32_t *acc0, int32_t *acc1, void *workspace,
                         size_t ws_bytes, cudaStream_t stream, int nmat, const float *norm_g = nullptr,
-                        float norm_eps = 0.0f)
+                        float norm_eps = 0.0f, const IoOpts &io = IoOpts())
 {
     bitnet_status_t st = check_shape(M, N, K);
     if (st != BITNET_OK) return st;
@@ -495,7 +518,17 @@ bitnet_status_t forward(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_
     if (!x || !w0 || !gamma0 || !y || (nmat == 2 && (!w1 || !gamma1))) return BITNET_ERR_INVALID_ARG;
     if (norm_g && (K > kNormMaxK || !(norm_eps >= 0.0f) || !std::isfinite(norm_eps)))
         return norm_g && K > kNormMaxK ? BITNET_ERR_UNSUPPORTED_SHAPE : BITNET_ERR_INVALID_ARG;
-    const void *ptrs[] = {x, w0, gamma0, w1, gamma1, y, x_q_out, s_out, acc0, acc1, workspace, norm_g};
+    // the maxima of the raw input are not those of its normalised form; the
+    // given and the emitted maxima must not share memory (one is read while
+    // the other is zeroed and folded)
+    if (io.x_amax && norm_g) return BITNET_ERR_INVALID_ARG;
+    if (io.x_amax && io.y_amax) {
+        const uintptr_t a0 = reinterpret_cast<uintptr_t>(io.x_amax), b0 = reinterpret_cast<uintptr_t>(io.y_amax);
+        const uintptr_t bytes = (uintptr_t)M * 4;
+        if (a0 < b0 + bytes && b0 < a0 + bytes) return BITNET_ERR_INVALID_ARG;
+    }
+    const void *ptrs[] = {x, w0, gamma0, w1, gamma1, y, x_q_out, s_out, acc0, acc1, workspace, norm_g,
+                          io.x_amax, io.y_amax};
     for (const void *p : ptrs)
         if (p && !aligned16(p)) return BITNET_ERR_MISALIGNED;
     if (!workspace || ws_bytes < ws_bytes_for(M, K)) return BITNET_ERR_WORKSPACE;
@@ -509,9 +542,10 @@ bitnet_status_t forward(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_
     float *s = s_out ? s_out : ws.s;
 
     // the normalising quantiser runs as its own kernel ahead of the GEMM
+    // and zeroes the emitted maxima for the contraction kernel's epilogue
     auto quantise = [&](int8_t *q, float *sc, int32_t *rs) {
-        return norm_g ? launch_norm_quant(x, xf32, M, K, norm_g, norm_eps, q, sc, rs, stream)
-                      : launch_quant(x, xf32, M, K, q, sc, rs, stream);
+        return norm_g ? launch_norm_quant(x, xf32, M, K, norm_g, norm_eps, q, sc, rs, stream, io.y_amax)
+                      : launch_quant(x, xf32, M, K, q, sc, rs, stream, io.x_amax, io.y_amax);
     };
     if (M <= kDecodeMaxM && dispatch != BITNET_DISPATCH_PREFILL) {
         // cluster kernel with the quantiser fused in (automatic choice for decode)
@@ -519,7 +553,7 @@ bitnet_status_t forward(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_
             const DcCfg c = dc_config(N, K, nmat, xf32, M <= 8, dev, sms);
             if (c.ok)
                 return dc_forward(c, x, xf32, M, K, w0, gamma0, w1, gamma1, N, y, x_q_out, s_out, acc0, acc1,
-                                  stream, nmat);
+                                  stream, nmat, io);
             if (dispatch == BITNET_DISPATCH_DECODE_FUSED) return BITNET_ERR_UNSUPPORTED_SHAPE;
         }
         if (norm_g && dispatch == BITNET_DISPATCH_DECODE_FUSED) return BITNET_ERR_UNSUPPORTED_SHAPE;
@@ -535,6 +569,8 @@ bitnet_status_t forward(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_
             a.gamma0 = gamma0;
             a.gamma1 = gamma1;
             a.y = y;
+            a.y_bf16 = io.y_bf16 ? 1 : 0;
+            a.y_amax = io.y_amax;
             a.acc0 = acc0;
             a.acc1 = acc1;
             a.M = (int)M;
@@ -567,9 +603,11 @@ bitnet_status_t forward(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_
     a.gamma1 = gamma1;
     a.s = s;
     a.y = y;
+    a.y_bf16 = io.y_bf16 ? 1 : 0;
+    a.y_amax = io.y_amax;
     a.acc0 = acc0;
     a.acc1 = acc1;
-    a.vec_ok = (N % 4) == 0;
+    a.vec_ok = (N % (io.y_bf16 ? 8 : 4)) == 0; // 16-byte rows
     CUtensorMap tmA, tmB0, tmB1, tmY;
     const uint32_t brows = nmat == 1 ? PF_BN : PF_BN / 2;
     if (!encode_u8_2d(&tmA, xq, (uint64_t)M, (uint64_t)K, PF_BM, PF_BK, true) ||
@@ -581,9 +619,10 @@ bitnet_status_t forward(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_
     } else {
         tmB1 = tmB0;
     }
-    // fp32 output through TMA stores (32 x 32 boxes, 128-byte swizzle) when rows are 16-byte multiples
+    // output through TMA stores when rows are 16-byte multiples: 32 x 32 boxes,
+    // 128-byte swizzle for fp32, 64-byte swizzle for bf16
     tmY = tmA;
-    if (a.vec_ok && !encode_f32_2d_sw128(&tmY, y, (uint64_t)M, (uint64_t)N, 32, 32)) return BITNET_ERR_CUDA;
+    if (a.vec_ok && !encode_2d_out(&tmY, y, (uint64_t)M, (uint64_t)N, 32, 32, io.y_bf16)) return BITNET_ERR_CUDA;
     cudaError_t e = quantise(xq, s, nullptr);
     if (e != cudaSuccess) return BITNET_ERR_CUDA;
     const int grid = std::min(a.num_tiles, sms);
@@ -1139,6 +1178,35 @@ bitnet_status_t bitnet_ffn_gate_up_norm(const void *x, bitnet_dtype_t x_dtype, i
     if (!g) return BITNET_ERR_INVALID_ARG;
     return forward(x, x_dtype, M, K, wg_packed, gamma_g, wu_packed, gamma_u, N, h, nullptr, nullptr, acc_g_out,
                    acc_u_out, workspace, ws_bytes, stream, 2, g, eps);
+}
+
+bitnet_status_t bitnet_linear_ex(const void *x, bitnet_dtype_t x_dtype, const float *x_amax, const float *norm_g,
+                                 float norm_eps, int64_t M, int64_t K, const uint8_t *w_packed, const float *gamma,
+                                 int64_t N, void *y, bitnet_dtype_t y_dtype, float *y_amax, void *workspace,
+                                 size_t ws_bytes, cudaStream_t stream)
+{
+    if (y_dtype != BITNET_DTYPE_BF16 && y_dtype != BITNET_DTYPE_F32) return BITNET_ERR_INVALID_ARG;
+    IoOpts io;
+    io.x_amax = x_amax;
+    io.y_bf16 = y_dtype == BITNET_DTYPE_BF16;
+    io.y_amax = y_amax;
+    return forward(x, x_dtype, M, K, w_packed, gamma, nullptr, nullptr, N, y, nullptr, nullptr, nullptr, nullptr,
+                   workspace, ws_bytes, stream, 1, norm_g, norm_eps, io);
+}
+
+bitnet_status_t bitnet_ffn_gate_up_ex(const void *x, bitnet_dtype_t x_dtype, const float *x_amax,
+                                      const float *norm_g, float norm_eps, int64_t M, int64_t K,
+                                      const uint8_t *wg_packed, const float *gamma_g, const uint8_t *wu_packed,
+                                      const float *gamma_u, int64_t N, void *h, bitnet_dtype_t h_dtype,
+                                      float *h_amax, void *workspace, size_t ws_bytes, cudaStream_t stream)
+{
+    if (h_dtype != BITNET_DTYPE_BF16 && h_dtype != BITNET_DTYPE_F32) return BITNET_ERR_INVALID_ARG;
+    IoOpts io;
+    io.x_amax = x_amax;
+    io.y_bf16 = h_dtype == BITNET_DTYPE_BF16;
+    io.y_amax = h_amax;
+    return forward(x, x_dtype, M, K, wg_packed, gamma_g, wu_packed, gamma_u, N, h, nullptr, nullptr, nullptr,
+                   nullptr, workspace, ws_bytes, stream, 2, norm_g, norm_eps, io);
 }
 
 bitnet_status_t bitnet_device_status(int clear, bitnet_status_t *status_out, cudaStream_t stream)

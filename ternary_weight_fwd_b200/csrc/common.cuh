@@ -298,6 +298,39 @@ BITNET_DEVINL uint32_t pack4_s8(int a, int b, int c, int d)
 BITNET_DEVINL float bf16_bits_lo(uint32_t w) { return __uint_as_float(w << 16); }
 BITNET_DEVINL float bf16_bits_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
+// ---- output stage: fp32, or bf16 = the fp32 value rounded to nearest even ----
+
+BITNET_DEVINL uint32_t bf16_rn_bits(float v) { return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v)); }
+
+// Magnitude of the value as stored, as the bit pattern of a non-negative fp32
+// (non-negative floats order like their bit patterns, so maxima are integer
+// maxima and atomicMax on the bits is exact and order-free).
+BITNET_DEVINL uint32_t out_mag_bits(float v, bool bf16)
+{
+    return bf16 ? (bf16_rn_bits(v) & 0x7fffu) << 16 : __float_as_uint(v) & 0x7fffffffu;
+}
+
+BITNET_DEVINL void out_store(void *y, size_t o, float v, bool bf16)
+{
+    if (bf16)
+        static_cast<uint16_t *>(y)[o] = (uint16_t)bf16_rn_bits(v);
+    else
+        static_cast<float *>(y)[o] = v;
+}
+
+// Fold each lane's magnitude bits into per-token maxima (shared memory, bits
+// of non-negative floats).  Lanes hold consecutive elements of an epilogue
+// whose token index j does not decrease from lane to lane; a lane without an
+// element passes bits 0 and a j no smaller than any active lane's.
+BITNET_DEVINL void warp_token_max(uint32_t bits, int j, unsigned *smax)
+{
+    const int jlo = __shfl_sync(0xffffffffu, j, 0), jhi = __shfl_sync(0xffffffffu, j, 31);
+    for (int t = jlo; t <= jhi; ++t) {
+        const unsigned m = __reduce_max_sync(0xffffffffu, j == t ? bits : 0u);
+        if ((threadIdx.x & 31) == 0 && m != 0u) atomicMax(&smax[t], m);
+    }
+}
+
 // ---- tcgen05 (5th-generation tensor cores, tensor memory) ----------------
 
 BITNET_DEVINL void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }

@@ -40,8 +40,10 @@ struct DecodeArgs {
     const int32_t *rs_in;   // [M] per-token sums of x_q
     const uint8_t *w0, *w1; // [N][K/4] packed
     const float *gamma0, *gamma1;
-    float *y;               // [M][N]
+    void *y;                // [M][N] fp32, or bf16 when y_bf16
+    float *y_amax;          // optional [M]: max |y| per token, atomicMax into zeroed memory
     int32_t *acc0, *acc1;   // [M][N] optional
+    int y_bf16;
     int M, N, K;
     int grid;               // CTAs sharing the N rows
     int rg;                 // row groups per matrix per CTA (<= DEC_RGM)
@@ -90,6 +92,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) k_decode(const DecodeArgs a)
     float *tok_s = reinterpret_cast<float *>(smem + 64);    // [8]
     int *tok_rs = reinterpret_cast<int *>(smem + 96);       // [8]
     float *tok_r = reinterpret_cast<float *>(smem + 128);   // [2][8]
+    unsigned *s_amax = reinterpret_cast<unsigned *>(smem + 192); // [8] per-token max magnitude bits
     uint8_t *sW = smem + DEC_HDR;
     const int rg = a.rg;
     const size_t w_bytes = (size_t)NMAT * rg * 16 * a.w_stride;
@@ -105,6 +108,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) k_decode(const DecodeArgs a)
         mbar_init(bar_w, 1);
         fence_mbarrier_init();
     }
+    if (tid < 8) s_amax[tid] = 0u;
     __syncthreads();
     // ---- weight prefetch: independent of the previous grid ----
     if (warp == 0) {
@@ -188,23 +192,35 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) k_decode(const DecodeArgs a)
         __syncthreads();
 
         // ---- epilogue: remove the code offset, dequantise, (gate), store ----
-        for (int idx = tid; idx < R * mt; idx += DEC_THREADS) {
-            const int row = idx % R, j = idx / R;
-            const size_t o = (size_t)(m0 + j) * a.N + r0 + row;
-            const int a0 = sRed[j * a.rp + row] - tok_rs[j];
-            if (a.acc0) a.acc0[o] = a0;
-            const float v0 = __fmul_rn((float)a0, tok_r[j]);
-            if constexpr (NMAT == 1) {
-                a.y[o] = v0;
-            } else {
-                const int a1 = sRed[(8 + j) * a.rp + row] - tok_rs[j];
-                if (a.acc1) a.acc1[o] = a1;
-                const float v1 = __fmul_rn((float)a1, tok_r[8 + j]);
-                const float gp = v0 > 0.0f ? v0 : 0.0f;
-                a.y[o] = __fmul_rn(__fmul_rn(gp, gp), v1);
+        const bool obf = a.y_bf16 != 0;
+        const int total = R * mt;
+        for (int base = warp * 32; base < total; base += DEC_THREADS) {
+            const int idx = base + lane;
+            const bool act = idx < total;
+            const int row = act ? idx % R : 0, j = act ? idx / R : mt - 1;
+            uint32_t mag = 0;
+            if (act) {
+                const size_t o = (size_t)(m0 + j) * a.N + r0 + row;
+                const int a0 = sRed[j * a.rp + row] - tok_rs[j];
+                if (a.acc0) a.acc0[o] = a0;
+                float v = __fmul_rn((float)a0, tok_r[j]);
+                if constexpr (NMAT == 2) {
+                    const int a1 = sRed[(8 + j) * a.rp + row] - tok_rs[j];
+                    if (a.acc1) a.acc1[o] = a1;
+                    const float v1 = __fmul_rn((float)a1, tok_r[8 + j]);
+                    const float gp = v > 0.0f ? v : 0.0f;
+                    v = __fmul_rn(__fmul_rn(gp, gp), v1);
+                }
+                out_store(a.y, o, v, obf);
+                mag = out_mag_bits(v, obf);
             }
+            if (a.y_amax) warp_token_max(mag, j, s_amax);
         }
         __syncthreads();
+        if (a.y_amax && tid < mt) {
+            if (s_amax[tid]) atomicMax(reinterpret_cast<unsigned *>(a.y_amax) + m0 + tid, s_amax[tid]);
+            s_amax[tid] = 0u;
+        }
     }
 }
 

@@ -38,9 +38,12 @@ constexpr int DC_RGW_MAX = 8; // max row groups (of 16 rows) per warp
 
 struct DcArgs {
     const void *x;
+    const float *x_amax;        // optional [M]: max |x| per token, given (no reduction, no exchange)
     const uint8_t *w0, *w1;     // packed [N][K/4]
     const float *gamma0, *gamma1;
-    float *y;
+    void *y;                    // fp32, or bf16 when y_bf16
+    float *y_amax;              // optional [M]: max |y| per token, atomicMax into zeroed memory
+    int y_bf16;
     int32_t *acc0, *acc1;
     int8_t *xq_out;
     float *s_out;
@@ -88,6 +91,7 @@ __global__ void __launch_bounds__(DC_THREADS, 2) k_decode_cluster(const DcArgs a
     float *tok_s = reinterpret_cast<float *>(smem + 64);
     int *tok_rs = reinterpret_cast<int *>(smem + 96);
     float *tok_r = reinterpret_cast<float *>(smem + 128);     // [2][8]
+    unsigned *s_amax = reinterpret_cast<unsigned *>(smem + 192); // [8] per-token max magnitude bits of y
     float *amax_slot = reinterpret_cast<float *>(smem + 256); // [C][8]
     unsigned char *sW = smem + DC_HDR;
     unsigned char *sXs = smem + a.xs_off;
@@ -125,6 +129,7 @@ __global__ void __launch_bounds__(DC_THREADS, 2) k_decode_cluster(const DcArgs a
         }
         fence_mbarrier_init();
     }
+    if (tid < 8) s_amax[tid] = 0u;
     __syncthreads();
     cluster_arrive(); // peers may send to this CTA once every CTA of the cluster has arrived here
     {
@@ -192,15 +197,16 @@ __global__ void __launch_bounds__(DC_THREADS, 2) k_decode_cluster(const DcArgs a
         const int mt = min(8, a.M - m0);
         const int pp = tile & 1;                        // which barrier of each pair
         const uint32_t ph = (uint32_t)(tile >> 1) & 1u; // its phase parity
+        const bool given = a.x_amax != nullptr; // per-token maxima supplied: no reduction, no exchange
         if (tid == 0) {
-            mbar_arrive_expect_tx(&bar_amax[pp], (uint32_t)(C - 1) * 32);
+            if (!given) mbar_arrive_expect_tx(&bar_amax[pp], (uint32_t)(C - 1) * 32);
             mbar_arrive_expect_tx(&bar_red[pp], (uint32_t)(C - 1) * a.blk_bytes);
             if (tile > 0) issue_x(m0, mt);
         }
         ok = mbar_wait(bar_x, (uint32_t)tile & 1u) && ok;
 
         // ---- partial absmax of this slice, warp j <-> token j ----
-        {
+        if (!given) {
             float mx = 0.0f;
             if (warp < mt && ok) {
                 const uint4 *src = reinterpret_cast<const uint4 *>(sXs + warp * a.xs_row);
@@ -211,17 +217,23 @@ __global__ void __launch_bounds__(DC_THREADS, 2) k_decode_cluster(const DcArgs a
         }
         __syncthreads();
         if (tile == 0) cluster_wait(); // every peer's barriers exist before anyone sends to them
-        if (tid < C && tid != (int)r) {
-            const float *v = &amax_slot[r * 8];
-            const uint32_t dst = mapa_shared(smem_u32(&amax_slot[r * 8]), tid);
-            const uint32_t bar = mapa_shared(smem_u32(&bar_amax[pp]), tid);
-            st_async_v4f(dst, v[0], v[1], v[2], v[3], bar);
-            st_async_v4f(dst + 16, v[4], v[5], v[6], v[7], bar);
+        if (!given) {
+            if (tid < C && tid != (int)r) {
+                const float *v = &amax_slot[r * 8];
+                const uint32_t dst = mapa_shared(smem_u32(&amax_slot[r * 8]), tid);
+                const uint32_t bar = mapa_shared(smem_u32(&bar_amax[pp]), tid);
+                st_async_v4f(dst, v[0], v[1], v[2], v[3], bar);
+                st_async_v4f(dst + 16, v[4], v[5], v[6], v[7], bar);
+            }
+            ok = mbar_wait_cluster(&bar_amax[pp], ph) && ok;
         }
-        ok = mbar_wait_cluster(&bar_amax[pp], ph) && ok;
         if (tid < 8) {
             float am = 0.0f;
-            for (int src = 0; src < C; ++src) am = fmaxf(am, amax_slot[src * 8 + tid]);
+            if (given) {
+                if (tid < mt) am = a.x_amax[m0 + tid];
+            } else {
+                for (int src = 0; src < C; ++src) am = fmaxf(am, amax_slot[src * 8 + tid]);
+            }
             tok_s[tid] = quant_scale(am);
         }
         __syncthreads();
@@ -343,27 +355,40 @@ __global__ void __launch_bounds__(DC_THREADS, 2) k_decode_cluster(const DcArgs a
         if (m0 + 8 >= a.M) cluster_arrive(); // this CTA needs nothing more from its peers
 
         // ---- owners: sum the C partials, dequantise, gate, store ----
-        for (int idx = tid; idx < nown * mt; idx += DC_THREADS) {
-            const int orow = idx % nown, j = idx / nown;
-            int s0 = 0, s1 = 0;
-            for (int src = 0; src < C; ++src) {
-                const int *blk = (src == (int)r ? part + (int)r * blk_ints : recv + src * blk_ints) + j * a.orp + orow;
-                s0 += blk[0];
-                if (NMAT == 2) s1 += blk[8 * a.orp];
+        const bool obf = a.y_bf16 != 0;
+        const int total = nown * mt;
+        for (int base = warp * 32; base < total; base += DC_THREADS) {
+            const int idx = base + lane;
+            const bool act = idx < total;
+            const int orow = act ? idx % nown : 0, j = act ? idx / nown : mt - 1;
+            uint32_t mag = 0;
+            if (act) {
+                int s0 = 0, s1 = 0;
+                for (int src = 0; src < C; ++src) {
+                    const int *blk =
+                        (src == (int)r ? part + (int)r * blk_ints : recv + src * blk_ints) + j * a.orp + orow;
+                    s0 += blk[0];
+                    if (NMAT == 2) s1 += blk[8 * a.orp];
+                }
+                const size_t o = (size_t)(m0 + j) * a.N + (size_t)(n0 + own0 + orow);
+                if (a.acc0) a.acc0[o] = s0;
+                float v = __fmul_rn((float)s0, tok_r[j]);
+                if constexpr (NMAT == 2) {
+                    if (a.acc1) a.acc1[o] = s1;
+                    const float v1 = __fmul_rn((float)s1, tok_r[8 + j]);
+                    const float gp = v > 0.0f ? v : 0.0f;
+                    v = __fmul_rn(__fmul_rn(gp, gp), v1);
+                }
+                out_store(a.y, o, v, obf);
+                mag = out_mag_bits(v, obf);
             }
-            const size_t o = (size_t)(m0 + j) * a.N + (size_t)(n0 + own0 + orow);
-            if (a.acc0) a.acc0[o] = s0;
-            const float v0 = __fmul_rn((float)s0, tok_r[j]);
-            if constexpr (NMAT == 1) {
-                a.y[o] = v0;
-            } else {
-                if (a.acc1) a.acc1[o] = s1;
-                const float v1 = __fmul_rn((float)s1, tok_r[8 + j]);
-                const float gp = v0 > 0.0f ? v0 : 0.0f;
-                a.y[o] = __fmul_rn(__fmul_rn(gp, gp), v1);
-            }
+            if (a.y_amax) warp_token_max(mag, j, s_amax);
         }
         __syncthreads();
+        if (a.y_amax && tid < mt) {
+            if (s_amax[tid]) atomicMax(reinterpret_cast<unsigned *>(a.y_amax) + m0 + tid, s_amax[tid]);
+            s_amax[tid] = 0u;
+        }
     }
     if (!wready && tid == 0) mbar_wait_drain(bar_w, 0);
     // no CTA leaves while a peer's bulk copy may still read its shared memory:

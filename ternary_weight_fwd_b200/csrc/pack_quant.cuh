@@ -119,7 +119,8 @@ BITNET_DEVINL uint2 chunk_quant(const uint4 v, float sc, int &rs)
 template <bool XF32>
 __global__ void __launch_bounds__(256) k_quant_rows(const void *__restrict__ x, int64_t M, int64_t K,
                                                     int8_t *__restrict__ x_q, float *__restrict__ s,
-                                                    int32_t *__restrict__ rowsum)
+                                                    int32_t *__restrict__ rowsum, const float *__restrict__ amax_in,
+                                                    float *__restrict__ amax_zero)
 {
     pdl_launch_dependents();
     pdl_wait();
@@ -131,14 +132,18 @@ __global__ void __launch_bounds__(256) k_quant_rows(const void *__restrict__ x, 
     const uint4 *row = reinterpret_cast<const uint4 *>(static_cast<const char *>(x) + m * K * (XF32 ? 4 : 2));
     float amax = 0.0f;
     int64_t c = lane;
-    for (; c + 96 < nch; c += 128) {
-        const uint4 v0 = __ldg(row + c), v1 = __ldg(row + c + 32), v2 = __ldg(row + c + 64),
-                    v3 = __ldg(row + c + 96);
-        amax = fmaxf(amax, fmaxf(fmaxf(chunk_absmax<XF32>(v0), chunk_absmax<XF32>(v1)),
-                                 fmaxf(chunk_absmax<XF32>(v2), chunk_absmax<XF32>(v3))));
+    if (amax_in) {
+        amax = amax_in[m]; // the row maximum is given: one pass over x
+    } else {
+        for (; c + 96 < nch; c += 128) {
+            const uint4 v0 = __ldg(row + c), v1 = __ldg(row + c + 32), v2 = __ldg(row + c + 64),
+                        v3 = __ldg(row + c + 96);
+            amax = fmaxf(amax, fmaxf(fmaxf(chunk_absmax<XF32>(v0), chunk_absmax<XF32>(v1)),
+                                     fmaxf(chunk_absmax<XF32>(v2), chunk_absmax<XF32>(v3))));
+        }
+        for (; c < nch; c += 32) amax = fmaxf(amax, chunk_absmax<XF32>(__ldg(row + c)));
+        amax = warp_max(amax);
     }
-    for (; c < nch; c += 32) amax = fmaxf(amax, chunk_absmax<XF32>(__ldg(row + c)));
-    amax = warp_max(amax);
     const float sc = quant_scale(amax);
     int rs = 0;
     int8_t *qrow = x_q + m * K;
@@ -153,6 +158,7 @@ __global__ void __launch_bounds__(256) k_quant_rows(const void *__restrict__ x, 
     if (lane == 0) {
         s[m] = sc;
         if (rowsum) rowsum[m] = rs;
+        if (amax_zero) amax_zero[m] = 0.0f;
     }
 }
 
@@ -166,7 +172,9 @@ constexpr int QR_NCH = 16;
 template <bool XF32, int WPR>
 __global__ void __launch_bounds__(256) k_quant_rows_reg(const void *__restrict__ x, int64_t M, int64_t K,
                                                         int8_t *__restrict__ x_q, float *__restrict__ s,
-                                                        int32_t *__restrict__ rowsum)
+                                                        int32_t *__restrict__ rowsum,
+                                                        const float *__restrict__ amax_in,
+                                                        float *__restrict__ amax_zero)
 {
     __shared__ float red_max[8];
     __shared__ int red_sum[8];
@@ -191,13 +199,17 @@ __global__ void __launch_bounds__(256) k_quant_rows_reg(const void *__restrict__
             amax = fmaxf(amax, chunk_absmax<XF32>(v[i]));
         }
     }
-    amax = warp_max(amax);
-    if (WPR > 1) {
-        if (lane == 0) red_max[warp] = amax;
-        __syncthreads();
-        const int w0 = warp - wr;
+    if (amax_in) {
+        amax = live ? amax_in[m] : 0.0f; // the row maximum is given: no reduction
+    } else {
+        amax = warp_max(amax);
+        if (WPR > 1) {
+            if (lane == 0) red_max[warp] = amax;
+            __syncthreads();
+            const int w0 = warp - wr;
 #pragma unroll
-        for (int i = 0; i < WPR; ++i) amax = fmaxf(amax, red_max[w0 + i]);
+            for (int i = 0; i < WPR; ++i) amax = fmaxf(amax, red_max[w0 + i]);
+        }
     }
     const float sc = quant_scale(amax);
     int rs = 0;
@@ -225,7 +237,17 @@ __global__ void __launch_bounds__(256) k_quant_rows_reg(const void *__restrict__
     if (live && wr == 0 && lane == 0) {
         s[m] = sc;
         if (rowsum) rowsum[m] = rs;
+        if (amax_zero) amax_zero[m] = 0.0f;
     }
+}
+
+// amax[0 .. n) <- 0 ahead of a kernel that folds row maxima into it with
+// atomicMax (after the previous kernel, which may still read or write it).
+__global__ void __launch_bounds__(128) k_zero_f32(float *__restrict__ amax, int n)
+{
+    pdl_launch_dependents();
+    pdl_wait();
+    for (int i = threadIdx.x; i < n; i += blockDim.x) amax[i] = 0.0f;
 }
 
 // ---------------------------------------------------------------------------
@@ -250,7 +272,7 @@ template <bool XF32, int TPR>
 __global__ void __launch_bounds__(256) k_rmsnorm_quant_rows(const void *__restrict__ x, int64_t M, int64_t K,
                                                             const float *__restrict__ g, float eps,
                                                             int8_t *__restrict__ x_q, float *__restrict__ s,
-                                                            int32_t *__restrict__ rowsum)
+                                                            int32_t *__restrict__ rowsum, float *__restrict__ amax_zero)
 {
     constexpr int RPC = 256 / TPR;         // rows per CTA
     constexpr int WPR = TPR / 32;          // warps per row
@@ -335,6 +357,7 @@ __global__ void __launch_bounds__(256) k_rmsnorm_quant_rows(const void *__restri
         for (int w = 0; w < WPR; ++w) tot += red_sum[lr][w];
         s[m] = sc;
         if (rowsum) rowsum[m] = tot;
+        if (amax_zero) amax_zero[m] = 0.0f;
     }
 }
 

@@ -55,9 +55,11 @@ struct PrefillArgs {
     int num_m, num_n, num_k, num_tiles;
     const float *gamma0, *gamma1;
     const float *s;       // [M] per-token scales
-    float *y;             // [M][N]
+    void *y;              // [M][N] fp32, or bf16 when y_bf16
+    float *y_amax;        // optional [M]: max |y| per row, folded in with atomicMax (zeroed beforehand)
     int32_t *acc0, *acc1; // optional [M][N]
-    int vec_ok;           // N % 4 == 0 (16-byte row chunks are aligned)
+    int y_bf16;           // store y as bf16 (nearest even of the fp32 value)
+    int vec_ok;           // rows of y are 16-byte multiples: TMA stores
 };
 
 // codes {0,1,2} (one per byte) -> int8 {-1,0,1}: per byte (c | 0x80) - 1 cannot
@@ -102,6 +104,13 @@ BITNET_DEVINL void pf_store_row32(float *dst, const float (&v)[32], int ncols, b
         for (int j = 0; j < 32; ++j)
             if (j < ncols) dst[j] = v[j];
     }
+}
+
+BITNET_DEVINL void pf_store_row32_bf16(uint16_t *dst, const uint32_t (&pk)[16], int ncols)
+{
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+        if (j < ncols) dst[j] = (uint16_t)(j & 1 ? pk[j >> 1] >> 16 : pk[j >> 1] & 0xffffu);
 }
 
 BITNET_DEVINL void pf_store_row32_i(int32_t *dst, const uint32_t (&v)[32], int ncols, bool vec, int off)
@@ -270,24 +279,50 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         }
     } else {
         // ---------------- epilogue (warps 0-3: TMEM lanes 32w..32w+31) ----------------
-        // fp32 chunks of 32 rows x 32 columns go through a 128-byte-swizzled
-        // staging buffer (chunk j of row l at l*128 + ((j ^ (l & 7)) << 4), so
-        // the writes are conflict-free) and one TMA store; two buffers per warp.
+        // Chunks of 32 rows x 32 columns go through a swizzled staging buffer
+        // and one TMA store; two buffers per warp.  fp32: 128-byte rows, chunk
+        // j of row l at l*128 + ((j ^ (l & 7)) << 4); bf16: 64-byte rows, chunk
+        // j at l*64 + ((j ^ ((l >> 1) & 3)) << 4) (the 64-byte swizzle).  Both
+        // keep the eight lanes of a shared-memory wavefront on distinct banks.
         pdl_wait();
         const float g0 = a.gamma0[0];
         const float g1 = FFN ? a.gamma1[0] : 0.0f;
         const bool tma_out = a.vec_ok != 0;
+        const bool obf = a.y_bf16 != 0;
         unsigned char *wbuf = epi_bufs + warp * 2 * PF_EPI_BUF;
         int nbuf = 0;
+        uint32_t rmax = 0; // this lane's row: max magnitude bits of the stored values of the tile
         auto emit = [&](const float (&o)[32], int m, int n, bool mok) {
+            const int nv = a.N - n; // valid columns of this chunk (the rest is never stored)
+            uint32_t pk[16];
+            if (obf) {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) pk[j] = bf16_rn_bits(o[2 * j]) | (bf16_rn_bits(o[2 * j + 1]) << 16);
+                if (a.y_amax) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (j < nv) rmax = max(rmax, ((j & 1 ? pk[j >> 1] >> 16 : pk[j >> 1]) & 0x7fffu) << 16);
+                }
+            } else if (a.y_amax) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    if (j < nv) rmax = max(rmax, __float_as_uint(o[j]) & 0x7fffffffu);
+            }
             if (tma_out) {
                 unsigned char *buf = wbuf + nbuf * PF_EPI_BUF;
                 if (lane == 0) bulk_wait_group_read<1>(); // the store that used this buffer has read it
                 __syncwarp();
+                if (obf) {
 #pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    *reinterpret_cast<float4 *>(buf + lane * 128 + ((j ^ (lane & 7)) << 4)) =
-                        make_float4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+                    for (int j = 0; j < 4; ++j)
+                        *reinterpret_cast<uint4 *>(buf + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4)) =
+                            make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        *reinterpret_cast<float4 *>(buf + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                            make_float4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+                }
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
@@ -296,7 +331,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 }
                 nbuf ^= 1;
             } else if (mok && n < a.N) {
-                pf_store_row32(a.y + (size_t)m * a.N + n, o, a.N - n, false);
+                if (obf)
+                    pf_store_row32_bf16(static_cast<uint16_t *>(a.y) + (size_t)m * a.N + n, pk, nv);
+                else
+                    pf_store_row32(static_cast<float *>(a.y) + (size_t)m * a.N + n, o, nv, false);
             }
         };
         int acc = 0;
@@ -319,11 +357,11 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                     tmem_wait_ld();
                     const int n = nb * PF_BN + 32 * c;
                     if (n < a.N) {
+                        if (a.acc0 && mok) pf_store_row32_i(a.acc0 + (size_t)m * a.N + n, v, a.N - n, false, 0);
                         float o[32];
 #pragma unroll
                         for (int j = 0; j < 32; ++j) o[j] = __fmul_rn((float)(int)v[j], r0);
                         emit(o, m, n, mok);
-                        if (a.acc0 && mok) pf_store_row32_i(a.acc0 + (size_t)m * a.N + n, v, a.N - n, false, 0);
                     }
                 }
             } else {
@@ -335,6 +373,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                     tmem_wait_ld();
                     const int n = nb * (PF_BN / 2) + 32 * c;
                     if (n < a.N) {
+                        if (mok && a.acc0) pf_store_row32_i(a.acc0 + (size_t)m * a.N + n, vg, a.N - n, false, 0);
+                        if (mok && a.acc1) pf_store_row32_i(a.acc1 + (size_t)m * a.N + n, vu, a.N - n, false, 0);
                         float o[32];
 #pragma unroll
                         for (int j = 0; j < 32; ++j) {
@@ -344,10 +384,12 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                             o[j] = __fmul_rn(__fmul_rn(gp, gp), uv);
                         }
                         emit(o, m, n, mok);
-                        if (mok && a.acc0) pf_store_row32_i(a.acc0 + (size_t)m * a.N + n, vg, a.N - n, false, 0);
-                        if (mok && a.acc1) pf_store_row32_i(a.acc1 + (size_t)m * a.N + n, vu, a.N - n, false, 0);
                     }
                 }
+            }
+            if (a.y_amax) {
+                if (mok && rmax != 0u) atomicMax(reinterpret_cast<unsigned *>(a.y_amax) + m, rmax);
+                rmax = 0;
             }
             tc_fence_before();
             __syncwarp();

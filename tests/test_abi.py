@@ -139,3 +139,34 @@ def test_norm_entry_points_reject_before_launch(lib):
     assert ln(P, 0, 4, 256, P + 4, 1e-5, P, P, 256, P, None, None, None, P, ws, None) == tw.BITNET_ERR_MISALIGNED
     fn = lib.bitnet_ffn_gate_up_norm
     assert fn(P, 0, 4, 256, None, 1e-5, P, P, P, P, 256, P, None, None, P, ws, None) == tw.BITNET_ERR_INVALID_ARG
+
+
+def test_ex_entry_points_reject_before_launch(lib):
+    """bitnet_linear_ex / bitnet_ffn_gate_up_ex: bad output dtype, given maxima
+    together with normalisation, given and emitted maxima sharing memory, and
+    misaligned maxima are rejected on the host."""
+    P = 1 << 40
+    A = P + (1 << 20)  # a second, disjoint address
+    ws = tw.bitnet_workspace_size(4, 256, 256)
+    lx = lib.bitnet_linear_ex
+    ok_args = dict(x=P, xd=0, xa=None, g=None, eps=1e-5, m=4, k=256, w=P, gam=P, n=256, y=P, yd=0, ya=None)
+
+    def call(**kw):
+        a = dict(ok_args, **kw)
+        return lx(a["x"], a["xd"], a["xa"], a["g"], a["eps"], a["m"], a["k"], a["w"], a["gam"], a["n"], a["y"],
+                  a["yd"], a["ya"], P, ws, None)
+
+    assert call(yd=7) == tw.BITNET_ERR_INVALID_ARG
+    assert call(xd=7) == tw.BITNET_ERR_INVALID_ARG
+    assert call(xa=A, g=P) == tw.BITNET_ERR_INVALID_ARG
+    assert call(xa=A, ya=A + 8) == tw.BITNET_ERR_INVALID_ARG
+    assert call(xa=A, ya=A) == tw.BITNET_ERR_INVALID_ARG
+    assert call(ya=A + 4) == tw.BITNET_ERR_MISALIGNED
+    assert call(xa=A + 4) == tw.BITNET_ERR_MISALIGNED
+    assert call(y=None) == tw.BITNET_ERR_INVALID_ARG
+    assert call(k=96) == tw.BITNET_ERR_UNSUPPORTED_SHAPE
+    fx = lib.bitnet_ffn_gate_up_ex
+    assert fx(P, 0, None, None, 1e-5, 4, 256, P, P, P, P, 256, P, 5, None, P, ws, None) == tw.BITNET_ERR_INVALID_ARG
+    assert fx(P, 0, A, P, 1e-5, 4, 256, P, P, P, P, 256, P, 0, None, P, ws, None) == tw.BITNET_ERR_INVALID_ARG
+    assert fx(P, 0, None, None, 1e-5, 4, 256, P, P, None, P, 256, P, 0, None, P, ws, None) == \
+        tw.BITNET_ERR_INVALID_ARG
