@@ -57,6 +57,8 @@ def parse_args():
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--cpu-seconds", type=float, default=10.0, help="budget of the oracle CPU baseline")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--seq-partitions", type=int, default=0,
+                   help="decode-sequence partition count (0: chosen by the library's planner)")
     p.add_argument("--decode-path", choices=["sequence", "per-op"], default="sequence",
                    help="decode step as one persistent bitnet_decode_sequence launch (default) or one "
                         "bitnet_linear / bitnet_ffn_gate_up call per projection")
@@ -79,6 +81,7 @@ def workload_config(a, n_gpus):
         "prefill_tokens": a.prefill_tokens, "decode_steps": a.decode_steps, "decode_batch": a.decode_batch,
         "activations": "bf16 N(0,1), fresh per projection; ternary weights from N(0,0.02) latents",
         "decode_path": a.decode_path,
+        "decode_outputs": "one set per layer",
         "l2": "inputs larger than L2: every pass streams 496 MB of packed weights; prefill activations rotate "
               "over 168 MB",
         "parallelism": f"replicas x{n_gpus} (data parallel, no collective)",
@@ -249,6 +252,12 @@ class Stack:
                         "o": torch.empty((B, HIDDEN), dtype=f32, device=device),
                         "h": torch.empty((B, INTER), dtype=f32, device=device),
                         "down": torch.empty((B, HIDDEN), dtype=f32, device=device)}
+        # the decode step's outputs, one set per layer: the layers of a step share no buffers, so the
+        # only dependency inside a step is gate/up -> down of each layer (fresh x for every other op)
+        self.dec_out_l = [{"q": torch.empty((B, HIDDEN), dtype=f32, device=device),
+                           "o": torch.empty((B, HIDDEN), dtype=f32, device=device),
+                           "h": torch.empty((B, INTER), dtype=f32, device=device),
+                           "down": torch.empty((B, HIDDEN), dtype=f32, device=device)} for _ in range(a.layers)]
         ws = max(tw.bitnet_workspace_size(M, INTER, INTER), tw.bitnet_workspace_size(M, HIDDEN, HIDDEN))
         self.ws_pre = torch.empty(ws, dtype=torch.uint8, device=device)
         self.ws_dec = torch.empty(tw.bitnet_workspace_size(B, INTER, INTER), dtype=torch.uint8, device=device)
@@ -303,9 +312,9 @@ class Stack:
     def decode_ops(self, t):
         """The projections of decode step t as bitnet_op_t records (one sequence launch)."""
         if t not in self.seq_ops:
-            tw, out, ops = self.tw, self.dec_out, []
+            tw, ops = self.tw, []
             for l in range(self.a.layers):
-                L = self.layers[l]
+                L, out = self.layers[l], self.dec_out_l[l]
                 base = t * 3 * self.a.layers + 3 * l
                 ops += [tw.linear_op(self.dec_x[base % self.n_dec], L["q"][0], L["q"][1], out["q"]),
                         tw.linear_op(self.dec_x[(base + 1) % self.n_dec], L["o"][0], L["o"][1], out["o"]),
@@ -321,10 +330,11 @@ class Stack:
             return
         for l in range(self.a.layers):
             base = t * 3 * self.a.layers + 3 * l
-            self.q(l, self.dec_x[base % self.n_dec], self.dec_out, self.ws_dec, s)
-            self.o(l, self.dec_x[(base + 1) % self.n_dec], self.dec_out, self.ws_dec, s)
-            self.gate_up(l, self.dec_x[(base + 2) % self.n_dec], self.dec_out, self.ws_dec, s)
-            self.down(l, self.dec_out, self.ws_dec, s)
+            out = self.dec_out_l[l]
+            self.q(l, self.dec_x[base % self.n_dec], out, self.ws_dec, s)
+            self.o(l, self.dec_x[(base + 1) % self.n_dec], out, self.ws_dec, s)
+            self.gate_up(l, self.dec_x[(base + 2) % self.n_dec], out, self.ws_dec, s)
+            self.down(l, out, self.ws_dec, s)
 
 
 def reduce_max(v, dist, device):
@@ -422,6 +432,7 @@ def our_arm(a, n_gpus):
         return reduce_max(v, dist, dev)
 
     st = Stack(a, dev, seed=1234 + rank)
+    st.tw.bitnet_set_sequence_partitions(a.seq_partitions)
     stream = torch.cuda.Stream(device=dev)
     stream.wait_stream(torch.cuda.current_stream())
 
@@ -604,7 +615,7 @@ def our_arm(a, n_gpus):
     if a.e2e_steps > 0:
         h_pre = [x.cpu().pin_memory() for x in st.pre_x]
         h_dec = [x.cpu().pin_memory() for x in st.dec_x]
-        outs = list(st.pre_out.values()) + list(st.dec_out.values())
+        outs = list(st.pre_out.values()) + list(st.dec_out_l[-1].values())  # the last layer's results
         h_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
         h2d = sum(x.numel() * x.element_size() for x in h_pre + h_dec)
         d2h = sum(o.numel() * o.element_size() for o in outs)

@@ -395,6 +395,43 @@ bitnet_status_t bitnet_decode_sequence(const bitnet_op_t *ops, int32_t n_ops, in
 int bitnet_set_sequence_cluster(int cluster_size);
 
 /*
+ * Partition count of the sequence kernel: 0 (default) lets the planner pick
+ * the count with the smallest estimated duration; 1 .. 8 forces that count
+ * (capped by the number of independent groups of ops).  Returns the previous
+ * value, or -1 if the value is not allowed.  Every count gives bit-identical
+ * results.  For tests and tuning; not synchronised with other threads.
+ */
+int bitnet_set_sequence_partitions(int partitions);
+
+/*
+ * Largest share of a CTA's shared-memory weight ring one op of a sequence may
+ * occupy: 1 / share, share = 1 .. 4 (default 1).  Projections larger than
+ * that are cut into more row slices.  With share >= 2 the next op's weights
+ * stream in while an op computes; with 1 fewer, larger slices wait for their
+ * weights.  Returns the previous value, or -1 if not allowed.  Every value
+ * gives bit-identical results.  For tests and tuning.
+ */
+int bitnet_set_sequence_ring_share(int share);
+
+/*
+ * The plan bitnet_decode_sequence would run, computed on the host only (no
+ * device is touched): for `clusters` clusters of `cluster_size` CTAs.
+ *   order[k]         index into ops of the k-th op executed
+ *   part_of[k]       its partition: a contiguous range of clusters that runs
+ *                    only its partition's ops; partitions never wait for each
+ *                    other (their ops share no memory)
+ *   slices[k]        the number of consecutive kernel ops it is cut into, over
+ *                    equal slices of its output rows (each slice's weights fit
+ *                    one CTA's shared-memory ring)
+ *   n_parts, part_clusters[0 .. n_parts)   partition count and sizes
+ * All arrays have n_ops entries (part_clusters: 8).  Errors as
+ * bitnet_decode_sequence (BITNET_ERR_UNSUPPORTED_SHAPE when no plan fits).
+ */
+bitnet_status_t bitnet_sequence_layout(const bitnet_op_t *ops, int32_t n_ops, int64_t M, int32_t cluster_size,
+                                       int32_t clusters, int32_t *order, int32_t *part_of, int32_t *slices,
+                                       int32_t *n_parts, int32_t *part_clusters);
+
+/*
  * Device-side status word.  Kernels whose waits are bounded record
  * BITNET_ERR_TIMEOUT there (and exit) instead of spinning forever.  This call
  * synchronises `stream`, copies the word to *status_out and, if clear != 0,

@@ -89,6 +89,10 @@ def load_library(path: str = LIB_PATH):
         "bitnet_sequence_schedule": ([ctypes.POINTER(bitnet_op_t), ctypes.c_int32, I64,
                                       ctypes.POINTER(ctypes.c_int32)], I),
         "bitnet_set_sequence_cluster": ([I], I),
+        "bitnet_set_sequence_partitions": ([I], I),
+        "bitnet_set_sequence_ring_share": ([I], I),
+        "bitnet_sequence_layout": ([ctypes.POINTER(bitnet_op_t), ctypes.c_int32, I64, ctypes.c_int32, ctypes.c_int32,
+                                    P, P, P, P, P], I),
         "bitnet_linear_ex": ([P, I, P, P, F, I64, I64, P, P, I64, P, I, P, P, SZ, P], I),
         "bitnet_ffn_gate_up_ex": ([P, I, P, P, F, I64, I64, P, P, P, P, I64, P, I, P, P, SZ, P], I),
     }
@@ -388,4 +392,37 @@ def bitnet_set_sequence_cluster(cluster_size: int) -> int:
     prev = load_library().bitnet_set_sequence_cluster(int(cluster_size))
     if prev < 0:
         raise ValueError(f"invalid sequence cluster size {cluster_size}")
+    return prev
+
+
+def bitnet_set_sequence_partitions(partitions: int) -> int:
+    """0: partition count chosen by the planner; 1..8: forced.  Returns the previous value."""
+    prev = load_library().bitnet_set_sequence_partitions(int(partitions))
+    if prev < 0:
+        raise ValueError(f"partition count must be 0..8, got {partitions}")
+    return prev
+
+
+def bitnet_sequence_layout(ops, m, cluster_size, clusters):
+    """Host-only plan of a sequence launch: dict(order, part_of, slices, part_clusters)."""
+    import numpy as np
+    n = len(ops)
+    order = np.zeros(n, np.int32)
+    part_of = np.zeros(n, np.int32)
+    slices = np.zeros(n, np.int32)
+    n_parts = np.zeros(1, np.int32)
+    part_cl = np.zeros(8, np.int32)
+    arr = _op_array(ops)
+    _check(load_library().bitnet_sequence_layout(arr, n, m, cluster_size, clusters, order.ctypes.data, part_of.ctypes.data,
+                                                 slices.ctypes.data, n_parts.ctypes.data, part_cl.ctypes.data),
+           "bitnet_sequence_layout")
+    return dict(order=order.tolist(), part_of=part_of.tolist(), slices=slices.tolist(),
+                part_clusters=part_cl[:int(n_parts[0])].tolist())
+
+
+def bitnet_set_sequence_ring_share(share: int) -> int:
+    """Largest share 1/share of the weight ring one sequence op may fill (1..4).  Returns the previous value."""
+    prev = load_library().bitnet_set_sequence_ring_share(int(share))
+    if prev < 0:
+        raise ValueError(f"ring share must be 1..4, got {share}")
     return prev

@@ -787,53 +787,93 @@ int seq_clusters(int dev, int C)
     return v;
 }
 
-// Per-op layout and the launch-wide shared-memory map for G clusters of C CTAs.
-// Partitions of the grid: op i runs on clusters [cl0[of[i]], cl0[of[i]] + ncl[of[i]]).
+// Partitions of the grid: user op i runs on clusters [cl0[of[i]], cl0[of[i]] +
+// ncl[of[i]]) as slices[i] consecutive ops over slices of its output rows.
 struct SeqParts {
     int n = 1;
     int cl0[DS_MAX_PARTS] = {0}, ncl[DS_MAX_PARTS] = {0};
-    std::vector<int> of;
+    std::vector<int> of;     // partition of each user op
+    std::vector<int> slices; // row slices of each user op
+    int ring_share = 1;      // an op's weights may fill 1 / ring_share of the ring
 };
 
-bitnet_status_t seq_build(DsProgram &p, const bitnet_op_t *ops, int n, int64_t M, int C, int G, const SeqParts &parts,
-                          const int32_t *wx, const int32_t *wy)
+// Rows per cluster of `rows` output rows spread over ncl clusters.
+inline int seq_rpc(int64_t rows, int ncl) { return (int)align_up((size_t)cdiv(rows, ncl), 16); }
+
+// Fewest row slices of an op (nmat matrices, N rows) for which every warp holds
+// at most DS_RGW row groups on ncl clusters.
+int seq_min_slices(int64_t N, int nmat, int ncl)
 {
+    int s = 1;
+    while ((int64_t)nmat * (seq_rpc(cdiv(N, s), ncl) / 16) > 8 * DS_RGW) ++s;
+    return s;
+}
+
+// Per-op layout and the launch-wide shared-memory map for G clusters of C CTAs.
+// The user ops (in execution order, waits wx / wy between them) are cut into
+// parts.slices[i] consecutive ops over slices of their output rows.  A slice
+// waits for the last slice of the op its user op waits for; later slices of an
+// op need no wait of their own (the first one's wait held on every CTA of the
+// partition), and with one token tile they reuse the first slice's quantised x.
+// too_big: set to the first user op whose weight piece does not fit the ring.
+bitnet_status_t seq_build(DsProgram &p, const bitnet_op_t *ops, int n, int64_t M, int C, int G, const SeqParts &parts,
+                          const int32_t *wx, const int32_t *wy, int *too_big = nullptr)
+{
+    if (too_big) *too_big = -1;
+    int total = 0;
+    for (int i = 0; i < n; ++i) total += parts.slices[i];
+    if (total > DS_MAX_OPS) return BITNET_ERR_UNSUPPORTED_SHAPE;
+    std::vector<int> last_of(n), user_of(total);
     int ks_max = 1;
     uint32_t blk_max = 0;
+    int idx = 0;
     for (int i = 0; i < n; ++i) {
         const bitnet_op_t &o = ops[i];
-        DsOp &d = p.ops[i];
-        d = DsOp{};
         const int part = parts.of[i];
-        d.cl0 = parts.cl0[part];
-        d.ncl = parts.ncl[part];
+        const int ncl = parts.ncl[part];
         const int nmat = o.kind == BITNET_OP_FFN_GATE_UP ? 2 : 1;
         const int KS = (int)(o.K / 64);
-        d.ks = (int)cdiv(KS, C);
-        if (d.ks > DS_MAX_KS) return BITNET_ERR_UNSUPPORTED_SHAPE;
-        d.rpc = (int)align_up((size_t)cdiv(o.N, d.ncl), 16);
-        const int64_t per_warp = cdiv((int64_t)nmat * (d.rpc / 16), 8);
-        if (per_warp > DS_RGW) return BITNET_ERR_UNSUPPORTED_SHAPE;
-        d.own_rows = d.rpc / C;
-        d.orp = (int)align_up((size_t)d.own_rows, 4);
-        if (d.orp % 8 == 0) d.orp += 4; // token rows of a block land 8 banks apart
-        d.box_w = 16 * (d.ks | 1);      // odd number of 16-byte chunks: conflict-free fragment loads
-        d.x = o.x;
-        d.w0 = o.w0;
-        d.w1 = nmat == 2 ? o.w1 : nullptr;
-        d.gamma0 = o.gamma0;
-        d.gamma1 = nmat == 2 ? o.gamma1 : nullptr;
-        d.y = o.y;
-        d.K = (int)o.K;
-        d.N = (int)o.N;
-        d.nmat = nmat;
-        d.xf32 = o.x_dtype == BITNET_DTYPE_F32;
-        d.wait_x = wx[i];
-        d.wait_y = wy[i];
-        ks_max = std::max(ks_max, d.ks);
-        blk_max = std::max(blk_max, (uint32_t)(nmat * 8 * d.orp * 4));
+        const int ks = (int)cdiv(KS, C);
+        if (ks > DS_MAX_KS) return BITNET_ERR_UNSUPPORTED_SHAPE;
+        const int ns = parts.slices[i];
+        const size_t row_bytes = (size_t)(o.K / 4);
+        for (int t = 0; t < ns; ++t, ++idx) {
+            const int64_t r0 = o.N * t / ns, r1 = o.N * (t + 1) / ns;
+            DsOp &d = p.ops[idx];
+            d = DsOp{};
+            user_of[idx] = i;
+            d.cl0 = (int16_t)parts.cl0[part];
+            d.ncl = (int16_t)ncl;
+            d.ks = (int16_t)ks;
+            const int rpc = seq_rpc(r1 - r0, ncl);
+            if ((int64_t)nmat * (rpc / 16) > 8 * DS_RGW) return BITNET_ERR_UNSUPPORTED_SHAPE;
+            d.rpc = (int16_t)rpc;
+            const int own = rpc / C;
+            int orp = (int)align_up((size_t)own, 4);
+            if (orp % 8 == 0) orp += 4; // token rows of a block land 8 banks apart
+            d.own_rows = (int16_t)own;
+            d.orp = (int16_t)orp;
+            d.box_w = (int16_t)(16 * (ks | 1)); // odd number of 16-byte chunks: conflict-free fragment loads
+            d.x = o.x;
+            d.w0 = o.w0 + (size_t)r0 * row_bytes;
+            d.w1 = nmat == 2 ? o.w1 + (size_t)r0 * row_bytes : nullptr;
+            d.gamma0 = o.gamma0;
+            d.gamma1 = nmat == 2 ? o.gamma1 : nullptr;
+            d.y = o.y + r0;
+            d.K = (int)o.K;
+            d.N = (int)(r1 - r0);
+            d.ldy = (int)o.N;
+            d.nmat = (uint8_t)nmat;
+            d.xf32 = o.x_dtype == BITNET_DTYPE_F32;
+            d.reuse = (t > 0 && M <= 8) ? 1 : 0;
+            d.wait_x = (wx[i] >= 0 && !d.reuse) ? last_of[wx[i]] : -1;
+            d.wait_y = (t == 0 && wy[i] >= 0) ? last_of[wy[i]] : -1;
+            blk_max = std::max(blk_max, (uint32_t)(nmat * 8 * orp * 4));
+        }
+        last_of[i] = idx - 1;
+        ks_max = std::max(ks_max, ks);
     }
-    p.n_ops = n;
+    p.n_ops = total;
     p.M = (int)M;
     p.C = C;
     p.n_ctas = G * C;
@@ -847,14 +887,15 @@ bitnet_status_t seq_build(DsProgram &p, const bitnet_op_t *ops, int n, int64_t M
     {
         int last[DS_MAX_PARTS];
         for (int q = 0; q < DS_MAX_PARTS; ++q) last[q] = -1;
-        for (int i = 0; i < n; ++i) {
+        for (int j = 0; j < total; ++j) {
+            const int i = user_of[j];
             const int q = parts.of[i];
-            p.ops[i].nxt = -1;
+            p.ops[j].nxt = -1;
             if (last[q] < 0)
-                p.part_first[q] = i;
+                p.part_first[q] = j;
             else
-                p.ops[last[q]].nxt = i;
-            last[q] = i;
+                p.ops[last[q]].nxt = j;
+            last[q] = j;
             // every op an op waits for runs in its partition
             if ((wx[i] >= 0 && parts.of[wx[i]] != q) || (wy[i] >= 0 && parts.of[wy[i]] != q))
                 return BITNET_ERR_INVALID_ARG;
@@ -864,16 +905,19 @@ bitnet_status_t seq_build(DsProgram &p, const bitnet_op_t *ops, int n, int64_t M
     }
     // x staging: ops whose x no op of the launch writes alternate between buffers 0 and 1 (the
     // next one is fetched while the current one runs); ops reading an earlier op's output use
-    // buffer 2 (loaded when their wait is over).  Rows as long as the largest K slice in the buffer.
+    // buffer 2 (loaded when their wait is over); ops reusing the previous op's x load nothing.
+    // Rows as long as the largest K slice in the buffer.
     uint32_t pitch[3] = {16, 16, 16};
     int alt[DS_MAX_PARTS] = {0};
-    for (int i = 0; i < n; ++i) {
-        DsOp &d = p.ops[i];
+    for (int j = 0; j < total; ++j) {
+        DsOp &d = p.ops[j];
+        if (d.reuse) continue;
+        const int q = parts.of[user_of[j]];
         if (d.wait_x >= 0) {
             d.xbuf = 2;
         } else {
-            d.xbuf = alt[parts.of[i]];
-            alt[parts.of[i]] ^= 1;
+            d.xbuf = (uint8_t)alt[q];
+            alt[q] ^= 1;
         }
         pitch[d.xbuf] = std::max(pitch[d.xbuf], (uint32_t)(d.ks * 64 * (d.xf32 ? 4 : 2)));
     }
@@ -894,70 +938,214 @@ bitnet_status_t seq_build(DsProgram &p, const bitnet_op_t *ops, int n, int64_t M
     const size_t usable = kSmemLimit - 128; // the kernel aligns its base to 128 bytes
     if (p.ring_off + 4096 > usable) return BITNET_ERR_UNSUPPORTED_SHAPE;
     p.ring_bytes = (uint32_t)((usable - p.ring_off) & ~size_t(127));
-    for (int i = 0; i < n; ++i)
-        if ((size_t)ds_piece_bytes(p.ops[i]) * p.ops[i].nmat > p.ring_bytes) return BITNET_ERR_UNSUPPORTED_SHAPE;
+    for (int j = 0; j < total; ++j)
+        if ((size_t)ds_piece_bytes(p.ops[j]) * p.ops[j].nmat * parts.ring_share > p.ring_bytes) {
+            if (too_big) *too_big = user_of[j];
+            return BITNET_ERR_UNSUPPORTED_SHAPE;
+        }
     return BITNET_OK;
 }
 
-// Independent groups of ops run side by side: the connected components of the
-// hazard graph never wait for each other.  The component with the most weight
-// bytes gets most clusters; the rest share the others, sized by their weight
-// bytes, as long as every weight piece still fits a CTA's ring.  A single
-// partition (every cluster runs every op) when there is one component or no
-// split fits.
-bitnet_status_t seq_partitioned_build(DsProgram &p, const bitnet_op_t *ops, int n, int64_t M, int C, int G,
-                                      const int32_t *wx, const int32_t *wy)
+// Partition count for decode sequences: 0 = chosen by the cost estimate below.
+std::atomic<int> g_seq_parts{0};
+// Share of the weight ring one op may fill (1 = all of it).  Half the ring
+// lets the next op's weights stream in while an op computes, but the extra row
+// slices cost more than the wait (measured on the 30-layer decode step: 4
+// partitions fit 256 ops at share 1, only 2 at share 2).
+std::atomic<int> g_seq_ring_share{1};
+
+// Estimated duration (µs) of the busiest partition of a built program: per op
+// a fixed exchange / epilogue cost, the x staging, absmax exchange and
+// quantisation unless the op reuses the previous op's, the contraction at
+// ~40 cycles per mma.sync per warp (measured, 1.9 GHz), and a producer's
+// completion latency when an op reads the output of the op just before it; or
+// the weight stream at ~45 GB/s per SM if that takes longer.
+double seq_estimate(const DsProgram &p)
 {
-    SeqParts one;
-    one.n = 1;
-    one.ncl[0] = G;
-    one.of.assign(n, 0);
-    if (G < 2) return seq_build(p, ops, n, M, C, G, one, wx, wy);
-    // components over the hazard waits (union-find)
+    double t_ops[DS_MAX_PARTS] = {0.0}, bytes[DS_MAX_PARTS] = {0.0};
+    for (int q = 0; q < p.n_parts; ++q) {
+        int prev = -1;
+        for (int j = p.part_first[q]; j >= 0; j = p.ops[j].nxt) {
+            const DsOp &d = p.ops[j];
+            const double mma_per_warp = (double)d.nmat * (d.rpc / 16) * d.ks * 2.0 / 8.0;
+            double t = 1.3 + mma_per_warp * 0.021;
+            if (!d.reuse) t += 1.6;
+            if (d.wait_x >= 0 && d.wait_x == prev) t += 2.3;
+            t_ops[q] += t;
+            bytes[q] += (double)d.nmat * d.N * (d.K / 4);
+            prev = j;
+        }
+    }
+    double worst = 0.0;
+    for (int q = 0; q < p.n_parts; ++q) {
+        const double stream_us = bytes[q] / (p.part_ncl[q] * p.C * 45e3);
+        worst = std::max(worst, std::max(t_ops[q], stream_us));
+    }
+    return worst;
+}
+
+// Independent groups of ops run side by side: the connected components of the
+// hazard graph never wait for each other.  For each partition count P (up to
+// DS_MAX_PARTS, or the count set by bitnet_set_sequence_partitions) the
+// components are dealt to P partitions by weight bytes (largest first, to the
+// lightest partition), each partition gets clusters in proportion to its
+// bytes, its ops are re-scheduled among themselves, and each op is cut into
+// the fewest row slices whose weight pieces fit a CTA's ring.  The program with
+// the smallest estimated duration is kept.  ops / wx / wy are rewritten in the
+// chosen execution order.
+// What the planner chose, per op of the returned execution order.
+struct SeqLayout {
+    std::vector<int> perm;    // index of the op in the list the planner was given
+    std::vector<int> part_of; // partition
+    std::vector<int> slices;  // row slices
+};
+
+bitnet_status_t seq_partitioned_build(DsProgram &p, bitnet_op_t *ops, int n, int64_t M, int C, int G, int32_t *wx,
+                                      int32_t *wy, ByteRange extra, SeqLayout *layout = nullptr)
+{
+    std::vector<ByteRange> xr, yr;
+    if (seq_validate(ops, n, M, extra, xr, yr) != BITNET_OK) return BITNET_ERR_INVALID_ARG;
+    // components over the hazards (union-find)
     std::vector<int> root(n);
     for (int i = 0; i < n; ++i) root[i] = i;
     auto find = [&](int i) {
         while (root[i] != i) i = root[i] = root[root[i]];
         return i;
     };
-    std::vector<ByteRange> xr, yr;
-    if (seq_validate(ops, n, M, ByteRange{0, 0}, xr, yr) != BITNET_OK) return BITNET_ERR_INVALID_ARG;
     for (int j = 0; j < n; ++j)
         for (int i = 0; i < j; ++i)
             if (hazard(xr, yr, i, j)) root[find(i)] = find(j);
-    std::vector<double> bytes(n, 0.0);
+    std::vector<double> cbytes(n, 0.0);
     double total = 0.0;
     for (int i = 0; i < n; ++i) {
         const double b = (ops[i].kind == BITNET_OP_FFN_GATE_UP ? 2.0 : 1.0) * (double)ops[i].N * (double)(ops[i].K / 4);
-        bytes[find(i)] += b;
+        cbytes[find(i)] += b;
         total += b;
     }
-    int main_root = find(0);
+    std::vector<int> comps;
     for (int i = 0; i < n; ++i)
-        if (bytes[find(i)] > bytes[main_root]) main_root = find(i);
-    const double side = total - bytes[main_root];
-    if (side <= 0.0) return seq_build(p, ops, n, M, C, G, one, wx, wy);
-    SeqParts two;
-    two.n = 2;
-    two.of.resize(n);
-    for (int i = 0; i < n; ++i) two.of[i] = find(i) == main_root ? 1 : 0;
-    // the side's share of clusters rounded down: the main component is one long dependency
-    // chain, so its per-op latency (fewer rows per CTA) sets the launch time
-    const int target = std::min(G - 1, std::max(1, (int)(G * side / total)));
-    for (int pass = 0; pass < 2; ++pass)
-        for (int s = pass == 0 ? target : target - 1; pass == 0 ? s < G : s >= 1; s += pass == 0 ? 1 : -1) {
-            two.cl0[0] = 0;
-            two.ncl[0] = s;
-            two.cl0[1] = s;
-            two.ncl[1] = G - s;
-            if (seq_build(p, ops, n, M, C, G, two, wx, wy) == BITNET_OK) return BITNET_OK;
+        if (find(i) == i) comps.push_back(i);
+    std::sort(comps.begin(), comps.end(), [&](int a, int b) { return cbytes[a] > cbytes[b] || (cbytes[a] == cbytes[b] && a < b); });
+
+    const int forced = g_seq_parts.load();
+    const int p_max = std::min({DS_MAX_PARTS, G, (int)comps.size()});
+    double best_t = 0.0;
+    bool have = false;
+    static DsProgram cand_proto;
+    DsProgram cand = cand_proto;
+    std::vector<bitnet_op_t> best_ops;
+    std::vector<int32_t> best_wx, best_wy;
+    SeqLayout best_layout;
+    for (int P = 1; P <= p_max; ++P) {
+        if (forced > 0 && P != std::min(forced, p_max)) continue;
+        // components to partitions: largest first, each to the lightest partition
+        std::vector<double> pbytes(P, 0.0);
+        std::vector<int> part_of_root(n, 0);
+        for (int c : comps) {
+            int q = 0;
+            for (int k = 1; k < P; ++k)
+                if (pbytes[k] < pbytes[q]) q = k;
+            part_of_root[c] = q;
+            pbytes[q] += cbytes[c];
         }
-    return seq_build(p, ops, n, M, C, G, one, wx, wy);
+        // clusters in proportion to bytes, at least one each
+        SeqParts parts;
+        parts.n = P;
+        int used = 0;
+        for (int q = 0; q < P; ++q) {
+            parts.ncl[q] = std::max(1, (int)(G * pbytes[q] / total));
+            used += parts.ncl[q];
+        }
+        while (used > G) { // only when many partitions are tiny
+            int q = 0;
+            for (int k = 1; k < P; ++k)
+                if (parts.ncl[k] > parts.ncl[q]) q = k;
+            --parts.ncl[q];
+            --used;
+        }
+        while (used < G) {
+            int q = 0;
+            for (int k = 1; k < P; ++k)
+                if (pbytes[k] / parts.ncl[k] > pbytes[q] / parts.ncl[q]) q = k;
+            ++parts.ncl[q];
+            ++used;
+        }
+        for (int q = 1; q < P; ++q) parts.cl0[q] = parts.cl0[q - 1] + parts.ncl[q - 1];
+        // execution order: partition by partition, each re-scheduled among its own ops
+        std::vector<bitnet_op_t> ord;
+        std::vector<int> perm;
+        ord.reserve(n);
+        for (int q = 0; q < P; ++q) {
+            std::vector<bitnet_op_t> sub;
+            std::vector<int> sub_idx;
+            for (int i = 0; i < n; ++i)
+                if (part_of_root[find(i)] == q) {
+                    sub.push_back(ops[i]);
+                    sub_idx.push_back(i);
+                }
+            if (sub.empty()) continue;
+            std::vector<int32_t> o(sub.size());
+            if (seq_schedule(sub.data(), (int)sub.size(), M, o.data(), extra) != BITNET_OK) return BITNET_ERR_INVALID_ARG;
+            for (int32_t k : o) {
+                ord.push_back(sub[k]);
+                perm.push_back(sub_idx[k]);
+            }
+        }
+        std::vector<int32_t> cwx(n), cwy(n);
+        if (seq_plan(ord.data(), n, M, cwx.data(), cwy.data(), extra) != BITNET_OK) return BITNET_ERR_INVALID_ARG;
+        // partition of each op in the new order
+        parts.of.assign(n, 0);
+        {
+            int pos = 0;
+            for (int q = 0; q < P; ++q)
+                for (int i = 0; i < n; ++i)
+                    if (part_of_root[find(i)] == q) parts.of[pos++] = q;
+        }
+        parts.ring_share = g_seq_ring_share.load();
+        parts.slices.resize(n);
+        for (int i = 0; i < n; ++i)
+            parts.slices[i] = seq_min_slices(ord[i].N, ord[i].kind == BITNET_OP_FFN_GATE_UP ? 2 : 1,
+                                             parts.ncl[parts.of[i]]);
+        // cut ops whose pieces do not fit the ring finer until they do (the ring grows as
+        // slices shrink: smaller partial-sum blocks)
+        bitnet_status_t st = BITNET_ERR_UNSUPPORTED_SHAPE;
+        for (int iter = 0; iter < 4 * DS_MAX_OPS; ++iter) {
+            int big = -1;
+            st = seq_build(cand, ord.data(), n, M, C, G, parts, cwx.data(), cwy.data(), &big);
+            if (st == BITNET_OK || big < 0) break;
+            if (parts.slices[big] >= ord[big].N) break;
+            ++parts.slices[big];
+        }
+        if (st != BITNET_OK) {
+            if (st == BITNET_ERR_INVALID_ARG) return st;
+            continue;
+        }
+        const double t = seq_estimate(cand);
+        if (!have || t < best_t) {
+            have = true;
+            best_t = t;
+            p = cand;
+            best_ops = ord;
+            best_wx = cwx;
+            best_wy = cwy;
+            best_layout.perm = perm;
+            best_layout.part_of = parts.of;
+            best_layout.slices = parts.slices;
+        }
+    }
+    if (!have) return BITNET_ERR_UNSUPPORTED_SHAPE;
+    for (int i = 0; i < n; ++i) {
+        ops[i] = best_ops[i];
+        wx[i] = best_wx[i];
+        wy[i] = best_wy[i];
+    }
+    if (layout) *layout = best_layout;
+    return BITNET_OK;
 }
 
-constexpr size_t kSeqWorkspaceBytes = 1024;
+constexpr size_t kSeqWorkspaceBytes = 2048;
 static_assert(4 * (DS_MAX_OPS + 1) <= (int)kSeqWorkspaceBytes, "sequence counters");
-static_assert(DS_MAX_OPS == BITNET_SEQ_MAX_OPS, "sequence op limit");
+static_assert(DS_MAX_OPS >= BITNET_SEQ_MAX_OPS, "sequence op limit: every op fits unsliced");
 static_assert(sizeof(DsProgram) <= 32000, "kernel parameter space");
 
 bitnet_status_t decode_sequence(const bitnet_op_t *ops, int n, int64_t M, void *workspace, size_t ws_bytes,
@@ -980,7 +1168,7 @@ bitnet_status_t decode_sequence(const bitnet_op_t *ops, int n, int64_t M, void *
     if (G < 1) return BITNET_ERR_CUDA;
     static DsProgram prog_proto; // zero-initialised template; each call fills a copy
     DsProgram p = prog_proto;
-    st = seq_partitioned_build(p, ops, n, M, C, G, wx, wy);
+    st = seq_partitioned_build(p, sched, n, M, C, G, wx, wy, wsr);
     if (st != BITNET_OK) return st;
     p.counters = static_cast<unsigned *>(workspace);
     cudaLaunchConfig_t cfg = {};
@@ -1140,10 +1328,51 @@ bitnet_status_t bitnet_sequence_schedule(const bitnet_op_t *ops, int32_t n_ops, 
     return seq_schedule(ops, n_ops, M, order, ByteRange{0, 0});
 }
 
+bitnet_status_t bitnet_sequence_layout(const bitnet_op_t *ops, int32_t n_ops, int64_t M, int32_t cluster_size,
+                                       int32_t clusters, int32_t *order, int32_t *part_of, int32_t *slices,
+                                       int32_t *n_parts, int32_t *part_clusters)
+{
+    if (!ops || n_ops < 1 || n_ops > BITNET_SEQ_MAX_OPS || !order || !part_of || !slices || !n_parts || !part_clusters)
+        return BITNET_ERR_INVALID_ARG;
+    if ((cluster_size != 4 && cluster_size != 8) || clusters < 1) return BITNET_ERR_INVALID_ARG;
+    int32_t wx[BITNET_SEQ_MAX_OPS], wy[BITNET_SEQ_MAX_OPS], ord0[BITNET_SEQ_MAX_OPS];
+    bitnet_status_t st = seq_schedule(ops, n_ops, M, ord0, ByteRange{0, 0});
+    if (st != BITNET_OK) return st;
+    bitnet_op_t sched[BITNET_SEQ_MAX_OPS];
+    for (int k = 0; k < n_ops; ++k) sched[k] = ops[ord0[k]];
+    st = seq_plan(sched, n_ops, M, wx, wy, ByteRange{0, 0});
+    if (st != BITNET_OK) return st;
+    static DsProgram proto;
+    DsProgram p = proto;
+    SeqLayout lay;
+    st = seq_partitioned_build(p, sched, n_ops, M, cluster_size, clusters, wx, wy, ByteRange{0, 0}, &lay);
+    if (st != BITNET_OK) return st;
+    for (int k = 0; k < n_ops; ++k) {
+        order[k] = ord0[lay.perm[k]];
+        part_of[k] = lay.part_of[k];
+        slices[k] = lay.slices[k];
+    }
+    *n_parts = p.n_parts;
+    for (int q = 0; q < p.n_parts; ++q) part_clusters[q] = p.part_ncl[q];
+    return BITNET_OK;
+}
+
 int bitnet_set_sequence_cluster(int cluster_size)
 {
     if (cluster_size != 4 && cluster_size != 8) return -1;
     return g_seq_cluster.exchange(cluster_size);
+}
+
+int bitnet_set_sequence_partitions(int partitions)
+{
+    if (partitions < 0 || partitions > DS_MAX_PARTS) return -1;
+    return g_seq_parts.exchange(partitions);
+}
+
+int bitnet_set_sequence_ring_share(int share)
+{
+    if (share < 1 || share > 4) return -1;
+    return g_seq_ring_share.exchange(share);
 }
 
 bitnet_status_t bitnet_rmsnorm_quant(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_t K, const float *g,

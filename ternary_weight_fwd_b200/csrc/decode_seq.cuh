@@ -40,36 +40,42 @@
 
 namespace bitnet {
 
-constexpr int DS_MAX_OPS = 128;   // ops per launch (kernel-parameter space)
+constexpr int DS_MAX_OPS = 256;   // ops per launch, after row slicing (kernel-parameter space)
 constexpr int DS_COMPUTE = 256;   // eight compute warps
 constexpr int DS_CONTROL = 128;   // control warps: weight copies and completion signals
 constexpr int DS_THREADS = DS_COMPUTE + DS_CONTROL;
 constexpr int DS_SLOTS = 8;       // ops whose weights may be in the ring at once
 constexpr int DS_PSLOTS = 16;     // weight pieces in the ring at once (one per matrix of an op)
-constexpr int DS_HDR = 1024 + 8 * 112; // header: barriers, per-token scalars, staged op descriptors
+constexpr int DS_HDR = 1024 + 8 * 96; // header: barriers, per-token scalars, staged op descriptors
 constexpr int DS_MAX_KS = 32;     // 64-wide k-steps per CTA
-constexpr int DS_MAX_PARTS = 4;   // partitions: independent groups of ops on disjoint clusters
+constexpr int DS_MAX_PARTS = 8;   // partitions: independent groups of ops on disjoint clusters
 constexpr int DS_RGW = 8;         // row groups (of 16 output rows) per compute warp (host limit)
 
+// One op of a sequence: a BitLinear or gated FFN over N output rows.  The host
+// may cut a projection into several ops over consecutive slices of its output
+// rows (w0/w1 and y then point at the slice's first row / column).
 struct __align__(16) DsOp {
     const void *x;               // [M][K] bf16 or fp32
     const uint8_t *w0, *w1;      // packed [N][K/4]; w1 (up) only for the gated FFN
     const float *gamma0, *gamma1;
-    float *y;                    // [M][N]
+    float *y;                    // y[m][n] at y + m * ldy + n, n < N
     int K, N;
-    int nmat;                    // 1 = BitLinear, 2 = gate/up + ReLU^2
-    int xf32;                    // x is fp32 (else bf16)
-    int ks;                      // 64-wide k-steps per CTA (the last CTAs may have fewer)
-    int rpc;                     // output rows per cluster (multiple of 16)
-    int own_rows;                // rows finished by each CTA of a cluster (rpc / C)
-    int orp;                     // row pitch (ints) of a partial-sum block, == 4 mod 8
-    int box_w;                   // shared bytes per weight row: 16 * odd (conflict-free rows)
+    int ldy;                     // row pitch of y (elements)
     int wait_x;                  // earlier op that must be complete before x is read (-1: none)
     int wait_y;                  // earlier op that must be complete before y is written (-1: none)
-    int xbuf;                    // x staging buffer: 0/1 alternate among ops whose x can be
-                                 // prefetched, 2 for ops that read an earlier op's output
-    int cl0, ncl;                // clusters running this op: [cl0, cl0 + ncl) (its partition)
     int nxt;                     // next op of the same partition (-1: last)
+    int16_t ks;                  // 64-wide k-steps per CTA (the last CTAs may have fewer)
+    int16_t rpc;                 // output rows per cluster (multiple of 16)
+    int16_t own_rows;            // rows finished by each CTA of a cluster (rpc / C)
+    int16_t orp;                 // row pitch (ints) of a partial-sum block, == 4 mod 8
+    int16_t box_w;               // shared bytes per weight row: 16 * odd (conflict-free rows)
+    int16_t cl0, ncl;            // clusters running this op: [cl0, cl0 + ncl) (its partition)
+    uint8_t nmat;                // 1 = BitLinear, 2 = gate/up + ReLU^2
+    uint8_t xf32;                // x is fp32 (else bf16)
+    uint8_t xbuf;                // x staging buffer: 0/1 alternate among ops whose x can be
+                                 // prefetched, 2 for ops that read an earlier op's output
+    uint8_t reuse;               // same x as the previous op of the partition, one token tile:
+                                 // its quantised slice, scales and row sums are still in place
 };
 
 struct DsProgram {
@@ -103,7 +109,7 @@ constexpr int DS_OP_P0 = 720;                      // uint32 [DS_SLOTS]: first p
 constexpr int DS_DESC = 1024;                      // DsOp [DS_DESC_SLOTS]: this CTA's k-th op in slot k % DS_DESC_SLOTS
 constexpr int DS_DESC_SLOTS = 8;
 
-static_assert(sizeof(DsOp) == 112 && DS_DESC + DS_DESC_SLOTS * 112 <= DS_HDR, "staged op descriptors");
+static_assert(sizeof(DsOp) == 96 && DS_DESC + DS_DESC_SLOTS * 96 <= DS_HDR, "staged op descriptors");
 
 // Descriptor of this CTA's k-th op, staged in shared memory (slot k % DS_DESC_SLOTS).
 BITNET_DEVINL const DsOp &ds_desc(unsigned char *smem, int k)
@@ -344,7 +350,8 @@ BITNET_DEVINL void ds_signal(const DsProgram &p, int j)
 
 // Per-CTA launch state shared by the ops (uniform across the CTA's threads).
 struct DsState {
-    int tile;        // token tiles done in this launch (exchange barriers and parity)
+    int tile;        // token tiles done in this launch (partial-sum exchange barriers and parity)
+    int atile;       // token tiles whose maxima were exchanged (absmax barriers and parity)
     uint32_t xw;     // completed waits on x staging buffer b (0..2) in bit b (its next parity)
     bool ok;
 };
@@ -425,18 +432,21 @@ __device__ __forceinline__ void ds_op(const DsProgram &p, const DsOp &op, int j,
 
     const float gam0 = op.gamma0[0];
     const float gam1 = nmat == 2 ? op.gamma1[0] : 0.0f;
+    const bool reuse = op.reuse != 0; // x_q, tok_s and tok_rs of the previous op stand
 
     for (int m0 = 0; m0 < p.M; m0 += 8, ++st.tile) {
         const int mt = min(8, p.M - m0);
         const int pp = st.tile & 1;
         const uint32_t ph = (uint32_t)(st.tile >> 1) & 1u;
+        const int app = st.atile & 1;
+        const uint32_t aph = (uint32_t)(st.atile >> 1) & 1u;
         if (tid == 0) {
-            mbar_arrive_expect_tx(&bar_amax[pp], (uint32_t)(C - 1) * 32);
+            if (!reuse) mbar_arrive_expect_tx(&bar_amax[app], (uint32_t)(C - 1) * 32);
             mbar_arrive_expect_tx(&bar_red[pp], (uint32_t)(C - 1) * blk_bytes);
         }
         // the first tile of an op that reads nothing this launch writes was fetched
         // during this CTA's previous op
-        if (warp == 0 && (m0 > 0 || k == 0 || op.wait_x >= 0)) {
+        if (warp == 0 && !reuse && (m0 > 0 || k == 0 || op.wait_x >= 0)) {
             if (m0 == 0 && op.wait_x >= 0) { // x is written by an earlier op of this launch
                 if (lane == 0) {
                     if (prev >= 0 && op.wait_x == prev) ds_signal(p, prev); // the previous op: publish it right here
@@ -451,65 +461,68 @@ __device__ __forceinline__ void ds_op(const DsProgram &p, const DsOp &op, int j,
             // the next op's first tile reads memory no op of this launch writes: fetch it now
             wait_local(reinterpret_cast<const uint32_t *>(smem + DS_DESC_READY), (uint32_t)k + 2);
             const DsOp &nx = ds_desc(smem, k + 1);
-            if (nx.wait_x < 0) { // its buffer (0/1) is not this op's and no earlier op still uses it
+            if (nx.wait_x < 0 && !nx.reuse) { // its buffer (0/1) is not this op's and no earlier op still uses it
                 const int nks0 = (int)r * nx.ks;
                 ds_load_x(p, nx, smem, nx.xbuf, 0, min(8, p.M), nks0, max(0, min(nx.ks, nx.K / 64 - nks0)), lane);
             }
         }
 
-        // ---- partial absmax of this warp's token over the staged slice ----
-        st.ok = mbar_spin(&bar_x[xb], (st.xw >> xb) & 1u) && st.ok;
-        st.xw ^= 1u << xb;
-        float mx = 0.0f;
-        if (warp < mt) {
-            const uint4 *src = reinterpret_cast<const uint4 *>(sXs + warp * xs_pitch);
-            if (xf32) {
-#pragma unroll 4
-                for (int c = lane; c < nchunk; c += 32) mx = fmaxf(mx, chunk_absmax<true>(src[c]));
-            } else {
-#pragma unroll 4
-                for (int c = lane; c < nchunk; c += 32) mx = fmaxf(mx, chunk_absmax<false>(src[c]));
-            }
-        }
-        mx = warp_max(mx);
-        if (lane == 0) amax_slot[r * 8 + warp] = mx;
-        compute_sync();
-        if (st.tile == 0) cluster_wait(); // every peer's barriers exist before anyone sends to them
-        if (tid < C && tid != (int)r) {
-            const float *v = &amax_slot[r * 8];
-            const uint32_t dst = mapa_shared(smem_u32(&amax_slot[r * 8]), tid);
-            const uint32_t bar = mapa_shared(smem_u32(&bar_amax[pp]), tid);
-            st_async_v4f(dst, v[0], v[1], v[2], v[3], bar);
-            st_async_v4f(dst + 16, v[4], v[5], v[6], v[7], bar);
-        }
-        st.ok = mbar_spin(&bar_amax[pp], ph, true) && st.ok;
-        if (tid < 8) {
-            float am = 0.0f;
-            for (int src = 0; src < C; ++src) am = fmaxf(am, amax_slot[src * 8 + tid]);
-            tok_s[tid] = quant_scale(am);
-        }
-        compute_sync();
-
-        // ---- quantise the staged slice (exact scale known), row sums ----
-        {
-            int rs = 0;
+        if (!reuse) {
+            // ---- partial absmax of this warp's token over the staged slice ----
+            st.ok = mbar_spin(&bar_x[xb], (st.xw >> xb) & 1u) && st.ok;
+            st.xw ^= 1u << xb;
+            float mx = 0.0f;
             if (warp < mt) {
-                const float sc = tok_s[warp];
                 const uint4 *src = reinterpret_cast<const uint4 *>(sXs + warp * xs_pitch);
-                unsigned char *dst = sXq + warp * p.xq_stride;
                 if (xf32) {
 #pragma unroll 4
-                    for (int c = lane; c < nchunk; c += 32)
-                        reinterpret_cast<uint32_t *>(dst)[c] = chunk_quant<true>(src[c], sc, rs).x;
+                    for (int c = lane; c < nchunk; c += 32) mx = fmaxf(mx, chunk_absmax<true>(src[c]));
                 } else {
 #pragma unroll 4
-                    for (int c = lane; c < nchunk; c += 32)
-                        reinterpret_cast<uint2 *>(dst)[c] = chunk_quant<false>(src[c], sc, rs);
+                    for (int c = lane; c < nchunk; c += 32) mx = fmaxf(mx, chunk_absmax<false>(src[c]));
                 }
             }
-            rs = warp_sum(rs);
-            if (lane == 0) tok_rs[warp] = rs;
-        }
+            mx = warp_max(mx);
+            if (lane == 0) amax_slot[r * 8 + warp] = mx;
+            compute_sync();
+            if (st.tile == 0) cluster_wait(); // every peer's barriers exist before anyone sends to them
+            if (tid < C && tid != (int)r) {
+                const float *v = &amax_slot[r * 8];
+                const uint32_t dst = mapa_shared(smem_u32(&amax_slot[r * 8]), tid);
+                const uint32_t bar = mapa_shared(smem_u32(&bar_amax[app]), tid);
+                st_async_v4f(dst, v[0], v[1], v[2], v[3], bar);
+                st_async_v4f(dst + 16, v[4], v[5], v[6], v[7], bar);
+            }
+            st.ok = mbar_spin(&bar_amax[app], aph, true) && st.ok;
+            ++st.atile;
+            if (tid < 8) {
+                float am = 0.0f;
+                for (int src = 0; src < C; ++src) am = fmaxf(am, amax_slot[src * 8 + tid]);
+                tok_s[tid] = quant_scale(am);
+            }
+            compute_sync();
+
+            // ---- quantise the staged slice (exact scale known), row sums ----
+            {
+                int rs = 0;
+                if (warp < mt) {
+                    const float sc = tok_s[warp];
+                    const uint4 *src = reinterpret_cast<const uint4 *>(sXs + warp * xs_pitch);
+                    unsigned char *dst = sXq + warp * p.xq_stride;
+                    if (xf32) {
+#pragma unroll 4
+                        for (int c = lane; c < nchunk; c += 32)
+                            reinterpret_cast<uint32_t *>(dst)[c] = chunk_quant<true>(src[c], sc, rs).x;
+                    } else {
+#pragma unroll 4
+                        for (int c = lane; c < nchunk; c += 32)
+                            reinterpret_cast<uint2 *>(dst)[c] = chunk_quant<false>(src[c], sc, rs);
+                    }
+                }
+                rs = warp_sum(rs);
+                if (lane == 0) tok_rs[warp] = rs;
+            }
+        } // !reuse
         if (tid < 16) {
             const int mat = tid >> 3, jj = tid & 7;
             if (mat < nmat) tok_r[tid] = __fdiv_rn(mat ? gam1 : gam0, tok_s[jj]);
@@ -618,7 +631,7 @@ __device__ __forceinline__ void ds_op(const DsProgram &p, const DsOp &op, int j,
                 s0 += blk[0];
                 if (nmat == 2) s1 += blk[8 * orp];
             }
-            const size_t o = (size_t)(m0 + jj) * op.N + (size_t)(n0 + own0 + orow);
+            const size_t o = (size_t)(m0 + jj) * op.ldy + (size_t)(n0 + own0 + orow);
             const float v0 = __fmul_rn((float)s0, tok_r[jj]);
             if (nmat == 1) {
                 op.y[o] = v0;
@@ -720,7 +733,7 @@ __global__ void __launch_bounds__(DS_THREADS, 1) k_decode_seq(const __grid_const
         cluster_arrive();
     } else {
         uint32_t head = 0;
-        DsState st = {0, 0u, true};
+        DsState st = {0, 0, 0u, true};
         const uint32_t *desc_ready = reinterpret_cast<const uint32_t *>(smem + DS_DESC_READY);
         int prev = -1, k = 0, pieces = 0;
         for (int j = first; j >= 0; ++k) {

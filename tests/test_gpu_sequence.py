@@ -198,15 +198,86 @@ def test_one_launch_graph_and_repeat(cluster):
     assert torch.count_nonzero(ws) == 0
 
 
-def test_too_large_for_the_weight_slice_is_rejected(cluster):
+def test_huge_projection_is_cut_into_row_slices(cluster):
+    """A gated FFN with 60000 output rows: its weights exceed every CTA's ring,
+    so the planner cuts it into row slices; the result is bit-identical to the
+    per-op call and matches the oracle on sampled rows."""
+    m, k, n = 8, 256, 60000
+    x, xf = make_x(m, k, 700, "outliers")
+    G, U = make_weights(n, k, 701), make_weights(n, k, 702)
+    y = torch.full((m, n), float("nan"), dtype=torch.float32, device=DEV)
+    ws = tw.bitnet_sequence_workspace(DEV)
+    c0 = tw.bitnet_launch_count()
+    tw.bitnet_decode_sequence([tw.ffn_gate_up_op(x, G["p"], G["g"], U["p"], U["g"], y)], m, ws)
+    torch.cuda.synchronize()
+    assert tw.bitnet_launch_count() - c0 == 1
+    ref = tw.bitnet_ffn_gate_up(x, G["p"], G["g"], U["p"], U["g"])
+    assert torch.equal(y.view(torch.int32), ref.view(torch.int32))
+    cols = np.random.default_rng(703).choice(n, 512, replace=False)
+    Gs = dict(p_ref=G["p_ref"][cols], g_ref=G["g_ref"])
+    Us = dict(p_ref=U["p_ref"][cols], g_ref=U["g_ref"])
+    assert_rel_close(y.cpu().numpy()[:, cols], oracle_ffn(xf, Gs, Us, k))
+    assert torch.count_nonzero(ws) == 0
+
+
+def test_k_above_the_limit_is_rejected(cluster):
     m = 8
-    x = torch.zeros((m, 256), dtype=torch.bfloat16, device=DEV)
-    w = torch.zeros((60000, 64), dtype=torch.uint8, device=DEV)
+    x = torch.zeros((m, 8256), dtype=torch.bfloat16, device=DEV)
+    w = torch.zeros((256, 8256 // 4), dtype=torch.uint8, device=DEV)
     g = torch.ones(4, dtype=torch.float32, device=DEV)
-    y = torch.empty((m, 60000), dtype=torch.float32, device=DEV)
+    y = torch.empty((m, 256), dtype=torch.float32, device=DEV)
     ws = tw.bitnet_sequence_workspace(DEV)
     c0 = tw.bitnet_launch_count()
     with pytest.raises(tw.BitnetError) as e:
-        tw.bitnet_decode_sequence([tw.ffn_gate_up_op(x, w, g, w, g, y)], m, ws)
+        tw.bitnet_decode_sequence([tw.linear_op(x, w, g, y)], m, ws)
     assert e.value.status == tw.BITNET_ERR_UNSUPPORTED_SHAPE
     assert tw.bitnet_launch_count() == c0
+
+
+# ---------------------------------------------------------------- partitions of independent layers
+@pytest.mark.parametrize("parts", [0, 1, 2, 4])
+@pytest.mark.parametrize("m", [1, 8, 13])
+def test_private_layer_stack_partitions_and_slices(m, parts, cluster):
+    """Layers with their own output buffers are independent groups: they run on
+    separate partitions, with projections cut into row slices to fit the
+    smaller partitions.  Every partition count gives the per-op results bit for
+    bit; the oracle checks the gate/up -> down chain on sampled rows."""
+    nl = 4
+    layers = []
+    for l in range(nl):
+        s = 3000 + 100 * l + m
+        L = dict(q=make_weights(H, H, s + 1), o=make_weights(H, H, s + 2), g=make_weights(I, H, s + 3),
+                 u=make_weights(I, H, s + 4), d=make_weights(H, I, s + 5))
+        L["x"] = [make_x(m, H, s + 10 + i) for i in range(3)]
+        L["out"] = {k: torch.full((m, n), float("nan"), dtype=torch.float32, device=DEV)
+                    for k, n in (("q", H), ("o", H), ("h", I), ("down", H))}
+        layers.append(L)
+    ops = []
+    for L in layers:
+        (xq, _), (xo, _), (xg, _) = L["x"]
+        o = L["out"]
+        ops += [tw.linear_op(xq, L["q"]["p"], L["q"]["g"], o["q"]),
+                tw.linear_op(xo, L["o"]["p"], L["o"]["g"], o["o"]),
+                tw.ffn_gate_up_op(xg, L["g"]["p"], L["g"]["g"], L["u"]["p"], L["u"]["g"], o["h"]),
+                tw.linear_op(o["h"], L["d"]["p"], L["d"]["g"], o["down"])]
+    prev = tw.bitnet_set_sequence_partitions(parts)
+    try:
+        lay = tw.bitnet_sequence_layout(ops, m, cluster, 33 if cluster == 4 else 16)
+        ws = run_seq(ops, m)
+    finally:
+        tw.bitnet_set_sequence_partitions(prev)
+    if parts:
+        assert len(lay["part_clusters"]) == parts
+    assert torch.count_nonzero(ws) == 0
+    rows = np.arange(m) if m <= 8 else np.array([0, m // 2, m - 1])
+    for L in layers:
+        (xq, fq), (xo, fo), (xg, fg) = L["x"]
+        o = {k: v.cpu().numpy() for k, v in L["out"].items()}
+        ref_q = tw.bitnet_linear(xq, L["q"]["p"], L["q"]["g"])
+        ref_o = tw.bitnet_linear(xo, L["o"]["p"], L["o"]["g"])
+        ref_h = tw.bitnet_ffn_gate_up(xg, L["g"]["p"], L["g"]["g"], L["u"]["p"], L["u"]["g"])
+        ref_d = tw.bitnet_linear(ref_h, L["d"]["p"], L["d"]["g"])
+        for got, ref in ((o["q"], ref_q), (o["o"], ref_o), (o["h"], ref_h), (o["down"], ref_d)):
+            assert np.array_equal(got.view(np.uint32), ref.cpu().numpy().view(np.uint32))
+        assert_rel_close(o["h"][rows], oracle_ffn(fg[rows], L["g"], L["u"], H))
+        assert_rel_close(o["down"][rows], oracle_linear(o["h"][rows], L["d"], I))

@@ -275,3 +275,80 @@ def test_cluster_size_setter():
         assert tw.bitnet_set_sequence_cluster(4) == 4
     finally:
         tw.bitnet_set_sequence_cluster(prev)
+
+
+# ---------------------------------------------------------------- partitions and row slices
+def producers(ops, m):
+    wx, wy = brute_force(ops, m)
+    return [{w for w in (wx[j], wy[j]) if w >= 0} for j in range(len(ops))]
+
+
+def check_layout(ops, m, L, clusters):
+    n = len(ops)
+    order, part_of, slices = L["order"], L["part_of"], L["slices"]
+    assert sorted(order) == list(range(n)), "order is a permutation of the ops"
+    assert sum(L["part_clusters"]) == clusters and min(L["part_clusters"]) >= 1
+    assert sum(slices) <= 256 and min(slices) >= 1
+    pos = {i: k for k, i in enumerate(order)}
+    for j, pre in enumerate(producers(ops, m)):
+        for i in pre:
+            # every earlier conflicting op runs first, in the same partition
+            assert pos[i] < pos[j] and part_of[pos[i]] == part_of[pos[j]]
+    # partitions never share memory: ops of different partitions never conflict
+    wx, wy = brute_force([ops[i] for i in order], m)
+    for j in range(n):
+        for w in (wx[j], wy[j]):
+            assert w < 0 or part_of[w] == part_of[j]
+
+
+@pytest.mark.parametrize("forced", [0, 1, 2, 3, 4, 8])
+@pytest.mark.parametrize("shared", [True, False], ids=["shared_outputs", "private_outputs"])
+def test_layout_of_the_layer_stack(forced, shared):
+    ops = layer_stack(30, 8, shared_outputs=shared)
+    prev = tw.bitnet_set_sequence_partitions(forced)
+    try:
+        try:
+            L = tw.bitnet_sequence_layout(ops, 8, 4, 33)
+        except tw.BitnetError as e:
+            # more partitions than slices allow (every op cut to fit 4 clusters): refused, never wrong
+            assert forced >= 6 and e.status == tw.BITNET_ERR_UNSUPPORTED_SHAPE
+            return
+    finally:
+        tw.bitnet_set_sequence_partitions(prev)
+    check_layout(ops, 8, L, 33)
+    n_parts = len(L["part_clusters"])
+    if shared:
+        assert n_parts <= 3  # the gate/up -> down chain, the q chain and the o chain
+    if forced:
+        assert n_parts == min(forced, 3 if shared else 120)
+    # a gate/up op and the down op that reads its h share a partition
+    for l in range(30):
+        k_gu, k_dn = L["order"].index(4 * l + 2), L["order"].index(4 * l + 3)
+        assert L["part_of"][k_gu] == L["part_of"][k_dn] and k_gu < k_dn
+
+
+def test_layout_private_outputs_runs_layers_side_by_side():
+    ops = layer_stack(30, 8, shared_outputs=False)
+    L = tw.bitnet_sequence_layout(ops, 8, 4, 33)
+    assert len(L["part_clusters"]) >= 2
+    # big projections are cut into row slices on the smaller partitions
+    k_gu = L["order"].index(2)
+    assert L["slices"][k_gu] >= 2
+
+
+def test_layout_cuts_one_huge_projection_into_slices():
+    m, k, n = 8, 256, 60000
+    ops = [op(tw.BITNET_OP_FFN_GATE_UP, BASE, k, n, BASE + (1 << 30), BASE + (2 << 30), BASE + (3 << 30),
+              BASE + (4 << 30), BASE + (5 << 30))]
+    L = tw.bitnet_sequence_layout(ops, m, 4, 33)
+    assert L["part_clusters"] == [33] and L["slices"][0] >= 2
+    # rows per cluster of each slice within 8 row groups per warp (1024 rows of both matrices)
+    assert 2 * ((-(-(n // L["slices"][0] + 1) // 33) + 15) // 16) <= 64
+
+
+def test_partition_setter():
+    assert tw.bitnet_set_sequence_partitions(2) == 0
+    assert tw.bitnet_set_sequence_partitions(0) == 2
+    with pytest.raises(ValueError):
+        tw.bitnet_set_sequence_partitions(9)
+    assert tw.bitnet_set_sequence_partitions(0) == 0
