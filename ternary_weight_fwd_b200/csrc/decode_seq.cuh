@@ -417,6 +417,12 @@ __device__ __forceinline__ void ds_op(const DsProgram &p, const DsOp &op, int j,
     const int ksn = max(0, min(op.ks, KS - ks0));
     const int own0 = (int)r * op.own_rows;
     const int nown = max(0, min(op.own_rows, R - own0));
+    // Quotients by runtime row counts without integer division: for 0 <= i <
+    // 2^11 and 1 <= d <= 2^10, (i + 0.5) * fl(1/d) lies at least 0.5/d from
+    // every integer while its rounding error stays below 2^-12, so truncation
+    // gives floor(i / d) exactly.
+    const float inv_own = 1.0f / (float)op.own_rows;
+    const float inv_nown = 1.0f / (float)max(nown, 1);
     const int RG = op.rpc / 16;
     const int nrgi = nmat * RG; // row groups of the cluster: rgi = warp + 8 i (matrix rgi / RG)
     const uint32_t box_w = (uint32_t)op.box_w;
@@ -592,7 +598,7 @@ __device__ __forceinline__ void ds_op(const DsProgram &p, const DsOp &op, int j,
                     for (int h = 0; h < 2; ++h) {
                         const int row = rg * 16 + g + 8 * h;
                         if (row < R) {
-                            const int jo = row / op.own_rows, orow = row - jo * op.own_rows;
+                            const int jo = (int)(((float)row + 0.5f) * inv_own), orow = row - jo * op.own_rows;
                             int *blk = part + jo * blk_ints + (mat * 8 + 2 * t4) * orp + orow;
                             blk[0] = a[0][2 * h] + a[1][2 * h] + a[2][2 * h] + a[3][2 * h] - rs0;
                             blk[orp] = a[0][2 * h + 1] + a[1][2 * h + 1] + a[2][2 * h + 1] + a[3][2 * h + 1] - rs1;
@@ -624,7 +630,7 @@ __device__ __forceinline__ void ds_op(const DsProgram &p, const DsOp &op, int j,
 
         // ---- owners: sum the C partials, dequantise, gate, store ----
         for (int idx = tid; idx < nown * mt; idx += DS_COMPUTE) {
-            const int orow = idx % nown, jj = idx / nown;
+            const int jj = (int)(((float)idx + 0.5f) * inv_nown), orow = idx - jj * nown;
             int s0 = 0, s1 = 0;
             for (int src = 0; src < C; ++src) {
                 const int *blk = (src == (int)r ? part + (int)r * blk_ints : recv + src * blk_ints) + jj * orp + orow;
