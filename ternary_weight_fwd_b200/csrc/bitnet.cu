@@ -904,9 +904,10 @@ bitnet_status_t seq_build(DsProgram &p, const bitnet_op_t *ops, int n, int64_t M
             if (p.part_first[q] < 0) return BITNET_ERR_INVALID_ARG;
     }
     // x staging: ops whose x no op of the launch writes alternate between buffers 0 and 1 (the
-    // next one is fetched while the current one runs); ops reading an earlier op's output use
-    // buffer 2 (loaded when their wait is over); ops reusing the previous op's x load nothing.
-    // Rows as long as the largest K slice in the buffer.
+    // next one is fetched while the current one runs); ops reading an earlier op's output are
+    // marked buffer 2 and read their x in place from L2 once their wait is over (no staging);
+    // ops reusing the previous op's x load nothing.  Rows as long as the largest K slice in
+    // the buffer.
     uint32_t pitch[3] = {16, 16, 16};
     int alt[DS_MAX_PARTS] = {0};
     for (int j = 0; j < total; ++j) {
@@ -919,7 +920,7 @@ bitnet_status_t seq_build(DsProgram &p, const bitnet_op_t *ops, int n, int64_t M
             d.xbuf = (uint8_t)alt[q];
             alt[q] ^= 1;
         }
-        pitch[d.xbuf] = std::max(pitch[d.xbuf], (uint32_t)(d.ks * 64 * (d.xf32 ? 4 : 2)));
+        if (d.xbuf != 2) pitch[d.xbuf] = std::max(pitch[d.xbuf], (uint32_t)(d.ks * 64 * (d.xf32 ? 4 : 2)));
     }
     size_t off = DS_HDR;
     for (int b = 0; b < 3; ++b) {
@@ -954,12 +955,13 @@ std::atomic<int> g_seq_parts{0};
 // partitions fit 256 ops at share 1, only 2 at share 2).
 std::atomic<int> g_seq_ring_share{1};
 
-// Estimated duration (µs) of the busiest partition of a built program: per op
-// a fixed exchange / epilogue cost, the x staging, absmax exchange and
-// quantisation unless the op reuses the previous op's, the contraction at
-// ~40 cycles per mma.sync per warp (measured, 1.9 GHz), and a producer's
-// completion latency when an op reads the output of the op just before it; or
-// the weight stream at ~45 GB/s per SM if that takes longer.
+// Estimated duration (µs) of the busiest partition of a built program, from
+// per-phase timestamps of the 30-layer decode step on B200: per op ~2 µs of
+// partial-sum exchange, epilogue and hand-over, ~2 µs more for x, the absmax
+// exchange and quantisation unless the op reuses the previous op's, the
+// contraction at ~0.055 µs per mma.sync per warp, and a producer's completion
+// latency when an op reads the output of the op just before it; or the weight
+// stream at ~45 GB/s per SM if that takes longer.
 double seq_estimate(const DsProgram &p)
 {
     double t_ops[DS_MAX_PARTS] = {0.0}, bytes[DS_MAX_PARTS] = {0.0};
@@ -968,8 +970,8 @@ double seq_estimate(const DsProgram &p)
         for (int j = p.part_first[q]; j >= 0; j = p.ops[j].nxt) {
             const DsOp &d = p.ops[j];
             const double mma_per_warp = (double)d.nmat * (d.rpc / 16) * d.ks * 2.0 / 8.0;
-            double t = 1.3 + mma_per_warp * 0.021;
-            if (!d.reuse) t += 1.6;
+            double t = 2.0 + mma_per_warp * 0.055;
+            if (!d.reuse) t += 2.0;
             if (d.wait_x >= 0 && d.wait_x == prev) t += 2.3;
             t_ops[q] += t;
             bytes[q] += (double)d.nmat * d.N * (d.K / 4);

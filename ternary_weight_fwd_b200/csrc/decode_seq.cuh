@@ -40,7 +40,7 @@
 
 namespace bitnet {
 
-constexpr int DS_MAX_OPS = 256;   // ops per launch, after row slicing (kernel-parameter space)
+constexpr int DS_MAX_OPS = 320;   // ops per launch, after row slicing (kernel-parameter space)
 constexpr int DS_COMPUTE = 256;   // eight compute warps
 constexpr int DS_CONTROL = 128;   // control warps: weight copies and completion signals
 constexpr int DS_THREADS = DS_COMPUTE + DS_CONTROL;
@@ -439,6 +439,10 @@ __device__ __forceinline__ void ds_op(const DsProgram &p, const DsOp &op, int j,
     const float gam0 = op.gamma0[0];
     const float gam1 = nmat == 2 ? op.gamma1[0] : 0.0f;
     const bool reuse = op.reuse != 0; // x_q, tok_s and tok_rs of the previous op stand
+    // x written earlier in this launch (buffer 2) is read in place from L2 by both
+    // passes below instead of being staged: it leaves that shared memory to the ring
+    const bool direct = xb == 2;
+    const int esz = xf32 ? 4 : 2;
 
     for (int m0 = 0; m0 < p.M; m0 += 8, ++st.tile) {
         const int mt = min(8, p.M - m0);
@@ -459,9 +463,8 @@ __device__ __forceinline__ void ds_op(const DsProgram &p, const DsOp &op, int j,
                     st.ok = wait_count(&p.counters[op.wait_x], target) && st.ok;
                 }
                 __syncwarp();
-                asm volatile("fence.proxy.async.global;" ::: "memory"); // generic writes -> bulk copy reads
             }
-            ds_load_x(p, op, smem, xb, m0, mt, ks0, ksn, lane);
+            if (!direct) ds_load_x(p, op, smem, xb, m0, mt, ks0, ksn, lane);
         }
         if (warp == 7 && m0 == 0 && op.nxt >= 0) {
             // the next op's first tile reads memory no op of this launch writes: fetch it now
@@ -474,18 +477,24 @@ __device__ __forceinline__ void ds_op(const DsProgram &p, const DsOp &op, int j,
         }
 
         if (!reuse) {
-            // ---- partial absmax of this warp's token over the staged slice ----
-            st.ok = mbar_spin(&bar_x[xb], (st.xw >> xb) & 1u) && st.ok;
-            st.xw ^= 1u << xb;
+            // ---- partial absmax of this warp's token over the staged (or in-place) slice ----
+            if (direct) {
+                compute_sync(); // warp 0's acquire of the producer's completion precedes every read
+            } else {
+                st.ok = mbar_spin(&bar_x[xb], (st.xw >> xb) & 1u) && st.ok;
+                st.xw ^= 1u << xb;
+            }
+            const uint4 *src = reinterpret_cast<const uint4 *>(sXs + warp * xs_pitch);
+            const char *gx = static_cast<const char *>(op.x) + ((size_t)(m0 + warp) * op.K + (size_t)ks0 * 64) * esz;
+            auto xchunk = [&](int c) { return direct ? ld_cg_v4(gx + 16 * (size_t)c) : src[c]; };
             float mx = 0.0f;
             if (warp < mt) {
-                const uint4 *src = reinterpret_cast<const uint4 *>(sXs + warp * xs_pitch);
                 if (xf32) {
 #pragma unroll 4
-                    for (int c = lane; c < nchunk; c += 32) mx = fmaxf(mx, chunk_absmax<true>(src[c]));
+                    for (int c = lane; c < nchunk; c += 32) mx = fmaxf(mx, chunk_absmax<true>(xchunk(c)));
                 } else {
 #pragma unroll 4
-                    for (int c = lane; c < nchunk; c += 32) mx = fmaxf(mx, chunk_absmax<false>(src[c]));
+                    for (int c = lane; c < nchunk; c += 32) mx = fmaxf(mx, chunk_absmax<false>(xchunk(c)));
                 }
             }
             mx = warp_max(mx);
@@ -513,16 +522,15 @@ __device__ __forceinline__ void ds_op(const DsProgram &p, const DsOp &op, int j,
                 int rs = 0;
                 if (warp < mt) {
                     const float sc = tok_s[warp];
-                    const uint4 *src = reinterpret_cast<const uint4 *>(sXs + warp * xs_pitch);
                     unsigned char *dst = sXq + warp * p.xq_stride;
                     if (xf32) {
 #pragma unroll 4
                         for (int c = lane; c < nchunk; c += 32)
-                            reinterpret_cast<uint32_t *>(dst)[c] = chunk_quant<true>(src[c], sc, rs).x;
+                            reinterpret_cast<uint32_t *>(dst)[c] = chunk_quant<true>(xchunk(c), sc, rs).x;
                     } else {
 #pragma unroll 4
                         for (int c = lane; c < nchunk; c += 32)
-                            reinterpret_cast<uint2 *>(dst)[c] = chunk_quant<false>(src[c], sc, rs);
+                            reinterpret_cast<uint2 *>(dst)[c] = chunk_quant<false>(xchunk(c), sc, rs);
                     }
                 }
                 rs = warp_sum(rs);

@@ -235,7 +235,7 @@ def test_k_above_the_limit_is_rejected(cluster):
 
 
 # ---------------------------------------------------------------- partitions of independent layers
-@pytest.mark.parametrize("parts", [0, 1, 2, 4])
+@pytest.mark.parametrize("parts", [0, 1, 2, 4, 8])
 @pytest.mark.parametrize("m", [1, 8, 13])
 def test_private_layer_stack_partitions_and_slices(m, parts, cluster):
     """Layers with their own output buffers are independent groups: they run on
