@@ -106,6 +106,7 @@ constexpr int DS_DONE = 708;                       // uint32: ops complete on th
 constexpr int DS_DESC_READY = 712;                 // uint32: op descriptors staged in shared memory
 constexpr int DS_Y_CLEAR = 716;                    // uint32: ops whose y-region ordering wait is satisfied
 constexpr int DS_OP_P0 = 720;                      // uint32 [DS_SLOTS]: first piece of each op in the ring
+constexpr int DS_GAMMA = 768;                      // float [DS_DESC_SLOTS][2]: gammas of the staged ops
 constexpr int DS_DESC = 1024;                      // DsOp [DS_DESC_SLOTS]: this CTA's k-th op in slot k % DS_DESC_SLOTS
 constexpr int DS_DESC_SLOTS = 8;
 
@@ -117,9 +118,13 @@ BITNET_DEVINL const DsOp &ds_desc(unsigned char *smem, int k)
     return *reinterpret_cast<const DsOp *>(smem + DS_DESC + (k % DS_DESC_SLOTS) * (int)sizeof(DsOp));
 }
 
-// Stage op j (program index) as this CTA's k-th op (one thread).
+// Stage op j (program index) as this CTA's k-th op (one thread), with the
+// values of its gammas (read here, well ahead of the op, not on its critical path).
 BITNET_DEVINL void ds_stage_desc(const DsProgram &p, unsigned char *smem, int j, int k)
 {
+    float *gam = reinterpret_cast<float *>(smem + DS_GAMMA) + 2 * (k % DS_DESC_SLOTS);
+    gam[0] = p.ops[j].gamma0[0];
+    gam[1] = p.ops[j].nmat == 2 ? p.ops[j].gamma1[0] : 0.0f;
     const uint4 *src = reinterpret_cast<const uint4 *>(&p.ops[j]);
     uint4 *dst = reinterpret_cast<uint4 *>(smem + DS_DESC + (k % DS_DESC_SLOTS) * (int)sizeof(DsOp));
 #pragma unroll
@@ -421,8 +426,8 @@ __device__ __forceinline__ void ds_op(const DsProgram &p, const DsOp &op, int j,
     // 2^11 and 1 <= d <= 2^10, (i + 0.5) * fl(1/d) lies at least 0.5/d from
     // every integer while its rounding error stays below 2^-12, so truncation
     // gives floor(i / d) exactly.
-    const float inv_own = 1.0f / (float)op.own_rows;
-    const float inv_nown = 1.0f / (float)max(nown, 1);
+    const float inv_own = __frcp_rn((float)op.own_rows); // correctly rounded, as 1.0f / x
+    const float inv_nown = __frcp_rn((float)max(nown, 1));
     const int RG = op.rpc / 16;
     const int nrgi = nmat * RG; // row groups of the cluster: rgi = warp + 8 i (matrix rgi / RG)
     const uint32_t box_w = (uint32_t)op.box_w;
@@ -436,8 +441,9 @@ __device__ __forceinline__ void ds_op(const DsProgram &p, const DsOp &op, int j,
     const uint32_t xs_pitch = p.xs_pitch[xb];
     const unsigned target = (unsigned)(op.ncl * C); // CTAs of this partition (every op it waits for is in it)
 
-    const float gam0 = op.gamma0[0];
-    const float gam1 = nmat == 2 ? op.gamma1[0] : 0.0f;
+    const float *gam = reinterpret_cast<const float *>(smem + DS_GAMMA) + 2 * (k % DS_DESC_SLOTS);
+    const float gam0 = gam[0];
+    const float gam1 = gam[1];
     const bool reuse = op.reuse != 0; // x_q, tok_s and tok_rs of the previous op stand
     // x written earlier in this launch (buffer 2) is read in place from L2 by both
     // passes below instead of being staged: it leaves that shared memory to the ring

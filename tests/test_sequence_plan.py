@@ -288,7 +288,7 @@ def check_layout(ops, m, L, clusters):
     order, part_of, slices = L["order"], L["part_of"], L["slices"]
     assert sorted(order) == list(range(n)), "order is a permutation of the ops"
     assert sum(L["part_clusters"]) == clusters and min(L["part_clusters"]) >= 1
-    assert sum(slices) <= 256 and min(slices) >= 1
+    assert sum(slices) <= 320 and min(slices) >= 1  # kernel ops per launch
     pos = {i: k for k, i in enumerate(order)}
     for j, pre in enumerate(producers(ops, m)):
         for i in pre:
