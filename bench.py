@@ -373,10 +373,23 @@ def time_graph(torch, stream, graph, reps):
     return e0.elapsed_time(e1) / reps
 
 
-def source_digest():
+# The sources each measured kernel family is built from (its device code, the headers that code
+# includes, and the host code that plans and launches it).
+KIND_SOURCES = {
+    "decode_sequence": ["bitnet.cu", "common.cuh", "decode.cuh", "decode_cluster.cuh", "decode_seq.cuh",
+                        "pack_quant.cuh"],
+    "prefill": ["bitnet.cu", "common.cuh", "pack_quant.cuh", "prefill.cuh"],
+}
+
+
+def source_digest(kind=None):
+    """sha256 (first 16 hex digits) of the kernel sources of `kind` (all of csrc/ when None)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "ternary_weight_fwd_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    files = sorted(os.listdir(csrc))
+    if kind is not None:
+        files = sorted(KIND_SOURCES["prefill" if kind.startswith("prefill") else kind])
+    for f in files:
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode())
             h.update(fh.read())
@@ -393,7 +406,7 @@ def dram_traffic(kernel_key):
     except (OSError, ValueError):
         return None
     e = d.get(kernel_key)
-    if not e or e.get("source_digest") != source_digest():
+    if not e or e.get("source_digest") != source_digest(kernel_key):
         return None
     return e.get("bytes_per_launch")
 
