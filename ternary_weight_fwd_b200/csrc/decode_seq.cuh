@@ -33,6 +33,8 @@
 // to finish zeroes them again.  Every wait is bounded (device status word).
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "decode.cuh"
 #include "decode_cluster.cuh"
@@ -570,40 +572,65 @@ __device__ __forceinline__ void ds_op(const DsProgram &p, const DsOp &op, int j,
                 // four independent accumulator chains per row group: k-step parity x k half
                 int a0[4][4] = {}, a1[4][4] = {};
                 if (st.ok && ksn > 0) {
-#pragma unroll 1
-                    for (int ks = 0; ks < ksn; ks += 2) {
-                        const bool has2 = ks + 1 < ksn;
-                        const int kb = has2 ? ks + 1 : ks;
+                    // Branch-free bodies: one variant with the second row group (TWO) and
+                    // one without, pairs of k-steps, then the odd last k-step.
+                    auto kstep_pair = [&](int ks, auto two_c) {
+                        constexpr bool TWO = decltype(two_c)::value;
                         const uint4 xa = lds128(xq_lane + ks * 64);
-                        const uint4 xb2 = lds128(xq_lane + kb * 64);
+                        const uint4 xb2 = lds128(xq_lane + (ks + 1) * 64);
                         const uint32_t la0 = lds32(w0 + ks * 16);
                         const uint32_t ha0 = lds32(w0 + hi_off + ks * 16);
-                        const uint32_t lb0 = lds32(w0 + kb * 16);
-                        const uint32_t hb0 = lds32(w0 + hi_off + kb * 16);
-                        const uint32_t la1 = two ? lds32(w1 + ks * 16) : 0u;
-                        const uint32_t ha1 = two ? lds32(w1 + hi_off + ks * 16) : 0u;
-                        const uint32_t lb1 = two ? lds32(w1 + kb * 16) : 0u;
-                        const uint32_t hb1 = two ? lds32(w1 + hi_off + kb * 16) : 0u;
+                        const uint32_t lb0 = lds32(w0 + (ks + 1) * 16);
+                        const uint32_t hb0 = lds32(w0 + hi_off + (ks + 1) * 16);
+                        uint32_t la1 = 0u, ha1 = 0u, lb1 = 0u, hb1 = 0u;
+                        if constexpr (TWO) {
+                            la1 = lds32(w1 + ks * 16);
+                            ha1 = lds32(w1 + hi_off + ks * 16);
+                            lb1 = lds32(w1 + (ks + 1) * 16);
+                            hb1 = lds32(w1 + hi_off + (ks + 1) * 16);
+                        }
                         mma_u8s8_16832(a0[0], la0 & M3, ha0 & M3, (la0 >> 2) & M3, (ha0 >> 2) & M3, xa.x, xa.y);
                         mma_u8s8_16832(a0[1], (la0 >> 4) & M3, (ha0 >> 4) & M3, (la0 >> 6) & M3, (ha0 >> 6) & M3,
                                        xa.z, xa.w);
-                        if (has2) {
-                            mma_u8s8_16832(a0[2], lb0 & M3, hb0 & M3, (lb0 >> 2) & M3, (hb0 >> 2) & M3, xb2.x, xb2.y);
-                            mma_u8s8_16832(a0[3], (lb0 >> 4) & M3, (hb0 >> 4) & M3, (lb0 >> 6) & M3,
-                                           (hb0 >> 6) & M3, xb2.z, xb2.w);
-                        }
-                        if (two) {
+                        mma_u8s8_16832(a0[2], lb0 & M3, hb0 & M3, (lb0 >> 2) & M3, (hb0 >> 2) & M3, xb2.x, xb2.y);
+                        mma_u8s8_16832(a0[3], (lb0 >> 4) & M3, (hb0 >> 4) & M3, (lb0 >> 6) & M3, (hb0 >> 6) & M3,
+                                       xb2.z, xb2.w);
+                        if constexpr (TWO) {
                             mma_u8s8_16832(a1[0], la1 & M3, ha1 & M3, (la1 >> 2) & M3, (ha1 >> 2) & M3, xa.x, xa.y);
                             mma_u8s8_16832(a1[1], (la1 >> 4) & M3, (ha1 >> 4) & M3, (la1 >> 6) & M3,
                                            (ha1 >> 6) & M3, xa.z, xa.w);
-                            if (has2) {
-                                mma_u8s8_16832(a1[2], lb1 & M3, hb1 & M3, (lb1 >> 2) & M3, (hb1 >> 2) & M3, xb2.x,
-                                               xb2.y);
-                                mma_u8s8_16832(a1[3], (lb1 >> 4) & M3, (hb1 >> 4) & M3, (lb1 >> 6) & M3,
-                                               (hb1 >> 6) & M3, xb2.z, xb2.w);
-                            }
+                            mma_u8s8_16832(a1[2], lb1 & M3, hb1 & M3, (lb1 >> 2) & M3, (hb1 >> 2) & M3, xb2.x,
+                                           xb2.y);
+                            mma_u8s8_16832(a1[3], (lb1 >> 4) & M3, (hb1 >> 4) & M3, (lb1 >> 6) & M3,
+                                           (hb1 >> 6) & M3, xb2.z, xb2.w);
                         }
-                    }
+                    };
+                    auto kstep_last = [&](int ks, auto two_c) {
+                        constexpr bool TWO = decltype(two_c)::value;
+                        const uint4 xa = lds128(xq_lane + ks * 64);
+                        const uint32_t la0 = lds32(w0 + ks * 16);
+                        const uint32_t ha0 = lds32(w0 + hi_off + ks * 16);
+                        mma_u8s8_16832(a0[0], la0 & M3, ha0 & M3, (la0 >> 2) & M3, (ha0 >> 2) & M3, xa.x, xa.y);
+                        mma_u8s8_16832(a0[1], (la0 >> 4) & M3, (ha0 >> 4) & M3, (la0 >> 6) & M3, (ha0 >> 6) & M3,
+                                       xa.z, xa.w);
+                        if constexpr (TWO) {
+                            const uint32_t la1 = lds32(w1 + ks * 16);
+                            const uint32_t ha1 = lds32(w1 + hi_off + ks * 16);
+                            mma_u8s8_16832(a1[0], la1 & M3, ha1 & M3, (la1 >> 2) & M3, (ha1 >> 2) & M3, xa.x, xa.y);
+                            mma_u8s8_16832(a1[1], (la1 >> 4) & M3, (ha1 >> 4) & M3, (la1 >> 6) & M3,
+                                           (ha1 >> 6) & M3, xa.z, xa.w);
+                        }
+                    };
+                    auto run = [&](auto two_c) {
+                        int ks = 0;
+#pragma unroll 1
+                        for (; ks + 1 < ksn; ks += 2) kstep_pair(ks, two_c);
+                        if (ks < ksn) kstep_last(ks, two_c);
+                    };
+                    if (two)
+                        run(std::true_type{});
+                    else
+                        run(std::false_type{});
                 }
                 auto store = [&](const int (&a)[4][4], int rgi) {
                     const int mat = rgi >= RG ? 1 : 0;
