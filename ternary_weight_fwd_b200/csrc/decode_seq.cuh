@@ -329,9 +329,11 @@ __device__ __forceinline__ void ds_issue(const DsProgram &p, unsigned char *smem
             unsigned char *dst0 = smem + p.ring_off + start % p.ring_bytes;
             const uint8_t *w = (mat ? op.w1 : op.w0) + (size_t)n0 * (op.K / 4) + (size_t)ks0 * 16;
             const size_t row_bytes = (size_t)op.K / 4;
-            // (row, chunk) of chunk index c = tid + DS_CONTROL i, advanced incrementally
-            const int dq = DS_CONTROL / ksn, dr = DS_CONTROL % ksn;
-            int kc = tid % ksn, row = tid / ksn;
+            // (row, chunk) of chunk index c = tid + DS_CONTROL i, advanced incrementally; the
+            // quotients by ksn (<= 32) of numbers below 2^11 are exact through a rounded reciprocal
+            const float inv_ksn = __frcp_rn((float)ksn);
+            const int dq = (int)(((float)DS_CONTROL + 0.5f) * inv_ksn), dr = DS_CONTROL - dq * ksn;
+            int row = (int)(((float)tid + 0.5f) * inv_ksn), kc = tid - row * ksn;
             for (int c = tid; c < total; c += DS_CONTROL) {
                 cp_async16(dst0 + (uint32_t)row * op.box_w + kc * 16, w + (size_t)row * row_bytes + (size_t)kc * 16);
                 kc += dr;
@@ -779,7 +781,7 @@ __global__ void __launch_bounds__(DS_THREADS, 1) k_decode_seq(const __grid_const
         cluster_wait();
         cluster_arrive();
     } else {
-        uint32_t head = 0;
+        uint32_t off = 0; // ring offset where the next op's pieces may start (no wrap inside an op)
         DsState st = {0, 0, 0u, true};
         const uint32_t *desc_ready = reinterpret_cast<const uint32_t *>(smem + DS_DESC_READY);
         int prev = -1, k = 0, pieces = 0;
@@ -787,13 +789,14 @@ __global__ void __launch_bounds__(DS_THREADS, 1) k_decode_seq(const __grid_const
             st.ok = wait_local(desc_ready, (uint32_t)k + 1) && st.ok;
             const DsOp &op = ds_desc(smem, k);
             const int nxt = op.nxt; // read before the slot can be restaged (after this op)
-            // ring positions of the op's pieces: the same sequence the control warps place
+            // ring positions of the op's pieces: the sequence the control warps place (ring_place on
+            // monotone positions), kept here as the offset within the ring (no division)
             const uint32_t size = ds_piece_bytes(op);
-            const uint32_t start0 = ring_place(head, size * op.nmat, p.ring_bytes);
-            const uint32_t start1 = start0 + size; // the up projection's piece (gated FFN)
-            head = start0 + size * op.nmat;
-            ds_op(p, op, j, k, prev, pieces, p.ring_off + start0 % p.ring_bytes, p.ring_off + start1 % p.ring_bytes,
-                  smem, st, nxt < 0);
+            const uint32_t total = size * op.nmat;
+            if (off + total > p.ring_bytes) off = 0; // the op would straddle the end: it starts over
+            const uint32_t start0 = off, start1 = off + size; // start1: the up projection's piece (gated FFN)
+            off += total;
+            ds_op(p, op, j, k, prev, pieces, p.ring_off + start0, p.ring_off + start1, smem, st, nxt < 0);
             pieces += op.nmat;
             prev = j;
             j = nxt;
