@@ -382,17 +382,41 @@ KIND_SOURCES = {
 }
 
 
+def strip_comments(src):
+    """C/C++ source without comments and blank lines (string and character literals kept)."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    return "\n".join(l.rstrip() for l in "".join(out).splitlines() if l.strip())
+
+
 def source_digest(kind=None):
-    """sha256 (first 16 hex digits) of the kernel sources of `kind` (all of csrc/ when None)."""
+    """sha256 (first 16 hex digits) of the code of the kernel sources of `kind` (all of csrc/ when
+    None); comments do not count, so a documentation change keeps counters taken on the same code."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "ternary_weight_fwd_b200", "csrc")
     files = sorted(os.listdir(csrc))
     if kind is not None:
         files = sorted(KIND_SOURCES["prefill" if kind.startswith("prefill") else kind])
     for f in files:
-        with open(os.path.join(csrc, f), "rb") as fh:
+        with open(os.path.join(csrc, f), encoding="utf-8") as fh:
             h.update(f.encode())
-            h.update(fh.read())
+            h.update(strip_comments(fh.read()).encode())
     return h.hexdigest()[:16]
 
 
