@@ -27,8 +27,18 @@
 //     overlaps this op's output (write after read / write).  After an op, every
 //     CTA adds one to that op's completion counter (release, device scope);
 //     a dependent op waits (acquire) until the counter reaches the number of
-//     CTAs before it reads x, resp. before it stores y.  Ops run in the same
-//     order on every CTA, so waiting for op i covers every op before i.
+//     CTAs of its partition before it reads x, resp. before it stores y.  Ops
+//     run in the same order on every CTA of a partition, so waiting for op i
+//     covers every op before i;
+//   * groups of ops that share no memory (connected components of the hazard
+//     graph, e.g. the layers of a decode step with their own output buffers)
+//     run side by side on disjoint partitions of the clusters; the host deals
+//     them out by weight bytes and picks the partition count;
+//   * a projection whose weights do not fit a CTA's ring on its partition is
+//     cut into consecutive slices of its output rows, each one op; with one
+//     token tile the later slices reuse the first slice's quantised x;
+//   * an op that reads an earlier op's output reads its x slice in place from
+//     L2 (no staging), which leaves that shared memory to the weight ring.
 // The counters live in a caller-provided zero-filled workspace; the last CTA
 // to finish zeroes them again.  Every wait is bounded (device status word).
 #pragma once
