@@ -374,7 +374,7 @@ def time_graph(torch, stream, graph, reps):
 
 
 # The sources each measured kernel family is built from (its device code, the headers that code
-# includes, and the host code that plans and launches it).
+# includes, and the host code that plans and launches it); include/bitnet.h is always added.
 KIND_SOURCES = {
     "decode_sequence": ["bitnet.cu", "common.cuh", "decode.cuh", "decode_cluster.cuh", "decode_seq.cuh",
                         "pack_quant.cuh"],
@@ -413,9 +413,10 @@ def source_digest(kind=None):
     files = sorted(os.listdir(csrc))
     if kind is not None:
         files = sorted(KIND_SOURCES["prefill" if kind.startswith("prefill") else kind])
-    for f in files:
-        with open(os.path.join(csrc, f), encoding="utf-8") as fh:
-            h.update(f.encode())
+    paths = [os.path.join(csrc, f) for f in files] + [os.path.join(ROOT, "include", "bitnet.h")]
+    for path in paths:
+        with open(path, encoding="utf-8") as fh:
+            h.update(os.path.basename(path).encode())
             h.update(strip_comments(fh.read()).encode())
     return h.hexdigest()[:16]
 

@@ -364,7 +364,11 @@ bitnet_status_t bitnet_sequence_schedule(const bitnet_op_t *ops, int32_t n_ops, 
  * before any ordering wait), and an op waits for another op only where the
  * byte ranges of their activations and outputs overlap (see
  * bitnet_sequence_plan), and independent ops may be reordered (see
- * bitnet_sequence_schedule) with the same results.
+ * bitnet_sequence_schedule) with the same results.  Groups of ops that share
+ * no memory run side by side on disjoint sets of clusters, and projections
+ * too large for one CTA's weight ring there run as consecutive slices of
+ * their output rows (see bitnet_sequence_layout for the plan); neither
+ * changes any result.
  *
  *   ops, n_ops  1 <= n_ops <= BITNET_SEQ_MAX_OPS ops (host array, read
  *               during the call only; the launch keeps its own copy)
@@ -377,8 +381,9 @@ bitnet_status_t bitnet_sequence_schedule(const bitnet_op_t *ops, int32_t n_ops, 
  * Errors (nothing is launched): BITNET_ERR_INVALID_ARG for a null pointer, a
  * bad kind or dtype, an op whose y overlaps its own x, any op's weights or
  * gammas, or the workspace; BITNET_ERR_UNSUPPORTED_SHAPE for K not a
- * multiple of 64 or above 8192, or an op too large for the per-CTA weight
- * slice on this GPU; BITNET_ERR_MISALIGNED; BITNET_ERR_WORKSPACE.
+ * multiple of 64 or above 8192, or a list whose row slices would exceed the
+ * kernel's 320 ops per launch on this GPU (split the list over several
+ * calls); BITNET_ERR_MISALIGNED; BITNET_ERR_WORKSPACE.
  * The launch is stream-ordered (it starts once earlier work on `stream` has
  * finished).  Weights and gammas must not be written by other work while it
  * runs: they are read ahead of every ordering wait.
