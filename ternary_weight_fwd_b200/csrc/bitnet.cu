@@ -815,11 +815,12 @@ int seq_min_slices(int64_t N, int nmat, int ncl)
 // waits for the last slice of the op its user op waits for; later slices of an
 // op need no wait of their own (the first one's wait held on every CTA of the
 // partition), and with one token tile they reuse the first slice's quantised x.
-// too_big: set to the first user op whose weight piece does not fit the ring.
+// too_big (optional, n entries): set to 1 for every user op one of whose
+// slices does not fit the ring, else 0.
 bitnet_status_t seq_build(DsProgram &p, const bitnet_op_t *ops, int n, int64_t M, int C, int G, const SeqParts &parts,
-                          const int32_t *wx, const int32_t *wy, int *too_big = nullptr)
+                          const int32_t *wx, const int32_t *wy, std::vector<char> *too_big = nullptr)
 {
-    if (too_big) *too_big = -1;
+    if (too_big) too_big->assign(n, 0);
     int total = 0;
     for (int i = 0; i < n; ++i) total += parts.slices[i];
     if (total > DS_MAX_OPS) return BITNET_ERR_UNSUPPORTED_SHAPE;
@@ -939,12 +940,13 @@ bitnet_status_t seq_build(DsProgram &p, const bitnet_op_t *ops, int n, int64_t M
     const size_t usable = kSmemLimit - 128; // the kernel aligns its base to 128 bytes
     if (p.ring_off + 4096 > usable) return BITNET_ERR_UNSUPPORTED_SHAPE;
     p.ring_bytes = (uint32_t)((usable - p.ring_off) & ~size_t(127));
+    bool fits = true;
     for (int j = 0; j < total; ++j)
         if ((size_t)ds_piece_bytes(p.ops[j]) * p.ops[j].nmat * parts.ring_share > p.ring_bytes) {
-            if (too_big) *too_big = user_of[j];
-            return BITNET_ERR_UNSUPPORTED_SHAPE;
+            fits = false;
+            if (too_big) (*too_big)[user_of[j]] = 1;
         }
-    return BITNET_OK;
+    return fits ? BITNET_OK : BITNET_ERR_UNSUPPORTED_SHAPE;
 }
 
 // Partition count for decode sequences: 0 = chosen by the cost estimate below.
@@ -1108,15 +1110,21 @@ bitnet_status_t seq_partitioned_build(DsProgram &p, bitnet_op_t *ops, int n, int
         for (int i = 0; i < n; ++i)
             parts.slices[i] = seq_min_slices(ord[i].N, ord[i].kind == BITNET_OP_FFN_GATE_UP ? 2 : 1,
                                              parts.ncl[parts.of[i]]);
-        // cut ops whose pieces do not fit the ring finer until they do (the ring grows as
-        // slices shrink: smaller partial-sum blocks)
+        // cut ops whose pieces do not fit the ring finer until they do: each pass adds one slice
+        // to every op that does not fit (the ring grows as slices shrink, through smaller
+        // partial-sum blocks, so an op is cut no finer than the ring of its pass requires)
         bitnet_status_t st = BITNET_ERR_UNSUPPORTED_SHAPE;
-        for (int iter = 0; iter < 4 * DS_MAX_OPS; ++iter) {
-            int big = -1;
+        std::vector<char> big;
+        for (int pass = 0; pass < 4 * DS_MAX_OPS; ++pass) {
             st = seq_build(cand, ord.data(), n, M, C, G, parts, cwx.data(), cwy.data(), &big);
-            if (st == BITNET_OK || big < 0) break;
-            if (parts.slices[big] >= ord[big].N) break;
-            ++parts.slices[big];
+            if (st == BITNET_OK) break;
+            bool grew = false;
+            for (int i = 0; i < n; ++i)
+                if (big[i] && parts.slices[i] < ord[i].N) {
+                    ++parts.slices[i];
+                    grew = true;
+                }
+            if (!grew) break;
         }
         if (st != BITNET_OK) {
             if (st == BITNET_ERR_INVALID_ARG) return st;
@@ -1150,11 +1158,86 @@ static_assert(4 * (DS_MAX_OPS + 1) <= (int)kSeqWorkspaceBytes, "sequence counter
 static_assert(DS_MAX_OPS >= BITNET_SEQ_MAX_OPS, "sequence op limit: every op fits unsliced");
 static_assert(sizeof(DsProgram) <= 32000, "kernel parameter space");
 
+// Plans of recent sequence calls.  A decode loop calls with the same op list
+// every step; planning it (schedule, partitions, row slices) takes about 2 ms
+// of host time for a 120-op layer stack, the launch itself microseconds.
+struct SeqCacheEntry {
+    bool used = false;
+    uint64_t stamp = 0;
+    int n = 0, dev = -1, C = 0, parts = 0, share = 0;
+    int64_t M = 0;
+    const void *ws = nullptr;
+    bitnet_op_t ops[BITNET_SEQ_MAX_OPS];
+    DsProgram prog;
+};
+constexpr int kSeqCacheEntries = 8;
+SeqCacheEntry g_seq_cache[kSeqCacheEntries];
+std::mutex g_seq_cache_mu;
+uint64_t g_seq_cache_clock = 0;
+
+bool same_op(const bitnet_op_t &a, const bitnet_op_t &b)
+{
+    return a.kind == b.kind && a.x_dtype == b.x_dtype && a.x == b.x && a.K == b.K && a.N == b.N && a.w0 == b.w0 &&
+           a.gamma0 == b.gamma0 && a.w1 == b.w1 && a.gamma1 == b.gamma1 && a.y == b.y;
+}
+
+bool seq_cache_match(const SeqCacheEntry &e, const bitnet_op_t *ops, int n, int64_t M, int dev, int C, int parts,
+                     int share, const void *ws)
+{
+    if (!e.used || e.n != n || e.M != M || e.dev != dev || e.C != C || e.parts != parts || e.share != share ||
+        e.ws != ws)
+        return false;
+    for (int i = 0; i < n; ++i)
+        if (!same_op(e.ops[i], ops[i])) return false;
+    return true;
+}
+
+cudaError_t seq_launch(const DsProgram &p, cudaStream_t stream)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)p.n_ctas);
+    cfg.blockDim = dim3(DS_THREADS);
+    cfg.dynamicSmemBytes = kSmemLimit;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = p.C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return cudaLaunchKernelEx(&cfg, k_decode_seq, p);
+}
+
 bitnet_status_t decode_sequence(const bitnet_op_t *ops, int n, int64_t M, void *workspace, size_t ws_bytes,
                                 cudaStream_t stream)
 {
     if (workspace && !aligned16(workspace)) return BITNET_ERR_MISALIGNED;
+    const int parts_set = g_seq_parts.load(), share_set = g_seq_ring_share.load();
+    // the plan of an op list seen before (validated then) on this device, workspace and settings
+    if (ops && n >= 1 && n <= BITNET_SEQ_MAX_OPS && workspace && ws_bytes >= kSeqWorkspaceBytes) {
+        int dev = -1;
+        if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0) {
+            const int C = g_seq_cluster.load();
+            static DsProgram hit_proto;
+            DsProgram p = hit_proto;
+            bool hit = false;
+            {
+                std::lock_guard<std::mutex> lk(g_seq_cache_mu);
+                for (SeqCacheEntry &e : g_seq_cache)
+                    if (seq_cache_match(e, ops, n, M, dev, C, parts_set, share_set, workspace)) {
+                        p = e.prog;
+                        e.stamp = ++g_seq_cache_clock;
+                        hit = true;
+                        break;
+                    }
+            }
+            if (hit) return cuda_status(seq_launch(p, stream));
+        }
+    }
     int32_t wx[BITNET_SEQ_MAX_OPS], wy[BITNET_SEQ_MAX_OPS], order[BITNET_SEQ_MAX_OPS];
+    const bitnet_op_t *user_ops = ops;
     const ByteRange wsr = workspace ? range_of(workspace, kSeqWorkspaceBytes) : ByteRange{0, 0};
     bitnet_status_t st = seq_schedule(ops, n, M, order, wsr);
     if (st != BITNET_OK) return st;
@@ -1173,20 +1256,30 @@ bitnet_status_t decode_sequence(const bitnet_op_t *ops, int n, int64_t M, void *
     st = seq_partitioned_build(p, sched, n, M, C, G, wx, wy, wsr);
     if (st != BITNET_OK) return st;
     p.counters = static_cast<unsigned *>(workspace);
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(G * C));
-    cfg.blockDim = dim3(DS_THREADS);
-    cfg.dynamicSmemBytes = kSmemLimit;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = C;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    g_launches.fetch_add(1, std::memory_order_relaxed);
-    return cuda_status(cudaLaunchKernelEx(&cfg, k_decode_seq, p));
+    {
+        // remember the plan under the caller's op list (least recently used entry replaced)
+        std::lock_guard<std::mutex> lk(g_seq_cache_mu);
+        SeqCacheEntry *slot = &g_seq_cache[0];
+        for (SeqCacheEntry &e : g_seq_cache) {
+            if (!e.used) {
+                slot = &e;
+                break;
+            }
+            if (e.stamp < slot->stamp) slot = &e;
+        }
+        slot->used = true;
+        slot->stamp = ++g_seq_cache_clock;
+        slot->n = n;
+        slot->M = M;
+        slot->dev = dev;
+        slot->C = C;
+        slot->parts = parts_set;
+        slot->share = share_set;
+        slot->ws = workspace;
+        for (int i = 0; i < n; ++i) slot->ops[i] = user_ops[i];
+        slot->prog = p;
+    }
+    return cuda_status(seq_launch(p, stream));
 }
 
 // ---- fixed scratch for bitnet_linear_noalloc -------------------------------
