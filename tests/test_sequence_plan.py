@@ -356,7 +356,7 @@ def test_partition_setter():
 
 def test_layout_auto_choice_for_the_bench_decode_step():
     """The plan the bench times (30 layers, per-layer outputs, M = 8, 33 clusters of 4): eight
-    partitions of ~4 layers, q / o whole, gate/up in 3-4 row slices, down in 2, 266 kernel ops.
+    partitions of ~4 layers, q / o whole, gate/up in 4-5 row slices, down in 2, 266 kernel ops.
     Measured on B200: 3, 4, 5, 6, 7, 8 partitions -> 434, 432, 404, 385, 405, 368 us per step."""
     ops = layer_stack(30, 8, shared_outputs=False)
     L = tw.bitnet_sequence_layout(ops, 8, 4, 33)
@@ -365,4 +365,4 @@ def test_layout_auto_choice_for_the_bench_decode_step():
     kinds = {}
     for k, i in enumerate(L["order"]):
         kinds.setdefault(i % 4, set()).add(L["slices"][k])
-    assert kinds[0] == {1} and kinds[1] == {1} and kinds[2] <= {3, 4} and kinds[3] == {2}
+    assert kinds[0] == {1} and kinds[1] == {1} and kinds[2] <= {4, 5} and kinds[3] == {2}
