@@ -40,6 +40,7 @@ if ROOT not in sys.path:
 METRIC = "BitLinear GB/s and TOPS (% of HBM / INT8 roofline); decode tokens/s per layer"
 UNIT = "tokens/s per layer"
 HIDDEN, INTER = 2560, 6912
+QKV = HIDDEN + 2 * 640  # fused q, k, v projection of the grouped-query attention (k / v: 2560 -> 640)
 NOMINAL_INT8_PER_BF16 = 2.0  # dense int8 / dense bf16 tensor rate on B200 (4.5 / 2.25 PFLOP/s)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -266,6 +267,7 @@ class Stack:
         self.q_buf = torch.empty((M, HIDDEN), dtype=torch.int8, device=device)
         self.s_buf = torch.empty(M, dtype=torch.float32, device=device)
         self.rs_buf = torch.empty(M, dtype=torch.int32, device=device)
+        self.gen = gen
         # bf16 gate/up -> down chain through the emitted per-token maxima of h
         bf = torch.bfloat16
         self.pre_hb = torch.empty((M, INTER), dtype=bf, device=device)
@@ -275,7 +277,7 @@ class Stack:
         self.dec_db = torch.empty((B, HIDDEN), dtype=bf, device=device)
         self.dec_ha = torch.empty(B, dtype=f32, device=device)
         self.seq_ops = {}
-        self.packed_bytes = sum(p.numel() for L in self.layers for (p, _) in L.values())
+        self.packed_bytes = sum(L[k][0].numel() for L in self.layers for k in ("q", "o", "gate", "up", "down"))
 
     # one projection of each kind -------------------------------------------
     def q(self, l, x, out, ws, s):
@@ -294,6 +296,24 @@ class Stack:
     def down(self, l, out, ws, s):
         L = self.layers[l]
         self.tw.bitnet_linear(out["h"], L["down"][0], L["down"][1], y=out["down"], workspace=ws, stream=s)
+
+    def ensure_qkv(self):
+        """Fused QKV projection weights and outputs, made only when those kinds are timed (after the
+        step), so the step's launch sequence does not change."""
+        if hasattr(self, "pre_qkv"):
+            return
+        torch, tw = self.torch, self.tw
+        for layer in self.layers:
+            w = torch.randn((QKV, HIDDEN), generator=self.gen, device=self.dev, dtype=torch.float32).mul_(0.02)
+            layer["qkv"] = tw.bitnet_pack_weights(w)
+            del w
+        self.dec_qkv = torch.empty((self.a.decode_batch, QKV), dtype=torch.float32, device=self.dev)
+        self.pre_qkv = torch.empty((self.a.prefill_tokens, QKV), dtype=torch.float32, device=self.dev)
+        torch.cuda.synchronize()
+
+    def qkv(self, l, x, out, ws, s):
+        L = self.layers[l]
+        self.tw.bitnet_linear(x, L["qkv"][0], L["qkv"][1], y=out, workspace=ws, stream=s)
 
     def ffn_bf16_chain(self, l, x, hb, ha, db, ws, s):
         """gate/up with bf16 h and its emitted maxima, then down fed those maxima."""
@@ -613,14 +633,36 @@ def our_arm(a, n_gpus):
                                                  for _ in range(R) for l in range(Lyr)],
                                       3 * INTER * HIDDEN // 4 + B * HIDDEN * 2 + 2 * B * INTER * 2 + B * HIDDEN * 2,
                                       "hbm", 0, R * Lyr, False),
+            # fused QKV BitLinear 2560 -> 3840 (q 2560 + k 640 + v 640), not in the step
+            "decode_qkv": (lambda s: [st.qkv(l, st.dec_x[l % st.n_dec], st.dec_qkv, st.ws_dec, s)
+                                      for _ in range(R) for l in range(Lyr)],
+                           QKV * HIDDEN // 4 + B * HIDDEN * 2 + B * QKV * 4, "hbm", 0, R * Lyr, False),
+            "prefill_qkv": (lambda s: [st.qkv(l, st.pre_x[l % st.n_pre], st.pre_qkv, st.ws_pre, s)
+                                       for l in range(Lyr)], 2 * M * QKV * HIDDEN, "tensor", 0, Lyr, False),
         }
         for name, (fn, work, bound, per_step, n_ops, in_step) in specs.items():
             if name == "decode_sequence" and not seq:
                 continue
+            if not in_step:
+                # kinds outside the step run once eagerly first: one that fails is reported, not fatal
+                try:
+                    if name.endswith("_qkv"):
+                        st.ensure_qkv()
+                    fn(stream)
+                    stream.synchronize()
+                except Exception as e:  # noqa: BLE001
+                    kinds[name] = {"error": f"{type(e).__name__}: {e}", "in_step": False, "share_est": 0.0}
+                    continue
             c0 = tw.bitnet_launch_count()
-            g = capture(torch, stream, fn)
-            kern = tw.bitnet_launch_count() - c0
-            ms = time_graph(torch, stream, g, 3) / n_ops
+            try:
+                g = capture(torch, stream, fn)
+                kern = tw.bitnet_launch_count() - c0
+                ms = time_graph(torch, stream, g, 3) / n_ops
+            except Exception as e:  # noqa: BLE001
+                if in_step:
+                    raise
+                kinds[name] = {"error": f"{type(e).__name__}: {e}", "in_step": False, "share_est": 0.0}
+                continue
             reps_step = per_step * (a.decode_steps if name.startswith("decode") else 1)
             kinds[name] = {"us_per_op": ms * 1e3, "kernels_per_op": kern / n_ops, "bound": bound,
                            "work_per_op": work, "in_step": in_step,
