@@ -22,7 +22,11 @@
 //   5. partial int32 sums are scattered to the CTA that owns each output row
 //      (st.async into its shared memory); int32 addition is exact and
 //      order-free, so the result equals the single-CTA contraction;
-//   6. owners finish: dequantise (acc * gamma / s), optional ReLU^2 gate, store.
+//   6. owners finish: dequantise (acc * gamma / s), optional ReLU^2 gate, store
+//      (fp32 or bf16), optionally folding the per-token maxima of the stored
+//      values into a zeroed [M] vector (warp reduction, one atomicMax per CTA).
+// Given per-token maxima of x (from the epilogue of the BitLinear that wrote
+// x) replace step 2's reduction and exchange: every CTA reads them directly.
 // All waits are bounded mbarrier waits; every CTA runs the whole exchange
 // protocol even after a timeout so that no peer is left waiting.
 #pragma once

@@ -6,8 +6,11 @@
 //
 // One persistent CTA per SM, warp-specialised, 448 threads:
 //   warps 0-3  epilogue: tcgen05.ld the int32 tile, dequantise (acc * gamma/s),
-//              optional ReLU^2 gate; 32 x 32 fp32 chunks are staged in
-//              128-byte-swizzled shared memory and written by TMA stores
+//              optional ReLU^2 gate; 32 x 32 chunks are staged in swizzled
+//              shared memory (fp32: 128-byte swizzle; bf16 outputs, rounded to
+//              nearest even: 64-byte swizzle) and written by TMA stores; the
+//              optional per-token maxima of the stored values are folded in
+//              with one integer atomicMax per row and tile
 //   warp 4     producer: TMA (no multicast) of the int8 activation tile
 //              (128 tokens x 128 k, 128-byte swizzle) and of the packed
 //              ternary tile (256 rows x 32 bytes)
