@@ -252,38 +252,74 @@ void oracle_relu2_gate(const double *g, const double *u, int64_t count, double *
  * no formula): y = x / sqrt(mean_k(x_k^2) + eps) * g, with a per-feature
  * weight g and no bias; BitLinear then quantises y per token as above.
  *
- * Order and precision (the page is silent; one ulp in 1/rms can move a
- * quantised code, so this reading fixes them):
- *   S_t = sum of x_k^2 over k = t, t + 256, t + 512, ... in ascending k, in
- *         binary64, for t = 0 .. 255 (x_k^2 of a bf16 or fp32 value is exact);
- *   the partials of each group t = 32w .. 32w + 31 are combined by pairing
- *         halves: P_i = S_i + S_{i+16} (i < 16), then P_i + P_{i+8} (i < 8),
- *         then + P_{i+4}, + P_{i+2}, + P_{i+1}, giving G_w;
- *   ss  = the same pairing over the 8 group sums: G_i + G_{i+4}, + G_{i+2},
- *         + G_{i+1};
+ * Precision (the page is silent; one ulp in 1/rms can move a quantised code,
+ * so this reading fixes it):
+ *   ss  = sum_k x_k^2, the exact sum (every x_k^2 of a binary32 value is an
+ *         exact binary64 number), rounded ONCE to the nearest binary64, ties
+ *         to even -- the correctly rounded sum, independent of any order;
  *   r   = (float)(1 / sqrt(ss / K + eps)), every step in binary64 (correctly
  *         rounded division and square root), rounded once to binary32;
- *   y_k = (x_k * r) * g_k in binary32, two roundings in this order. */
+ *   y_k = (x_k * r) * g_k in binary32, two roundings in this order.
+ *
+ * The exact sum is kept as an integer.  A finite binary32 value is
+ * v = +-mant * 2^(e - 150) with mant < 2^24 an integer and e the biased
+ * exponent field (e = 1 for subnormals, whose mant has no hidden bit), so
+ * v^2 = mant^2 * 2^(2e - 2) * 2^-298: an integer multiple of 2^-298 below
+ * 2^256.  The integers mant^2 * 2^(2e - 2) are added into a long accumulator
+ * of SS_DIGITS little-endian 32-bit digits (640 bits; 2^31 terms need at most
+ * 587), then the accumulator is rounded to 53 significant bits. */
+#define SS_DIGITS 20
 
-/* pair v[i] with v[i + n/2] until one value is left (n a power of two) */
-static double oracle_pairing_sum(double *v, int n)
+/* acc += mant2 * 2^shift, carries propagated (mant2 < 2^48, shift < 512) */
+static void ss_add(uint32_t *acc, uint64_t mant2, int shift)
 {
-    for (int half = n / 2; half >= 1; half /= 2)
-        for (int i = 0; i < half; ++i) v[i] = v[i] + v[i + half];
-    return v[0];
+    const int d = shift / 32, b = shift % 32;
+    const uint64_t lo = mant2 << b;                  /* bits 0..63 of mant2 * 2^b */
+    const uint64_t hi = b ? mant2 >> (64 - b) : 0;    /* bits 64..79 */
+    const uint32_t piece[3] = {(uint32_t)lo, (uint32_t)(lo >> 32), (uint32_t)hi};
+    uint64_t carry = 0;
+    for (int i = 0; d + i < SS_DIGITS; ++i) {
+        const uint64_t t = (uint64_t)acc[d + i] + (i < 3 ? piece[i] : 0) + carry;
+        acc[d + i] = (uint32_t)t;
+        carry = t >> 32;
+        if (i >= 2 && carry == 0) break;
+    }
+}
+
+static int ss_bit(const uint32_t *acc, int i) { return (int)((acc[i / 32] >> (i % 32)) & 1u); }
+
+/* the accumulator times 2^-298, rounded to the nearest binary64, ties to even */
+static double ss_round(const uint32_t *acc)
+{
+    int top = -1; /* position of the highest set bit */
+    for (int i = 32 * SS_DIGITS - 1; i >= 0 && top < 0; --i)
+        if (ss_bit(acc, i)) top = i;
+    if (top < 0) return 0.0;
+    const int sh = top > 52 ? top - 52 : 0; /* bits below the 53 kept ones */
+    uint64_t mant = 0;
+    for (int i = top; i >= sh; --i) mant = (mant << 1) | (uint64_t)ss_bit(acc, i);
+    if (sh > 0) {
+        const int round = ss_bit(acc, sh - 1);
+        int sticky = 0;
+        for (int i = 0; i < sh - 1; ++i) sticky |= ss_bit(acc, i);
+        if (round && (sticky || (mant & 1u))) mant += 1; /* mant <= 2^53: exact in binary64 */
+    }
+    return ldexp((double)mant, sh - 298);
 }
 
 double oracle_sumsq(const float *row, int64_t k_cols)
 {
-    double part[256];
-    for (int t = 0; t < 256; ++t) {
-        double acc = 0.0;
-        for (int64_t k = t; k < k_cols; k += 256) acc += (double)row[k] * (double)row[k];
-        part[t] = acc;
+    uint32_t acc[SS_DIGITS];
+    memset(acc, 0, sizeof(acc));
+    for (int64_t k = 0; k < k_cols; ++k) {
+        uint32_t bits;
+        memcpy(&bits, &row[k], 4);
+        const int field = (int)((bits >> 23) & 0xffu);
+        const uint64_t mant = (bits & 0x7fffffu) | (field ? 0x800000u : 0u);
+        const int e = field ? field : 1;
+        ss_add(acc, mant * mant, 2 * e - 2);
     }
-    double group[8];
-    for (int w = 0; w < 8; ++w) group[w] = oracle_pairing_sum(part + 32 * w, 32);
-    return oracle_pairing_sum(group, 8);
+    return ss_round(acc);
 }
 
 /* x, y: [m_rows][k_cols]; g: [k_cols]; r_out: [m_rows] (may be NULL). */

@@ -374,15 +374,85 @@ def pin_rmsnorm_weight_per_feature():
     assert np.array_equal(yg, (y1 * g[None, :]).astype(np.float32))
 
 
-def pin_rmsnorm_sumsq_rounding_bound():
-    """Against the correctly rounded sum (math.fsum): the binary64 partial/pairing sum of n
-    exact squares is within n * 2^-53 relative; the mean square of the output is
-    mean(x^2) / (mean(x^2) + eps) to fp32 accuracy."""
+def _sq_terms(p):
+    """binary32 values whose squares add up to exactly 2^p."""
+    return [2.0 ** (p // 2)] if p % 2 == 0 else [2.0 ** ((p - 1) // 2)] * 2
+
+
+def _exact_sumsq(row):
+    return sum(Fraction(float(v)) ** 2 for v in row)
+
+
+def _sumsq_rows():
+    """Rows for the sum-of-squares pins: the workloads' rows, wide dynamic ranges, subnormals,
+    one large value among many tiny ones, and exact ties between two binary64 neighbours."""
+    rows = list(synth.bf16_bits_to_f32(synth.activations(4, 2560, 306, "outliers")))
+    rows += list(synth.bf16_bits_to_f32(synth.activations(2, 6912, 307)))
+    rows += list(synth.bf16_bits_to_f32(synth.activations(8, 333, 309, "student_t_rows"))[6:])
+    rng = np.random.default_rng(310)
+    for n in (64, 700, 2560, 6912):
+        rows.append((rng.standard_normal(n) * 2.0 ** rng.integers(-60, 61, n)).astype(np.float32))
+    rows.append((rng.standard_normal(300) * 2.0 ** rng.integers(-149, -126, 300)).astype(np.float32))
+    rows.append(np.array([2.0 ** -149, 3 * 2.0 ** -149, 2.0 ** -126], np.float32))
+    rows.append(np.array([1.0] + [2.0 ** -27] * 4095, np.float32))
+    rows.append(np.array([2.0 ** 100, 2.0 ** -100, -(2.0 ** 60)], np.float32))
+    for v0 in rng.uniform(1.0, 2.0, 6).astype(np.float32):
+        e = math.frexp(float(v0) * float(v0))[1] - 1  # binary64 ulp of v0^2 is 2^(e - 52)
+        rows.append(np.array([v0] + _sq_terms(e - 53), np.float32))                        # tie, even below
+        rows.append(np.array([v0] + _sq_terms(e - 52) + _sq_terms(e - 53), np.float32))    # tie, odd below
+        rows.append(np.array([v0] + _sq_terms(e - 53) + [2.0 ** -40], np.float32))         # just above a tie
+        rows.append(np.array([-v0] + _sq_terms(e - 54), np.float32))                       # below a tie
+    return rows
+
+
+def pin_rmsnorm_sumsq_correctly_rounded():
+    """The sum of squares is the exact sum rounded once to the nearest binary64, ties to even:
+    equal to the exact rational sum converted by Python and to math.fsum of the (exact) squares,
+    two correctly rounded sums that share nothing with the oracle.  The rows include ones on
+    which a binary64 sum in list order, in reverse order or by strided partials gives another
+    value, so no fixed summation order passes."""
+    rows = _sumsq_rows()
+    wrong = {"forward": 0, "reverse": 0, "strided": 0}
+    for row in rows:
+        want = float(_exact_sumsq(row))
+        assert math.fsum(float(v) * float(v) for v in row) == want
+        assert oracle.sumsq(row) == want
+        sq = [float(v) * float(v) for v in row]
+        fwd = 0.0
+        for q in sq:
+            fwd += q
+        rev = 0.0
+        for q in reversed(sq):
+            rev += q
+        part = [0.0] * 256
+        for i, q in enumerate(sq):
+            part[i % 256] += q
+        strided = 0.0
+        for q in part:
+            strided += q
+        wrong["forward"] += fwd != want
+        wrong["reverse"] += rev != want
+        wrong["strided"] += strided != want
+    assert all(v > 0 for v in wrong.values()), wrong
+
+
+def pin_rmsnorm_sumsq_ties_hand_cases():
+    """Hand-worked rounding of 1 + small squares: 1 + 2^-53 is the midpoint between 1 and
+    1 + 2^-52 and goes to the even 1; anything above it goes up; (1 + 2^-23)^2 is exact."""
+    cases = [([1.0, 2.0 ** -27, 2.0 ** -27], 1.0),
+             ([1.0, 2.0 ** -27, 2.0 ** -27, 2.0 ** -60], 1.0 + 2.0 ** -52),
+             ([1.0, 2.0 ** -26, 2.0 ** -27, 2.0 ** -27], 1.0 + 2.0 ** -51),
+             ([1.0 + 2.0 ** -23], 1.0 + 2.0 ** -22 + 2.0 ** -46),
+             ([2.0 ** -149], 2.0 ** -298),
+             ([0.0, -0.0], 0.0)]
+    for row, want in cases:
+        assert oracle.sumsq(np.array(row, np.float32)) == want, row
+
+
+def pin_rmsnorm_output_mean_square():
+    """The mean square of the normalised row is mean(x^2) / (mean(x^2) + eps) to fp32 accuracy."""
     for n, seed in ((2560, 306), (6912, 307), (100, 308), (333, 309)):
         x = synth.bf16_bits_to_f32(synth.activations(2, n, seed, "outliers"))
-        for row in x:
-            exact = math.fsum(float(v) * float(v) for v in row)
-            assert abs(oracle.sumsq(row) - exact) <= n * 2.0 ** -53 * exact
         y, _ = oracle.rmsnorm(x, np.ones(n, np.float32))
         ms = np.mean(x.astype(np.float64) ** 2, axis=1)
         got = np.mean(y.astype(np.float64) ** 2, axis=1)

@@ -50,9 +50,21 @@ MUTANTS = {
                          "(float)(sqrt(ss / (double)k_cols + (double)eps));"),
     "rms_weight_dropped": ("y[m * k_cols + k] = xr * g[k];", "y[m * k_cols + k] = xr;"),
     "rms_weight_first_only": ("y[m * k_cols + k] = xr * g[k];", "y[m * k_cols + k] = xr * g[0];"),
-    "sumsq_stride_255": ("for (int64_t k = t; k < k_cols; k += 256)", "for (int64_t k = t; k < k_cols; k += 255)"),
-    "sumsq_abs": ("acc += (double)row[k] * (double)row[k];", "acc += fabs((double)row[k]);"),
-    "pairing_drops_last_group": ("return oracle_pairing_sum(group, 8);", "return oracle_pairing_sum(group, 4);"),
+    # sum of squares: any fixed binary64 order, a wrong rounding, a lost carry or exponent
+    "sumsq_forward_binary64": ("return ss_round(acc);",
+                               "double f = 0.0; for (int64_t k = 0; k < k_cols; ++k) f += (double)row[k] * (double)row[k]; return f;"),
+    "sumsq_reverse_binary64": ("return ss_round(acc);",
+                               "double f = 0.0; for (int64_t k = k_cols - 1; k >= 0; --k) f += (double)row[k] * (double)row[k]; return f;"),
+    "sumsq_strided_partials": ("return ss_round(acc);",
+                               "double pt[256] = {0}; for (int64_t k = 0; k < k_cols; ++k) pt[k % 256] += (double)row[k] * (double)row[k]; "
+                               "double f = 0.0; for (int t = 0; t < 256; ++t) f += pt[t]; return f;"),
+    "sumsq_ties_away": ("if (round && (sticky || (mant & 1u))) mant += 1;", "if (round) mant += 1;"),
+    "sumsq_truncates": ("if (round && (sticky || (mant & 1u))) mant += 1;", ""),
+    "sumsq_sticky_dropped": ("if (round && (sticky || (mant & 1u)))", "if (round && (mant & 1u))"),
+    "sumsq_carry_lost": ("carry = t >> 32;", "carry = 0;"),
+    "sumsq_subnormal_hidden_bit": ("(field ? 0x800000u : 0u)", "0x800000u"),
+    "sumsq_exponent_off": ("ss_add(acc, mant * mant, 2 * e - 2);", "ss_add(acc, mant * mant, 2 * e);"),
+    "sumsq_abs_not_square": ("ss_add(acc, mant * mant, 2 * e - 2);", "ss_add(acc, mant, e + 149);"),
     "bf16_truncate": ("if (lower > 0x8000u || (lower == 0x8000u && (upper & 1u))) upper += 1u;", ""),
     "bf16_ties_away": ("if (lower > 0x8000u || (lower == 0x8000u && (upper & 1u))) upper += 1u;",
                        "if (lower >= 0x8000u) upper += 1u;"),
