@@ -215,12 +215,11 @@ bitnet_status_t bitnet_ffn_gate_up(const void *x, bitnet_dtype_t x_dtype, int64_
  * rms_norm_eps = 1e-5):
  *   y_k = (x_k * r) * g_k,  r = 1 / sqrt(mean_k(x_k^2) + eps)
  * followed by the per-token absmax quantiser of bitnet_quant_act applied to y.
- * Order and precision are fixed so that results are reproducible: the sum of
- * squares is accumulated in fp64 as 256 partials (partial t sums k = t,
- * t + 256, ... in ascending k), combined by pairing halves within each group
- * of 32 partials (16, 8, 4, 2, 1) and then over the 8 groups (4, 2, 1); r is
- * computed in fp64 with correctly rounded division and square root and
- * rounded once to fp32; y is two fp32 products in the order shown.
+ * Precision is fixed so that results are reproducible: the sum of squares
+ * is the exact sum of the (exact) squares rounded once to the nearest fp64,
+ * ties to even -- independent of any summation order; r is computed in fp64
+ * with correctly rounded division and square root and rounded once to fp32;
+ * y is two fp32 products in the order shown.
  *
  *   x      [M][K] activations of type x_dtype (device, read); K <= 8192
  *   g      [K] fp32 normalisation weight (device, read)

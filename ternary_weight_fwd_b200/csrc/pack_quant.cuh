@@ -7,6 +7,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "exact_sumsq.cuh"
 
 namespace bitnet {
 
@@ -255,19 +256,15 @@ __global__ void __launch_bounds__(128) k_zero_f32(float *__restrict__ amax, int 
 // y = (x * r) * g with r = 1 / sqrt(mean(x^2) + eps), then the quantiser on y.
 // BitNet model page, "Model details" / "Architecture" (subln normalisation, no
 // bias) and BitNetConfig (rms_norm_eps).  Each row is held in registers by
-// 128 or 256 threads, so x is read once.  The sum of squares follows the fixed order of this library's
-// definition: per-thread binary64 partials in ascending k, combined within
-// each warp by pairing halves (16, 8, 4, 2, 1) and then over the 8 warps by
-// pairing halves (4, 2, 1); r is computed in binary64 (correctly rounded
-// division and square root) and rounded once to binary32.
+// 128 or 256 threads, so x is read once.  The sum of squares is the exact sum
+// rounded once to binary64 (exact_sumsq.cuh: 128-bit integer partials, or a
+// long accumulator for rows of very wide range), so no summation order enters
+// the result; r is computed in binary64 (correctly rounded division and square
+// root) and rounded once to binary32.
 // ---------------------------------------------------------------------------
-constexpr int RQ_PARTIALS = 256;      // binary64 partial sums of squares per row (fixed by the definition)
 constexpr int RQ_MAX_PER_THREAD = 32; // elements a thread holds in registers
 
-// TPR threads per row (128 or 256), 256 / TPR rows per CTA; thread t of a row
-// owns partials t + j * TPR (j < 256 / TPR).  Each warp runs the pairing tree
-// once per partial set, so the group sums (and hence every rounding) are those
-// of the definition whatever TPR is.
+// TPR threads per row (128 or 256), 256 / TPR rows per CTA.
 template <bool XF32, int TPR>
 __global__ void __launch_bounds__(256) k_rmsnorm_quant_rows(const void *__restrict__ x, int64_t M, int64_t K,
                                                             const float *__restrict__ g, float eps,
@@ -276,8 +273,10 @@ __global__ void __launch_bounds__(256) k_rmsnorm_quant_rows(const void *__restri
 {
     constexpr int RPC = 256 / TPR;         // rows per CTA
     constexpr int WPR = TPR / 32;          // warps per row
-    constexpr int PSETS = RQ_PARTIALS / TPR; // partial sets per thread
-    __shared__ double red_ss[RPC][8];
+    __shared__ uint64_t red_lo[RPC][WPR], red_hi[RPC][WPR];
+    __shared__ unsigned long long dig[RPC][SS_LONG_DIGITS];
+    __shared__ uint32_t red_e[RPC][WPR];
+    __shared__ int red_fit[RPC][WPR];
     __shared__ float red_max[RPC][WPR];
     __shared__ int red_sum[RPC][WPR];
     __shared__ float bcast[RPC][2];
@@ -289,7 +288,6 @@ __global__ void __launch_bounds__(256) k_rmsnorm_quant_rows(const void *__restri
     const int64_t m = (int64_t)blockIdx.x * RPC + lr;
     const bool live = m < M;
     float v[RQ_MAX_PER_THREAD];
-    // element e of this thread: partial set j = e % PSETS, step i = e / PSETS, k = t + j * TPR + 256 i
     const int n = live ? (int)((K + TPR - 1 - t) / TPR) : 0; // elements k = t + TPR * e, e < n
     if constexpr (XF32) {
         const float *row = static_cast<const float *>(x) + (live ? m : 0) * K;
@@ -302,23 +300,60 @@ __global__ void __launch_bounds__(256) k_rmsnorm_quant_rows(const void *__restri
         for (int e = 0; e < RQ_MAX_PER_THREAD; ++e)
             if (e < n) v[e] = __uint_as_float((uint32_t)__ldg(row + t + (int64_t)e * TPR) << 16);
     }
-    // partial j holds k = t + j * TPR + 256 i = t + TPR * (j + PSETS * i), i.e. e = j + PSETS * i
+    // largest exponent of the row (anchors the 128-bit window)
+    uint32_t emax = 0;
 #pragma unroll
-    for (int j = 0; j < PSETS; ++j) {
-        double part = 0.0;
+    for (int e = 0; e < RQ_MAX_PER_THREAD; ++e)
+        if (e < n) emax = max(emax, ss_exponent(v[e]));
+    emax = __reduce_max_sync(0xffffffffu, emax);
+    if (lane == 0) red_e[lr][wr] = emax;
+    if (t < SS_LONG_DIGITS) dig[lr][t] = 0ull;
+    __syncthreads();
+    uint32_t E = 0;
 #pragma unroll
-        for (int e = j; e < RQ_MAX_PER_THREAD; e += PSETS)
-            if (e < n) part = __dadd_rn(part, __dmul_rn((double)v[e], (double)v[e]));
-        for (int d = 16; d >= 1; d >>= 1) part = __dadd_rn(part, __shfl_down_sync(0xffffffffu, part, d));
-        if (lane == 0) red_ss[lr][wr + j * WPR] = part; // group (t + j * TPR) / 32
+    for (int w = 0; w < WPR; ++w) E = max(E, red_e[lr][w]);
+    SsWindow acc;
+    if (E != 0) {
+#pragma unroll
+        for (int e = 0; e < RQ_MAX_PER_THREAD; ++e)
+            if (e < n) ss_window_add(acc, v[e], E);
+    }
+    ss_warp_sum(acc.lo, acc.hi);
+    const bool fits = __all_sync(0xffffffffu, acc.fits);
+    if (lane == 0) {
+        red_lo[lr][wr] = acc.lo;
+        red_hi[lr][wr] = acc.hi;
+        red_fit[lr][wr] = fits ? 1 : 0;
     }
     __syncthreads();
+    // a row with a value too far below its largest takes the long accumulator
+    bool row_slow = false, any_slow = false;
+#pragma unroll
+    for (int q = 0; q < RPC; ++q) {
+        bool f = true;
+#pragma unroll
+        for (int w = 0; w < WPR; ++w) f = f && red_fit[q][w] != 0;
+        if (q == lr) row_slow = !f;
+        any_slow = any_slow || !f;
+    }
+    if (any_slow) { // uniform over the CTA
+        if (row_slow) {
+#pragma unroll
+            for (int e = 0; e < RQ_MAX_PER_THREAD; ++e)
+                if (e < n) ss_long_add(dig[lr], v[e]);
+        }
+        __syncthreads();
+    }
     if (t == 0) {
-        double gsum[8];
-        for (int w = 0; w < 8; ++w) gsum[w] = red_ss[lr][w];
-        for (int half = 4; half >= 1; half >>= 1)
-            for (int i = 0; i < half; ++i) gsum[i] = __dadd_rn(gsum[i], gsum[i + half]);
-        const double mean = __ddiv_rn(gsum[0], (double)K);
+        double ss;
+        if (row_slow) {
+            ss = ss_long_round(dig[lr]);
+        } else {
+            uint64_t lo = 0, hi = 0;
+            for (int w = 0; w < WPR; ++w) ss_add128(lo, hi, red_lo[lr][w], red_hi[lr][w]);
+            ss = E ? ss_window_round(lo, hi, E) : 0.0;
+        }
+        const double mean = __ddiv_rn(ss, (double)K);
         bcast[lr][0] = __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(mean, (double)eps))));
     }
     __syncthreads();

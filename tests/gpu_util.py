@@ -50,11 +50,12 @@ def assert_rel_close(y_gpu, y_ref, rel=REL_TOL):
 
 
 def sample_rows(m, count, seed):
-    """Row indices for spot checks: both ends of every 128-row tile edge plus random rows."""
+    """Row indices for spot checks: the first and last row of every 128-row tile, one random
+    row inside every tile, plus random rows up to `count`."""
     r = np.random.default_rng(seed)
     fixed = [0, 1, m - 1, m // 2]
-    for t in range(128, m, 128 * 7):
-        fixed += [t - 1, t]
+    for t in range(0, m, 128):
+        fixed += [t, min(t + 127, m - 1), int(r.integers(t, min(t + 128, m)))]
     rows = set(i for i in fixed if 0 <= i < m)
     while len(rows) < min(count, m):
         rows.add(int(r.integers(0, m)))

@@ -1,8 +1,11 @@
 """RMS normalisation fused in front of the quantiser, on the GPU through the C ABI.
 
 Bit-exact against the oracle: x_q, per-token scales, row sums and int32
-accumulators; BitLinear / FFN outputs within 1e-6 relative.  The oracle takes
-the same reduction order (see the C header), so equality is exact."""
+accumulators; BitLinear / FFN outputs within 1e-6 relative.  Both sides use
+the correctly rounded sum of squares (the exact sum rounded once), so no
+reduction order enters and equality is exact."""
+import math
+
 import numpy as np
 import pytest
 import torch
@@ -58,6 +61,54 @@ def test_rmsnorm_quant_special_rows():
     assert np.array_equal(x_q.cpu().numpy(), rq)
     assert np.array_equal(s.cpu().numpy().view(np.uint32), rsc.view(np.uint32))
     assert np.all(x_q.cpu().numpy()[1] == 0)
+
+
+def _sq_terms(p):
+    """binary32 values whose squares add up to exactly 2^p."""
+    return [2.0 ** (p // 2)] if p % 2 == 0 else [2.0 ** ((p - 1) // 2)] * 2
+
+
+def _range_rows(k, seed):
+    """Rows whose sums of squares need more than a 128-bit window (a value more than 33
+    binades below the largest), rows sitting exactly on a rounding tie of the sum, rows of
+    subnormals, and ordinary rows next to them (two rows share a CTA at K <= 4096)."""
+    rng = np.random.default_rng(seed)
+    rows = []
+    rows.append((rng.standard_normal(k) * 2.0 ** rng.integers(-70, 60, k)).astype(np.float32))
+    rows.append(rng.standard_normal(k).astype(np.float32))
+    r = rng.standard_normal(k).astype(np.float32)
+    r[k // 3] = np.float32(2.0 ** -60)  # one value 60 binades down: long accumulator
+    rows.append(r)
+    rows.append((rng.standard_normal(k) * 2.0 ** rng.integers(-149, -120, k)).astype(np.float32))
+    for v0 in rng.uniform(1.0, 2.0, 3).astype(np.float32):
+        e = math.frexp(float(v0) * float(v0))[1] - 1
+        for terms in (_sq_terms(e - 53), _sq_terms(e - 52) + _sq_terms(e - 53), _sq_terms(e - 53) + [2.0 ** -40]):
+            row = np.zeros(k, np.float32)
+            vals = [v0] + terms
+            row[rng.choice(k, len(vals), replace=False)] = vals
+            rows.append(row)
+    r = np.zeros(k, np.float32)
+    r[0] = 1.0
+    r[1:4096 if k > 4096 else k] = 2.0 ** -27  # one large square among many tiny ones
+    rows.append(r)
+    return np.stack(rows).astype(np.float32)
+
+
+@pytest.mark.parametrize("k", [256, 2560, 6912])
+def test_rmsnorm_sumsq_wide_range_and_ties(k):
+    """Exact sums of squares on rows of every path: the 128-bit window, the long accumulator
+    (values more than 33 binades below the row's largest), exact ties and subnormals."""
+    x_all = _range_rows(k, 950 + k)
+    g = norm_weight(k, 951)
+    for eps in (1e-5, 0.0):
+        # with eps = 0 the subnormal row (index 3) would give 1/rms beyond binary32
+        x = x_all if eps else np.delete(x_all, 3, axis=0)
+        x_q, s, rs = tw.bitnet_rmsnorm_quant(f32_to_dev(x), f32_to_dev(g), eps)
+        torch.cuda.synchronize()
+        rq, rsc, rrs, _, _ = oracle.rmsnorm_quant_act(x, g, eps)
+        assert np.array_equal(x_q.cpu().numpy(), rq)
+        assert np.array_equal(s.cpu().numpy().view(np.uint32), rsc.view(np.uint32))
+        assert np.array_equal(rs.cpu().numpy(), rrs)
 
 
 @pytest.mark.parametrize("m,k,n", [(1, 2560, 2560), (8, 2560, 640), (8, 6912, 2560), (300, 2560, 512), (4096, 2560, 256)])
