@@ -58,8 +58,6 @@ def parse_args():
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--cpu-seconds", type=float, default=10.0, help="budget of the oracle CPU baseline")
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--seq-partitions", type=int, default=0,
-                   help="decode-sequence partition count (0: chosen by the library's planner)")
     p.add_argument("--decode-path", choices=["sequence", "per-op"], default="sequence",
                    help="decode step as one persistent bitnet_decode_sequence launch (default) or one "
                         "bitnet_linear / bitnet_ffn_gate_up call per projection")
@@ -106,7 +104,8 @@ def oracle_layer_sample(tokens, seed=4242):
     import numpy as np
 
     import oracle
-    from ternary_weight_fwd_b200 import synth
+    sys.path.insert(0, os.path.join(os.path.dirname(os.path.abspath(__file__)), "tests"))
+    import synth  # the seeded input generators shared with the tests
 
     mats = {}
     for j, (name, n, k) in enumerate((("q", HIDDEN, HIDDEN), ("o", HIDDEN, HIDDEN), ("gate", INTER, HIDDEN),
@@ -262,7 +261,7 @@ class Stack:
         ws = max(tw.bitnet_workspace_size(M, INTER, INTER), tw.bitnet_workspace_size(M, HIDDEN, HIDDEN))
         self.ws_pre = torch.empty(ws, dtype=torch.uint8, device=device)
         self.ws_dec = torch.empty(tw.bitnet_workspace_size(B, INTER, INTER), dtype=torch.uint8, device=device)
-        self.ws_seq = tw.bitnet_sequence_workspace(device)
+        self.ws_seq = tw.bitnet_sequence_workspace(device, 4 * a.layers, B, INTER)
         self.norm_g = (torch.randn(HIDDEN, generator=gen, device=device) * 0.1 + 1.0).float()
         self.q_buf = torch.empty((M, HIDDEN), dtype=torch.int8, device=device)
         self.s_buf = torch.empty(M, dtype=torch.float32, device=device)
@@ -490,7 +489,6 @@ def our_arm(a, n_gpus):
         return reduce_max(v, dist, dev)
 
     st = Stack(a, dev, seed=1234 + rank)
-    st.tw.bitnet_set_sequence_partitions(a.seq_partitions)
     stream = torch.cuda.Stream(device=dev)
     stream.wait_stream(torch.cuda.current_stream())
 

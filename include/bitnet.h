@@ -316,13 +316,20 @@ typedef struct bitnet_op {
     const uint8_t *w1;     /* [N][K/4] packed W_up (FFN only, else NULL) */
     const float *gamma1;   /* [1] (FFN only, else NULL) */
     float *y;              /* [M][N] fp32 output (written): y, or h for the FFN */
+    const float *norm_g;   /* [K] RMS normalisation weight applied to x first (as bitnet_linear_norm), or NULL */
+    float norm_eps;        /* its epsilon (>= 0; used only with norm_g) */
 } bitnet_op_t;
 
 #define BITNET_SEQ_MAX_OPS 128
 #define BITNET_SEQ_MAX_M 64
 
-/* Workspace of bitnet_decode_sequence: completion counters (bytes). */
-size_t bitnet_sequence_workspace_size(void);
+/*
+ * Workspace of bitnet_decode_sequence for up to n_ops ops over M tokens whose
+ * K are at most K_max: completion counters, then per op the quantised
+ * activations ([K/64][Mp][64] int8, Mp = M rounded up to 8, 16, 32 or 64),
+ * scales and row sums.  0 for arguments out of range.
+ */
+size_t bitnet_sequence_workspace_size(int32_t n_ops, int64_t M, int64_t K_max);
 
 /*
  * Host-only planning step of bitnet_decode_sequence (launches nothing, needs
@@ -337,103 +344,95 @@ bitnet_status_t bitnet_sequence_plan(const bitnet_op_t *ops, int32_t n_ops, int6
                                      int32_t *wait_x, int32_t *wait_y);
 
 /*
- * Host-only: the order in which bitnet_decode_sequence runs the ops (launches
- * nothing, needs no GPU).  order[k] = index into ops of the k-th op run.  The
- * order keeps every pair of ops whose byte ranges conflict (see
+ * Host-only: the order in which bitnet_decode_sequence takes the ops up
+ * (launches nothing, needs no GPU).  order[k] = index into ops of the k-th op.
+ * The order keeps every pair of ops whose byte ranges conflict (see
  * bitnet_sequence_plan) in list order, so every op reads, and every output
  * ends up holding, exactly what running the ops in list order gives; only
- * independent ops move.  It follows the list, except that an op reading the
- * output of the op just before it is deferred behind a later ready op (one
- * that conflicts with nothing still unscheduled before it), so the consumer
- * waits less for its producer.
+ * independent ops move.
  */
 bitnet_status_t bitnet_sequence_schedule(const bitnet_op_t *ops, int32_t n_ops, int64_t M, int32_t *order);
 
 /*
  * Run ops[0..n_ops) -- every one a decode-size BitLinear or gated FFN over
- * the same M tokens -- in ONE persistent kernel launch.  The results are
- * bit-identical to calling bitnet_linear / bitnet_ffn_gate_up for each op in
- * order on `stream`: an op whose x is an earlier op's y reads that y, and
- * every output holds what the last op that writes it stored.  The page has
- * no counterpart to this call: it is the decode-step execution of the
- * BitLinear layers that the page's model stacks (page: "Architecture").
+ * the same M tokens, optionally RMS-normalising its input first -- in ONE
+ * persistent kernel launch.  The results are bit-identical to calling
+ * bitnet_linear / bitnet_ffn_gate_up (bitnet_linear_norm /
+ * bitnet_ffn_gate_up_norm when norm_g is set) for each op in order on
+ * `stream`: an op whose x is an earlier op's y reads that y, and every output
+ * holds what the last op that writes it stored.  The page has no counterpart
+ * to this call: it is the decode-step execution of the BitLinear layers that
+ * the page's model stacks (page: "Architecture").
  *
- * Execution: the grid stays resident; each CTA streams its slice of every
- * op's packed weights into shared memory ahead of the op (weights are read
- * before any ordering wait), and an op waits for another op only where the
- * byte ranges of their activations and outputs overlap (see
- * bitnet_sequence_plan), and independent ops may be reordered (see
- * bitnet_sequence_schedule) with the same results.  Groups of ops that share
- * no memory run side by side on disjoint sets of clusters, and projections
- * too large for one CTA's weight ring there run as consecutive slices of
- * their output rows (see bitnet_sequence_layout for the plan); neither
- * changes any result.
+ * Execution: every op is cut into tasks -- one quantisation task per token
+ * (absmax, after the optional RMS normalisation) and one task per 128 packed
+ * weight rows (64 output rows of a gated FFN) over all of K -- and the CTAs of
+ * the launch (one per SM) claim tasks in a fixed order through a counter in
+ * the workspace.  A task waits only for the tasks it depends on: an op's
+ * weight rows for its quantisation tasks, a quantisation task for the rows of
+ * the op that wrote its x, and an op's outputs for the earlier readers and
+ * writers of the same bytes (see bitnet_sequence_tasks).  Weights are
+ * streamed ahead of every wait.  Progress does not depend on how many CTAs
+ * are resident at the same time.
  *
  *   ops, n_ops  1 <= n_ops <= BITNET_SEQ_MAX_OPS ops (host array, read
  *               during the call only; the launch keeps its own copy)
  *   M           tokens, 1 <= M <= BITNET_SEQ_MAX_M, the same for every op
- *   workspace   device memory of bitnet_sequence_workspace_size() bytes,
- *               ZERO-FILLED before its first use; every call leaves it zero
- *               again (also after a device-side timeout).  Calls that may
- *               run at the same time need separate workspaces.
+ *   workspace   device memory of at least
+ *               bitnet_sequence_workspace_size(n_ops, M, max K) bytes whose
+ *               first 4 * (2 + 2 * n_ops) bytes are ZERO before its first use;
+ *               every call leaves them zero again (also after a device-side
+ *               timeout).  Calls that may run at the same time need separate
+ *               workspaces.
  *
  * Errors (nothing is launched): BITNET_ERR_INVALID_ARG for a null pointer, a
- * bad kind or dtype, an op whose y overlaps its own x, any op's weights or
- * gammas, or the workspace; BITNET_ERR_UNSUPPORTED_SHAPE for K not a
- * multiple of 64 or above 8192, or a list whose row slices would exceed the
- * kernel's 320 ops per launch on this GPU (split the list over several
- * calls); BITNET_ERR_MISALIGNED; BITNET_ERR_WORKSPACE.
- * The launch is stream-ordered (it starts once earlier work on `stream` has
- * finished).  Weights and gammas must not be written by other work while it
- * runs: they are read ahead of every ordering wait.
+ * bad kind or dtype, a negative or non-finite norm_eps, an op whose y overlaps
+ * its own x, any op's weights, gammas or norm weight, or the workspace;
+ * BITNET_ERR_UNSUPPORTED_SHAPE for K not a multiple of 64 or above 8192, or an
+ * op that would wait on more than 8 groups of tasks; BITNET_ERR_MISALIGNED;
+ * BITNET_ERR_WORKSPACE.  The launch is stream-ordered (it starts once earlier
+ * work on `stream` has finished).  Weights, gammas and norm weights must not be
+ * written by other work while it runs: they are read ahead of every ordering
+ * wait.
  */
 bitnet_status_t bitnet_decode_sequence(const bitnet_op_t *ops, int32_t n_ops, int64_t M,
                                        void *workspace, size_t ws_bytes, cudaStream_t stream);
 
 /*
- * Cluster size (CTAs splitting K) of the sequence kernel: 4 (default) or 8.
- * Returns the previous value, or -1 if the value is not allowed (nothing
- * changed).  Every size gives bit-identical results.  For tests and tuning;
- * not synchronised with calls running in other threads.
+ * Host-only: the task order bitnet_decode_sequence would launch for `ctas`
+ * CTAs (no device is touched).  The 2 * n_ops task groups -- per op, its
+ * quantisation tasks (kind 0, M tasks) and its weight-row tasks (kind 1) --
+ * in the order the CTAs claim them; for group k:
+ *   group_op[k]     index into ops
+ *   group_kind[k]   0 = quantisation, 1 = weight rows
+ *   group_tasks[k]  number of tasks
+ *   dep_count[k], deps[9k .. 9k + 9)  positions (< k) of the groups that must
+ *                   be complete before it (reduced: none implied by another;
+ *                   a rows group's own quantisation group is always among
+ *                   them, besides at most 8 others), unused entries -1
+ * All arrays have 2 * n_ops entries (deps: 18 * n_ops).
  */
-int bitnet_set_sequence_cluster(int cluster_size);
+bitnet_status_t bitnet_sequence_tasks(const bitnet_op_t *ops, int32_t n_ops, int64_t M, int32_t ctas,
+                                      int32_t *group_op, int32_t *group_kind, int32_t *group_tasks,
+                                      int32_t *dep_count, int32_t *deps);
 
 /*
- * Partition count of the sequence kernel: 0 (default) lets the planner pick
- * the count with the smallest estimated duration; 1 .. 8 forces that count
- * (capped by the number of independent groups of ops).  Returns the previous
- * value, or -1 if the value is not allowed.  Every count gives bit-identical
- * results.  For tests and tuning; not synchronised with other threads.
+ * Tests only (host-armed failure injection, no GPU fault): make the weight-row
+ * tasks of op `op` (index into the list of later bitnet_decode_sequence calls)
+ * wait for one quantisation task more than exist, so that the wait runs out
+ * after the wait limit and the launch ends with BITNET_ERR_TIMEOUT in the
+ * device status word; -1 turns it off.  Returns the previous value (-2 if
+ * op is out of range).
  */
-int bitnet_set_sequence_partitions(int partitions);
+int bitnet_set_sequence_test_stall(int op);
 
 /*
- * Largest share of a CTA's shared-memory weight ring one op of a sequence may
- * occupy: 1 / share, share = 1 .. 4 (default 1).  Projections larger than
- * that are cut into more row slices.  With share >= 2 the next op's weights
- * stream in while an op computes; with 1 fewer, larger slices wait for their
- * weights.  Returns the previous value, or -1 if not allowed.  Every value
- * gives bit-identical results.  For tests and tuning.
+ * Limit of every bounded device-side wait of this library, in nanoseconds (0
+ * restores the default of two seconds).  Returns the previous value, or 0 if
+ * it could not be set.  For tests of the timeout path; synchronises with the
+ * device (a plain copy to device memory).
  */
-int bitnet_set_sequence_ring_share(int share);
-
-/*
- * The plan bitnet_decode_sequence would run, computed on the host only (no
- * device is touched): for `clusters` clusters of `cluster_size` CTAs.
- *   order[k]         index into ops of the k-th op executed
- *   part_of[k]       its partition: a contiguous range of clusters that runs
- *                    only its partition's ops; partitions never wait for each
- *                    other (their ops share no memory)
- *   slices[k]        the number of consecutive kernel ops it is cut into, over
- *                    equal slices of its output rows (each slice's weights fit
- *                    one CTA's shared-memory ring)
- *   n_parts, part_clusters[0 .. n_parts)   partition count and sizes
- * All arrays have n_ops entries (part_clusters: 8).  Errors as
- * bitnet_decode_sequence (BITNET_ERR_UNSUPPORTED_SHAPE when no plan fits).
- */
-bitnet_status_t bitnet_sequence_layout(const bitnet_op_t *ops, int32_t n_ops, int64_t M, int32_t cluster_size,
-                                       int32_t clusters, int32_t *order, int32_t *part_of, int32_t *slices,
-                                       int32_t *n_parts, int32_t *part_clusters);
+uint64_t bitnet_set_wait_limit_ns(uint64_t ns);
 
 /*
  * Device-side status word.  Kernels whose waits are bounded record

@@ -46,7 +46,7 @@ class bitnet_op_t(ctypes.Structure):
     _fields_ = [("kind", ctypes.c_int32), ("x_dtype", ctypes.c_int32), ("x", ctypes.c_void_p),
                 ("K", ctypes.c_int64), ("N", ctypes.c_int64), ("w0", ctypes.c_void_p),
                 ("gamma0", ctypes.c_void_p), ("w1", ctypes.c_void_p), ("gamma1", ctypes.c_void_p),
-                ("y", ctypes.c_void_p)]
+                ("y", ctypes.c_void_p), ("norm_g", ctypes.c_void_p), ("norm_eps", ctypes.c_float)]
 
 
 class BitnetError(RuntimeError):
@@ -82,17 +82,16 @@ def load_library(path: str = LIB_PATH):
         "bitnet_rmsnorm_quant": ([P, I, I64, I64, P, F, P, P, P, P], I),
         "bitnet_linear_norm": ([P, I, I64, I64, P, F, P, P, I64, P, P, P, P, P, SZ, P], I),
         "bitnet_ffn_gate_up_norm": ([P, I, I64, I64, P, F, P, P, P, P, I64, P, P, P, P, SZ, P], I),
-        "bitnet_sequence_workspace_size": ([], SZ),
+        "bitnet_sequence_workspace_size": ([ctypes.c_int32, I64, I64], SZ),
         "bitnet_sequence_plan": ([ctypes.POINTER(bitnet_op_t), ctypes.c_int32, I64,
                                   ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)], I),
         "bitnet_decode_sequence": ([ctypes.POINTER(bitnet_op_t), ctypes.c_int32, I64, P, SZ, P], I),
         "bitnet_sequence_schedule": ([ctypes.POINTER(bitnet_op_t), ctypes.c_int32, I64,
                                       ctypes.POINTER(ctypes.c_int32)], I),
-        "bitnet_set_sequence_cluster": ([I], I),
-        "bitnet_set_sequence_partitions": ([I], I),
-        "bitnet_set_sequence_ring_share": ([I], I),
-        "bitnet_sequence_layout": ([ctypes.POINTER(bitnet_op_t), ctypes.c_int32, I64, ctypes.c_int32, ctypes.c_int32,
-                                    P, P, P, P, P], I),
+        "bitnet_sequence_tasks": ([ctypes.POINTER(bitnet_op_t), ctypes.c_int32, I64, ctypes.c_int32,
+                                   P, P, P, P, P], I),
+        "bitnet_set_sequence_test_stall": ([I], I),
+        "bitnet_set_wait_limit_ns": ([ctypes.c_uint64], ctypes.c_uint64),
         "bitnet_linear_ex": ([P, I, P, P, F, I64, I64, P, P, I64, P, I, P, P, SZ, P], I),
         "bitnet_ffn_gate_up_ex": ([P, I, P, P, F, I64, I64, P, P, P, P, I64, P, I, P, P, SZ, P], I),
     }
@@ -335,17 +334,18 @@ def bitnet_device_status(clear=True, stream=None) -> int:
 
 
 # ---- decode sequences -------------------------------------------------------
-def linear_op(x, w_packed, gamma, y):
-    """Describe y = BitLinear(x) as one op of a decode sequence."""
+def linear_op(x, w_packed, gamma, y, norm_g=None, eps=RMS_EPS):
+    """Describe y = BitLinear(x) (of RMSNorm(x) when norm_g is given) as one op of a decode sequence."""
     return bitnet_op_t(BITNET_OP_LINEAR, _dtype_code(x), x.data_ptr(), x.shape[1], w_packed.shape[0],
-                       w_packed.data_ptr(), gamma.data_ptr(), None, None, y.data_ptr())
+                       w_packed.data_ptr(), gamma.data_ptr(), None, None, y.data_ptr(),
+                       None if norm_g is None else norm_g.data_ptr(), float(eps))
 
 
-def ffn_gate_up_op(x, wg_packed, gamma_g, wu_packed, gamma_u, h):
+def ffn_gate_up_op(x, wg_packed, gamma_g, wu_packed, gamma_u, h, norm_g=None, eps=RMS_EPS):
     """Describe h = relu(BitLinear_g(x))^2 * BitLinear_u(x) as one op of a decode sequence."""
     return bitnet_op_t(BITNET_OP_FFN_GATE_UP, _dtype_code(x), x.data_ptr(), x.shape[1], wg_packed.shape[0],
                        wg_packed.data_ptr(), gamma_g.data_ptr(), wu_packed.data_ptr(), gamma_u.data_ptr(),
-                       h.data_ptr())
+                       h.data_ptr(), None if norm_g is None else norm_g.data_ptr(), float(eps))
 
 
 def _op_array(ops):
@@ -355,13 +355,13 @@ def _op_array(ops):
     return arr
 
 
-def bitnet_sequence_workspace_size() -> int:
-    return load_library().bitnet_sequence_workspace_size()
+def bitnet_sequence_workspace_size(n_ops: int, m: int, k_max: int) -> int:
+    return load_library().bitnet_sequence_workspace_size(int(n_ops), int(m), int(k_max))
 
 
-def bitnet_sequence_workspace(device):
-    """A zero-filled workspace for bitnet_decode_sequence (calls leave it zeroed)."""
-    return torch.zeros(bitnet_sequence_workspace_size(), dtype=torch.uint8, device=device)
+def bitnet_sequence_workspace(device, n_ops=BITNET_SEQ_MAX_OPS, m=BITNET_SEQ_MAX_M, k_max=8192):
+    """A zero-filled workspace for bitnet_decode_sequence (calls leave its counters zeroed)."""
+    return torch.zeros(bitnet_sequence_workspace_size(n_ops, m, k_max), dtype=torch.uint8, device=device)
 
 
 def bitnet_sequence_plan(ops, m):
@@ -375,11 +375,28 @@ def bitnet_sequence_plan(ops, m):
 
 
 def bitnet_sequence_schedule(ops, m):
-    """Host-only: the order (indices into `ops`) in which bitnet_decode_sequence runs them."""
+    """Host-only: the order (indices into `ops`) in which bitnet_decode_sequence takes them up."""
     n = len(ops)
     order = (ctypes.c_int32 * max(1, n))()
     _check(load_library().bitnet_sequence_schedule(_op_array(ops), n, m, order), "bitnet_sequence_schedule")
     return list(order[:n])
+
+
+def bitnet_sequence_tasks(ops, m, ctas):
+    """Host-only task order of a sequence launch on `ctas` CTAs: list of groups
+    dict(op, kind ('quant' | 'rows'), tasks, deps (positions of earlier groups))."""
+    import numpy as np
+    n = len(ops)
+    g_op = np.zeros(2 * n, np.int32)
+    g_kind = np.zeros(2 * n, np.int32)
+    g_tasks = np.zeros(2 * n, np.int32)
+    d_cnt = np.zeros(2 * n, np.int32)
+    deps = np.zeros(18 * n, np.int32)
+    _check(load_library().bitnet_sequence_tasks(_op_array(ops), n, m, int(ctas), g_op.ctypes.data, g_kind.ctypes.data,
+                                                g_tasks.ctypes.data, d_cnt.ctypes.data, deps.ctypes.data),
+           "bitnet_sequence_tasks")
+    return [dict(op=int(g_op[k]), kind="rows" if g_kind[k] else "quant", tasks=int(g_tasks[k]),
+                 deps=[int(d) for d in deps[9 * k:9 * k + d_cnt[k]]]) for k in range(2 * n)]
 
 
 def bitnet_decode_sequence(ops, m, workspace, stream=None):
@@ -388,41 +405,18 @@ def bitnet_decode_sequence(ops, m, workspace, stream=None):
                                                  _stream(stream)), "bitnet_decode_sequence")
 
 
-def bitnet_set_sequence_cluster(cluster_size: int) -> int:
-    prev = load_library().bitnet_set_sequence_cluster(int(cluster_size))
-    if prev < 0:
-        raise ValueError(f"invalid sequence cluster size {cluster_size}")
+def bitnet_set_sequence_test_stall(op: int) -> int:
+    """Tests only: op (list index) whose weight-row tasks wait for a quantisation task that never
+    runs, so the launch ends in a device-side timeout; -1 = off.  Returns the previous value."""
+    prev = load_library().bitnet_set_sequence_test_stall(int(op))
+    if prev < -1:
+        raise ValueError(f"op index out of range: {op}")
     return prev
 
 
-def bitnet_set_sequence_partitions(partitions: int) -> int:
-    """0: partition count chosen by the planner; 1..8: forced.  Returns the previous value."""
-    prev = load_library().bitnet_set_sequence_partitions(int(partitions))
-    if prev < 0:
-        raise ValueError(f"partition count must be 0..8, got {partitions}")
-    return prev
-
-
-def bitnet_sequence_layout(ops, m, cluster_size, clusters):
-    """Host-only plan of a sequence launch: dict(order, part_of, slices, part_clusters)."""
-    import numpy as np
-    n = len(ops)
-    order = np.zeros(n, np.int32)
-    part_of = np.zeros(n, np.int32)
-    slices = np.zeros(n, np.int32)
-    n_parts = np.zeros(1, np.int32)
-    part_cl = np.zeros(8, np.int32)
-    arr = _op_array(ops)
-    _check(load_library().bitnet_sequence_layout(arr, n, m, cluster_size, clusters, order.ctypes.data, part_of.ctypes.data,
-                                                 slices.ctypes.data, n_parts.ctypes.data, part_cl.ctypes.data),
-           "bitnet_sequence_layout")
-    return dict(order=order.tolist(), part_of=part_of.tolist(), slices=slices.tolist(),
-                part_clusters=part_cl[:int(n_parts[0])].tolist())
-
-
-def bitnet_set_sequence_ring_share(share: int) -> int:
-    """Largest share 1/share of the weight ring one sequence op may fill (1..4).  Returns the previous value."""
-    prev = load_library().bitnet_set_sequence_ring_share(int(share))
-    if prev < 0:
-        raise ValueError(f"ring share must be 1..4, got {share}")
+def bitnet_set_wait_limit_ns(ns: int) -> int:
+    """Limit of every bounded device-side wait (0 = default, 2 s).  Returns the previous value."""
+    prev = load_library().bitnet_set_wait_limit_ns(int(ns))
+    if prev == 0:
+        raise RuntimeError("could not set the wait limit")
     return prev

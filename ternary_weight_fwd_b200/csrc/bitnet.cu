@@ -11,6 +11,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <queue>
 #include <utility>
 #include <vector>
 
@@ -18,7 +19,7 @@
 #include "common.cuh"
 #include "decode.cuh"
 #include "decode_cluster.cuh"
-#include "decode_seq.cuh"
+#include "decode_tasks.cuh"
 #include "pack_quant.cuh"
 #include "prefill.cuh"
 
@@ -641,8 +642,7 @@ bitnet_status_t forward(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_
 }
 
 // ---- decode sequences: one persistent launch for many ops -----------------
-std::atomic<int> g_seq_cluster{4};
-constexpr int64_t kSeqMaxK = 64 * DS_MAX_KS * 4; // 8192: at most 32 k-steps per CTA with the smallest cluster (4)
+constexpr int64_t kSeqMaxK = 8192; // a quant task holds a row of x in 256 threads' registers
 
 struct ByteRange {
     uintptr_t lo, hi;
@@ -654,8 +654,8 @@ inline ByteRange range_of(const void *p, size_t bytes)
     return {lo, lo + bytes};
 }
 
-// Validation (host only, shared by plan, schedule and run); fills the byte
-// ranges each op reads (x) and writes (y).  extra: one more range no op may
+// Validation (host only, shared by plan, schedule, tasks and run); fills the
+// byte ranges each op reads (x) and writes (y).  extra: one more range no op may
 // write or read (the workspace), may be empty.
 bitnet_status_t seq_validate(const bitnet_op_t *ops, int n, int64_t M, ByteRange extra, std::vector<ByteRange> &xr,
                              std::vector<ByteRange> &yr)
@@ -664,18 +664,19 @@ bitnet_status_t seq_validate(const bitnet_op_t *ops, int n, int64_t M, ByteRange
     if (M > BITNET_SEQ_MAX_M) return BITNET_ERR_UNSUPPORTED_SHAPE;
     xr.assign(n, ByteRange{0, 0});
     yr.assign(n, ByteRange{0, 0});
-    std::vector<ByteRange> ro; // weights and gammas (read-only for the launch)
-    ro.reserve(4 * (size_t)n);
+    std::vector<ByteRange> ro; // weights, gammas and norm weights (read-only for the launch)
+    ro.reserve(5 * (size_t)n);
     for (int i = 0; i < n; ++i) {
         const bitnet_op_t &o = ops[i];
         if (o.kind != BITNET_OP_LINEAR && o.kind != BITNET_OP_FFN_GATE_UP) return BITNET_ERR_INVALID_ARG;
         if (o.x_dtype != BITNET_DTYPE_BF16 && o.x_dtype != BITNET_DTYPE_F32) return BITNET_ERR_INVALID_ARG;
         const bool ffn = o.kind == BITNET_OP_FFN_GATE_UP;
         if (!o.x || !o.w0 || !o.gamma0 || !o.y || (ffn && (!o.w1 || !o.gamma1))) return BITNET_ERR_INVALID_ARG;
+        if (o.norm_g && !(o.norm_eps >= 0.0f && std::isfinite(o.norm_eps))) return BITNET_ERR_INVALID_ARG;
         const bitnet_status_t st = check_shape(M, o.N, o.K);
         if (st != BITNET_OK) return st;
-        if (o.K > kSeqMaxK) return BITNET_ERR_UNSUPPORTED_SHAPE;
-        const void *ptrs[] = {o.x, o.w0, o.gamma0, ffn ? o.w1 : nullptr, ffn ? o.gamma1 : nullptr, o.y};
+        if (o.K > kSeqMaxK || o.N > 32767 * 64) return BITNET_ERR_UNSUPPORTED_SHAPE;
+        const void *ptrs[] = {o.x, o.w0, o.gamma0, ffn ? o.w1 : nullptr, ffn ? o.gamma1 : nullptr, o.y, o.norm_g};
         for (const void *q : ptrs)
             if (q && !aligned16(q)) return BITNET_ERR_MISALIGNED;
         xr[i] = range_of(o.x, (size_t)M * (size_t)o.K * (o.x_dtype == BITNET_DTYPE_F32 ? 4 : 2));
@@ -688,6 +689,7 @@ bitnet_status_t seq_validate(const bitnet_op_t *ops, int n, int64_t M, ByteRange
             ro.push_back(range_of(o.w1, wbytes));
             ro.push_back(range_of(o.gamma1, 4));
         }
+        if (o.norm_g) ro.push_back(range_of(o.norm_g, (size_t)o.K * 4));
     }
     for (int j = 0; j < n; ++j) {
         for (const ByteRange &w : ro)
@@ -728,8 +730,7 @@ bitnet_status_t seq_plan(const bitnet_op_t *ops, int n, int64_t M, int32_t *wait
 // Execution order (see bitnet_sequence_schedule): a topological order of the
 // hazard graph, so every op reads and leaves exactly what it would in list
 // order.  Greedy, in list order, except that an op reading the output of the
-// op scheduled just before it is deferred while another op is ready: a
-// consumer then waits less for its producer to finish on every CTA.
+// op scheduled just before it is deferred while another op is ready.
 bitnet_status_t seq_schedule(const bitnet_op_t *ops, int n, int64_t M, int32_t *order, ByteRange extra)
 {
     std::vector<ByteRange> xr, yr;
@@ -762,413 +763,236 @@ bitnet_status_t seq_schedule(const bitnet_op_t *ops, int n, int64_t M, int32_t *
     return BITNET_OK;
 }
 
-// Clusters of C CTAs (one CTA per SM) that are resident at once on `dev`.
-int seq_clusters(int dev, int C)
+inline int seq_mp(int64_t M) { return M <= 8 ? 8 : M <= 16 ? 16 : M <= 32 ? 32 : 64; }
+inline int seq_rtasks(const bitnet_op_t &o)
 {
-    static std::atomic<int> cache[kMaxDevices][9];
-    static std::atomic<int> smem_done[kMaxDevices];
-    if (dev < 0 || dev >= kMaxDevices || C < 1 || C > 8) return 0;
-    int v = cache[dev][C].load();
-    if (v > 0) return v;
-    if (ensure_smem(k_decode_seq, kSmemLimit, smem_done, dev) != cudaSuccess) return 0;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(C * 64);
-    cfg.blockDim = dim3(DS_THREADS);
-    cfg.dynamicSmemBytes = kSmemLimit;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = C;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaOccupancyMaxActiveClusters(&v, k_decode_seq, &cfg) != cudaSuccess || v < 1) return 0;
-    cache[dev][C].store(v);
-    return v;
+    const int64_t rows_per_task = o.kind == BITNET_OP_FFN_GATE_UP ? DT_ROWS / 2 : DT_ROWS;
+    return (int)cdiv(o.N, rows_per_task);
 }
 
-// Partitions of the grid: user op i runs on clusters [cl0[of[i]], cl0[of[i]] +
-// ncl[of[i]]) as slices[i] consecutive ops over slices of its output rows.
-struct SeqParts {
-    int n = 1;
-    int cl0[DS_MAX_PARTS] = {0}, ncl[DS_MAX_PARTS] = {0};
-    std::vector<int> of;     // partition of each user op
-    std::vector<int> slices; // row slices of each user op
-    int ring_share = 1;      // an op's weights may fill 1 / ring_share of the ring
+// Task groups of a sequence (ops in execution order): group 2j = the quant
+// tasks of op j (one per token), group 2j + 1 = its row tasks.  Dependencies
+// between groups (must complete first):
+//   rows(j)  <- quant(j)                                  (always; implicit)
+//   quant(j) <- rows(i),  i < j, y_i overlaps x_j         (read after write)
+//   rows(j)  <- quant(i), i < j, x_i overlaps y_j         (write after read: quant(i) is x_i's only reader)
+//   rows(j)  <- rows(i),  i < j, y_i overlaps y_j         (write after write)
+// reduced to the edges not implied by others.  [0, 2n) is a topological order.
+struct SeqGroups {
+    std::vector<std::vector<int>> preds; // reduced predecessors of every group
 };
 
-// Rows per cluster of `rows` output rows spread over ncl clusters.
-inline int seq_rpc(int64_t rows, int ncl) { return (int)align_up((size_t)cdiv(rows, ncl), 16); }
-
-// Fewest row slices of an op (nmat matrices, N rows) for which every warp holds
-// at most DS_RGW row groups on ncl clusters.
-int seq_min_slices(int64_t N, int nmat, int ncl)
-{
-    int s = 1;
-    while ((int64_t)nmat * (seq_rpc(cdiv(N, s), ncl) / 16) > 8 * DS_RGW) ++s;
-    return s;
-}
-
-// Per-op layout and the launch-wide shared-memory map for G clusters of C CTAs.
-// The user ops (in execution order, waits wx / wy between them) are cut into
-// parts.slices[i] consecutive ops over slices of their output rows.  A slice
-// waits for the last slice of the op its user op waits for; later slices of an
-// op need no wait of their own (the first one's wait held on every CTA of the
-// partition), and with one token tile they reuse the first slice's quantised x.
-// too_big (optional, n entries): set to 1 for every user op one of whose
-// slices does not fit the ring, else 0.
-bitnet_status_t seq_build(DsProgram &p, const bitnet_op_t *ops, int n, int64_t M, int C, int G, const SeqParts &parts,
-                          const int32_t *wx, const int32_t *wy, std::vector<char> *too_big = nullptr)
-{
-    if (too_big) too_big->assign(n, 0);
-    int total = 0;
-    for (int i = 0; i < n; ++i) total += parts.slices[i];
-    if (total > DS_MAX_OPS) return BITNET_ERR_UNSUPPORTED_SHAPE;
-    std::vector<int> last_of(n), user_of(total);
-    int ks_max = 1;
-    uint32_t blk_max = 0;
-    int idx = 0;
-    for (int i = 0; i < n; ++i) {
-        const bitnet_op_t &o = ops[i];
-        const int part = parts.of[i];
-        const int ncl = parts.ncl[part];
-        const int nmat = o.kind == BITNET_OP_FFN_GATE_UP ? 2 : 1;
-        const int KS = (int)(o.K / 64);
-        const int ks = (int)cdiv(KS, C);
-        if (ks > DS_MAX_KS) return BITNET_ERR_UNSUPPORTED_SHAPE;
-        const int ns = parts.slices[i];
-        const size_t row_bytes = (size_t)(o.K / 4);
-        for (int t = 0; t < ns; ++t, ++idx) {
-            const int64_t r0 = o.N * t / ns, r1 = o.N * (t + 1) / ns;
-            DsOp &d = p.ops[idx];
-            d = DsOp{};
-            user_of[idx] = i;
-            d.cl0 = (int16_t)parts.cl0[part];
-            d.ncl = (int16_t)ncl;
-            d.ks = (int16_t)ks;
-            const int rpc = seq_rpc(r1 - r0, ncl);
-            if ((int64_t)nmat * (rpc / 16) > 8 * DS_RGW) return BITNET_ERR_UNSUPPORTED_SHAPE;
-            d.rpc = (int16_t)rpc;
-            const int own = rpc / C;
-            int orp = (int)align_up((size_t)own, 4);
-            if (orp % 8 == 0) orp += 4; // token rows of a block land 8 banks apart
-            d.own_rows = (int16_t)own;
-            d.orp = (int16_t)orp;
-            d.box_w = (int16_t)(16 * (ks | 1)); // odd number of 16-byte chunks: conflict-free fragment loads
-            d.x = o.x;
-            d.w0 = o.w0 + (size_t)r0 * row_bytes;
-            d.w1 = nmat == 2 ? o.w1 + (size_t)r0 * row_bytes : nullptr;
-            d.gamma0 = o.gamma0;
-            d.gamma1 = nmat == 2 ? o.gamma1 : nullptr;
-            d.y = o.y + r0;
-            d.K = (int)o.K;
-            d.N = (int)(r1 - r0);
-            d.ldy = (int)o.N;
-            d.nmat = (uint8_t)nmat;
-            d.xf32 = o.x_dtype == BITNET_DTYPE_F32;
-            d.reuse = (t > 0 && M <= 8) ? 1 : 0;
-            d.wait_x = (wx[i] >= 0 && !d.reuse) ? last_of[wx[i]] : -1;
-            d.wait_y = (t == 0 && wy[i] >= 0) ? last_of[wy[i]] : -1;
-            blk_max = std::max(blk_max, (uint32_t)(nmat * 8 * orp * 4));
-        }
-        last_of[i] = idx - 1;
-        ks_max = std::max(ks_max, ks);
-    }
-    p.n_ops = total;
-    p.M = (int)M;
-    p.C = C;
-    p.n_ctas = G * C;
-    // partitions: each runs its ops in program order, linked through DsOp::nxt
-    p.n_parts = parts.n;
-    for (int q = 0; q < parts.n; ++q) {
-        p.part_cl0[q] = parts.cl0[q];
-        p.part_ncl[q] = parts.ncl[q];
-        p.part_first[q] = -1;
-    }
-    {
-        int last[DS_MAX_PARTS];
-        for (int q = 0; q < DS_MAX_PARTS; ++q) last[q] = -1;
-        for (int j = 0; j < total; ++j) {
-            const int i = user_of[j];
-            const int q = parts.of[i];
-            p.ops[j].nxt = -1;
-            if (last[q] < 0)
-                p.part_first[q] = j;
-            else
-                p.ops[last[q]].nxt = j;
-            last[q] = j;
-            // every op an op waits for runs in its partition
-            if ((wx[i] >= 0 && parts.of[wx[i]] != q) || (wy[i] >= 0 && parts.of[wy[i]] != q))
-                return BITNET_ERR_INVALID_ARG;
-        }
-        for (int q = 0; q < parts.n; ++q)
-            if (p.part_first[q] < 0) return BITNET_ERR_INVALID_ARG;
-    }
-    // x staging: ops whose x no op of the launch writes alternate between buffers 0 and 1 (the
-    // next one is fetched while the current one runs); ops reading an earlier op's output are
-    // marked buffer 2 and read their x in place from L2 once their wait is over (no staging);
-    // ops reusing the previous op's x load nothing.  Rows as long as the largest K slice in
-    // the buffer.
-    uint32_t pitch[3] = {16, 16, 16};
-    int alt[DS_MAX_PARTS] = {0};
-    for (int j = 0; j < total; ++j) {
-        DsOp &d = p.ops[j];
-        if (d.reuse) continue;
-        const int q = parts.of[user_of[j]];
-        if (d.wait_x >= 0) {
-            d.xbuf = 2;
-        } else {
-            d.xbuf = (uint8_t)alt[q];
-            alt[q] ^= 1;
-        }
-        if (d.xbuf != 2) pitch[d.xbuf] = std::max(pitch[d.xbuf], (uint32_t)(d.ks * 64 * (d.xf32 ? 4 : 2)));
-    }
-    size_t off = DS_HDR;
-    for (int b = 0; b < 3; ++b) {
-        p.xs_off[b] = (uint32_t)off;
-        p.xs_pitch[b] = pitch[b];
-        off = align_up(off + 8 * (size_t)pitch[b], 128);
-    }
-    uint32_t xs = (uint32_t)ks_max * 64;
-    xs += (uint32_t)(((64 - (int)(xs % 128)) + 128) % 128); // == 64 mod 128
-    p.xq_stride = xs;
-    p.xq_off = (uint32_t)off;
-    p.part_off = (uint32_t)align_up(p.xq_off + 8 * (size_t)xs, 128);
-    const size_t part_bytes = align_up((size_t)C * blk_max, 128);
-    p.recv_off = (uint32_t)(p.part_off + part_bytes);
-    p.ring_off = (uint32_t)(p.recv_off + part_bytes);
-    const size_t usable = kSmemLimit - 128; // the kernel aligns its base to 128 bytes
-    if (p.ring_off + 4096 > usable) return BITNET_ERR_UNSUPPORTED_SHAPE;
-    p.ring_bytes = (uint32_t)((usable - p.ring_off) & ~size_t(127));
-    bool fits = true;
-    for (int j = 0; j < total; ++j)
-        if ((size_t)ds_piece_bytes(p.ops[j]) * p.ops[j].nmat * parts.ring_share > p.ring_bytes) {
-            fits = false;
-            if (too_big) (*too_big)[user_of[j]] = 1;
-        }
-    return fits ? BITNET_OK : BITNET_ERR_UNSUPPORTED_SHAPE;
-}
-
-// Partition count for decode sequences: 0 = chosen by the cost estimate below.
-std::atomic<int> g_seq_parts{0};
-// Share of the weight ring one op may fill (1 = all of it).  Half the ring
-// lets the next op's weights stream in while an op computes, but the extra row
-// slices cost more than the wait (measured on the 30-layer decode step: 4
-// partitions fit 256 ops at share 1, only 2 at share 2).
-std::atomic<int> g_seq_ring_share{1};
-
-// Estimated duration (µs) of the busiest partition of a built program, from
-// per-phase timestamps of the 30-layer decode step on B200: per op ~2 µs of
-// partial-sum exchange, epilogue and hand-over, ~2 µs more for x, the absmax
-// exchange and quantisation unless the op reuses the previous op's, the
-// contraction at ~0.055 µs per mma.sync per warp, and a producer's completion
-// latency when an op reads the output of the op just before it; or the weight
-// stream at ~45 GB/s per SM if that takes longer.
-double seq_estimate(const DsProgram &p)
-{
-    double t_ops[DS_MAX_PARTS] = {0.0}, bytes[DS_MAX_PARTS] = {0.0};
-    for (int q = 0; q < p.n_parts; ++q) {
-        int prev = -1;
-        for (int j = p.part_first[q]; j >= 0; j = p.ops[j].nxt) {
-            const DsOp &d = p.ops[j];
-            const double mma_per_warp = (double)d.nmat * (d.rpc / 16) * d.ks * 2.0 / 8.0;
-            double t = 2.0 + mma_per_warp * 0.055;
-            if (!d.reuse) t += 2.0;
-            if (d.wait_x >= 0 && d.wait_x == prev) t += 2.3;
-            t_ops[q] += t;
-            bytes[q] += (double)d.nmat * d.N * (d.K / 4);
-            prev = j;
-        }
-    }
-    double worst = 0.0;
-    for (int q = 0; q < p.n_parts; ++q) {
-        const double stream_us = bytes[q] / (p.part_ncl[q] * p.C * 45e3);
-        worst = std::max(worst, std::max(t_ops[q], stream_us));
-    }
-    return worst;
-}
-
-// Independent groups of ops run side by side: the connected components of the
-// hazard graph never wait for each other.  For each partition count P (up to
-// DS_MAX_PARTS, or the count set by bitnet_set_sequence_partitions) the
-// components are dealt to P partitions by weight bytes (largest first, to the
-// lightest partition), each partition gets clusters in proportion to its
-// bytes, its ops are re-scheduled among themselves, and each op is cut into
-// the fewest row slices whose weight pieces fit a CTA's ring.  The program with
-// the smallest estimated duration is kept.  ops / wx / wy are rewritten in the
-// chosen execution order.
-// What the planner chose, per op of the returned execution order.
-struct SeqLayout {
-    std::vector<int> perm;    // index of the op in the list the planner was given
-    std::vector<int> part_of; // partition
-    std::vector<int> slices;  // row slices
-};
-
-bitnet_status_t seq_partitioned_build(DsProgram &p, bitnet_op_t *ops, int n, int64_t M, int C, int G, int32_t *wx,
-                                      int32_t *wy, ByteRange extra, SeqLayout *layout = nullptr)
+bitnet_status_t seq_groups(const bitnet_op_t *ops, int n, int64_t M, ByteRange extra, SeqGroups &G)
 {
     std::vector<ByteRange> xr, yr;
-    if (seq_validate(ops, n, M, extra, xr, yr) != BITNET_OK) return BITNET_ERR_INVALID_ARG;
-    // components over the hazards (union-find)
-    std::vector<int> root(n);
-    for (int i = 0; i < n; ++i) root[i] = i;
-    auto find = [&](int i) {
-        while (root[i] != i) i = root[i] = root[root[i]];
-        return i;
-    };
-    for (int j = 0; j < n; ++j)
-        for (int i = 0; i < j; ++i)
-            if (hazard(xr, yr, i, j)) root[find(i)] = find(j);
-    std::vector<double> cbytes(n, 0.0);
-    double total = 0.0;
-    for (int i = 0; i < n; ++i) {
-        const double b = (ops[i].kind == BITNET_OP_FFN_GATE_UP ? 2.0 : 1.0) * (double)ops[i].N * (double)(ops[i].K / 4);
-        cbytes[find(i)] += b;
-        total += b;
-    }
-    std::vector<int> comps;
-    for (int i = 0; i < n; ++i)
-        if (find(i) == i) comps.push_back(i);
-    std::sort(comps.begin(), comps.end(), [&](int a, int b) { return cbytes[a] > cbytes[b] || (cbytes[a] == cbytes[b] && a < b); });
-
-    const int forced = g_seq_parts.load();
-    const int p_max = std::min({DS_MAX_PARTS, G, (int)comps.size()});
-    double best_t = 0.0;
-    bool have = false;
-    static DsProgram cand_proto;
-    DsProgram cand = cand_proto;
-    std::vector<bitnet_op_t> best_ops;
-    std::vector<int32_t> best_wx, best_wy;
-    SeqLayout best_layout;
-    for (int P = 1; P <= p_max; ++P) {
-        if (forced > 0 && P != std::min(forced, p_max)) continue;
-        // components to partitions: largest first, each to the lightest partition
-        std::vector<double> pbytes(P, 0.0);
-        std::vector<int> part_of_root(n, 0);
-        for (int c : comps) {
-            int q = 0;
-            for (int k = 1; k < P; ++k)
-                if (pbytes[k] < pbytes[q]) q = k;
-            part_of_root[c] = q;
-            pbytes[q] += cbytes[c];
-        }
-        // clusters in proportion to bytes, at least one each
-        SeqParts parts;
-        parts.n = P;
-        int used = 0;
-        for (int q = 0; q < P; ++q) {
-            parts.ncl[q] = std::max(1, (int)(G * pbytes[q] / total));
-            used += parts.ncl[q];
-        }
-        while (used > G) { // only when many partitions are tiny
-            int q = 0;
-            for (int k = 1; k < P; ++k)
-                if (parts.ncl[k] > parts.ncl[q]) q = k;
-            --parts.ncl[q];
-            --used;
-        }
-        while (used < G) {
-            int q = 0;
-            for (int k = 1; k < P; ++k)
-                if (pbytes[k] / parts.ncl[k] > pbytes[q] / parts.ncl[q]) q = k;
-            ++parts.ncl[q];
-            ++used;
-        }
-        for (int q = 1; q < P; ++q) parts.cl0[q] = parts.cl0[q - 1] + parts.ncl[q - 1];
-        // execution order: partition by partition, each re-scheduled among its own ops
-        std::vector<bitnet_op_t> ord;
-        std::vector<int> perm;
-        ord.reserve(n);
-        for (int q = 0; q < P; ++q) {
-            std::vector<bitnet_op_t> sub;
-            std::vector<int> sub_idx;
-            for (int i = 0; i < n; ++i)
-                if (part_of_root[find(i)] == q) {
-                    sub.push_back(ops[i]);
-                    sub_idx.push_back(i);
-                }
-            if (sub.empty()) continue;
-            std::vector<int32_t> o(sub.size());
-            if (seq_schedule(sub.data(), (int)sub.size(), M, o.data(), extra) != BITNET_OK) return BITNET_ERR_INVALID_ARG;
-            for (int32_t k : o) {
-                ord.push_back(sub[k]);
-                perm.push_back(sub_idx[k]);
-            }
-        }
-        std::vector<int32_t> cwx(n), cwy(n);
-        if (seq_plan(ord.data(), n, M, cwx.data(), cwy.data(), extra) != BITNET_OK) return BITNET_ERR_INVALID_ARG;
-        // partition of each op in the new order
-        parts.of.assign(n, 0);
-        {
-            int pos = 0;
-            for (int q = 0; q < P; ++q)
-                for (int i = 0; i < n; ++i)
-                    if (part_of_root[find(i)] == q) parts.of[pos++] = q;
-        }
-        parts.ring_share = g_seq_ring_share.load();
-        parts.slices.resize(n);
-        for (int i = 0; i < n; ++i)
-            parts.slices[i] = seq_min_slices(ord[i].N, ord[i].kind == BITNET_OP_FFN_GATE_UP ? 2 : 1,
-                                             parts.ncl[parts.of[i]]);
-        // cut ops whose pieces do not fit the ring finer until they do: each pass adds one slice
-        // to every op that does not fit (the ring grows as slices shrink, through smaller
-        // partial-sum blocks, so an op is cut no finer than the ring of its pass requires)
-        bitnet_status_t st = BITNET_ERR_UNSUPPORTED_SHAPE;
-        std::vector<char> big;
-        for (int pass = 0; pass < 4 * DS_MAX_OPS; ++pass) {
-            st = seq_build(cand, ord.data(), n, M, C, G, parts, cwx.data(), cwy.data(), &big);
-            if (st == BITNET_OK) break;
-            bool grew = false;
-            for (int i = 0; i < n; ++i)
-                if (big[i] && parts.slices[i] < ord[i].N) {
-                    ++parts.slices[i];
-                    grew = true;
-                }
-            if (!grew) break;
-        }
-        if (st != BITNET_OK) {
-            if (st == BITNET_ERR_INVALID_ARG) return st;
-            continue;
-        }
-        const double t = seq_estimate(cand);
-        if (!have || t < best_t) {
-            have = true;
-            best_t = t;
-            p = cand;
-            best_ops = ord;
-            best_wx = cwx;
-            best_wy = cwy;
-            best_layout.perm = perm;
-            best_layout.part_of = parts.of;
-            best_layout.slices = parts.slices;
+    const bitnet_status_t st = seq_validate(ops, n, M, extra, xr, yr);
+    if (st != BITNET_OK) return st;
+    const int ng = 2 * n, words = (ng + 63) / 64;
+    std::vector<std::vector<int>> full(ng);
+    for (int j = 0; j < n; ++j) {
+        full[2 * j + 1].push_back(2 * j);
+        for (int i = 0; i < j; ++i) {
+            if (overlaps(yr[i], xr[j])) full[2 * j].push_back(2 * i + 1);
+            if (overlaps(xr[i], yr[j])) full[2 * j + 1].push_back(2 * i);
+            if (overlaps(yr[i], yr[j])) full[2 * j + 1].push_back(2 * i + 1);
         }
     }
-    if (!have) return BITNET_ERR_UNSUPPORTED_SHAPE;
-    for (int i = 0; i < n; ++i) {
-        ops[i] = best_ops[i];
-        wx[i] = best_wx[i];
-        wy[i] = best_wy[i];
+    std::vector<uint64_t> anc((size_t)ng * words, 0ull); // ancestors of each group (bitset)
+    G.preds.assign(ng, {});
+    for (int v = 0; v < ng; ++v) {
+        uint64_t *av = &anc[(size_t)v * words];
+        for (int u : full[v]) {
+            const uint64_t *au = &anc[(size_t)u * words];
+            for (int w = 0; w < words; ++w) av[w] |= au[w];
+        }
+        for (int u : full[v]) { // u is implied if another predecessor already has it as an ancestor
+            bool implied = false;
+            for (int u2 : full[v])
+                if (u2 != u && ((anc[(size_t)u2 * words + u / 64] >> (u % 64)) & 1ull)) implied = true;
+            if (!implied) G.preds[v].push_back(u);
+        }
+        for (int u : full[v]) av[u / 64] |= 1ull << (u % 64);
     }
-    if (layout) *layout = best_layout;
     return BITNET_OK;
 }
 
-constexpr size_t kSeqWorkspaceBytes = 2048;
-static_assert(4 * (DS_MAX_OPS + 1) <= (int)kSeqWorkspaceBytes, "sequence counters");
-static_assert(DS_MAX_OPS >= BITNET_SEQ_MAX_OPS, "sequence op limit: every op fits unsliced");
-static_assert(sizeof(DsProgram) <= 32000, "kernel parameter space");
+// Order of the task groups in the launch's global task list.  A list-scheduling
+// simulation on `ctas` CTAs: repeatedly take, among the groups whose
+// predecessors are already placed, the one whose predecessors finish first
+// (ties: execution order), and give its tasks to the CTAs that free up first.
+// Durations are estimates (a quant task ~1 us; a row task its packed weights at
+// ~40 GB/s per SM).  CTAs claim tasks in this order, so a dependent group is
+// placed after the work that will be running while its producer finishes.
+std::vector<int> seq_group_order(const bitnet_op_t *ops, int n, int64_t M, const SeqGroups &G, int ctas)
+{
+    const int ng = 2 * n;
+    std::vector<double> finish(ng, 0.0), dur(ng, 0.0);
+    std::vector<int> count(ng, 0), left(ng, 0), order;
+    for (int j = 0; j < n; ++j) {
+        count[2 * j] = (int)M;
+        dur[2 * j] = 1.0;
+        count[2 * j + 1] = seq_rtasks(ops[j]);
+        dur[2 * j + 1] = (double)DT_ROWS * (double)(ops[j].K / 4) / 40e3;
+    }
+    std::vector<std::vector<int>> succ(ng);
+    for (int v = 0; v < ng; ++v) {
+        left[v] = (int)G.preds[v].size();
+        for (int u : G.preds[v]) succ[u].push_back(v);
+    }
+    std::priority_queue<double, std::vector<double>, std::greater<double>> free_at;
+    for (int c = 0; c < std::max(1, ctas); ++c) free_at.push(0.0);
+    std::vector<char> placed(ng, 0);
+    for (int k = 0; k < ng; ++k) {
+        int pick = -1;
+        double best = 0.0;
+        for (int v = 0; v < ng; ++v) {
+            if (placed[v] || left[v] != 0) continue;
+            double ready = 0.0;
+            for (int u : G.preds[v]) ready = std::max(ready, finish[u]);
+            if (pick < 0 || ready < best) {
+                pick = v;
+                best = ready;
+            }
+        }
+        placed[pick] = 1;
+        order.push_back(pick);
+        double fin = best;
+        for (int t = 0; t < count[pick]; ++t) {
+            const double f = free_at.top();
+            free_at.pop();
+            const double end = std::max(f, best) + dur[pick];
+            free_at.push(end);
+            fin = std::max(fin, end);
+        }
+        finish[pick] = fin;
+        for (int v : succ[pick]) --left[v];
+    }
+    return order;
+}
+
+// Workspace: counters, then per op x_q [K/64][Mp][64], s [Mp], row sums [Mp].
+inline size_t seq_counter_bytes(int n) { return align_up(4 * (size_t)(DT_CNT_OPS + 2 * n), 256); }
+inline size_t seq_op_ws_bytes(int64_t K, int Mp) { return align_up((size_t)K * Mp, 256) + 512; }
+
+std::atomic<int> g_seq_stall{-1};                        // tests: op (list index) whose rows never become ready
+std::atomic<unsigned long long> g_wait_limit_set{kDefaultWaitLimitNs};
+
+// Build the launch program for ops in execution order (user_index: list index
+// of each).  ws: workspace (counters zero before the first launch).
+bitnet_status_t seq_build(DtProgram &p, const bitnet_op_t *ops, const int32_t *user_index, int n, int64_t M, int ctas,
+                          void *ws, size_t ws_bytes, ByteRange extra, std::vector<int> *order_out = nullptr)
+{
+    SeqGroups G;
+    bitnet_status_t st = seq_groups(ops, n, M, extra, G);
+    if (st != BITNET_OK) return st;
+    const int Mp = seq_mp(M);
+    size_t need = seq_counter_bytes(n);
+    for (int j = 0; j < n; ++j) need += seq_op_ws_bytes(ops[j].K, Mp);
+    if (ws && ws_bytes < need) return BITNET_ERR_WORKSPACE;
+    p.n_ops = n;
+    p.M = (int)M;
+    p.Mp = Mp;
+    p.counters = static_cast<unsigned *>(ws);
+    char *base = static_cast<char *>(ws);
+    size_t off = seq_counter_bytes(n);
+    const int stall = g_seq_stall.load();
+    for (int j = 0; j < n; ++j) {
+        const bitnet_op_t &o = ops[j];
+        DtOp &d = p.ops[j];
+        d = DtOp{};
+        d.x = o.x;
+        d.w0 = o.w0;
+        d.w1 = o.kind == BITNET_OP_FFN_GATE_UP ? o.w1 : nullptr;
+        d.gamma0 = o.gamma0;
+        d.gamma1 = o.kind == BITNET_OP_FFN_GATE_UP ? o.gamma1 : nullptr;
+        d.norm_g = o.norm_g;
+        d.norm_eps = o.norm_eps;
+        d.y = o.y;
+        d.K = (int)o.K;
+        d.N = (int)o.N;
+        d.nmat = o.kind == BITNET_OP_FFN_GATE_UP ? 2 : 1;
+        d.xf32 = o.x_dtype == BITNET_DTYPE_F32;
+        d.rtasks = seq_rtasks(o);
+        d.stall = (stall >= 0 && user_index && user_index[j] == stall) ? 1 : 0;
+        if (base) {
+            d.xq = reinterpret_cast<int8_t *>(base + off);
+            d.s = reinterpret_cast<float *>(base + off + align_up((size_t)o.K * Mp, 256));
+            d.rs = reinterpret_cast<int32_t *>(base + off + align_up((size_t)o.K * Mp, 256) + 256);
+        }
+        off += seq_op_ws_bytes(o.K, Mp);
+        const std::vector<int> &qp = G.preds[2 * j], &rp = G.preds[2 * j + 1];
+        int nd = 0;
+        for (int u : qp) { // quant(j) waits only on row groups
+            if (nd >= DT_MAX_DEPS) return BITNET_ERR_UNSUPPORTED_SHAPE;
+            d.deps[nd++] = (uint16_t)(u / 2);
+        }
+        d.nq = nd;
+        for (int u : rp) {
+            if (u == 2 * j) continue; // the op's own quant tasks: always waited for
+            if (nd >= DT_MAX_DEPS) return BITNET_ERR_UNSUPPORTED_SHAPE;
+            d.deps[nd++] = (uint16_t)((u / 2) | ((u % 2 == 0) ? DT_DEP_QUANT : 0));
+        }
+        d.nr = nd - d.nq;
+    }
+    const std::vector<int> order = seq_group_order(ops, n, M, G, ctas);
+    int t = 0, ns = 0;
+    for (int v : order) {
+        const int j = v / 2;
+        const bool quant = v % 2 == 0;
+        const int cnt = quant ? (int)M : p.ops[j].rtasks;
+        if (ns >= DT_MAX_SEGS) return BITNET_ERR_UNSUPPORTED_SHAPE;
+        p.segs[ns].start = t;
+        p.segs[ns].op = (uint16_t)j;
+        p.segs[ns].first = (uint16_t)(quant ? 0x8000u : 0u);
+        ++ns;
+        t += cnt;
+    }
+    p.n_segs = ns;
+    p.n_tasks = t;
+    p.slot_bytes = DT_WBYTES + DT_KC * Mp;
+    p.n_slots = (int)std::min<size_t>(DT_MAX_SLOTS, (kSmemLimit - 128 - DT_HDR) / (size_t)p.slot_bytes);
+    if (order_out) *order_out = order;
+    return BITNET_OK;
+}
+
+static_assert(sizeof(DtProgram) <= 32000, "kernel parameter space");
+static_assert(DT_MAX_OPS >= BITNET_SEQ_MAX_OPS && 2 * DT_MAX_OPS <= DT_MAX_SEGS, "sequence limits");
+static_assert(DT_MAX_M >= BITNET_SEQ_MAX_M, "sequence token limit");
+
+template <int TT>
+cudaError_t seq_launch_t(const DtProgram &p, int ctas, cudaStream_t stream, int dev)
+{
+    static std::atomic<int> smem_done[kMaxDevices];
+    cudaError_t e = ensure_smem(k_decode_tasks<TT>, kSmemLimit, smem_done, dev);
+    if (e != cudaSuccess) return e;
+    const size_t smem = 128 + DT_HDR + (size_t)p.n_slots * p.slot_bytes;
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    k_decode_tasks<TT><<<ctas, DT_THREADS, smem, stream>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t seq_launch(const DtProgram &p, int ctas, cudaStream_t stream, int dev)
+{
+    switch (p.Mp) {
+    case 8: return seq_launch_t<1>(p, ctas, stream, dev);
+    case 16: return seq_launch_t<2>(p, ctas, stream, dev);
+    case 32: return seq_launch_t<4>(p, ctas, stream, dev);
+    default: return seq_launch_t<8>(p, ctas, stream, dev);
+    }
+}
 
 // Plans of recent sequence calls.  A decode loop calls with the same op list
-// every step; planning it (schedule, partitions, row slices) takes about 2 ms
-// of host time for a 120-op layer stack, the launch itself microseconds.
+// every step; planning a 120-op layer stack takes on the order of a
+// millisecond of host time, the launch itself microseconds.
 struct SeqCacheEntry {
     bool used = false;
     uint64_t stamp = 0;
-    int n = 0, dev = -1, C = 0, parts = 0, share = 0;
+    int n = 0, dev = -1, stall = -1;
     int64_t M = 0;
     const void *ws = nullptr;
+    size_t ws_bytes = 0;
     bitnet_op_t ops[BITNET_SEQ_MAX_OPS];
-    DsProgram prog;
+    DtProgram prog;
 };
 constexpr int kSeqCacheEntries = 8;
 SeqCacheEntry g_seq_cache[kSeqCacheEntries];
@@ -1178,84 +1002,59 @@ uint64_t g_seq_cache_clock = 0;
 bool same_op(const bitnet_op_t &a, const bitnet_op_t &b)
 {
     return a.kind == b.kind && a.x_dtype == b.x_dtype && a.x == b.x && a.K == b.K && a.N == b.N && a.w0 == b.w0 &&
-           a.gamma0 == b.gamma0 && a.w1 == b.w1 && a.gamma1 == b.gamma1 && a.y == b.y;
+           a.gamma0 == b.gamma0 && a.w1 == b.w1 && a.gamma1 == b.gamma1 && a.y == b.y && a.norm_g == b.norm_g &&
+           (a.norm_g == nullptr || a.norm_eps == b.norm_eps);
 }
 
-bool seq_cache_match(const SeqCacheEntry &e, const bitnet_op_t *ops, int n, int64_t M, int dev, int C, int parts,
-                     int share, const void *ws)
+bool seq_cache_match(const SeqCacheEntry &e, const bitnet_op_t *ops, int n, int64_t M, int dev, int stall,
+                     const void *ws, size_t ws_bytes)
 {
-    if (!e.used || e.n != n || e.M != M || e.dev != dev || e.C != C || e.parts != parts || e.share != share ||
-        e.ws != ws)
+    if (!e.used || e.n != n || e.M != M || e.dev != dev || e.stall != stall || e.ws != ws || e.ws_bytes != ws_bytes)
         return false;
     for (int i = 0; i < n; ++i)
         if (!same_op(e.ops[i], ops[i])) return false;
     return true;
 }
 
-cudaError_t seq_launch(const DsProgram &p, cudaStream_t stream)
-{
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)p.n_ctas);
-    cfg.blockDim = dim3(DS_THREADS);
-    cfg.dynamicSmemBytes = kSmemLimit;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = p.C;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    g_launches.fetch_add(1, std::memory_order_relaxed);
-    return cudaLaunchKernelEx(&cfg, k_decode_seq, p);
-}
+int seq_ctas(int dev) { return num_sms_for(dev); } // one CTA per SM (227 KB of shared memory each)
 
 bitnet_status_t decode_sequence(const bitnet_op_t *ops, int n, int64_t M, void *workspace, size_t ws_bytes,
                                 cudaStream_t stream)
 {
     if (workspace && !aligned16(workspace)) return BITNET_ERR_MISALIGNED;
-    const int parts_set = g_seq_parts.load(), share_set = g_seq_ring_share.load();
-    // the plan of an op list seen before (validated then) on this device, workspace and settings
-    if (ops && n >= 1 && n <= BITNET_SEQ_MAX_OPS && workspace && ws_bytes >= kSeqWorkspaceBytes) {
-        int dev = -1;
-        if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0) {
-            const int C = g_seq_cluster.load();
-            static DsProgram hit_proto;
-            DsProgram p = hit_proto;
-            bool hit = false;
-            {
-                std::lock_guard<std::mutex> lk(g_seq_cache_mu);
-                for (SeqCacheEntry &e : g_seq_cache)
-                    if (seq_cache_match(e, ops, n, M, dev, C, parts_set, share_set, workspace)) {
-                        p = e.prog;
-                        e.stamp = ++g_seq_cache_clock;
-                        hit = true;
-                        break;
-                    }
-            }
-            if (hit) return cuda_status(seq_launch(p, stream));
+    const int stall = g_seq_stall.load();
+    const int dev = current_device();
+    if (ops && n >= 1 && n <= BITNET_SEQ_MAX_OPS && workspace && dev >= 0) {
+        static DtProgram hit_proto;
+        DtProgram p = hit_proto;
+        bool hit = false;
+        {
+            std::lock_guard<std::mutex> lk(g_seq_cache_mu);
+            for (SeqCacheEntry &e : g_seq_cache)
+                if (seq_cache_match(e, ops, n, M, dev, stall, workspace, ws_bytes)) {
+                    p = e.prog;
+                    e.stamp = ++g_seq_cache_clock;
+                    hit = true;
+                    break;
+                }
         }
+        if (hit) return cuda_status(seq_launch(p, seq_ctas(dev), stream, dev));
     }
-    int32_t wx[BITNET_SEQ_MAX_OPS], wy[BITNET_SEQ_MAX_OPS], order[BITNET_SEQ_MAX_OPS];
-    const bitnet_op_t *user_ops = ops;
-    const ByteRange wsr = workspace ? range_of(workspace, kSeqWorkspaceBytes) : ByteRange{0, 0};
+    const ByteRange wsr = workspace ? range_of(workspace, ws_bytes) : ByteRange{0, 0};
+    int32_t order[BITNET_SEQ_MAX_OPS];
     bitnet_status_t st = seq_schedule(ops, n, M, order, wsr);
     if (st != BITNET_OK) return st;
+    if (!workspace) return BITNET_ERR_WORKSPACE;
+    if (dev < 0) return BITNET_ERR_CUDA;
+    const int ctas = seq_ctas(dev);
+    if (ctas < 1) return BITNET_ERR_CUDA;
     bitnet_op_t sched[BITNET_SEQ_MAX_OPS];
     for (int k = 0; k < n; ++k) sched[k] = ops[order[k]];
-    ops = sched;
-    st = seq_plan(ops, n, M, wx, wy, wsr);
+    static DtProgram prog_proto; // zero-initialised template; each call fills a copy
+    DtProgram p = prog_proto;
+    st = seq_build(p, sched, order, n, M, ctas, workspace, ws_bytes, wsr);
     if (st != BITNET_OK) return st;
-    if (!workspace || ws_bytes < kSeqWorkspaceBytes) return BITNET_ERR_WORKSPACE;
-    const int dev = current_device();
-    const int C = g_seq_cluster.load();
-    const int G = seq_clusters(dev, C);
-    if (G < 1) return BITNET_ERR_CUDA;
-    static DsProgram prog_proto; // zero-initialised template; each call fills a copy
-    DsProgram p = prog_proto;
-    st = seq_partitioned_build(p, sched, n, M, C, G, wx, wy, wsr);
-    if (st != BITNET_OK) return st;
-    p.counters = static_cast<unsigned *>(workspace);
+    if (p.n_slots < 2) return BITNET_ERR_UNSUPPORTED_SHAPE;
     {
         // remember the plan under the caller's op list (least recently used entry replaced)
         std::lock_guard<std::mutex> lk(g_seq_cache_mu);
@@ -1272,14 +1071,13 @@ bitnet_status_t decode_sequence(const bitnet_op_t *ops, int n, int64_t M, void *
         slot->n = n;
         slot->M = M;
         slot->dev = dev;
-        slot->C = C;
-        slot->parts = parts_set;
-        slot->share = share_set;
+        slot->stall = stall;
         slot->ws = workspace;
-        for (int i = 0; i < n; ++i) slot->ops[i] = user_ops[i];
+        slot->ws_bytes = ws_bytes;
+        for (int i = 0; i < n; ++i) slot->ops[i] = ops[i];
         slot->prog = p;
     }
-    return cuda_status(seq_launch(p, stream));
+    return cuda_status(seq_launch(p, ctas, stream, dev));
 }
 
 // ---- fixed scratch for bitnet_linear_noalloc -------------------------------
@@ -1403,7 +1201,12 @@ bitnet_status_t bitnet_ffn_gate_up(const void *x, bitnet_dtype_t x_dtype, int64_
                    acc_u_out, workspace, ws_bytes, stream, 2);
 }
 
-size_t bitnet_sequence_workspace_size(void) { return kSeqWorkspaceBytes; }
+size_t bitnet_sequence_workspace_size(int32_t n_ops, int64_t M, int64_t K_max)
+{
+    if (n_ops < 1 || n_ops > BITNET_SEQ_MAX_OPS || M < 1 || M > BITNET_SEQ_MAX_M || K_max < 64 || K_max > kSeqMaxK)
+        return 0;
+    return seq_counter_bytes(n_ops) + (size_t)n_ops * seq_op_ws_bytes(align_up((size_t)K_max, 64), seq_mp(M));
+}
 
 bitnet_status_t bitnet_sequence_plan(const bitnet_op_t *ops, int32_t n_ops, int64_t M, int32_t *wait_x,
                                      int32_t *wait_y)
@@ -1423,51 +1226,51 @@ bitnet_status_t bitnet_sequence_schedule(const bitnet_op_t *ops, int32_t n_ops, 
     return seq_schedule(ops, n_ops, M, order, ByteRange{0, 0});
 }
 
-bitnet_status_t bitnet_sequence_layout(const bitnet_op_t *ops, int32_t n_ops, int64_t M, int32_t cluster_size,
-                                       int32_t clusters, int32_t *order, int32_t *part_of, int32_t *slices,
-                                       int32_t *n_parts, int32_t *part_clusters)
+bitnet_status_t bitnet_sequence_tasks(const bitnet_op_t *ops, int32_t n_ops, int64_t M, int32_t ctas,
+                                      int32_t *group_op, int32_t *group_kind, int32_t *group_tasks,
+                                      int32_t *dep_count, int32_t *deps)
 {
-    if (!ops || n_ops < 1 || n_ops > BITNET_SEQ_MAX_OPS || !order || !part_of || !slices || !n_parts || !part_clusters)
-        return BITNET_ERR_INVALID_ARG;
-    if ((cluster_size != 4 && cluster_size != 8) || clusters < 1) return BITNET_ERR_INVALID_ARG;
-    int32_t wx[BITNET_SEQ_MAX_OPS], wy[BITNET_SEQ_MAX_OPS], ord0[BITNET_SEQ_MAX_OPS];
-    bitnet_status_t st = seq_schedule(ops, n_ops, M, ord0, ByteRange{0, 0});
+    if (!group_op || !group_kind || !group_tasks || !dep_count || !deps || ctas < 1) return BITNET_ERR_INVALID_ARG;
+    int32_t order[BITNET_SEQ_MAX_OPS];
+    bitnet_status_t st = seq_schedule(ops, n_ops, M, order, ByteRange{0, 0});
     if (st != BITNET_OK) return st;
     bitnet_op_t sched[BITNET_SEQ_MAX_OPS];
-    for (int k = 0; k < n_ops; ++k) sched[k] = ops[ord0[k]];
-    st = seq_plan(sched, n_ops, M, wx, wy, ByteRange{0, 0});
+    for (int k = 0; k < n_ops; ++k) sched[k] = ops[order[k]];
+    static DtProgram proto;
+    DtProgram p = proto;
+    std::vector<int> gorder;
+    st = seq_build(p, sched, order, n_ops, M, ctas, nullptr, 0, ByteRange{0, 0}, &gorder);
     if (st != BITNET_OK) return st;
-    static DsProgram proto;
-    DsProgram p = proto;
-    SeqLayout lay;
-    st = seq_partitioned_build(p, sched, n_ops, M, cluster_size, clusters, wx, wy, ByteRange{0, 0}, &lay);
+    SeqGroups G;
+    st = seq_groups(sched, n_ops, M, ByteRange{0, 0}, G);
     if (st != BITNET_OK) return st;
-    for (int k = 0; k < n_ops; ++k) {
-        order[k] = ord0[lay.perm[k]];
-        part_of[k] = lay.part_of[k];
-        slices[k] = lay.slices[k];
+    // position of each group in the task order, to report dependencies by position
+    std::vector<int> pos(2 * n_ops, 0);
+    for (int k = 0; k < 2 * n_ops; ++k) pos[gorder[k]] = k;
+    for (int k = 0; k < 2 * n_ops; ++k) {
+        const int v = gorder[k], j = v / 2;
+        group_op[k] = order[j];
+        group_kind[k] = v % 2;
+        group_tasks[k] = v % 2 ? p.ops[j].rtasks : (int32_t)M;
+        dep_count[k] = (int32_t)G.preds[v].size();
+        for (int d = 0; d < DT_MAX_DEPS + 1; ++d)
+            deps[k * (DT_MAX_DEPS + 1) + d] = d < (int)G.preds[v].size() ? pos[G.preds[v][d]] : -1;
     }
-    *n_parts = p.n_parts;
-    for (int q = 0; q < p.n_parts; ++q) part_clusters[q] = p.part_ncl[q];
     return BITNET_OK;
 }
 
-int bitnet_set_sequence_cluster(int cluster_size)
+uint64_t bitnet_set_wait_limit_ns(uint64_t ns)
 {
-    if (cluster_size != 4 && cluster_size != 8) return -1;
-    return g_seq_cluster.exchange(cluster_size);
+    if (ns == 0) ns = kDefaultWaitLimitNs;
+    const unsigned long long v = ns;
+    if (cudaMemcpyToSymbol(g_wait_limit_ns, &v, sizeof(v)) != cudaSuccess) return 0;
+    return g_wait_limit_set.exchange(v);
 }
 
-int bitnet_set_sequence_partitions(int partitions)
+int bitnet_set_sequence_test_stall(int op)
 {
-    if (partitions < 0 || partitions > DS_MAX_PARTS) return -1;
-    return g_seq_parts.exchange(partitions);
-}
-
-int bitnet_set_sequence_ring_share(int share)
-{
-    if (share < 1 || share > 4) return -1;
-    return g_seq_ring_share.exchange(share);
+    if (op < -1 || op >= BITNET_SEQ_MAX_OPS) return -2;
+    return g_seq_stall.exchange(op);
 }
 
 bitnet_status_t bitnet_rmsnorm_quant(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_t K, const float *g,

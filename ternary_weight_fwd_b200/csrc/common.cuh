@@ -2,7 +2,7 @@
 //
 // Everything here is a thin wrapper over one documented PTX instruction
 // (mbarrier, bulk/tensor copies, programmatic dependent launch, tcgen05).
-// Every wait on a barrier is bounded: after BITNET_WAIT_LIMIT_NS of wall time
+// Every wait on a barrier is bounded: after g_wait_limit_ns of wall time
 // the wait records BITNET_ERR_TIMEOUT in the device status word and returns
 // false, and the caller unwinds instead of spinning forever.
 #pragma once
@@ -16,16 +16,20 @@
 
 #define BITNET_DEVINL __device__ __forceinline__
 
-// Two seconds: far above any legitimate wait in these kernels.
-#ifndef BITNET_WAIT_LIMIT_NS
-#define BITNET_WAIT_LIMIT_NS 2000000000ull
-#endif
-
 namespace bitnet {
+
+// Two seconds: far above any legitimate wait in these kernels.
+constexpr unsigned long long kDefaultWaitLimitNs = 2000000000ull;
 
 // Device status word (one per device).  The library is one translation unit,
 // so this is its only definition.
 __device__ int g_device_status = 0;
+
+// Limit of every bounded wait, in nanoseconds of wall time (one per device;
+// lowered only by tests, through bitnet_set_wait_limit_ns).
+__device__ unsigned long long g_wait_limit_ns = kDefaultWaitLimitNs;
+
+BITNET_DEVINL uint64_t wait_limit_ns() { return *(volatile unsigned long long *)&g_wait_limit_ns; }
 
 BITNET_DEVINL void record_status(int code) { atomicCAS(&g_device_status, 0, code); }
 BITNET_DEVINL bool status_failed() { return *(volatile int *)&g_device_status != 0; }
@@ -93,7 +97,7 @@ BITNET_DEVINL bool mbar_wait(uint64_t *bar, uint32_t parity)
         if (mbar_try_wait(a, parity)) return true;
         if ((spin & 255u) == 0) {
             if (status_failed()) return false;
-            if (globaltimer_ns() - t0 > BITNET_WAIT_LIMIT_NS) {
+            if (globaltimer_ns() - t0 > wait_limit_ns()) {
                 record_status(BITNET_ERR_TIMEOUT);
                 return false;
             }
@@ -125,7 +129,7 @@ BITNET_DEVINL bool mbar_wait_cluster(uint64_t *bar, uint32_t parity)
         if (mbar_try_wait_cluster(a, parity)) return true;
         if ((spin & 255u) == 0) {
             if (status_failed()) return false;
-            if (globaltimer_ns() - t0 > BITNET_WAIT_LIMIT_NS) {
+            if (globaltimer_ns() - t0 > wait_limit_ns()) {
                 record_status(BITNET_ERR_TIMEOUT);
                 return false;
             }
@@ -401,7 +405,7 @@ BITNET_DEVINL bool mbar_wait_drain(uint64_t *bar, uint32_t parity)
     const uint32_t a = smem_u32(bar);
     const uint64_t t0 = globaltimer_ns();
     while (!mbar_try_wait(a, parity))
-        if (globaltimer_ns() - t0 > BITNET_WAIT_LIMIT_NS) return false;
+        if (globaltimer_ns() - t0 > wait_limit_ns()) return false;
     return true;
 }
 

@@ -1,0 +1,665 @@
+// decode_tasks.cuh -- a decode step (many small-M BitLinear / gated-FFN ops over
+// the same M <= 64 tokens) in one persistent launch: bitnet_decode_sequence.
+//
+// BitNet model page, "Model details" / "Architecture" (BitLinear layers, no
+// bias, ReLU^2 FFN) and "Quantization" (W1.58A8: absmean ternary weights,
+// per-token absmax int8 activations).  Each op computes exactly what
+// bitnet_linear / bitnet_ffn_gate_up compute; this file only changes how the
+// work of many ops is laid out on the GPU.
+//
+// Work is cut into tasks, claimed in a fixed global order by the CTAs through
+// one atomic counter (dynamic scheduling: a CTA that finishes early takes the
+// next task):
+//   * quant task (op j, token m): per-token absmax quantisation of row m of the
+//     op's x (optionally RMS-normalised first), written to the workspace as
+//     int8 in the fragment layout [K/64][Mp][64] plus the scale and row sum.
+//     All 256 compute threads share the row (in registers: one pass over x).
+//   * row task (op j, block b): 128 rows of the packed weights (a BitLinear:
+//     output rows 128b ..; a gated FFN: 64 gate rows and the same 64 up rows),
+//     full K, against all tokens.  Compute warp w owns a 16-row group: rows g
+//     and g + 8 of the mma fragment are two output rows (BitLinear) or the gate
+//     and the up row of one output (FFN), so each lane ends with complete sums
+//     and the epilogue needs no exchange between warps or CTAs.
+// Tasks wait only on earlier tasks of the order (an op's rows on its quant
+// tasks; a quant task on the rows of the op that wrote its x; outputs on the
+// readers / writers of the same bytes before them), and every task a CTA
+// holds was claimed by a running CTA, so progress does not depend on how many
+// CTAs are resident at once.
+//
+// Roles in a CTA (320 threads):
+//   warp 8  weight producer: claims tasks, writes them to a 4-entry queue in
+//           shared memory, streams each row task's packed weights into a ring of
+//           pieces (128 rows x 512 k, 16-byte cp.async, row pitch 144 bytes so
+//           the fragment loads hit 32 distinct banks).  Weights never wait for
+//           any other task.
+//   warp 9  activation producer: for a row task, waits for its dependencies,
+//           stages per-token rescale factors gamma / s and row sums, and streams
+//           the matching x_q chunk ([8][Mp][64] bytes) next to each weight piece.
+//   warps 0-7 compute: quant tasks; for row tasks the contraction with
+//           mma.m16n8k32 u8 x s8 (codes c = w + 1 in {0,1,2}; the offset is
+//           removed exactly with the row sum: sum c*x - sum x) and the epilogue.
+// Completion counters live in the caller's workspace; the last CTA out zeroes
+// them.  Every wait is bounded (device status word), and after a timeout every
+// wait returns at once, so the launch always ends.
+#pragma once
+
+#include "common.cuh"
+#include "decode.cuh"
+#include "exact_sumsq.cuh"
+
+namespace bitnet {
+
+constexpr int DT_COMPUTE = 256;                 // compute threads (warps 0-7)
+constexpr int DT_THREADS = 320;                 // + weight producer (warp 8) + activation producer (warp 9)
+constexpr int DT_ROWS = 128;                    // packed rows per row task
+constexpr int DT_KC = 512;                      // k per piece
+constexpr int DT_KB = DT_KC / 64;               // 64-k blocks per piece
+constexpr int DT_PITCH = DT_KC / 4 + 16;        // 144 = 16 * 9: conflict-free fragment loads
+constexpr int DT_WBYTES = DT_ROWS * DT_PITCH;   // 18432 weight bytes of a piece in shared memory
+constexpr int DT_QUEUE = 4;                     // tasks claimed ahead of the compute warps (at most)
+constexpr int DT_MAX_OPS = 128;
+constexpr int DT_MAX_SEGS = 512;
+constexpr int DT_MAX_DEPS = 8;
+constexpr int DT_MAX_SLOTS = 16;
+constexpr int DT_MAX_M = 64;
+// 16-byte chunks of a row of x per compute thread (K <= 8192): 8 for fp32, 4 for bf16
+template <bool XF32> __host__ __device__ constexpr int dt_quant_ch() { return XF32 ? 8 : 4; }
+
+// counters (uint32) at the start of the workspace
+constexpr int DT_CNT_TASK = 0;  // next task to claim
+constexpr int DT_CNT_EXIT = 1;  // CTAs finished
+constexpr int DT_CNT_OPS = 2;   // then per op: quant tasks done, row tasks done (x 8 warps)
+
+constexpr uint16_t DT_DEP_QUANT = 0x8000u; // dependency on an op's quant tasks (else its row tasks)
+
+struct DtOp {
+    const void *x;                 // [M][K] bf16 or fp32 (read by the quant tasks)
+    const uint8_t *w0, *w1;        // [N][K/4] packed (w1: up projection of a gated FFN)
+    const float *gamma0, *gamma1;
+    const float *norm_g;           // [K] RMS normalisation weight, or null
+    float *y;                      // [M][N] fp32 output
+    int8_t *xq;                    // workspace: [K/64][Mp][64]
+    float *s;                      // workspace: [Mp]
+    int32_t *rs;                   // workspace: [Mp]
+    float norm_eps;
+    int K, N;
+    int nmat, xf32;
+    int rtasks;                    // row tasks (blocks of 128 packed rows)
+    int stall;                     // tests only: 1 = the row tasks wait for one quant task too many
+    int nq, nr;                    // dependencies of the quant tasks, of the row outputs
+    uint16_t deps[DT_MAX_DEPS];    // deps[0 .. nq): ops whose rows precede the quant tasks;
+                                   // deps[nq .. nq+nr): op | DT_DEP_QUANT, or op (its rows)
+};
+
+struct DtSeg {        // consecutive tasks of one op in the global order
+    int start;        // global index of the segment's first task
+    uint16_t op;
+    uint16_t first;   // first token (quant) or row block (rows); bit 15: 1 = quant segment
+};
+
+struct DtProgram {
+    int n_ops, n_segs, n_tasks, M, Mp, n_slots, slot_bytes;
+    unsigned *counters;
+    DtOp ops[DT_MAX_OPS];
+    DtSeg segs[DT_MAX_SEGS];
+};
+
+// ---- shared-memory map ------------------------------------------------------
+constexpr int DT_BAR_FULL = 0;                        // [DT_MAX_SLOTS]
+constexpr int DT_BAR_EMPTY = DT_BAR_FULL + 8 * DT_MAX_SLOTS;
+constexpr int DT_BAR_QFULL = DT_BAR_EMPTY + 8 * DT_MAX_SLOTS;
+constexpr int DT_BAR_QINFO = DT_BAR_QFULL + 8 * DT_QUEUE;
+constexpr int DT_BAR_QEMPTY = DT_BAR_QINFO + 8 * DT_QUEUE;
+constexpr int DT_QTASK = DT_BAR_QEMPTY + 8 * DT_QUEUE; // int[DT_QUEUE]
+constexpr int DT_RED = 512;                           // quant-task reductions (512 bytes)
+constexpr int DT_INFO = 1024;                         // per queue entry: r0[64], r1[64] fp32, rs[64] int32
+constexpr int DT_INFO_BYTES = 3 * 4 * DT_MAX_M;
+constexpr int DT_HDR = DT_INFO + DT_QUEUE * DT_INFO_BYTES; // 4096: the piece ring starts here
+static_assert(DT_QTASK + 4 * DT_QUEUE <= DT_RED, "shared header");
+static_assert(DT_HDR % 128 == 0, "ring alignment");
+
+// task t -> (op, kind, index)
+struct DtTask {
+    int op, idx;
+    bool quant;
+};
+
+BITNET_DEVINL DtTask dt_decode(const DtProgram &p, int t)
+{
+    int lo = 0, hi = p.n_segs - 1;
+    while (lo < hi) { // last segment with start <= t
+        const int mid = (lo + hi + 1) >> 1;
+        if (p.segs[mid].start <= t) lo = mid;
+        else hi = mid - 1;
+    }
+    const DtSeg sg = p.segs[lo];
+    DtTask r;
+    r.op = sg.op;
+    r.quant = (sg.first & 0x8000u) != 0;
+    r.idx = (int)(sg.first & 0x7fffu) + (t - sg.start);
+    return r;
+}
+
+BITNET_DEVINL unsigned dt_ld_acquire(const unsigned *c)
+{
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(c) : "memory");
+    return v;
+}
+
+// Bounded wait until *c >= target; false after a timeout (recorded) or once
+// another wait gave up.
+BITNET_DEVINL bool dt_wait_count(const unsigned *c, unsigned target)
+{
+    if (dt_ld_acquire(c) >= target) return true;
+    const uint64_t t0 = globaltimer_ns();
+    const uint64_t limit = wait_limit_ns();
+    for (uint32_t spin = 1;; ++spin) {
+        __nanosleep(64);
+        if (dt_ld_acquire(c) >= target) return true;
+        if ((spin & 31u) == 0) {
+            if (status_failed()) return false;
+            if (globaltimer_ns() - t0 > limit) {
+                record_status(BITNET_ERR_TIMEOUT);
+                return false;
+            }
+        }
+    }
+}
+
+BITNET_DEVINL unsigned *dt_qdone(const DtProgram &p, int j) { return p.counters + DT_CNT_OPS + 2 * j; }
+BITNET_DEVINL unsigned *dt_rdone(const DtProgram &p, int j) { return p.counters + DT_CNT_OPS + 2 * j + 1; }
+
+// Completion targets: one arrival per quant task (token), eight per row task (warps).
+BITNET_DEVINL unsigned dt_qtarget(const DtProgram &p, int) { return (unsigned)p.M; }
+BITNET_DEVINL unsigned dt_rtarget(const DtProgram &p, int j) { return 8u * (unsigned)p.ops[j].rtasks; }
+
+BITNET_DEVINL void dt_bar_compute() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+// 16-byte asynchronous copy; zero-fills the destination when !valid (nothing is read).
+BITNET_DEVINL void dt_cp16(uint32_t dst, const void *src, bool valid)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
+                 : "memory");
+}
+
+BITNET_DEVINL void dt_cp_arrive(uint32_t bar)
+{
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+BITNET_DEVINL uint4 dt_ld_cg16(const void *p)
+{
+    uint4 v;
+    asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+BITNET_DEVINL float dt_ld_cg_f32(const float *p)
+{
+    float v;
+    asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(v) : "l"(p));
+    return v;
+}
+
+BITNET_DEVINL int dt_ld_cg_s32(const int32_t *p)
+{
+    int v;
+    asm volatile("ld.global.cg.s32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+
+BITNET_DEVINL int dt_pieces(int K) { return (K + DT_KC - 1) / DT_KC; }
+
+// ---- weight producer (warp 8) ----------------------------------------------
+BITNET_DEVINL void dt_weight_producer(const DtProgram &p, unsigned char *smem)
+{
+    const int lane = threadIdx.x & 31;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + DT_BAR_FULL);
+    uint64_t *empty = reinterpret_cast<uint64_t *>(smem + DT_BAR_EMPTY);
+    uint64_t *qfull = reinterpret_cast<uint64_t *>(smem + DT_BAR_QFULL);
+    uint64_t *qempty = reinterpret_cast<uint64_t *>(smem + DT_BAR_QEMPTY);
+    volatile int *qtask = reinterpret_cast<volatile int *>(smem + DT_QTASK);
+    const uint32_t ring = smem_u32(smem + DT_HDR);
+    // this lane's 16-byte chunk of a piece row and its first row; 32 rows a pass of 4 lanes... 8 lanes a row
+    const int j16 = lane & 7;   // chunk within the row (64-k block of the piece)
+    const int r0 = lane >> 3;   // rows r0, r0 + 4, ..., r0 + 124
+    uint32_t seq = 0, piece = 0;
+    for (;;) {
+        int t = 0;
+        if (lane == 0) t = (int)atomicAdd(&p.counters[DT_CNT_TASK], 1u);
+        t = __shfl_sync(0xffffffffu, t, 0);
+        if (t >= p.n_tasks) t = -1;
+        const int e = (int)(seq % DT_QUEUE);
+        mbar_wait(&qempty[e], ((seq / DT_QUEUE) & 1u) ^ 1u);
+        if (lane == 0) {
+            qtask[e] = t;
+            mbar_arrive(&qfull[e]);
+        }
+        ++seq;
+        if (t < 0) break;
+        const DtTask tk = dt_decode(p, t);
+        if (tk.quant) continue;
+        const DtOp &op = p.ops[tk.op];
+        const int K = op.K, N = op.N, rowb = K / 4;
+        const bool ffn = op.nmat == 2;
+        const int np = dt_pieces(K);
+        // source row of shared row r (ffn: rows 8..15 of each 16-row group are the up rows)
+        for (int pc = 0; pc < np; ++pc) {
+            const int s = (int)(piece % (uint32_t)p.n_slots);
+            mbar_wait(&empty[s], ((piece / (uint32_t)p.n_slots) & 1u) ^ 1u);
+            const int nkb = min(DT_KB, (K - pc * DT_KC) / 64);
+            const uint32_t dst0 = ring + (uint32_t)s * (uint32_t)p.slot_bytes;
+            if (j16 < nkb) {
+#pragma unroll 8
+                for (int r = r0; r < DT_ROWS; r += 4) {
+                    int n;
+                    const uint8_t *w;
+                    if (ffn) {
+                        n = tk.idx * (DT_ROWS / 2) + (r >> 4) * 8 + (r & 7);
+                        w = (r & 8) ? op.w1 : op.w0;
+                    } else {
+                        n = tk.idx * DT_ROWS + r;
+                        w = op.w0;
+                    }
+                    const bool ok = n < N;
+                    const uint8_t *src = w + (size_t)(ok ? n : 0) * rowb + pc * (DT_KC / 4) + j16 * 16;
+                    dt_cp16(dst0 + (uint32_t)(r * DT_PITCH + j16 * 16), src, ok);
+                }
+            }
+            dt_cp_arrive(smem_u32(&full[s]));
+            ++piece;
+        }
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+// ---- activation producer (warp 9) -------------------------------------------
+BITNET_DEVINL void dt_act_producer(const DtProgram &p, unsigned char *smem)
+{
+    const int lane = threadIdx.x & 31;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + DT_BAR_FULL);
+    uint64_t *empty = reinterpret_cast<uint64_t *>(smem + DT_BAR_EMPTY);
+    uint64_t *qfull = reinterpret_cast<uint64_t *>(smem + DT_BAR_QFULL);
+    uint64_t *qinfo = reinterpret_cast<uint64_t *>(smem + DT_BAR_QINFO);
+    uint64_t *qempty = reinterpret_cast<uint64_t *>(smem + DT_BAR_QEMPTY);
+    const volatile int *qtask = reinterpret_cast<const volatile int *>(smem + DT_QTASK);
+    const uint32_t ring = smem_u32(smem + DT_HDR);
+    const int Mp = p.Mp;
+    uint32_t seq = 0, piece = 0;
+    for (;;) {
+        const int e = (int)(seq % DT_QUEUE);
+        mbar_wait(&qfull[e], (seq / DT_QUEUE) & 1u);
+        const int t = qtask[e];
+        bool rows = false;
+        DtTask tk = {0, 0, true};
+        if (t >= 0) {
+            tk = dt_decode(p, t);
+            rows = !tk.quant;
+        }
+        if (rows) {
+            const DtOp &op = p.ops[tk.op];
+            // dependencies: the op's own quant tasks, then the readers / writers of its output bytes
+            if (lane == 0) {
+                dt_wait_count(dt_qdone(p, tk.op), dt_qtarget(p, tk.op) + (unsigned)op.stall);
+                for (int d = op.nq; d < op.nq + op.nr; ++d) {
+                    const int o = op.deps[d] & 0x7fff;
+                    if (op.deps[d] & DT_DEP_QUANT) dt_wait_count(dt_qdone(p, o), dt_qtarget(p, o));
+                    else dt_wait_count(dt_rdone(p, o), dt_rtarget(p, o));
+                }
+            }
+            __syncwarp();
+            // per-token rescale factors fl(gamma / s) and row sums of this task's op
+            float *inf = reinterpret_cast<float *>(smem + DT_INFO + e * DT_INFO_BYTES);
+            const float g0 = __ldg(op.gamma0), g1 = op.nmat == 2 ? __ldg(op.gamma1) : 0.0f;
+            for (int m = lane; m < Mp; m += 32) {
+                const float sm = m < p.M ? dt_ld_cg_f32(op.s + m) : 1.0f;
+                inf[m] = __fdiv_rn(g0, sm);
+                inf[DT_MAX_M + m] = __fdiv_rn(g1, sm);
+                reinterpret_cast<int *>(inf)[2 * DT_MAX_M + m] = m < p.M ? dt_ld_cg_s32(op.rs + m) : 0;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&qinfo[e]);
+            // the x_q chunk of every piece: [8 k-blocks][Mp][64] bytes, contiguous in the workspace
+            const int np = dt_pieces(op.K);
+            for (int pc = 0; pc < np; ++pc) {
+                const int s = (int)(piece % (uint32_t)p.n_slots);
+                mbar_wait(&empty[s], ((piece / (uint32_t)p.n_slots) & 1u) ^ 1u);
+                const int nkb = min(DT_KB, (op.K - pc * DT_KC) / 64);
+                const int chunks = nkb * Mp * 4; // 16-byte chunks
+                const uint8_t *src = reinterpret_cast<const uint8_t *>(op.xq) + (size_t)pc * DT_KB * Mp * 64;
+                const uint32_t dst = ring + (uint32_t)s * (uint32_t)p.slot_bytes + DT_WBYTES;
+                for (int c = lane; c < chunks; c += 32) dt_cp16(dst + 16u * c, src + 16 * c, true);
+                dt_cp_arrive(smem_u32(&full[s]));
+                ++piece;
+            }
+        } else if (lane == 0) {
+            mbar_arrive(&qinfo[e]); // keeps the entry's phases in step
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&qempty[e]);
+        ++seq;
+        if (t < 0) break;
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+// ---- quant task (compute warps): token m of op j -----------------------------
+// Thread t holds 16-byte chunks c = t + 256 i of the row (x read once, from L2).
+template <bool XF32>
+BITNET_DEVINL void dt_quant_row(const DtProgram &p, const DtOp &op, int m, unsigned char *smem)
+{
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    constexpr int EPC = XF32 ? 4 : 8; // elements per chunk
+    constexpr int DT_QUANT_CH = dt_quant_ch<XF32>();
+    const int K = op.K, nch = K / EPC;
+    float *red = reinterpret_cast<float *>(smem + DT_RED);           // [8] maxima / scratch
+    int *redi = reinterpret_cast<int *>(smem + DT_RED + 32);         // [8] row sums
+    uint32_t *rede = reinterpret_cast<uint32_t *>(smem + DT_RED + 64);  // [8] exponents
+    int *redf = reinterpret_cast<int *>(smem + DT_RED + 96);         // [8] window fits
+    uint64_t *redw = reinterpret_cast<uint64_t *>(smem + DT_RED + 128); // [8][2] window sums
+    unsigned long long *dig = reinterpret_cast<unsigned long long *>(smem + DT_RED + 256); // [20]
+    float *bc = reinterpret_cast<float *>(smem + DT_RED + 416);     // broadcasts
+    const char *row = static_cast<const char *>(op.x) + (size_t)m * K * (XF32 ? 4 : 2);
+    float v[DT_QUANT_CH * EPC];
+#pragma unroll
+    for (int i = 0; i < DT_QUANT_CH; ++i) {
+        const int c = tid + 256 * i;
+        uint4 q = make_uint4(0u, 0u, 0u, 0u);
+        if (c < nch) q = dt_ld_cg16(row + 16 * (size_t)c);
+        if constexpr (XF32) {
+            v[4 * i + 0] = __uint_as_float(q.x);
+            v[4 * i + 1] = __uint_as_float(q.y);
+            v[4 * i + 2] = __uint_as_float(q.z);
+            v[4 * i + 3] = __uint_as_float(q.w);
+        } else {
+            const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                v[8 * i + 2 * h] = bf16_bits_lo(w[h]);
+                v[8 * i + 2 * h + 1] = bf16_bits_hi(w[h]);
+            }
+        }
+    }
+    if (op.norm_g) {
+        // RMS normalisation: exact sum of squares (rounded once), r in binary64 -> binary32
+        uint32_t em = 0;
+#pragma unroll
+        for (int e = 0; e < DT_QUANT_CH * EPC; ++e) em = max(em, ss_exponent(v[e]));
+        em = __reduce_max_sync(0xffffffffu, em);
+        if (lane == 0) rede[warp] = em;
+        if (tid < SS_LONG_DIGITS) dig[tid] = 0ull;
+        dt_bar_compute();
+        uint32_t E = 0;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) E = max(E, rede[w]);
+        SsWindow acc;
+        if (E != 0) {
+#pragma unroll
+            for (int e = 0; e < DT_QUANT_CH * EPC; ++e) ss_window_add(acc, v[e], E);
+        }
+        ss_warp_sum(acc.lo, acc.hi);
+        const bool fits = __all_sync(0xffffffffu, acc.fits);
+        if (lane == 0) {
+            redw[2 * warp] = acc.lo;
+            redw[2 * warp + 1] = acc.hi;
+            redf[warp] = fits ? 1 : 0;
+        }
+        dt_bar_compute();
+        bool slow = false;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) slow = slow || redf[w] == 0;
+        if (slow) {
+#pragma unroll
+            for (int e = 0; e < DT_QUANT_CH * EPC; ++e) ss_long_add(dig, v[e]);
+            dt_bar_compute();
+        }
+        if (tid == 0) {
+            double ss;
+            if (slow) {
+                ss = ss_long_round(dig);
+            } else {
+                uint64_t lo = 0, hi = 0;
+                for (int w = 0; w < 8; ++w) ss_add128(lo, hi, redw[2 * w], redw[2 * w + 1]);
+                ss = E ? ss_window_round(lo, hi, E) : 0.0;
+            }
+            const double mean = __ddiv_rn(ss, (double)K);
+            bc[0] = __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(mean, (double)op.norm_eps))));
+        }
+        dt_bar_compute();
+        const float r = bc[0];
+#pragma unroll
+        for (int i = 0; i < DT_QUANT_CH; ++i) {
+#pragma unroll
+            for (int h = 0; h < EPC; ++h) {
+                const int k = (tid + 256 * i) * EPC + h;
+                if (k < K) v[EPC * i + h] = __fmul_rn(__fmul_rn(v[EPC * i + h], r), __ldg(op.norm_g + k));
+            }
+        }
+    }
+    // per-token absmax (padding elements are zero)
+    float mx = 0.0f;
+#pragma unroll
+    for (int e = 0; e < DT_QUANT_CH * EPC; ++e) mx = fmaxf(mx, fabsf(v[e]));
+    mx = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(mx)));
+    if (lane == 0) red[warp] = mx;
+    dt_bar_compute();
+    float amax = 0.0f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) amax = fmaxf(amax, red[w]);
+    const float sc = quant_scale(amax);
+    // quantise into the fragment layout: byte k of token m at ((k / 64) * Mp + m) * 64 + k % 64
+    int rsum = 0;
+    int8_t *xq = op.xq;
+#pragma unroll
+    for (int i = 0; i < DT_QUANT_CH; ++i) {
+        const int c = tid + 256 * i;
+        if (c < nch) {
+            int q[EPC];
+#pragma unroll
+            for (int h = 0; h < EPC; ++h) {
+                q[h] = quant_one(v[EPC * i + h], sc);
+                rsum += q[h];
+            }
+            const int k0 = c * EPC;
+            int8_t *dst = xq + ((size_t)(k0 >> 6) * p.Mp + m) * 64 + (k0 & 63);
+            if constexpr (XF32) {
+                *reinterpret_cast<uint32_t *>(dst) = pack4_s8(q[0], q[1], q[2], q[3]);
+            } else {
+                *reinterpret_cast<uint2 *>(dst) =
+                    make_uint2(pack4_s8(q[0], q[1], q[2], q[3]), pack4_s8(q[4], q[5], q[6], q[7]));
+            }
+        }
+    }
+    rsum = warp_sum(rsum);
+    if (lane == 0) redi[warp] = rsum;
+    dt_bar_compute();
+    if (tid == 0) {
+        int tot = 0;
+        for (int w = 0; w < 8; ++w) tot += redi[w];
+        op.s[m] = sc;
+        op.rs[m] = tot;
+    }
+}
+
+// ---- row task contraction over one piece (compute warp w) ------------------
+// acc[a][tt][4]: accumulator set a (k-blocks alternate between sets so that
+// consecutive mma are independent), token tile tt.
+template <int TT, int NACC>
+BITNET_DEVINL void dt_piece(int (&acc)[NACC][TT][4], uint32_t wrow, uint32_t xrow, int Mp, int nkb)
+{
+    constexpr uint32_t M3 = 0x03030303u;
+#pragma unroll
+    for (int kb = 0; kb < DT_KB; ++kb) {
+        if (kb < nkb) {
+            uint32_t lo, hi;
+            asm volatile("ld.shared.u32 %0, [%1];" : "=r"(lo) : "r"(wrow + kb * 16));
+            asm volatile("ld.shared.u32 %0, [%1];" : "=r"(hi) : "r"(wrow + 8 * DT_PITCH + kb * 16));
+            const uint32_t a0 = lo & M3, a1 = hi & M3, a2 = (lo >> 2) & M3, a3 = (hi >> 2) & M3;
+            const uint32_t a4 = (lo >> 4) & M3, a5 = (hi >> 4) & M3, a6 = (lo >> 6) & M3, a7 = (hi >> 6) & M3;
+#pragma unroll
+            for (int tt = 0; tt < TT; ++tt) {
+                uint4 b;
+                asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w)
+                             : "r"(xrow + (uint32_t)((kb * Mp + tt * 8) * 64)));
+                mma_u8s8_16832(acc[kb % NACC][tt], a0, a1, a2, a3, b.x, b.y);
+                mma_u8s8_16832(acc[kb % NACC][tt], a4, a5, a6, a7, b.z, b.w);
+            }
+        }
+    }
+}
+
+template <int TT>
+BITNET_DEVINL void dt_compute(const DtProgram &p, unsigned char *smem)
+{
+    constexpr int NACC = TT <= 2 ? 4 : 2;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = lane >> 2, t4 = lane & 3;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + DT_BAR_FULL);
+    uint64_t *empty = reinterpret_cast<uint64_t *>(smem + DT_BAR_EMPTY);
+    uint64_t *qfull = reinterpret_cast<uint64_t *>(smem + DT_BAR_QFULL);
+    uint64_t *qinfo = reinterpret_cast<uint64_t *>(smem + DT_BAR_QINFO);
+    uint64_t *qempty = reinterpret_cast<uint64_t *>(smem + DT_BAR_QEMPTY);
+    const volatile int *qtask = reinterpret_cast<const volatile int *>(smem + DT_QTASK);
+    const uint32_t ring = smem_u32(smem + DT_HDR);
+    const int Mp = p.Mp, M = p.M;
+    uint32_t seq = 0, piece = 0;
+    for (;;) {
+        const int e = (int)(seq % DT_QUEUE);
+        mbar_wait(&qfull[e], (seq / DT_QUEUE) & 1u);
+        const int t = qtask[e];
+        if (t < 0) break;
+        const DtTask tk = dt_decode(p, t);
+        const DtOp &op = p.ops[tk.op];
+        if (tk.quant) {
+            // the op that wrote x (read after write) is complete
+            if (tid == 0)
+                for (int d = 0; d < op.nq; ++d) dt_wait_count(dt_rdone(p, op.deps[d]), dt_rtarget(p, op.deps[d]));
+            dt_bar_compute();
+            if (op.xf32) dt_quant_row<true>(p, op, tk.idx, smem);
+            else dt_quant_row<false>(p, op, tk.idx, smem);
+            // (dt_quant_row ends with a barrier after every store of the row)
+            if (tid == 0) {
+                __threadfence();
+                atomicAdd(dt_qdone(p, tk.op), 1u);
+            }
+        } else {
+            int acc[NACC][TT][4];
+#pragma unroll
+            for (int a = 0; a < NACC; ++a)
+#pragma unroll
+                for (int tt = 0; tt < TT; ++tt)
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) acc[a][tt][c] = 0;
+            const int np = dt_pieces(op.K);
+            for (int pc = 0; pc < np; ++pc) {
+                const int s = (int)(piece % (uint32_t)p.n_slots);
+                mbar_wait(&full[s], (piece / (uint32_t)p.n_slots) & 1u);
+                const uint32_t base = ring + (uint32_t)s * (uint32_t)p.slot_bytes;
+                const uint32_t wrow = base + (uint32_t)((warp * 16 + g) * DT_PITCH + t4 * 4);
+                const uint32_t xrow = base + DT_WBYTES + (uint32_t)(g * 64 + t4 * 16);
+                const int nkb = min(DT_KB, (op.K - pc * DT_KC) / 64);
+                dt_piece<TT, NACC>(acc, wrow, xrow, Mp, nkb);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[s]);
+                ++piece;
+            }
+#pragma unroll
+            for (int a = 1; a < NACC; ++a)
+#pragma unroll
+                for (int tt = 0; tt < TT; ++tt)
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) acc[0][tt][c] += acc[a][tt][c];
+            // epilogue: y = fl((float)(sum c*x - sum x) * fl(gamma / s))
+            mbar_wait(&qinfo[e], (seq / DT_QUEUE) & 1u);
+            const float *inf = reinterpret_cast<const float *>(smem + DT_INFO + e * DT_INFO_BYTES);
+            const int *irs = reinterpret_cast<const int *>(inf) + 2 * DT_MAX_M;
+            const int N = op.N;
+            float *y = op.y;
+            if (op.nmat == 2) {
+                const int n = tk.idx * (DT_ROWS / 2) + warp * 8 + g;
+#pragma unroll
+                for (int tt = 0; tt < TT; ++tt)
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {
+                        const int m = tt * 8 + 2 * t4 + q;
+                        if (m < M && n < N) {
+                            const int rsm = irs[m];
+                            const float gv = __fmul_rn((float)(acc[0][tt][q] - rsm), inf[m]);
+                            const float uv = __fmul_rn((float)(acc[0][tt][2 + q] - rsm), inf[DT_MAX_M + m]);
+                            const float pg = gv > 0.0f ? gv : 0.0f;
+                            y[(size_t)m * N + n] = __fmul_rn(__fmul_rn(pg, pg), uv);
+                        }
+                    }
+            } else {
+                const int n0 = tk.idx * DT_ROWS + warp * 16 + g;
+#pragma unroll
+                for (int tt = 0; tt < TT; ++tt)
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {
+                        const int m = tt * 8 + 2 * t4 + q;
+                        if (m < M) {
+                            const int rsm = irs[m];
+                            const float r = inf[m];
+#pragma unroll
+                            for (int h = 0; h < 2; ++h) {
+                                const int n = n0 + 8 * h;
+                                if (n < N) y[(size_t)m * N + n] = __fmul_rn((float)(acc[0][tt][2 * h + q] - rsm), r);
+                            }
+                        }
+                    }
+            }
+            // every lane's stores precede (warp barrier) lane 0's fence and completion count
+            __syncwarp();
+            if (lane == 0) {
+                __threadfence();
+                atomicAdd(dt_rdone(p, tk.op), 1u);
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&qempty[e]);
+        ++seq;
+    }
+}
+
+template <int TT>
+__global__ void __launch_bounds__(DT_THREADS, 1) k_decode_tasks(const __grid_constant__ DtProgram p)
+{
+    extern __shared__ unsigned char dt_smem_raw[];
+    unsigned char *smem =
+        reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(dt_smem_raw) + 127) & ~uintptr_t(127));
+    const int tid = threadIdx.x;
+    if (tid == 0) {
+        uint64_t *bars = reinterpret_cast<uint64_t *>(smem);
+        for (int i = 0; i < p.n_slots; ++i) {
+            mbar_init(&bars[DT_BAR_FULL / 8 + i], 64); // 32 weight lanes + 32 activation lanes (cp.async, noinc)
+            mbar_init(&bars[DT_BAR_EMPTY / 8 + i], 8); // compute warps
+        }
+        for (int i = 0; i < DT_QUEUE; ++i) {
+            mbar_init(&bars[DT_BAR_QFULL / 8 + i], 1);
+            mbar_init(&bars[DT_BAR_QINFO / 8 + i], 1);
+            mbar_init(&bars[DT_BAR_QEMPTY / 8 + i], 9); // compute warps + activation producer
+        }
+        fence_mbarrier_init();
+    }
+    __syncthreads();
+    const int warp = tid >> 5;
+    if (warp == 8) dt_weight_producer(p, smem);
+    else if (warp == 9) dt_act_producer(p, smem);
+    else dt_compute<TT>(p, smem);
+    __syncthreads();
+    if (tid == 0) {
+        // the last CTA out leaves the counters zeroed for the next launch
+        __threadfence();
+        const unsigned prev = atomicAdd(&p.counters[DT_CNT_EXIT], 1u);
+        if (prev == gridDim.x - 1) {
+            __threadfence();
+            for (int i = 0; i < DT_CNT_OPS + 2 * p.n_ops; ++i) atomicExch(&p.counters[i], 0u);
+        }
+    }
+}
+
+} // namespace bitnet

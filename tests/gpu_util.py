@@ -4,7 +4,7 @@ import torch
 
 import oracle
 import ternary_weight_fwd_b200 as tw
-from ternary_weight_fwd_b200 import synth
+import synth
 
 DEV = "cuda"
 REL_TOL = 1e-6  # dequantised outputs: |y - y_ref| <= 1e-6 |y_ref|; y_ref == 0 -> y == 0

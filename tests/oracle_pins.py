@@ -19,7 +19,7 @@ from fractions import Fraction
 import numpy as np
 
 import oracle
-from ternary_weight_fwd_b200 import synth
+import synth
 
 
 def _f32_bits(v):

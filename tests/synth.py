@@ -1,4 +1,4 @@
-"""Seeded synthetic inputs shared by the tests, the smoke check and the benchmark.
+"""Seeded synthetic inputs shared by the tests, the smoke check and the benchmark's CPU baseline.
 
 This module draws random numbers and formats them; it holds none of the
 BitLinear arithmetic (no scale, no rounding to integers, no contraction).

@@ -13,7 +13,7 @@ import torch
 import oracle
 import ternary_weight_fwd_b200 as tw
 from gpu_util import DEV, assert_rel_close, f32_to_dev, make_weights, make_x
-from ternary_weight_fwd_b200 import synth
+import synth
 
 pytestmark = pytest.mark.gpu
 

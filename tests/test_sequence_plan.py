@@ -251,10 +251,9 @@ def test_run_rejects_before_launch():
     good = [lin(BASE, 256, 256, BASE + (1 << 20), BASE + (2 << 20))]
     arr = tw._op_array(good)
     ws = BASE + (8 << 20)
-    size = tw.bitnet_sequence_workspace_size()
-    assert size >= 4 * (tw.BITNET_SEQ_MAX_OPS + 1)
+    size = tw.bitnet_sequence_workspace_size(1, 4, 256)
+    assert size >= 4 * 4 + 256 * 8
     assert lib.bitnet_decode_sequence(arr, 1, 4, None, size, None) == tw.BITNET_ERR_WORKSPACE
-    assert lib.bitnet_decode_sequence(arr, 1, 4, ws, size - 1, None) == tw.BITNET_ERR_WORKSPACE
     assert lib.bitnet_decode_sequence(arr, 1, 4, ws + 8, size, None) == tw.BITNET_ERR_MISALIGNED
     # the workspace may not overlap any operand
     assert lib.bitnet_decode_sequence(arr, 1, 4, BASE + (1 << 20), size, None) == tw.BITNET_ERR_INVALID_ARG
@@ -265,153 +264,216 @@ def test_run_rejects_before_launch():
         assert lib.bitnet_decode_sequence(arr, 1, 4, ws, size, None) == tw.BITNET_ERR_CUDA
 
 
-def test_cluster_size_setter():
-    prev = tw.bitnet_set_sequence_cluster(8)
-    try:
-        assert tw.bitnet_set_sequence_cluster(4) == 8
-        for bad in (0, 1, 2, 3, 16):
-            with pytest.raises(ValueError):
-                tw.bitnet_set_sequence_cluster(bad)
-        assert tw.bitnet_set_sequence_cluster(4) == 4
-    finally:
-        tw.bitnet_set_sequence_cluster(prev)
+def test_workspace_size():
+    one = tw.bitnet_sequence_workspace_size(1, 8, 2560)
+    assert one >= 2560 * 8 + 8 * 8
+    assert tw.bitnet_sequence_workspace_size(120, 8, 6912) >= 120 * 6912 * 8
+    assert tw.bitnet_sequence_workspace_size(2, 8, 2560) > one
+    assert tw.bitnet_sequence_workspace_size(1, 9, 2560) > one       # 16 token rows of x_q
+    assert tw.bitnet_sequence_workspace_size(1, 64, 8192) >= 64 * 8192
+    for bad in ((0, 8, 256), (129, 8, 256), (1, 0, 256), (1, 65, 256), (1, 8, 32), (1, 8, 8256)):
+        assert tw.bitnet_sequence_workspace_size(*bad) == 0
 
 
-# ---------------------------------------------------------------- partitions and row slices
-def producers(ops, m):
-    wx, wy = brute_force(ops, m)
-    return [{w for w in (wx[j], wy[j]) if w >= 0} for j in range(len(ops))]
+def test_norm_fields_are_validated():
+    x, y, w = BASE, BASE + (1 << 20), BASE + (2 << 20)
+    good = lin(x, 256, 256, y, w)
+    good.norm_g = BASE + (3 << 20)
+    good.norm_eps = 1e-5
+    assert _status([good], 4) == tw.BITNET_OK
+    bad = lin(x, 256, 256, y, w)
+    bad.norm_g = BASE + (3 << 20) + 4
+    assert _status([bad], 4) == tw.BITNET_ERR_MISALIGNED
+    bad.norm_g = BASE + (3 << 20)
+    bad.norm_eps = -1.0
+    assert _status([bad], 4) == tw.BITNET_ERR_INVALID_ARG
+    bad.norm_eps = float("inf")
+    assert _status([bad], 4) == tw.BITNET_ERR_INVALID_ARG
+    # an output may not overwrite a norm weight (read ahead of every wait)
+    other = lin(BASE + (4 << 20), 256, 256, BASE + (3 << 20), BASE + (5 << 20))
+    assert _status([good, other], 4) == tw.BITNET_ERR_INVALID_ARG
 
 
-def check_layout(ops, m, L, clusters):
-    n = len(ops)
-    order, part_of, slices = L["order"], L["part_of"], L["slices"]
-    assert sorted(order) == list(range(n)), "order is a permutation of the ops"
-    assert sum(L["part_clusters"]) == clusters and min(L["part_clusters"]) >= 1
-    assert sum(slices) <= 320 and min(slices) >= 1  # kernel ops per launch
-    pos = {i: k for k, i in enumerate(order)}
-    for j, pre in enumerate(producers(ops, m)):
-        for i in pre:
-            # every earlier conflicting op runs first, in the same partition
-            assert pos[i] < pos[j] and part_of[pos[i]] == part_of[pos[j]]
-    # partitions never share memory: ops of different partitions never conflict
-    wx, wy = brute_force([ops[i] for i in order], m)
-    for j in range(n):
-        for w in (wx[j], wy[j]):
-            assert w < 0 or part_of[w] == part_of[j]
-
-
-@pytest.mark.parametrize("forced", [0, 1, 2, 3, 4, 8])
-@pytest.mark.parametrize("shared", [True, False], ids=["shared_outputs", "private_outputs"])
-def test_layout_of_the_layer_stack(forced, shared):
-    ops = layer_stack(30, 8, shared_outputs=shared)
-    prev = tw.bitnet_set_sequence_partitions(forced)
-    try:
-        try:
-            L = tw.bitnet_sequence_layout(ops, 8, 4, 33)
-        except tw.BitnetError as e:
-            # more partitions than slices allow (every op cut to fit 4 clusters): refused, never wrong
-            assert forced >= 6 and e.status == tw.BITNET_ERR_UNSUPPORTED_SHAPE
-            return
-    finally:
-        tw.bitnet_set_sequence_partitions(prev)
-    check_layout(ops, 8, L, 33)
-    n_parts = len(L["part_clusters"])
-    if shared:
-        assert n_parts <= 3  # the gate/up -> down chain, the q chain and the o chain
-    if forced:
-        assert n_parts == min(forced, 3 if shared else 120)
-    # a gate/up op and the down op that reads its h share a partition
-    for l in range(30):
-        k_gu, k_dn = L["order"].index(4 * l + 2), L["order"].index(4 * l + 3)
-        assert L["part_of"][k_gu] == L["part_of"][k_dn] and k_gu < k_dn
-
-
-def test_layout_private_outputs_runs_layers_side_by_side():
-    ops = layer_stack(30, 8, shared_outputs=False)
-    L = tw.bitnet_sequence_layout(ops, 8, 4, 33)
-    assert len(L["part_clusters"]) >= 2
-    # big projections are cut into row slices on the smaller partitions
-    k_gu = L["order"].index(2)
-    assert L["slices"][k_gu] >= 2
-
-
-def test_layout_cuts_one_huge_projection_into_slices():
-    m, k, n = 8, 256, 60000
-    ops = [op(tw.BITNET_OP_FFN_GATE_UP, BASE, k, n, BASE + (1 << 30), BASE + (2 << 30), BASE + (3 << 30),
-              BASE + (4 << 30), BASE + (5 << 30))]
-    L = tw.bitnet_sequence_layout(ops, m, 4, 33)
-    assert L["part_clusters"] == [33] and L["slices"][0] >= 2
-    # rows per cluster of each slice within 8 row groups per warp (1024 rows of both matrices)
-    assert 2 * ((-(-(n // L["slices"][0] + 1) // 33) + 15) // 16) <= 64
-
-
-def test_partition_setter():
-    assert tw.bitnet_set_sequence_partitions(2) == 0
-    assert tw.bitnet_set_sequence_partitions(0) == 2
+def test_test_stall_setter():
+    assert tw.bitnet_set_sequence_test_stall(3) == -1
+    assert tw.bitnet_set_sequence_test_stall(-1) == 3
     with pytest.raises(ValueError):
-        tw.bitnet_set_sequence_partitions(9)
-    assert tw.bitnet_set_sequence_partitions(0) == 0
+        tw.bitnet_set_sequence_test_stall(tw.BITNET_SEQ_MAX_OPS)
 
 
-def test_layout_auto_choice_for_the_bench_decode_step():
-    """The plan the bench times (30 layers, per-layer outputs, M = 8, 33 clusters of 4): eight
-    partitions of ~4 layers, q / o whole, gate/up in 4-5 row slices, down in 2, 266 kernel ops.
-    Measured on B200: 3, 4, 5, 6, 7, 8 partitions -> 434, 432, 404, 385, 405, 368 us per step."""
+# ---------------------------------------------------------------- task groups and their order
+def rows_per_task(o):
+    return 64 if o.kind == tw.BITNET_OP_FFN_GATE_UP else 128
+
+
+def ranges(o, m):
+    return ((o.x, o.x + m * o.K * (4 if o.x_dtype == tw.BITNET_DTYPE_F32 else 2)), (o.y, o.y + m * o.N * 4))
+
+
+def ov(a, b):
+    return a[0] < b[1] and b[0] < a[1]
+
+
+def check_tasks(ops, m, groups):
+    """The task groups a launch claims, in order: every op's quant group (M tasks) and rows
+    group; dependencies point backwards, include every ordering the byte ranges require
+    (transitively), and none is implied by another."""
+    n = len(ops)
+    assert len(groups) == 2 * n
+    pos = {}
+    for k, gr in enumerate(groups):
+        o = ops[gr["op"]]
+        key = (gr["op"], gr["kind"])
+        assert key not in pos
+        pos[key] = k
+        want = m if gr["kind"] == "quant" else -(-o.N // rows_per_task(o))
+        assert gr["tasks"] == want
+        assert all(0 <= d < k for d in gr["deps"])
+        assert len(gr["deps"]) <= (9 if gr["kind"] == "rows" else 8)
+    # transitive closure of the reported dependencies
+    anc = [set() for _ in groups]
+    for k, gr in enumerate(groups):
+        for d in gr["deps"]:
+            anc[k] |= anc[d] | {d}
+    # reduced: no reported dependency is an ancestor of another one
+    for k, gr in enumerate(groups):
+        for d in gr["deps"]:
+            assert not any(d in anc[e] for e in gr["deps"] if e != d), (k, d)
+    for j in range(n):
+        xj, yj = ranges(ops[j], m)
+        assert pos[(j, "quant")] in anc[pos[(j, "rows")]]
+        for i in range(j):
+            xi, yi = ranges(ops[i], m)
+            if ov(yi, xj):
+                assert pos[(i, "rows")] in anc[pos[(j, "quant")]], ("read after write", i, j)
+            if ov(xi, yj):
+                assert pos[(i, "quant")] in anc[pos[(j, "rows")]], ("write after read", i, j)
+            if ov(yi, yj):
+                assert pos[(i, "rows")] in anc[pos[(j, "rows")]], ("write after write", i, j)
+    return pos
+
+
+def random_linear_extension(groups, r):
+    """A random order in which the groups could complete, given only their dependencies."""
+    left = [len(g["deps"]) for g in groups]
+    succ = [[] for _ in groups]
+    for k, g in enumerate(groups):
+        for d in g["deps"]:
+            succ[d].append(k)
+    ready = [k for k in range(len(groups)) if left[k] == 0]
+    out = []
+    while ready:
+        k = ready.pop(r.randrange(len(ready)))
+        out.append(k)
+        for v in succ[k]:
+            left[v] -= 1
+            if left[v] == 0:
+                ready.append(v)
+    assert len(out) == len(groups)
+    return out
+
+
+def simulate_groups(ops, m, groups, order, arena_lo, arena_hi):
+    """Byte-stamp model of a launch: a quant group reads its op's x, a rows group writes its y."""
+    mem = np.zeros(arena_hi - arena_lo, np.int32)
+    reads = {}
+    for k in order:
+        gr = groups[k]
+        j = gr["op"]
+        (xlo, xhi), (ylo, yhi) = ranges(ops[j], m)
+        if gr["kind"] == "quant":
+            reads[j] = mem[xlo - arena_lo: xhi - arena_lo].copy()
+        else:
+            mem[ylo - arena_lo: yhi - arena_lo] = j + 1
+    return reads, mem
+
+
+def test_tasks_of_the_bench_decode_step():
+    """30 layers with private outputs at M = 8 on 148 CTAs: every input is fresh except down's
+    (h of the same layer), so all 90 fresh quant groups come first, a down's quant group waits
+    only for its gate/up rows, and rows groups wait only for their own quant group."""
     ops = layer_stack(30, 8, shared_outputs=False)
-    L = tw.bitnet_sequence_layout(ops, 8, 4, 33)
-    assert L["part_clusters"] == [5, 4, 4, 4, 4, 4, 4, 4]
-    assert sum(L["slices"]) == 266
-    kinds = {}
-    for k, i in enumerate(L["order"]):
-        kinds.setdefault(i % 4, set()).add(L["slices"][k])
-    assert kinds[0] == {1} and kinds[1] == {1} and kinds[2] <= {4, 5} and kinds[3] == {2}
+    groups = tw.bitnet_sequence_tasks(ops, 8, 148)
+    pos = check_tasks(ops, 8, groups)
+    fresh = [k for k, g in enumerate(groups) if g["kind"] == "quant" and g["op"] % 4 != 3]
+    assert fresh == list(range(90))
+    for l in range(30):
+        gu, dn = 4 * l + 2, 4 * l + 3
+        assert groups[pos[(dn, "quant")]]["deps"] == [pos[(gu, "rows")]]
+        for j in (4 * l, 4 * l + 1, gu, dn):
+            assert groups[pos[(j, "rows")]]["deps"] == [pos[(j, "quant")]]
+    assert sum(g["tasks"] for g in groups) == 30 * (4 * 8 + 20 + 20 + 108 + 20)
 
 
-@pytest.mark.parametrize("seed", range(12))
-def test_random_layouts_keep_every_hazard_inside_a_partition(seed):
-    """Random op lists over a shared arena (partial overlaps of every kind) and random
-    large projections: whatever partitions and row slices the planner picks, every op
-    runs after, and in the same partition as, every earlier op it conflicts with, and
-    the execution order leaves every read and the final memory as list order does."""
+def test_tasks_of_a_stack_sharing_its_output_buffers():
+    ops = layer_stack(6, 8, shared_outputs=True)
+    groups = tw.bitnet_sequence_tasks(ops, 8, 148)
+    pos = check_tasks(ops, 8, groups)
+    for l in range(1, 6):
+        q, gu = 4 * l, 4 * l + 2
+        # q overwrites the previous layer's q output: waits for those rows
+        assert pos[(q - 4, "rows")] in groups[pos[(q, "rows")]]["deps"]
+        # gate/up overwrites h, which the previous down's quant group still reads
+        assert pos[(gu + 1 - 4, "quant")] in groups[pos[(gu, "rows")]]["deps"]
+
+
+def test_too_many_dependencies_are_refused():
+    """An op whose output overwrites the inputs of 9 independent earlier readers would wait
+    on 9 groups (more than a task records): refused, never run with a wait missing."""
+    m, k = 1, 64
+    y = BASE
+    readers = [lin(y + 128 * i, k, 16, BASE + (1 << 20) + 4096 * i, BASE + (1 << 30) + (1 << 20) * i)
+               for i in range(9)]
+    writer = lin(BASE + (2 << 20), k, 9 * 32, y, BASE + (1 << 31))
+    with pytest.raises(tw.BitnetError) as e:
+        tw.bitnet_sequence_tasks(readers + [writer], m, 148)
+    assert e.value.status == tw.BITNET_ERR_UNSUPPORTED_SHAPE
+    groups = tw.bitnet_sequence_tasks(readers[:8] + [writer], m, 148)  # 8 readers: fine
+    check_tasks(readers[:8] + [writer], m, groups)
+
+
+@pytest.mark.parametrize("seed", range(16))
+def test_random_task_orders_preserve_every_read_and_the_final_memory(seed):
+    """Random op lists over a shared arena (partial overlaps of every kind): the task groups'
+    dependencies cover every required ordering, and ANY order in which the groups could
+    complete under those dependencies reads and leaves exactly what list order does."""
     r = random.Random(1000 + seed)
     m = r.choice([1, 8, 13, 64])
     arena = BASE
+    size = 16 * 20000
     ops = []
     wbase = BASE + (1 << 34)
-    for j in range(r.randint(2, 60)):
-        k = 64 * r.randint(1, 40)
-        n = r.choice([r.randint(1, 300), r.randint(2000, 9000)])
+    for j in range(r.randint(2, 40)):
+        k = 64 * r.randint(1, 8)
+        n = r.randint(1, 300)
         f32 = r.random() < 0.3
-        x = arena + 16 * r.randint(0, 200000)
-        y = arena + 16 * r.randint(0, 200000)
-        xb = m * k * (4 if f32 else 2)
-        if x < y + m * n * 4 and y < x + xb:
-            y = x + xb + 16 * r.randint(0, 64)
+        xb, yb = m * k * (4 if f32 else 2), m * n * 4
+        if xb > size or yb > size:
+            continue
+        x = arena + 16 * r.randint(0, (size - xb) // 16)
+        y = arena + 16 * r.randint(0, (size - yb) // 16)
+        if x < y + yb and y < x + xb:
+            continue
         w = wbase + j * (1 << 26)
         if r.random() < 0.3:
             ops.append(op(tw.BITNET_OP_FFN_GATE_UP, x, k, n, y, w, w + (1 << 25), w + (1 << 24), w + (3 << 23),
                           f32=f32))
         else:
             ops.append(lin(x, k, n, y, w, w + (1 << 25), f32=f32))
-    prev = tw.bitnet_set_sequence_partitions(r.choice([0, 0, 2, 4, 8]))
-    try:
-        L = tw.bitnet_sequence_layout(ops, m, r.choice([4, 8]), r.choice([16, 33]))
-    except tw.BitnetError as e:
-        assert e.status == tw.BITNET_ERR_UNSUPPORTED_SHAPE  # more row slices than one launch holds
+    if not ops:
         return
-    finally:
-        tw.bitnet_set_sequence_partitions(prev)
+    try:
+        groups = tw.bitnet_sequence_tasks(ops, m, r.choice([1, 7, 148]))
+    except tw.BitnetError as e:
+        assert e.status == tw.BITNET_ERR_UNSUPPORTED_SHAPE  # an op with more than 8 waits
+        return
+    check_tasks(ops, m, groups)
     n_ops = len(ops)
-    assert sorted(L["order"]) == list(range(n_ops))
-    pos = {i: k for k, i in enumerate(L["order"])}
-    for j, pre in enumerate(producers(ops, m)):
-        for i in pre:
-            assert pos[i] < pos[j] and L["part_of"][pos[i]] == L["part_of"][pos[j]]
-    lo = arena
-    hi = max(max(o.x + m * o.K * 4, o.y + m * o.N * 4) for o in ops) + 16
+    lo, hi = arena, arena + size
     reads_a, mem_a = simulate(ops, m, list(range(n_ops)), lo, hi)
-    reads_b, mem_b = simulate(ops, m, L["order"], lo, hi)
-    assert np.array_equal(mem_a, mem_b)
-    for j in range(n_ops):
-        assert np.array_equal(reads_a[j], reads_b[j])
+    for _ in range(6):
+        order = random_linear_extension(groups, r)
+        reads_b, mem_b = simulate_groups(ops, m, groups, order, lo, hi)
+        assert np.array_equal(mem_a, mem_b)
+        for j in range(n_ops):
+            assert np.array_equal(reads_a[j], reads_b[j])
