@@ -58,6 +58,8 @@ def parse_args():
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--cpu-seconds", type=float, default=10.0, help="budget of the oracle CPU baseline")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-configs", action="store_true",
+                   help="skip the single-BitLinear and FFN lines at decode sizes (configs 2 and 3)")
     p.add_argument("--decode-path", choices=["sequence", "per-op"], default="sequence",
                    help="decode step as one persistent bitnet_decode_sequence launch (default) or one "
                         "bitnet_linear / bitnet_ffn_gate_up call per projection")
@@ -124,18 +126,67 @@ def oracle_layer_sample(tokens, seed=4242):
                  f"single thread; tokens/s per layer = tokens / time")
 
 
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
+_WORKER_RUN = []
+
+
+def _oracle_init(tokens, seed):
+    """Pool initializer: pack the one-layer oracle sample's weights once per worker process."""
+    _WORKER_RUN.append(oracle_layer_sample(tokens, seed=seed)[0])
+
+
+def _oracle_worker(reps):
+    """One pool task: `reps` passes of the worker's oracle sample; returns its run time."""
+    run = _WORKER_RUN[0]
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        run()
+    return time.perf_counter() - t0
+
+
 def cpu_baseline(budget_s, tokens=8):
+    """The oracle as it stands, on the host: single-threaded, then one independent copy per host core
+    (a spawn-started process pool; the oracle itself is unchanged and single-threaded)."""
     run, desc = oracle_layer_sample(tokens)
     run()  # warm
     times = []
-    t_end = time.perf_counter() + budget_s
+    t_end = time.perf_counter() + budget_s / 2
     while time.perf_counter() < t_end or len(times) < 2:
         t0 = time.perf_counter()
         run()
         times.append(time.perf_counter() - t0)
-    mean = statistics.mean(times)
-    return {"value": tokens / mean, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"{desc}; {len(times)} repetitions, {sum(times):.1f} s"}
+    single = tokens / statistics.mean(times)
+    cores = os.cpu_count() or 1
+    out = {"value": single, "unit": UNIT, "cores": 1, "kind": "oracle",
+           "sample": f"{desc}; {len(times)} repetitions, {sum(times):.1f} s",
+           "host_cores": cores, "cpu_model": cpu_model()}
+    if cores > 1:
+        import multiprocessing as mp
+        reps = max(1, int(budget_s / 2 / statistics.mean(times)))
+        try:
+            with mp.get_context("spawn").Pool(cores, initializer=_oracle_init, initargs=(tokens, 4242)) as pool:
+                pool.map(_oracle_worker, [0] * cores, chunksize=1)  # every worker started and packed, untimed
+                t0 = time.perf_counter()
+                pool.map(_oracle_worker, [reps] * cores, chunksize=1)
+                wall = time.perf_counter() - t0
+            out["value"] = cores * reps * tokens / wall
+            out["cores"] = cores
+            out["sample"] = (f"{desc.replace('single thread', f'{cores} processes (one per host core)')}; "
+                             f"{reps} repetitions per process, {wall:.1f} s wall")
+            out["single_thread"] = {"value": single, "cores": 1}
+        except Exception as e:  # noqa: BLE001 - the single-thread figure stands
+            out["all_cores_error"] = f"{type(e).__name__}: {e}"
+    return out
 
 
 def reference_arm(a, n_gpus):
@@ -212,6 +263,102 @@ class ClockSampler:
         reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
                 "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ configs 2 and 3
+def check_context(torch, tw, where):
+    """Raise if the CUDA context holds a sticky error or a device-side wait gave up: numbers taken
+    after that would come from a broken context."""
+    torch.cuda.synchronize()
+    stat = tw.bitnet_device_status(clear=False)
+    if stat != 0:
+        raise RuntimeError(f"{where}: device status {tw.bitnet_status_string(stat)}")
+
+
+def decode_configs(st, stream, hbm_peak, l2_bytes):
+    """Single BitLinears and FFNs at decode sizes, each timed two ways (CUDA events over a CUDA graph):
+      per_op    one bitnet_linear / bitnet_ffn_gate_up call per projection, consecutive calls rotating
+                over distinct weight copies (>= 3 x L2 of weights), so every call streams from HBM;
+      sequence  the same projections as independent ops of one bitnet_decode_sequence launch.
+    GEMV at M = 1: 2560 -> 2560, 2560 -> 6912, 6912 -> 2560.  FFN at M in {1, 8, 16, 32, 64}: gate/up
+    2560 -> 2 x 6912 with relu(gate)^2 * up, then down 6912 -> 2560 on its h (the stack's 30 layers of
+    weights, 398 MB).  Bytes = packed weights + activations in + outputs."""
+    torch, tw = st.torch, st.tw
+    dev = st.dev
+    f32 = torch.float32
+    out = {"gemv_m1": {}, "ffn": {}}
+
+    def timed(fn, n_calls, reps=5):
+        g = capture(torch, stream, fn)
+        ms = time_graph(torch, stream, g, reps)
+        del g
+        return ms / n_calls
+
+    def line(us, nbytes, tokens=None):
+        gbs = nbytes / (us / 1e6) / 1e9
+        d = {"us": us, "bytes": nbytes, "gbs": gbs, "frac_hbm": gbs / hbm_peak}
+        if tokens is not None:
+            d["tokens_per_s"] = tokens / (us / 1e6)
+        return d
+
+    with torch.cuda.stream(stream):
+        # ---- config 2: GEMV at M = 1 ----
+        x1 = torch.randn((1, INTER), generator=st.gen, device=dev).to(torch.bfloat16)
+        for (k, n) in ((HIDDEN, HIDDEN), (HIDDEN, INTER), (INTER, HIDDEN)):
+            lat = torch.randn((n, k), generator=st.gen, device=dev, dtype=f32).mul_(0.02)
+            p0, g0 = tw.bitnet_pack_weights(lat)
+            del lat
+            wbytes = n * k // 4
+            copies = max(128, -(-3 * l2_bytes // wbytes))
+            ws = torch.empty(copies * wbytes, dtype=torch.uint8, device=dev).view(copies, n, k // 4)
+            ws.copy_(p0.unsqueeze(0).expand(copies, n, k // 4))
+            x = x1[:, :k].contiguous()
+            ys = torch.empty((copies, 1, n), dtype=f32, device=dev)
+            wsp = torch.empty(tw.bitnet_workspace_size(1, n, k), dtype=torch.uint8, device=dev)
+            per_call = wbytes + k * 2 + n * 4
+            us = timed(lambda s: [tw.bitnet_linear(x, ws[c], g0, y=ys[c], workspace=wsp, stream=s)
+                                  for c in range(copies)], copies) * 1e3
+            key = f"{k}x{n}"
+            out["gemv_m1"][key] = {"per_op": line(us, per_call), "copies": copies}
+            # one launch of 128 independent GEMVs (two alternating halves of the copies)
+            nseq = 128
+            halves = [[tw.linear_op(x, ws[(h * nseq + c) % copies], g0, ys[(h * nseq + c) % copies])
+                       for c in range(nseq)] for h in range(2)]
+            wsq = tw.bitnet_sequence_workspace(dev, nseq, 1, k)
+            us = timed(lambda s: [tw.bitnet_decode_sequence(halves[r % 2], 1, wsq, stream=s) for r in range(4)],
+                       4) * 1e3
+            out["gemv_m1"][key]["sequence"] = line(us / nseq, per_call)
+            out["gemv_m1"][key]["sequence"]["ops_per_launch"] = nseq
+            del ws, ys, wsq
+            check_context(torch, tw, f"gemv {key}")
+        # ---- config 3: FFN (gate/up + down) at M in {1, 8, 16, 32, 64} ----
+        L = st.layers
+        nl = len(L)
+        for m in (1, 8, 16, 32, 64):
+            xs = [torch.randn((m, HIDDEN), generator=st.gen, device=dev).to(torch.bfloat16) for _ in range(nl)]
+            hs = [torch.empty((m, INTER), dtype=f32, device=dev) for _ in range(nl)]
+            ds = [torch.empty((m, HIDDEN), dtype=f32, device=dev) for _ in range(nl)]
+            wsp = torch.empty(tw.bitnet_workspace_size(m, INTER, INTER), dtype=torch.uint8, device=dev)
+            per_ffn = 3 * INTER * HIDDEN // 4 + m * HIDDEN * 2 + 2 * m * INTER * 4 + m * HIDDEN * 4
+
+            def per_op(s):
+                for l in range(nl):
+                    tw.bitnet_ffn_gate_up(xs[l], L[l]["gate"][0], L[l]["gate"][1], L[l]["up"][0], L[l]["up"][1],
+                                          h=hs[l], workspace=wsp, stream=s)
+                    tw.bitnet_linear(hs[l], L[l]["down"][0], L[l]["down"][1], y=ds[l], workspace=wsp, stream=s)
+            us = timed(per_op, nl) * 1e3
+            ops = []
+            for l in range(nl):
+                ops += [tw.ffn_gate_up_op(xs[l], L[l]["gate"][0], L[l]["gate"][1], L[l]["up"][0], L[l]["up"][1],
+                                          hs[l]),
+                        tw.linear_op(hs[l], L[l]["down"][0], L[l]["down"][1], ds[l])]
+            wsq = tw.bitnet_sequence_workspace(dev, len(ops), m, INTER)
+            us_seq = timed(lambda s: [tw.bitnet_decode_sequence(ops, m, wsq, stream=s) for _ in range(3)], 3) * 1e3
+            out["ffn"][f"M={m}"] = {"per_op": line(us, per_ffn, m), "sequence": line(us_seq / nl, per_ffn, m)}
+            out["ffn"][f"M={m}"]["sequence"]["ffns_per_launch"] = nl
+            del xs, hs, ds, wsp, wsq
+            check_context(torch, tw, f"ffn M={m}")
+    return out
 
 
 # ------------------------------------------------------------------ our arm
@@ -395,7 +542,7 @@ def time_graph(torch, stream, graph, reps):
 # The sources each measured kernel family is built from (its device code, the headers that code
 # includes, and the host code that plans and launches it); include/bitnet.h is always added.
 KIND_SOURCES = {
-    "decode_sequence": ["bitnet.cu", "common.cuh", "decode.cuh", "decode_cluster.cuh", "decode_seq.cuh",
+    "decode_sequence": ["bitnet.cu", "common.cuh", "decode.cuh", "decode_tasks.cuh", "exact_sumsq.cuh",
                         "pack_quant.cuh"],
     "prefill": ["bitnet.cu", "common.cuh", "pack_quant.cuh", "prefill.cuh"],
 }
@@ -571,6 +718,7 @@ def our_arm(a, n_gpus):
     pre_tops = pre_ops / (pre_ms / 1e3) / 1e12
     int8_peak_sust = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]) * \
         NOMINAL_INT8_PER_BF16
+    int8_peak_burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]) * NOMINAL_INT8_PER_BF16
     pk_w = st.packed_bytes
     act_dec = Lyr * (B * HIDDEN * 2 * 3 + B * INTER * 4 + B * HIDDEN * 4 * 3 + B * INTER * 4)
     dec_bytes_step = pk_w + act_dec
@@ -583,7 +731,9 @@ def our_arm(a, n_gpus):
         "prefill_tokens_per_s_per_layer": M * Lyr / (pre_ms / 1e3),
         "decode_ms_per_step": dec_step_ms, "decode_gbs": dec_gbs, "decode_frac_hbm": dec_gbs / hbm_peak,
         "decode_tokens_per_s_per_layer": B * Lyr / (dec_step_ms / 1e3),
-        "peaks": f"{peaks_src}: HBM {hbm_peak} GB/s; int8 = sustained bf16 x {NOMINAL_INT8_PER_BF16}",
+        "peaks": (f"{peaks_src}: HBM {hbm_peak} GB/s; int8 of the prefill pass (a long phase) = sustained "
+                  f"bf16 x {NOMINAL_INT8_PER_BF16}; int8 of a kind timed alone = burst bf16 x "
+                  f"{NOMINAL_INT8_PER_BF16} = {int8_peak_burst:.0f} TOPS"),
     }
 
     # ---- per-kernel averages (CUDA events over graphs of one projection kind) ----
@@ -649,6 +799,8 @@ def our_arm(a, n_gpus):
                     fn(stream)
                     stream.synchronize()
                 except Exception as e:  # noqa: BLE001
+                    # a host-side refusal is reported; a broken context ends the run
+                    check_context(torch, tw, name)
                     kinds[name] = {"error": f"{type(e).__name__}: {e}", "in_step": False, "share_est": 0.0}
                     continue
             c0 = tw.bitnet_launch_count()
@@ -659,11 +811,15 @@ def our_arm(a, n_gpus):
             except Exception as e:  # noqa: BLE001
                 if in_step:
                     raise
+                check_context(torch, tw, name)
                 kinds[name] = {"error": f"{type(e).__name__}: {e}", "in_step": False, "share_est": 0.0}
                 continue
             reps_step = per_step * (a.decode_steps if name.startswith("decode") else 1)
+            rate = work / (ms / 1e3) / (1e12 if bound == "tensor" else 1e9)
+            peak = int8_peak_burst if bound == "tensor" else hbm_peak
             kinds[name] = {"us_per_op": ms * 1e3, "kernels_per_op": kern / n_ops, "bound": bound,
-                           "work_per_op": work, "in_step": in_step,
+                           "work_per_op": work, "rate": rate, "rate_unit": "TOPS" if bound == "tensor" else "GB/s",
+                           "frac_peak": rate / peak, "in_step": in_step,
                            "ops_per_step": reps_step if in_step else 0,
                            "share_est": ms * reps_step / ms_step if in_step else 0.0}
             del g
@@ -675,8 +831,8 @@ def our_arm(a, n_gpus):
                 "frac": achieved / hbm_peak}
     else:
         achieved = d["work_per_op"] / (d["us_per_op"] / 1e6) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": int8_peak_sust, "unit": "TFLOP/s",
-                "frac": achieved / int8_peak_sust}
+        roof = {"bound": "tensor", "achieved": achieved, "peak": int8_peak_burst, "unit": "TFLOP/s",
+                "frac": achieved / int8_peak_burst}
     roof["traffic"] = dram_traffic(dom)
     roof["kernel"] = dom
     roof["peak_source"] = f"{peaks_src} (MEASURED_PEAKS.json)" if peaks_src == "measured" else "fallback"
@@ -687,6 +843,16 @@ def our_arm(a, n_gpus):
     else:
         roof["note"] = ("achieved = algorithmic bytes (packed weights + activations in + outputs) per op / "
                         "mean op time in a CUDA graph of consecutive ops (CUDA events on the launch stream)")
+
+    # ---- configs 2 and 3: single BitLinears and FFNs at decode sizes ----
+    configs = None
+    if not a.no_configs:
+        try:
+            l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+            configs = decode_configs(st, stream, hbm_peak, l2)
+        except Exception as e:  # noqa: BLE001
+            check_context(torch, tw, "decode configs")
+            configs = {"error": f"{type(e).__name__}: {e}"}
 
     # ---- end to end: pinned host inputs -> device, step, outputs -> host ----
     e2e = None
@@ -712,7 +878,30 @@ def our_arm(a, n_gpus):
         e1.synchronize()
         e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / a.e2e_steps
         e2e = {"value": aggregate_value(n_gpus, tokens_step, Lyr, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "launch": "CUDA graphs of the step's calls"}
+        # the same, with every projection called eagerly through the C ABI (argument checks, plan-cache
+        # lookups and launches on the host, no graphs): what a caller without graphs gets
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        barrier()
+        t_host = time.perf_counter()
+        e0.record(stream)
+        with torch.cuda.stream(stream):
+            for _ in range(a.e2e_steps):
+                for dx, hx in zip(st.pre_x + st.dec_x, h_pre + h_dec):
+                    dx.copy_(hx, non_blocking=True)
+                st.prefill_pass(stream)
+                for t in range(a.decode_steps):
+                    st.decode_step(t, stream)
+                for ho, o in zip(h_out, outs):
+                    ho.copy_(o, non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+        host_ms = (time.perf_counter() - t_host) * 1e3 / a.e2e_steps
+        eager_ms = max_over_ranks(e0.elapsed_time(e1)) / a.e2e_steps
+        e2e["eager"] = {"value": aggregate_value(n_gpus, tokens_step, Lyr, eager_ms), "ms_per_step": eager_ms,
+                        "host_ms_per_step": host_ms,
+                        "calls_per_step": Lyr * 4 + (a.decode_steps if seq else a.decode_steps * Lyr * 4)}
 
     cpu = None
     if rank == 0 and n_gpus == 1 and not a.no_cpu_baseline:
@@ -724,6 +913,7 @@ def our_arm(a, n_gpus):
             "warmup": a.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "int8", "data": "synthetic (seeded random activations and latents)",
             "config": workload_config(a, n_gpus), "phases": phases, "roofline": roof, "kernels": kinds,
+            "decode_configs": configs,
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int((launches_pre + launches_dec) * a.steps),
             "gpu_launches_per_step": {"prefill": int(launches_pre), "decode": int(launches_dec)},
             "clocks": clk, "gpu": torch.cuda.get_device_name(dev),

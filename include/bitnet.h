@@ -173,8 +173,9 @@ bitnet_status_t bitnet_linear(const void *x, bitnet_dtype_t x_dtype, int64_t M, 
  * > 8 MiB, are rejected with BITNET_ERR_WORKSPACE before anything is launched.
  *
  * The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress, with that device current); make that first call
- * before any stream capture.  No call allocates or frees memory.  All calls
+ * (cudaGetSymbolAddress, with that device current), and so does the first
+ * call after the device's context has been destroyed and created again
+ * (cudaDeviceReset); make those calls before any stream capture.  No call allocates or frees memory.  All calls
  * share the one array and it keeps the last call's contents (nothing in it
  * needs to start at zero): calls that can overlap on the GPU -- on different
  * streams, or on different host threads -- race on it and give wrong

@@ -1084,21 +1084,50 @@ bitnet_status_t decode_sequence(const bitnet_op_t *ops, int n, int64_t M, void *
 // Callers of that entry point cannot allocate, so its scratch is a static
 // device array (every GPU that loads the library holds it until exit).  Host
 // code must not use the symbol as a pointer: it is a host-side stand-in, and
-// the device address is looked up once per device below.
+// the device address is looked up once per device and context below.
 constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 // Device address of g_noalloc_scratch on the current device (looked up on the
-// first call per device, with that device current); nullptr on failure.
+// first call per device and context, with that device current); nullptr on
+// failure.  The context is part of the key: if the primary context is torn
+// down and created again (cudaDeviceReset), the module is loaded again and
+// the array may live at another address.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+
+CUcontext current_context()
+{
+    static CtxGetCurrentFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(p);
+    });
+    CUcontext c = nullptr;
+    if (!fn || fn(&c) != CUDA_SUCCESS) return nullptr;
+    return c;
+}
+
 void *noalloc_scratch(int dev)
 {
-    static std::atomic<void *> cache[kMaxDevices];
+    struct Entry {
+        CUcontext ctx = nullptr;
+        void *ptr = nullptr;
+    };
+    static Entry cache[kMaxDevices];
+    static std::mutex mu;
     if (dev < 0 || dev >= kMaxDevices) return nullptr;
-    void *p = cache[dev].load();
-    if (p) return p;
+    const CUcontext ctx = current_context();
+    if (!ctx) return nullptr;
+    std::lock_guard<std::mutex> lk(mu);
+    if (cache[dev].ptr && cache[dev].ctx == ctx) return cache[dev].ptr;
     void *q = nullptr;
     if (cudaGetSymbolAddress(&q, g_noalloc_scratch) != cudaSuccess || q == nullptr) return nullptr;
-    cache[dev].store(q);
+    cache[dev].ctx = ctx;
+    cache[dev].ptr = q;
     return q;
 }
 
