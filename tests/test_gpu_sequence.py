@@ -284,7 +284,11 @@ def test_workspace_too_small_is_rejected():
     m = 8
     L = make_layer(800, m)
     ops = layer_ops(L)
-    need = tw.bitnet_sequence_workspace_size(4, m, I)
+    up = lambda v: (v + 255) // 256 * 256  # noqa: E731
+    need = up(4 * (2 + 2 * 4)) + sum(up(o.K * 8) + 512 for o in ops)  # the documented exact size, Mp = 8
+    assert need < tw.bitnet_sequence_workspace_size(4, m, I)
+    tw.bitnet_decode_sequence(ops, m, torch.zeros(need, dtype=torch.uint8, device=DEV))  # exactly enough
+    torch.cuda.synchronize()
     ws = torch.zeros(need - 256, dtype=torch.uint8, device=DEV)
     c0 = tw.bitnet_launch_count()
     with pytest.raises(tw.BitnetError) as e:
