@@ -99,6 +99,8 @@ LINEAR_SHAPES = [
     (40, 1024, 1000, "outliers", "f32"),      # 5 token tiles, fp32 input
     (8, 2560, 640, "normal", "bf16"),         # K / V projections of the 2B4T layer (GQA, 5 KV heads)
     (8, 2560, 3840, "normal", "bf16"),        # fused q|k|v projection
+    (32, 6912, 2560, "normal", "f32"),        # batched decode down projections (M = 32, 64)
+    (64, 6912, 2560, "outliers", "f32"),
 ]
 
 
@@ -142,10 +144,13 @@ def test_linear_prefill_full_size_sampled(k, n):
     W = make_weights(n, k, 700 + k)
     xd, xf = make_x(m, k, 800 + k, "student_t_rows", "bf16")
     y, acc, x_q, s = run_linear(xd, W, tw.BITNET_DISPATCH_AUTO, m, k, n)
+    # the quantiser on every row
+    xq_all, s_all, _ = oracle.quant_act(xf)
+    assert np.array_equal(x_q, xq_all)
+    assert np.array_equal(s.view(np.uint32), s_all.view(np.uint32))
+    # the contraction and epilogue on sampled rows: both ends and one random row of every 128-row tile
     rows = sample_rows(m, 48, 9)
     y_ref, acc_ref, xq_ref, s_ref = oracle.bitlinear(xf[rows], W["p_ref"], W["g_ref"], k)
-    assert np.array_equal(x_q[rows], xq_ref)
-    assert np.array_equal(s[rows].view(np.uint32), s_ref.view(np.uint32))
     assert np.array_equal(acc[rows].astype(np.int64), acc_ref)
     assert_rel_close(y[rows], y_ref)
     # properties that hold for every output: |acc| <= 127 * K, and y == 0 iff acc == 0
@@ -167,9 +172,19 @@ FFN_SHAPES = [
     (12, 576, 136, "outliers"),
     (1, 2560, 6912, "normal"),
     (8, 2560, 6912, "normal"),
+    (16, 2560, 6912, "outliers"),             # batched decode FFN at the 2B4T shape (M = 16, 32, 64)
+    (32, 2560, 6912, "normal"),
+    (64, 2560, 6912, "normal"),
     (32, 320, 200, "outliers"),
     (64, 256, 256, "normal"),
 ]
+
+
+def token_rows(m):
+    """All tokens up to 16; beyond, the first and last token of every 8-token tile."""
+    if m <= 16:
+        return np.arange(m)
+    return np.array(sorted({r for t in range(0, m, 8) for r in (t, min(t + 7, m - 1))}))
 
 
 @pytest.mark.parametrize("dispatch", DECODE, ids=lambda d: DNAME[d])
@@ -179,10 +194,11 @@ def test_ffn_small_m(dispatch, m, k, n, kind):
     U = make_weights(n, k, 950 + n)
     xd, xf = make_x(m, k, 1000 + m, kind)
     h, ag, au = run_ffn(xd, G, U, dispatch, m, n)
-    h_ref, ag_ref, au_ref, _, _ = oracle.ffn_gate_up(xf, G["p_ref"], G["g_ref"], U["p_ref"], U["g_ref"], k)
-    assert np.array_equal(ag.astype(np.int64), ag_ref)
-    assert np.array_equal(au.astype(np.int64), au_ref)
-    assert_rel_close(h, h_ref)
+    rows = token_rows(m)
+    h_ref, ag_ref, au_ref, _, _ = oracle.ffn_gate_up(xf[rows], G["p_ref"], G["g_ref"], U["p_ref"], U["g_ref"], k)
+    assert np.array_equal(ag[rows].astype(np.int64), ag_ref)
+    assert np.array_equal(au[rows].astype(np.int64), au_ref)
+    assert_rel_close(h[rows], h_ref)
 
 
 @pytest.mark.parametrize("m,k,n", [(4096, 2560, 6912), (200, 192, 130)])
