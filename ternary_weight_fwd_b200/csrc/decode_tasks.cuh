@@ -33,11 +33,17 @@
 //           the fragment loads hit 32 distinct banks).  Weights never wait for
 //           any other task.
 //   warp 9  activation producer: for a row task, waits for its dependencies,
-//           stages per-token rescale factors gamma / s and row sums, and streams
-//           the matching x_q chunk ([8][Mp][64] bytes) next to each weight piece.
+//           copies the per-token scales and row sums and the gammas, and streams
+//           the matching x_q chunk ([8][Mp][64] bytes) next to each weight piece
+//           (all with cp.async: it never waits for its own loads).
 //   warps 0-7 compute: quant tasks; for row tasks the contraction with
 //           mma.m16n8k32 u8 x s8 (codes c = w + 1 in {0,1,2}; the offset is
 //           removed exactly with the row sum: sum c*x - sum x) and the epilogue.
+//           They only arrive on a shared-memory barrier when a task's stores
+//           are issued.
+//   warp 10 completion: per task, once the compute warps arrived, makes their
+//           stores visible device-wide (fence) and counts the task done, so
+//           the fence's round trip stays off the compute warps.
 // Completion counters live in the caller's workspace; the last CTA out zeroes
 // them.  Every wait is bounded (device status word), and after a timeout every
 // wait returns at once, so the launch always ends.
@@ -50,7 +56,7 @@
 namespace bitnet {
 
 constexpr int DT_COMPUTE = 256;                 // compute threads (warps 0-7)
-constexpr int DT_THREADS = 320;                 // + weight producer (warp 8) + activation producer (warp 9)
+constexpr int DT_THREADS = 352;                 // + weight producer (8), activation producer (9), completion (10)
 constexpr int DT_ROWS = 128;                    // packed rows per row task
 constexpr int DT_KC = 512;                      // k per piece
 constexpr int DT_KB = DT_KC / 64;               // 64-k blocks per piece
@@ -110,11 +116,14 @@ constexpr int DT_BAR_EMPTY = DT_BAR_FULL + 8 * DT_MAX_SLOTS;
 constexpr int DT_BAR_QFULL = DT_BAR_EMPTY + 8 * DT_MAX_SLOTS;
 constexpr int DT_BAR_QINFO = DT_BAR_QFULL + 8 * DT_QUEUE;
 constexpr int DT_BAR_QEMPTY = DT_BAR_QINFO + 8 * DT_QUEUE;
-constexpr int DT_QTASK = DT_BAR_QEMPTY + 8 * DT_QUEUE; // int[DT_QUEUE]
+constexpr int DT_BAR_CDONE = DT_BAR_QEMPTY + 8 * DT_QUEUE; // compute warps done with the entry's task
+constexpr int DT_QTASK = DT_BAR_CDONE + 8 * DT_QUEUE; // int[DT_QUEUE]
 constexpr int DT_RED = 512;                           // quant-task reductions (512 bytes)
-constexpr int DT_INFO = 1024;                         // per queue entry: r0[64], r1[64] fp32, rs[64] int32
-constexpr int DT_INFO_BYTES = 3 * 4 * DT_MAX_M;
-constexpr int DT_HDR = DT_INFO + DT_QUEUE * DT_INFO_BYTES; // 4096: the piece ring starts here
+constexpr int DT_INFO = 1024;                         // per queue entry: s[64] fp32, rs[64] int32, gamma0, gamma1
+constexpr int DT_INFO_S = 0, DT_INFO_RS = 4 * DT_MAX_M, DT_INFO_G = 8 * DT_MAX_M;
+constexpr int DT_INFO_BYTES = 8 * DT_MAX_M + 16;
+constexpr int DT_HDR = 4096; // the piece ring starts here
+static_assert(DT_INFO + DT_QUEUE * DT_INFO_BYTES <= DT_HDR, "shared header");
 static_assert(DT_QTASK + 4 * DT_QUEUE <= DT_RED, "shared header");
 static_assert(DT_HDR % 128 == 0, "ring alignment");
 
@@ -170,9 +179,9 @@ BITNET_DEVINL bool dt_wait_count(const unsigned *c, unsigned target)
 BITNET_DEVINL unsigned *dt_qdone(const DtProgram &p, int j) { return p.counters + DT_CNT_OPS + 2 * j; }
 BITNET_DEVINL unsigned *dt_rdone(const DtProgram &p, int j) { return p.counters + DT_CNT_OPS + 2 * j + 1; }
 
-// Completion targets: one arrival per quant task (token), eight per row task (warps).
+// Completion targets: one count per quant task (token) and per row task.
 BITNET_DEVINL unsigned dt_qtarget(const DtProgram &p, int) { return (unsigned)p.M; }
-BITNET_DEVINL unsigned dt_rtarget(const DtProgram &p, int j) { return 8u * (unsigned)p.ops[j].rtasks; }
+BITNET_DEVINL unsigned dt_rtarget(const DtProgram &p, int j) { return (unsigned)p.ops[j].rtasks; }
 
 BITNET_DEVINL void dt_bar_compute() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
@@ -181,6 +190,11 @@ BITNET_DEVINL void dt_cp16(uint32_t dst, const void *src, bool valid)
 {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
                  : "memory");
+}
+
+BITNET_DEVINL void dt_cp4(uint32_t dst, const void *src)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
 }
 
 BITNET_DEVINL void dt_cp_arrive(uint32_t bar)
@@ -214,6 +228,11 @@ BITNET_DEVINL int dt_ld_cg_s32(const int32_t *p)
 BITNET_DEVINL int dt_pieces(int K) { return (K + DT_KC - 1) / DT_KC; }
 
 // ---- weight producer (warp 8) ----------------------------------------------
+// Lane l copies 16-byte chunk j = l % 8 (a 64-k block of the piece) of shared
+// rows r = l / 8 + 4 i, i = 0 .. 31.  Shared row r of a BitLinear task is packed
+// row 128 b + r; of a gated-FFN task (rows 8 .. 15 of each 16-row group are the
+// up rows) it is row 64 b + 8 (r / 16) + r % 8 of the gate or the up matrix.
+// For i = 4 g + q the source row is rb[q] + g * rstep: four base rows per task.
 BITNET_DEVINL void dt_weight_producer(const DtProgram &p, unsigned char *smem)
 {
     const int lane = threadIdx.x & 31;
@@ -223,9 +242,8 @@ BITNET_DEVINL void dt_weight_producer(const DtProgram &p, unsigned char *smem)
     uint64_t *qempty = reinterpret_cast<uint64_t *>(smem + DT_BAR_QEMPTY);
     volatile int *qtask = reinterpret_cast<volatile int *>(smem + DT_QTASK);
     const uint32_t ring = smem_u32(smem + DT_HDR);
-    // this lane's 16-byte chunk of a piece row and its first row; 32 rows a pass of 4 lanes... 8 lanes a row
-    const int j16 = lane & 7;   // chunk within the row (64-k block of the piece)
-    const int r0 = lane >> 3;   // rows r0, r0 + 4, ..., r0 + 124
+    const int j16 = lane & 7;
+    const int r0 = lane >> 3;
     uint32_t seq = 0, piece = 0;
     for (;;) {
         int t = 0;
@@ -243,30 +261,40 @@ BITNET_DEVINL void dt_weight_producer(const DtProgram &p, unsigned char *smem)
         const DtTask tk = dt_decode(p, t);
         if (tk.quant) continue;
         const DtOp &op = p.ops[tk.op];
-        const int K = op.K, N = op.N, rowb = K / 4;
+        const int K = op.K, N = op.N;
+        const size_t rowb = (size_t)(K / 4);
         const bool ffn = op.nmat == 2;
+        int rb[4];
+        const uint8_t *wb[4];
+        int rstep;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            if (ffn) {
+                rb[q] = tk.idx * (DT_ROWS / 2) + r0 + 4 * (q & 1);
+                wb[q] = q >= 2 ? op.w1 : op.w0;
+            } else {
+                rb[q] = tk.idx * DT_ROWS + r0 + 4 * q;
+                wb[q] = op.w0;
+            }
+        }
+        rstep = ffn ? 8 : 16;
         const int np = dt_pieces(K);
-        // source row of shared row r (ffn: rows 8..15 of each 16-row group are the up rows)
         for (int pc = 0; pc < np; ++pc) {
             const int s = (int)(piece % (uint32_t)p.n_slots);
             mbar_wait(&empty[s], ((piece / (uint32_t)p.n_slots) & 1u) ^ 1u);
             const int nkb = min(DT_KB, (K - pc * DT_KC) / 64);
-            const uint32_t dst0 = ring + (uint32_t)s * (uint32_t)p.slot_bytes;
+            const uint32_t dst0 = ring + (uint32_t)s * (uint32_t)p.slot_bytes + (uint32_t)(r0 * DT_PITCH + j16 * 16);
+            const size_t koff = (size_t)pc * (DT_KC / 4) + (size_t)j16 * 16;
             if (j16 < nkb) {
-#pragma unroll 8
-                for (int r = r0; r < DT_ROWS; r += 4) {
-                    int n;
-                    const uint8_t *w;
-                    if (ffn) {
-                        n = tk.idx * (DT_ROWS / 2) + (r >> 4) * 8 + (r & 7);
-                        w = (r & 8) ? op.w1 : op.w0;
-                    } else {
-                        n = tk.idx * DT_ROWS + r;
-                        w = op.w0;
+#pragma unroll
+                for (int g = 0; g < 8; ++g) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int n = rb[q] + g * rstep;
+                        const bool ok = n < N;
+                        const uint8_t *src = wb[q] + (ok ? (size_t)n * rowb + koff : 0);
+                        dt_cp16(dst0 + (uint32_t)((16 * g + 4 * q) * DT_PITCH), src, ok);
                     }
-                    const bool ok = n < N;
-                    const uint8_t *src = w + (size_t)(ok ? n : 0) * rowb + pc * (DT_KC / 4) + j16 * 16;
-                    dt_cp16(dst0 + (uint32_t)(r * DT_PITCH + j16 * 16), src, ok);
                 }
             }
             dt_cp_arrive(smem_u32(&full[s]));
@@ -311,17 +339,15 @@ BITNET_DEVINL void dt_act_producer(const DtProgram &p, unsigned char *smem)
                 }
             }
             __syncwarp();
-            // per-token rescale factors fl(gamma / s) and row sums of this task's op
-            float *inf = reinterpret_cast<float *>(smem + DT_INFO + e * DT_INFO_BYTES);
-            const float g0 = __ldg(op.gamma0), g1 = op.nmat == 2 ? __ldg(op.gamma1) : 0.0f;
-            for (int m = lane; m < Mp; m += 32) {
-                const float sm = m < p.M ? dt_ld_cg_f32(op.s + m) : 1.0f;
-                inf[m] = __fdiv_rn(g0, sm);
-                inf[DT_MAX_M + m] = __fdiv_rn(g1, sm);
-                reinterpret_cast<int *>(inf)[2 * DT_MAX_M + m] = m < p.M ? dt_ld_cg_s32(op.rs + m) : 0;
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&qinfo[e]);
+            // scales, row sums and gammas of this task's op into the entry (asynchronous: the
+            // entry's info barrier completes when they have landed)
+            const uint32_t inf = smem_u32(smem + DT_INFO + e * DT_INFO_BYTES);
+            const int ch = Mp / 4; // 16-byte chunks of Mp floats
+            if (lane < ch) dt_cp16(inf + DT_INFO_S + 16 * lane, op.s + 4 * lane, true);
+            else if (lane >= 16 && lane < 16 + ch) dt_cp16(inf + DT_INFO_RS + 16 * (lane - 16), op.rs + 4 * (lane - 16), true);
+            else if (lane == 30) dt_cp4(inf + DT_INFO_G, op.gamma0);
+            else if (lane == 31 && op.nmat == 2) dt_cp4(inf + DT_INFO_G + 4, op.gamma1);
+            dt_cp_arrive(smem_u32(&qinfo[e]));
             // the x_q chunk of every piece: [8 k-blocks][Mp][64] bytes, contiguous in the workspace
             const int np = dt_pieces(op.K);
             for (int pc = 0; pc < np; ++pc) {
@@ -335,8 +361,8 @@ BITNET_DEVINL void dt_act_producer(const DtProgram &p, unsigned char *smem)
                 dt_cp_arrive(smem_u32(&full[s]));
                 ++piece;
             }
-        } else if (lane == 0) {
-            mbar_arrive(&qinfo[e]); // keeps the entry's phases in step
+        } else {
+            mbar_arrive(&qinfo[e]); // keeps the entry's phases in step (every lane: the count is 32)
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&qempty[e]);
@@ -523,6 +549,7 @@ BITNET_DEVINL void dt_compute(const DtProgram &p, unsigned char *smem)
     uint64_t *qfull = reinterpret_cast<uint64_t *>(smem + DT_BAR_QFULL);
     uint64_t *qinfo = reinterpret_cast<uint64_t *>(smem + DT_BAR_QINFO);
     uint64_t *qempty = reinterpret_cast<uint64_t *>(smem + DT_BAR_QEMPTY);
+    uint64_t *cdone = reinterpret_cast<uint64_t *>(smem + DT_BAR_CDONE);
     const volatile int *qtask = reinterpret_cast<const volatile int *>(smem + DT_QTASK);
     const uint32_t ring = smem_u32(smem + DT_HDR);
     const int Mp = p.Mp, M = p.M;
@@ -541,11 +568,10 @@ BITNET_DEVINL void dt_compute(const DtProgram &p, unsigned char *smem)
             dt_bar_compute();
             if (op.xf32) dt_quant_row<true>(p, op, tk.idx, smem);
             else dt_quant_row<false>(p, op, tk.idx, smem);
-            // (dt_quant_row ends with a barrier after every store of the row)
-            if (tid == 0) {
-                __threadfence();
-                atomicAdd(dt_qdone(p, tk.op), 1u);
-            }
+            // (dt_quant_row ends with a barrier after every x_q store; thread 0 stored s and the
+            // row sum after it): the completion warp counts the task once every warp arrived
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&cdone[e]);
         } else {
             int acc[NACC][TT][4];
 #pragma unroll
@@ -575,11 +601,14 @@ BITNET_DEVINL void dt_compute(const DtProgram &p, unsigned char *smem)
                     for (int c = 0; c < 4; ++c) acc[0][tt][c] += acc[a][tt][c];
             // epilogue: y = fl((float)(sum c*x - sum x) * fl(gamma / s))
             mbar_wait(&qinfo[e], (seq / DT_QUEUE) & 1u);
-            const float *inf = reinterpret_cast<const float *>(smem + DT_INFO + e * DT_INFO_BYTES);
-            const int *irs = reinterpret_cast<const int *>(inf) + 2 * DT_MAX_M;
+            const unsigned char *inf = smem + DT_INFO + e * DT_INFO_BYTES;
+            const float *is = reinterpret_cast<const float *>(inf + DT_INFO_S);
+            const int *irs = reinterpret_cast<const int *>(inf + DT_INFO_RS);
+            const float g0 = *reinterpret_cast<const float *>(inf + DT_INFO_G);
             const int N = op.N;
             float *y = op.y;
             if (op.nmat == 2) {
+                const float g1 = *reinterpret_cast<const float *>(inf + DT_INFO_G + 4);
                 const int n = tk.idx * (DT_ROWS / 2) + warp * 8 + g;
 #pragma unroll
                 for (int tt = 0; tt < TT; ++tt)
@@ -588,8 +617,9 @@ BITNET_DEVINL void dt_compute(const DtProgram &p, unsigned char *smem)
                         const int m = tt * 8 + 2 * t4 + q;
                         if (m < M && n < N) {
                             const int rsm = irs[m];
-                            const float gv = __fmul_rn((float)(acc[0][tt][q] - rsm), inf[m]);
-                            const float uv = __fmul_rn((float)(acc[0][tt][2 + q] - rsm), inf[DT_MAX_M + m]);
+                            const float sm = is[m];
+                            const float gv = __fmul_rn((float)(acc[0][tt][q] - rsm), __fdiv_rn(g0, sm));
+                            const float uv = __fmul_rn((float)(acc[0][tt][2 + q] - rsm), __fdiv_rn(g1, sm));
                             const float pg = gv > 0.0f ? gv : 0.0f;
                             y[(size_t)m * N + n] = __fmul_rn(__fmul_rn(pg, pg), uv);
                         }
@@ -603,7 +633,7 @@ BITNET_DEVINL void dt_compute(const DtProgram &p, unsigned char *smem)
                         const int m = tt * 8 + 2 * t4 + q;
                         if (m < M) {
                             const int rsm = irs[m];
-                            const float r = inf[m];
+                            const float r = __fdiv_rn(g0, is[m]);
 #pragma unroll
                             for (int h = 0; h < 2; ++h) {
                                 const int n = n0 + 8 * h;
@@ -612,16 +642,42 @@ BITNET_DEVINL void dt_compute(const DtProgram &p, unsigned char *smem)
                         }
                     }
             }
-            // every lane's stores precede (warp barrier) lane 0's fence and completion count
+            // every lane's stores precede (warp barrier) lane 0's arrival; the completion warp
+            // makes them visible device-wide and counts the task
             __syncwarp();
-            if (lane == 0) {
-                __threadfence();
-                atomicAdd(dt_rdone(p, tk.op), 1u);
-            }
+            if (lane == 0) mbar_arrive(&cdone[e]);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&qempty[e]);
         ++seq;
+    }
+}
+
+// ---- completion warp (warp 10) ----------------------------------------------
+// Tasks in queue order: once the eight compute warps arrived (their stores are
+// issued and ordered before the arrival), one fence makes the stores visible
+// at device scope and one atomic counts the task.
+BITNET_DEVINL void dt_completion(const DtProgram &p, unsigned char *smem)
+{
+    const int lane = threadIdx.x & 31;
+    uint64_t *qfull = reinterpret_cast<uint64_t *>(smem + DT_BAR_QFULL);
+    uint64_t *qempty = reinterpret_cast<uint64_t *>(smem + DT_BAR_QEMPTY);
+    uint64_t *cdone = reinterpret_cast<uint64_t *>(smem + DT_BAR_CDONE);
+    const volatile int *qtask = reinterpret_cast<const volatile int *>(smem + DT_QTASK);
+    for (uint32_t seq = 0;; ++seq) {
+        const int e = (int)(seq % DT_QUEUE);
+        const uint32_t par = (seq / DT_QUEUE) & 1u;
+        mbar_wait(&qfull[e], par);
+        const int t = qtask[e];
+        if (t < 0) break;
+        const DtTask tk = dt_decode(p, t);
+        mbar_wait(&cdone[e], par);
+        if (lane == 0) {
+            __threadfence();
+            atomicAdd(tk.quant ? dt_qdone(p, tk.op) : dt_rdone(p, tk.op), 1u);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&qempty[e]);
     }
 }
 
@@ -640,8 +696,9 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_decode_tasks(const __grid_con
         }
         for (int i = 0; i < DT_QUEUE; ++i) {
             mbar_init(&bars[DT_BAR_QFULL / 8 + i], 1);
-            mbar_init(&bars[DT_BAR_QINFO / 8 + i], 1);
-            mbar_init(&bars[DT_BAR_QEMPTY / 8 + i], 9); // compute warps + activation producer
+            mbar_init(&bars[DT_BAR_QINFO / 8 + i], 32);  // activation producer lanes (cp.async, noinc)
+            mbar_init(&bars[DT_BAR_QEMPTY / 8 + i], 10); // compute warps, activation producer, completion warp
+            mbar_init(&bars[DT_BAR_CDONE / 8 + i], 8);   // compute warps
         }
         fence_mbarrier_init();
     }
@@ -649,6 +706,7 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_decode_tasks(const __grid_con
     const int warp = tid >> 5;
     if (warp == 8) dt_weight_producer(p, smem);
     else if (warp == 9) dt_act_producer(p, smem);
+    else if (warp == 10) dt_completion(p, smem);
     else dt_compute<TT>(p, smem);
     __syncthreads();
     if (tid == 0) {
