@@ -21,9 +21,9 @@ def test_digest_ignores_comments_but_tracks_code(tmp_path, monkeypatch):
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     d0 = bench.source_digest("decode_sequence")
     p0 = bench.source_digest("prefill_q_o")
-    (csrc / "decode_seq.cuh").write_text("// a different comment\nint decode_seq_v = 1;  /* and another */\n")
+    (csrc / "decode_tasks.cuh").write_text("// a different comment\nint decode_tasks_v = 1;  /* and another */\n")
     assert bench.source_digest("decode_sequence") == d0          # comments only
-    (csrc / "decode_seq.cuh").write_text("int decode_seq_v = 2;\n")
+    (csrc / "decode_tasks.cuh").write_text("int decode_tasks_v = 2;\n")
     assert bench.source_digest("decode_sequence") != d0          # code changed
     assert bench.source_digest("prefill_gate_up") == p0          # not a prefill source
     (csrc / "bitnet.cu").write_text("int bitnet_v = 3;\n")
