@@ -342,11 +342,13 @@ BITNET_DEVINL void dt_act_producer(const DtProgram &p, unsigned char *smem)
             // scales, row sums and gammas of this task's op into the entry (asynchronous: the
             // entry's info barrier completes when they have landed)
             const uint32_t inf = smem_u32(smem + DT_INFO + e * DT_INFO_BYTES);
-            const int ch = Mp / 4; // 16-byte chunks of Mp floats
-            if (lane < ch) dt_cp16(inf + DT_INFO_S + 16 * lane, op.s + 4 * lane, true);
-            else if (lane >= 16 && lane < 16 + ch) dt_cp16(inf + DT_INFO_RS + 16 * (lane - 16), op.rs + 4 * (lane - 16), true);
-            else if (lane == 30) dt_cp4(inf + DT_INFO_G, op.gamma0);
-            else if (lane == 31 && op.nmat == 2) dt_cp4(inf + DT_INFO_G + 4, op.gamma1);
+            const int ch = Mp / 4; // 16-byte chunks of Mp values (at most 16)
+            if (lane < ch) {
+                dt_cp16(inf + DT_INFO_S + 16 * lane, op.s + 4 * lane, true);
+                dt_cp16(inf + DT_INFO_RS + 16 * lane, op.rs + 4 * lane, true);
+            }
+            if (lane == 0) dt_cp4(inf + DT_INFO_G, op.gamma0);
+            if (lane == 1 && op.nmat == 2) dt_cp4(inf + DT_INFO_G + 4, op.gamma1);
             dt_cp_arrive(smem_u32(&qinfo[e]));
             // the x_q chunk of every piece: [8 k-blocks][Mp][64] bytes, contiguous in the workspace
             const int np = dt_pieces(op.K);
