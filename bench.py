@@ -405,7 +405,8 @@ class Stack:
                            "o": torch.empty((B, HIDDEN), dtype=f32, device=device),
                            "h": torch.empty((B, INTER), dtype=f32, device=device),
                            "down": torch.empty((B, HIDDEN), dtype=f32, device=device)} for _ in range(a.layers)]
-        ws = max(tw.bitnet_workspace_size(M, INTER, INTER), tw.bitnet_workspace_size(M, HIDDEN, HIDDEN))
+        ws = max(tw.bitnet_workspace_size(M, n, k) for n, k in ((HIDDEN, HIDDEN), (INTER, HIDDEN), (HIDDEN, INTER),
+                                                                 (QKV, HIDDEN)))
         self.ws_pre = torch.empty(ws, dtype=torch.uint8, device=device)
         self.ws_dec = torch.empty(tw.bitnet_workspace_size(B, INTER, INTER), dtype=torch.uint8, device=device)
         self.ws_seq = tw.bitnet_sequence_workspace(device, 4 * a.layers, B, INTER)

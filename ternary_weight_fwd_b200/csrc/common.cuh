@@ -269,6 +269,16 @@ BITNET_DEVINL void pdl_launch_dependents() { asm volatile("griddepcontrol.launch
 
 // ---- small utilities -----------------------------------------------------
 
+// 16-byte load through L2 only (data written by other CTAs during the kernel).
+BITNET_DEVINL uint4 ld_cg_v4(const void *p)
+{
+    uint4 v;
+    asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
 BITNET_DEVINL float warp_max(float v)
 {
 #pragma unroll

@@ -20,6 +20,11 @@
 // Tile: 128 tokens x 256 output columns x 128 k per stage, 3-stage ring.
 // Accumulators double-buffered in TMEM (2 x 256 columns) so the epilogue of
 // tile i overlaps the main loop of tile i+1.
+// Work units: the first full waves of tiles (a multiple of the grid) are whole
+// tiles; the tiles of a last, partly filled wave are split along K into S
+// parts so that the last wave fills more SMs.  A part stores its raw int32
+// sums in the workspace; per 32-row slice, the last part to arrive (integer
+// sums are exact and order-free) adds the S partials and runs the epilogue.
 // For the gate/up FFN the 256 B-rows of a tile are 128 gate rows followed by
 // the same 128 up rows, so one N=256 MMA yields both halves of h's tile.
 #pragma once
@@ -63,7 +68,42 @@ struct PrefillArgs {
     int32_t *acc0, *acc1; // optional [M][N]
     int y_bf16;           // store y as bf16 (nearest even of the fp32 value)
     int vec_ok;           // rows of y are 16-byte multiples: TMA stores
+    int full_units;       // whole tiles (units [0, full_units))
+    int split;            // K parts of each remaining tile (1: no split)
+    int num_units;        // full_units + (num_tiles - full_units) * split
+    int32_t *part;        // [tail tiles][split][PF_BM][PF_BN] int32 partial sums (split > 1)
+    unsigned *part_cnt;   // [tail tiles][4] arrivals per 32-row slice, zero before the kernel
 };
+
+// Unit u of the persistent loop: a tile (mb, nb) and a range of k-stages.
+struct PfUnit {
+    int mb, nb, kb0, kb1;
+    int part; // -1: whole tile
+    int slot; // tail tile index (split parts)
+};
+
+BITNET_DEVINL PfUnit pf_unit(const PrefillArgs &a, int u)
+{
+    PfUnit r;
+    int tile;
+    if (u < a.full_units) {
+        tile = u;
+        r.kb0 = 0;
+        r.kb1 = a.num_k;
+        r.part = -1;
+        r.slot = 0;
+    } else {
+        const int v = u - a.full_units;
+        r.slot = v / a.split;
+        r.part = v - r.slot * a.split;
+        tile = a.full_units + r.slot;
+        r.kb0 = r.part * a.num_k / a.split;
+        r.kb1 = (r.part + 1) * a.num_k / a.split;
+    }
+    r.mb = tile % a.num_m;
+    r.nb = tile / a.num_m;
+    return r;
+}
 
 // codes {0,1,2} (one per byte) -> int8 {-1,0,1}: per byte (c | 0x80) - 1 cannot
 // borrow across bytes, xor 0x80 restores the sign.
@@ -186,9 +226,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             uint32_t phase = 0;
             uint32_t issued = 0, last_par = 0; // per stage bit flags
             bool ok = true;
-            for (int tile = blockIdx.x; tile < a.num_tiles && ok; tile += gridDim.x) {
-                const int mb = tile % a.num_m, nb = tile / a.num_m;
-                for (int kb = 0; kb < a.num_k; ++kb) {
+            for (int u = blockIdx.x; u < a.num_units && ok; u += gridDim.x) {
+                const PfUnit un = pf_unit(a, u);
+                const int mb = un.mb, nb = un.nb;
+                for (int kb = un.kb0; kb < un.kb1; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1)) {
                         ok = false;
                         break;
@@ -223,11 +264,12 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             int acc = 0;
             uint32_t acc_phase = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < a.num_tiles && ok; tile += gridDim.x) {
+            for (int u = blockIdx.x; u < a.num_units && ok; u += gridDim.x) {
+                const PfUnit un = pf_unit(a, u);
                 if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * PF_BN);
-                for (int kb = 0; kb < a.num_k; ++kb) {
+                for (int kb = un.kb0; kb < un.kb1; ++kb) {
                     if (!mbar_wait(&full[stage], phase) || !mbar_wait(&unpacked[stage], phase)) {
                         ok = false;
                         break;
@@ -238,7 +280,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                     const uint64_t bdesc = umma_desc_k_sw128(st + PF_A_BYTES);
 #pragma unroll
                     for (int j = 0; j < PF_BK / 32; ++j)
-                        umma_i8(d_tmem, adesc + 2 * j, bdesc + 2 * j, PF_IDESC, (kb | j) != 0);
+                        umma_i8(d_tmem, adesc + 2 * j, bdesc + 2 * j, PF_IDESC, (kb != un.kb0 || j != 0) ? 1u : 0u);
                     umma_commit(&empty[stage]);
                     if (++stage == PF_STAGES) {
                         stage = 0;
@@ -263,8 +305,9 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; tile < a.num_tiles && ok; tile += gridDim.x) {
-            for (int kb = 0; kb < a.num_k; ++kb) {
+        for (int u = blockIdx.x; u < a.num_units && ok; u += gridDim.x) {
+            const PfUnit un = pf_unit(a, u);
+            for (int kb = un.kb0; kb < un.kb1; ++kb) {
                 if (!mbar_wait(&full[stage], phase)) {
                     ok = false;
                     break;
@@ -340,53 +383,131 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                     pf_store_row32(static_cast<float *>(a.y) + (size_t)m * a.N + n, o, nv, false);
             }
         };
+        // the epilogue of one 32-column chunk (BitLinear) or of one 32-column chunk of h
+        // (gate columns c, up columns c + PF_BN / 2) from its int32 sums
+        auto fin_lin = [&](const uint32_t (&v)[32], int c, int nb, int m, bool mok, float r0) {
+            const int n = nb * PF_BN + 32 * c;
+            if (n < a.N) {
+                if (a.acc0 && mok) pf_store_row32_i(a.acc0 + (size_t)m * a.N + n, v, a.N - n, false, 0);
+                float o[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) o[j] = __fmul_rn((float)(int)v[j], r0);
+                emit(o, m, n, mok);
+            }
+        };
+        auto fin_ffn = [&](const uint32_t (&vg)[32], const uint32_t (&vu)[32], int c, int nb, int m, bool mok,
+                           float r0, float r1) {
+            const int n = nb * (PF_BN / 2) + 32 * c;
+            if (n < a.N) {
+                if (mok && a.acc0) pf_store_row32_i(a.acc0 + (size_t)m * a.N + n, vg, a.N - n, false, 0);
+                if (mok && a.acc1) pf_store_row32_i(a.acc1 + (size_t)m * a.N + n, vu, a.N - n, false, 0);
+                float o[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const float gv = __fmul_rn((float)(int)vg[j], r0);
+                    const float uv = __fmul_rn((float)(int)vu[j], r1);
+                    const float gp = gv > 0.0f ? gv : 0.0f;
+                    o[j] = __fmul_rn(__fmul_rn(gp, gp), uv);
+                }
+                emit(o, m, n, mok);
+            }
+        };
+        // sum of the split parts of columns [col, col + 32) of this lane's row
+        auto part_sum = [&](const int32_t *row0, int col, uint32_t (&v)[32]) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = 0u;
+            for (int q = 0; q < a.split; ++q) {
+                const int32_t *src = row0 + (size_t)q * PF_BM * PF_BN + col;
+#pragma unroll
+                for (int j = 0; j < 32; j += 4) {
+                    const uint4 w = ld_cg_v4(src + j);
+                    v[j] += w.x;
+                    v[j + 1] += w.y;
+                    v[j + 2] += w.z;
+                    v[j + 3] += w.w;
+                }
+            }
+        };
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int tile = blockIdx.x; tile < a.num_tiles; tile += gridDim.x) {
-            const int mb = tile % a.num_m, nb = tile / a.num_m;
+        for (int u = blockIdx.x; u < a.num_units; u += gridDim.x) {
+            const PfUnit un = pf_unit(a, u);
             if (!mbar_wait(&acc_full[acc], acc_phase)) break;
             tc_fence_after();
-            const int m = mb * PF_BM + warp * 32 + lane;
+            const int m = un.mb * PF_BM + warp * 32 + lane;
             const bool mok = m < a.M;
             const float sm = mok ? a.s[m] : 1.0f;
             const float r0 = __fdiv_rn(g0, sm);
             const float r1 = FFN ? __fdiv_rn(g1, sm) : 0.0f;
             const uint32_t tb = tmem_base + ((uint32_t)(warp * 32) << 16) + (uint32_t)(acc * PF_BN);
-            if constexpr (!FFN) {
+            if (un.part < 0) {
+                if constexpr (!FFN) {
+#pragma unroll 1
+                    for (int c = 0; c < PF_BN / 32; ++c) {
+                        uint32_t v[32];
+                        tmem_ld32(tb + 32 * c, v);
+                        tmem_wait_ld();
+                        fin_lin(v, c, un.nb, m, mok, r0);
+                    }
+                } else {
+#pragma unroll 1
+                    for (int c = 0; c < PF_BN / 64; ++c) {
+                        uint32_t vg[32], vu[32];
+                        tmem_ld32(tb + 32 * c, vg);
+                        tmem_ld32(tb + PF_BN / 2 + 32 * c, vu);
+                        tmem_wait_ld();
+                        fin_ffn(vg, vu, c, un.nb, m, mok, r0, r1);
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acc_empty[acc]);
+            } else {
+                // a part of a split tile: raw sums of this row to the workspace, then the
+                // accumulator is free for the next unit
+                int32_t *prow = a.part + ((size_t)(un.slot * a.split + un.part) * PF_BM + warp * 32 + lane) * PF_BN;
 #pragma unroll 1
                 for (int c = 0; c < PF_BN / 32; ++c) {
                     uint32_t v[32];
                     tmem_ld32(tb + 32 * c, v);
                     tmem_wait_ld();
-                    const int n = nb * PF_BN + 32 * c;
-                    if (n < a.N) {
-                        if (a.acc0 && mok) pf_store_row32_i(a.acc0 + (size_t)m * a.N + n, v, a.N - n, false, 0);
-                        float o[32];
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) o[j] = __fmul_rn((float)(int)v[j], r0);
-                        emit(o, m, n, mok);
-                    }
+                    for (int j = 0; j < 32; j += 4)
+                        *reinterpret_cast<uint4 *>(prow + 32 * c + j) = make_uint4(v[j], v[j + 1], v[j + 2], v[j + 3]);
                 }
-            } else {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acc_empty[acc]);
+                // every lane's partial stores precede lane 0's fence and arrival count
+                unsigned prev = 0u;
+                if (lane == 0) {
+                    __threadfence();
+                    prev = atomicAdd(&a.part_cnt[un.slot * 4 + warp], 1u);
+                }
+                prev = __shfl_sync(0xffffffffu, prev, 0);
+                if (prev == (unsigned)(a.split - 1)) {
+                    // the last part of this 32-row slice: every other part's sums are visible
+                    if (lane == 0) {
+                        __threadfence();
+                        a.part_cnt[un.slot * 4 + warp] = 0u;
+                    }
+                    __syncwarp();
+                    const int32_t *row0 = a.part + ((size_t)un.slot * a.split * PF_BM + warp * 32 + lane) * PF_BN;
+                    if constexpr (!FFN) {
 #pragma unroll 1
-                for (int c = 0; c < PF_BN / 64; ++c) {
-                    uint32_t vg[32], vu[32];
-                    tmem_ld32(tb + 32 * c, vg);
-                    tmem_ld32(tb + PF_BN / 2 + 32 * c, vu);
-                    tmem_wait_ld();
-                    const int n = nb * (PF_BN / 2) + 32 * c;
-                    if (n < a.N) {
-                        if (mok && a.acc0) pf_store_row32_i(a.acc0 + (size_t)m * a.N + n, vg, a.N - n, false, 0);
-                        if (mok && a.acc1) pf_store_row32_i(a.acc1 + (size_t)m * a.N + n, vu, a.N - n, false, 0);
-                        float o[32];
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            const float gv = __fmul_rn((float)(int)vg[j], r0);
-                            const float uv = __fmul_rn((float)(int)vu[j], r1);
-                            const float gp = gv > 0.0f ? gv : 0.0f;
-                            o[j] = __fmul_rn(__fmul_rn(gp, gp), uv);
+                        for (int c = 0; c < PF_BN / 32; ++c) {
+                            uint32_t v[32];
+                            part_sum(row0, 32 * c, v);
+                            fin_lin(v, c, un.nb, m, mok, r0);
                         }
-                        emit(o, m, n, mok);
+                    } else {
+#pragma unroll 1
+                        for (int c = 0; c < PF_BN / 64; ++c) {
+                            uint32_t vg[32], vu[32];
+                            part_sum(row0, 32 * c, vg);
+                            part_sum(row0, PF_BN / 2 + 32 * c, vu);
+                            fin_ffn(vg, vu, c, un.nb, m, mok, r0, r1);
+                        }
                     }
                 }
             }
@@ -394,9 +515,6 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 if (mok && rmax != 0u) atomicMax(reinterpret_cast<unsigned *>(a.y_amax) + m, rmax);
                 rmax = 0;
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[acc]);
             if (++acc == 2) {
                 acc = 0;
                 acc_phase ^= 1;
