@@ -265,35 +265,50 @@ BITNET_DEVINL void dt_weight_producer(const DtProgram &p, unsigned char *smem)
         const size_t rowb = (size_t)(K / 4);
         const bool ffn = op.nmat == 2;
         int rb[4];
-        const uint8_t *wb[4];
-        int rstep;
+        const uint8_t *pb[4]; // source of this lane's chunk in row rb[q], k-offset 0
+        const int rstep = ffn ? 8 : 16;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
+            const uint8_t *w;
             if (ffn) {
                 rb[q] = tk.idx * (DT_ROWS / 2) + r0 + 4 * (q & 1);
-                wb[q] = q >= 2 ? op.w1 : op.w0;
+                w = q >= 2 ? op.w1 : op.w0;
             } else {
                 rb[q] = tk.idx * DT_ROWS + r0 + 4 * q;
-                wb[q] = op.w0;
+                w = op.w0;
             }
+            pb[q] = w + (size_t)rb[q] * rowb + (size_t)j16 * 16;
         }
-        rstep = ffn ? 8 : 16;
+        const size_t gstep = (size_t)rstep * rowb; // bytes between rows rb[q] + g * rstep, consecutive g
+        const bool all_rows = (ffn ? (tk.idx + 1) * (DT_ROWS / 2) : (tk.idx + 1) * DT_ROWS) <= N;
         const int np = dt_pieces(K);
         for (int pc = 0; pc < np; ++pc) {
             const int s = (int)(piece % (uint32_t)p.n_slots);
             mbar_wait(&empty[s], ((piece / (uint32_t)p.n_slots) & 1u) ^ 1u);
             const int nkb = min(DT_KB, (K - pc * DT_KC) / 64);
             const uint32_t dst0 = ring + (uint32_t)s * (uint32_t)p.slot_bytes + (uint32_t)(r0 * DT_PITCH + j16 * 16);
-            const size_t koff = (size_t)pc * (DT_KC / 4) + (size_t)j16 * 16;
+            const size_t koff = (size_t)pc * (DT_KC / 4);
             if (j16 < nkb) {
-#pragma unroll
-                for (int g = 0; g < 8; ++g) {
+                if (all_rows) {
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
-                        const int n = rb[q] + g * rstep;
-                        const bool ok = n < N;
-                        const uint8_t *src = wb[q] + (ok ? (size_t)n * rowb + koff : 0);
-                        dt_cp16(dst0 + (uint32_t)((16 * g + 4 * q) * DT_PITCH), src, ok);
+                        const uint8_t *src = pb[q] + koff;
+#pragma unroll
+                        for (int g = 0; g < 8; ++g)
+                            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                                             dst0 + (uint32_t)((16 * g + 4 * q) * DT_PITCH)),
+                                         "l"(src + g * gstep)
+                                         : "memory");
+                    }
+                } else {
+#pragma unroll
+                    for (int g = 0; g < 8; ++g) {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const bool ok = rb[q] + g * rstep < N;
+                            const uint8_t *src = ok ? pb[q] + koff + g * gstep : op.w0; // nothing read when !ok
+                            dt_cp16(dst0 + (uint32_t)((16 * g + 4 * q) * DT_PITCH), src, ok);
+                        }
                     }
                 }
             }
@@ -540,6 +555,49 @@ BITNET_DEVINL void dt_piece(int (&acc)[NACC][TT][4], uint32_t wrow, uint32_t xro
     }
 }
 
+// A full piece (8 k-blocks): every fragment is loaded before the first mma, so
+// the shared-memory latency is paid once per piece; the two mma of a k-block
+// go to different accumulator sets.
+template <int TT, int NACC>
+BITNET_DEVINL void dt_piece_full(int (&acc)[NACC][TT][4], uint32_t wrow, uint32_t xrow, int Mp)
+{
+    constexpr uint32_t M3 = 0x03030303u;
+    uint32_t lo[DT_KB], hi[DT_KB];
+#pragma unroll
+    for (int kb = 0; kb < DT_KB; ++kb) {
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(lo[kb]) : "r"(wrow + kb * 16));
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(hi[kb]) : "r"(wrow + 8 * DT_PITCH + kb * 16));
+    }
+    constexpr int BPRE = TT == 1 ? DT_KB : 1; // activation fragments held ahead (all of them for one tile)
+    uint4 bq[BPRE];
+    if constexpr (TT == 1) {
+#pragma unroll
+        for (int kb = 0; kb < DT_KB; ++kb)
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(bq[kb].x), "=r"(bq[kb].y), "=r"(bq[kb].z), "=r"(bq[kb].w)
+                         : "r"(xrow + (uint32_t)(kb * Mp * 64)));
+    }
+#pragma unroll
+    for (int kb = 0; kb < DT_KB; ++kb) {
+        const uint32_t l = lo[kb], h = hi[kb];
+        const uint32_t a0 = l & M3, a1 = h & M3, a2 = (l >> 2) & M3, a3 = (h >> 2) & M3;
+        const uint32_t a4 = (l >> 4) & M3, a5 = (h >> 4) & M3, a6 = (l >> 6) & M3, a7 = (h >> 6) & M3;
+#pragma unroll
+        for (int tt = 0; tt < TT; ++tt) {
+            uint4 b;
+            if constexpr (TT == 1) {
+                b = bq[kb];
+            } else {
+                asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w)
+                             : "r"(xrow + (uint32_t)((kb * Mp + tt * 8) * 64)));
+            }
+            mma_u8s8_16832(acc[(2 * kb) % NACC][tt], a0, a1, a2, a3, b.x, b.y);
+            mma_u8s8_16832(acc[(2 * kb + 1) % NACC][tt], a4, a5, a6, a7, b.z, b.w);
+        }
+    }
+}
+
 template <int TT>
 BITNET_DEVINL void dt_compute(const DtProgram &p, unsigned char *smem)
 {
@@ -590,7 +648,10 @@ BITNET_DEVINL void dt_compute(const DtProgram &p, unsigned char *smem)
                 const uint32_t wrow = base + (uint32_t)((warp * 16 + g) * DT_PITCH + t4 * 4);
                 const uint32_t xrow = base + DT_WBYTES + (uint32_t)(g * 64 + t4 * 16);
                 const int nkb = min(DT_KB, (op.K - pc * DT_KC) / 64);
-                dt_piece<TT, NACC>(acc, wrow, xrow, Mp, nkb);
+                if (nkb == DT_KB)
+                    dt_piece_full<TT, NACC>(acc, wrow, xrow, Mp);
+                else
+                    dt_piece<TT, NACC>(acc, wrow, xrow, Mp, nkb);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&empty[s]);
                 ++piece;

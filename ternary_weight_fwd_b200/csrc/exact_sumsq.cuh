@@ -140,7 +140,7 @@ BITNET_DEVINL void ss_long_add(unsigned long long *dig, float v)
 // Slow-path result: resolve the carries, take the top 128 bits (lower nonzero
 // digits folded into the lowest bit, which lies below the rounding bit) and
 // round once.
-BITNET_DEVINL double ss_long_round(const unsigned long long *dig)
+__device__ __noinline__ double ss_long_round(const unsigned long long *dig)
 {
     uint32_t w[SS_LONG_DIGITS];
     unsigned long long c = 0;

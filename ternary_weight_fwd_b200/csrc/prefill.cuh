@@ -446,7 +446,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                     for (int c = 0; c < PF_BN / 32; ++c) {
                         uint32_t v[32];
                         tmem_ld32(tb + 32 * c, v);
-                        tmem_wait_ld();
+                        tmem_wait_ld(v);
                         fin_lin(v, c, un.nb, m, mok, r0);
                     }
                 } else {
@@ -455,7 +455,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                         uint32_t vg[32], vu[32];
                         tmem_ld32(tb + 32 * c, vg);
                         tmem_ld32(tb + PF_BN / 2 + 32 * c, vu);
-                        tmem_wait_ld();
+                        tmem_wait_ld(vg);
+                        tmem_regs_fence(vu);
                         fin_ffn(vg, vu, c, un.nb, m, mok, r0, r1);
                     }
                 }
@@ -470,7 +471,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 for (int c = 0; c < PF_BN / 32; ++c) {
                     uint32_t v[32];
                     tmem_ld32(tb + 32 * c, v);
-                    tmem_wait_ld();
+                    tmem_wait_ld(v);
 #pragma unroll
                     for (int j = 0; j < 32; j += 4)
                         *reinterpret_cast<uint4 *>(prow + 32 * c + j) = make_uint4(v[j], v[j + 1], v[j + 2], v[j + 3]);
