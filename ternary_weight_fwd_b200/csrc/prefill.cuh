@@ -226,8 +226,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             uint32_t phase = 0;
             uint32_t issued = 0, last_par = 0; // per stage bit flags
             bool ok = true;
-            for (int u = blockIdx.x; u < a.num_units && ok; u += gridDim.x) {
-                const PfUnit un = pf_unit(a, u);
+            for (int unit = blockIdx.x; unit < a.num_units && ok; unit += gridDim.x) {
+                const PfUnit un = pf_unit(a, unit);
                 const int mb = un.mb, nb = un.nb;
                 for (int kb = un.kb0; kb < un.kb1; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1)) {
@@ -264,8 +264,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             int acc = 0;
             uint32_t acc_phase = 0;
             bool ok = true;
-            for (int u = blockIdx.x; u < a.num_units && ok; u += gridDim.x) {
-                const PfUnit un = pf_unit(a, u);
+            for (int unit = blockIdx.x; unit < a.num_units && ok; unit += gridDim.x) {
+                const PfUnit un = pf_unit(a, unit);
                 if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * PF_BN);
@@ -305,8 +305,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
-        for (int u = blockIdx.x; u < a.num_units && ok; u += gridDim.x) {
-            const PfUnit un = pf_unit(a, u);
+        for (int unit = blockIdx.x; unit < a.num_units && ok; unit += gridDim.x) {
+            const PfUnit un = pf_unit(a, unit);
             for (int kb = un.kb0; kb < un.kb1; ++kb) {
                 if (!mbar_wait(&full[stage], phase)) {
                     ok = false;
@@ -430,8 +430,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         };
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int u = blockIdx.x; u < a.num_units; u += gridDim.x) {
-            const PfUnit un = pf_unit(a, u);
+        for (int unit = blockIdx.x; unit < a.num_units; unit += gridDim.x) {
+            const PfUnit un = pf_unit(a, unit);
             if (!mbar_wait(&acc_full[acc], acc_phase)) break;
             tc_fence_after();
             const int m = un.mb * PF_BM + warp * 32 + lane;
