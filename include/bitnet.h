@@ -129,13 +129,8 @@ bitnet_status_t bitnet_quant_act(const void *x, bitnet_dtype_t x_dtype, int64_t 
                                  cudaStream_t stream);
 
 /*
- * Workspace needed by bitnet_linear / bitnet_ffn_gate_up for the given shape:
- * the quantised activations, scales and row sums between kernels, and, for
- * prefill shapes whose last wave of output tiles is partly filled, the int32
- * partial sums of that wave's tiles, which run split along K.  The size of
- * the latter depends on the SM count of the current device (148 on a B200,
- * which is also assumed when no device is current).  A smaller workspace of
- * at least the first part gives the same results without the split.
+ * Workspace needed by bitnet_linear / bitnet_ffn_gate_up for the given shape
+ * (holds the quantised activations, scales and row sums between kernels).
  */
 size_t bitnet_workspace_size(int64_t M, int64_t N, int64_t K);
 

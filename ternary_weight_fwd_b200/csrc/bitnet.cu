@@ -121,46 +121,20 @@ Workspace carve(void *ws, int64_t M, int64_t K)
     return w;
 }
 
-// ---- prefill split-K tail (see k_prefill) ---------------------------------------
-// The tiles of a last, partly filled wave (at most half the grid) are split along K
-// into S parts.  S balances the shorter tail (a tile's k-stages / S) against the
-// partial-sum round trip through L2 that every part adds: about 0.6 us per k-stage
-// of a tile against about 1.3 us per part (B200 measurements), so S ~ sqrt(0.46 k).
-struct PfTail {
-    int full = 0, rem = 0, split = 1;
-};
-
-PfTail pf_tail(int64_t M, int64_t N, int64_t K, int nmat, int sms)
+// ---- prefill: the partly filled last wave of tiles (see k_prefill) -------------
+// A BitLinear whose last wave holds at most a quarter (half) of the grid runs each
+// of its tiles as 4 (2) sub-tiles of 64 (128) output columns on separate CTAs.
+int pf_tail_q(int64_t M, int64_t N, int nmat, int sms)
 {
-    PfTail t;
-    const int64_t tiles = cdiv(M, PF_BM) * cdiv(N, nmat == 1 ? PF_BN : PF_BN / 2);
+    if (nmat != 1) return 1;
+    const int64_t tiles = cdiv(M, PF_BM) * cdiv(N, PF_BN);
     const int64_t grid = std::min<int64_t>(tiles, sms);
-    if (grid <= 0) return t;
+    if (grid <= 0) return 1;
     const int64_t full = tiles / grid * grid, rem = tiles - full;
-    if (full == 0 || rem == 0 || 2 * rem > grid) return t;
-    const int64_t num_k = cdiv(K, PF_BK);
-    int64_t S = (int64_t)std::lround(std::sqrt(0.46 * (double)num_k));
-    S = std::max<int64_t>(1, std::min<int64_t>({S, num_k, grid / rem}));
-    if (S == 1) return t;
-    t.full = (int)full;
-    t.rem = (int)rem;
-    t.split = (int)S;
-    return t;
-}
-
-// workspace bytes of the partial sums and arrival counters of a tail
-inline size_t pf_tail_bytes(const PfTail &t)
-{
-    if (t.split <= 1) return 0;
-    return (size_t)t.rem * t.split * PF_BM * PF_BN * 4 + align_up((size_t)t.rem * 4 * 4, 256);
-}
-
-// SM count the workspace size query plans for: the current device's, else a B200's.
-int planning_sms()
-{
-    const int dev = current_device();
-    const int sms = dev >= 0 ? num_sms_for(dev) : 0;
-    return sms > 0 ? sms : 148;
+    if (full == 0 || rem == 0) return 1;
+    if (4 * rem <= grid) return 4;
+    if (2 * rem <= grid) return 2;
+    return 1;
 }
 
 // ---- TMA descriptors ---------------------------------------------------------
@@ -282,24 +256,24 @@ cudaError_t launch_decode(const DecodeArgs &a, const DecodeCfg &c, cudaStream_t 
 // amax_zero: optional [M] zeroed for the next kernel's atomicMax.
 template <bool XF32>
 cudaError_t launch_quant_t(const void *x, int64_t M, int64_t K, int8_t *xq, float *s, int32_t *rs,
-                           const float *amax_in, float *amax_zero, ZeroList zl, cudaStream_t stream)
+                           const float *amax_in, float *amax_zero, cudaStream_t stream)
 {
     const int64_t nch = K / (XF32 ? 4 : 8);
     const int64_t per_warp = 32 * QR_NCH;
     if (nch <= per_warp)
         return launch_pdl(k_quant_rows_reg<XF32, 1>, dim3((unsigned)cdiv(M, 8)), dim3(256), 0, stream, x, M, K, xq,
-                          s, rs, amax_in, amax_zero, zl);
+                          s, rs, amax_in, amax_zero);
     if (nch <= 2 * per_warp)
         return launch_pdl(k_quant_rows_reg<XF32, 2>, dim3((unsigned)cdiv(M, 4)), dim3(256), 0, stream, x, M, K, xq,
-                          s, rs, amax_in, amax_zero, zl);
+                          s, rs, amax_in, amax_zero);
     if (nch <= 4 * per_warp)
         return launch_pdl(k_quant_rows_reg<XF32, 4>, dim3((unsigned)cdiv(M, 2)), dim3(256), 0, stream, x, M, K, xq,
-                          s, rs, amax_in, amax_zero, zl);
+                          s, rs, amax_in, amax_zero);
     if (nch <= 8 * per_warp)
         return launch_pdl(k_quant_rows_reg<XF32, 8>, dim3((unsigned)M), dim3(256), 0, stream, x, M, K, xq, s, rs,
-                          amax_in, amax_zero, zl);
+                          amax_in, amax_zero);
     return launch_pdl(k_quant_rows<XF32>, dim3((unsigned)cdiv(M, 8)), dim3(256), 0, stream, x, M, K, xq, s, rs,
-                      amax_in, amax_zero, zl);
+                      amax_in, amax_zero);
 }
 
 // RMS normalisation + quantiser: rows of up to 4096 elements on 128 threads (two rows
@@ -308,29 +282,27 @@ constexpr int64_t kNormMaxK = 256 * RQ_MAX_PER_THREAD;
 
 template <bool XF32>
 cudaError_t launch_norm_quant_t(const void *x, int64_t M, int64_t K, const float *g, float eps, int8_t *xq, float *s,
-                                int32_t *rs, float *amax_zero, ZeroList zl, cudaStream_t stream)
+                                int32_t *rs, float *amax_zero, cudaStream_t stream)
 {
     if (K <= 128 * RQ_MAX_PER_THREAD)
         return launch_pdl(k_rmsnorm_quant_rows<XF32, 128>, dim3((unsigned)cdiv(M, 2)), dim3(256), 0, stream, x, M, K,
-                          g, eps, xq, s, rs, amax_zero, zl);
+                          g, eps, xq, s, rs, amax_zero);
     return launch_pdl(k_rmsnorm_quant_rows<XF32, 256>, dim3((unsigned)M), dim3(256), 0, stream, x, M, K, g, eps, xq, s,
-                      rs, amax_zero, zl);
+                      rs, amax_zero);
 }
 
 cudaError_t launch_norm_quant(const void *x, bool xf32, int64_t M, int64_t K, const float *g, float eps, int8_t *xq,
-                              float *s, int32_t *rs, cudaStream_t stream, float *amax_zero = nullptr,
-                              ZeroList zl = ZeroList{nullptr, 0})
+                              float *s, int32_t *rs, cudaStream_t stream, float *amax_zero = nullptr)
 {
-    return xf32 ? launch_norm_quant_t<true>(x, M, K, g, eps, xq, s, rs, amax_zero, zl, stream)
-                : launch_norm_quant_t<false>(x, M, K, g, eps, xq, s, rs, amax_zero, zl, stream);
+    return xf32 ? launch_norm_quant_t<true>(x, M, K, g, eps, xq, s, rs, amax_zero, stream)
+                : launch_norm_quant_t<false>(x, M, K, g, eps, xq, s, rs, amax_zero, stream);
 }
 
 cudaError_t launch_quant(const void *x, bool xf32, int64_t M, int64_t K, int8_t *xq, float *s, int32_t *rs,
-                         cudaStream_t stream, const float *amax_in = nullptr, float *amax_zero = nullptr,
-                         ZeroList zl = ZeroList{nullptr, 0})
+                         cudaStream_t stream, const float *amax_in = nullptr, float *amax_zero = nullptr)
 {
-    return xf32 ? launch_quant_t<true>(x, M, K, xq, s, rs, amax_in, amax_zero, zl, stream)
-                : launch_quant_t<false>(x, M, K, xq, s, rs, amax_in, amax_zero, zl, stream);
+    return xf32 ? launch_quant_t<true>(x, M, K, xq, s, rs, amax_in, amax_zero, stream)
+                : launch_quant_t<false>(x, M, K, xq, s, rs, amax_in, amax_zero, stream);
 }
 
 // ---- cluster (K-split, fused quantiser) decode kernel -------------------------
@@ -664,31 +636,22 @@ bitnet_status_t forward(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_
     } else {
         tmB1 = tmB0;
     }
+    // the last, partly filled wave of a BitLinear as sub-tiles (tmB1: a box of their rows)
+    const int grid = std::min(a.num_tiles, sms);
+    a.tail_q = pf_tail_q(M, N, nmat, sms);
+    a.full_units = a.num_tiles;
+    a.num_units = a.num_tiles;
+    if (a.tail_q > 1) {
+        a.full_units = a.num_tiles / grid * grid;
+        a.num_units = a.full_units + (a.num_tiles - a.full_units) * a.tail_q;
+        if (!encode_u8_2d(&tmB1, w0, (uint64_t)N, (uint64_t)(K / 4), (uint32_t)(PF_BN / a.tail_q), PF_BK / 4, false))
+            return BITNET_ERR_CUDA;
+    }
     // output through TMA stores when rows are 16-byte multiples: 32 x 32 boxes,
     // 128-byte swizzle for fp32, 64-byte swizzle for bf16
     tmY = tmA;
     if (a.vec_ok && !encode_2d_out(&tmY, y, (uint64_t)M, (uint64_t)N, 32, 32, io.y_bf16)) return BITNET_ERR_CUDA;
-    const int grid = std::min(a.num_tiles, sms);
-    // the last, partly filled wave split along K when the workspace holds its partial sums
-    a.full_units = a.num_tiles;
-    a.split = 1;
-    a.num_units = a.num_tiles;
-    ZeroList zl{nullptr, 0};
-    {
-        const PfTail t = pf_tail(M, N, K, nmat, sms);
-        const size_t base = ws_bytes_for(M, K);
-        if (t.split > 1 && ws_bytes >= base + pf_tail_bytes(t)) {
-            char *p = static_cast<char *>(workspace) + base;
-            a.part = reinterpret_cast<int32_t *>(p);
-            a.part_cnt = reinterpret_cast<unsigned *>(p + (size_t)t.rem * t.split * PF_BM * PF_BN * 4);
-            a.full_units = t.full;
-            a.split = t.split;
-            a.num_units = t.full + t.rem * t.split;
-            zl = ZeroList{a.part_cnt, 4 * t.rem};
-        }
-    }
-    cudaError_t e = norm_g ? launch_norm_quant(x, xf32, M, K, norm_g, norm_eps, xq, s, nullptr, stream, io.y_amax, zl)
-                           : launch_quant(x, xf32, M, K, xq, s, nullptr, stream, io.x_amax, io.y_amax, zl);
+    cudaError_t e = quantise(xq, s, nullptr);
     if (e != cudaSuccess) return BITNET_ERR_CUDA;
     if (nmat == 1) {
         static std::atomic<int> done[kMaxDevices];
@@ -1257,13 +1220,9 @@ bitnet_status_t bitnet_quant_act(const void *x, bitnet_dtype_t x_dtype, int64_t 
 
 size_t bitnet_workspace_size(int64_t M, int64_t N, int64_t K)
 {
+    (void)N;
     if (M < 1 || K < 1) return 0;
-    size_t tail = 0;
-    if (N >= 1) {
-        const int sms = planning_sms();
-        tail = std::max(pf_tail_bytes(pf_tail(M, N, K, 1, sms)), pf_tail_bytes(pf_tail(M, N, K, 2, sms)));
-    }
-    return ws_bytes_for(M, K) + tail;
+    return ws_bytes_for(M, K);
 }
 
 bitnet_status_t bitnet_linear(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_t K, const uint8_t *w_packed,

@@ -117,28 +117,14 @@ BITNET_DEVINL uint2 chunk_quant(const uint4 v, float sc, int &rs)
     return q;
 }
 
-// Words the quantiser zeroes (block 0) for the kernel that follows it: the
-// prefill GEMM's split-K tail counters.
-struct ZeroList {
-    unsigned *p;
-    int n;
-};
-
-BITNET_DEVINL void zero_words(const ZeroList &z)
-{
-    if (blockIdx.x == 0)
-        for (int i = threadIdx.x; i < z.n; i += blockDim.x) z.p[i] = 0u;
-}
-
 template <bool XF32>
 __global__ void __launch_bounds__(256) k_quant_rows(const void *__restrict__ x, int64_t M, int64_t K,
                                                     int8_t *__restrict__ x_q, float *__restrict__ s,
                                                     int32_t *__restrict__ rowsum, const float *__restrict__ amax_in,
-                                                    float *__restrict__ amax_zero, const ZeroList zl)
+                                                    float *__restrict__ amax_zero)
 {
     pdl_launch_dependents();
     pdl_wait();
-    zero_words(zl);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t m = (int64_t)blockIdx.x * 8 + warp;
     if (m >= M) return;
@@ -189,13 +175,12 @@ __global__ void __launch_bounds__(256) k_quant_rows_reg(const void *__restrict__
                                                         int8_t *__restrict__ x_q, float *__restrict__ s,
                                                         int32_t *__restrict__ rowsum,
                                                         const float *__restrict__ amax_in,
-                                                        float *__restrict__ amax_zero, const ZeroList zl)
+                                                        float *__restrict__ amax_zero)
 {
     __shared__ float red_max[8];
     __shared__ int red_sum[8];
     pdl_launch_dependents();
     pdl_wait();
-    zero_words(zl);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr int RPC = 8 / WPR; // rows per CTA
     const int wr = warp % WPR;   // this warp's part of the row
@@ -284,8 +269,7 @@ template <bool XF32, int TPR>
 __global__ void __launch_bounds__(256) k_rmsnorm_quant_rows(const void *__restrict__ x, int64_t M, int64_t K,
                                                             const float *__restrict__ g, float eps,
                                                             int8_t *__restrict__ x_q, float *__restrict__ s,
-                                                            int32_t *__restrict__ rowsum, float *__restrict__ amax_zero,
-                                                            const ZeroList zl)
+                                                            int32_t *__restrict__ rowsum, float *__restrict__ amax_zero)
 {
     constexpr int RPC = 256 / TPR;         // rows per CTA
     constexpr int WPR = TPR / 32;          // warps per row
@@ -298,7 +282,6 @@ __global__ void __launch_bounds__(256) k_rmsnorm_quant_rows(const void *__restri
     __shared__ float bcast[RPC][2];
     pdl_launch_dependents();
     pdl_wait();
-    zero_words(zl);
     const int lr = threadIdx.x / TPR;      // row of this CTA
     const int t = threadIdx.x % TPR;       // thread within the row
     const int wr = t >> 5, lane = t & 31;  // warp within the row

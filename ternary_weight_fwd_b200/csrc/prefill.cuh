@@ -20,11 +20,11 @@
 // Tile: 128 tokens x 256 output columns x 128 k per stage, 3-stage ring.
 // Accumulators double-buffered in TMEM (2 x 256 columns) so the epilogue of
 // tile i overlaps the main loop of tile i+1.
-// Work units: the first full waves of tiles (a multiple of the grid) are whole
-// tiles; the tiles of a last, partly filled wave are split along K into S
-// parts so that the last wave fills more SMs.  A part stores its raw int32
-// sums in the workspace; per 32-row slice, the last part to arrive (integer
-// sums are exact and order-free) adds the S partials and runs the epilogue.
+// Work units (BitLinear): the first full waves of tiles (a multiple of the
+// grid) are whole tiles; each tile of a last, partly filled wave runs as Q
+// sub-tiles of 256 / Q output columns (Q = 2 or 4, an N = 128 or 64 MMA) on Q
+// CTAs, so the last wave takes 1 / Q of a tile's time.  Sub-tiles own disjoint
+// outputs: nothing is combined across CTAs.
 // For the gate/up FFN the 256 B-rows of a tile are 128 gate rows followed by
 // the same 128 up rows, so one N=256 MMA yields both halves of h's tile.
 #pragma once
@@ -69,17 +69,14 @@ struct PrefillArgs {
     int y_bf16;           // store y as bf16 (nearest even of the fp32 value)
     int vec_ok;           // rows of y are 16-byte multiples: TMA stores
     int full_units;       // whole tiles (units [0, full_units))
-    int split;            // K parts of each remaining tile (1: no split)
-    int num_units;        // full_units + (num_tiles - full_units) * split
-    int32_t *part;        // [tail tiles][split][PF_BM][PF_BN] int32 partial sums (split > 1)
-    unsigned *part_cnt;   // [tail tiles][4] arrivals per 32-row slice, zero before the kernel
+    int tail_q;           // sub-tiles per remaining tile (1: none; 2 or 4, BitLinear only)
+    int num_units;        // full_units + (num_tiles - full_units) * tail_q
 };
 
-// Unit u of the persistent loop: a tile (mb, nb) and a range of k-stages.
+// Unit u of the persistent loop: tile (mb, nb), output columns [col0, col0 + ncols)
+// of its PF_BN (B rows of the tile).
 struct PfUnit {
-    int mb, nb, kb0, kb1;
-    int part; // -1: whole tile
-    int slot; // tail tile index (split parts)
+    int mb, nb, col0, ncols;
 };
 
 BITNET_DEVINL PfUnit pf_unit(const PrefillArgs &a, int u)
@@ -88,21 +85,24 @@ BITNET_DEVINL PfUnit pf_unit(const PrefillArgs &a, int u)
     int tile;
     if (u < a.full_units) {
         tile = u;
-        r.kb0 = 0;
-        r.kb1 = a.num_k;
-        r.part = -1;
-        r.slot = 0;
+        r.col0 = 0;
+        r.ncols = PF_BN;
     } else {
         const int v = u - a.full_units;
-        r.slot = v / a.split;
-        r.part = v - r.slot * a.split;
-        tile = a.full_units + r.slot;
-        r.kb0 = r.part * a.num_k / a.split;
-        r.kb1 = (r.part + 1) * a.num_k / a.split;
+        const int q = v % a.tail_q;
+        tile = a.full_units + v / a.tail_q;
+        r.ncols = PF_BN / a.tail_q;
+        r.col0 = q * r.ncols;
     }
     r.mb = tile % a.num_m;
     r.nb = tile / a.num_m;
     return r;
+}
+
+// kind::i8 instruction descriptor with N = ncols (a multiple of 16, <= 256).
+BITNET_DEVINL uint32_t pf_idesc(int ncols)
+{
+    return (PF_IDESC & ~(0x3Fu << 17)) | ((uint32_t)(ncols >> 3) << 17);
 }
 
 // codes {0,1,2} (one per byte) -> int8 {-1,0,1}: per byte (c | 0x80) - 1 cannot
@@ -112,14 +112,15 @@ BITNET_DEVINL uint32_t codes_to_s8(uint32_t c)
     return ((c | 0x80808080u) - 0x01010101u) ^ 0x80808080u;
 }
 
-// 256 threads turn one packed stage (256 rows x 32 B) into 256 rows x 128 B of
+// 256 threads turn one packed stage (rows x 32 B, rows <= 256) into rows x 128 B of
 // int8, 16-byte chunk c of row r stored at r*128 + ((c ^ (r & 7)) << 4).
-BITNET_DEVINL void pf_unpack_stage(const unsigned char *bp, unsigned char *bu, int u)
+BITNET_DEVINL void pf_unpack_stage(const unsigned char *bp, unsigned char *bu, int u, int rows)
 {
     constexpr uint32_t M3 = 0x03030303u;
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
         const int t = u + PF_UNPACK_THREADS * i;
+        if (t >= 2 * rows) break;
         const int row = t >> 1, half = t & 1;
         const uint4 p = *reinterpret_cast<const uint4 *>(bp + row * 32 + half * 16);
         const uint32_t wv[4] = {p.x, p.y, p.z, p.w};
@@ -229,20 +230,23 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             for (int unit = blockIdx.x; unit < a.num_units && ok; unit += gridDim.x) {
                 const PfUnit un = pf_unit(a, unit);
                 const int mb = un.mb, nb = un.nb;
-                for (int kb = un.kb0; kb < un.kb1; ++kb) {
+                for (int kb = 0; kb < a.num_k; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1)) {
                         ok = false;
                         break;
                     }
                     unsigned char *st = stages + stage * PF_STAGE_BYTES;
-                    mbar_arrive_expect_tx(&full[stage], PF_A_BYTES + PF_BP_BYTES);
+                    mbar_arrive_expect_tx(&full[stage], PF_A_BYTES + un.ncols * (PF_BK / 4));
                     tma_load_2d(st, &tmA, kb * PF_BK, mb * PF_BM, &full[stage]);
                     unsigned char *bp = st + PF_A_BYTES + PF_BU_BYTES;
                     if constexpr (FFN) {
                         tma_load_2d(bp, &tmB0, kb * (PF_BK / 4), nb * (PF_BN / 2), &full[stage]);
                         tma_load_2d(bp + PF_BP_BYTES / 2, &tmB1, kb * (PF_BK / 4), nb * (PF_BN / 2), &full[stage]);
-                    } else {
+                    } else if (un.ncols == PF_BN) {
                         tma_load_2d(bp, &tmB0, kb * (PF_BK / 4), nb * PF_BN, &full[stage]);
+                    } else {
+                        // a sub-tile: tmB1's box is ncols rows
+                        tma_load_2d(bp, &tmB1, kb * (PF_BK / 4), nb * PF_BN + un.col0, &full[stage]);
                     }
                     issued |= 1u << stage;
                     last_par = (last_par & ~(1u << stage)) | (phase << stage);
@@ -269,7 +273,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * PF_BN);
-                for (int kb = un.kb0; kb < un.kb1; ++kb) {
+                const uint32_t idesc = pf_idesc(un.ncols);
+                for (int kb = 0; kb < a.num_k; ++kb) {
                     if (!mbar_wait(&full[stage], phase) || !mbar_wait(&unpacked[stage], phase)) {
                         ok = false;
                         break;
@@ -280,7 +285,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                     const uint64_t bdesc = umma_desc_k_sw128(st + PF_A_BYTES);
 #pragma unroll
                     for (int j = 0; j < PF_BK / 32; ++j)
-                        umma_i8(d_tmem, adesc + 2 * j, bdesc + 2 * j, PF_IDESC, (kb != un.kb0 || j != 0) ? 1u : 0u);
+                        umma_i8(d_tmem, adesc + 2 * j, bdesc + 2 * j, idesc, (kb | j) != 0);
                     umma_commit(&empty[stage]);
                     if (++stage == PF_STAGES) {
                         stage = 0;
@@ -307,13 +312,13 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         bool ok = true;
         for (int unit = blockIdx.x; unit < a.num_units && ok; unit += gridDim.x) {
             const PfUnit un = pf_unit(a, unit);
-            for (int kb = un.kb0; kb < un.kb1; ++kb) {
+            for (int kb = 0; kb < a.num_k; ++kb) {
                 if (!mbar_wait(&full[stage], phase)) {
                     ok = false;
                     break;
                 }
                 unsigned char *st = stages + stage * PF_STAGE_BYTES;
-                pf_unpack_stage(st + PF_A_BYTES + PF_BU_BYTES, st + PF_A_BYTES, u);
+                pf_unpack_stage(st + PF_A_BYTES + PF_BU_BYTES, st + PF_A_BYTES, u, un.ncols);
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&unpacked[stage]);
@@ -412,22 +417,6 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 emit(o, m, n, mok);
             }
         };
-        // sum of the split parts of columns [col, col + 32) of this lane's row
-        auto part_sum = [&](const int32_t *row0, int col, uint32_t (&v)[32]) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = 0u;
-            for (int q = 0; q < a.split; ++q) {
-                const int32_t *src = row0 + (size_t)q * PF_BM * PF_BN + col;
-#pragma unroll
-                for (int j = 0; j < 32; j += 4) {
-                    const uint4 w = ld_cg_v4(src + j);
-                    v[j] += w.x;
-                    v[j + 1] += w.y;
-                    v[j + 2] += w.z;
-                    v[j + 3] += w.w;
-                }
-            }
-        };
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int unit = blockIdx.x; unit < a.num_units; unit += gridDim.x) {
@@ -440,78 +429,28 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             const float r0 = __fdiv_rn(g0, sm);
             const float r1 = FFN ? __fdiv_rn(g1, sm) : 0.0f;
             const uint32_t tb = tmem_base + ((uint32_t)(warp * 32) << 16) + (uint32_t)(acc * PF_BN);
-            if (un.part < 0) {
-                if constexpr (!FFN) {
+            if constexpr (!FFN) {
 #pragma unroll 1
-                    for (int c = 0; c < PF_BN / 32; ++c) {
-                        uint32_t v[32];
-                        tmem_ld32(tb + 32 * c, v);
-                        tmem_wait_ld(v);
-                        fin_lin(v, c, un.nb, m, mok, r0);
-                    }
-                } else {
-#pragma unroll 1
-                    for (int c = 0; c < PF_BN / 64; ++c) {
-                        uint32_t vg[32], vu[32];
-                        tmem_ld32(tb + 32 * c, vg);
-                        tmem_ld32(tb + PF_BN / 2 + 32 * c, vu);
-                        tmem_wait_ld(vg);
-                        tmem_regs_fence(vu);
-                        fin_ffn(vg, vu, c, un.nb, m, mok, r0, r1);
-                    }
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&acc_empty[acc]);
-            } else {
-                // a part of a split tile: raw sums of this row to the workspace, then the
-                // accumulator is free for the next unit
-                int32_t *prow = a.part + ((size_t)(un.slot * a.split + un.part) * PF_BM + warp * 32 + lane) * PF_BN;
-#pragma unroll 1
-                for (int c = 0; c < PF_BN / 32; ++c) {
+                for (int c = 0; c < un.ncols / 32; ++c) {
                     uint32_t v[32];
                     tmem_ld32(tb + 32 * c, v);
                     tmem_wait_ld(v);
-#pragma unroll
-                    for (int j = 0; j < 32; j += 4)
-                        *reinterpret_cast<uint4 *>(prow + 32 * c + j) = make_uint4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+                    fin_lin(v, un.col0 / 32 + c, un.nb, m, mok, r0);
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&acc_empty[acc]);
-                // every lane's partial stores precede lane 0's fence and arrival count
-                unsigned prev = 0u;
-                if (lane == 0) {
-                    __threadfence();
-                    prev = atomicAdd(&a.part_cnt[un.slot * 4 + warp], 1u);
-                }
-                prev = __shfl_sync(0xffffffffu, prev, 0);
-                if (prev == (unsigned)(a.split - 1)) {
-                    // the last part of this 32-row slice: every other part's sums are visible
-                    if (lane == 0) {
-                        __threadfence();
-                        a.part_cnt[un.slot * 4 + warp] = 0u;
-                    }
-                    __syncwarp();
-                    const int32_t *row0 = a.part + ((size_t)un.slot * a.split * PF_BM + warp * 32 + lane) * PF_BN;
-                    if constexpr (!FFN) {
+            } else {
 #pragma unroll 1
-                        for (int c = 0; c < PF_BN / 32; ++c) {
-                            uint32_t v[32];
-                            part_sum(row0, 32 * c, v);
-                            fin_lin(v, c, un.nb, m, mok, r0);
-                        }
-                    } else {
-#pragma unroll 1
-                        for (int c = 0; c < PF_BN / 64; ++c) {
-                            uint32_t vg[32], vu[32];
-                            part_sum(row0, 32 * c, vg);
-                            part_sum(row0, PF_BN / 2 + 32 * c, vu);
-                            fin_ffn(vg, vu, c, un.nb, m, mok, r0, r1);
-                        }
-                    }
+                for (int c = 0; c < PF_BN / 64; ++c) {
+                    uint32_t vg[32], vu[32];
+                    tmem_ld32(tb + 32 * c, vg);
+                    tmem_ld32(tb + PF_BN / 2 + 32 * c, vu);
+                    tmem_wait_ld(vg);
+                    tmem_regs_fence(vu);
+                    fin_ffn(vg, vu, c, un.nb, m, mok, r0, r1);
                 }
             }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[acc]);
             if (a.y_amax) {
                 if (mok && rmax != 0u) atomicMax(reinterpret_cast<unsigned *>(a.y_amax) + m, rmax);
                 rmax = 0;

@@ -140,8 +140,7 @@ def test_linear_prefill_ragged(m, k, n, kind, dtype):
 @pytest.mark.parametrize("k,n", [(2560, 6912), (6912, 2560), (2560, 3840), (2560, 640), (2560, 2560)])
 def test_linear_prefill_full_size_sampled(k, n):
     """M = 4096 prefill at the 2B4T shapes; every output of 48 sampled rows.  N = 2560 and 3840
-    leave a partly filled last wave of tiles, which runs split along K (partial sums combined
-    in the workspace)."""
+    leave a partly filled last wave of tiles, which runs as sub-tiles of 64 output columns."""
     m = 4096
     W = make_weights(n, k, 700 + k)
     xd, xf = make_x(m, k, 800 + k, "student_t_rows", "bf16")
@@ -209,7 +208,7 @@ def test_ffn_prefill(m, k, n):
     U = make_weights(n, k, 1150 + n)
     xd, xf = make_x(m, k, 1200 + m, "student_t_rows")
     h, ag, au = run_ffn(xd, G, U, tw.BITNET_DISPATCH_AUTO if m > 64 else tw.BITNET_DISPATCH_PREFILL, m, n)
-    rows = sample_rows(m, 40, 11) if m > 512 else np.arange(m)  # (n = 2560: split tail tiles)
+    rows = sample_rows(m, 40, 11) if m > 512 else np.arange(m)
     h_ref, ag_ref, au_ref, _, _ = oracle.ffn_gate_up(xf[rows], G["p_ref"], G["g_ref"], U["p_ref"], U["g_ref"], k)
     assert np.array_equal(ag[rows].astype(np.int64), ag_ref)
     assert np.array_equal(au[rows].astype(np.int64), au_ref)
