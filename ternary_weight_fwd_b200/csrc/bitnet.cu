@@ -790,9 +790,12 @@ bitnet_status_t seq_schedule(const bitnet_op_t *ops, int n, int64_t M, int32_t *
 }
 
 inline int seq_mp(int64_t M) { return M <= 8 ? 8 : M <= 16 ? 16 : M <= 32 ? 32 : 64; }
-inline int seq_rtasks(const bitnet_op_t &o)
+// Row groups per compute warp: two at one token tile (each activation fragment feeds two
+// weight fragments, halving the activation loads from shared memory), else one.
+inline int seq_rg(int64_t M) { return M <= 8 ? 2 : 1; }
+inline int seq_rtasks(const bitnet_op_t &o, int64_t M)
 {
-    const int64_t rows_per_task = o.kind == BITNET_OP_FFN_GATE_UP ? DT_ROWS / 2 : DT_ROWS;
+    const int64_t rows_per_task = (o.kind == BITNET_OP_FFN_GATE_UP ? DT_ROWS / 2 : DT_ROWS) * seq_rg(M);
     return (int)cdiv(o.N, rows_per_task);
 }
 
@@ -857,8 +860,8 @@ std::vector<int> seq_group_order(const bitnet_op_t *ops, int n, int64_t M, const
     for (int j = 0; j < n; ++j) {
         count[2 * j] = (int)M;
         dur[2 * j] = 1.0;
-        count[2 * j + 1] = seq_rtasks(ops[j]);
-        dur[2 * j + 1] = (double)DT_ROWS * (double)(ops[j].K / 4) / 40e3;
+        count[2 * j + 1] = seq_rtasks(ops[j], M);
+        dur[2 * j + 1] = (double)(DT_ROWS * seq_rg(M)) * (double)(ops[j].K / 4) / 40e3;
     }
     std::vector<std::vector<int>> succ(ng);
     for (int v = 0; v < ng; ++v) {
@@ -938,7 +941,7 @@ bitnet_status_t seq_build(DtProgram &p, const bitnet_op_t *ops, const int32_t *u
         d.N = (int)o.N;
         d.nmat = o.kind == BITNET_OP_FFN_GATE_UP ? 2 : 1;
         d.xf32 = o.x_dtype == BITNET_DTYPE_F32;
-        d.rtasks = seq_rtasks(o);
+        d.rtasks = seq_rtasks(o, M);
         d.stall = (stall >= 0 && user_index && user_index[j] == stall) ? 1 : 0;
         if (base) {
             d.xq = reinterpret_cast<int8_t *>(base + off);
@@ -975,7 +978,7 @@ bitnet_status_t seq_build(DtProgram &p, const bitnet_op_t *ops, const int32_t *u
     }
     p.n_segs = ns;
     p.n_tasks = t;
-    p.slot_bytes = DT_WBYTES + DT_KC * Mp;
+    p.slot_bytes = seq_rg(M) * DT_WBYTES + DT_KC * Mp;
     p.n_slots = (int)std::min<size_t>(DT_MAX_SLOTS, (kSmemLimit - 128 - DT_HDR) / (size_t)p.slot_bytes);
     if (order_out) *order_out = order;
     return BITNET_OK;
@@ -985,25 +988,25 @@ static_assert(sizeof(DtProgram) <= 32000, "kernel parameter space");
 static_assert(DT_MAX_OPS >= BITNET_SEQ_MAX_OPS && 2 * DT_MAX_OPS <= DT_MAX_SEGS, "sequence limits");
 static_assert(DT_MAX_M >= BITNET_SEQ_MAX_M, "sequence token limit");
 
-template <int TT>
+template <int TT, int RG>
 cudaError_t seq_launch_t(const DtProgram &p, int ctas, cudaStream_t stream, int dev)
 {
     static std::atomic<int> smem_done[kMaxDevices];
-    cudaError_t e = ensure_smem(k_decode_tasks<TT>, kSmemLimit, smem_done, dev);
+    cudaError_t e = ensure_smem(k_decode_tasks<TT, RG>, kSmemLimit, smem_done, dev);
     if (e != cudaSuccess) return e;
     const size_t smem = 128 + DT_HDR + (size_t)p.n_slots * p.slot_bytes;
     g_launches.fetch_add(1, std::memory_order_relaxed);
-    k_decode_tasks<TT><<<ctas, DT_THREADS, smem, stream>>>(p);
+    k_decode_tasks<TT, RG><<<ctas, DT_THREADS, smem, stream>>>(p);
     return cudaGetLastError();
 }
 
 cudaError_t seq_launch(const DtProgram &p, int ctas, cudaStream_t stream, int dev)
 {
-    switch (p.Mp) {
-    case 8: return seq_launch_t<1>(p, ctas, stream, dev);
-    case 16: return seq_launch_t<2>(p, ctas, stream, dev);
-    case 32: return seq_launch_t<4>(p, ctas, stream, dev);
-    default: return seq_launch_t<8>(p, ctas, stream, dev);
+    switch (p.Mp) { // row groups per warp as seq_rg
+    case 8: return seq_launch_t<1, 2>(p, ctas, stream, dev);
+    case 16: return seq_launch_t<2, 1>(p, ctas, stream, dev);
+    case 32: return seq_launch_t<4, 1>(p, ctas, stream, dev);
+    default: return seq_launch_t<8, 1>(p, ctas, stream, dev);
     }
 }
 

@@ -57,11 +57,11 @@ namespace bitnet {
 
 constexpr int DT_COMPUTE = 256;                 // compute threads (warps 0-7)
 constexpr int DT_THREADS = 352;                 // + weight producer (8), activation producer (9), completion (10)
-constexpr int DT_ROWS = 128;                    // packed rows per row task
+constexpr int DT_ROWS = 128;                    // packed rows per row task and 16-row group per warp
 constexpr int DT_KC = 512;                      // k per piece
 constexpr int DT_KB = DT_KC / 64;               // 64-k blocks per piece
 constexpr int DT_PITCH = DT_KC / 4 + 16;        // 144 = 16 * 9: conflict-free fragment loads
-constexpr int DT_WBYTES = DT_ROWS * DT_PITCH;   // 18432 weight bytes of a piece in shared memory
+constexpr int DT_WBYTES = DT_ROWS * DT_PITCH;   // 18432 weight bytes of a piece in shared memory, per row-group set
 constexpr int DT_QUEUE = 4;                     // tasks claimed ahead of the compute warps (at most)
 constexpr int DT_MAX_OPS = 128;
 constexpr int DT_MAX_SEGS = 512;
@@ -227,12 +227,26 @@ BITNET_DEVINL int dt_ld_cg_s32(const int32_t *p)
 
 BITNET_DEVINL int dt_pieces(int K) { return (K + DT_KC - 1) / DT_KC; }
 
+// Position in the piece ring: slot and the parity of its current use.
+struct DtRing {
+    int slot = 0;
+    uint32_t par = 0;
+    BITNET_DEVINL void next(int n_slots)
+    {
+        if (++slot == n_slots) {
+            slot = 0;
+            par ^= 1u;
+        }
+    }
+};
+
 // ---- weight producer (warp 8) ----------------------------------------------
 // Lane l copies 16-byte chunk j = l % 8 (a 64-k block of the piece) of shared
 // rows r = l / 8 + 4 i, i = 0 .. 31.  Shared row r of a BitLinear task is packed
 // row 128 b + r; of a gated-FFN task (rows 8 .. 15 of each 16-row group are the
 // up rows) it is row 64 b + 8 (r / 16) + r % 8 of the gate or the up matrix.
 // For i = 4 g + q the source row is rb[q] + g * rstep: four base rows per task.
+template <int RG>
 BITNET_DEVINL void dt_weight_producer(const DtProgram &p, unsigned char *smem)
 {
     const int lane = threadIdx.x & 31;
@@ -244,7 +258,8 @@ BITNET_DEVINL void dt_weight_producer(const DtProgram &p, unsigned char *smem)
     const uint32_t ring = smem_u32(smem + DT_HDR);
     const int j16 = lane & 7;
     const int r0 = lane >> 3;
-    uint32_t seq = 0, piece = 0;
+    uint32_t seq = 0;
+    DtRing ring_pos;
     for (;;) {
         int t = 0;
         if (lane == 0) t = (int)atomicAdd(&p.counters[DT_CNT_TASK], 1u);
@@ -271,20 +286,20 @@ BITNET_DEVINL void dt_weight_producer(const DtProgram &p, unsigned char *smem)
         for (int q = 0; q < 4; ++q) {
             const uint8_t *w;
             if (ffn) {
-                rb[q] = tk.idx * (DT_ROWS / 2) + r0 + 4 * (q & 1);
+                rb[q] = tk.idx * (RG * DT_ROWS / 2) + r0 + 4 * (q & 1);
                 w = q >= 2 ? op.w1 : op.w0;
             } else {
-                rb[q] = tk.idx * DT_ROWS + r0 + 4 * q;
+                rb[q] = tk.idx * (RG * DT_ROWS) + r0 + 4 * q;
                 w = op.w0;
             }
             pb[q] = w + (size_t)rb[q] * rowb + (size_t)j16 * 16;
         }
         const size_t gstep = (size_t)rstep * rowb; // bytes between rows rb[q] + g * rstep, consecutive g
-        const bool all_rows = (ffn ? (tk.idx + 1) * (DT_ROWS / 2) : (tk.idx + 1) * DT_ROWS) <= N;
+        const bool all_rows = (ffn ? (tk.idx + 1) * (RG * DT_ROWS / 2) : (tk.idx + 1) * (RG * DT_ROWS)) <= N;
         const int np = dt_pieces(K);
-        for (int pc = 0; pc < np; ++pc) {
-            const int s = (int)(piece % (uint32_t)p.n_slots);
-            mbar_wait(&empty[s], ((piece / (uint32_t)p.n_slots) & 1u) ^ 1u);
+        for (int pc = 0; pc < np; ++pc, ring_pos.next(p.n_slots)) {
+            const int s = ring_pos.slot;
+            mbar_wait(&empty[s], ring_pos.par ^ 1u);
             const int nkb = min(DT_KB, (K - pc * DT_KC) / 64);
             const uint32_t dst0 = ring + (uint32_t)s * (uint32_t)p.slot_bytes + (uint32_t)(r0 * DT_PITCH + j16 * 16);
             const size_t koff = (size_t)pc * (DT_KC / 4);
@@ -294,7 +309,7 @@ BITNET_DEVINL void dt_weight_producer(const DtProgram &p, unsigned char *smem)
                     for (int q = 0; q < 4; ++q) {
                         const uint8_t *src = pb[q] + koff;
 #pragma unroll
-                        for (int g = 0; g < 8; ++g)
+                        for (int g = 0; g < 8 * RG; ++g)
                             asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
                                              dst0 + (uint32_t)((16 * g + 4 * q) * DT_PITCH)),
                                          "l"(src + g * gstep)
@@ -302,7 +317,7 @@ BITNET_DEVINL void dt_weight_producer(const DtProgram &p, unsigned char *smem)
                     }
                 } else {
 #pragma unroll
-                    for (int g = 0; g < 8; ++g) {
+                    for (int g = 0; g < 8 * RG; ++g) {
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
                             const bool ok = rb[q] + g * rstep < N;
@@ -313,13 +328,13 @@ BITNET_DEVINL void dt_weight_producer(const DtProgram &p, unsigned char *smem)
                 }
             }
             dt_cp_arrive(smem_u32(&full[s]));
-            ++piece;
         }
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
 // ---- activation producer (warp 9) -------------------------------------------
+template <int RG>
 BITNET_DEVINL void dt_act_producer(const DtProgram &p, unsigned char *smem)
 {
     const int lane = threadIdx.x & 31;
@@ -331,7 +346,8 @@ BITNET_DEVINL void dt_act_producer(const DtProgram &p, unsigned char *smem)
     const volatile int *qtask = reinterpret_cast<const volatile int *>(smem + DT_QTASK);
     const uint32_t ring = smem_u32(smem + DT_HDR);
     const int Mp = p.Mp;
-    uint32_t seq = 0, piece = 0;
+    uint32_t seq = 0;
+    DtRing ring_pos;
     for (;;) {
         const int e = (int)(seq % DT_QUEUE);
         mbar_wait(&qfull[e], (seq / DT_QUEUE) & 1u);
@@ -367,16 +383,15 @@ BITNET_DEVINL void dt_act_producer(const DtProgram &p, unsigned char *smem)
             dt_cp_arrive(smem_u32(&qinfo[e]));
             // the x_q chunk of every piece: [8 k-blocks][Mp][64] bytes, contiguous in the workspace
             const int np = dt_pieces(op.K);
-            for (int pc = 0; pc < np; ++pc) {
-                const int s = (int)(piece % (uint32_t)p.n_slots);
-                mbar_wait(&empty[s], ((piece / (uint32_t)p.n_slots) & 1u) ^ 1u);
+            for (int pc = 0; pc < np; ++pc, ring_pos.next(p.n_slots)) {
+                const int s = ring_pos.slot;
+                mbar_wait(&empty[s], ring_pos.par ^ 1u);
                 const int nkb = min(DT_KB, (op.K - pc * DT_KC) / 64);
                 const int chunks = nkb * Mp * 4; // 16-byte chunks
                 const uint8_t *src = reinterpret_cast<const uint8_t *>(op.xq) + (size_t)pc * DT_KB * Mp * 64;
-                const uint32_t dst = ring + (uint32_t)s * (uint32_t)p.slot_bytes + DT_WBYTES;
+                const uint32_t dst = ring + (uint32_t)s * (uint32_t)p.slot_bytes + RG * DT_WBYTES;
                 for (int c = lane; c < chunks; c += 32) dt_cp16(dst + 16u * c, src + 16 * c, true);
                 dt_cp_arrive(smem_u32(&full[s]));
-                ++piece;
             }
         } else {
             mbar_arrive(&qinfo[e]); // keeps the entry's phases in step (every lane: the count is 32)
@@ -528,77 +543,85 @@ BITNET_DEVINL void dt_quant_row(const DtProgram &p, const DtOp &op, int m, unsig
 }
 
 // ---- row task contraction over one piece (compute warp w) ------------------
-// acc[a][tt][4]: accumulator set a (k-blocks alternate between sets so that
-// consecutive mma are independent), token tile tt.
-template <int TT, int NACC>
-BITNET_DEVINL void dt_piece(int (&acc)[NACC][TT][4], uint32_t wrow, uint32_t xrow, int Mp, int nkb)
+// acc[r][a][tt][4]: row group r of the warp (rows 16 (w + 8 r) ..), accumulator
+// set a (the two mma of a k-block go to different sets so that consecutive mma
+// are independent), token tile tt.  wrow: this lane's word in row group 0; row
+// group r is r * 128 rows further.
+template <int TT, int NACC, int RG>
+BITNET_DEVINL void dt_kblock(int (&acc)[RG][NACC][TT][4], const uint32_t (&lo)[RG], const uint32_t (&hi)[RG],
+                             const uint4 *bpre, uint32_t xrow, int Mp, int kb)
 {
     constexpr uint32_t M3 = 0x03030303u;
 #pragma unroll
-    for (int kb = 0; kb < DT_KB; ++kb) {
-        if (kb < nkb) {
-            uint32_t lo, hi;
-            asm volatile("ld.shared.u32 %0, [%1];" : "=r"(lo) : "r"(wrow + kb * 16));
-            asm volatile("ld.shared.u32 %0, [%1];" : "=r"(hi) : "r"(wrow + 8 * DT_PITCH + kb * 16));
-            const uint32_t a0 = lo & M3, a1 = hi & M3, a2 = (lo >> 2) & M3, a3 = (hi >> 2) & M3;
-            const uint32_t a4 = (lo >> 4) & M3, a5 = (hi >> 4) & M3, a6 = (lo >> 6) & M3, a7 = (hi >> 6) & M3;
+    for (int tt = 0; tt < TT; ++tt) {
+        uint4 b;
+        if (bpre) {
+            b = bpre[tt];
+        } else {
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w)
+                         : "r"(xrow + (uint32_t)((kb * Mp + tt * 8) * 64)));
+        }
 #pragma unroll
-            for (int tt = 0; tt < TT; ++tt) {
-                uint4 b;
-                asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                             : "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w)
-                             : "r"(xrow + (uint32_t)((kb * Mp + tt * 8) * 64)));
-                mma_u8s8_16832(acc[kb % NACC][tt], a0, a1, a2, a3, b.x, b.y);
-                mma_u8s8_16832(acc[kb % NACC][tt], a4, a5, a6, a7, b.z, b.w);
-            }
+        for (int r = 0; r < RG; ++r) {
+            const uint32_t l = lo[r], h = hi[r];
+            mma_u8s8_16832(acc[r][(2 * kb) % NACC][tt], l & M3, h & M3, (l >> 2) & M3, (h >> 2) & M3, b.x, b.y);
+            mma_u8s8_16832(acc[r][(2 * kb + 1) % NACC][tt], (l >> 4) & M3, (h >> 4) & M3, (l >> 6) & M3,
+                           (h >> 6) & M3, b.z, b.w);
         }
     }
 }
 
-// A full piece (8 k-blocks): every fragment is loaded before the first mma, so
-// the shared-memory latency is paid once per piece; the two mma of a k-block
-// go to different accumulator sets.
-template <int TT, int NACC>
-BITNET_DEVINL void dt_piece_full(int (&acc)[NACC][TT][4], uint32_t wrow, uint32_t xrow, int Mp)
+// A ragged piece (fewer than 8 k-blocks).
+template <int TT, int NACC, int RG>
+BITNET_DEVINL void dt_piece(int (&acc)[RG][NACC][TT][4], uint32_t wrow, uint32_t xrow, int Mp, int nkb)
 {
-    constexpr uint32_t M3 = 0x03030303u;
-    uint32_t lo[DT_KB], hi[DT_KB];
 #pragma unroll
     for (int kb = 0; kb < DT_KB; ++kb) {
-        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(lo[kb]) : "r"(wrow + kb * 16));
-        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(hi[kb]) : "r"(wrow + 8 * DT_PITCH + kb * 16));
+        if (kb < nkb) {
+            uint32_t lo[RG], hi[RG];
+#pragma unroll
+            for (int r = 0; r < RG; ++r) {
+                const uint32_t a = wrow + (uint32_t)(r * DT_ROWS * DT_PITCH) + kb * 16;
+                asm volatile("ld.shared.u32 %0, [%1];" : "=r"(lo[r]) : "r"(a));
+                asm volatile("ld.shared.u32 %0, [%1];" : "=r"(hi[r]) : "r"(a + 8 * DT_PITCH));
+            }
+            dt_kblock<TT, NACC, RG>(acc, lo, hi, nullptr, xrow, Mp, kb);
+        }
     }
-    constexpr int BPRE = TT == 1 ? DT_KB : 1; // activation fragments held ahead (all of them for one tile)
-    uint4 bq[BPRE];
+}
+
+// A full piece (8 k-blocks): every weight fragment (and, for one token tile,
+// every activation fragment) is loaded before the first mma, so the
+// shared-memory latency is paid once per piece.
+template <int TT, int NACC, int RG>
+BITNET_DEVINL void dt_piece_full(int (&acc)[RG][NACC][TT][4], uint32_t wrow, uint32_t xrow, int Mp)
+{
+    uint32_t lo[DT_KB][RG], hi[DT_KB][RG];
+#pragma unroll
+    for (int kb = 0; kb < DT_KB; ++kb)
+#pragma unroll
+        for (int r = 0; r < RG; ++r) {
+            const uint32_t a = wrow + (uint32_t)(r * DT_ROWS * DT_PITCH) + kb * 16;
+            asm volatile("ld.shared.u32 %0, [%1];" : "=r"(lo[kb][r]) : "r"(a));
+            asm volatile("ld.shared.u32 %0, [%1];" : "=r"(hi[kb][r]) : "r"(a + 8 * DT_PITCH));
+        }
     if constexpr (TT == 1) {
+        uint4 bq[DT_KB];
 #pragma unroll
         for (int kb = 0; kb < DT_KB; ++kb)
             asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
                          : "=r"(bq[kb].x), "=r"(bq[kb].y), "=r"(bq[kb].z), "=r"(bq[kb].w)
                          : "r"(xrow + (uint32_t)(kb * Mp * 64)));
-    }
 #pragma unroll
-    for (int kb = 0; kb < DT_KB; ++kb) {
-        const uint32_t l = lo[kb], h = hi[kb];
-        const uint32_t a0 = l & M3, a1 = h & M3, a2 = (l >> 2) & M3, a3 = (h >> 2) & M3;
-        const uint32_t a4 = (l >> 4) & M3, a5 = (h >> 4) & M3, a6 = (l >> 6) & M3, a7 = (h >> 6) & M3;
+        for (int kb = 0; kb < DT_KB; ++kb) dt_kblock<TT, NACC, RG>(acc, lo[kb], hi[kb], &bq[kb], xrow, Mp, kb);
+    } else {
 #pragma unroll
-        for (int tt = 0; tt < TT; ++tt) {
-            uint4 b;
-            if constexpr (TT == 1) {
-                b = bq[kb];
-            } else {
-                asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                             : "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w)
-                             : "r"(xrow + (uint32_t)((kb * Mp + tt * 8) * 64)));
-            }
-            mma_u8s8_16832(acc[(2 * kb) % NACC][tt], a0, a1, a2, a3, b.x, b.y);
-            mma_u8s8_16832(acc[(2 * kb + 1) % NACC][tt], a4, a5, a6, a7, b.z, b.w);
-        }
+        for (int kb = 0; kb < DT_KB; ++kb) dt_kblock<TT, NACC, RG>(acc, lo[kb], hi[kb], nullptr, xrow, Mp, kb);
     }
 }
 
-template <int TT>
+template <int TT, int RG>
 BITNET_DEVINL void dt_compute(const DtProgram &p, unsigned char *smem)
 {
     constexpr int NACC = TT <= 2 ? 4 : 2;
@@ -613,7 +636,8 @@ BITNET_DEVINL void dt_compute(const DtProgram &p, unsigned char *smem)
     const volatile int *qtask = reinterpret_cast<const volatile int *>(smem + DT_QTASK);
     const uint32_t ring = smem_u32(smem + DT_HDR);
     const int Mp = p.Mp, M = p.M;
-    uint32_t seq = 0, piece = 0;
+    uint32_t seq = 0;
+    DtRing ring_pos;
     for (;;) {
         const int e = (int)(seq % DT_QUEUE);
         mbar_wait(&qfull[e], (seq / DT_QUEUE) & 1u);
@@ -633,35 +657,39 @@ BITNET_DEVINL void dt_compute(const DtProgram &p, unsigned char *smem)
             __syncwarp();
             if (lane == 0) mbar_arrive(&cdone[e]);
         } else {
-            int acc[NACC][TT][4];
+            int acc[RG][NACC][TT][4];
 #pragma unroll
-            for (int a = 0; a < NACC; ++a)
+            for (int r = 0; r < RG; ++r)
 #pragma unroll
-                for (int tt = 0; tt < TT; ++tt)
+                for (int a = 0; a < NACC; ++a)
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) acc[a][tt][c] = 0;
-            const int np = dt_pieces(op.K);
-            for (int pc = 0; pc < np; ++pc) {
-                const int s = (int)(piece % (uint32_t)p.n_slots);
-                mbar_wait(&full[s], (piece / (uint32_t)p.n_slots) & 1u);
+                    for (int tt = 0; tt < TT; ++tt)
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) acc[r][a][tt][c] = 0;
+            const int K = op.K;
+            const int np = dt_pieces(K);
+            const uint32_t wlane = (uint32_t)((warp * 16 + g) * DT_PITCH + t4 * 4);
+            const uint32_t xlane = (uint32_t)(RG * DT_WBYTES + g * 64 + t4 * 16);
+            for (int pc = 0; pc < np; ++pc, ring_pos.next(p.n_slots)) {
+                const int s = ring_pos.slot;
+                mbar_wait(&full[s], ring_pos.par);
                 const uint32_t base = ring + (uint32_t)s * (uint32_t)p.slot_bytes;
-                const uint32_t wrow = base + (uint32_t)((warp * 16 + g) * DT_PITCH + t4 * 4);
-                const uint32_t xrow = base + DT_WBYTES + (uint32_t)(g * 64 + t4 * 16);
-                const int nkb = min(DT_KB, (op.K - pc * DT_KC) / 64);
+                const int nkb = min(DT_KB, (K - pc * DT_KC) >> 6);
                 if (nkb == DT_KB)
-                    dt_piece_full<TT, NACC>(acc, wrow, xrow, Mp);
+                    dt_piece_full<TT, NACC, RG>(acc, base + wlane, base + xlane, Mp);
                 else
-                    dt_piece<TT, NACC>(acc, wrow, xrow, Mp, nkb);
+                    dt_piece<TT, NACC, RG>(acc, base + wlane, base + xlane, Mp, nkb);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&empty[s]);
-                ++piece;
             }
 #pragma unroll
-            for (int a = 1; a < NACC; ++a)
+            for (int r = 0; r < RG; ++r)
 #pragma unroll
-                for (int tt = 0; tt < TT; ++tt)
+                for (int a = 1; a < NACC; ++a)
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) acc[0][tt][c] += acc[a][tt][c];
+                    for (int tt = 0; tt < TT; ++tt)
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) acc[r][0][tt][c] += acc[r][a][tt][c];
             // epilogue: y = fl((float)(sum c*x - sum x) * fl(gamma / s))
             mbar_wait(&qinfo[e], (seq / DT_QUEUE) & 1u);
             const unsigned char *inf = smem + DT_INFO + e * DT_INFO_BYTES;
@@ -672,23 +700,6 @@ BITNET_DEVINL void dt_compute(const DtProgram &p, unsigned char *smem)
             float *y = op.y;
             if (op.nmat == 2) {
                 const float g1 = *reinterpret_cast<const float *>(inf + DT_INFO_G + 4);
-                const int n = tk.idx * (DT_ROWS / 2) + warp * 8 + g;
-#pragma unroll
-                for (int tt = 0; tt < TT; ++tt)
-#pragma unroll
-                    for (int q = 0; q < 2; ++q) {
-                        const int m = tt * 8 + 2 * t4 + q;
-                        if (m < M && n < N) {
-                            const int rsm = irs[m];
-                            const float sm = is[m];
-                            const float gv = __fmul_rn((float)(acc[0][tt][q] - rsm), __fdiv_rn(g0, sm));
-                            const float uv = __fmul_rn((float)(acc[0][tt][2 + q] - rsm), __fdiv_rn(g1, sm));
-                            const float pg = gv > 0.0f ? gv : 0.0f;
-                            y[(size_t)m * N + n] = __fmul_rn(__fmul_rn(pg, pg), uv);
-                        }
-                    }
-            } else {
-                const int n0 = tk.idx * DT_ROWS + warp * 16 + g;
 #pragma unroll
                 for (int tt = 0; tt < TT; ++tt)
 #pragma unroll
@@ -696,11 +707,38 @@ BITNET_DEVINL void dt_compute(const DtProgram &p, unsigned char *smem)
                         const int m = tt * 8 + 2 * t4 + q;
                         if (m < M) {
                             const int rsm = irs[m];
-                            const float r = __fdiv_rn(g0, is[m]);
+                            const float sm = is[m];
+                            const float rg0 = __fdiv_rn(g0, sm), rg1 = __fdiv_rn(g1, sm);
 #pragma unroll
-                            for (int h = 0; h < 2; ++h) {
-                                const int n = n0 + 8 * h;
-                                if (n < N) y[(size_t)m * N + n] = __fmul_rn((float)(acc[0][tt][2 * h + q] - rsm), r);
+                            for (int r = 0; r < RG; ++r) {
+                                const int n = tk.idx * (RG * DT_ROWS / 2) + (warp + 8 * r) * 8 + g;
+                                if (n < N) {
+                                    const float gv = __fmul_rn((float)(acc[r][0][tt][q] - rsm), rg0);
+                                    const float uv = __fmul_rn((float)(acc[r][0][tt][2 + q] - rsm), rg1);
+                                    const float pg = gv > 0.0f ? gv : 0.0f;
+                                    y[(size_t)m * N + n] = __fmul_rn(__fmul_rn(pg, pg), uv);
+                                }
+                            }
+                        }
+                    }
+            } else {
+#pragma unroll
+                for (int tt = 0; tt < TT; ++tt)
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {
+                        const int m = tt * 8 + 2 * t4 + q;
+                        if (m < M) {
+                            const int rsm = irs[m];
+                            const float rsc = __fdiv_rn(g0, is[m]);
+#pragma unroll
+                            for (int r = 0; r < RG; ++r) {
+                                const int n0 = tk.idx * (RG * DT_ROWS) + (warp + 8 * r) * 16 + g;
+#pragma unroll
+                                for (int h = 0; h < 2; ++h) {
+                                    const int n = n0 + 8 * h;
+                                    if (n < N)
+                                        y[(size_t)m * N + n] = __fmul_rn((float)(acc[r][0][tt][2 * h + q] - rsm), rsc);
+                                }
                             }
                         }
                     }
@@ -744,7 +782,7 @@ BITNET_DEVINL void dt_completion(const DtProgram &p, unsigned char *smem)
     }
 }
 
-template <int TT>
+template <int TT, int RG>
 __global__ void __launch_bounds__(DT_THREADS, 1) k_decode_tasks(const __grid_constant__ DtProgram p)
 {
     extern __shared__ unsigned char dt_smem_raw[];
@@ -767,10 +805,10 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_decode_tasks(const __grid_con
     }
     __syncthreads();
     const int warp = tid >> 5;
-    if (warp == 8) dt_weight_producer(p, smem);
-    else if (warp == 9) dt_act_producer(p, smem);
+    if (warp == 8) dt_weight_producer<RG>(p, smem);
+    else if (warp == 9) dt_act_producer<RG>(p, smem);
     else if (warp == 10) dt_completion(p, smem);
-    else dt_compute<TT>(p, smem);
+    else dt_compute<TT, RG>(p, smem);
     __syncthreads();
     if (tid == 0) {
         // the last CTA out leaves the counters zeroed for the next launch

@@ -302,8 +302,11 @@ def test_test_stall_setter():
 
 
 # ---------------------------------------------------------------- task groups and their order
-def rows_per_task(o):
-    return 64 if o.kind == tw.BITNET_OP_FFN_GATE_UP else 128
+def rows_per_task(o, m):
+    """Packed rows of a task: 128 (a gated FFN: 64 outputs) per 16-row group of each of the 8
+    compute warps; two groups per warp when the tokens fit one 8-token tile."""
+    rg = 2 if m <= 8 else 1
+    return (64 if o.kind == tw.BITNET_OP_FFN_GATE_UP else 128) * rg
 
 
 def ranges(o, m):
@@ -326,7 +329,7 @@ def check_tasks(ops, m, groups):
         key = (gr["op"], gr["kind"])
         assert key not in pos
         pos[key] = k
-        want = m if gr["kind"] == "quant" else -(-o.N // rows_per_task(o))
+        want = m if gr["kind"] == "quant" else -(-o.N // rows_per_task(o, m))
         assert gr["tasks"] == want
         assert all(0 <= d < k for d in gr["deps"])
         assert len(gr["deps"]) <= (9 if gr["kind"] == "rows" else 8)
@@ -402,7 +405,7 @@ def test_tasks_of_the_bench_decode_step():
         assert groups[pos[(dn, "quant")]]["deps"] == [pos[(gu, "rows")]]
         for j in (4 * l, 4 * l + 1, gu, dn):
             assert groups[pos[(j, "rows")]]["deps"] == [pos[(j, "quant")]]
-    assert sum(g["tasks"] for g in groups) == 30 * (4 * 8 + 20 + 20 + 108 + 20)
+    assert sum(g["tasks"] for g in groups) == 30 * (4 * 8 + 10 + 10 + 54 + 10)  # 256-row tasks at M = 8
 
 
 def test_tasks_of_a_stack_sharing_its_output_buffers():
