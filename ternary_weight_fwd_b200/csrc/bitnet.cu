@@ -276,18 +276,24 @@ cudaError_t launch_quant_t(const void *x, int64_t M, int64_t K, int8_t *xq, floa
                       amax_in, amax_zero);
 }
 
-// RMS normalisation + quantiser: rows of up to 4096 elements on 128 threads (two rows
-// per CTA), longer rows (up to 8192) on 256.
-constexpr int64_t kNormMaxK = 256 * RQ_MAX_PER_THREAD;
-
+// RMS normalisation + quantiser: the row layout of launch_quant_t (1, 2, 4 or 8
+// warps per row by the number of 16-byte chunks), rows of up to kNormMaxK.
 template <bool XF32>
 cudaError_t launch_norm_quant_t(const void *x, int64_t M, int64_t K, const float *g, float eps, int8_t *xq, float *s,
                                 int32_t *rs, float *amax_zero, cudaStream_t stream)
 {
-    if (K <= 128 * RQ_MAX_PER_THREAD)
-        return launch_pdl(k_rmsnorm_quant_rows<XF32, 128>, dim3((unsigned)cdiv(M, 2)), dim3(256), 0, stream, x, M, K,
+    const int64_t nch = K / (XF32 ? 4 : 8);
+    const int64_t per_warp = 32 * QR_NCH;
+    if (nch <= per_warp)
+        return launch_pdl(k_rmsnorm_quant_rows<XF32, 1>, dim3((unsigned)cdiv(M, 8)), dim3(256), 0, stream, x, M, K,
                           g, eps, xq, s, rs, amax_zero);
-    return launch_pdl(k_rmsnorm_quant_rows<XF32, 256>, dim3((unsigned)M), dim3(256), 0, stream, x, M, K, g, eps, xq, s,
+    if (nch <= 2 * per_warp)
+        return launch_pdl(k_rmsnorm_quant_rows<XF32, 2>, dim3((unsigned)cdiv(M, 4)), dim3(256), 0, stream, x, M, K,
+                          g, eps, xq, s, rs, amax_zero);
+    if (nch <= 4 * per_warp)
+        return launch_pdl(k_rmsnorm_quant_rows<XF32, 4>, dim3((unsigned)cdiv(M, 2)), dim3(256), 0, stream, x, M, K,
+                          g, eps, xq, s, rs, amax_zero);
+    return launch_pdl(k_rmsnorm_quant_rows<XF32, 8>, dim3((unsigned)M), dim3(256), 0, stream, x, M, K, g, eps, xq, s,
                       rs, amax_zero);
 }
 

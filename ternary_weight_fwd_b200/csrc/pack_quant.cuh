@@ -255,143 +255,205 @@ __global__ void __launch_bounds__(128) k_zero_f32(float *__restrict__ amax, int 
 // RMS normalisation (subln) fused in front of the per-token absmax quantiser:
 // y = (x * r) * g with r = 1 / sqrt(mean(x^2) + eps), then the quantiser on y.
 // BitNet model page, "Model details" / "Architecture" (subln normalisation, no
-// bias) and BitNetConfig (rms_norm_eps).  Each row is held in registers by
-// 128 or 256 threads, so x is read once.  The sum of squares is the exact sum
-// rounded once to binary64 (exact_sumsq.cuh: 128-bit integer partials, or a
-// long accumulator for rows of very wide range), so no summation order enters
-// the result; r is computed in binary64 (correctly rounded division and square
-// root) and rounded once to binary32.
+// bias) and BitNetConfig (rms_norm_eps).  Same row layout as k_quant_rows_reg
+// (WPR warps per row, 16-byte chunks in registers), so x is read from HBM once
+// and x_q written in 8- or 4-byte pieces.  The sum of squares is the exact sum
+// rounded once to binary64 (exact_sumsq.cuh: 128-bit integer partials anchored
+// at the exponent of the row maximum, or a long accumulator for rows of very
+// wide range), so no summation order enters the result; r is computed in
+// binary64 (correctly rounded division and square root) and rounded once to
+// binary32.  y is recomputed for the quantise step rather than kept.
 // ---------------------------------------------------------------------------
-constexpr int RQ_MAX_PER_THREAD = 32; // elements a thread holds in registers
+constexpr int64_t kNormMaxK = 8192; // the 128-bit window and the long accumulator are sized for 8192 terms
 
-// TPR threads per row (128 or 256), 256 / TPR rows per CTA.
-template <bool XF32, int TPR>
+// The EPC values of a 16-byte chunk as fp32.
+template <bool XF32>
+BITNET_DEVINL void chunk_values(const uint4 v, float (&f)[XF32 ? 4 : 8])
+{
+    if constexpr (XF32) {
+        f[0] = __uint_as_float(v.x), f[1] = __uint_as_float(v.y);
+        f[2] = __uint_as_float(v.z), f[3] = __uint_as_float(v.w);
+    } else {
+        f[0] = bf16_bits_lo(v.x), f[1] = bf16_bits_hi(v.x), f[2] = bf16_bits_lo(v.y), f[3] = bf16_bits_hi(v.y);
+        f[4] = bf16_bits_lo(v.z), f[5] = bf16_bits_hi(v.z), f[6] = bf16_bits_lo(v.w), f[7] = bf16_bits_hi(v.w);
+    }
+}
+
+// y = (x * r) * g for the EPC values of chunk c.
+template <bool XF32>
+BITNET_DEVINL void chunk_norm(const uint4 v, int c, float r, const float *__restrict__ g, float (&y)[XF32 ? 4 : 8])
+{
+    constexpr int EPC = XF32 ? 4 : 8;
+    float gg[EPC];
+    const float4 g0 = __ldg(reinterpret_cast<const float4 *>(g) + (EPC / 4) * c);
+    gg[0] = g0.x, gg[1] = g0.y, gg[2] = g0.z, gg[3] = g0.w;
+    if constexpr (!XF32) {
+        const float4 g1 = __ldg(reinterpret_cast<const float4 *>(g) + 2 * c + 1);
+        gg[4] = g1.x, gg[5] = g1.y, gg[6] = g1.z, gg[7] = g1.w;
+    }
+    chunk_values<XF32>(v, y);
+#pragma unroll
+    for (int j = 0; j < EPC; ++j) y[j] = __fmul_rn(__fmul_rn(y[j], r), gg[j]);
+}
+
+template <bool XF32, int WPR>
 __global__ void __launch_bounds__(256) k_rmsnorm_quant_rows(const void *__restrict__ x, int64_t M, int64_t K,
                                                             const float *__restrict__ g, float eps,
                                                             int8_t *__restrict__ x_q, float *__restrict__ s,
                                                             int32_t *__restrict__ rowsum, float *__restrict__ amax_zero)
 {
-    constexpr int RPC = 256 / TPR;         // rows per CTA
-    constexpr int WPR = TPR / 32;          // warps per row
-    __shared__ uint64_t red_lo[RPC][WPR], red_hi[RPC][WPR];
+    constexpr int RPC = 8 / WPR;       // rows per CTA
+    constexpr int EPC = XF32 ? 4 : 8;  // elements per 16-byte chunk
+    __shared__ float red_x[8], red_y[8];
+    __shared__ uint64_t red_lo[8], red_hi[8];
+    __shared__ int red_fit[8], red_sum[8];
     __shared__ unsigned long long dig[RPC][SS_LONG_DIGITS];
-    __shared__ uint32_t red_e[RPC][WPR];
-    __shared__ int red_fit[RPC][WPR];
-    __shared__ float red_max[RPC][WPR];
-    __shared__ int red_sum[RPC][WPR];
-    __shared__ float bcast[RPC][2];
     pdl_launch_dependents();
     pdl_wait();
-    const int lr = threadIdx.x / TPR;      // row of this CTA
-    const int t = threadIdx.x % TPR;       // thread within the row
-    const int wr = t >> 5, lane = t & 31;  // warp within the row
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int wr = warp % WPR, lr = warp / WPR, w0 = warp - wr;
     const int64_t m = (int64_t)blockIdx.x * RPC + lr;
     const bool live = m < M;
-    float v[RQ_MAX_PER_THREAD];
-    const int n = live ? (int)((K + TPR - 1 - t) / TPR) : 0; // elements k = t + TPR * e, e < n
-    if constexpr (XF32) {
-        const float *row = static_cast<const float *>(x) + (live ? m : 0) * K;
+    const int nch = (int)(K / EPC);
+    const int c0 = wr * 32 + lane;
+    const uint4 *row = reinterpret_cast<const uint4 *>(static_cast<const char *>(x) + (live ? m : 0) * K * (XF32 ? 4 : 2));
+    uint4 v[QR_NCH];
+    float xmax = 0.0f;
 #pragma unroll
-        for (int e = 0; e < RQ_MAX_PER_THREAD; ++e)
-            if (e < n) v[e] = __ldg(row + t + (int64_t)e * TPR);
-    } else {
-        const unsigned short *row = static_cast<const unsigned short *>(x) + (live ? m : 0) * K;
-#pragma unroll
-        for (int e = 0; e < RQ_MAX_PER_THREAD; ++e)
-            if (e < n) v[e] = __uint_as_float((uint32_t)__ldg(row + t + (int64_t)e * TPR) << 16);
+    for (int i = 0; i < QR_NCH; ++i) {
+        const int c = c0 + i * 32 * WPR;
+        if (live && c < nch) {
+            v[i] = __ldg(row + c);
+            xmax = fmaxf(xmax, chunk_absmax<XF32>(v[i]));
+        }
     }
-    // largest exponent of the row (anchors the 128-bit window)
-    uint32_t emax = 0;
+    // the exponent of the row maximum anchors the 128-bit window
+    xmax = warp_max(xmax);
+    if constexpr (WPR > 1) {
+        if (lane == 0) red_x[warp] = xmax;
+        __syncthreads();
 #pragma unroll
-    for (int e = 0; e < RQ_MAX_PER_THREAD; ++e)
-        if (e < n) emax = max(emax, ss_exponent(v[e]));
-    emax = __reduce_max_sync(0xffffffffu, emax);
-    if (lane == 0) red_e[lr][wr] = emax;
-    if (t < SS_LONG_DIGITS) dig[lr][t] = 0ull;
-    __syncthreads();
-    uint32_t E = 0;
-#pragma unroll
-    for (int w = 0; w < WPR; ++w) E = max(E, red_e[lr][w]);
+        for (int i = 0; i < WPR; ++i) xmax = fmaxf(xmax, red_x[w0 + i]);
+    }
+    const uint32_t E = ss_exponent(xmax);
     SsWindow acc;
     if (E != 0) {
 #pragma unroll
-        for (int e = 0; e < RQ_MAX_PER_THREAD; ++e)
-            if (e < n) ss_window_add(acc, v[e], E);
+        for (int i = 0; i < QR_NCH; ++i) {
+            const int c = c0 + i * 32 * WPR;
+            if (live && c < nch) {
+                float f[EPC];
+                chunk_values<XF32>(v[i], f);
+#pragma unroll
+                for (int j = 0; j < EPC; ++j) ss_window_add(acc, f[j], E);
+            }
+        }
     }
     ss_warp_sum(acc.lo, acc.hi);
-    const bool fits = __all_sync(0xffffffffu, acc.fits);
-    if (lane == 0) {
-        red_lo[lr][wr] = acc.lo;
-        red_hi[lr][wr] = acc.hi;
-        red_fit[lr][wr] = fits ? 1 : 0;
-    }
-    __syncthreads();
-    // a row with a value too far below its largest takes the long accumulator
-    bool row_slow = false, any_slow = false;
-#pragma unroll
-    for (int q = 0; q < RPC; ++q) {
-        bool f = true;
-#pragma unroll
-        for (int w = 0; w < WPR; ++w) f = f && red_fit[q][w] != 0;
-        if (q == lr) row_slow = !f;
-        any_slow = any_slow || !f;
-    }
-    if (any_slow) { // uniform over the CTA
-        if (row_slow) {
-#pragma unroll
-            for (int e = 0; e < RQ_MAX_PER_THREAD; ++e)
-                if (e < n) ss_long_add(dig[lr], v[e]);
+    bool row_slow = !__all_sync(0xffffffffu, acc.fits);
+    uint64_t lo = acc.lo, hi = acc.hi;
+    if constexpr (WPR > 1) {
+        if (lane == 0) {
+            red_lo[warp] = lo;
+            red_hi[warp] = hi;
+            red_fit[warp] = row_slow ? 0 : 1;
         }
+        // a row with a value too far below its maximum takes the long accumulator
+        const int any_slow = __syncthreads_or(row_slow ? 1 : 0);
+        lo = hi = 0;
+        row_slow = false;
+#pragma unroll
+        for (int i = 0; i < WPR; ++i) {
+            ss_add128(lo, hi, red_lo[w0 + i], red_hi[w0 + i]);
+            row_slow = row_slow || red_fit[w0 + i] == 0;
+        }
+        if (any_slow) { // uniform over the CTA
+            if (wr == 0 && lane < SS_LONG_DIGITS) dig[lr][lane] = 0ull;
+            __syncthreads();
+            if (row_slow) {
+#pragma unroll
+                for (int i = 0; i < QR_NCH; ++i) {
+                    const int c = c0 + i * 32 * WPR;
+                    if (live && c < nch) {
+                        float f[EPC];
+                        chunk_values<XF32>(v[i], f);
+#pragma unroll
+                        for (int j = 0; j < EPC; ++j) ss_long_add(dig[lr], f[j]);
+                    }
+                }
+            }
+            __syncthreads();
+        }
+    } else if (row_slow) { // uniform over the warp, which holds the whole row
+        if (lane < SS_LONG_DIGITS) dig[lr][lane] = 0ull;
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < QR_NCH; ++i) {
+            const int c = c0 + i * 32;
+            if (live && c < nch) {
+                float f[EPC];
+                chunk_values<XF32>(v[i], f);
+#pragma unroll
+                for (int j = 0; j < EPC; ++j) ss_long_add(dig[lr], f[j]);
+            }
+        }
+        __syncwarp();
+    }
+    // every lane evaluates r (the same binary64 operations, no broadcast needed)
+    const double ss = row_slow ? ss_long_round(dig[lr]) : (E ? ss_window_round(lo, hi, E) : 0.0);
+    const double mean = __ddiv_rn(ss, (double)K);
+    const float r = __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(mean, (double)eps))));
+    float ymax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < QR_NCH; ++i) {
+        const int c = c0 + i * 32 * WPR;
+        if (live && c < nch) {
+            float y[EPC];
+            chunk_norm<XF32>(v[i], c, r, g, y);
+#pragma unroll
+            for (int j = 0; j < EPC; ++j) ymax = fmaxf(ymax, fabsf(y[j]));
+        }
+    }
+    ymax = warp_max(ymax);
+    if constexpr (WPR > 1) {
+        if (lane == 0) red_y[warp] = ymax;
         __syncthreads();
-    }
-    if (t == 0) {
-        double ss;
-        if (row_slow) {
-            ss = ss_long_round(dig[lr]);
-        } else {
-            uint64_t lo = 0, hi = 0;
-            for (int w = 0; w < WPR; ++w) ss_add128(lo, hi, red_lo[lr][w], red_hi[lr][w]);
-            ss = E ? ss_window_round(lo, hi, E) : 0.0;
-        }
-        const double mean = __ddiv_rn(ss, (double)K);
-        bcast[lr][0] = __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(mean, (double)eps))));
-    }
-    __syncthreads();
-    const float r = bcast[lr][0];
-    float mx = 0.0f;
 #pragma unroll
-    for (int e = 0; e < RQ_MAX_PER_THREAD; ++e)
-        if (e < n) {
-            v[e] = __fmul_rn(__fmul_rn(v[e], r), __ldg(g + t + e * TPR));
-            mx = fmaxf(mx, fabsf(v[e]));
-        }
-    mx = warp_max(mx);
-    if (lane == 0) red_max[lr][wr] = mx;
-    __syncthreads();
-    if (t == 0) {
-        float am = 0.0f;
-        for (int w = 0; w < WPR; ++w) am = fmaxf(am, red_max[lr][w]);
-        bcast[lr][1] = quant_scale(am);
+        for (int i = 0; i < WPR; ++i) ymax = fmaxf(ymax, red_y[w0 + i]);
     }
-    __syncthreads();
-    const float sc = bcast[lr][1];
+    const float sc = quant_scale(ymax);
     int rs = 0;
     int8_t *qrow = x_q + (live ? m : 0) * K;
 #pragma unroll
-    for (int e = 0; e < RQ_MAX_PER_THREAD; ++e)
-        if (e < n) {
-            const int q = quant_one(v[e], sc);
-            qrow[t + e * TPR] = (int8_t)q;
-            rs += q;
+    for (int i = 0; i < QR_NCH; ++i) {
+        const int c = c0 + i * 32 * WPR;
+        if (live && c < nch) {
+            float y[EPC];
+            chunk_norm<XF32>(v[i], c, r, g, y);
+            int q[EPC];
+#pragma unroll
+            for (int j = 0; j < EPC; ++j) {
+                q[j] = quant_one(y[j], sc);
+                rs += q[j];
+            }
+            if constexpr (XF32)
+                reinterpret_cast<uint32_t *>(qrow)[c] = pack4_s8(q[0], q[1], q[2], q[3]);
+            else
+                reinterpret_cast<uint2 *>(qrow)[c] = make_uint2(pack4_s8(q[0], q[1], q[2], q[3]),
+                                                                pack4_s8(q[4], q[5], q[6], q[7]));
         }
+    }
     rs = warp_sum(rs);
-    if (lane == 0) red_sum[lr][wr] = rs;
-    __syncthreads();
-    if (t == 0 && live) {
-        int tot = 0;
-        for (int w = 0; w < WPR; ++w) tot += red_sum[lr][w];
+    if constexpr (WPR > 1) {
+        if (lane == 0) red_sum[warp] = rs;
+        __syncthreads();
+        rs = 0;
+#pragma unroll
+        for (int i = 0; i < WPR; ++i) rs += red_sum[w0 + i];
+    }
+    if (live && wr == 0 && lane == 0) {
         s[m] = sc;
-        if (rowsum) rowsum[m] = tot;
+        if (rowsum) rowsum[m] = rs;
         if (amax_zero) amax_zero[m] = 0.0f;
     }
 }
