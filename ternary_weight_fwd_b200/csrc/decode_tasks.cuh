@@ -543,50 +543,90 @@ BITNET_DEVINL void dt_quant_row(const DtProgram &p, const DtOp &op, int m, unsig
 }
 
 // ---- row task contraction over one piece (compute warp w) ------------------
-// acc[r][a][tt][4]: row group r of the warp (rows 16 (w + 8 r) ..), accumulator
-// set a (the two mma of a k-block go to different sets so that consecutive mma
-// are independent), token tile tt.  wrow: this lane's word in row group 0; row
-// group r is r * 128 rows further.
-template <int TT, int NACC, int RG>
-BITNET_DEVINL void dt_kblock(int (&acc)[RG][NACC][TT][4], const uint32_t (&lo)[RG], const uint32_t (&hi)[RG],
-                             const uint4 *bpre, uint32_t xrow, int Mp, int kb)
+// The A fragments are the packed words masked in place, without shifting:
+// (w & (0x03030303 << 2j)) holds the codes of position j of each byte scaled
+// by 4^j (at most 2 * 64 = 128: still a u8 operand).  Accumulator set
+// acc[r][j] (SC = 4) therefore collects 4^j * sum c*x, exactly (|sum c*x| <
+// 2^21 for K <= 8192, so 64 * it fits int32), and the sets are combined with
+// exact arithmetic shifts at the end of the task.  With SC = 2 (many token
+// tiles, fewer registers) the word is used as is for positions 0, 1 and
+// shifted by 4 for positions 2, 3: set j & 1 holds 4^(j & 1) * its sum.
+// One mma covers a pair of k-blocks (its two k halves) at one position j.
+// acc[r][j][tt][4]: row group r of the warp (rows 16 (w + 8 r) ..), set j,
+// token tile tt.  wrow: this lane's word in row group 0 (row group r is
+// r * 128 rows further).
+template <int SC>
+BITNET_DEVINL uint32_t dt_code_bits(uint32_t w, uint32_t w4, int j)
 {
-    constexpr uint32_t M3 = 0x03030303u;
+    if constexpr (SC == 4) return w & (0x03030303u << (2 * j));
+    else return (j < 2 ? w : w4) & (0x03030303u << (2 * (j & 1)));
+}
+
+template <int TT, int SC, int RG>
+BITNET_DEVINL void dt_kpair(int (&acc)[RG][SC][TT][4], const uint32_t (&l0)[RG], const uint32_t (&h0)[RG],
+                            const uint32_t (&l1)[RG], const uint32_t (&h1)[RG], const uint4 (&b0)[TT],
+                            const uint4 (&b1)[TT])
+{
 #pragma unroll
-    for (int tt = 0; tt < TT; ++tt) {
-        uint4 b;
-        if (bpre) {
-            b = bpre[tt];
-        } else {
-            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                         : "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w)
-                         : "r"(xrow + (uint32_t)((kb * Mp + tt * 8) * 64)));
-        }
+    for (int r = 0; r < RG; ++r) {
+        const uint32_t L0 = l0[r], H0 = h0[r], L1 = l1[r], H1 = h1[r];
+        const uint32_t L04 = SC == 4 ? 0u : L0 >> 4, H04 = SC == 4 ? 0u : H0 >> 4;
+        const uint32_t L14 = SC == 4 ? 0u : L1 >> 4, H14 = SC == 4 ? 0u : H1 >> 4;
 #pragma unroll
-        for (int r = 0; r < RG; ++r) {
-            const uint32_t l = lo[r], h = hi[r];
-            mma_u8s8_16832(acc[r][(2 * kb) % NACC][tt], l & M3, h & M3, (l >> 2) & M3, (h >> 2) & M3, b.x, b.y);
-            mma_u8s8_16832(acc[r][(2 * kb + 1) % NACC][tt], (l >> 4) & M3, (h >> 4) & M3, (l >> 6) & M3,
-                           (h >> 6) & M3, b.z, b.w);
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t a0 = dt_code_bits<SC>(L0, L04, j), a1 = dt_code_bits<SC>(H0, H04, j);
+            const uint32_t a2 = dt_code_bits<SC>(L1, L14, j), a3 = dt_code_bits<SC>(H1, H14, j);
+#pragma unroll
+            for (int tt = 0; tt < TT; ++tt) {
+                const uint32_t bj0 = j == 0 ? b0[tt].x : j == 1 ? b0[tt].y : j == 2 ? b0[tt].z : b0[tt].w;
+                const uint32_t bj1 = j == 0 ? b1[tt].x : j == 1 ? b1[tt].y : j == 2 ? b1[tt].z : b1[tt].w;
+                mma_u8s8_16832(acc[r][SC == 4 ? j : (j & 1)][tt], a0, a1, a2, a3, bj0, bj1);
+            }
         }
     }
 }
 
-// A ragged piece (fewer than 8 k-blocks).
-template <int TT, int NACC, int RG>
-BITNET_DEVINL void dt_piece(int (&acc)[RG][NACC][TT][4], uint32_t wrow, uint32_t xrow, int Mp, int nkb)
+BITNET_DEVINL uint4 dt_ld_b(uint32_t addr)
+{
+    uint4 b;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w) : "r"(addr));
+    return b;
+}
+
+template <int RG>
+BITNET_DEVINL void dt_ld_a(uint32_t (&lo)[RG], uint32_t (&hi)[RG], uint32_t wrow, int kb)
 {
 #pragma unroll
-    for (int kb = 0; kb < DT_KB; ++kb) {
-        if (kb < nkb) {
-            uint32_t lo[RG], hi[RG];
+    for (int r = 0; r < RG; ++r) {
+        const uint32_t a = wrow + (uint32_t)(r * DT_ROWS * DT_PITCH) + kb * 16;
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(lo[r]) : "r"(a));
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(hi[r]) : "r"(a + 8 * DT_PITCH));
+    }
+}
+
+// A ragged piece (fewer than 8 k-blocks; an odd last block is paired with zeros).
+template <int TT, int SC, int RG>
+BITNET_DEVINL void dt_piece(int (&acc)[RG][SC][TT][4], uint32_t wrow, uint32_t xrow, int Mp, int nkb)
+{
 #pragma unroll
-            for (int r = 0; r < RG; ++r) {
-                const uint32_t a = wrow + (uint32_t)(r * DT_ROWS * DT_PITCH) + kb * 16;
-                asm volatile("ld.shared.u32 %0, [%1];" : "=r"(lo[r]) : "r"(a));
-                asm volatile("ld.shared.u32 %0, [%1];" : "=r"(hi[r]) : "r"(a + 8 * DT_PITCH));
+    for (int kp = 0; kp < DT_KB / 2; ++kp) {
+        if (2 * kp < nkb) {
+            const bool two = 2 * kp + 1 < nkb;
+            uint32_t l0[RG], h0[RG], l1[RG], h1[RG];
+            uint4 b0[TT], b1[TT];
+            dt_ld_a<RG>(l0, h0, wrow, 2 * kp);
+            if (two) {
+                dt_ld_a<RG>(l1, h1, wrow, 2 * kp + 1);
+            } else {
+#pragma unroll
+                for (int r = 0; r < RG; ++r) l1[r] = h1[r] = 0u;
             }
-            dt_kblock<TT, NACC, RG>(acc, lo, hi, nullptr, xrow, Mp, kb);
+#pragma unroll
+            for (int tt = 0; tt < TT; ++tt) {
+                b0[tt] = dt_ld_b(xrow + (uint32_t)((2 * kp * Mp + tt * 8) * 64));
+                b1[tt] = two ? dt_ld_b(xrow + (uint32_t)(((2 * kp + 1) * Mp + tt * 8) * 64)) : make_uint4(0, 0, 0, 0);
+            }
+            dt_kpair<TT, SC, RG>(acc, l0, h0, l1, h1, b0, b1);
         }
     }
 }
@@ -594,37 +634,38 @@ BITNET_DEVINL void dt_piece(int (&acc)[RG][NACC][TT][4], uint32_t wrow, uint32_t
 // A full piece (8 k-blocks): every weight fragment (and, for one token tile,
 // every activation fragment) is loaded before the first mma, so the
 // shared-memory latency is paid once per piece.
-template <int TT, int NACC, int RG>
-BITNET_DEVINL void dt_piece_full(int (&acc)[RG][NACC][TT][4], uint32_t wrow, uint32_t xrow, int Mp)
+template <int TT, int SC, int RG>
+BITNET_DEVINL void dt_piece_full(int (&acc)[RG][SC][TT][4], uint32_t wrow, uint32_t xrow, int Mp)
 {
     uint32_t lo[DT_KB][RG], hi[DT_KB][RG];
 #pragma unroll
-    for (int kb = 0; kb < DT_KB; ++kb)
-#pragma unroll
-        for (int r = 0; r < RG; ++r) {
-            const uint32_t a = wrow + (uint32_t)(r * DT_ROWS * DT_PITCH) + kb * 16;
-            asm volatile("ld.shared.u32 %0, [%1];" : "=r"(lo[kb][r]) : "r"(a));
-            asm volatile("ld.shared.u32 %0, [%1];" : "=r"(hi[kb][r]) : "r"(a + 8 * DT_PITCH));
-        }
+    for (int kb = 0; kb < DT_KB; ++kb) dt_ld_a<RG>(lo[kb], hi[kb], wrow, kb);
     if constexpr (TT == 1) {
-        uint4 bq[DT_KB];
+        uint4 bq[DT_KB][1];
 #pragma unroll
-        for (int kb = 0; kb < DT_KB; ++kb)
-            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                         : "=r"(bq[kb].x), "=r"(bq[kb].y), "=r"(bq[kb].z), "=r"(bq[kb].w)
-                         : "r"(xrow + (uint32_t)(kb * Mp * 64)));
+        for (int kb = 0; kb < DT_KB; ++kb) bq[kb][0] = dt_ld_b(xrow + (uint32_t)(kb * Mp * 64));
 #pragma unroll
-        for (int kb = 0; kb < DT_KB; ++kb) dt_kblock<TT, NACC, RG>(acc, lo[kb], hi[kb], &bq[kb], xrow, Mp, kb);
+        for (int kp = 0; kp < DT_KB / 2; ++kp)
+            dt_kpair<TT, SC, RG>(acc, lo[2 * kp], hi[2 * kp], lo[2 * kp + 1], hi[2 * kp + 1], bq[2 * kp],
+                                 bq[2 * kp + 1]);
     } else {
 #pragma unroll
-        for (int kb = 0; kb < DT_KB; ++kb) dt_kblock<TT, NACC, RG>(acc, lo[kb], hi[kb], nullptr, xrow, Mp, kb);
+        for (int kp = 0; kp < DT_KB / 2; ++kp) {
+            uint4 b0[TT], b1[TT];
+#pragma unroll
+            for (int tt = 0; tt < TT; ++tt) {
+                b0[tt] = dt_ld_b(xrow + (uint32_t)((2 * kp * Mp + tt * 8) * 64));
+                b1[tt] = dt_ld_b(xrow + (uint32_t)(((2 * kp + 1) * Mp + tt * 8) * 64));
+            }
+            dt_kpair<TT, SC, RG>(acc, lo[2 * kp], hi[2 * kp], lo[2 * kp + 1], hi[2 * kp + 1], b0, b1);
+        }
     }
 }
 
 template <int TT, int RG>
 BITNET_DEVINL void dt_compute(const DtProgram &p, unsigned char *smem)
 {
-    constexpr int NACC = TT <= 2 ? 4 : 2;
+    constexpr int SC = TT <= 2 ? 4 : 2; // accumulator sets (scales of the masked codes)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, t4 = lane & 3;
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + DT_BAR_FULL);
@@ -657,11 +698,11 @@ BITNET_DEVINL void dt_compute(const DtProgram &p, unsigned char *smem)
             __syncwarp();
             if (lane == 0) mbar_arrive(&cdone[e]);
         } else {
-            int acc[RG][NACC][TT][4];
+            int acc[RG][SC][TT][4];
 #pragma unroll
             for (int r = 0; r < RG; ++r)
 #pragma unroll
-                for (int a = 0; a < NACC; ++a)
+                for (int a = 0; a < SC; ++a)
 #pragma unroll
                     for (int tt = 0; tt < TT; ++tt)
 #pragma unroll
@@ -676,20 +717,21 @@ BITNET_DEVINL void dt_compute(const DtProgram &p, unsigned char *smem)
                 const uint32_t base = ring + (uint32_t)s * (uint32_t)p.slot_bytes;
                 const int nkb = min(DT_KB, (K - pc * DT_KC) >> 6);
                 if (nkb == DT_KB)
-                    dt_piece_full<TT, NACC, RG>(acc, base + wlane, base + xlane, Mp);
+                    dt_piece_full<TT, SC, RG>(acc, base + wlane, base + xlane, Mp);
                 else
-                    dt_piece<TT, NACC, RG>(acc, base + wlane, base + xlane, Mp, nkb);
+                    dt_piece<TT, SC, RG>(acc, base + wlane, base + xlane, Mp, nkb);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&empty[s]);
             }
+            // set a holds 4^a times its sum: exact arithmetic shifts
 #pragma unroll
             for (int r = 0; r < RG; ++r)
 #pragma unroll
-                for (int a = 1; a < NACC; ++a)
+                for (int a = 1; a < SC; ++a)
 #pragma unroll
                     for (int tt = 0; tt < TT; ++tt)
 #pragma unroll
-                        for (int c = 0; c < 4; ++c) acc[r][0][tt][c] += acc[r][a][tt][c];
+                        for (int c = 0; c < 4; ++c) acc[r][0][tt][c] += acc[r][a][tt][c] >> (2 * a);
             // epilogue: y = fl((float)(sum c*x - sum x) * fl(gamma / s))
             mbar_wait(&qinfo[e], (seq / DT_QUEUE) & 1u);
             const unsigned char *inf = smem + DT_INFO + e * DT_INFO_BYTES;
