@@ -260,10 +260,11 @@ BITNET_DEVINL void dt_weight_producer(const DtProgram &p, unsigned char *smem)
     const int r0 = lane >> 3;
     uint32_t seq = 0;
     DtRing ring_pos;
+    // the claim of the next task is issued one task ahead, so its latency overlaps the copies
+    unsigned claim = 0;
+    if (lane == 0) claim = atomicAdd(&p.counters[DT_CNT_TASK], 1u);
     for (;;) {
-        int t = 0;
-        if (lane == 0) t = (int)atomicAdd(&p.counters[DT_CNT_TASK], 1u);
-        t = __shfl_sync(0xffffffffu, t, 0);
+        int t = (int)__shfl_sync(0xffffffffu, claim, 0);
         if (t >= p.n_tasks) t = -1;
         const int e = (int)(seq % DT_QUEUE);
         mbar_wait(&qempty[e], ((seq / DT_QUEUE) & 1u) ^ 1u);
@@ -273,6 +274,7 @@ BITNET_DEVINL void dt_weight_producer(const DtProgram &p, unsigned char *smem)
         }
         ++seq;
         if (t < 0) break;
+        if (lane == 0) claim = atomicAdd(&p.counters[DT_CNT_TASK], 1u);
         const DtTask tk = dt_decode(p, t);
         if (tk.quant) continue;
         const DtOp &op = p.ops[tk.op];
