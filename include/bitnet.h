@@ -326,12 +326,13 @@ typedef struct bitnet_op {
 
 /*
  * Workspace of bitnet_decode_sequence for up to n_ops ops over M tokens whose
- * K are at most K_max: completion counters, then per op the quantised
- * activations ([K/64][Mp][64] int8, Mp = M rounded up to 8, 16, 32 or 64),
- * scales and row sums.  A list of n ops needs exactly
- *   up256(4 * (2 + 2n)) + sum over ops of (up256(K * Mp) + 512) bytes
- * (up256 = rounded up to a multiple of 256); this returns that for n_ops ops
- * of K = K_max.  0 for arguments out of range.
+ * K are at most K_max: completion counters, the TMA tensor maps of the ops'
+ * weights (made by the kernel), then per op the quantised activations
+ * ([K/64][Mp][64] int8, Mp = M rounded up to 8, 16, 32 or 64), scales and row
+ * sums.  A list of n ops needs exactly
+ *   up256(4 * (2 + 3n)) + up256(256n + 128) + sum over ops of (up256(K * Mp) + 512)
+ * bytes (up256 = rounded up to a multiple of 256); this returns that for
+ * n_ops ops of K = K_max.  0 for arguments out of range.
  */
 size_t bitnet_sequence_workspace_size(int32_t n_ops, int64_t M, int64_t K_max);
 

@@ -905,8 +905,11 @@ std::vector<int> seq_group_order(const bitnet_op_t *ops, int n, int64_t M, const
     return order;
 }
 
-// Workspace: counters, then per op x_q [K/64][Mp][64], s [Mp], row sums [Mp].
-inline size_t seq_counter_bytes(int n) { return align_up(4 * (size_t)(DT_CNT_OPS + 2 * n), 256); }
+// Workspace: counters (per op: quant tasks done, row tasks done, state of its
+// tensor maps), the ops' weight tensor maps [n][2] x 128 bytes, then per op
+// x_q [K/64][Mp][64], s [Mp], row sums [Mp].
+inline size_t seq_counter_bytes(int n) { return align_up(4 * (size_t)(DT_CNT_OPS + 3 * n), 256); }
+inline size_t seq_map_bytes(int n) { return align_up((size_t)n * 2 * sizeof(CUtensorMap) + 128, 256); } // + alignment
 inline size_t seq_op_ws_bytes(int64_t K, int Mp) { return align_up((size_t)K * Mp, 256) + 512; }
 
 std::atomic<int> g_seq_stall{-1};                        // tests: op (list index) whose rows never become ready
@@ -921,7 +924,7 @@ bitnet_status_t seq_build(DtProgram &p, const bitnet_op_t *ops, const int32_t *u
     bitnet_status_t st = seq_groups(ops, n, M, extra, G);
     if (st != BITNET_OK) return st;
     const int Mp = seq_mp(M);
-    size_t need = seq_counter_bytes(n);
+    size_t need = seq_counter_bytes(n) + seq_map_bytes(n);
     for (int j = 0; j < n; ++j) need += seq_op_ws_bytes(ops[j].K, Mp);
     if (ws && ws_bytes < need) return BITNET_ERR_WORKSPACE;
     p.n_ops = n;
@@ -929,7 +932,11 @@ bitnet_status_t seq_build(DtProgram &p, const bitnet_op_t *ops, const int32_t *u
     p.Mp = Mp;
     p.counters = static_cast<unsigned *>(ws);
     char *base = static_cast<char *>(ws);
-    size_t off = seq_counter_bytes(n);
+    // tensor maps want 128-byte alignment; the workspace is only required to be 16-byte aligned
+    p.wmaps = base ? reinterpret_cast<CUtensorMap *>(align_up(reinterpret_cast<uintptr_t>(base) + seq_counter_bytes(n),
+                                                              (uintptr_t)128))
+                   : nullptr;
+    size_t off = seq_counter_bytes(n) + seq_map_bytes(n);
     const int stall = g_seq_stall.load();
     for (int j = 0; j < n; ++j) {
         const bitnet_op_t &o = ops[j];
@@ -985,7 +992,7 @@ bitnet_status_t seq_build(DtProgram &p, const bitnet_op_t *ops, const int32_t *u
     p.n_segs = ns;
     p.n_tasks = t;
     p.slot_bytes = seq_rg(M) * DT_WBYTES + DT_KC * Mp;
-    p.n_slots = (int)std::min<size_t>(DT_MAX_SLOTS, (kSmemLimit - 128 - DT_HDR) / (size_t)p.slot_bytes);
+    p.n_slots = (int)std::min<size_t>(DT_MAX_SLOTS, (kSmemLimit - 1024 - DT_HDR) / (size_t)p.slot_bytes);
     if (order_out) *order_out = order;
     return BITNET_OK;
 }
@@ -1000,7 +1007,7 @@ cudaError_t seq_launch_t(const DtProgram &p, int ctas, cudaStream_t stream, int 
     static std::atomic<int> smem_done[kMaxDevices];
     cudaError_t e = ensure_smem(k_decode_tasks<TT, RG>, kSmemLimit, smem_done, dev);
     if (e != cudaSuccess) return e;
-    const size_t smem = 128 + DT_HDR + (size_t)p.n_slots * p.slot_bytes;
+    const size_t smem = 1024 + DT_HDR + (size_t)p.n_slots * p.slot_bytes; // + alignment to 1024 bytes
     g_launches.fetch_add(1, std::memory_order_relaxed);
     k_decode_tasks<TT, RG><<<ctas, DT_THREADS, smem, stream>>>(p);
     return cudaGetLastError();
@@ -1090,6 +1097,10 @@ bitnet_status_t decode_sequence(const bitnet_op_t *ops, int n, int64_t M, void *
     st = seq_build(p, sched, order, n, M, ctas, workspace, ws_bytes, wsr);
     if (st != BITNET_OK) return st;
     if (p.n_slots < 2) return BITNET_ERR_UNSUPPORTED_SHAPE;
+    // the template of the weight maps (any op's first matrix: address, extent and pitch are replaced per op)
+    if (!encode_u8_2d(&p.wtmpl, sched[0].w0, (uint64_t)sched[0].N, (uint64_t)(sched[0].K / 4), DT_BOX_ROWS,
+                      DT_KC / 4, true))
+        return BITNET_ERR_CUDA;
     {
         // remember the plan under the caller's op list (least recently used entry replaced)
         std::lock_guard<std::mutex> lk(g_seq_cache_mu);
@@ -1269,7 +1280,8 @@ size_t bitnet_sequence_workspace_size(int32_t n_ops, int64_t M, int64_t K_max)
 {
     if (n_ops < 1 || n_ops > BITNET_SEQ_MAX_OPS || M < 1 || M > BITNET_SEQ_MAX_M || K_max < 64 || K_max > kSeqMaxK)
         return 0;
-    return seq_counter_bytes(n_ops) + (size_t)n_ops * seq_op_ws_bytes(align_up((size_t)K_max, 64), seq_mp(M));
+    return seq_counter_bytes(n_ops) + seq_map_bytes(n_ops) +
+           (size_t)n_ops * seq_op_ws_bytes(align_up((size_t)K_max, 64), seq_mp(M));
 }
 
 bitnet_status_t bitnet_sequence_plan(const bitnet_op_t *ops, int32_t n_ops, int64_t M, int32_t *wait_x,

@@ -29,9 +29,11 @@
 // Roles in a CTA (320 threads):
 //   warp 8  weight producer: claims tasks, writes them to a 4-entry queue in
 //           shared memory, streams each row task's packed weights into a ring of
-//           pieces (128 rows x 512 k, 16-byte cp.async, row pitch 144 bytes so
-//           the fragment loads hit 32 distinct banks).  Weights never wait for
-//           any other task.
+//           pieces (128 rows x 512 k: two TMA boxes of 64 rows x 128 bytes, with
+//           the 128-byte swizzle so the fragment loads hit 32 distinct banks).
+//           The tensor maps are made on the device, once per op and launch, from
+//           a template map (the matrix's address, extent and row pitch put in
+//           with tensormap.replace).  Weights never wait for any other task.
 //   warp 9  activation producer: for a row task, waits for its dependencies,
 //           copies the per-token scales and row sums and the gammas, and streams
 //           the matching x_q chunk ([8][Mp][64] bytes) next to each weight piece
@@ -60,8 +62,9 @@ constexpr int DT_THREADS = 352;                 // + weight producer (8), activa
 constexpr int DT_ROWS = 128;                    // packed rows per row task and 16-row group per warp
 constexpr int DT_KC = 512;                      // k per piece
 constexpr int DT_KB = DT_KC / 64;               // 64-k blocks per piece
-constexpr int DT_PITCH = DT_KC / 4 + 16;        // 144 = 16 * 9: conflict-free fragment loads
-constexpr int DT_WBYTES = DT_ROWS * DT_PITCH;   // 18432 weight bytes of a piece in shared memory, per row-group set
+constexpr int DT_PITCH = DT_KC / 4;             // 128-byte rows, 16-byte chunk c of row r at chunk c ^ (r & 7)
+constexpr int DT_WBYTES = DT_ROWS * DT_PITCH;   // 16384 weight bytes of a piece in shared memory, per row-group set
+constexpr int DT_BOX_ROWS = 64;                 // rows of one TMA box of weights
 constexpr int DT_QUEUE = 4;                     // tasks claimed ahead of the compute warps (at most)
 constexpr int DT_MAX_OPS = 128;
 constexpr int DT_MAX_SEGS = 512;
@@ -74,7 +77,8 @@ template <bool XF32> __host__ __device__ constexpr int dt_quant_ch() { return XF
 // counters (uint32) at the start of the workspace
 constexpr int DT_CNT_TASK = 0;  // next task to claim
 constexpr int DT_CNT_EXIT = 1;  // CTAs finished
-constexpr int DT_CNT_OPS = 2;   // then per op: quant tasks done, row tasks done (x 8 warps)
+constexpr int DT_CNT_OPS = 2;   // then per op: quant tasks done, row tasks done; then per op the
+                                // state of its tensor maps (0 none, 1 being made, 2 ready)
 
 constexpr uint16_t DT_DEP_QUANT = 0x8000u; // dependency on an op's quant tasks (else its row tasks)
 
@@ -104,8 +108,10 @@ struct DtSeg {        // consecutive tasks of one op in the global order
 };
 
 struct DtProgram {
+    CUtensorMap wtmpl;   // template of the weight maps: uint8 [N][K/4], box 64 rows x 128 bytes, 128-byte swizzle
     int n_ops, n_segs, n_tasks, M, Mp, n_slots, slot_bytes;
     unsigned *counters;
+    CUtensorMap *wmaps;  // workspace: [n_ops][2] maps of w0, w1 (made by the first CTA to need them)
     DtOp ops[DT_MAX_OPS];
     DtSeg segs[DT_MAX_SEGS];
 };
@@ -122,10 +128,12 @@ constexpr int DT_RED = 512;                           // quant-task reductions (
 constexpr int DT_INFO = 1024;                         // per queue entry: s[64] fp32, rs[64] int32, gamma0, gamma1
 constexpr int DT_INFO_S = 0, DT_INFO_RS = 4 * DT_MAX_M, DT_INFO_G = 8 * DT_MAX_M;
 constexpr int DT_INFO_BYTES = 8 * DT_MAX_M + 16;
+constexpr int DT_MAPS = 3584;                         // two 128-byte tensor maps being made
 constexpr int DT_HDR = 4096; // the piece ring starts here
-static_assert(DT_INFO + DT_QUEUE * DT_INFO_BYTES <= DT_HDR, "shared header");
+static_assert(DT_INFO + DT_QUEUE * DT_INFO_BYTES <= DT_MAPS, "shared header");
+static_assert(DT_MAPS + 256 <= DT_HDR && DT_MAPS % 128 == 0, "shared header");
 static_assert(DT_QTASK + 4 * DT_QUEUE <= DT_RED, "shared header");
-static_assert(DT_HDR % 128 == 0, "ring alignment");
+static_assert(DT_HDR % 1024 == 0 && DT_WBYTES % 1024 == 0, "ring alignment (128-byte swizzle)");
 
 // task t -> (op, kind, index)
 struct DtTask {
@@ -240,12 +248,80 @@ struct DtRing {
     }
 };
 
-// ---- weight producer (warp 8) ----------------------------------------------
-// Lane l copies 16-byte chunk j = l % 8 (a 64-k block of the piece) of shared
-// rows r = l / 8 + 4 i, i = 0 .. 31.  Shared row r of a BitLinear task is packed
-// row 128 b + r; of a gated-FFN task (rows 8 .. 15 of each 16-row group are the
-// up rows) it is row 64 b + 8 (r / 16) + r % 8 of the gate or the up matrix.
-// For i = 4 g + q the source row is rb[q] + g * rstep: four base rows per task.
+// ---- tensor maps of the weights -------------------------------------------
+// Made on the device from the template: the first warp to need op j's maps
+// (CAS 0 -> 1 on its state) writes them to the workspace and publishes them
+// (state 2, release); every weight producer acquires them before its first
+// copy with them.  The maker is a running CTA with no other wait in between,
+// so a warp that waits for state 2 always sees it.
+BITNET_DEVINL void dt_tmap_set(uint32_t sm, const void *w, int K, int N)
+{
+    asm volatile("tensormap.replace.tile.global_address.shared::cta.b1024.b64 [%0], %1;" ::"r"(sm), "l"(w)
+                 : "memory");
+    asm volatile("tensormap.replace.tile.global_dim.shared::cta.b1024.b32 [%0], 0, %1;" ::"r"(sm), "r"(K / 4)
+                 : "memory");
+    asm volatile("tensormap.replace.tile.global_dim.shared::cta.b1024.b32 [%0], 1, %1;" ::"r"(sm), "r"(N)
+                 : "memory");
+    asm volatile("tensormap.replace.tile.global_stride.shared::cta.b1024.b64 [%0], 0, %1;" ::"r"(sm),
+                 "l"((unsigned long long)(K / 4))
+                 : "memory");
+}
+
+// Whole warp: the 128-byte map at sm to global g, with a release fence for the tensor-map proxy.
+BITNET_DEVINL void dt_tmap_publish(CUtensorMap *g, uint32_t sm)
+{
+    asm volatile("tensormap.cp_fenceproxy.global.shared::cta.tensormap::generic.release.gpu.sync.aligned [%0], [%1], "
+                 "128;" ::"l"(g),
+                 "r"(sm)
+                 : "memory");
+}
+
+BITNET_DEVINL void dt_tmap_acquire(const CUtensorMap *g)
+{
+    asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(g) : "memory");
+}
+
+// Whole warp; lane 0 may then copy with op j's maps.  false: the wait for
+// another warp's maps ran out (status set).
+BITNET_DEVINL bool dt_maps_acquire(const DtProgram &p, int j, unsigned char *smem, uint32_t (&have)[DT_MAX_OPS / 32])
+{
+    const int lane = threadIdx.x & 31;
+    if (have[j >> 5] & (1u << (j & 31))) return true;
+    const DtOp &op = p.ops[j];
+    unsigned *state = &p.counters[DT_CNT_OPS + 2 * p.n_ops + j];
+    CUtensorMap *g = p.wmaps + 2 * j;
+    unsigned st = 0;
+    if (lane == 0) st = atomicCAS(state, 0u, 1u);
+    st = __shfl_sync(0xffffffffu, st, 0);
+    bool ok = true;
+    if (st == 0) {
+        for (int m = 0; m < op.nmat; ++m) {
+            unsigned char *sm = smem + DT_MAPS + 128 * m;
+            if (lane < 8) reinterpret_cast<uint4 *>(sm)[lane] = reinterpret_cast<const uint4 *>(&p.wtmpl)[lane];
+            __syncwarp();
+            if (lane == 0) dt_tmap_set(smem_u32(sm), m ? op.w1 : op.w0, op.K, op.N);
+            __syncwarp();
+            dt_tmap_publish(g + m, smem_u32(sm));
+        }
+        __syncwarp();
+        if (lane == 0) asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(state), "r"(2u) : "memory");
+    } else if (lane == 0) {
+        ok = dt_wait_count(state, 2u);
+    }
+    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    if (!ok) return false;
+    if (lane == 0)
+        for (int m = 0; m < op.nmat; ++m) dt_tmap_acquire(g + m);
+    __syncwarp();
+    have[j >> 5] |= 1u << (j & 31);
+    return true;
+}
+
+// ---- weight producer (warp 8) -------------------------------------------------
+// A piece of a row task: for each of its RG 128-row groups, two boxes of 64
+// rows x 128 bytes at k-bytes 128 pc (rows past N and bytes past K/4 read as
+// zero).  BitLinear: rows 128 q .. of the task's block; gated FFN: the group's
+// 64 gate rows, then the same 64 up rows.
 template <int RG>
 BITNET_DEVINL void dt_weight_producer(const DtProgram &p, unsigned char *smem)
 {
@@ -255,11 +331,11 @@ BITNET_DEVINL void dt_weight_producer(const DtProgram &p, unsigned char *smem)
     uint64_t *qfull = reinterpret_cast<uint64_t *>(smem + DT_BAR_QFULL);
     uint64_t *qempty = reinterpret_cast<uint64_t *>(smem + DT_BAR_QEMPTY);
     volatile int *qtask = reinterpret_cast<volatile int *>(smem + DT_QTASK);
-    const uint32_t ring = smem_u32(smem + DT_HDR);
-    const int j16 = lane & 7;
-    const int r0 = lane >> 3;
+    unsigned char *ring = smem + DT_HDR;
     uint32_t seq = 0;
     DtRing ring_pos;
+    uint32_t have[DT_MAX_OPS / 32] = {0u, 0u, 0u, 0u}; // ops whose maps this warp has acquired
+    uint32_t issued = 0, last_par = 0;               // slots with copies issued, and their last phase
     // the claim of the next task is issued one task ahead, so its latency overlaps the copies
     unsigned claim = 0;
     if (lane == 0) claim = atomicAdd(&p.counters[DT_CNT_TASK], 1u);
@@ -278,61 +354,44 @@ BITNET_DEVINL void dt_weight_producer(const DtProgram &p, unsigned char *smem)
         const DtTask tk = dt_decode(p, t);
         if (tk.quant) continue;
         const DtOp &op = p.ops[tk.op];
-        const int K = op.K, N = op.N;
-        const size_t rowb = (size_t)(K / 4);
+        const bool maps = dt_maps_acquire(p, tk.op, smem, have);
+        const CUtensorMap *g0 = p.wmaps + 2 * tk.op;
         const bool ffn = op.nmat == 2;
-        int rb[4];
-        const uint8_t *pb[4]; // source of this lane's chunk in row rb[q], k-offset 0
-        const int rstep = ffn ? 8 : 16;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const uint8_t *w;
-            if (ffn) {
-                rb[q] = tk.idx * (RG * DT_ROWS / 2) + r0 + 4 * (q & 1);
-                w = q >= 2 ? op.w1 : op.w0;
-            } else {
-                rb[q] = tk.idx * (RG * DT_ROWS) + r0 + 4 * q;
-                w = op.w0;
-            }
-            pb[q] = w + (size_t)rb[q] * rowb + (size_t)j16 * 16;
-        }
-        const size_t gstep = (size_t)rstep * rowb; // bytes between rows rb[q] + g * rstep, consecutive g
-        const bool all_rows = (ffn ? (tk.idx + 1) * (RG * DT_ROWS / 2) : (tk.idx + 1) * (RG * DT_ROWS)) <= N;
-        const int np = dt_pieces(K);
+        const int np = dt_pieces(op.K);
         for (int pc = 0; pc < np; ++pc, ring_pos.next(p.n_slots)) {
             const int s = ring_pos.slot;
             mbar_wait(&empty[s], ring_pos.par ^ 1u);
-            const int nkb = min(DT_KB, (K - pc * DT_KC) / 64);
-            const uint32_t dst0 = ring + (uint32_t)s * (uint32_t)p.slot_bytes + (uint32_t)(r0 * DT_PITCH + j16 * 16);
-            const size_t koff = (size_t)pc * (DT_KC / 4);
-            if (j16 < nkb) {
-                if (all_rows) {
+            if (lane == 0) {
+                if (maps) {
+                    unsigned char *dst = ring + (size_t)s * (size_t)p.slot_bytes;
+                    mbar_arrive_expect_tx(&full[s], RG * DT_WBYTES);
+                    const int x = pc * (DT_KC / 4);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const uint8_t *src = pb[q] + koff;
-#pragma unroll
-                        for (int g = 0; g < 8 * RG; ++g)
-                            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
-                                             dst0 + (uint32_t)((16 * g + 4 * q) * DT_PITCH)),
-                                         "l"(src + g * gstep)
-                                         : "memory");
-                    }
-                } else {
-#pragma unroll
-                    for (int g = 0; g < 8 * RG; ++g) {
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const bool ok = rb[q] + g * rstep < N;
-                            const uint8_t *src = ok ? pb[q] + koff + g * gstep : op.w0; // nothing read when !ok
-                            dt_cp16(dst0 + (uint32_t)((16 * g + 4 * q) * DT_PITCH), src, ok);
+                    for (int q = 0; q < RG; ++q) {
+                        unsigned char *d = dst + q * DT_WBYTES;
+                        if (ffn) {
+                            const int row = tk.idx * (RG * DT_ROWS / 2) + q * (DT_ROWS / 2);
+                            tma_load_2d(d, g0, x, row, &full[s]);
+                            tma_load_2d(d + DT_BOX_ROWS * DT_PITCH, g0 + 1, x, row, &full[s]);
+                        } else {
+                            const int row = tk.idx * (RG * DT_ROWS) + q * DT_ROWS;
+                            tma_load_2d(d, g0, x, row, &full[s]);
+                            tma_load_2d(d + DT_BOX_ROWS * DT_PITCH, g0, x, row + DT_BOX_ROWS, &full[s]);
                         }
                     }
+                } else {
+                    mbar_arrive(&full[s]); // maps unavailable (status set): keep the phases in step
                 }
+                issued |= 1u << s;
+                last_par = (last_par & ~(1u << s)) | (ring_pos.par << s);
             }
-            dt_cp_arrive(smem_u32(&full[s]));
         }
     }
-    asm volatile("cp.async.wait_all;" ::: "memory");
+    // every copy this warp issued has landed before the CTA can exit
+    if (lane == 0)
+        for (int s = 0; s < p.n_slots; ++s)
+            if (issued & (1u << s)) mbar_wait_drain(&full[s], (last_par >> s) & 1u);
+    __syncwarp();
 }
 
 // ---- activation producer (warp 9) -------------------------------------------
@@ -554,9 +613,12 @@ BITNET_DEVINL void dt_quant_row(const DtProgram &p, const DtOp &op, int m, unsig
 // tiles, fewer registers) the word is used as is for positions 0, 1 and
 // shifted by 4 for positions 2, 3: set j & 1 holds 4^(j & 1) * its sum.
 // One mma covers a pair of k-blocks (its two k halves) at one position j.
-// acc[r][j][tt][4]: row group r of the warp (rows 16 (w + 8 r) ..), set j,
-// token tile tt.  wrow: this lane's word in row group 0 (row group r is
-// r * 128 rows further).
+// acc[r][j][tt][4]: row group r of the warp, set j, token tile tt.  The
+// fragment's rows g and g + 8 are slot rows lo and hi of row group 0 (row
+// group r is 128 rows further): BitLinear 16 w + g and 16 w + g + 8, gated FFN
+// 8 w + g (gate) and 64 + 8 w + g (up).  Rows are 128 bytes with the 16-byte
+// chunks swizzled by (row & 7) = g, so k-block kb of a row is its chunk
+// kb ^ g; wlo / whi: this lane's word in chunk 0 of rows lo / hi, g16 = g << 4.
 template <int SC>
 BITNET_DEVINL uint32_t dt_code_bits(uint32_t w, uint32_t w4, int j)
 {
@@ -595,20 +657,24 @@ BITNET_DEVINL uint4 dt_ld_b(uint32_t addr)
     return b;
 }
 
+struct DtArow {
+    uint32_t lo, hi, g16;
+};
+
 template <int RG>
-BITNET_DEVINL void dt_ld_a(uint32_t (&lo)[RG], uint32_t (&hi)[RG], uint32_t wrow, int kb)
+BITNET_DEVINL void dt_ld_a(uint32_t (&lo)[RG], uint32_t (&hi)[RG], const DtArow &w, int kb)
 {
+    const uint32_t kx = ((uint32_t)kb << 4) ^ w.g16;
 #pragma unroll
     for (int r = 0; r < RG; ++r) {
-        const uint32_t a = wrow + (uint32_t)(r * DT_ROWS * DT_PITCH) + kb * 16;
-        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(lo[r]) : "r"(a));
-        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(hi[r]) : "r"(a + 8 * DT_PITCH));
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(lo[r]) : "r"(w.lo + (uint32_t)(r * DT_WBYTES) + kx));
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(hi[r]) : "r"(w.hi + (uint32_t)(r * DT_WBYTES) + kx));
     }
 }
 
 // A ragged piece (fewer than 8 k-blocks; an odd last block is paired with zeros).
 template <int TT, int SC, int RG>
-BITNET_DEVINL void dt_piece(int (&acc)[RG][SC][TT][4], uint32_t wrow, uint32_t xrow, int Mp, int nkb)
+BITNET_DEVINL void dt_piece(int (&acc)[RG][SC][TT][4], const DtArow &wrow, uint32_t xrow, int Mp, int nkb)
 {
 #pragma unroll
     for (int kp = 0; kp < DT_KB / 2; ++kp) {
@@ -637,7 +703,7 @@ BITNET_DEVINL void dt_piece(int (&acc)[RG][SC][TT][4], uint32_t wrow, uint32_t x
 // every activation fragment) is loaded before the first mma, so the
 // shared-memory latency is paid once per piece.
 template <int TT, int SC, int RG>
-BITNET_DEVINL void dt_piece_full(int (&acc)[RG][SC][TT][4], uint32_t wrow, uint32_t xrow, int Mp)
+BITNET_DEVINL void dt_piece_full(int (&acc)[RG][SC][TT][4], const DtArow &wrow, uint32_t xrow, int Mp)
 {
     uint32_t lo[DT_KB][RG], hi[DT_KB][RG];
 #pragma unroll
@@ -711,17 +777,21 @@ BITNET_DEVINL void dt_compute(const DtProgram &p, unsigned char *smem)
                         for (int c = 0; c < 4; ++c) acc[r][a][tt][c] = 0;
             const int K = op.K;
             const int np = dt_pieces(K);
-            const uint32_t wlane = (uint32_t)((warp * 16 + g) * DT_PITCH + t4 * 4);
+            const bool ffn = op.nmat == 2;
+            const uint32_t row_lo = ffn ? (uint32_t)(warp * 8 + g) : (uint32_t)(warp * 16 + g);
+            const uint32_t row_hi = row_lo + (ffn ? (uint32_t)DT_BOX_ROWS : 8u);
             const uint32_t xlane = (uint32_t)(RG * DT_WBYTES + g * 64 + t4 * 16);
             for (int pc = 0; pc < np; ++pc, ring_pos.next(p.n_slots)) {
                 const int s = ring_pos.slot;
                 mbar_wait(&full[s], ring_pos.par);
                 const uint32_t base = ring + (uint32_t)s * (uint32_t)p.slot_bytes;
                 const int nkb = min(DT_KB, (K - pc * DT_KC) >> 6);
+                const DtArow wr = {base + row_lo * DT_PITCH + t4 * 4, base + row_hi * DT_PITCH + t4 * 4,
+                                   (uint32_t)g << 4};
                 if (nkb == DT_KB)
-                    dt_piece_full<TT, SC, RG>(acc, base + wlane, base + xlane, Mp);
+                    dt_piece_full<TT, SC, RG>(acc, wr, base + xlane, Mp);
                 else
-                    dt_piece<TT, SC, RG>(acc, base + wlane, base + xlane, Mp, nkb);
+                    dt_piece<TT, SC, RG>(acc, wr, base + xlane, Mp, nkb);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&empty[s]);
             }
@@ -831,12 +901,12 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_decode_tasks(const __grid_con
 {
     extern __shared__ unsigned char dt_smem_raw[];
     unsigned char *smem =
-        reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(dt_smem_raw) + 127) & ~uintptr_t(127));
+        reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(dt_smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x;
     if (tid == 0) {
         uint64_t *bars = reinterpret_cast<uint64_t *>(smem);
         for (int i = 0; i < p.n_slots; ++i) {
-            mbar_init(&bars[DT_BAR_FULL / 8 + i], 64); // 32 weight lanes + 32 activation lanes (cp.async, noinc)
+            mbar_init(&bars[DT_BAR_FULL / 8 + i], 33); // weight producer (expect_tx) + 32 activation lanes (cp.async, noinc)
             mbar_init(&bars[DT_BAR_EMPTY / 8 + i], 8); // compute warps
         }
         for (int i = 0; i < DT_QUEUE; ++i) {
@@ -860,7 +930,7 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_decode_tasks(const __grid_con
         const unsigned prev = atomicAdd(&p.counters[DT_CNT_EXIT], 1u);
         if (prev == gridDim.x - 1) {
             __threadfence();
-            for (int i = 0; i < DT_CNT_OPS + 2 * p.n_ops; ++i) atomicExch(&p.counters[i], 0u);
+            for (int i = 0; i < DT_CNT_OPS + 3 * p.n_ops; ++i) atomicExch(&p.counters[i], 0u);
         }
     }
 }

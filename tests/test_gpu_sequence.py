@@ -45,7 +45,7 @@ def workspace(n_ops, m, k_max=I):
 
 
 def counters_zero(ws, n_ops):
-    return torch.count_nonzero(ws[:4 * (2 + 2 * n_ops)]) == 0
+    return torch.count_nonzero(ws[:4 * (2 + 3 * n_ops)]) == 0
 
 
 def run_seq(ops, m, ws=None):
@@ -285,7 +285,7 @@ def test_workspace_too_small_is_rejected():
     L = make_layer(800, m)
     ops = layer_ops(L)
     up = lambda v: (v + 255) // 256 * 256  # noqa: E731
-    need = up(4 * (2 + 2 * 4)) + sum(up(o.K * 8) + 512 for o in ops)  # the documented exact size, Mp = 8
+    need = up(4 * (2 + 3 * 4)) + up(256 * 4 + 128) + sum(up(o.K * 8) + 512 for o in ops)  # documented exact size
     assert need < tw.bitnet_sequence_workspace_size(4, m, I)
     tw.bitnet_decode_sequence(ops, m, torch.zeros(need, dtype=torch.uint8, device=DEV))  # exactly enough
     torch.cuda.synchronize()
