@@ -46,6 +46,9 @@ def test_pack_deterministic():
     (1, 256, "normal", "bf16"), (4, 256, "normal", "bf16"), (7, 320, "outliers", "bf16"),
     (64, 2560, "student_t_rows", "bf16"), (33, 6912, "outliers", "bf16"), (4096, 2560, "student_t_rows", "bf16"),
     (5, 2560, "normal", "f32"), (300, 6912, "normal", "f32"),
+    # the streaming kernel (M >= 256, rows of up to 32 KB in shared memory): ragged grids, the
+    # largest row it takes, and rows of a single 128-byte chunk per lane group
+    (257, 6912, "outliers", "bf16"), (600, 8192, "normal", "f32"), (1024, 64, "student_t_rows", "bf16"),
     # row held by 8 warps (fp32, K = 16384) and the two-pass kernel for rows longer than that
     (3, 16384, "normal", "f32"), (2, 65536, "outliers", "bf16"), (9, 65536, "normal", "f32"),
 ])
