@@ -369,9 +369,11 @@ bitnet_status_t bitnet_sequence_schedule(const bitnet_op_t *ops, int32_t n_ops, 
  * to this call: it is the decode-step execution of the BitLinear layers that
  * the page's model stacks (page: "Architecture").
  *
- * Execution: every op is cut into tasks -- one quantisation task per token
- * (absmax, after the optional RMS normalisation) and one task per 128 packed
- * weight rows (64 output rows of a gated FFN) over all of K -- and the CTAs of
+ * Execution: every op is cut into tasks -- quantisation tasks (absmax, after
+ * the optional RMS normalisation: one per token for M <= 8, else one per 8
+ * tokens with a warp per token) and one
+ * task per 128 packed weight rows (256 when M <= 8; half of them output rows
+ * of a gated FFN) over all of K -- and the CTAs of
  * the launch (one per SM) claim tasks in a fixed order through a counter in
  * the workspace.  A task waits only for the tasks it depends on: an op's
  * weight rows for its quantisation tasks, a quantisation task for the rows of
@@ -406,7 +408,8 @@ bitnet_status_t bitnet_decode_sequence(const bitnet_op_t *ops, int32_t n_ops, in
 /*
  * Host-only: the task order bitnet_decode_sequence would launch for `ctas`
  * CTAs (no device is touched).  The 2 * n_ops task groups -- per op, its
- * quantisation tasks (kind 0, M tasks) and its weight-row tasks (kind 1) --
+ * quantisation tasks (kind 0: M tasks for M <= 8, else ceil(M / 8)) and its weight-row
+ * tasks (kind 1) --
  * in the order the CTAs claim them; for group k:
  *   group_op[k]     index into ops
  *   group_kind[k]   0 = quantisation, 1 = weight rows

@@ -674,7 +674,7 @@ bitnet_status_t forward(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_
 }
 
 // ---- decode sequences: one persistent launch for many ops -----------------
-constexpr int64_t kSeqMaxK = 8192; // a quant task holds a row of x in 256 threads' registers
+constexpr int64_t kSeqMaxK = 8192; // the exact sum of squares and the x_q fragment layout are sized for this
 
 struct ByteRange {
     uintptr_t lo, hi;
@@ -798,6 +798,9 @@ bitnet_status_t seq_schedule(const bitnet_op_t *ops, int n, int64_t M, int32_t *
 inline int seq_mp(int64_t M) { return M <= 8 ? 8 : M <= 16 ? 16 : M <= 32 ? 32 : 64; }
 // Row groups per compute warp: two at one token tile (each activation fragment feeds two
 // weight fragments, halving the activation loads from shared memory), else one.
+// quantisation tasks of an op: one per token for M <= 8 (on all compute warps),
+// else one per 8 tokens (a compute warp per token)
+inline int seq_qtasks(int64_t M) { return (int)(M <= 8 ? M : (M + 7) / 8); }
 inline int seq_rg(int64_t M) { return M <= 8 ? 2 : 1; }
 inline int seq_rtasks(const bitnet_op_t &o, int64_t M)
 {
@@ -855,7 +858,7 @@ bitnet_status_t seq_groups(const bitnet_op_t *ops, int n, int64_t M, ByteRange e
 // simulation on `ctas` CTAs: repeatedly take, among the groups whose
 // predecessors are already placed, the one whose predecessors finish first
 // (ties: execution order), and give its tasks to the CTAs that free up first.
-// Durations are estimates (a quant task ~1 us; a row task its packed weights at
+// Durations are estimates (a quant task 1.5 us for one token, 3 us for 8; a row task its packed weights at
 // ~40 GB/s per SM).  CTAs claim tasks in this order, so a dependent group is
 // placed after the work that will be running while its producer finishes.
 std::vector<int> seq_group_order(const bitnet_op_t *ops, int n, int64_t M, const SeqGroups &G, int ctas)
@@ -864,8 +867,8 @@ std::vector<int> seq_group_order(const bitnet_op_t *ops, int n, int64_t M, const
     std::vector<double> finish(ng, 0.0), dur(ng, 0.0);
     std::vector<int> count(ng, 0), left(ng, 0), order;
     for (int j = 0; j < n; ++j) {
-        count[2 * j] = (int)M;
-        dur[2 * j] = 1.0;
+        count[2 * j] = seq_qtasks(M);
+        dur[2 * j] = M <= 8 ? 1.5 : 3.0;
         count[2 * j + 1] = seq_rtasks(ops[j], M);
         dur[2 * j + 1] = (double)(DT_ROWS * seq_rg(M)) * (double)(ops[j].K / 4) / 40e3;
     }
@@ -981,7 +984,7 @@ bitnet_status_t seq_build(DtProgram &p, const bitnet_op_t *ops, const int32_t *u
     for (int v : order) {
         const int j = v / 2;
         const bool quant = v % 2 == 0;
-        const int cnt = quant ? (int)M : p.ops[j].rtasks;
+        const int cnt = quant ? seq_qtasks(M) : p.ops[j].rtasks;
         if (ns >= DT_MAX_SEGS) return BITNET_ERR_UNSUPPORTED_SHAPE;
         p.segs[ns].start = t;
         p.segs[ns].op = (uint16_t)j;
@@ -1327,7 +1330,7 @@ bitnet_status_t bitnet_sequence_tasks(const bitnet_op_t *ops, int32_t n_ops, int
         const int v = gorder[k], j = v / 2;
         group_op[k] = order[j];
         group_kind[k] = v % 2;
-        group_tasks[k] = v % 2 ? p.ops[j].rtasks : (int32_t)M;
+        group_tasks[k] = v % 2 ? p.ops[j].rtasks : (int32_t)seq_qtasks(M);
         dep_count[k] = (int32_t)G.preds[v].size();
         for (int d = 0; d < DT_MAX_DEPS + 1; ++d)
             deps[k * (DT_MAX_DEPS + 1) + d] = d < (int)G.preds[v].size() ? pos[G.preds[v][d]] : -1;

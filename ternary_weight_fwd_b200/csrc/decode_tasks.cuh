@@ -10,23 +10,25 @@
 // Work is cut into tasks, claimed in a fixed global order by the CTAs through
 // one atomic counter (dynamic scheduling: a CTA that finishes early takes the
 // next task):
-//   * quant task (op j, token m): per-token absmax quantisation of row m of the
-//     op's x (optionally RMS-normalised first), written to the workspace as
-//     int8 in the fragment layout [K/64][Mp][64] plus the scale and row sum.
-//     All 256 compute threads share the row (in registers: one pass over x).
-//   * row task (op j, block b): 128 rows of the packed weights (a BitLinear:
-//     output rows 128b ..; a gated FFN: 64 gate rows and the same 64 up rows),
-//     full K, against all tokens.  Compute warp w owns a 16-row group: rows g
-//     and g + 8 of the mma fragment are two output rows (BitLinear) or the gate
-//     and the up row of one output (FFN), so each lane ends with complete sums
-//     and the epilogue needs no exchange between warps or CTAs.
+//   * quant task (op j, token m for M <= 8, else tokens 8 i .. 8 i + 7):
+//     per-token absmax quantisation of the op's x (optionally RMS-normalised
+//     first) on all compute warps (one token), or one compute warp per token,
+//     written to the workspace as int8 in the fragment layout [K/64][Mp][64]
+//     plus the scale and row sum.
+//   * row task (op j, block b): 128 RG rows of the packed weights (RG = 2 for
+//     M <= 8, else 1; a BitLinear: output rows 128 RG b ..; a gated FFN: 64 RG
+//     gate rows and the same up rows), full K, against all tokens.  Compute
+//     warp w owns RG 16-row groups: rows g and g + 8 of the mma fragment are
+//     two output rows (BitLinear) or the gate and the up row of one output
+//     (FFN), so each lane ends with complete sums and the epilogue needs no
+//     exchange between warps or CTAs.
 // Tasks wait only on earlier tasks of the order (an op's rows on its quant
 // tasks; a quant task on the rows of the op that wrote its x; outputs on the
 // readers / writers of the same bytes before them), and every task a CTA
 // holds was claimed by a running CTA, so progress does not depend on how many
 // CTAs are resident at once.
 //
-// Roles in a CTA (320 threads):
+// Roles in a CTA (352 threads):
 //   warp 8  weight producer: claims tasks, writes them to a 4-entry queue in
 //           shared memory, streams each row task's packed weights into a ring of
 //           pieces (128 rows x 512 k: two TMA boxes of 64 rows x 128 bytes, with
@@ -129,9 +131,11 @@ constexpr int DT_INFO = 1024;                         // per queue entry: s[64] 
 constexpr int DT_INFO_S = 0, DT_INFO_RS = 4 * DT_MAX_M, DT_INFO_G = 8 * DT_MAX_M;
 constexpr int DT_INFO_BYTES = 8 * DT_MAX_M + 16;
 constexpr int DT_MAPS = 3584;                         // two 128-byte tensor maps being made
-constexpr int DT_HDR = 4096; // the piece ring starts here
+constexpr int DT_DIG = 3840;                          // [8 warps][20] long accumulators (quant tasks)
+constexpr int DT_HDR = 5120; // the piece ring starts here
 static_assert(DT_INFO + DT_QUEUE * DT_INFO_BYTES <= DT_MAPS, "shared header");
-static_assert(DT_MAPS + 256 <= DT_HDR && DT_MAPS % 128 == 0, "shared header");
+static_assert(DT_MAPS + 256 <= DT_DIG && DT_MAPS % 128 == 0, "shared header");
+static_assert(DT_DIG + 8 * 8 * SS_LONG_DIGITS <= DT_HDR && DT_DIG % 8 == 0, "shared header");
 static_assert(DT_QTASK + 4 * DT_QUEUE <= DT_RED, "shared header");
 static_assert(DT_HDR % 1024 == 0 && DT_WBYTES % 1024 == 0, "ring alignment (128-byte swizzle)");
 
@@ -184,14 +188,17 @@ BITNET_DEVINL bool dt_wait_count(const unsigned *c, unsigned target)
     }
 }
 
+// named barrier of the eight compute warps
+BITNET_DEVINL void dt_bar_compute() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
 BITNET_DEVINL unsigned *dt_qdone(const DtProgram &p, int j) { return p.counters + DT_CNT_OPS + 2 * j; }
 BITNET_DEVINL unsigned *dt_rdone(const DtProgram &p, int j) { return p.counters + DT_CNT_OPS + 2 * j + 1; }
 
 // Completion targets: one count per quant task (token) and per row task.
-BITNET_DEVINL unsigned dt_qtarget(const DtProgram &p, int) { return (unsigned)p.M; }
+// quant tasks of an op: one per token for M <= 8, else one per 8 tokens (a warp per token)
+BITNET_DEVINL unsigned dt_qtarget(const DtProgram &p, int) { return (unsigned)(p.M <= 8 ? p.M : (p.M + 7) / 8); }
 BITNET_DEVINL unsigned dt_rtarget(const DtProgram &p, int j) { return (unsigned)p.ops[j].rtasks; }
 
-BITNET_DEVINL void dt_bar_compute() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 // 16-byte asynchronous copy; zero-fills the destination when !valid (nothing is read).
 BITNET_DEVINL void dt_cp16(uint32_t dst, const void *src, bool valid)
@@ -465,8 +472,184 @@ BITNET_DEVINL void dt_act_producer(const DtProgram &p, unsigned char *smem)
     asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
-// ---- quant task (compute warps): token m of op j -----------------------------
-// Thread t holds 16-byte chunks c = t + 256 i of the row (x read once, from L2).
+// ---- quant task (compute warps): tokens 8 i .. 8 i + 7 of op j, one per warp --
+// Warp w quantises token m = 8 i + w (m < M).  The row is read from L2 in
+// passes, so any K <= 8192 fits and no barrier between warps is needed: the
+// absmax pass and the quantise pass; with the RMS normalisation first, a pass
+// for the exponent of the row maximum and one for the exact sum of squares
+// (128-bit window, or the warp's long accumulator in shared memory for a row
+// of very wide range), and the normalised values are recomputed in the later
+// passes.  x_q goes to the fragment layout: byte k of token m at
+// ((k / 64) * Mp + m) * 64 + k % 64.
+template <bool XF32>
+BITNET_DEVINL void dt_chunk_vals(const uint4 q, float (&f)[XF32 ? 4 : 8])
+{
+    if constexpr (XF32) {
+        f[0] = __uint_as_float(q.x), f[1] = __uint_as_float(q.y), f[2] = __uint_as_float(q.z);
+        f[3] = __uint_as_float(q.w);
+    } else {
+        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            f[2 * h] = bf16_bits_lo(w[h]);
+            f[2 * h + 1] = bf16_bits_hi(w[h]);
+        }
+    }
+}
+
+// A batch of QB chunks c0 + 32 b of the row (b < QB, c < nch), loaded before any
+// is used (one L2 round trip per batch), as fp32 values; normalised when g is
+// set: fl(fl(x r) g).  Chunks past the row are left zero.
+template <bool XF32, bool NORM, int QB>
+BITNET_DEVINL void dt_batch(const char *row, int c0, int nch, const float *g, float r,
+                            float (&f)[QB][XF32 ? 4 : 8])
+{
+    constexpr int EPC = XF32 ? 4 : 8;
+    uint4 q[QB];
+    float4 gv[NORM ? QB * (EPC / 4) : 1];
+#pragma unroll
+    for (int b = 0; b < QB; ++b) {
+        const int c = c0 + 32 * b;
+        q[b] = make_uint4(0u, 0u, 0u, 0u);
+        if (c < nch) {
+            q[b] = dt_ld_cg16(row + 16 * (size_t)c);
+            if constexpr (NORM) {
+#pragma unroll
+                for (int u = 0; u < EPC / 4; ++u)
+                    gv[b * (EPC / 4) + u] = __ldg(reinterpret_cast<const float4 *>(g) + (EPC / 4) * c + u);
+            }
+        }
+    }
+#pragma unroll
+    for (int b = 0; b < QB; ++b) {
+        dt_chunk_vals<XF32>(q[b], f[b]);
+        if constexpr (NORM) {
+            if (c0 + 32 * b < nch) {
+#pragma unroll
+                for (int h = 0; h < EPC; ++h) {
+                    const float4 gq = gv[b * (EPC / 4) + h / 4];
+                    const float gh = (h & 3) == 0 ? gq.x : (h & 3) == 1 ? gq.y : (h & 3) == 2 ? gq.z : gq.w;
+                    f[b][h] = __fmul_rn(__fmul_rn(f[b][h], r), gh);
+                }
+            }
+        }
+    }
+}
+
+// The absmax pass and the quantise pass over the (normalised) row of token m.
+template <bool XF32, bool NORM, int QB>
+BITNET_DEVINL void dt_quant_pass(const DtProgram &p, const DtOp &op, int m, const char *row, int nch, float r)
+{
+    const int lane = threadIdx.x & 31;
+    constexpr int EPC = XF32 ? 4 : 8;
+    float mx = 0.0f;
+    for (int c0 = lane; c0 < nch; c0 += 32 * QB) {
+        float fr[QB][EPC];
+        dt_batch<XF32, NORM, QB>(row, c0, nch, op.norm_g, r, fr);
+#pragma unroll
+        for (int b = 0; b < QB; ++b)
+#pragma unroll
+            for (int h = 0; h < EPC; ++h) mx = fmaxf(mx, fabsf(fr[b][h]));
+    }
+    mx = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(mx)));
+    const float sc = quant_scale(mx);
+    int rsum = 0;
+    int8_t *xq = op.xq;
+    for (int c0 = lane; c0 < nch; c0 += 32 * QB) {
+        float fr[QB][EPC];
+        dt_batch<XF32, NORM, QB>(row, c0, nch, op.norm_g, r, fr);
+#pragma unroll
+        for (int b = 0; b < QB; ++b) {
+            const int c = c0 + 32 * b;
+            if (c < nch) {
+                int q[EPC];
+#pragma unroll
+                for (int h = 0; h < EPC; ++h) {
+                    q[h] = quant_one(fr[b][h], sc);
+                    rsum += q[h];
+                }
+                const int k0 = c * EPC;
+                int8_t *dst = xq + ((size_t)(k0 >> 6) * p.Mp + m) * 64 + (k0 & 63);
+                if constexpr (XF32) {
+                    *reinterpret_cast<uint32_t *>(dst) = pack4_s8(q[0], q[1], q[2], q[3]);
+                } else {
+                    *reinterpret_cast<uint2 *>(dst) =
+                        make_uint2(pack4_s8(q[0], q[1], q[2], q[3]), pack4_s8(q[4], q[5], q[6], q[7]));
+                }
+            }
+        }
+    }
+    rsum = warp_sum(rsum);
+    if (lane == 0) {
+        op.s[m] = sc;
+        op.rs[m] = rsum;
+    }
+}
+
+template <bool XF32, int SHRINK>
+BITNET_DEVINL void dt_quant_warp(const DtProgram &p, const DtOp &op, int m, unsigned char *smem)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr int EPC = XF32 ? 4 : 8; // elements per 16-byte chunk
+    // chunks per lane per batch: 32 values in the absmax and quantise passes, 16 in the sum-of-squares
+    // and normalised ones; halved (SHRINK = 2) where the contraction of many token tiles holds more registers
+    constexpr int QB = (XF32 ? 8 : 4) / SHRINK;
+    constexpr int QS = (XF32 ? 4 : 2) / SHRINK;
+    const int K = op.K, nch = K / EPC;
+    const char *row = static_cast<const char *>(op.x) + (size_t)m * K * (XF32 ? 4 : 2);
+    float r = 1.0f;
+    if (op.norm_g) {
+        // RMS normalisation: exact sum of squares (rounded once), r in binary64 -> binary32
+        float xm = 0.0f;
+        for (int c0 = lane; c0 < nch; c0 += 32 * QS) {
+            float f[QS][EPC];
+            dt_batch<XF32, false, QS>(row, c0, nch, nullptr, 1.0f, f);
+#pragma unroll
+            for (int b = 0; b < QB; ++b)
+#pragma unroll
+                for (int h = 0; h < EPC; ++h) xm = fmaxf(xm, fabsf(f[b][h]));
+        }
+        xm = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(xm)));
+        const uint32_t E = ss_exponent(xm); // the largest exponent of the row
+        SsWindow acc;
+        if (E != 0)
+            for (int c0 = lane; c0 < nch; c0 += 32 * QS) {
+                float f[QS][EPC];
+                dt_batch<XF32, false, QS>(row, c0, nch, nullptr, 1.0f, f);
+#pragma unroll
+                for (int b = 0; b < QS; ++b)
+#pragma unroll
+                    for (int h = 0; h < EPC; ++h) ss_window_add(acc, f[b][h], E);
+            }
+        ss_warp_sum(acc.lo, acc.hi);
+        double ss;
+        if (!__all_sync(0xffffffffu, acc.fits)) { // warp-uniform
+            unsigned long long *dig = reinterpret_cast<unsigned long long *>(smem + DT_DIG) + warp * SS_LONG_DIGITS;
+            if (lane < SS_LONG_DIGITS) dig[lane] = 0ull;
+            __syncwarp();
+            for (int c0 = lane; c0 < nch; c0 += 32 * QS) {
+                float f[QS][EPC];
+                dt_batch<XF32, false, QS>(row, c0, nch, nullptr, 1.0f, f);
+#pragma unroll
+                for (int b = 0; b < QS; ++b)
+#pragma unroll
+                    for (int h = 0; h < EPC; ++h) ss_long_add(dig, f[b][h]);
+            }
+            __syncwarp();
+            ss = ss_long_round(dig);
+        } else {
+            ss = E ? ss_window_round(acc.lo, acc.hi, E) : 0.0;
+        }
+        r = __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(__ddiv_rn(ss, (double)K), (double)op.norm_eps))));
+    }
+    if (op.norm_g) dt_quant_pass<XF32, true, QS>(p, op, m, row, nch, r); // + the weights: smaller batches
+    else dt_quant_pass<XF32, false, QB>(p, op, m, row, nch, r);
+}
+
+// ---- quant task of one token on all compute warps (M <= 8) --------------------
+// Thread t holds 16-byte chunks c = t + 256 i of the row (x read once, from L2,
+// in one round trip): the shortest latency for a single row, which is what a
+// decode step of few tokens waits on.
 template <bool XF32>
 BITNET_DEVINL void dt_quant_row(const DtProgram &p, const DtOp &op, int m, unsigned char *smem)
 {
@@ -755,14 +938,28 @@ BITNET_DEVINL void dt_compute(const DtProgram &p, unsigned char *smem)
         const DtTask tk = dt_decode(p, t);
         const DtOp &op = p.ops[tk.op];
         if (tk.quant) {
-            // the op that wrote x (read after write) is complete
-            if (tid == 0)
-                for (int d = 0; d < op.nq; ++d) dt_wait_count(dt_rdone(p, op.deps[d]), dt_rtarget(p, op.deps[d]));
-            dt_bar_compute();
-            if (op.xf32) dt_quant_row<true>(p, op, tk.idx, smem);
-            else dt_quant_row<false>(p, op, tk.idx, smem);
-            // (dt_quant_row ends with a barrier after every x_q store; thread 0 stored s and the
-            // row sum after it): the completion warp counts the task once every warp arrived
+            if constexpr (TT == 1) {
+                // one token on all compute warps; the op that wrote x (read after write) is complete
+                if (tid == 0)
+                    for (int d = 0; d < op.nq; ++d)
+                        dt_wait_count(dt_rdone(p, op.deps[d]), dt_rtarget(p, op.deps[d]));
+                dt_bar_compute();
+                if (op.xf32) dt_quant_row<true>(p, op, tk.idx, smem);
+                else dt_quant_row<false>(p, op, tk.idx, smem);
+            } else {
+                const int m = tk.idx * 8 + warp;
+                if (m < M) {
+                    // the op that wrote x (read after write) is complete
+                    if (lane == 0)
+                        for (int d = 0; d < op.nq; ++d)
+                            dt_wait_count(dt_rdone(p, op.deps[d]), dt_rtarget(p, op.deps[d]));
+                    __syncwarp();
+                    if (op.xf32) dt_quant_warp<true, TT >= 8 ? 2 : 1>(p, op, m, smem);
+                    else dt_quant_warp<false, TT >= 8 ? 2 : 1>(p, op, m, smem);
+                }
+            }
+            // every lane's stores precede lane 0's arrival; the completion warp counts the
+            // task once every warp arrived
             __syncwarp();
             if (lane == 0) mbar_arrive(&cdone[e]);
         } else {

@@ -325,9 +325,9 @@ def ov(a, b):
 
 
 def check_tasks(ops, m, groups):
-    """The task groups a launch claims, in order: every op's quant group (M tasks) and rows
-    group; dependencies point backwards, include every ordering the byte ranges require
-    (transitively), and none is implied by another."""
+    """The task groups a launch claims, in order: every op's quant group (a task per token for
+    M <= 8, else per 8 tokens) and rows group; dependencies point backwards, include every
+    ordering the byte ranges require (transitively), and none is implied by another."""
     n = len(ops)
     assert len(groups) == 2 * n
     pos = {}
@@ -336,7 +336,7 @@ def check_tasks(ops, m, groups):
         key = (gr["op"], gr["kind"])
         assert key not in pos
         pos[key] = k
-        want = m if gr["kind"] == "quant" else -(-o.N // rows_per_task(o, m))
+        want = (m if m <= 8 else -(-m // 8)) if gr["kind"] == "quant" else -(-o.N // rows_per_task(o, m))
         assert gr["tasks"] == want
         assert all(0 <= d < k for d in gr["deps"])
         assert len(gr["deps"]) <= (9 if gr["kind"] == "rows" else 8)
