@@ -330,7 +330,7 @@ typedef struct bitnet_op {
  * weights (made by the kernel), then per op the quantised activations
  * ([K/64][Mp][64] int8, Mp = M rounded up to 8, 16, 32 or 64), scales and row
  * sums.  A list of n ops needs exactly
- *   up256(4 * (2 + 3n)) + up256(256n + 128) + sum over ops of (up256(K * Mp) + 512)
+ *   up256(4 * (2 + 2n)) + up256(256n + 128) + sum over ops of (up256(K * Mp) + 512)
  * bytes (up256 = rounded up to a multiple of 256); this returns that for
  * n_ops ops of K = K_max.  0 for arguments out of range.
  */
@@ -361,7 +361,9 @@ bitnet_status_t bitnet_sequence_schedule(const bitnet_op_t *ops, int32_t n_ops, 
 /*
  * Run ops[0..n_ops) -- every one a decode-size BitLinear or gated FFN over
  * the same M tokens, optionally RMS-normalising its input first -- in ONE
- * persistent kernel launch.  The results are bit-identical to calling
+ * persistent kernel launch (preceded by a one-wave kernel that writes the
+ * weights' TMA tensor maps into the workspace: two launches per call).  The
+ * results are bit-identical to calling
  * bitnet_linear / bitnet_ffn_gate_up (bitnet_linear_norm /
  * bitnet_ffn_gate_up_norm when norm_g is set) for each op in order on
  * `stream`: an op whose x is an earlier op's y reads that y, and every output

@@ -908,10 +908,10 @@ std::vector<int> seq_group_order(const bitnet_op_t *ops, int n, int64_t M, const
     return order;
 }
 
-// Workspace: counters (per op: quant tasks done, row tasks done, state of its
-// tensor maps), the ops' weight tensor maps [n][2] x 128 bytes, then per op
-// x_q [K/64][Mp][64], s [Mp], row sums [Mp].
-inline size_t seq_counter_bytes(int n) { return align_up(4 * (size_t)(DT_CNT_OPS + 3 * n), 256); }
+// Workspace: counters (per op: quant tasks done, row tasks done), the ops'
+// weight tensor maps [n][2] x 128 bytes, then per op x_q [K/64][Mp][64],
+// s [Mp], row sums [Mp].
+inline size_t seq_counter_bytes(int n) { return align_up(4 * (size_t)(DT_CNT_OPS + 2 * n), 256); }
 inline size_t seq_map_bytes(int n) { return align_up((size_t)n * 2 * sizeof(CUtensorMap) + 128, 256); } // + alignment
 inline size_t seq_op_ws_bytes(int64_t K, int Mp) { return align_up((size_t)K * Mp, 256) + 512; }
 
@@ -1011,7 +1011,9 @@ cudaError_t seq_launch_t(const DtProgram &p, int ctas, cudaStream_t stream, int 
     cudaError_t e = ensure_smem(k_decode_tasks<TT, RG>, kSmemLimit, smem_done, dev);
     if (e != cudaSuccess) return e;
     const size_t smem = 1024 + DT_HDR + (size_t)p.n_slots * p.slot_bytes; // + alignment to 1024 bytes
-    g_launches.fetch_add(1, std::memory_order_relaxed);
+    // the weights' tensor maps, then the sequence
+    g_launches.fetch_add(2, std::memory_order_relaxed);
+    k_decode_maps<<<p.n_ops, 32, 0, stream>>>(p);
     k_decode_tasks<TT, RG><<<ctas, DT_THREADS, smem, stream>>>(p);
     return cudaGetLastError();
 }

@@ -33,9 +33,10 @@
 //           shared memory, streams each row task's packed weights into a ring of
 //           pieces (128 rows x 512 k: two TMA boxes of 64 rows x 128 bytes, with
 //           the 128-byte swizzle so the fragment loads hit 32 distinct banks).
-//           The tensor maps are made on the device, once per op and launch, from
-//           a template map (the matrix's address, extent and row pitch put in
-//           with tensormap.replace).  Weights never wait for any other task.
+//           The tensor maps are made on the device by a small kernel launched
+//           before this one, from a template map (the matrix's address, extent
+//           and row pitch put in with tensormap.replace).  Weights never wait
+//           for any other task.
 //   warp 9  activation producer: for a row task, waits for its dependencies,
 //           copies the per-token scales and row sums and the gammas, and streams
 //           the matching x_q chunk ([8][Mp][64] bytes) next to each weight piece
@@ -79,8 +80,7 @@ template <bool XF32> __host__ __device__ constexpr int dt_quant_ch() { return XF
 // counters (uint32) at the start of the workspace
 constexpr int DT_CNT_TASK = 0;  // next task to claim
 constexpr int DT_CNT_EXIT = 1;  // CTAs finished
-constexpr int DT_CNT_OPS = 2;   // then per op: quant tasks done, row tasks done; then per op the
-                                // state of its tensor maps (0 none, 1 being made, 2 ready)
+constexpr int DT_CNT_OPS = 2;   // then per op: quant tasks done, row tasks done
 
 constexpr uint16_t DT_DEP_QUANT = 0x8000u; // dependency on an op's quant tasks (else its row tasks)
 
@@ -113,7 +113,7 @@ struct DtProgram {
     CUtensorMap wtmpl;   // template of the weight maps: uint8 [N][K/4], box 64 rows x 128 bytes, 128-byte swizzle
     int n_ops, n_segs, n_tasks, M, Mp, n_slots, slot_bytes;
     unsigned *counters;
-    CUtensorMap *wmaps;  // workspace: [n_ops][2] maps of w0, w1 (made by the first CTA to need them)
+    CUtensorMap *wmaps;  // workspace: [n_ops][2] maps of w0, w1 (made by k_decode_maps)
     DtOp ops[DT_MAX_OPS];
     DtSeg segs[DT_MAX_SEGS];
 };
@@ -130,11 +130,9 @@ constexpr int DT_RED = 512;                           // quant-task reductions (
 constexpr int DT_INFO = 1024;                         // per queue entry: s[64] fp32, rs[64] int32, gamma0, gamma1
 constexpr int DT_INFO_S = 0, DT_INFO_RS = 4 * DT_MAX_M, DT_INFO_G = 8 * DT_MAX_M;
 constexpr int DT_INFO_BYTES = 8 * DT_MAX_M + 16;
-constexpr int DT_MAPS = 3584;                         // two 128-byte tensor maps being made
-constexpr int DT_DIG = 3840;                          // [8 warps][20] long accumulators (quant tasks)
+constexpr int DT_DIG = 3584;                          // [8 warps][20] long accumulators (quant tasks)
 constexpr int DT_HDR = 5120; // the piece ring starts here
-static_assert(DT_INFO + DT_QUEUE * DT_INFO_BYTES <= DT_MAPS, "shared header");
-static_assert(DT_MAPS + 256 <= DT_DIG && DT_MAPS % 128 == 0, "shared header");
+static_assert(DT_INFO + DT_QUEUE * DT_INFO_BYTES <= DT_DIG, "shared header");
 static_assert(DT_DIG + 8 * 8 * SS_LONG_DIGITS <= DT_HDR && DT_DIG % 8 == 0, "shared header");
 static_assert(DT_QTASK + 4 * DT_QUEUE <= DT_RED, "shared header");
 static_assert(DT_HDR % 1024 == 0 && DT_WBYTES % 1024 == 0, "ring alignment (128-byte swizzle)");
@@ -256,11 +254,11 @@ struct DtRing {
 };
 
 // ---- tensor maps of the weights -------------------------------------------
-// Made on the device from the template: the first warp to need op j's maps
-// (CAS 0 -> 1 on its state) writes them to the workspace and publishes them
-// (state 2, release); every weight producer acquires them before its first
-// copy with them.  The maker is a running CTA with no other wait in between,
-// so a warp that waits for state 2 always sees it.
+// Made on the device, by a small kernel launched just before the sequence
+// kernel (k_decode_maps, one CTA per op): the template with the matrix's
+// address, extent and row pitch put in, published to the workspace with a
+// release fence for the tensor-map proxy.  The sequence kernel's weight
+// producer acquires an op's maps once before its first copy with them.
 BITNET_DEVINL void dt_tmap_set(uint32_t sm, const void *w, int K, int N)
 {
     asm volatile("tensormap.replace.tile.global_address.shared::cta.b1024.b64 [%0], %1;" ::"r"(sm), "l"(w)
@@ -274,54 +272,31 @@ BITNET_DEVINL void dt_tmap_set(uint32_t sm, const void *w, int K, int N)
                  : "memory");
 }
 
-// Whole warp: the 128-byte map at sm to global g, with a release fence for the tensor-map proxy.
-BITNET_DEVINL void dt_tmap_publish(CUtensorMap *g, uint32_t sm)
+__global__ void __launch_bounds__(32) k_decode_maps(const __grid_constant__ DtProgram p)
 {
-    asm volatile("tensormap.cp_fenceproxy.global.shared::cta.tensormap::generic.release.gpu.sync.aligned [%0], [%1], "
-                 "128;" ::"l"(g),
-                 "r"(sm)
-                 : "memory");
-}
-
-BITNET_DEVINL void dt_tmap_acquire(const CUtensorMap *g)
-{
-    asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(g) : "memory");
-}
-
-// Whole warp; lane 0 may then copy with op j's maps.  false: the wait for
-// another warp's maps ran out (status set).
-BITNET_DEVINL bool dt_maps_acquire(const DtProgram &p, int j, unsigned char *smem, uint32_t (&have)[DT_MAX_OPS / 32])
-{
-    const int lane = threadIdx.x & 31;
-    if (have[j >> 5] & (1u << (j & 31))) return true;
+    __shared__ alignas(128) unsigned char sm[2][128];
+    const int j = blockIdx.x, lane = threadIdx.x;
+    if (j >= p.n_ops) return;
     const DtOp &op = p.ops[j];
-    unsigned *state = &p.counters[DT_CNT_OPS + 2 * p.n_ops + j];
-    CUtensorMap *g = p.wmaps + 2 * j;
-    unsigned st = 0;
-    if (lane == 0) st = atomicCAS(state, 0u, 1u);
-    st = __shfl_sync(0xffffffffu, st, 0);
-    bool ok = true;
-    if (st == 0) {
-        for (int m = 0; m < op.nmat; ++m) {
-            unsigned char *sm = smem + DT_MAPS + 128 * m;
-            if (lane < 8) reinterpret_cast<uint4 *>(sm)[lane] = reinterpret_cast<const uint4 *>(&p.wtmpl)[lane];
-            __syncwarp();
-            if (lane == 0) dt_tmap_set(smem_u32(sm), m ? op.w1 : op.w0, op.K, op.N);
-            __syncwarp();
-            dt_tmap_publish(g + m, smem_u32(sm));
-        }
+    for (int m = 0; m < op.nmat; ++m) {
+        if (lane < 8) reinterpret_cast<uint4 *>(sm[m])[lane] = reinterpret_cast<const uint4 *>(&p.wtmpl)[lane];
         __syncwarp();
-        if (lane == 0) asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(state), "r"(2u) : "memory");
-    } else if (lane == 0) {
-        ok = dt_wait_count(state, 2u);
+        if (lane == 0) dt_tmap_set(smem_u32(sm[m]), m ? op.w1 : op.w0, op.K, op.N);
+        __syncwarp();
+        asm volatile("tensormap.cp_fenceproxy.global.shared::cta.tensormap::generic.release.gpu.sync.aligned [%0], "
+                     "[%1], 128;" ::"l"(p.wmaps + 2 * j + m),
+                     "r"(smem_u32(sm[m]))
+                     : "memory");
     }
-    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-    if (!ok) return false;
-    if (lane == 0)
-        for (int m = 0; m < op.nmat; ++m) dt_tmap_acquire(g + m);
-    __syncwarp();
+}
+
+// Lane 0: acquire op j's maps (once per op and CTA).
+BITNET_DEVINL void dt_maps_acquire(const DtProgram &p, int j, uint32_t (&have)[DT_MAX_OPS / 32])
+{
+    if (have[j >> 5] & (1u << (j & 31))) return;
+    for (int m = 0; m < p.ops[j].nmat; ++m)
+        asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(p.wmaps + 2 * j + m) : "memory");
     have[j >> 5] |= 1u << (j & 31);
-    return true;
 }
 
 // ---- weight producer (warp 8) -------------------------------------------------
@@ -361,7 +336,7 @@ BITNET_DEVINL void dt_weight_producer(const DtProgram &p, unsigned char *smem)
         const DtTask tk = dt_decode(p, t);
         if (tk.quant) continue;
         const DtOp &op = p.ops[tk.op];
-        const bool maps = dt_maps_acquire(p, tk.op, smem, have);
+        if (lane == 0) dt_maps_acquire(p, tk.op, have);
         const CUtensorMap *g0 = p.wmaps + 2 * tk.op;
         const bool ffn = op.nmat == 2;
         const int np = dt_pieces(op.K);
@@ -369,7 +344,7 @@ BITNET_DEVINL void dt_weight_producer(const DtProgram &p, unsigned char *smem)
             const int s = ring_pos.slot;
             mbar_wait(&empty[s], ring_pos.par ^ 1u);
             if (lane == 0) {
-                if (maps) {
+                {
                     unsigned char *dst = ring + (size_t)s * (size_t)p.slot_bytes;
                     mbar_arrive_expect_tx(&full[s], RG * DT_WBYTES);
                     const int x = pc * (DT_KC / 4);
@@ -386,8 +361,6 @@ BITNET_DEVINL void dt_weight_producer(const DtProgram &p, unsigned char *smem)
                             tma_load_2d(d + DT_BOX_ROWS * DT_PITCH, g0, x, row + DT_BOX_ROWS, &full[s]);
                         }
                     }
-                } else {
-                    mbar_arrive(&full[s]); // maps unavailable (status set): keep the phases in step
                 }
                 issued |= 1u << s;
                 last_par = (last_par & ~(1u << s)) | (ring_pos.par << s);
@@ -1127,7 +1100,7 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_decode_tasks(const __grid_con
         const unsigned prev = atomicAdd(&p.counters[DT_CNT_EXIT], 1u);
         if (prev == gridDim.x - 1) {
             __threadfence();
-            for (int i = 0; i < DT_CNT_OPS + 3 * p.n_ops; ++i) atomicExch(&p.counters[i], 0u);
+            for (int i = 0; i < DT_CNT_OPS + 2 * p.n_ops; ++i) atomicExch(&p.counters[i], 0u);
         }
     }
 }

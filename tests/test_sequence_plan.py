@@ -273,12 +273,12 @@ def test_workspace_size():
     assert tw.bitnet_sequence_workspace_size(1, 64, 8192) >= 64 * 8192
     for bad in ((0, 8, 256), (129, 8, 256), (1, 0, 256), (1, 65, 256), (1, 8, 32), (1, 8, 8256)):
         assert tw.bitnet_sequence_workspace_size(*bad) == 0
-    # the documented size: counters (3 per op + 2), tensor maps (2 x 128 bytes per op, 128-byte
+    # the documented size: counters (2 per op + 2), tensor maps (2 x 128 bytes per op, 128-byte
     # alignment slack), then per op x_q [K/64][Mp][64] + 512 bytes of scales and row sums
     up = lambda v: (v + 255) // 256 * 256  # noqa: E731
     for n, m, k in ((1, 1, 256), (4, 8, 2560), (120, 8, 6912), (128, 64, 8192), (3, 13, 640)):
         mp = 8 if m <= 8 else 16 if m <= 16 else 32 if m <= 32 else 64
-        want = up(4 * (2 + 3 * n)) + up(256 * n + 128) + n * (up(k * mp) + 512)
+        want = up(4 * (2 + 2 * n)) + up(256 * n + 128) + n * (up(k * mp) + 512)
         assert tw.bitnet_sequence_workspace_size(n, m, k) == want
 
 
