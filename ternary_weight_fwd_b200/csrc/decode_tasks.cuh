@@ -445,6 +445,28 @@ BITNET_DEVINL void dt_act_producer(const DtProgram &p, unsigned char *smem)
     asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
+// Byte offset of x_q element k of token m in the fragment layout.  A k-block
+// (64 bytes per token) holds, at 16 t4 .. 16 t4 + 15, the 16 values that lane
+// group t4 of an mma over that block multiplies.  Ragged last piece (fewer than
+// 512 k): block k / 64, position k % 64.  Full piece pc: block 8 pc + kb of the
+// piece holds, at 16 t4, the values of packed word 8 t4 + kb of the piece (k =
+// 512 pc + 128 t4 + 16 kb ..), so that lane group t4 reads the weight words
+// 8 t4 .. 8 t4 + 7 of a row as two 16-byte chunks (both operands use the same
+// order of k inside the piece, which leaves the dot product unchanged).
+BITNET_DEVINL size_t dt_xq_offset(int k, int m, int Mp, int K)
+{
+    const int pc = k >> 9, kk = k & 511;
+    int blk, pos;
+    if ((pc + 1) * DT_KC <= K) {
+        blk = 8 * pc + ((kk >> 4) & 7);
+        pos = ((kk >> 7) << 4) | (kk & 15);
+    } else {
+        blk = k >> 6;
+        pos = k & 63;
+    }
+    return ((size_t)blk * Mp + m) * 64 + pos;
+}
+
 // ---- quant task (compute warps): tokens 8 i .. 8 i + 7 of op j, one per warp --
 // Warp w quantises token m = 8 i + w (m < M).  The row is read from L2 in
 // passes, so any K <= 8192 fits and no barrier between warps is needed: the
@@ -542,7 +564,7 @@ BITNET_DEVINL void dt_quant_pass(const DtProgram &p, const DtOp &op, int m, cons
                     rsum += q[h];
                 }
                 const int k0 = c * EPC;
-                int8_t *dst = xq + ((size_t)(k0 >> 6) * p.Mp + m) * 64 + (k0 & 63);
+                int8_t *dst = xq + dt_xq_offset(k0, m, p.Mp, op.K);
                 if constexpr (XF32) {
                     *reinterpret_cast<uint32_t *>(dst) = pack4_s8(q[0], q[1], q[2], q[3]);
                 } else {
@@ -739,7 +761,7 @@ BITNET_DEVINL void dt_quant_row(const DtProgram &p, const DtOp &op, int m, unsig
                 rsum += q[h];
             }
             const int k0 = c * EPC;
-            int8_t *dst = xq + ((size_t)(k0 >> 6) * p.Mp + m) * 64 + (k0 & 63);
+            int8_t *dst = xq + dt_xq_offset(k0, m, p.Mp, K);
             if constexpr (XF32) {
                 *reinterpret_cast<uint32_t *>(dst) = pack4_s8(q[0], q[1], q[2], q[3]);
             } else {
@@ -855,15 +877,35 @@ BITNET_DEVINL void dt_piece(int (&acc)[RG][SC][TT][4], const DtArow &wrow, uint3
     }
 }
 
-// A full piece (8 k-blocks): every weight fragment (and, for one token tile,
-// every activation fragment) is loaded before the first mma, so the
-// shared-memory latency is paid once per piece.
+// A full piece (8 k-blocks) in the permuted order of dt_xq_offset: lane group
+// t4 of k-block kb uses word 8 t4 + kb of each row, so a row's eight words for
+// the lane are its chunks 2 t4 and 2 t4 + 1 (two 16-byte loads; chunk c sits
+// at c ^ g).  Every weight fragment (and, for one token tile, every activation
+// fragment) is loaded before the first mma.
+template <int RG>
+BITNET_DEVINL void dt_ld_a_full(uint32_t (&lo)[DT_KB][RG], uint32_t (&hi)[DT_KB][RG], const DtArow &w, uint32_t t4)
+{
+    const uint32_t base_lo = w.lo - 4 * t4, base_hi = w.hi - 4 * t4; // chunk 0 of rows lo / hi
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const uint32_t cx = ((2 * t4 + h) << 4) ^ w.g16;
+#pragma unroll
+        for (int r = 0; r < RG; ++r) {
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(lo[4 * h][r]), "=r"(lo[4 * h + 1][r]), "=r"(lo[4 * h + 2][r]), "=r"(lo[4 * h + 3][r])
+                         : "r"(base_lo + (uint32_t)(r * DT_WBYTES) + cx));
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(hi[4 * h][r]), "=r"(hi[4 * h + 1][r]), "=r"(hi[4 * h + 2][r]), "=r"(hi[4 * h + 3][r])
+                         : "r"(base_hi + (uint32_t)(r * DT_WBYTES) + cx));
+        }
+    }
+}
+
 template <int TT, int SC, int RG>
-BITNET_DEVINL void dt_piece_full(int (&acc)[RG][SC][TT][4], const DtArow &wrow, uint32_t xrow, int Mp)
+BITNET_DEVINL void dt_piece_full(int (&acc)[RG][SC][TT][4], const DtArow &wrow, uint32_t xrow, int Mp, uint32_t t4)
 {
     uint32_t lo[DT_KB][RG], hi[DT_KB][RG];
-#pragma unroll
-    for (int kb = 0; kb < DT_KB; ++kb) dt_ld_a<RG>(lo[kb], hi[kb], wrow, kb);
+    dt_ld_a_full<RG>(lo, hi, wrow, t4);
     if constexpr (TT == 1) {
         uint4 bq[DT_KB][1];
 #pragma unroll
@@ -959,7 +1001,7 @@ BITNET_DEVINL void dt_compute(const DtProgram &p, unsigned char *smem)
                 const DtArow wr = {base + row_lo * DT_PITCH + t4 * 4, base + row_hi * DT_PITCH + t4 * 4,
                                    (uint32_t)g << 4};
                 if (nkb == DT_KB)
-                    dt_piece_full<TT, SC, RG>(acc, wr, base + xlane, Mp);
+                    dt_piece_full<TT, SC, RG>(acc, wr, base + xlane, Mp, (uint32_t)t4);
                 else
                     dt_piece<TT, SC, RG>(acc, wr, base + xlane, Mp, nkb);
                 __syncwarp();
