@@ -83,6 +83,7 @@ constexpr int DT_CNT_EXIT = 1;  // CTAs finished
 constexpr int DT_CNT_OPS = 2;   // then per op: quant tasks done, row tasks done
 
 constexpr uint16_t DT_DEP_QUANT = 0x8000u; // dependency on an op's quant tasks (else its row tasks)
+constexpr int DT_QEND = 0x7fffffff;         // queue entry: no more tasks
 
 struct DtOp {
     const void *x;                 // [M][K] bf16 or fp32 (read by the quant tasks)
@@ -156,6 +157,18 @@ BITNET_DEVINL DtTask dt_decode(const DtProgram &p, int t)
     r.op = sg.op;
     r.quant = (sg.first & 0x8000u) != 0;
     r.idx = (int)(sg.first & 0x7fffu) + (t - sg.start);
+    return r;
+}
+
+// Queue entries hold the decoded task (the weight producer decodes each claim
+// once): quant << 31 | op << 24 | idx; -1 ends the queue.
+BITNET_DEVINL int dt_pack(const DtTask &k) { return (k.quant ? (int)0x80000000u : 0) | (k.op << 24) | k.idx; }
+BITNET_DEVINL DtTask dt_unpack(int w)
+{
+    DtTask r;
+    r.quant = w < 0;
+    r.op = (w >> 24) & 0x7f;
+    r.idx = w & 0xffffff;
     return r;
 }
 
@@ -324,16 +337,17 @@ BITNET_DEVINL void dt_weight_producer(const DtProgram &p, unsigned char *smem)
     for (;;) {
         int t = (int)__shfl_sync(0xffffffffu, claim, 0);
         if (t >= p.n_tasks) t = -1;
+        DtTask tk = {0, 0, false};
+        if (t >= 0) tk = dt_decode(p, t);
         const int e = (int)(seq % DT_QUEUE);
         mbar_wait(&qempty[e], ((seq / DT_QUEUE) & 1u) ^ 1u);
         if (lane == 0) {
-            qtask[e] = t;
+            qtask[e] = t < 0 ? DT_QEND : dt_pack(tk);
             mbar_arrive(&qfull[e]);
         }
         ++seq;
         if (t < 0) break;
         if (lane == 0) claim = atomicAdd(&p.counters[DT_CNT_TASK], 1u);
-        const DtTask tk = dt_decode(p, t);
         if (tk.quant) continue;
         const DtOp &op = p.ops[tk.op];
         if (lane == 0) dt_maps_acquire(p, tk.op, have);
@@ -395,8 +409,8 @@ BITNET_DEVINL void dt_act_producer(const DtProgram &p, unsigned char *smem)
         const int t = qtask[e];
         bool rows = false;
         DtTask tk = {0, 0, true};
-        if (t >= 0) {
-            tk = dt_decode(p, t);
+        if (t != DT_QEND) {
+            tk = dt_unpack(t);
             rows = !tk.quant;
         }
         if (rows) {
@@ -440,7 +454,7 @@ BITNET_DEVINL void dt_act_producer(const DtProgram &p, unsigned char *smem)
         __syncwarp();
         if (lane == 0) mbar_arrive(&qempty[e]);
         ++seq;
-        if (t < 0) break;
+        if (t == DT_QEND) break;
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
 }
@@ -949,8 +963,8 @@ BITNET_DEVINL void dt_compute(const DtProgram &p, unsigned char *smem)
         const int e = (int)(seq % DT_QUEUE);
         mbar_wait(&qfull[e], (seq / DT_QUEUE) & 1u);
         const int t = qtask[e];
-        if (t < 0) break;
-        const DtTask tk = dt_decode(p, t);
+        if (t == DT_QEND) break;
+        const DtTask tk = dt_unpack(t);
         const DtOp &op = p.ops[tk.op];
         if (tk.quant) {
             if constexpr (TT == 1) {
@@ -1096,8 +1110,8 @@ BITNET_DEVINL void dt_completion(const DtProgram &p, unsigned char *smem)
         const uint32_t par = (seq / DT_QUEUE) & 1u;
         mbar_wait(&qfull[e], par);
         const int t = qtask[e];
-        if (t < 0) break;
-        const DtTask tk = dt_decode(p, t);
+        if (t == DT_QEND) break;
+        const DtTask tk = dt_unpack(t);
         mbar_wait(&cdone[e], par);
         if (lane == 0) {
             __threadfence();
