@@ -250,6 +250,23 @@ cudaError_t launch_decode(const DecodeArgs &a, const DecodeCfg &c, cudaStream_t 
     }
 }
 
+template <bool XF32, int WPR>
+cudaError_t launch_quant_w(const void *x, int64_t M, int64_t K, int8_t *xq, float *s, int32_t *rs,
+                           const float *amax_in, float *amax_zero, cudaStream_t stream)
+{
+    const int64_t nch = K / (XF32 ? 4 : 8);
+    const int64_t per_lane = cdiv(nch, 32 * WPR); // chunks a lane holds
+    const dim3 grid((unsigned)cdiv(M, 8 / WPR));
+    if (per_lane <= 8)
+        return launch_pdl(k_quant_rows_reg<XF32, WPR, 8>, grid, dim3(256), 0, stream, x, M, K, xq, s, rs, amax_in,
+                          amax_zero);
+    if (per_lane <= 12)
+        return launch_pdl(k_quant_rows_reg<XF32, WPR, 12>, grid, dim3(256), 0, stream, x, M, K, xq, s, rs, amax_in,
+                          amax_zero);
+    return launch_pdl(k_quant_rows_reg<XF32, WPR, QR_NCH>, grid, dim3(256), 0, stream, x, M, K, xq, s, rs, amax_in,
+                      amax_zero);
+}
+
 // Per-token quantiser: rows held in registers (one HBM read) when a row fits
 // in 8 warps x 32 lanes x QR_NCH chunks, otherwise the two-pass kernel (one
 // pass when the row maxima are given).  amax_in: optional given row maxima;
@@ -260,18 +277,10 @@ cudaError_t launch_quant_t(const void *x, int64_t M, int64_t K, int8_t *xq, floa
 {
     const int64_t nch = K / (XF32 ? 4 : 8);
     const int64_t per_warp = 32 * QR_NCH;
-    if (nch <= per_warp)
-        return launch_pdl(k_quant_rows_reg<XF32, 1>, dim3((unsigned)cdiv(M, 8)), dim3(256), 0, stream, x, M, K, xq,
-                          s, rs, amax_in, amax_zero);
-    if (nch <= 2 * per_warp)
-        return launch_pdl(k_quant_rows_reg<XF32, 2>, dim3((unsigned)cdiv(M, 4)), dim3(256), 0, stream, x, M, K, xq,
-                          s, rs, amax_in, amax_zero);
-    if (nch <= 4 * per_warp)
-        return launch_pdl(k_quant_rows_reg<XF32, 4>, dim3((unsigned)cdiv(M, 2)), dim3(256), 0, stream, x, M, K, xq,
-                          s, rs, amax_in, amax_zero);
-    if (nch <= 8 * per_warp)
-        return launch_pdl(k_quant_rows_reg<XF32, 8>, dim3((unsigned)M), dim3(256), 0, stream, x, M, K, xq, s, rs,
-                          amax_in, amax_zero);
+    if (nch <= per_warp) return launch_quant_w<XF32, 1>(x, M, K, xq, s, rs, amax_in, amax_zero, stream);
+    if (nch <= 2 * per_warp) return launch_quant_w<XF32, 2>(x, M, K, xq, s, rs, amax_in, amax_zero, stream);
+    if (nch <= 4 * per_warp) return launch_quant_w<XF32, 4>(x, M, K, xq, s, rs, amax_in, amax_zero, stream);
+    if (nch <= 8 * per_warp) return launch_quant_w<XF32, 8>(x, M, K, xq, s, rs, amax_in, amax_zero, stream);
     return launch_pdl(k_quant_rows<XF32>, dim3((unsigned)cdiv(M, 8)), dim3(256), 0, stream, x, M, K, xq, s, rs,
                       amax_in, amax_zero);
 }

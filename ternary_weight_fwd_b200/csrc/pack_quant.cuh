@@ -167,11 +167,12 @@ __global__ void __launch_bounds__(256) k_quant_rows(const void *__restrict__ x, 
 // quantise step, so x is read from HBM exactly once (the two-pass kernel above
 // re-reads rows that no longer sit in cache once the input exceeds L2).  WPR
 // warps share a row (8 / WPR rows per 256-thread CTA); every lane holds up to
-// QR_NCH 16-byte chunks of it.  Same arithmetic as k_quant_rows.
+// NCH <= QR_NCH 16-byte chunks of it (the fewest that hold the row: fewer
+// registers, more rows in flight per SM).  Same arithmetic as k_quant_rows.
 constexpr int QR_NCH = 16;
 
-template <bool XF32, int WPR>
-__global__ void __launch_bounds__(256) k_quant_rows_reg(const void *__restrict__ x, int64_t M, int64_t K,
+template <bool XF32, int WPR, int NCH>
+__global__ void __launch_bounds__(256, NCH <= 12 ? 3 : 2) k_quant_rows_reg(const void *__restrict__ x, int64_t M, int64_t K,
                                                         int8_t *__restrict__ x_q, float *__restrict__ s,
                                                         int32_t *__restrict__ rowsum,
                                                         const float *__restrict__ amax_in,
@@ -190,10 +191,10 @@ __global__ void __launch_bounds__(256) k_quant_rows_reg(const void *__restrict__
     const int nch = (int)(K / EPC);
     const int c0 = wr * 32 + lane;
     const uint4 *row = reinterpret_cast<const uint4 *>(static_cast<const char *>(x) + (live ? m : 0) * K * (XF32 ? 4 : 2));
-    uint4 v[QR_NCH];
+    uint4 v[NCH];
     float amax = 0.0f;
 #pragma unroll
-    for (int i = 0; i < QR_NCH; ++i) {
+    for (int i = 0; i < NCH; ++i) {
         const int c = c0 + i * 32 * WPR;
         if (live && c < nch) {
             v[i] = __ldg(row + c);
@@ -216,7 +217,7 @@ __global__ void __launch_bounds__(256) k_quant_rows_reg(const void *__restrict__
     int rs = 0;
     int8_t *qrow = x_q + (live ? m : 0) * K;
 #pragma unroll
-    for (int i = 0; i < QR_NCH; ++i) {
+    for (int i = 0; i < NCH; ++i) {
         const int c = c0 + i * 32 * WPR;
         if (live && c < nch) {
             const uint2 q = chunk_quant<XF32>(v[i], sc, rs);
