@@ -1020,11 +1020,15 @@ cudaError_t seq_launch_t(const DtProgram &p, int ctas, cudaStream_t stream, int 
     cudaError_t e = ensure_smem(k_decode_tasks<TT, RG>, kSmemLimit, smem_done, dev);
     if (e != cudaSuccess) return e;
     const size_t smem = 1024 + DT_HDR + (size_t)p.n_slots * p.slot_bytes; // + alignment to 1024 bytes
-    // the weights' tensor maps, then the sequence
-    g_launches.fetch_add(2, std::memory_order_relaxed);
+    // the weights' tensor maps (after everything before it on the stream: a previous
+    // sequence on this workspace may still read the old ones), then the sequence as its
+    // programmatic dependent: everything but the weight producer starts while the maps
+    // are written
+    g_launches.fetch_add(1, std::memory_order_relaxed);
     k_decode_maps<<<p.n_ops, 32, 0, stream>>>(p);
-    k_decode_tasks<TT, RG><<<ctas, DT_THREADS, smem, stream>>>(p);
-    return cudaGetLastError();
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return launch_pdl(k_decode_tasks<TT, RG>, dim3(ctas), dim3(DT_THREADS), smem, stream, p);
 }
 
 cudaError_t seq_launch(const DtProgram &p, int ctas, cudaStream_t stream, int dev)

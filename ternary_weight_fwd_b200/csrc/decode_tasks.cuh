@@ -289,6 +289,7 @@ __global__ void __launch_bounds__(32) k_decode_maps(const __grid_constant__ DtPr
 {
     __shared__ alignas(128) unsigned char sm[2][128];
     const int j = blockIdx.x, lane = threadIdx.x;
+    pdl_launch_dependents(); // the sequence kernel starts now; its weight producer waits for this grid
     if (j >= p.n_ops) return;
     const DtOp &op = p.ops[j];
     for (int m = 0; m < op.nmat; ++m) {
@@ -331,6 +332,7 @@ BITNET_DEVINL void dt_weight_producer(const DtProgram &p, unsigned char *smem)
     DtRing ring_pos;
     uint32_t have[DT_MAX_OPS / 32] = {0u, 0u, 0u, 0u}; // ops whose maps this warp has acquired
     uint32_t issued = 0, last_par = 0;               // slots with copies issued, and their last phase
+    pdl_wait(); // the tensor maps written by k_decode_maps are visible
     // the claim of the next task is issued one task ahead, so its latency overlaps the copies
     unsigned claim = 0;
     if (lane == 0) claim = atomicAdd(&p.counters[DT_CNT_TASK], 1u);
