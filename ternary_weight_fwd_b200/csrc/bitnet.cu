@@ -864,50 +864,76 @@ bitnet_status_t seq_groups(const bitnet_op_t *ops, int n, int64_t M, ByteRange e
 }
 
 // Order of the task groups in the launch's global task list.  A list-scheduling
-// simulation on `ctas` CTAs: repeatedly take, among the groups whose
-// predecessors are already placed, the one whose predecessors finish first
-// (ties: execution order), and give its tasks to the CTAs that free up first.
-// Durations are estimates (a quant task 1.5 us for one token, 3 us for 8; a row task its packed weights at
-// ~40 GB/s per SM).  CTAs claim tasks in this order, so a dependent group is
-// placed after the work that will be running while its producer finishes.
+// simulation on `ctas` CTAs: at the time the first CTA frees up, among the
+// groups whose predecessors are placed and finished by then, take the one with
+// the longest chain of work after it (its own duration plus the longest chain
+// of its successors), ties in execution order; if none is ready, the one whose
+// predecessors finish first.  Its tasks go to the CTAs that free up first.
+// Durations are estimates (a quant task 1.5 us for one token, 3 us for 8; a row
+// task its packed weights at ~28 GB/s per SM, the rate a CTA sustains in a full
+// step; a dependent group is ready kSeqHandOver after its predecessors finish:
+// completion fence, counter, the consumer's poll and copies).  Chains such as gate/up -> down
+// therefore start early and short independent work is left for the end, where
+// it fills the CTAs instead of a few long tasks running on a mostly idle GPU.
+// CTAs claim tasks in this order; every dependency points to an earlier group.
+constexpr double kSeqHandOver = 3.0; // us
+
 std::vector<int> seq_group_order(const bitnet_op_t *ops, int n, int64_t M, const SeqGroups &G, int ctas)
 {
     const int ng = 2 * n;
-    std::vector<double> finish(ng, 0.0), dur(ng, 0.0);
+    const int nc = std::max(1, ctas);
+    std::vector<double> finish(ng, 0.0), dur(ng, 0.0), chain(ng, 0.0);
     std::vector<int> count(ng, 0), left(ng, 0), order;
     for (int j = 0; j < n; ++j) {
         count[2 * j] = seq_qtasks(M);
         dur[2 * j] = M <= 8 ? 1.5 : 3.0;
         count[2 * j + 1] = seq_rtasks(ops[j], M);
-        dur[2 * j + 1] = (double)(DT_ROWS * seq_rg(M)) * (double)(ops[j].K / 4) / 40e3;
+        dur[2 * j + 1] = (double)(DT_ROWS * seq_rg(M)) * (double)(ops[j].K / 4) / 28e3;
     }
     std::vector<std::vector<int>> succ(ng);
     for (int v = 0; v < ng; ++v) {
         left[v] = (int)G.preds[v].size();
         for (int u : G.preds[v]) succ[u].push_back(v);
     }
+    // successors are later groups (dependencies point to earlier ops, or from an op's
+    // rows to its own quant tasks), so one backward pass computes every chain
+    for (int v = ng - 1; v >= 0; --v) {
+        double after = 0.0;
+        for (int w : succ[v]) after = std::max(after, chain[w]);
+        chain[v] = dur[v] * (double)((count[v] + nc - 1) / nc) + after;
+    }
     std::priority_queue<double, std::vector<double>, std::greater<double>> free_at;
-    for (int c = 0; c < std::max(1, ctas); ++c) free_at.push(0.0);
+    for (int c = 0; c < nc; ++c) free_at.push(0.0);
     std::vector<char> placed(ng, 0);
     for (int k = 0; k < ng; ++k) {
-        int pick = -1;
-        double best = 0.0;
+        const double now = free_at.top();
+        int pick = -1, first = -1;
+        double best_chain = -1.0, first_ready = 0.0, pick_ready = 0.0;
         for (int v = 0; v < ng; ++v) {
             if (placed[v] || left[v] != 0) continue;
             double ready = 0.0;
-            for (int u : G.preds[v]) ready = std::max(ready, finish[u]);
-            if (pick < 0 || ready < best) {
-                pick = v;
-                best = ready;
+            for (int u : G.preds[v]) ready = std::max(ready, finish[u] + kSeqHandOver);
+            if (first < 0 || ready < first_ready) {
+                first = v;
+                first_ready = ready;
             }
+            if (ready <= now && chain[v] > best_chain) {
+                pick = v;
+                best_chain = chain[v];
+                pick_ready = ready;
+            }
+        }
+        if (pick < 0) {
+            pick = first;
+            pick_ready = first_ready;
         }
         placed[pick] = 1;
         order.push_back(pick);
-        double fin = best;
+        double fin = pick_ready;
         for (int t = 0; t < count[pick]; ++t) {
             const double f = free_at.top();
             free_at.pop();
-            const double end = std::max(f, best) + dur[pick];
+            const double end = std::max(f, pick_ready) + dur[pick];
             free_at.push(end);
             fin = std::max(fin, end);
         }

@@ -400,13 +400,16 @@ def simulate_groups(ops, m, groups, order, arena_lo, arena_hi):
 
 def test_tasks_of_the_bench_decode_step():
     """30 layers with private outputs at M = 8 on 148 CTAs: every input is fresh except down's
-    (h of the same layer), so all 90 fresh quant groups come first, a down's quant group waits
-    only for its gate/up rows, and rows groups wait only for their own quant group."""
+    (h of the same layer), so a down's quant group waits only for its gate/up rows, and rows
+    groups wait only for their own quant group.  The order starts the longest chains (gate/up
+    -> down) first and leaves the short independent q / o rows for the end."""
     ops = layer_stack(30, 8, shared_outputs=False)
     groups = tw.bitnet_sequence_tasks(ops, 8, 148)
     pos = check_tasks(ops, 8, groups)
-    fresh = [k for k, g in enumerate(groups) if g["kind"] == "quant" and g["op"] % 4 != 3]
-    assert fresh == list(range(90))
+    assert [g["op"] % 4 for g in groups[:30]] == [2] * 30 and all(g["kind"] == "quant" for g in groups[:30])
+    assert all(g["kind"] == "rows" and g["op"] % 4 in (0, 1) for g in groups[-20:])
+    for l in range(30):
+        assert pos[(4 * l + 3, "rows")] < pos[(4 * l, "rows")]  # each down before its layer's q
     for l in range(30):
         gu, dn = 4 * l + 2, 4 * l + 3
         assert groups[pos[(dn, "quant")]]["deps"] == [pos[(gu, "rows")]]
