@@ -122,16 +122,18 @@ Workspace carve(void *ws, int64_t M, int64_t K)
 }
 
 // ---- prefill: the partly filled last wave of tiles (see k_prefill) -------------
-// When the last wave holds at most a sixth (third, half) of the grid, each of its
-// tiles runs as 6 (3, 2) units of 32 (64, 96) tokens on separate CTAs.
-int pf_tail_q(int64_t tiles, int sms)
+// A BitLinear whose last wave holds at most a quarter (half) of the grid runs each
+// of its tiles as 4 (2) sub-tiles of 64 (128) output columns on separate CTAs.
+int pf_tail_q(int64_t M, int64_t N, int nmat, int sms)
 {
+    if (nmat != 1) return 1;
+    const int64_t tiles = cdiv(M, PF_BM) * cdiv(N, PF_BN);
     const int64_t grid = std::min<int64_t>(tiles, sms);
     if (grid <= 0) return 1;
     const int64_t full = tiles / grid * grid, rem = tiles - full;
     if (full == 0 || rem == 0) return 1;
-    for (int q : {6, 3, 2})
-        if (q * rem <= grid) return q;
+    if (4 * rem <= grid) return 4;
+    if (2 * rem <= grid) return 2;
     return 1;
 }
 
@@ -171,7 +173,8 @@ bool encode_u8_2d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t co
     return r == CUDA_SUCCESS;
 }
 
-// 2-D output tensor [rows][cols] of fp32 or bf16, box [box_rows][box_cols], no swizzle.
+// 2-D output tensor [rows][cols] of fp32 (128-byte swizzle) or bf16 (64-byte
+// swizzle), box [box_rows][box_cols]: the box rows are exactly one swizzle span.
 bool encode_2d_out(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows,
                    uint32_t box_cols, bool bf16)
 {
@@ -183,7 +186,8 @@ bool encode_2d_out(CUtensorMap *map, const void *base, uint64_t rows, uint64_t c
     cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
                     const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                    bf16 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
@@ -623,10 +627,10 @@ bitnet_status_t forward(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_
     a.M = (int)M;
     a.N = (int)N;
     a.K = (int)K;
-    a.num_t = (int)cdiv(M, PF_TN);
-    a.num_w = (int)cdiv(N, nmat == 1 ? PF_WM : PF_WM / 2);
+    a.num_m = (int)cdiv(M, PF_BM);
+    a.num_n = (int)cdiv(N, nmat == 1 ? PF_BN : PF_BN / 2);
     a.num_k = (int)cdiv(K, PF_BK);
-    a.num_tiles = a.num_t * a.num_w;
+    a.num_tiles = a.num_m * a.num_n;
     a.gamma0 = gamma0;
     a.gamma1 = gamma1;
     a.s = s;
@@ -635,44 +639,45 @@ bitnet_status_t forward(const void *x, bitnet_dtype_t x_dtype, int64_t M, int64_
     a.y_amax = io.y_amax;
     a.acc0 = acc0;
     a.acc1 = acc1;
-    // x_q in 64-token boxes of 128 k (128-byte swizzle); packed weights in boxes of
-    // 128 rows (BitLinear) or 16 rows (FFN: gate and up rows interleaved per tile);
-    // outputs in chunks of 32 tokens x 32 (FFN: 16) columns when rows are 16-byte multiples
-    CUtensorMap tmX, tmW0, tmW1, tmY;
-    const uint32_t wrows = nmat == 1 ? PF_WM : 16;
-    if (!encode_u8_2d(&tmX, xq, (uint64_t)M, (uint64_t)K, PF_XBOX, PF_BK, true) ||
-        !encode_u8_2d(&tmW0, w0, (uint64_t)N, (uint64_t)(K / 4), wrows, PF_BK / 4, false))
+    a.vec_ok = (N % (io.y_bf16 ? 8 : 4)) == 0; // 16-byte rows
+    CUtensorMap tmA, tmB0, tmB1, tmY;
+    const uint32_t brows = nmat == 1 ? PF_BN : PF_BN / 2;
+    if (!encode_u8_2d(&tmA, xq, (uint64_t)M, (uint64_t)K, PF_BM, PF_BK, true) ||
+        !encode_u8_2d(&tmB0, w0, (uint64_t)N, (uint64_t)(K / 4), brows, PF_BK / 4, false))
         return BITNET_ERR_CUDA;
     if (nmat == 2) {
-        if (!encode_u8_2d(&tmW1, w1, (uint64_t)N, (uint64_t)(K / 4), wrows, PF_BK / 4, false))
+        if (!encode_u8_2d(&tmB1, w1, (uint64_t)N, (uint64_t)(K / 4), brows, PF_BK / 4, false))
             return BITNET_ERR_CUDA;
     } else {
-        tmW1 = tmW0;
+        tmB1 = tmB0;
     }
-    a.tma_out = (N % (io.y_bf16 ? 8 : 4)) == 0;
-    tmY = tmX;
-    if (a.tma_out && !encode_2d_out(&tmY, y, (uint64_t)M, (uint64_t)N, 32, nmat == 1 ? 32 : 16, io.y_bf16))
-        return BITNET_ERR_CUDA;
+    // the last, partly filled wave of a BitLinear as sub-tiles (tmB1: a box of their rows)
     const int grid = std::min(a.num_tiles, sms);
-    a.tail_q = pf_tail_q(a.num_tiles, sms);
+    a.tail_q = pf_tail_q(M, N, nmat, sms);
     a.full_units = a.num_tiles;
     a.num_units = a.num_tiles;
     if (a.tail_q > 1) {
         a.full_units = a.num_tiles / grid * grid;
         a.num_units = a.full_units + (a.num_tiles - a.full_units) * a.tail_q;
+        if (!encode_u8_2d(&tmB1, w0, (uint64_t)N, (uint64_t)(K / 4), (uint32_t)(PF_BN / a.tail_q), PF_BK / 4, false))
+            return BITNET_ERR_CUDA;
     }
+    // output through TMA stores when rows are 16-byte multiples: 32 x 32 boxes,
+    // 128-byte swizzle for fp32, 64-byte swizzle for bf16
+    tmY = tmA;
+    if (a.vec_ok && !encode_2d_out(&tmY, y, (uint64_t)M, (uint64_t)N, 32, 32, io.y_bf16)) return BITNET_ERR_CUDA;
     cudaError_t e = quantise(xq, s, nullptr);
     if (e != cudaSuccess) return BITNET_ERR_CUDA;
     if (nmat == 1) {
         static std::atomic<int> done[kMaxDevices];
         e = ensure_smem(k_prefill<false>, PF_SMEM, done, dev);
         if (e == cudaSuccess)
-            e = launch_pdl(k_prefill<false>, dim3(grid), dim3(PF_THREADS), PF_SMEM, stream, tmX, tmW0, tmW1, tmY, a);
+            e = launch_pdl(k_prefill<false>, dim3(grid), dim3(PF_THREADS), PF_SMEM, stream, tmA, tmB0, tmB1, tmY, a);
     } else {
         static std::atomic<int> done[kMaxDevices];
         e = ensure_smem(k_prefill<true>, PF_SMEM, done, dev);
         if (e == cudaSuccess)
-            e = launch_pdl(k_prefill<true>, dim3(grid), dim3(PF_THREADS), PF_SMEM, stream, tmX, tmW0, tmW1, tmY, a);
+            e = launch_pdl(k_prefill<true>, dim3(grid), dim3(PF_THREADS), PF_SMEM, stream, tmA, tmB0, tmB1, tmY, a);
     }
     return cuda_status(e);
 }

@@ -384,18 +384,6 @@ BITNET_DEVINL void umma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint
         : "memory");
 }
 
-// D[tmem] (+)= A[tmem] . B[smem]^T, int8 inputs, int32 accumulators.  A (M = 128)
-// sits on TMEM lanes 0-127, row m in lane m, k in byte k % 4 of column k / 4.
-BITNET_DEVINL void umma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc, uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
 // Arrive once on `bar` when every tcgen05 operation issued so far by this
 // thread has completed.
 BITNET_DEVINL void umma_commit(uint64_t *bar)
@@ -418,18 +406,6 @@ BITNET_DEVINL void tmem_ld32(uint32_t taddr, uint32_t (&v)[32])
                  : "r"(taddr)
                  : "memory");
 }
-// Warp-collective: 32 lanes x 16 consecutive 32-bit columns from registers.
-BITNET_DEVINL void tmem_st16(uint32_t taddr, const uint32_t (&v)[16])
-{
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-                 "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
-                 "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
-                 "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
-                 : "memory");
-}
-// This thread's tcgen05.st have completed.
-BITNET_DEVINL void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
 // The registers a tcgen05.ld writes are valid only after tcgen05.wait::ld, but
 // the compiler does not know that: these forms name them as operands of the
 // wait (or of an empty statement right after it), so no use of them can be
