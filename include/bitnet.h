@@ -321,7 +321,8 @@ typedef struct bitnet_op {
     float norm_eps;        /* its epsilon (>= 0; used only with norm_g) */
 } bitnet_op_t;
 
-#define BITNET_SEQ_MAX_OPS 128
+#define BITNET_SEQ_MAX_OPS 128        /* ops of one launch (and of the host planning calls) */
+#define BITNET_SEQ_MAX_OPS_TOTAL 1024 /* ops of one bitnet_decode_sequence call */
 #define BITNET_SEQ_MAX_M 64
 
 /*
@@ -332,7 +333,11 @@ typedef struct bitnet_op {
  * sums.  A list of n ops needs exactly
  *   up256(4 * (2 + 2n)) + up256(256n + 128) + sum over ops of (up256(K * Mp) + 512)
  * bytes (up256 = rounded up to a multiple of 256); this returns that for
- * n_ops ops of K = K_max.  0 for arguments out of range.
+ * n_ops ops of K = K_max.  A list longer than BITNET_SEQ_MAX_OPS runs as
+ * launches of BITNET_SEQ_MAX_OPS ops (the last one shorter), each with its own
+ * consecutive part of the workspace laid out as above for its ops, every op
+ * sized for the largest K of the whole list; the size is the sum of the parts.
+ * 1 <= n_ops <= BITNET_SEQ_MAX_OPS_TOTAL; 0 for arguments out of range.
  */
 size_t bitnet_sequence_workspace_size(int32_t n_ops, int64_t M, int64_t K_max);
 
@@ -384,15 +389,20 @@ bitnet_status_t bitnet_sequence_schedule(const bitnet_op_t *ops, int32_t n_ops, 
  * streamed ahead of every wait.  Progress does not depend on how many CTAs
  * are resident at the same time.
  *
- *   ops, n_ops  1 <= n_ops <= BITNET_SEQ_MAX_OPS ops (host array, read
- *               during the call only; the launch keeps its own copy)
+ *   ops, n_ops  1 <= n_ops <= BITNET_SEQ_MAX_OPS_TOTAL ops (host array,
+ *               read during the call only; the launch keeps its own copy).
+ *               Lists longer than BITNET_SEQ_MAX_OPS run as consecutive
+ *               launches of BITNET_SEQ_MAX_OPS ops in list order (two kernels
+ *               each); a later launch starts once the earlier one has
+ *               finished, so ops in different launches are ordered as in the
+ *               list.  All parts are validated before the first launch.
  *   M           tokens, 1 <= M <= BITNET_SEQ_MAX_M, the same for every op
  *   workspace   device memory of at least
  *               bitnet_sequence_workspace_size(n_ops, M, max K) bytes whose
- *               first 4 * (2 + 2 * n_ops) bytes are ZERO before its first use;
- *               every call leaves them zero again (also after a device-side
- *               timeout).  Calls that may run at the same time need separate
- *               workspaces.
+ *               counters (the first 4 * (2 + 2 * n) bytes of the part of each
+ *               launch of n ops) are ZERO before its first use; every call
+ *               leaves them zero again (also after a device-side timeout).
+ *               Calls that may run at the same time need separate workspaces.
  *
  * Errors (nothing is launched): BITNET_ERR_INVALID_ARG for a null pointer, a
  * bad kind or dtype, a negative or non-finite norm_eps, an op whose y overlaps

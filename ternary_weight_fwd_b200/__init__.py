@@ -33,7 +33,8 @@ BITNET_DISPATCH_PREFILL = 3
 
 BITNET_OP_LINEAR = 0
 BITNET_OP_FFN_GATE_UP = 1
-BITNET_SEQ_MAX_OPS = 128
+BITNET_SEQ_MAX_OPS = 128         # ops of one launch
+BITNET_SEQ_MAX_OPS_TOTAL = 1024  # ops of one bitnet_decode_sequence call (consecutive launches)
 BITNET_SEQ_MAX_M = 64
 
 QUANT_EPS = 1e-5
@@ -400,7 +401,8 @@ def bitnet_sequence_tasks(ops, m, ctas):
 
 
 def bitnet_decode_sequence(ops, m, workspace, stream=None):
-    """Run `ops` (bitnet_op_t records over the same m tokens) in one persistent launch."""
+    """Run `ops` (bitnet_op_t records over the same m tokens) in one persistent launch per
+    BITNET_SEQ_MAX_OPS ops."""
     _check(load_library().bitnet_decode_sequence(_op_array(ops), len(ops), m, _ptr(workspace), workspace.numel(),
                                                  _stream(stream)), "bitnet_decode_sequence")
 

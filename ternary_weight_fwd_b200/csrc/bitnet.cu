@@ -1104,8 +1104,10 @@ bool seq_cache_match(const SeqCacheEntry &e, const bitnet_op_t *ops, int n, int6
 
 int seq_ctas(int dev) { return num_sms_for(dev); } // one CTA per SM (227 KB of shared memory each)
 
+// One launch of at most BITNET_SEQ_MAX_OPS ops.  whole: the byte range no op may
+// touch (the caller's whole workspace), or null for this part's own.
 bitnet_status_t decode_sequence(const bitnet_op_t *ops, int n, int64_t M, void *workspace, size_t ws_bytes,
-                                cudaStream_t stream)
+                                cudaStream_t stream, const ByteRange *whole = nullptr)
 {
     if (workspace && !aligned16(workspace)) return BITNET_ERR_MISALIGNED;
     const int stall = g_seq_stall.load();
@@ -1126,7 +1128,7 @@ bitnet_status_t decode_sequence(const bitnet_op_t *ops, int n, int64_t M, void *
         }
         if (hit) return cuda_status(seq_launch(p, seq_ctas(dev), stream, dev));
     }
-    const ByteRange wsr = workspace ? range_of(workspace, ws_bytes) : ByteRange{0, 0};
+    const ByteRange wsr = whole ? *whole : workspace ? range_of(workspace, ws_bytes) : ByteRange{0, 0};
     int32_t order[BITNET_SEQ_MAX_OPS];
     bitnet_status_t st = seq_schedule(ops, n, M, order, wsr);
     if (st != BITNET_OK) return st;
@@ -1320,12 +1322,21 @@ bitnet_status_t bitnet_ffn_gate_up(const void *x, bitnet_dtype_t x_dtype, int64_
                    acc_u_out, workspace, ws_bytes, stream, 2);
 }
 
+// Workspace of one launch of n ops (all sized for K_max).
+size_t seq_part_ws_bytes(int n, int64_t M, int64_t K_max)
+{
+    return seq_counter_bytes(n) + seq_map_bytes(n) + (size_t)n * seq_op_ws_bytes(align_up((size_t)K_max, 64), seq_mp(M));
+}
+
 size_t bitnet_sequence_workspace_size(int32_t n_ops, int64_t M, int64_t K_max)
 {
-    if (n_ops < 1 || n_ops > BITNET_SEQ_MAX_OPS || M < 1 || M > BITNET_SEQ_MAX_M || K_max < 64 || K_max > kSeqMaxK)
+    if (n_ops < 1 || n_ops > BITNET_SEQ_MAX_OPS_TOTAL || M < 1 || M > BITNET_SEQ_MAX_M || K_max < 64 ||
+        K_max > kSeqMaxK)
         return 0;
-    return seq_counter_bytes(n_ops) + seq_map_bytes(n_ops) +
-           (size_t)n_ops * seq_op_ws_bytes(align_up((size_t)K_max, 64), seq_mp(M));
+    size_t total = 0;
+    for (int c0 = 0; c0 < n_ops; c0 += BITNET_SEQ_MAX_OPS)
+        total += seq_part_ws_bytes(std::min(BITNET_SEQ_MAX_OPS, n_ops - c0), M, K_max);
+    return total;
 }
 
 bitnet_status_t bitnet_sequence_plan(const bitnet_op_t *ops, int32_t n_ops, int64_t M, int32_t *wait_x,
@@ -1337,7 +1348,35 @@ bitnet_status_t bitnet_sequence_plan(const bitnet_op_t *ops, int32_t n_ops, int6
 bitnet_status_t bitnet_decode_sequence(const bitnet_op_t *ops, int32_t n_ops, int64_t M, void *workspace,
                                        size_t ws_bytes, cudaStream_t stream)
 {
-    return decode_sequence(ops, n_ops, M, workspace, ws_bytes, stream);
+    if (n_ops <= BITNET_SEQ_MAX_OPS) return decode_sequence(ops, n_ops, M, workspace, ws_bytes, stream);
+    // a longer list: consecutive launches of BITNET_SEQ_MAX_OPS ops, each on its own part of the
+    // workspace (sized for the largest K of the list), all validated before the first launch
+    if (!ops || n_ops > BITNET_SEQ_MAX_OPS_TOTAL || M < 1 || M > BITNET_SEQ_MAX_M) return BITNET_ERR_INVALID_ARG;
+    if (!workspace) return BITNET_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return BITNET_ERR_MISALIGNED;
+    int64_t K_max = 64;
+    for (int i = 0; i < n_ops; ++i) K_max = std::max(K_max, ops[i].K);
+    if (K_max > kSeqMaxK) return BITNET_ERR_UNSUPPORTED_SHAPE;
+    const ByteRange whole = range_of(workspace, ws_bytes);
+    size_t need = 0;
+    for (int c0 = 0; c0 < n_ops; c0 += BITNET_SEQ_MAX_OPS) {
+        const int nc = std::min(BITNET_SEQ_MAX_OPS, n_ops - c0);
+        int32_t order[BITNET_SEQ_MAX_OPS];
+        const bitnet_status_t st = seq_schedule(ops + c0, nc, M, order, whole);
+        if (st != BITNET_OK) return st;
+        need += seq_part_ws_bytes(nc, M, K_max);
+    }
+    if (need > ws_bytes) return BITNET_ERR_WORKSPACE;
+    size_t off = 0;
+    for (int c0 = 0; c0 < n_ops; c0 += BITNET_SEQ_MAX_OPS) {
+        const int nc = std::min(BITNET_SEQ_MAX_OPS, n_ops - c0);
+        const size_t part = seq_part_ws_bytes(nc, M, K_max);
+        const bitnet_status_t st =
+            decode_sequence(ops + c0, nc, M, static_cast<unsigned char *>(workspace) + off, part, stream, &whole);
+        if (st != BITNET_OK) return st;
+        off += part;
+    }
+    return BITNET_OK;
 }
 
 bitnet_status_t bitnet_sequence_schedule(const bitnet_op_t *ops, int32_t n_ops, int64_t M, int32_t *order)

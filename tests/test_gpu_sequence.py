@@ -344,6 +344,44 @@ def test_full_decode_step_of_the_benchmark():
             assert same_bits(got, ref), l
 
 
+def test_list_longer_than_one_launch():
+    """45 layers at M = 8: 180 ops in one call, run as two launches of 128 and 52 ops.  Layer
+    32's q reads layer 31's down output, so the first op of the second launch reads what the
+    last op of the first launch wrote.  Every output is bitwise equal to per-op calls in list
+    order, and the counters of both workspace parts are left zeroed."""
+    m, nl = 8, 45
+    gen = torch.Generator(device=DEV)
+    gen.manual_seed(777)
+    layers = [device_layer(l, m, gen) for l in range(nl)]
+    spec = []
+    for l, L in enumerate(layers):
+        (xq, _), (xo, _), (xg, _) = L["x"]
+        o = L["out"]
+        if l == 32:
+            xq = layers[31]["out"]["down"]
+        spec += [("lin", xq, L["q"], o["q"]), ("lin", xo, L["o"], o["o"]), ("ffn", xg, (L["g"], L["u"]), o["h"]),
+                 ("lin", o["h"], L["d"], o["down"])]
+    ops = [tw.linear_op(x, w["p"], w["g"], y) if k == "lin" else
+           tw.ffn_gate_up_op(x, w[0]["p"], w[0]["g"], w[1]["p"], w[1]["g"], y) for k, x, w, y in spec]
+    n, cap = len(ops), tw.BITNET_SEQ_MAX_OPS
+    assert n == 180 and spec[cap][1] is spec[cap - 1][3]
+    ws = workspace(n, m)
+    c0 = tw.bitnet_launch_count()
+    tw.bitnet_decode_sequence(ops, m, ws)
+    torch.cuda.synchronize()
+    assert tw.bitnet_launch_count() - c0 == 4  # two launches of (tensor maps, sequence)
+    assert tw.bitnet_device_status() == 0
+    part0 = tw.bitnet_sequence_workspace_size(cap, m, I)
+    assert counters_zero(ws, cap) and counters_zero(ws[part0:], n - cap)
+    ref = {}
+    for k, x, w, y in spec:
+        xin = ref.get(x.data_ptr(), x)
+        ref[y.data_ptr()] = (tw.bitnet_linear(xin, w["p"], w["g"]) if k == "lin" else
+                             tw.bitnet_ffn_gate_up(xin, w[0]["p"], w[0]["g"], w[1]["p"], w[1]["g"]))
+    for i, (k, x, w, y) in enumerate(spec):
+        assert same_bits(y, ref[y.data_ptr()]), i
+
+
 # ---------------------------------------------------------------- failure detection (no GPU fault)
 def test_bounded_wait_runs_out_and_the_next_launch_is_correct():
     """A host-armed stall makes one op's weight-row tasks wait for a quantisation task that

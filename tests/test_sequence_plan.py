@@ -271,7 +271,8 @@ def test_workspace_size():
     assert tw.bitnet_sequence_workspace_size(2, 8, 2560) > one
     assert tw.bitnet_sequence_workspace_size(1, 9, 2560) > one       # 16 token rows of x_q
     assert tw.bitnet_sequence_workspace_size(1, 64, 8192) >= 64 * 8192
-    for bad in ((0, 8, 256), (129, 8, 256), (1, 0, 256), (1, 65, 256), (1, 8, 32), (1, 8, 8256)):
+    for bad in ((0, 8, 256), (tw.BITNET_SEQ_MAX_OPS_TOTAL + 1, 8, 256), (1, 0, 256), (1, 65, 256), (1, 8, 32),
+                (1, 8, 8256)):
         assert tw.bitnet_sequence_workspace_size(*bad) == 0
     # the documented size: counters (2 per op + 2), tensor maps (2 x 128 bytes per op, 128-byte
     # alignment slack), then per op x_q [K/64][Mp][64] + 512 bytes of scales and row sums
@@ -280,6 +281,36 @@ def test_workspace_size():
         mp = 8 if m <= 8 else 16 if m <= 16 else 32 if m <= 32 else 64
         want = up(4 * (2 + 2 * n)) + up(256 * n + 128) + n * (up(k * mp) + 512)
         assert tw.bitnet_sequence_workspace_size(n, m, k) == want
+    # longer lists: one part per launch of at most BITNET_SEQ_MAX_OPS ops, laid out as above
+    part = lambda n, k: up(4 * (2 + 2 * n)) + up(256 * n + 128) + n * (up(k * 8) + 512)  # noqa: E731
+    cap = tw.BITNET_SEQ_MAX_OPS
+    for n in (cap + 1, 180, 2 * cap, tw.BITNET_SEQ_MAX_OPS_TOTAL):
+        want = sum(part(min(cap, n - c0), 6912) for c0 in range(0, n, cap))
+        assert tw.bitnet_sequence_workspace_size(n, 8, 6912) == want
+
+
+def test_long_lists_are_validated_before_any_launch():
+    """A list longer than one launch is validated as a whole first: an invalid op in its
+    second part is refused before the first part is launched (here: before the missing
+    GPU is noticed); a valid list without a GPU fails with a CUDA status."""
+    lib = tw.load_library()
+    n, m = tw.BITNET_SEQ_MAX_OPS + 50, 4
+    good = [lin(BASE + (2 * i << 20), 256, 256, BASE + ((2 * i + 1) << 20), BASE + ((1 << 12) + i << 20))
+            for i in range(n)]
+    size = tw.bitnet_sequence_workspace_size(n, m, 256)
+    ws = BASE + (1 << 34)
+    bad = list(good)
+    bad[tw.BITNET_SEQ_MAX_OPS + 10] = lin(BASE, 256, 256, BASE + 16, BASE + (8 << 30))  # y overlaps its own x
+    assert lib.bitnet_decode_sequence(tw._op_array(bad), n, m, ws, size, None) == tw.BITNET_ERR_INVALID_ARG
+    over = list(good)
+    over[-1] = lin(BASE + (2 * (n - 1) << 20), 256, 256, ws + 4096, BASE + (8 << 30))   # writes the workspace
+    assert lib.bitnet_decode_sequence(tw._op_array(over), n, m, ws, size, None) == tw.BITNET_ERR_INVALID_ARG
+    assert lib.bitnet_decode_sequence(tw._op_array(good), n, m, ws, size - 256, None) == tw.BITNET_ERR_WORKSPACE
+    assert lib.bitnet_decode_sequence(tw._op_array(good), tw.BITNET_SEQ_MAX_OPS_TOTAL + 1, m, ws, size,
+                                      None) == tw.BITNET_ERR_INVALID_ARG
+    import torch
+    if not torch.cuda.is_available():
+        assert lib.bitnet_decode_sequence(tw._op_array(good), n, m, ws, size, None) == tw.BITNET_ERR_CUDA
 
 
 def test_norm_fields_are_validated():
