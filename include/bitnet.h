@@ -438,7 +438,8 @@ bitnet_status_t bitnet_sequence_tasks(const bitnet_op_t *ops, int32_t n_ops, int
 
 /*
  * Tests only (host-armed failure injection, no GPU fault): make the weight-row
- * tasks of op `op` (index into the list of later bitnet_decode_sequence calls)
+ * tasks of op `op` (index into the whole list of later bitnet_decode_sequence
+ * calls, 0 <= op < BITNET_SEQ_MAX_OPS_TOTAL)
  * wait for one quantisation task more than exist, so that the wait runs out
  * after the wait limit and the launch ends with BITNET_ERR_TIMEOUT in the
  * device status word; -1 turns it off.  Returns the previous value (-2 if

@@ -954,9 +954,11 @@ std::atomic<int> g_seq_stall{-1};                        // tests: op (list inde
 std::atomic<unsigned long long> g_wait_limit_set{kDefaultWaitLimitNs};
 
 // Build the launch program for ops in execution order (user_index: list index
-// of each).  ws: workspace (counters zero before the first launch).
+// of each).  ws: workspace (counters zero before the first launch).  stall:
+// list index of the test stall's op, or -2 to read the test setting.
 bitnet_status_t seq_build(DtProgram &p, const bitnet_op_t *ops, const int32_t *user_index, int n, int64_t M, int ctas,
-                          void *ws, size_t ws_bytes, ByteRange extra, std::vector<int> *order_out = nullptr)
+                          void *ws, size_t ws_bytes, ByteRange extra, std::vector<int> *order_out = nullptr,
+                          int stall = -2)
 {
     SeqGroups G;
     bitnet_status_t st = seq_groups(ops, n, M, extra, G);
@@ -975,7 +977,7 @@ bitnet_status_t seq_build(DtProgram &p, const bitnet_op_t *ops, const int32_t *u
                                                               (uintptr_t)128))
                    : nullptr;
     size_t off = seq_counter_bytes(n) + seq_map_bytes(n);
-    const int stall = g_seq_stall.load();
+    if (stall == -2) stall = g_seq_stall.load();
     for (int j = 0; j < n; ++j) {
         const bitnet_op_t &o = ops[j];
         DtOp &d = p.ops[j];
@@ -1105,12 +1107,14 @@ bool seq_cache_match(const SeqCacheEntry &e, const bitnet_op_t *ops, int n, int6
 int seq_ctas(int dev) { return num_sms_for(dev); } // one CTA per SM (227 KB of shared memory each)
 
 // One launch of at most BITNET_SEQ_MAX_OPS ops.  whole: the byte range no op may
-// touch (the caller's whole workspace), or null for this part's own.
+// touch (the caller's whole workspace), or null for this part's own; base: the
+// list index of ops[0] in the caller's list (the test stall names a list index).
 bitnet_status_t decode_sequence(const bitnet_op_t *ops, int n, int64_t M, void *workspace, size_t ws_bytes,
-                                cudaStream_t stream, const ByteRange *whole = nullptr)
+                                cudaStream_t stream, const ByteRange *whole = nullptr, int base = 0)
 {
     if (workspace && !aligned16(workspace)) return BITNET_ERR_MISALIGNED;
-    const int stall = g_seq_stall.load();
+    const int stall_set = g_seq_stall.load();
+    const int stall = stall_set >= base && stall_set < base + n ? stall_set - base : -1;
     const int dev = current_device();
     if (ops && n >= 1 && n <= BITNET_SEQ_MAX_OPS && workspace && dev >= 0) {
         static DtProgram hit_proto;
@@ -1140,7 +1144,7 @@ bitnet_status_t decode_sequence(const bitnet_op_t *ops, int n, int64_t M, void *
     for (int k = 0; k < n; ++k) sched[k] = ops[order[k]];
     static DtProgram prog_proto; // zero-initialised template; each call fills a copy
     DtProgram p = prog_proto;
-    st = seq_build(p, sched, order, n, M, ctas, workspace, ws_bytes, wsr);
+    st = seq_build(p, sched, order, n, M, ctas, workspace, ws_bytes, wsr, nullptr, stall);
     if (st != BITNET_OK) return st;
     if (p.n_slots < 2) return BITNET_ERR_UNSUPPORTED_SHAPE;
     // the template of the weight maps (any op's first matrix: address, extent and pitch are replaced per op)
@@ -1372,7 +1376,7 @@ bitnet_status_t bitnet_decode_sequence(const bitnet_op_t *ops, int32_t n_ops, in
         const int nc = std::min(BITNET_SEQ_MAX_OPS, n_ops - c0);
         const size_t part = seq_part_ws_bytes(nc, M, K_max);
         const bitnet_status_t st =
-            decode_sequence(ops + c0, nc, M, static_cast<unsigned char *>(workspace) + off, part, stream, &whole);
+            decode_sequence(ops + c0, nc, M, static_cast<unsigned char *>(workspace) + off, part, stream, &whole, c0);
         if (st != BITNET_OK) return st;
         off += part;
     }
@@ -1428,7 +1432,7 @@ uint64_t bitnet_set_wait_limit_ns(uint64_t ns)
 
 int bitnet_set_sequence_test_stall(int op)
 {
-    if (op < -1 || op >= BITNET_SEQ_MAX_OPS) return -2;
+    if (op < -1 || op >= BITNET_SEQ_MAX_OPS_TOTAL) return -2;
     return g_seq_stall.exchange(op);
 }
 

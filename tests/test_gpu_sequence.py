@@ -407,6 +407,47 @@ def test_bounded_wait_runs_out_and_the_next_launch_is_correct():
     check_layer(L, m, np.arange(m))
 
 
+def test_bounded_wait_in_the_second_launch_of_a_long_list():
+    """A 132-op list (two launches) with the stall on op 130, the gate/up op of the last layer,
+    in the second launch: the first launch completes and its outputs equal the per-op calls;
+    the second ends by itself with BITNET_ERR_TIMEOUT; the counters of both workspace parts
+    are left zeroed, and the next call without the stall is correct throughout."""
+    m, nl = 8, 33
+    gen = torch.Generator(device=DEV)
+    gen.manual_seed(778)
+    layers = [device_layer(l, m, gen) for l in range(nl)]
+    ops = sum((layer_ops(L) for L in layers), [])
+    n, cap = len(ops), tw.BITNET_SEQ_MAX_OPS
+    ws = workspace(n, m)
+    part0 = tw.bitnet_sequence_workspace_size(cap, m, I)
+
+    def check(upto):
+        for L in layers[:upto]:
+            (xq, _), (xo, _), (xg, _) = L["x"]
+            o = L["out"]
+            ref_h = tw.bitnet_ffn_gate_up(xg, L["g"]["p"], L["g"]["g"], L["u"]["p"], L["u"]["g"])
+            for got, ref in ((o["q"], tw.bitnet_linear(xq, L["q"]["p"], L["q"]["g"])),
+                             (o["o"], tw.bitnet_linear(xo, L["o"]["p"], L["o"]["g"])), (o["h"], ref_h),
+                             (o["down"], tw.bitnet_linear(ref_h, L["d"]["p"], L["d"]["g"]))):
+                assert same_bits(got, ref)
+
+    prev_limit = tw.bitnet_set_wait_limit_ns(20_000_000)
+    prev_stall = tw.bitnet_set_sequence_test_stall(130)
+    try:
+        tw.bitnet_decode_sequence(ops, m, ws)
+        torch.cuda.synchronize()
+        assert tw.bitnet_device_status(clear=True) == tw.BITNET_ERR_TIMEOUT
+        assert counters_zero(ws, cap) and counters_zero(ws[part0:], n - cap)
+    finally:
+        tw.bitnet_set_sequence_test_stall(prev_stall)
+        tw.bitnet_set_wait_limit_ns(prev_limit)
+    check(cap // 4)  # the 32 layers of the first launch
+    run_seq(ops, m, ws)
+    assert counters_zero(ws[part0:], n - cap)
+    assert tw.bitnet_device_status(clear=False) == tw.BITNET_OK
+    check(nl)
+
+
 # ---------------------------------------------------------------- independent layers
 @pytest.mark.parametrize("m", [1, 8, 13])
 def test_private_layer_stack(m):

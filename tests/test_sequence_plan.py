@@ -335,8 +335,11 @@ def test_norm_fields_are_validated():
 def test_test_stall_setter():
     assert tw.bitnet_set_sequence_test_stall(3) == -1
     assert tw.bitnet_set_sequence_test_stall(-1) == 3
+    # an index of a list longer than one launch is accepted (it names an op of the whole list)
+    assert tw.bitnet_set_sequence_test_stall(tw.BITNET_SEQ_MAX_OPS + 5) == -1
+    assert tw.bitnet_set_sequence_test_stall(-1) == tw.BITNET_SEQ_MAX_OPS + 5
     with pytest.raises(ValueError):
-        tw.bitnet_set_sequence_test_stall(tw.BITNET_SEQ_MAX_OPS)
+        tw.bitnet_set_sequence_test_stall(tw.BITNET_SEQ_MAX_OPS_TOTAL)
 
 
 # ---------------------------------------------------------------- task groups and their order
