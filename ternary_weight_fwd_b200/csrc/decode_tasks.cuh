@@ -127,15 +127,26 @@ constexpr int DT_BAR_QINFO = DT_BAR_QFULL + 8 * DT_QUEUE;
 constexpr int DT_BAR_QEMPTY = DT_BAR_QINFO + 8 * DT_QUEUE;
 constexpr int DT_BAR_CDONE = DT_BAR_QEMPTY + 8 * DT_QUEUE; // compute warps done with the entry's task
 constexpr int DT_QTASK = DT_BAR_CDONE + 8 * DT_QUEUE; // int[DT_QUEUE]
+constexpr int DT_QOP = DT_QTASK + 4 * DT_QUEUE;       // DtEntry[DT_QUEUE]: the row task's op fields
 constexpr int DT_RED = 512;                           // quant-task reductions (512 bytes)
-constexpr int DT_INFO = 1024;                         // per queue entry: s[64] fp32, rs[64] int32, gamma0, gamma1
-constexpr int DT_INFO_S = 0, DT_INFO_RS = 4 * DT_MAX_M, DT_INFO_G = 8 * DT_MAX_M;
-constexpr int DT_INFO_BYTES = 8 * DT_MAX_M + 16;
-constexpr int DT_DIG = 3584;                          // [8 warps][20] long accumulators (quant tasks)
-constexpr int DT_HDR = 5120; // the piece ring starts here
+// per queue entry (row tasks): fl(gamma0 / s[m]), rowsum[m], fl(gamma1 / s[m]) for m < M
+constexpr int DT_INFO = 1024;
+constexpr int DT_INFO_R0 = 0, DT_INFO_RS = 4 * DT_MAX_M, DT_INFO_R1 = 8 * DT_MAX_M;
+constexpr int DT_INFO_BYTES = 12 * DT_MAX_M;
+constexpr int DT_DIG = 4096;                          // [8 warps][20] long accumulators (quant tasks)
+constexpr int DT_HDR = 6144; // the piece ring starts here
+
+// The fields of a row task's op that the compute warps use, written into the
+// queue entry by the weight producer (which reads the op anyway), so that the
+// compute warps read shared memory at a task's start instead of the op table
+// in kernel-parameter space.
+struct DtEntry {
+    float *y;
+    int K, N, nmat, pad;
+};
 static_assert(DT_INFO + DT_QUEUE * DT_INFO_BYTES <= DT_DIG, "shared header");
 static_assert(DT_DIG + 8 * 8 * SS_LONG_DIGITS <= DT_HDR && DT_DIG % 8 == 0, "shared header");
-static_assert(DT_QTASK + 4 * DT_QUEUE <= DT_RED, "shared header");
+static_assert(DT_QOP % 8 == 0 && DT_QOP + (int)sizeof(DtEntry) * DT_QUEUE <= DT_RED, "shared header");
 static_assert(DT_HDR % 1024 == 0 && DT_WBYTES % 1024 == 0, "ring alignment (128-byte swizzle)");
 
 // task t -> (op, kind, index)
@@ -345,6 +356,14 @@ BITNET_DEVINL void dt_weight_producer(const DtProgram &p, unsigned char *smem)
         mbar_wait(&qempty[e], ((seq / DT_QUEUE) & 1u) ^ 1u);
         if (lane == 0) {
             qtask[e] = t < 0 ? DT_QEND : dt_pack(tk);
+            if (t >= 0 && !tk.quant) {
+                const DtOp &op = p.ops[tk.op];
+                DtEntry *en = reinterpret_cast<DtEntry *>(smem + DT_QOP) + e;
+                en->y = op.y;
+                en->K = op.K;
+                en->N = op.N;
+                en->nmat = op.nmat;
+            }
             mbar_arrive(&qfull[e]);
         }
         ++seq;
@@ -427,17 +446,21 @@ BITNET_DEVINL void dt_act_producer(const DtProgram &p, unsigned char *smem)
                 }
             }
             __syncwarp();
-            // scales, row sums and gammas of this task's op into the entry (asynchronous: the
-            // entry's info barrier completes when they have landed)
-            const uint32_t inf = smem_u32(smem + DT_INFO + e * DT_INFO_BYTES);
-            const int ch = Mp / 4; // 16-byte chunks of Mp values (at most 16)
-            if (lane < ch) {
-                dt_cp16(inf + DT_INFO_S + 16 * lane, op.s + 4 * lane, true);
-                dt_cp16(inf + DT_INFO_RS + 16 * lane, op.rs + 4 * lane, true);
+            // the epilogue's factors fl(gamma / s[m]) and the row sums of this task's op into the
+            // entry (this warp runs a task ahead of the compute warps, so the divisions and the
+            // loads leave their path); every lane arrives on the entry's info barrier
+            {
+                unsigned char *inf = smem + DT_INFO + e * DT_INFO_BYTES;
+                const float g0 = dt_ld_cg_f32(op.gamma0);
+                const float g1 = op.nmat == 2 ? dt_ld_cg_f32(op.gamma1) : 0.0f;
+                for (int m = lane; m < p.M; m += 32) {
+                    const float sm = dt_ld_cg_f32(op.s + m);
+                    reinterpret_cast<int *>(inf + DT_INFO_RS)[m] = dt_ld_cg_s32(op.rs + m);
+                    reinterpret_cast<float *>(inf + DT_INFO_R0)[m] = __fdiv_rn(g0, sm);
+                    if (op.nmat == 2) reinterpret_cast<float *>(inf + DT_INFO_R1)[m] = __fdiv_rn(g1, sm);
+                }
+                mbar_arrive(&qinfo[e]);
             }
-            if (lane == 0) dt_cp4(inf + DT_INFO_G, op.gamma0);
-            if (lane == 1 && op.nmat == 2) dt_cp4(inf + DT_INFO_G + 4, op.gamma1);
-            dt_cp_arrive(smem_u32(&qinfo[e]));
             // the x_q chunk of every piece: [8 k-blocks][Mp][64] bytes, contiguous in the workspace
             const int np = dt_pieces(op.K);
             for (int pc = 0; pc < np; ++pc, ring_pos.next(p.n_slots)) {
@@ -967,8 +990,8 @@ BITNET_DEVINL void dt_compute(const DtProgram &p, unsigned char *smem)
         const int t = qtask[e];
         if (t == DT_QEND) break;
         const DtTask tk = dt_unpack(t);
-        const DtOp &op = p.ops[tk.op];
         if (tk.quant) {
+            const DtOp &op = p.ops[tk.op];
             if constexpr (TT == 1) {
                 // one token on all compute warps; the op that wrote x (read after write) is complete
                 if (tid == 0)
@@ -1003,9 +1026,10 @@ BITNET_DEVINL void dt_compute(const DtProgram &p, unsigned char *smem)
                     for (int tt = 0; tt < TT; ++tt)
 #pragma unroll
                         for (int c = 0; c < 4; ++c) acc[r][a][tt][c] = 0;
-            const int K = op.K;
+            // the entry's op fields (valid until this task's qempty arrival)
+            const int K = reinterpret_cast<const DtEntry *>(smem + DT_QOP)[e].K;
             const int np = dt_pieces(K);
-            const bool ffn = op.nmat == 2;
+            const bool ffn = reinterpret_cast<const DtEntry *>(smem + DT_QOP)[e].nmat == 2;
             const uint32_t row_lo = ffn ? (uint32_t)(warp * 8 + g) : (uint32_t)(warp * 16 + g);
             const uint32_t row_hi = row_lo + (ffn ? (uint32_t)DT_BOX_ROWS : 8u);
             const uint32_t xlane = (uint32_t)(RG * DT_WBYTES + g * 64 + t4 * 16);
@@ -1035,13 +1059,12 @@ BITNET_DEVINL void dt_compute(const DtProgram &p, unsigned char *smem)
             // epilogue: y = fl((float)(sum c*x - sum x) * fl(gamma / s))
             mbar_wait(&qinfo[e], (seq / DT_QUEUE) & 1u);
             const unsigned char *inf = smem + DT_INFO + e * DT_INFO_BYTES;
-            const float *is = reinterpret_cast<const float *>(inf + DT_INFO_S);
+            const float *ir0 = reinterpret_cast<const float *>(inf + DT_INFO_R0);
+            const float *ir1 = reinterpret_cast<const float *>(inf + DT_INFO_R1);
             const int *irs = reinterpret_cast<const int *>(inf + DT_INFO_RS);
-            const float g0 = *reinterpret_cast<const float *>(inf + DT_INFO_G);
-            const int N = op.N;
-            float *y = op.y;
-            if (op.nmat == 2) {
-                const float g1 = *reinterpret_cast<const float *>(inf + DT_INFO_G + 4);
+            const int N = reinterpret_cast<const DtEntry *>(smem + DT_QOP)[e].N;
+            float *y = reinterpret_cast<const DtEntry *>(smem + DT_QOP)[e].y;
+            if (ffn) {
 #pragma unroll
                 for (int tt = 0; tt < TT; ++tt)
 #pragma unroll
@@ -1049,8 +1072,7 @@ BITNET_DEVINL void dt_compute(const DtProgram &p, unsigned char *smem)
                         const int m = tt * 8 + 2 * t4 + q;
                         if (m < M) {
                             const int rsm = irs[m];
-                            const float sm = is[m];
-                            const float rg0 = __fdiv_rn(g0, sm), rg1 = __fdiv_rn(g1, sm);
+                            const float rg0 = ir0[m], rg1 = ir1[m];
 #pragma unroll
                             for (int r = 0; r < RG; ++r) {
                                 const int n = tk.idx * (RG * DT_ROWS / 2) + (warp + 8 * r) * 8 + g;
@@ -1071,7 +1093,7 @@ BITNET_DEVINL void dt_compute(const DtProgram &p, unsigned char *smem)
                         const int m = tt * 8 + 2 * t4 + q;
                         if (m < M) {
                             const int rsm = irs[m];
-                            const float rsc = __fdiv_rn(g0, is[m]);
+                            const float rsc = ir0[m];
 #pragma unroll
                             for (int r = 0; r < RG; ++r) {
                                 const int n0 = tk.idx * (RG * DT_ROWS) + (warp + 8 * r) * 16 + g;
@@ -1139,7 +1161,7 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_decode_tasks(const __grid_con
         }
         for (int i = 0; i < DT_QUEUE; ++i) {
             mbar_init(&bars[DT_BAR_QFULL / 8 + i], 1);
-            mbar_init(&bars[DT_BAR_QINFO / 8 + i], 32);  // activation producer lanes (cp.async, noinc)
+            mbar_init(&bars[DT_BAR_QINFO / 8 + i], 32);  // activation producer lanes
             mbar_init(&bars[DT_BAR_QEMPTY / 8 + i], 10); // compute warps, activation producer, completion warp
             mbar_init(&bars[DT_BAR_CDONE / 8 + i], 8);   // compute warps
         }
