@@ -344,12 +344,14 @@ def test_full_decode_step_of_the_benchmark():
             assert same_bits(got, ref), l
 
 
-def test_list_longer_than_one_launch():
-    """45 layers at M = 8: 180 ops in one call, run as two launches of 128 and 52 ops.  Layer
-    32's q reads layer 31's down output, so the first op of the second launch reads what the
-    last op of the first launch wrote.  Every output is bitwise equal to per-op calls in list
-    order, and the counters of both workspace parts are left zeroed."""
-    m, nl = 8, 45
+@pytest.mark.parametrize("m", [8, 13])
+def test_list_longer_than_one_launch(m):
+    """45 layers: 180 ops in one call, run as two launches of 128 and 52 ops.  Layer 32's q
+    reads layer 31's down output, so the first op of the second launch reads what the last op
+    of the first launch wrote.  Every output is bitwise equal to per-op calls in list order,
+    and the counters of both workspace parts are left zeroed.  M = 13 takes the two-token-tile
+    kernel and its larger workspace parts."""
+    nl = 45
     gen = torch.Generator(device=DEV)
     gen.manual_seed(777)
     layers = [device_layer(l, m, gen) for l in range(nl)]
