@@ -398,11 +398,13 @@ bitnet_status_t bitnet_sequence_schedule(const bitnet_op_t *ops, int32_t n_ops, 
  *               list.  All parts are validated before the first launch.
  *   M           tokens, 1 <= M <= BITNET_SEQ_MAX_M, the same for every op
  *   workspace   device memory of at least
- *               bitnet_sequence_workspace_size(n_ops, M, max K) bytes whose
- *               counters (the first 4 * (2 + 2 * n) bytes of the part of each
- *               launch of n ops) are ZERO before its first use; every call
- *               leaves them zero again (also after a device-side timeout).
- *               Calls that may run at the same time need separate workspaces.
+ *               bitnet_sequence_workspace_size(n_ops, M, max K) bytes, any
+ *               contents: each launch zeroes its own completion counters (the
+ *               first 4 * (2 + 2 * n) bytes of its part) before its sequence
+ *               kernel uses them, and leaves them zero again (also after a
+ *               device-side timeout), so one workspace may serve different op
+ *               lists one after the other.  Calls that may run at the same time
+ *               need separate workspaces.
  *
  * Errors (nothing is launched): BITNET_ERR_INVALID_ARG for a null pointer, a
  * bad kind or dtype, a negative or non-finite norm_eps, an op whose y overlaps

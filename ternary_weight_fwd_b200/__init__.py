@@ -361,7 +361,7 @@ def bitnet_sequence_workspace_size(n_ops: int, m: int, k_max: int) -> int:
 
 
 def bitnet_sequence_workspace(device, n_ops=BITNET_SEQ_MAX_OPS, m=BITNET_SEQ_MAX_M, k_max=8192):
-    """A zero-filled workspace for bitnet_decode_sequence (calls leave its counters zeroed)."""
+    """A workspace for bitnet_decode_sequence (each launch zeroes its counters before use)."""
     return torch.zeros(bitnet_sequence_workspace_size(n_ops, m, k_max), dtype=torch.uint8, device=device)
 
 

@@ -301,6 +301,11 @@ __global__ void __launch_bounds__(32) k_decode_maps(const __grid_constant__ DtPr
     __shared__ alignas(128) unsigned char sm[2][128];
     const int j = blockIdx.x, lane = threadIdx.x;
     pdl_launch_dependents(); // the sequence kernel starts now; its weight producer waits for this grid
+    // block 0 zeroes the completion counters: every counter access of the sequence kernel follows
+    // its weight producer's wait for this grid, and this grid starts after all earlier work on the
+    // stream, so the launch never depends on what an earlier call left in these bytes
+    if (j == 0)
+        for (int i = lane; i < DT_CNT_OPS + 2 * p.n_ops; i += 32) p.counters[i] = 0u;
     if (j >= p.n_ops) return;
     const DtOp &op = p.ops[j];
     for (int m = 0; m < op.nmat; ++m) {

@@ -384,6 +384,45 @@ def test_list_longer_than_one_launch(m):
         assert same_bits(y, ref[y.data_ptr()]), i
 
 
+def test_one_workspace_for_different_lists():
+    """One workspace serves a 4-layer list, then a 45-layer list (two launches whose counters sit
+    where the first list kept tensor maps and activations), then the 4-layer list again, then
+    the 45-layer list after the workspace was filled with 0xff: every run gives the per-op
+    results bit for bit."""
+    m = 8
+    gen = torch.Generator(device=DEV)
+    gen.manual_seed(779)
+    layers = [device_layer(l, m, gen) for l in range(45)]
+    short = sum((layer_ops(L) for L in layers[:4]), [])
+    long_ = sum((layer_ops(L) for L in layers), [])
+    ws = torch.empty(max(tw.bitnet_sequence_workspace_size(len(short), m, I),
+                         tw.bitnet_sequence_workspace_size(len(long_), m, I)), dtype=torch.uint8, device=DEV)
+    ws.fill_(0xff)
+
+    def check(ls):
+        for L in ls:
+            (xq, _), (xo, _), (xg, _) = L["x"]
+            o = L["out"]
+            ref_h = tw.bitnet_ffn_gate_up(xg, L["g"]["p"], L["g"]["g"], L["u"]["p"], L["u"]["g"])
+            for got, ref in ((o["q"], tw.bitnet_linear(xq, L["q"]["p"], L["q"]["g"])),
+                             (o["o"], tw.bitnet_linear(xo, L["o"]["p"], L["o"]["g"])), (o["h"], ref_h),
+                             (o["down"], tw.bitnet_linear(ref_h, L["d"]["p"], L["d"]["g"]))):
+                assert same_bits(got, ref)
+            for t in o.values():
+                t.fill_(float("nan"))
+
+    for ops, ls in ((short, layers[:4]), (long_, layers), (short, layers[:4])):
+        tw.bitnet_decode_sequence(ops, m, ws)
+        torch.cuda.synchronize()
+        assert tw.bitnet_device_status() == 0
+        check(ls)
+    ws.fill_(0xff)
+    tw.bitnet_decode_sequence(long_, m, ws)
+    torch.cuda.synchronize()
+    assert tw.bitnet_device_status() == 0
+    check(layers)
+
+
 # ---------------------------------------------------------------- failure detection (no GPU fault)
 def test_bounded_wait_runs_out_and_the_next_launch_is_correct():
     """A host-armed stall makes one op's weight-row tasks wait for a quantisation task that
