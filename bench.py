@@ -55,7 +55,8 @@ def parse_args():
     p.add_argument("--prefill-tokens", type=int, default=4096)
     p.add_argument("--decode-steps", type=int, default=128)
     p.add_argument("--decode-batch", type=int, default=8)
-    p.add_argument("--e2e-steps", type=int, default=3)
+    p.add_argument("--e2e-steps", type=int, default=None,
+                   help="steps of the end-to-end measurement (default: --steps; 0 skips it)")
     p.add_argument("--cpu-seconds", type=float, default=10.0, help="budget of the oracle CPU baseline")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-configs", action="store_true",
@@ -69,7 +70,10 @@ def parse_args():
                    help="profiling harness: build one layer, run this projection kind --profile-reps times "
                         "(no graphs, no timing, no JSON) and exit; for ncu captures of one kernel")
     p.add_argument("--profile-reps", type=int, default=3)
-    return p.parse_args()
+    a = p.parse_args()
+    if a.e2e_steps is None:
+        a.e2e_steps = a.steps
+    return a
 
 
 def workload_config(a, n_gpus):
