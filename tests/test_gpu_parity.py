@@ -87,6 +87,43 @@ def run_linear(xd, W, dispatch, m, k, n):
     return y.cpu().numpy(), acc.cpu().numpy(), x_q.cpu().numpy(), s.cpu().numpy()
 
 
+def weights_from(w):
+    """Packed weights of a given latent matrix, by both sides."""
+    p_ref, g_ref, w_q = oracle.pack_weights(w)
+    p, g = tw.bitnet_pack_weights(torch.from_numpy(w).to(DEV))
+    torch.cuda.synchronize()
+    return dict(w=w, w_q=w_q, p_ref=p_ref, g_ref=g_ref, p=p, g=g)
+
+
+@pytest.mark.parametrize("dispatch,m", [(d, 5) for d in DECODE] + [(tw.BITNET_DISPATCH_PREFILL, 130)],
+                         ids=lambda v: DNAME[v] if v in DNAME and v < 4 else str(v))
+def test_linear_degenerate_inputs(dispatch, m):
+    """Degenerate cases of the method on every path: an all-zero latent matrix (gamma = 0, so
+    every code is 0 and every output exactly 0), a matrix with one nonzero latent (gamma =
+    |w| / (N K), W_q one-hot), and activation rows that are all zero (s = 127 / 1e-5, x_q = 0,
+    y = 0) next to ordinary rows.  Integers bit-exact, outputs as the oracle (zero exact)."""
+    k, n = 320, 200
+    xd, xf = make_x(m, k, 4100 + m, "normal", "bf16")
+    xd = xd.clone()
+    xd[1].zero_()
+    xd[m - 1].zero_()
+    xf = xd.float().cpu().numpy()
+    one = np.zeros((n, k), np.float32)
+    one[37, 101] = -0.75
+    for w in (np.zeros((n, k), np.float32), one):
+        W = weights_from(w)
+        assert np.array_equal(W["p"].cpu().numpy(), W["p_ref"])
+        y, acc, x_q, s = run_linear(xd, W, dispatch, m, k, n)
+        y_ref, acc_ref, xq_ref, s_ref = oracle.bitlinear(xf, W["p_ref"], W["g_ref"], k)
+        assert np.array_equal(x_q, xq_ref)
+        assert np.array_equal(s.view(np.uint32), s_ref.view(np.uint32))
+        assert np.array_equal(acc.astype(np.int64), acc_ref)
+        assert_rel_close(y, y_ref)
+        assert not y[1].any() and not y[m - 1].any()
+        if not w.any():
+            assert not y.any() and not acc.any()
+
+
 LINEAR_SHAPES = [
     # (M, K, N, kind, dtype)
     (4, 256, 256, "normal", "bf16"),          # small single BitLinear
