@@ -209,6 +209,28 @@ def run_ffn(xd, G, U, dispatch, m, n):
     return h.cpu().numpy(), ag.cpu().numpy(), au.cpu().numpy()
 
 
+@pytest.mark.parametrize("dispatch,m", [(d, 5) for d in DECODE] + [(tw.BITNET_DISPATCH_PREFILL, 130)],
+                         ids=lambda v: DNAME[v] if v in DNAME and v < 4 else str(v))
+def test_ffn_degenerate_inputs(dispatch, m):
+    """The gated FFN with an all-zero gate matrix (h = relu(0)^2 * u = 0) and with an all-zero
+    up matrix (h = relu(g)^2 * 0 = 0), and all-zero activation rows, on every path: int32 sums
+    bit-exact, h as the oracle and exactly zero where the definition makes it zero."""
+    k, n = 320, 136
+    xd, _ = make_x(m, k, 4200 + m, "normal", "bf16")
+    xd = xd.clone()
+    xd[0].zero_()
+    xf = xd.float().cpu().numpy()
+    rnd = make_weights(n, k, 4300)
+    zero = weights_from(np.zeros((n, k), np.float32))
+    for G, U in ((zero, rnd), (rnd, zero)):
+        h, ag, au = run_ffn(xd, G, U, dispatch, m, n)
+        h_ref, ag_ref, au_ref, _, _ = oracle.ffn_gate_up(xf, G["p_ref"], G["g_ref"], U["p_ref"], U["g_ref"], k)
+        assert np.array_equal(ag.astype(np.int64), ag_ref)
+        assert np.array_equal(au.astype(np.int64), au_ref)
+        assert_rel_close(h, h_ref)
+        assert not h.any()
+
+
 FFN_SHAPES = [
     (12, 576, 136, "outliers"),
     (1, 2560, 6912, "normal"),

@@ -384,6 +384,26 @@ def test_list_longer_than_one_launch(m):
         assert same_bits(y, ref[y.data_ptr()]), i
 
 
+def test_degenerate_weights_in_a_sequence():
+    """A sequence whose q projection has all-zero latents (gamma = 0) and whose gated FFN has
+    an all-zero gate matrix, with one all-zero activation row: every output equals the per-op
+    call bit for bit and is exactly zero where the definition makes it zero."""
+    m = 8
+    L = make_layer(860, m)
+    zero = tw.bitnet_pack_weights(torch.zeros((H, H), device=DEV))
+    zero_g = tw.bitnet_pack_weights(torch.zeros((I, H), device=DEV))
+    (xq, _), (xo, _), (xg, _) = L["x"]
+    xo = xo.clone()
+    xo[3].zero_()
+    o = L["out"]
+    ops = [tw.linear_op(xq, zero[0], zero[1], o["q"]), tw.linear_op(xo, L["o"]["p"], L["o"]["g"], o["o"]),
+           tw.ffn_gate_up_op(xg, zero_g[0], zero_g[1], L["u"]["p"], L["u"]["g"], o["h"]),
+           tw.linear_op(o["h"], L["d"]["p"], L["d"]["g"], o["down"])]
+    run_seq(ops, m)
+    assert not o["q"].any() and not o["h"].any() and not o["down"].any() and not o["o"][3].any()
+    assert same_bits(o["o"], tw.bitnet_linear(xo, L["o"]["p"], L["o"]["g"]))
+
+
 def test_one_workspace_for_different_lists():
     """One workspace serves a 4-layer list, then a 45-layer list (two launches whose counters sit
     where the first list kept tensor maps and activations), then the 4-layer list again, then
